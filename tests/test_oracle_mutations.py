@@ -1,0 +1,88 @@
+"""Plants plausible mistakes in a copy of the oracle (on the CPU) and checks
+that at least one pin catches each: the pins are only worth something if a
+dropped term, a wrong sign or index, or a transposed operand fails them."""
+import importlib.util
+import os
+import shutil
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+sys.path.insert(0, HERE)
+import test_oracle_pins as pins  # noqa: E402
+
+# (name, original text, planted text, pins expected to catch it)
+MUTATIONS = [
+    ("philox_weyl_constant", "W0 = 0x9E3779B9u", "W0 = 0x9E3779B8u",
+     ["test_philox_known_answers"]),
+    ("philox_swapped_words", "uint32_t n0 = hi1 ^ c1 ^ k0;",
+     "uint32_t n0 = hi0 ^ c1 ^ k0;", ["test_philox_known_answers"]),
+    ("uniform_bits", "((double)(x >> 9) + 0.5)", "((double)(x >> 8) + 0.5)",
+     ["test_u01_exact_open_interval"]),
+    ("gumbel_sign", "g[k] = -log(-log((double)u[k]));",
+     "g[k] = log(-log((double)u[k]));", ["test_softmax_is_library_softmax"]),
+    ("dropped_temperature", "z[k] = (l[k] + g[k]) / tau;", "z[k] = (l[k] + g[k]);",
+     ["test_softmax_is_library_softmax", "test_gradients_match_central_differences"]),
+    ("jacobian_sign", "acc += yy[j] * (cand[p] - cand[j]);",
+     "acc += yy[j] * (cand[j] - cand[p]);",
+     ["test_gradients_match_central_differences"]),
+    ("ternary_dropped_p0", "double gm = a * (qp - qm) * p1 * p0;",
+     "double gm = a * (qp - qm) * p1;", ["test_gradients_match_central_differences"]),
+    ("scale_grad_dropped_v", "dsg += dw * v[c];", "dsg += dw;",
+     ["test_gradients_match_central_differences"]),
+    ("weight_grad_transposed", "double d = dY[t * N + n];", "double d = dY[n * N + t];",
+     ["test_loss_and_weight_grad_equal_library_gemm"]),
+    ("output_grad_factor", "dY[t * N + n] = (float)gsqo_bf16_round(2.0 * e);",
+     "dY[t * N + n] = (float)gsqo_bf16_round(e);",
+     ["test_loss_and_weight_grad_equal_library_gemm"]),
+    ("lion_beta_swap", "float c = fmaf(beta1, m, omb1 * g);",
+     "float c = fmaf(beta2, m, omb2 * g);", ["test_lion_second_step_closed_form"]),
+    ("rtn_ties_last", "if (d < bestd) {", "if (d <= bestd) {",
+     ["test_init_scales_and_rtn_bruteforce"]),
+    ("ternary_init_sign_of_zero", "(lev == 1 && !(w < 0.0f))", "(lev == 1 && (w > 0.0f))",
+     ["test_init_logits_layout"]),
+    ("local_shift_no_upper_clamp", "if (j > 7) j = 7;\n            c[k]", "c[k]",
+     ["test_local_shift_clamped_exhaustive"]),
+    ("ternary_harden_sign", "lev = nonzero ? (plus ? 2 : 0) : 1;",
+     "lev = nonzero ? (plus ? 0 : 2) : 1;", ["test_harden_bruteforce_and_pack_roundtrip"]),
+    ("pack_msb_first", "packed[n * wpr + bit / 32] |= (1u << (bit % 32));",
+     "packed[n * wpr + bit / 32] |= (1u << (31 - bit % 32));",
+     ["test_harden_bruteforce_and_pack_roundtrip"]),
+]
+
+MODES = {"test_softmax_is_library_softmax": [0, 2]}
+
+
+def _load_mutant(tmp_path, name, old, new):
+    dst = tmp_path / f"oracle_{name}"
+    shutil.copytree(os.path.join(ROOT, "oracle"), dst,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    src = (dst / "gsq_oracle.c").read_text()
+    assert src.count(old) == 1, f"mutation anchor not unique: {name}"
+    (dst / "gsq_oracle.c").write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", dst / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[spec.name] = mod
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new,catchers", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
+    mod = _load_mutant(tmp_path, name, old, new)
+    caught = []
+    for tname in catchers:
+        fn = getattr(pins, tname)
+        params = getattr(fn, "pytestmark", [])
+        modes = MODES.get(tname)
+        if modes is None:
+            modes = [0, 1, 2] if any(m.name == "parametrize" for m in params) else [None]
+        for mode in modes:
+            try:
+                fn(mod) if mode is None else fn(mod, mode)
+            except AssertionError:
+                caught.append((tname, mode))
+    assert caught, f"no pin caught the planted mistake {name}"
