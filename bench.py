@@ -1,0 +1,354 @@
+"""Benchmark of the GSQ layer-reconstruction step on B200.
+
+One step = one pass of the whole hot path over one synthetic layer: Philox
+Gumbel soft weight, forward GEMM with fused loss / output gradient, weight-
+gradient GEMM, fused logit/scale gradients with Lion.  The default workload is
+the Llama-3.1-8B q_proj-shaped layer (4096 x 4096, 4096 calibration tokens,
+2-bit grid).  Under torchrun each rank quantizes its own independent layer of
+that shape (weak scaling, no data-path collective).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...   # the oracle on the host cores
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from post_weight_quantization_philox_b200 import synth  # noqa: E402
+
+METRIC = "GSQ recon steps/s and grid coords updated/s per layer; % of TC / HBM roofline"
+UNIT = "coords/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def phase_bytes_flops(cfg, layer):
+    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch."""
+    NK = cfg.N * cfg.K
+    L = layer.L
+    extra = 1 if cfg.grid == synth.GRID_3BIT_LOCAL else 0  # initial level (int8)
+    groups = cfg.N * (cfg.K // 128)
+    soft = NK * (4 * L + 2 + extra) + groups * 4
+    back = NK * (4 + 16 * L + extra) + groups * 16
+    gemm = 2.0 * cfg.N * cfg.T * cfg.K
+    return {"soft_weight": ("hbm", soft), "forward_gemm": ("tensor", gemm),
+            "weight_grad_gemm": ("tensor", gemm), "backward_lion": ("hbm", back)}
+
+
+def run_gsq(args, rank, world, local_rank):
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    if rank == 0 or not os.path.exists(os.path.join(ROOT, "post_weight_quantization_philox_b200", "libgsq.so")):
+        build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    from post_weight_quantization_philox_b200 import gsq
+
+    torch.cuda.set_device(local_rank)
+    cfg = synth.CONFIGS[args.config]
+    # each rank quantizes its own independent layer of the same shape
+    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
+    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
+    Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    stream = torch.cuda.current_stream()
+    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=rank)
+    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
+    nt = len(taus)
+
+    def dist_barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for i in range(args.warmup):
+        lay.step(float(taus[i % nt]), cfg.lr)
+    torch.cuda.synchronize()
+    gsq.gsq_set_timing(lay, True)
+    gsq.gsq_phase_times(lay)  # reset
+    clocks = ClockSampler(local_rank)
+    dist_barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        lay.step(float(taus[(args.warmup + i) % nt]), cfg.lr)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    phase_ms, phase_n = gsq.gsq_phase_times(lay)
+    gsq.gsq_set_timing(lay, False)
+    loss = lay.last_loss()
+    lay.close()
+    del Wd, Xd
+    torch.cuda.empty_cache()
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end: host buffers through the C ABI, whole quantization job
+    e2e = None if args.no_e2e else run_e2e(gsq, torch, cfg, W, X, rank)
+
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    steps_per_s = args.steps / (ms / 1e3)
+    coords = cfg.N * cfg.K
+    value = world * coords * steps_per_s
+    names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion"]
+    work = phase_bytes_flops(cfg, lay)
+    phases = {}
+    for i, nm in enumerate(names):
+        per = phase_ms[i] / max(phase_n[i], 1)
+        bound, amount = work[nm]
+        if bound == "hbm":
+            ach = amount / (per / 1e3) / 1e9
+            peak, unit = hbm, "GB/s"
+        else:
+            ach = amount / (per / 1e3) / 1e12
+            peak, unit = tf_sus, "TFLOP/s"
+        phases[nm] = {"ms": round(per, 5), "bound": bound, "achieved": round(ach, 1),
+                      "unit": unit, "peak": peak, "frac": round(ach / peak, 4),
+                      "per_launch": amount}
+    dom = max(names, key=lambda n: phases[n]["ms"])
+    d = phases[dom]
+    traffic = load_traffic(dom, args.config)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "steps_per_s": steps_per_s, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state",
+        "data": "synthetic (seeded; W ~ N(0,0.02^2) bf16, X ~ N(0,1) bf16 with 1% outlier channels x20)",
+        "config": {"workload": cfg.name, "N": cfg.N, "K": cfg.K, "T": cfg.T,
+                   "grid": ["2bit", "ternary", "3bit_local"][cfg.grid], "group": 128,
+                   "parallelism": f"independent layer per GPU x{world}",
+                   "l2": "state (logits + Lion momenta, 537 MB) larger than L2; no flush"},
+        "roofline": {"bound": d["bound"], "kernel": dom, "achieved": d["achieved"],
+                     "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
+                     "peak_kind": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})",
+                     "traffic": traffic},
+        "phases": phases,
+        "gpu_launches": int(4 * args.steps),
+        "clocks": clk,
+        "last_loss": loss,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    return out
+
+
+def run_e2e(gsq, torch, cfg, W, X, rank):
+    """Whole quantization job from pinned host buffers through the C ABI:
+    upload + init, the config's steps, loss history read-back, harden+pack
+    into host memory."""
+    Wh = torch.from_numpy(W).to(torch.bfloat16).pin_memory()
+    Xh = torch.from_numpy(X).to(torch.bfloat16).pin_memory()
+    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
+    pb = gsq.gsq_packed_bytes(cfg.grid, cfg.N, cfg.K)
+    packed = torch.zeros(pb // 4, dtype=torch.int32).pin_memory()
+    h16 = torch.zeros((cfg.N, cfg.K // 128), dtype=torch.int16).pin_memory()
+    hist = np.zeros(min(cfg.steps, 4096), np.float64)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    lay = gsq.gsq_init(Wh, Xh, 128, cfg.grid, seed=rank)
+    for tau in taus:
+        lay.step(float(tau), cfg.lr)
+    gsq._check(gsq.lib().gsq_loss_history(lay.ctx, cfg.steps - hist.size, hist.size,
+                                          hist.ctypes.data), "gsq_loss_history")
+    gsq.gsq_harden_pack(lay, packed, h16, None)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    lay.close()
+    h2d = W.size * 2 + X.size * 2
+    d2h = pb + h16.numel() * 2 + hist.nbytes
+    return {"value": cfg.N * cfg.K * cfg.steps / dt, "unit": UNIT,
+            "h2d_bytes_per_step": h2d / cfg.steps, "d2h_bytes_per_step": d2h / cfg.steps,
+            "job": f"init from pinned host + {cfg.steps} steps + harden/pack to host",
+            "seconds": dt}
+
+
+def cpu_baseline(cfg, budget_s=15.0, steps=None):
+    """The oracle on the host cores: a row slice of the same layer (the loss
+    decomposes over rows), full K and T, timed per step."""
+    import oracle
+    oracle.build()
+    threads = os.cpu_count()
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    W = synth.make_weight(cfg)
+    X = synth.make_calib(cfg)
+    rows = 1
+    # calibrate: one step of one row, then scale rows to the budget
+    st = oracle.init(cfg.grid, W[:rows], seed=0)
+    Y = oracle.reference_output(W[:rows], X)
+    t0 = time.perf_counter()
+    oracle.step(st, X, Y, 1.0, cfg.lr)
+    one = time.perf_counter() - t0
+    nsteps = steps or 2
+    rows = int(max(1, min(cfg.N, budget_s / max(one * nsteps, 1e-6))))
+    st = oracle.init(cfg.grid, W[:rows], seed=0)
+    Y = oracle.reference_output(W[:rows], X)
+    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
+    t0 = time.perf_counter()
+    for i in range(nsteps):
+        oracle.step(st, X, Y, float(taus[i]), cfg.lr)
+    dt = time.perf_counter() - t0
+    return {"value": rows * cfg.K * nsteps / dt, "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows} of {cfg.N} rows x K={cfg.K} x T={cfg.T}, {nsteps} steps, {dt:.1f} s"}
+
+
+def load_traffic(kernel, config):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get(config, {}).get(kernel)
+    return None
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    per = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state to build
+    cb = None
+    for _ in range(args.steps):
+        cb = cpu_baseline(cfg, budget_s=args.cpu_seconds / max(args.steps, 1), steps=1)
+        per.append(cb["value"])
+    v = statistics.median(per)
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": cfg.name, "N": cfg.N, "K": cfg.K, "T": cfg.T},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cb["cores"],
+                             "kind": "oracle", "sample": cb["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c2_qproj_4096x4096", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end job (profiling runs)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out:
+            print(json.dumps(out))
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_gsq(args, rank, world, local_rank)
+    if out:
+        print(json.dumps(out))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,225 @@
+/*
+ * gsq.h -- C ABI of libgsq: the GSQ Gumbel-Softmax layer-reconstruction step
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * Method: "GSQ: Highly-Accurate Low-Precision Scalar Quantization for LLMs via
+ * Gumbel-Softmax Sampling" (Dadgarnia et al., arXiv 2604.18556).  The method
+ * paragraph of its summary on agihunt.info defines the state (per-coordinate
+ * logits over a symmetric, zero-point-free, group-wise scalar grid plus one
+ * learnable scale per group of 128), the relaxation (Gumbel-Softmax soft
+ * weighted sum of grid points, annealed to a hard choice), the three grids
+ * (2-bit: 4 levels, 4 logits; ternary: a mask choice times a sign choice;
+ * 3 bits: 5 logits for shifts -2..+2 around the initial level) and the
+ * objective (output reconstruction error on calibration inputs); its
+ * optimisation paragraph names Lion; the Approach section on atlas.scime.ai
+ * restates the same.  Noise comes from Philox4x32-10 (Salmon et al., SC'11).
+ *
+ * Notation: W (N x K) is the layer weight, X (T x K) the calibration inputs,
+ * G = K / group groups per row, L logits per coordinate (4, 2+2, 5),
+ * coord = n*K + k.  One step t computes
+ *     u   = Philox4x32-10(key = seed, ctr = (coord lo, coord hi, t, block))
+ *     g   = -log(-log u),  y = softmax((l + g) / tau),  v = sum y_k c_k,
+ *     What = bf16(s_g * v),
+ *     loss = || X What^T - X W^T ||_F^2,   dY = 2 E,   dWhat = dY^T X,
+ *     dl, ds from the softmax Jacobian;  Lion on logits and scales.
+ *
+ * Conventions for every entry point:
+ *   - returns GSQ_OK (0) or a negative status; never throws, never aborts;
+ *   - a CUDA error or a device-side failure puts the context into a sticky
+ *     failed state: later calls return GSQ_ERR_STATE;
+ *   - all device work is enqueued on the stream given to gsq_init (NULL =
+ *     the legacy default stream); calls documented as "syncs" wait for it;
+ *   - pointers documented "host or device" may point to pageable host,
+ *     pinned host or device memory (unified addressing decides);
+ *   - the context owns all of its device memory; callers own their buffers.
+ */
+#ifndef GSQ_H
+#define GSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GSQ_API __attribute__((visibility("default")))
+#else
+#define GSQ_API
+#endif
+
+typedef struct gsq_ctx gsq_ctx; /* opaque, library-owned */
+
+/* Grids (agihunt.info method paragraph).  Unit levels:
+ *   GSQ_GRID_2BIT        {-1.5, -0.5, 0.5, 1.5}, 4 logits, scale absmax/1.5
+ *   GSQ_GRID_TERNARY     {-1, 0, +1} as mask (zero, nonzero) x sign (-, +),
+ *                        2 + 2 logits, scale absmax
+ *   GSQ_GRID_3BIT_LOCAL  {-3.5 .. 3.5}, 5 logits for shifts -2..+2 around the
+ *                        initial level, clamped to [0, 7], scale absmax/3.5 */
+enum { GSQ_GRID_2BIT = 0, GSQ_GRID_TERNARY = 1, GSQ_GRID_3BIT_LOCAL = 2 };
+
+/* element types of caller inputs */
+enum { GSQ_F32 = 0, GSQ_BF16 = 1 };
+
+enum {
+    GSQ_OK = 0,
+    GSQ_ERR_INVALID_ARG = -1, /* bad size, null pointer, unknown mode, tau <= 0 */
+    GSQ_ERR_CUDA = -2,        /* a CUDA runtime call failed */
+    GSQ_ERR_OOM = -3,         /* device allocation failed */
+    GSQ_ERR_NONFINITE = -4,   /* a loss or an input was NaN / Inf */
+    GSQ_ERR_STATE = -5,       /* context already failed or destroyed */
+    GSQ_ERR_UNSUPPORTED = -6, /* e.g. group != 128, no sm_100 device */
+    GSQ_ERR_TIMEOUT = -7      /* a bounded device-side wait gave up */
+};
+
+/* Recon-error modes */
+enum { GSQ_RECON_HARD = 0, GSQ_RECON_SOFT = 1 };
+
+/*
+ * gsq_init -- A0 of the step: build the state of one layer.
+ *   W        N x K row-major, w_dtype GSQ_F32 or GSQ_BF16, host or device.
+ *   X        T x K row-major, x_dtype GSQ_F32 or GSQ_BF16, host or device.
+ *   group    must be 128 (the pages' group size); K % 128 == 0.
+ *   init_idx nullable; N x K int8 initial level index (2-bit 0..3, ternary
+ *            0..2 for -1/0/+1, 3-bit 0..7), host or device.  NULL selects
+ *            round-to-nearest (first level on ties) of W / s.  (The pages
+ *            start from GPTQ; round-to-nearest is the stand-in.)
+ *   seed     Philox key.
+ *   stream   cudaStream_t (NULL = legacy default stream).
+ * Computes bf16 X (and its transpose), Y_ref = bf16(X) W^T with fp32
+ * accumulation (W at its own precision), s_g = absmax_g / c_max, the initial
+ * levels, logits = +2 on the initial slot and 0 elsewhere, Lion momenta = 0,
+ * step counter t = 0.  W, X and init_idx are read only during the call.
+ * Syncs once at the end.  On failure *out is NULL.
+ */
+GSQ_API int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+             int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+             int grid_mode, const int8_t* init_idx, uint64_t seed,
+             void* stream);
+
+/*
+ * gsq_step -- one reconstruction step at temperature tau (asynchronous):
+ * soft weight (noise of step t), forward GEMM with fused loss and dY,
+ * weight-gradient GEMM, fused logit/scale gradients and Lion update
+ * (c = beta1 m + (1-beta1) g; theta -= lr sign(c); m = beta2 m + (1-beta2) g),
+ * then t += 1.  tau > 0, lr >= 0, 0 <= beta < 1.  The annealing schedule is
+ * the caller's.
+ */
+GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2);
+
+/* gsq_last_loss -- loss (sum of squared errors) of the last step.  Syncs.
+ * GSQ_ERR_NONFINITE if it was NaN / Inf; GSQ_ERR_STATE before any step. */
+GSQ_API int gsq_last_loss(gsq_ctx* ctx, double* loss);
+
+/* gsq_loss_history -- losses of steps [t0, t0 + n) (the last 4096 steps are
+ * kept); host output.  Syncs. */
+GSQ_API int gsq_loss_history(gsq_ctx* ctx, uint64_t t0, int64_t n, double* host_out);
+
+/* gsq_packed_bytes -- bytes of the packed code stream for an N x K layer:
+ * N * K * b / 8 with b = 2 (2-bit, ternary) or 3 (3-bit).  Host only. */
+GSQ_API int gsq_packed_bytes(int grid_mode, int64_t N, int64_t K, size_t* bytes);
+
+/*
+ * gsq_harden_pack -- A6: hard level = argmax of the logits (first maximum,
+ * no noise; 3-bit: clamp(i0 + argmax - 2, 0, 7); ternary: zero if the mask
+ * pair prefers zero, else the sign pair's choice), packed as an LSB-first
+ * bitstream per row of 32-bit little-endian words (code j of a row at bits
+ * [j b, j b + b)); the code is the level index (ternary: v + 1).
+ *   packed      gsq_packed_bytes() bytes, host or device.
+ *   scales_f16  N x G binary16 (round to nearest even), host or device,
+ *               nullable.
+ *   scales_f32  N x G fp32, host or device, nullable.
+ * Syncs.
+ */
+GSQ_API int gsq_harden_pack(gsq_ctx* ctx, void* packed, uint16_t* scales_f16,
+                    float* scales_f32);
+
+/*
+ * gsq_recon_error -- A7: abs = || bf16(X) Wq^T - Y_ref ||_F^2 and
+ * rel = abs / || Y_ref ||_F^2 with Wq the hard weight (GSQ_RECON_HARD) or
+ * the noiseless soft weight at tau (GSQ_RECON_SOFT; tau ignored for hard).
+ * Syncs.  Leaves the optimiser state untouched.
+ */
+GSQ_API int gsq_recon_error(gsq_ctx* ctx, int mode, float tau, double* abs_err,
+                    double* rel_err);
+
+/* Checkpoint: logits, momenta, scales, scale momenta, step counter.  The
+ * noise is a pure function of (seed, t, coord), so resuming is bit-exact.
+ * gsq_state_bytes gives the size; buffers are host memory.  Sync. */
+GSQ_API int gsq_state_bytes(gsq_ctx* ctx, size_t* bytes);
+GSQ_API int gsq_export_state(gsq_ctx* ctx, void* host_buf, size_t bytes);
+GSQ_API int gsq_import_state(gsq_ctx* ctx, const void* host_buf, size_t bytes);
+
+/* step counter t (the Philox counter word of the next step) */
+GSQ_API int gsq_get_step(gsq_ctx* ctx, uint64_t* t);
+
+/* gsq_destroy -- frees the context (syncs its stream).  NULL is a no-op. */
+GSQ_API int gsq_destroy(gsq_ctx* ctx);
+
+/* static string for a status code */
+GSQ_API const char* gsq_error_string(int status);
+
+/* ---------------------------------------------------------- measurement --
+ * gsq_set_timing(ctx, on): record CUDA events on the context stream around
+ * each phase of gsq_step.  gsq_phase_times(ctx, ms[4], launches[4]) returns
+ * and resets the accumulated milliseconds and launch counts of phases
+ * 0 soft weight, 1 forward GEMM + loss, 2 weight-gradient GEMM,
+ * 3 backward + Lion.  Syncs. */
+GSQ_API int gsq_set_timing(gsq_ctx* ctx, int on);
+GSQ_API int gsq_phase_times(gsq_ctx* ctx, double* ms, int64_t* launches);
+
+/* ------------------------------------------------------------- testing --
+ * These expose internal buffers and single phases so tests can compare each
+ * phase with an independent implementation on identical inputs.
+ *
+ * gsq_debug_uniforms: the L Philox uniforms of coords [coord0, coord0+count)
+ *   at step t, coordinate-major, into host memory.  Syncs.
+ * gsq_debug_get / gsq_debug_set: copy an internal buffer to / from host
+ *   memory; bytes must equal the buffer size.  Syncs.  Buffers:          */
+enum {
+    GSQ_DBG_LOGITS = 0,  /* L x N x K fp32 (planar)            */
+    GSQ_DBG_MOM = 1,     /* L x N x K fp32                     */
+    GSQ_DBG_SCALES = 2,  /* N x G fp32                         */
+    GSQ_DBG_SMOM = 3,    /* N x G fp32                         */
+    GSQ_DBG_I0 = 4,      /* N x K int8 initial level           */
+    GSQ_DBG_WHAT = 5,    /* N x K bf16 soft weight             */
+    GSQ_DBG_WSOFT32 = 6, /* N x K fp32 soft weight before rounding (filled
+                            by gsq_debug_soft_weight)           */
+    GSQ_DBG_DW = 7,      /* N x K fp32 weight gradient         */
+    GSQ_DBG_DYT = 8,     /* N x Tp bf16 output gradient (transposed, Tp =
+                            T rounded up to 64)                */
+    GSQ_DBG_YREFT = 9,   /* N x Tp fp32 reference output (transposed) */
+    GSQ_DBG_DL = 10,     /* L x N x K fp32 logit gradient (filled by
+                            gsq_debug_backward)                 */
+    GSQ_DBG_DS = 11      /* N x G fp32 scale gradient (ditto)   */
+};
+GSQ_API int gsq_debug_uniforms(gsq_ctx* ctx, uint32_t t, uint64_t coord0,
+                       int64_t count, float* host_out);
+GSQ_API int gsq_debug_get(gsq_ctx* ctx, int which, void* host, size_t bytes);
+GSQ_API int gsq_debug_set(gsq_ctx* ctx, int which, const void* host, size_t bytes);
+/* noise on (default) / off; off sets g = 0 */
+GSQ_API int gsq_debug_noise(gsq_ctx* ctx, int on);
+/* single phases at the current t (t is not advanced):
+ *   soft weight (also fills GSQ_DBG_WSOFT32), forward GEMM + loss (loss
+ *   returned, syncs), weight-gradient GEMM, backward + Lion from the
+ *   current dW (also fills GSQ_DBG_DL / GSQ_DBG_DS). */
+GSQ_API int gsq_debug_soft_weight(gsq_ctx* ctx, float tau);
+GSQ_API int gsq_debug_forward(gsq_ctx* ctx, double* loss);
+GSQ_API int gsq_debug_weight_grad(gsq_ctx* ctx);
+GSQ_API int gsq_debug_backward(gsq_ctx* ctx, float tau, float lr, float beta1,
+                       float beta2);
+
+/*
+ * gsq_gemm_bf16_abt -- the library's tcgen05 GEMM on its own:
+ * C (M x N fp32, row-major, ldc = N) = A (M x Kc bf16, row-major) .
+ * B (N x Kc bf16, row-major)^T with fp32 accumulation; device pointers,
+ * 16-byte aligned, Kc % 8 == 0.  Enqueued on `stream`; syncs.
+ */
+GSQ_API int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
+                      int64_t N, int64_t Kc, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GSQ_H */

@@ -1,0 +1,95 @@
+// gsq_internal.h -- launchers shared by the translation units of libgsq.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gsq {
+
+// device-side error codes written into the context's error word
+enum : int {
+  DEV_OK = 0,
+  DEV_ERR_TIMEOUT = 1,    // a bounded mbarrier wait gave up
+  DEV_ERR_NONFINITE = 2,  // NaN / Inf in an input or a loss
+  DEV_ERR_BAD_INIT = 3    // init_idx out of the grid's range
+};
+
+// ---------------------------------------------------------------- GEMM
+enum EpiMode : int {
+  EPI_STORE_F32 = 0,  // C = acc (fp32 store)
+  EPI_LOSS_DY = 1,    // E = acc - Yref; loss += sum E^2; dY = bf16(2E)
+  EPI_LOSS = 2        // E = acc - Yref; loss += sum E^2
+};
+
+struct EpiParams {
+  float* out;            // EPI_STORE_F32: M x ldo
+  int64_t ldo;
+  const float* yref;     // EPI_LOSS*: M x ldy
+  int64_t ldy;
+  __nv_bfloat16* dy;     // EPI_LOSS_DY: M x lddy
+  int64_t lddy;
+  double* partials;      // one slot per CTA
+  unsigned* ticket;      // zero between launches
+  double* loss_out;      // final loss (fp64)
+  int* err;              // device error word
+};
+
+// Encodes a 2-D bf16 tensor map (rows x cols, row stride ld elements) with
+// a box of box_rows x 64 elements and 128-byte swizzling.
+int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows,
+                   int64_t cols, int64_t ld, int box_rows);
+
+// C[M x N] = A[M x Kc] . B[N x Kc]^T with the epilogue selected by `mode`;
+// tmA / tmB made by make_tmap_bf16 with box rows 128 (A) and 256 (B).
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        int64_t M, int64_t N, int64_t Kc, int mode,
+                        const EpiParams& ep, int sm_count, cudaStream_t st);
+
+// ------------------------------------------------------- elementwise
+struct StepArgs {
+  int mode;
+  int64_t N, K, G;
+  const float* logits;   // L x N x K
+  float* logits_w;       // same buffer, written by the backward
+  float* mom;
+  float* s;
+  float* ms;
+  const int8_t* i0;
+  uint64_t seed;
+  uint32_t t;
+  int noise;
+  float tau;
+};
+
+cudaError_t launch_convert_x(const void* X, int dtype, int64_t T, int64_t K,
+                             int64_t Tp, __nv_bfloat16* Xb, __nv_bfloat16* Xt,
+                             __nv_bfloat16* Xcat, int* err, cudaStream_t st);
+cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
+                             float* W32, __nv_bfloat16* Wop, int split,
+                             int* err, cudaStream_t st);
+cudaError_t launch_init_state(int mode, const float* W32, const int8_t* init_idx,
+                              int64_t N, int64_t K, float* s, int8_t* i0,
+                              float* logits, int* err, cudaStream_t st);
+cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
+                               float* wsoft32, int sm_count, cudaStream_t st);
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr,
+                                 float b1, float b2, float* dl_dbg,
+                                 float* ds_dbg, int sm_count, cudaStream_t st);
+cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
+                               const float* logits, const float* s,
+                               const int8_t* i0, __nv_bfloat16* What,
+                               cudaStream_t st);
+cudaError_t launch_harden_pack(int mode, int64_t N, int64_t K,
+                               const float* logits, const int8_t* i0,
+                               uint32_t* packed, cudaStream_t st);
+cudaError_t launch_export_scales(const float* s, int64_t n, uint16_t* f16,
+                                 float* f32, cudaStream_t st);
+cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
+                            uint64_t coord0, int64_t count, float* out,
+                            cudaStream_t st);
+cudaError_t launch_sumsq(const float* x, int64_t n, double* partials,
+                         unsigned* ticket, double* out, cudaStream_t st);
+
+}  // namespace gsq

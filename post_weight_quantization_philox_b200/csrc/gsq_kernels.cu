@@ -1,0 +1,718 @@
+// gsq_kernels.cu -- the bandwidth-bound kernels of the GSQ step:
+//   init (operand conversion, scales, initial level, logits),
+//   soft weight (Philox Gumbel noise + tempered softmax + dequantisation),
+//   backward (softmax-Jacobian logit gradients, group-scale gradient by warp
+//   shuffle over the 128-wide group, Lion in place),
+//   harden + pack, scale export, and small reductions.
+// Method: GSQ (arXiv 2604.18556), method and optimisation paragraphs of the
+// agihunt.info summary; Approach section on atlas.scime.ai.
+#include "gsq_device.cuh"
+#include "gsq_internal.h"
+
+namespace gsq {
+
+namespace {
+
+constexpr int kGroup = 128;
+
+__device__ __forceinline__ void set_err(int* err, int code) {
+  atomicCAS(err, 0, code);
+}
+
+// ------------------------------------------------------------ conversion
+
+// X (T x K, fp32 or bf16) -> Xb (Tp x K bf16, row-major) and
+// Xt (K x Tp bf16, transposed); optional Xcat (Tp x 2K) = [Xb | Xb] for the
+// split-precision reference GEMM.  64 x 64 tiles through shared memory.
+__global__ void k_convert_x(const void* __restrict__ X, int dtype, int64_t T,
+                            int64_t K, int64_t Tp, __nv_bfloat16* __restrict__ Xb,
+                            __nv_bfloat16* __restrict__ Xt,
+                            __nv_bfloat16* __restrict__ Xcat, int* err) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int64_t t0 = (int64_t)blockIdx.y * 64, k0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 64 x 4
+  bool bad = false;
+  for (int r = ty; r < 64; r += 4) {
+    const int64_t t = t0 + r, k = k0 + tx;
+    float v = 0.f;
+    if (t < T && k < K) {
+      v = dtype == 0 ? ((const float*)X)[t * K + k]
+                     : __bfloat162float(((const __nv_bfloat16*)X)[t * K + k]);
+      bad |= !isfinite(v);
+    }
+    const __nv_bfloat16 b = __float2bfloat16_rn(v);
+    tile[r][tx] = b;
+    if (t < Tp && k < K) {
+      Xb[t * K + k] = b;
+      if (Xcat) {
+        Xcat[t * 2 * K + k] = b;
+        Xcat[t * 2 * K + K + k] = b;
+      }
+    }
+  }
+  if (bad) set_err(err, DEV_ERR_NONFINITE);
+  __syncthreads();
+  for (int r = ty; r < 64; r += 4) {
+    const int64_t k = k0 + r, t = t0 + tx;
+    if (k < K && t < Tp) Xt[k * Tp + t] = tile[tx][r];
+  }
+}
+
+// W (N x K, fp32 or bf16) -> W32 (fp32 copy for init) and the reference-GEMM
+// operand: bf16 W (split = 0) or [hi | lo] (N x 2K) with hi = bf16(W),
+// lo = bf16(W - hi) (split = 1), so that hi + lo carries ~16 bits of W.
+__global__ void k_convert_w(const void* __restrict__ W, int dtype, int64_t N,
+                            int64_t K, float* __restrict__ W32,
+                            __nv_bfloat16* __restrict__ Wop, int split,
+                            int* err) {
+  const int64_t n_el = N * K;
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float w = dtype == 0
+                        ? ((const float*)W)[i]
+                        : __bfloat162float(((const __nv_bfloat16*)W)[i]);
+    bad |= !isfinite(w);
+    W32[i] = w;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    if (split) {
+      const int64_t n = i / K, k = i % K;
+      Wop[n * 2 * K + k] = hi;
+      Wop[n * 2 * K + K + k] = __float2bfloat16_rn(w - __bfloat162float(hi));
+    } else {
+      Wop[i] = hi;
+    }
+  }
+  if (bad) set_err(err, DEV_ERR_NONFINITE);
+}
+
+// ------------------------------------------------------------------ init
+
+// One warp per group of 128: s = absmax / c_max; initial level by
+// round-to-nearest of w / s (first level on ties, s = 0 -> w / s := 0) or
+// from init_idx; logits +2 on the initial slot.  All comparisons in fp32.
+template <int MODE>
+__global__ void k_init_state(const float* __restrict__ W32,
+                             const int8_t* __restrict__ init_idx, int64_t N,
+                             int64_t K, float* __restrict__ s,
+                             int8_t* __restrict__ i0,
+                             float* __restrict__ logits, int* err) {
+  using Gr = GridT<MODE>;
+  const int64_t G = K / kGroup, NK = N * K;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t gi = warp; gi < N * G; gi += nwarps) {
+    const int64_t n = gi / G, g = gi % G;
+    const int64_t base = n * K + g * kGroup + lane * 4;
+    float w[4];
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      w[j] = W32[base + j];
+      amax = fmaxf(amax, fabsf(w[j]));
+    }
+    amax = warp_max(amax);
+    const float sg = amax / Gr::CMAX;
+    if (lane == 0) s[gi] = sg;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t c = base + j;
+      int lev;
+      if (init_idx) {
+        lev = init_idx[c];
+        if (lev < 0 || lev >= Gr::LEVELS) {
+          set_err(err, DEV_ERR_BAD_INIT);
+          lev = 0;
+        }
+      } else {
+        const float q = sg > 0.f ? w[j] / sg : 0.f;
+        lev = 0;
+        float best = fabsf(q - Gr::level(0));
+#pragma unroll
+        for (int l = 1; l < Gr::LEVELS; ++l) {
+          const float d = fabsf(q - Gr::level(l));
+          if (d < best) {
+            best = d;
+            lev = l;
+          }
+        }
+      }
+      i0[c] = (int8_t)lev;
+      float lg[Gr::L];
+#pragma unroll
+      for (int p = 0; p < Gr::L; ++p) lg[p] = 0.f;
+      if (MODE == GRID_2BIT) {
+#pragma unroll
+        for (int p = 0; p < Gr::L; ++p) lg[p] = (p == lev) ? 2.f : 0.f;
+      } else if (MODE == GRID_3BIT_LOCAL) {
+        lg[2] = 2.f;  // shift 0
+      } else {
+        // ternary: mask (zero, nonzero), sign (minus, plus); sign of w when
+        // the initial level is zero (w = 0 counts as plus)
+        const bool nonzero = lev != 1;
+        const bool plus = (lev == 2) || (lev == 1 && !(w[j] < 0.f));
+        lg[nonzero ? 1 : 0] = 2.f;
+        lg[plus ? 3 : 2] = 2.f;
+      }
+#pragma unroll
+      for (int p = 0; p < Gr::L; ++p) logits[p * NK + c] = lg[p];
+    }
+  }
+}
+
+// ----------------------------------------------------- soft weight (A1+A2)
+
+// Per coordinate: probabilities y and unit value v from logits l, noise g
+// and 1/tau.  Categorical modes use candidate values cand[]; ternary forms
+// v = p1 (q+ - q-).
+template <int MODE>
+__device__ __forceinline__ float coord_soft(const float* l, const float* g,
+                                            float inv_tau, const float* cand,
+                                            float* y) {
+  constexpr int L = GridT<MODE>::L;
+  float z[L];
+#pragma unroll
+  for (int k = 0; k < L; ++k) z[k] = (l[k] + g[k]) * inv_tau;
+  if (MODE == GRID_TERNARY) {
+    const float m0 = fmaxf(z[0], z[1]);
+    const float e0 = __expf(z[0] - m0), e1 = __expf(z[1] - m0);
+    const float r0 = 1.f / (e0 + e1);
+    y[0] = e0 * r0;
+    y[1] = e1 * r0;
+    const float m1 = fmaxf(z[2], z[3]);
+    const float e2 = __expf(z[2] - m1), e3 = __expf(z[3] - m1);
+    const float r1 = 1.f / (e2 + e3);
+    y[2] = e2 * r1;
+    y[3] = e3 * r1;
+    return y[1] * (y[3] - y[2]);
+  } else {
+    float zm = z[0];
+#pragma unroll
+    for (int k = 1; k < L; ++k) zm = fmaxf(zm, z[k]);
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < L; ++k) {
+      y[k] = __expf(z[k] - zm);
+      sum += y[k];
+    }
+    const float r = 1.f / sum;
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < L; ++k) {
+      y[k] *= r;
+      v = fmaf(y[k], cand[k], v);
+    }
+    return v;
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void candidates(int lev0, float* cand) {
+  if (MODE == GRID_2BIT) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cand[k] = (float)k - 1.5f;
+  } else if (MODE == GRID_3BIT_LOCAL) {
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const int j = min(max(lev0 + k - 2, 0), 7);
+      cand[k] = (float)j - 3.5f;
+    }
+  }
+}
+
+// Four consecutive coordinates per thread (128-bit loads per logit plane).
+template <int MODE, bool DBG>
+__global__ void __launch_bounds__(256) k_soft_weight(
+    const float* __restrict__ logits, const float* __restrict__ s,
+    const int8_t* __restrict__ i0, int64_t N, int64_t K, uint32_t k0,
+    uint32_t k1, uint32_t t, int noise, float inv_tau,
+    __nv_bfloat16* __restrict__ What, float* __restrict__ wsoft32) {
+  constexpr int L = GridT<MODE>::L;
+  const int64_t NK = N * K, G = K / kGroup, n4 = NK / 4;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c0 = q * 4;
+    const int64_t n = c0 / K, k = c0 - n * K;
+    const float sg = __ldg(s + n * G + k / kGroup);
+    float4 lp[L];
+#pragma unroll
+    for (int p = 0; p < L; ++p)
+      lp[p] = __ldg(reinterpret_cast<const float4*>(logits + p * NK + c0));
+    char4 iv = make_char4(0, 0, 0, 0);
+    if (MODE == GRID_3BIT_LOCAL)
+      iv = __ldg(reinterpret_cast<const char4*>(i0 + c0));
+    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
+    float wv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[L], g[5], y[L], cand[5];
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
+      if (noise) {
+        coord_noise5((uint64_t)(c0 + j), t, k0, k1, L == 5, g);
+      } else {
+#pragma unroll
+        for (int p = 0; p < 5; ++p) g[p] = 0.f;
+      }
+      candidates<MODE>(lev0[j], cand);
+      const float v = coord_soft<MODE>(l, g, inv_tau, cand, y);
+      wv[j] = sg * v;
+    }
+    __nv_bfloat162 b01 = __floats2bfloat162_rn(wv[0], wv[1]);
+    __nv_bfloat162 b23 = __floats2bfloat162_rn(wv[2], wv[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&b01);
+    pk.y = *reinterpret_cast<uint32_t*>(&b23);
+    *reinterpret_cast<uint2*>(What + c0) = pk;
+    if (DBG)
+      *reinterpret_cast<float4*>(wsoft32 + c0) =
+          make_float4(wv[0], wv[1], wv[2], wv[3]);
+  }
+}
+
+// ------------------------------------------------- backward + Lion (A5)
+
+// One warp per group of 128 coordinates, four per lane.  Recomputes the
+// step's probabilities from the same Philox counters, forms
+//   a = s dW / tau,  dl_k = a y_k sum_j y_j (c_k - c_j)   (categorical),
+//   dl_mask1 = a (q+ - q-) p1 p0 = -dl_mask0, dl_sign+ = 2 a p1 q+ q- =
+//   -dl_sign- (ternary),  ds = sum over the group of dW v (warp shuffle),
+// then applies Lion to the logits and, on lane 0, to the group scale.
+template <int MODE, bool DBG>
+__global__ void __launch_bounds__(256) k_backward_lion(
+    float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ s,
+    float* __restrict__ ms, const int8_t* __restrict__ i0,
+    const float* __restrict__ dW, int64_t N, int64_t K, uint32_t k0,
+    uint32_t k1, uint32_t t, int noise, float inv_tau, float lr, float b1,
+    float omb1, float b2, float omb2, float* __restrict__ dl_dbg,
+    float* __restrict__ ds_dbg) {
+  constexpr int L = GridT<MODE>::L;
+  const int64_t NK = N * K, G = K / kGroup;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t gi = warp; gi < N * G; gi += nwarps) {
+    const int64_t n = gi / G, g = gi - n * G;
+    const int64_t c0 = n * K + g * kGroup + lane * 4;
+    const float sg = s[gi];
+    const float4 dw4 = __ldg(reinterpret_cast<const float4*>(dW + c0));
+    float4 lp[L], mp[L];
+#pragma unroll
+    for (int p = 0; p < L; ++p) {
+      lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
+      mp[p] = *reinterpret_cast<const float4*>(mom + p * NK + c0);
+    }
+    char4 iv = make_char4(0, 0, 0, 0);
+    if (MODE == GRID_3BIT_LOCAL)
+      iv = __ldg(reinterpret_cast<const char4*>(i0 + c0));
+    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
+    const float dwv[4] = {dw4.x, dw4.y, dw4.z, dw4.w};
+    float ds_part = 0.f;
+    float lo[L][4], mo[L][4], dlo[L][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[L], m[L], gz[5], y[L], cand[5];
+#pragma unroll
+      for (int p = 0; p < L; ++p) {
+        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
+        m[p] = j == 0 ? mp[p].x : j == 1 ? mp[p].y : j == 2 ? mp[p].z : mp[p].w;
+      }
+      if (noise) {
+        coord_noise5((uint64_t)(c0 + j), t, k0, k1, L == 5, gz);
+      } else {
+#pragma unroll
+        for (int p = 0; p < 5; ++p) gz[p] = 0.f;
+      }
+      candidates<MODE>(lev0[j], cand);
+      const float v = coord_soft<MODE>(l, gz, inv_tau, cand, y);
+      ds_part = fmaf(dwv[j], v, ds_part);
+      const float a = sg * dwv[j] * inv_tau;
+      float dl[L];
+      if (MODE == GRID_TERNARY) {
+        const float gm = a * (y[3] - y[2]) * y[1] * y[0];
+        const float gs = 2.f * a * y[1] * y[3] * y[2];
+        dl[0] = -gm;
+        dl[1] = gm;
+        dl[2] = -gs;
+        dl[3] = gs;
+      } else {
+#pragma unroll
+        for (int p = 0; p < L; ++p) {
+          float acc = 0.f;
+#pragma unroll
+          for (int q = 0; q < L; ++q) acc = fmaf(y[q], cand[p] - cand[q], acc);
+          dl[p] = a * y[p] * acc;
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < L; ++p) {
+        float th = l[p], mm = m[p];
+        lion_update(th, mm, dl[p], lr, b1, omb1, b2, omb2);
+        lo[p][j] = th;
+        mo[p][j] = mm;
+        dlo[p][j] = dl[p];
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < L; ++p) {
+      *reinterpret_cast<float4*>(logits + p * NK + c0) =
+          make_float4(lo[p][0], lo[p][1], lo[p][2], lo[p][3]);
+      *reinterpret_cast<float4*>(mom + p * NK + c0) =
+          make_float4(mo[p][0], mo[p][1], mo[p][2], mo[p][3]);
+      if (DBG)
+        *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
+            make_float4(dlo[p][0], dlo[p][1], dlo[p][2], dlo[p][3]);
+    }
+    const float ds = warp_sum(ds_part);
+    if (lane == 0) {
+      float th = sg, mm = ms[gi];
+      lion_update(th, mm, ds, lr, b1, omb1, b2, omb2);
+      s[gi] = th;
+      ms[gi] = mm;
+      if (DBG) ds_dbg[gi] = ds;
+    }
+  }
+}
+
+// ---------------------------------------------------- harden + pack (A6)
+
+template <int MODE>
+__device__ __forceinline__ int hard_level(const float* l, int lev0) {
+  if (MODE == GRID_TERNARY) {
+    const bool nonzero = l[1] > l[0];  // first maximum: ties -> zero
+    const bool plus = l[3] > l[2];     // ties -> minus
+    return nonzero ? (plus ? 2 : 0) : 1;
+  }
+  constexpr int L = GridT<MODE>::L;
+  int best = 0;
+#pragma unroll
+  for (int k = 1; k < L; ++k)
+    if (l[k] > l[best]) best = k;
+  if (MODE == GRID_3BIT_LOCAL) return min(max(lev0 + best - 2, 0), 7);
+  return best;
+}
+
+// 2-bit / ternary: 16 codes -> one 32-bit word per thread.
+// 3-bit: 32 codes -> three 32-bit words per thread.  Codes never straddle
+// rows because K is a multiple of 128.
+template <int MODE>
+__global__ void __launch_bounds__(256) k_harden_pack(
+    const float* __restrict__ logits, const int8_t* __restrict__ i0,
+    int64_t N, int64_t K, uint32_t* __restrict__ packed) {
+  constexpr int L = GridT<MODE>::L;
+  constexpr int CPT = (MODE == GRID_3BIT_LOCAL) ? 32 : 16;  // codes / thread
+  const int64_t NK = N * K, nthr = NK / CPT;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nthr;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c0 = q * CPT;
+    uint32_t w[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int j4 = 0; j4 < CPT / 4; ++j4) {
+      float4 lp[L];
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        lp[p] = __ldg(reinterpret_cast<const float4*>(logits + p * NK + c0 + j4 * 4));
+      char4 iv = make_char4(0, 0, 0, 0);
+      if (MODE == GRID_3BIT_LOCAL)
+        iv = __ldg(reinterpret_cast<const char4*>(i0 + c0 + j4 * 4));
+      const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float l[L];
+#pragma unroll
+        for (int p = 0; p < L; ++p)
+          l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
+        const uint32_t code = (uint32_t)hard_level<MODE>(l, lev0[j]);
+        const int idx = j4 * 4 + j;
+        if (MODE == GRID_3BIT_LOCAL) {
+          const int bit = idx * 3;
+          w[bit >> 5] |= code << (bit & 31);
+          if ((bit & 31) > 29) w[(bit >> 5) + 1] |= code >> (32 - (bit & 31));
+        } else {
+          w[0] |= code << (idx * 2);
+        }
+      }
+    }
+    if (MODE == GRID_3BIT_LOCAL) {
+      packed[q * 3 + 0] = w[0];
+      packed[q * 3 + 1] = w[1];
+      packed[q * 3 + 2] = w[2];
+    } else {
+      packed[q] = w[0];
+    }
+  }
+}
+
+// bf16(s * level) of the hard choice, four coordinates per thread
+template <int MODE>
+__global__ void __launch_bounds__(256) k_hard_weight(
+    const float* __restrict__ logits, const float* __restrict__ s,
+    const int8_t* __restrict__ i0, int64_t N, int64_t K,
+    __nv_bfloat16* __restrict__ What) {
+  constexpr int L = GridT<MODE>::L;
+  const int64_t NK = N * K, G = K / kGroup, n4 = NK / 4;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c0 = q * 4;
+    const int64_t n = c0 / K, k = c0 - n * K;
+    const float sg = s[n * G + k / kGroup];
+    float4 lp[L];
+#pragma unroll
+    for (int p = 0; p < L; ++p)
+      lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
+    char4 iv = make_char4(0, 0, 0, 0);
+    if (MODE == GRID_3BIT_LOCAL) iv = *reinterpret_cast<const char4*>(i0 + c0);
+    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
+    float wv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[L];
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
+      wv[j] = sg * GridT<MODE>::level(hard_level<MODE>(l, lev0[j]));
+    }
+    __nv_bfloat162 b01 = __floats2bfloat162_rn(wv[0], wv[1]);
+    __nv_bfloat162 b23 = __floats2bfloat162_rn(wv[2], wv[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&b01);
+    pk.y = *reinterpret_cast<uint32_t*>(&b23);
+    *reinterpret_cast<uint2*>(What + c0) = pk;
+  }
+}
+
+__global__ void k_export_scales(const float* __restrict__ s, int64_t n,
+                                uint16_t* __restrict__ f16,
+                                float* __restrict__ f32) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = s[i];
+    if (f16) {
+      const __half h = __float2half_rn(v);
+      f16[i] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+    if (f32) f32[i] = v;
+  }
+}
+
+template <int MODE>
+__global__ void k_uniforms(uint64_t seed, uint32_t t, uint64_t coord0,
+                           int64_t count, float* __restrict__ out) {
+  constexpr int L = GridT<MODE>::L;
+  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t c = coord0 + (uint64_t)i;
+    const uint4 r = philox4x32_10(
+        make_uint4((uint32_t)c, (uint32_t)(c >> 32), t, 0u), k0, k1);
+    out[i * L + 0] = word_to_unit(r.x);
+    out[i * L + 1] = word_to_unit(r.y);
+    out[i * L + 2] = word_to_unit(r.z);
+    out[i * L + 3] = word_to_unit(r.w);
+    if (L == 5) {
+      const uint4 r2 = philox4x32_10(
+          make_uint4((uint32_t)c, (uint32_t)(c >> 32), t, 1u), k0, k1);
+      out[i * L + 4] = word_to_unit(r2.x);
+    }
+  }
+}
+
+// sum of squares with per-block fp64 partials; the last block to finish
+// adds the partials in block order (deterministic) and resets the ticket.
+__global__ void __launch_bounds__(256) k_sumsq(const float* __restrict__ x,
+                                               int64_t n,
+                                               double* __restrict__ partials,
+                                               unsigned* ticket,
+                                               double* __restrict__ out) {
+  __shared__ double red[8];
+  __shared__ bool last;
+  double acc = 0.0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const double v = x[i];
+    acc += v * v;
+  }
+  acc = warp_sum_d(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b += red[w];
+    partials[blockIdx.x] = b;
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    double tot = 0.0;
+    for (unsigned b = 0; b < gridDim.x; ++b)
+      tot += *((volatile double*)partials + b);
+    *out = tot;
+    *ticket = 0u;
+  }
+}
+
+int grid_for(int64_t work, int threads, int cap) {
+  int64_t b = (work + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > cap) b = cap;
+  return (int)b;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ launchers
+
+cudaError_t launch_convert_x(const void* X, int dtype, int64_t T, int64_t K,
+                             int64_t Tp, __nv_bfloat16* Xb, __nv_bfloat16* Xt,
+                             __nv_bfloat16* Xcat, int* err, cudaStream_t st) {
+  dim3 grid((unsigned)((K + 63) / 64), (unsigned)((Tp + 63) / 64));
+  k_convert_x<<<grid, dim3(64, 4), 0, st>>>(X, dtype, T, K, Tp, Xb, Xt, Xcat,
+                                            err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
+                             float* W32, __nv_bfloat16* Wop, int split,
+                             int* err, cudaStream_t st) {
+  k_convert_w<<<grid_for(N * K, 256, 4096), 256, 0, st>>>(W, dtype, N, K, W32,
+                                                          Wop, split, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_init_state(int mode, const float* W32,
+                              const int8_t* init_idx, int64_t N, int64_t K,
+                              float* s, int8_t* i0, float* logits, int* err,
+                              cudaStream_t st) {
+  const int64_t groups = N * (K / kGroup);
+  const int blocks = grid_for(groups * 32, 256, 8192);
+  switch (mode) {
+    case GRID_2BIT:
+      k_init_state<GRID_2BIT><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s,
+                                                       i0, logits, err);
+      break;
+    case GRID_TERNARY:
+      k_init_state<GRID_TERNARY><<<blocks, 256, 0, st>>>(W32, init_idx, N, K,
+                                                          s, i0, logits, err);
+      break;
+    default:
+      k_init_state<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(
+          W32, init_idx, N, K, s, i0, logits, err);
+  }
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static void soft_weight_mode(const StepArgs& a, __nv_bfloat16* What,
+                             float* wsoft32, int blocks, cudaStream_t st) {
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+  const float inv_tau = 1.0f / a.tau;
+  if (wsoft32)
+    k_soft_weight<MODE, true><<<blocks, 256, 0, st>>>(
+        a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
+        wsoft32);
+  else
+    k_soft_weight<MODE, false><<<blocks, 256, 0, st>>>(
+        a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
+        nullptr);
+}
+
+cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
+                               float* wsoft32, int sm_count, cudaStream_t st) {
+  const int blocks = grid_for(a.N * a.K / 4, 256, sm_count * 8);
+  switch (a.mode) {
+    case GRID_2BIT: soft_weight_mode<GRID_2BIT>(a, What, wsoft32, blocks, st); break;
+    case GRID_TERNARY: soft_weight_mode<GRID_TERNARY>(a, What, wsoft32, blocks, st); break;
+    default: soft_weight_mode<GRID_3BIT_LOCAL>(a, What, wsoft32, blocks, st);
+  }
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static void backward_mode(const StepArgs& a, const float* dW, float lr,
+                          float b1, float b2, float* dl_dbg, float* ds_dbg,
+                          int blocks, cudaStream_t st) {
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+  const float inv_tau = 1.0f / a.tau;
+  const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
+  if (dl_dbg)
+    k_backward_lion<MODE, true><<<blocks, 256, 0, st>>>(
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, a.N, a.K, k0, k1, a.t, a.noise,
+        inv_tau, lr, b1, omb1, b2, omb2, dl_dbg, ds_dbg);
+  else
+    k_backward_lion<MODE, false><<<blocks, 256, 0, st>>>(
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, a.N, a.K, k0, k1, a.t, a.noise,
+        inv_tau, lr, b1, omb1, b2, omb2, nullptr, nullptr);
+}
+
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr,
+                                 float b1, float b2, float* dl_dbg,
+                                 float* ds_dbg, int sm_count,
+                                 cudaStream_t st) {
+  const int64_t groups = a.N * (a.K / kGroup);
+  const int blocks = grid_for(groups * 32, 256, sm_count * 8);
+  switch (a.mode) {
+    case GRID_2BIT: backward_mode<GRID_2BIT>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st); break;
+    case GRID_TERNARY: backward_mode<GRID_TERNARY>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st); break;
+    default: backward_mode<GRID_3BIT_LOCAL>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
+                               const float* logits, const float* s,
+                               const int8_t* i0, __nv_bfloat16* What,
+                               cudaStream_t st) {
+  const int blocks = grid_for(N * K / 4, 256, 4096);
+  switch (mode) {
+    case GRID_2BIT: k_hard_weight<GRID_2BIT><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
+    case GRID_TERNARY: k_hard_weight<GRID_TERNARY><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
+    default: k_hard_weight<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_harden_pack(int mode, int64_t N, int64_t K,
+                               const float* logits, const int8_t* i0,
+                               uint32_t* packed, cudaStream_t st) {
+  switch (mode) {
+    case GRID_2BIT:
+      k_harden_pack<GRID_2BIT><<<grid_for(N * K / 16, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
+      break;
+    case GRID_TERNARY:
+      k_harden_pack<GRID_TERNARY><<<grid_for(N * K / 16, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
+      break;
+    default:
+      k_harden_pack<GRID_3BIT_LOCAL><<<grid_for(N * K / 32, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_export_scales(const float* s, int64_t n, uint16_t* f16,
+                                 float* f32, cudaStream_t st) {
+  k_export_scales<<<grid_for(n, 256, 1024), 256, 0, st>>>(s, n, f16, f32);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
+                            uint64_t coord0, int64_t count, float* out,
+                            cudaStream_t st) {
+  const int blocks = grid_for(count, 256, 4096);
+  switch (mode) {
+    case GRID_2BIT: k_uniforms<GRID_2BIT><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out); break;
+    case GRID_TERNARY: k_uniforms<GRID_TERNARY><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out); break;
+    default: k_uniforms<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sumsq(const float* x, int64_t n, double* partials,
+                         unsigned* ticket, double* out, cudaStream_t st) {
+  k_sumsq<<<grid_for(n, 256, 1024), 256, 0, st>>>(x, n, partials, ticket, out);
+  return cudaGetLastError();
+}
+
+}  // namespace gsq

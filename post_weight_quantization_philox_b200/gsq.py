@@ -1,0 +1,349 @@
+"""Thin ctypes binding of libgsq (the C ABI in include/gsq.h).
+
+Argument marshalling only: every step of the GSQ reconstruction path runs in
+the library's CUDA kernels.  PyTorch supplies device memory and the current
+stream; numpy arrays are accepted as host buffers.  There is no fallback: if
+the shared library is missing or fails to load, importing raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgsq.so")
+
+GSQ_GRID_2BIT, GSQ_GRID_TERNARY, GSQ_GRID_3BIT_LOCAL = 0, 1, 2
+GSQ_F32, GSQ_BF16 = 0, 1
+GSQ_OK = 0
+GSQ_ERR_INVALID_ARG, GSQ_ERR_CUDA, GSQ_ERR_OOM = -1, -2, -3
+GSQ_ERR_NONFINITE, GSQ_ERR_STATE, GSQ_ERR_UNSUPPORTED, GSQ_ERR_TIMEOUT = -4, -5, -6, -7
+GSQ_RECON_HARD, GSQ_RECON_SOFT = 0, 1
+(GSQ_DBG_LOGITS, GSQ_DBG_MOM, GSQ_DBG_SCALES, GSQ_DBG_SMOM, GSQ_DBG_I0,
+ GSQ_DBG_WHAT, GSQ_DBG_WSOFT32, GSQ_DBG_DW, GSQ_DBG_DYT, GSQ_DBG_YREFT,
+ GSQ_DBG_DL, GSQ_DBG_DS) = range(12)
+
+NUM_LOGITS = {GSQ_GRID_2BIT: 4, GSQ_GRID_TERNARY: 4, GSQ_GRID_3BIT_LOCAL: 5}
+
+# every symbol include/gsq.h declares (checked by the CPU tests)
+EXPORTS = [
+    "gsq_init", "gsq_step", "gsq_last_loss", "gsq_loss_history",
+    "gsq_packed_bytes", "gsq_harden_pack", "gsq_recon_error",
+    "gsq_state_bytes", "gsq_export_state", "gsq_import_state", "gsq_get_step",
+    "gsq_destroy", "gsq_error_string", "gsq_set_timing", "gsq_phase_times",
+    "gsq_debug_uniforms", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
+    "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
+    "gsq_debug_backward", "gsq_gemm_bf16_abt",
+]
+
+
+class GSQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {error_string(status)} ({status})")
+
+
+_i32, _i64, _u32, _u64 = C.c_int, C.c_int64, C.c_uint32, C.c_uint64
+_f32, _p, _sz = C.c_float, C.c_void_p, C.c_size_t
+_pp = C.POINTER(C.c_void_p)
+
+_SIGS = {
+    "gsq_init": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64, _p],
+    "gsq_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_last_loss": [_p, C.POINTER(C.c_double)],
+    "gsq_loss_history": [_p, _u64, _i64, _p],
+    "gsq_packed_bytes": [_i32, _i64, _i64, C.POINTER(_sz)],
+    "gsq_harden_pack": [_p, _p, _p, _p],
+    "gsq_recon_error": [_p, _i32, _f32, C.POINTER(C.c_double), C.POINTER(C.c_double)],
+    "gsq_state_bytes": [_p, C.POINTER(_sz)],
+    "gsq_export_state": [_p, _p, _sz],
+    "gsq_import_state": [_p, _p, _sz],
+    "gsq_get_step": [_p, C.POINTER(_u64)],
+    "gsq_destroy": [_p],
+    "gsq_error_string": [_i32],
+    "gsq_set_timing": [_p, _i32],
+    "gsq_phase_times": [_p, _p, _p],
+    "gsq_debug_uniforms": [_p, _u32, _u64, _i64, _p],
+    "gsq_debug_get": [_p, _i32, _p, _sz],
+    "gsq_debug_set": [_p, _i32, _p, _sz],
+    "gsq_debug_noise": [_p, _i32],
+    "gsq_debug_soft_weight": [_p, _f32],
+    "gsq_debug_forward": [_p, C.POINTER(C.c_double)],
+    "gsq_debug_weight_grad": [_p],
+    "gsq_debug_backward": [_p, _f32, _f32, _f32, _f32],
+    "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libgsq.so not found at {LIB_PATH}; build it with "
+            "`python -m post_weight_quantization_philox_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    for name, args in _SIGS.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = C.c_char_p if name == "gsq_error_string" else C.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def error_string(status: int) -> str:
+    return _lib.gsq_error_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != GSQ_OK:
+        raise GSQError(status, where)
+
+
+def _ptr_dtype(a):
+    """(pointer, GSQ dtype, keep-alive object) of a numpy array or torch tensor."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            if not a.is_contiguous():
+                a = a.contiguous()
+            if a.dtype == torch.float32:
+                return a.data_ptr(), GSQ_F32, a
+            if a.dtype == torch.bfloat16:
+                return a.data_ptr(), GSQ_BF16, a
+            raise TypeError(f"unsupported tensor dtype {a.dtype}")
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return a.ctypes.data, GSQ_F32, a
+
+
+def _stream_ptr(stream):
+    if stream is not None:
+        return int(getattr(stream, "cuda_stream", stream))
+    import torch
+    if torch.cuda.is_available():
+        return torch.cuda.current_stream().cuda_stream
+    return None
+
+
+def _host_ptr(a):
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.data_ptr()
+    except ImportError:  # pragma: no cover
+        pass
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+# --------------------------------------------------------------- C-ABI names
+
+def gsq_packed_bytes(grid_mode: int, N: int, K: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.gsq_packed_bytes(grid_mode, N, K, C.byref(b)), "gsq_packed_bytes")
+    return b.value
+
+
+def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
+             init_idx=None, seed: int = 0, stream=None) -> "Layer":
+    """W (N x K) and X (T x K): numpy fp32 or torch fp32/bf16, host or device."""
+    wp, wdt, wk = _ptr_dtype(W)
+    xp, xdt, xk = _ptr_dtype(X)
+    N, K = int(W.shape[0]), int(W.shape[1])
+    T = int(X.shape[0])
+    if int(X.shape[1]) != K:
+        raise ValueError("X and W disagree on K")
+    ip, ik = None, None
+    if init_idx is not None:
+        try:
+            import torch
+            if isinstance(init_idx, torch.Tensor):
+                ik = init_idx.to(torch.int8).contiguous()
+                ip = ik.data_ptr()
+        except ImportError:  # pragma: no cover
+            pass
+        if ip is None:
+            ik = np.ascontiguousarray(init_idx, dtype=np.int8)
+            ip = ik.ctypes.data
+    ctx = C.c_void_p()
+    st = _stream_ptr(stream)
+    _check(_lib.gsq_init(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group,
+                         grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
+           "gsq_init")
+    del wk, xk, ik
+    return Layer(ctx, grid_mode, N, K, T, group)
+
+
+def gsq_step(layer: "Layer", tau: float, lr: float, beta1: float = 0.9,
+             beta2: float = 0.99) -> None:
+    _check(_lib.gsq_step(layer.ctx, tau, lr, beta1, beta2), "gsq_step")
+
+
+def gsq_last_loss(layer: "Layer") -> float:
+    v = C.c_double()
+    _check(_lib.gsq_last_loss(layer.ctx, C.byref(v)), "gsq_last_loss")
+    return v.value
+
+
+def gsq_harden_pack(layer: "Layer", packed=None, scales_f16=None,
+                    scales_f32=None):
+    """Into the given buffers (host numpy or device tensors); allocates host
+    numpy outputs when none are given.  Returns (packed, scales_f16, scales_f32)."""
+    if packed is None:
+        packed = np.zeros(gsq_packed_bytes(layer.mode, layer.N, layer.K) // 4,
+                          np.uint32)
+        scales_f16 = np.zeros((layer.N, layer.G), np.uint16)
+        scales_f32 = np.zeros((layer.N, layer.G), np.float32)
+    _check(_lib.gsq_harden_pack(
+        layer.ctx, _host_ptr(packed),
+        None if scales_f16 is None else _host_ptr(scales_f16),
+        None if scales_f32 is None else _host_ptr(scales_f32)), "gsq_harden_pack")
+    return packed, scales_f16, scales_f32
+
+
+def gsq_recon_error(layer: "Layer", mode: int = GSQ_RECON_HARD,
+                    tau: float = 1.0):
+    a, r = C.c_double(), C.c_double()
+    _check(_lib.gsq_recon_error(layer.ctx, mode, tau, C.byref(a), C.byref(r)),
+           "gsq_recon_error")
+    return a.value, r.value
+
+
+def gsq_export_state(layer: "Layer") -> np.ndarray:
+    n = C.c_size_t()
+    _check(_lib.gsq_state_bytes(layer.ctx, C.byref(n)), "gsq_state_bytes")
+    buf = np.zeros(n.value, np.uint8)
+    _check(_lib.gsq_export_state(layer.ctx, buf.ctypes.data, n.value),
+           "gsq_export_state")
+    return buf
+
+
+def gsq_import_state(layer: "Layer", buf: np.ndarray) -> None:
+    buf = np.ascontiguousarray(buf, np.uint8)
+    _check(_lib.gsq_import_state(layer.ctx, buf.ctypes.data, buf.size),
+           "gsq_import_state")
+
+
+def gsq_get_step(layer: "Layer") -> int:
+    t = C.c_uint64()
+    _check(_lib.gsq_get_step(layer.ctx, C.byref(t)), "gsq_get_step")
+    return t.value
+
+
+def gsq_destroy(layer: "Layer") -> None:
+    if layer.ctx:
+        _check(_lib.gsq_destroy(layer.ctx), "gsq_destroy")
+        layer.ctx = None
+
+
+def gsq_set_timing(layer: "Layer", on: bool) -> None:
+    _check(_lib.gsq_set_timing(layer.ctx, int(on)), "gsq_set_timing")
+
+
+def gsq_phase_times(layer: "Layer"):
+    ms = np.zeros(4, np.float64)
+    n = np.zeros(4, np.int64)
+    _check(_lib.gsq_phase_times(layer.ctx, ms.ctypes.data, n.ctypes.data),
+           "gsq_phase_times")
+    return ms, n
+
+
+def gsq_gemm_bf16_abt(A, B, Cout, stream=None) -> None:
+    """Cout (M x N fp32) = A (M x Kc bf16) . B (N x Kc bf16)^T; torch device tensors."""
+    M, Kc = A.shape
+    N = B.shape[0]
+    _check(_lib.gsq_gemm_bf16_abt(A.data_ptr(), B.data_ptr(), Cout.data_ptr(),
+                                  M, N, Kc, _stream_ptr(stream)),
+           "gsq_gemm_bf16_abt")
+
+
+class Layer:
+    """A GSQ context for one linear layer (owner of the C handle)."""
+
+    def __init__(self, ctx, mode, N, K, T, group):
+        self.ctx, self.mode, self.N, self.K, self.T, self.group = ctx, mode, N, K, T, group
+        self.G = K // group
+        self.L = NUM_LOGITS[mode]
+        self.Tp = (T + 63) // 64 * 64
+
+    # debug accessors ---------------------------------------------------
+    _SHAPES = {
+        GSQ_DBG_LOGITS: ("L,N,K", np.float32), GSQ_DBG_MOM: ("L,N,K", np.float32),
+        GSQ_DBG_SCALES: ("N,G", np.float32), GSQ_DBG_SMOM: ("N,G", np.float32),
+        GSQ_DBG_I0: ("N,K", np.int8), GSQ_DBG_WHAT: ("N,K", np.uint16),
+        GSQ_DBG_WSOFT32: ("N,K", np.float32), GSQ_DBG_DW: ("N,K", np.float32),
+        GSQ_DBG_DYT: ("N,Tp", np.uint16), GSQ_DBG_YREFT: ("N,Tp", np.float32),
+        GSQ_DBG_DL: ("L,N,K", np.float32), GSQ_DBG_DS: ("N,G", np.float32),
+    }
+
+    def _shape(self, which):
+        spec, dt = self._SHAPES[which]
+        return tuple(getattr(self, d) for d in spec.split(",")), dt
+
+    def get(self, which) -> np.ndarray:
+        shape, dt = self._shape(which)
+        out = np.zeros(shape, dt)
+        _check(_lib.gsq_debug_get(self.ctx, which, out.ctypes.data, out.nbytes),
+               "gsq_debug_get")
+        return out
+
+    def set(self, which, arr) -> None:
+        shape, dt = self._shape(which)
+        a = np.ascontiguousarray(arr, dtype=dt).reshape(shape)
+        _check(_lib.gsq_debug_set(self.ctx, which, a.ctypes.data, a.nbytes),
+               "gsq_debug_set")
+
+    def uniforms(self, t: int, coord0: int, count: int) -> np.ndarray:
+        out = np.zeros((count, self.L), np.float32)
+        _check(_lib.gsq_debug_uniforms(self.ctx, t, coord0, count, out.ctypes.data),
+               "gsq_debug_uniforms")
+        return out
+
+    def noise(self, on: bool) -> None:
+        _check(_lib.gsq_debug_noise(self.ctx, int(on)), "gsq_debug_noise")
+
+    def soft_weight(self, tau: float) -> None:
+        _check(_lib.gsq_debug_soft_weight(self.ctx, tau), "gsq_debug_soft_weight")
+
+    def forward(self) -> float:
+        v = C.c_double()
+        _check(_lib.gsq_debug_forward(self.ctx, C.byref(v)), "gsq_debug_forward")
+        return v.value
+
+    def weight_grad(self) -> None:
+        _check(_lib.gsq_debug_weight_grad(self.ctx), "gsq_debug_weight_grad")
+
+    def backward(self, tau, lr, beta1=0.9, beta2=0.99) -> None:
+        _check(_lib.gsq_debug_backward(self.ctx, tau, lr, beta1, beta2),
+               "gsq_debug_backward")
+
+    # convenience -------------------------------------------------------
+    def step(self, tau, lr, beta1=0.9, beta2=0.99):
+        gsq_step(self, tau, lr, beta1, beta2)
+
+    def last_loss(self):
+        return gsq_last_loss(self)
+
+    def close(self):
+        gsq_destroy(self)
+
+    def __del__(self):
+        try:
+            if self.ctx:
+                _lib.gsq_destroy(self.ctx)
+                self.ctx = None
+        except Exception:
+            pass
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float32 values (exact)."""
+    return (b.astype(np.uint32) << 16).view(np.float32)
