@@ -281,11 +281,19 @@ def cpu_baseline(cfg, budget_s=15.0, steps=None):
 
 
 def load_traffic(kernel, config):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernels changed since those counters were taken."""
+    import glob
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return d.get(config, {}).get(kernel)
-    return None
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = sorted(glob.glob(os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc", "*")))
+    h = hashlib.sha256(b"".join(open(f, "rb").read() for f in src)).hexdigest()[:16]
+    if d.get("_csrc_sha256_16") != h:
+        return None
+    return d.get(config, {}).get(kernel)
 
 
 def run_reference(args, rank, world):
