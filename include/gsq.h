@@ -211,6 +211,29 @@ GSQ_API int gsq_debug_backward(gsq_ctx* ctx, float tau, float lr, float beta1,
                        float beta2);
 
 /*
+ * gsq_uniforms_noalloc -- the L Philox uniforms of coords
+ * [coord0, coord0 + count) at step t for grid_mode and seed (the values
+ * gsq_debug_uniforms returns for a context with that mode and seed),
+ * coordinate-major, into `out` (host or device, count * L floats), without
+ * allocating any device memory.  The pages have no counterpart: this is a
+ * convenience for callers that cannot call cudaMalloc, for example a process
+ * whose device memory is fully reserved by another allocator, or code inside
+ * a framework that forbids device allocation on its execution path.
+ * Device staging lives in a fixed array inside the library of
+ * GSQ_NOALLOC_MAX_COORDS x 5 floats (1.25 MiB), which every GPU that loads
+ * the library holds until exit; count above GSQ_NOALLOC_MAX_COORDS returns
+ * GSQ_ERR_INVALID_ARG.  The first call on a device looks up that array's
+ * device address (once per device); make that first call before any stream
+ * capture.  All calls share the array: calls whose work overlaps on the GPU
+ * (for example on two streams) race and may return each other's values.
+ * Enqueued on `stream` (NULL = legacy default stream); syncs.
+ */
+#define GSQ_NOALLOC_MAX_COORDS 65536
+GSQ_API int gsq_uniforms_noalloc(int grid_mode, uint64_t seed, uint32_t t,
+                                 uint64_t coord0, int64_t count, float* out,
+                                 void* stream);
+
+/*
  * gsq_gemm_bf16_abt -- the library's tcgen05 GEMM on its own:
  * C (M x N fp32, row-major, ldc = N) = A (M x Kc bf16, row-major) .
  * B (N x Kc bf16, row-major)^T with fp32 accumulation; device pointers,

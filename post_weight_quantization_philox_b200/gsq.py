@@ -21,6 +21,7 @@ GSQ_OK = 0
 GSQ_ERR_INVALID_ARG, GSQ_ERR_CUDA, GSQ_ERR_OOM = -1, -2, -3
 GSQ_ERR_NONFINITE, GSQ_ERR_STATE, GSQ_ERR_UNSUPPORTED, GSQ_ERR_TIMEOUT = -4, -5, -6, -7
 GSQ_RECON_HARD, GSQ_RECON_SOFT = 0, 1
+GSQ_NOALLOC_MAX_COORDS = 65536
 (GSQ_DBG_LOGITS, GSQ_DBG_MOM, GSQ_DBG_SCALES, GSQ_DBG_SMOM, GSQ_DBG_I0,
  GSQ_DBG_WHAT, GSQ_DBG_WSOFT32, GSQ_DBG_DW, GSQ_DBG_DYT, GSQ_DBG_YREFT,
  GSQ_DBG_DL, GSQ_DBG_DS) = range(12)
@@ -35,7 +36,7 @@ EXPORTS = [
     "gsq_destroy", "gsq_error_string", "gsq_set_timing", "gsq_phase_times",
     "gsq_debug_uniforms", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
-    "gsq_debug_backward", "gsq_gemm_bf16_abt",
+    "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
 ]
 
 
@@ -74,6 +75,7 @@ _SIGS = {
     "gsq_debug_weight_grad": [_p],
     "gsq_debug_backward": [_p, _f32, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
+    "gsq_uniforms_noalloc": [_i32, _u64, _u32, _u64, _i64, _p, _p],
 }
 
 
