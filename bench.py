@@ -96,16 +96,24 @@ class ClockSampler:
 
 
 def phase_bytes_flops(cfg, layer):
-    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch."""
+    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch.
+
+    soft weight:        read L logit planes + scale (+ initial level),
+                        write bf16 weight and the L noise planes;
+    backward + Lion:    read dW, logits, momenta, noise (+ initial level),
+                        write logits and momenta, 16 B per group of scales;
+    ... + next soft:    also write the next bf16 weight and noise planes."""
     NK = cfg.N * cfg.K
     L = layer.L
     extra = 1 if cfg.grid == synth.GRID_3BIT_LOCAL else 0  # initial level (int8)
     groups = cfg.N * (cfg.K // 128)
-    soft = NK * (4 * L + 2 + extra) + groups * 4
-    back = NK * (4 + 16 * L + extra) + groups * 16
+    soft = NK * (8 * L + 2 + extra) + groups * 4
+    back = NK * (4 + 20 * L + extra) + groups * 16
+    back_next = NK * (6 + 24 * L + extra) + groups * 16
     gemm = 2.0 * cfg.N * cfg.T * cfg.K
     return {"soft_weight": ("hbm", soft), "forward_gemm": ("tensor", gemm),
-            "weight_grad_gemm": ("tensor", gemm), "backward_lion": ("hbm", back)}
+            "weight_grad_gemm": ("tensor", gemm), "backward_lion": ("hbm", back),
+            "backward_lion_next_soft": ("hbm", back_next)}
 
 
 def run_gsq(args, rank, world, local_rank):
@@ -135,21 +143,20 @@ def run_gsq(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    for i in range(args.warmup):
-        lay.step(float(taus[i % nt]), cfg.lr)
-    torch.cuda.synchronize()
-    gsq.gsq_set_timing(lay, True)
-    gsq.gsq_phase_times(lay)  # reset
+    sched = np.array([taus[i % nt] for i in range(args.warmup + args.steps)], np.float32)
     clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)  # sampler up before the GPU work starts
+    # warm-up steps right before the timed region (clocks ramped up)
+    lay.run(sched[:args.warmup], cfg.lr)
+    gsq.gsq_set_timing(lay, True)
+    gsq.gsq_phase_times(lay)  # reset (syncs)
     dist_barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
-        lay.step(float(taus[(args.warmup + i) % nt]), cfg.lr)
+    lay.run(sched[args.warmup:], cfg.lr)
     e1.record(stream)
     torch.cuda.synchronize()
     dist_barrier()
@@ -177,11 +184,14 @@ def run_gsq(args, rank, world, local_rank):
     steps_per_s = args.steps / (ms / 1e3)
     coords = cfg.N * cfg.K
     value = world * coords * steps_per_s
-    names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion"]
+    names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion",
+             "backward_lion_next_soft"]
     work = phase_bytes_flops(cfg, lay)
     phases = {}
     for i, nm in enumerate(names):
-        per = phase_ms[i] / max(phase_n[i], 1)
+        if phase_n[i] == 0:
+            continue
+        per = phase_ms[i] / phase_n[i]
         bound, amount = work[nm]
         if bound == "hbm":
             ach = amount / (per / 1e3) / 1e9
@@ -189,10 +199,10 @@ def run_gsq(args, rank, world, local_rank):
         else:
             ach = amount / (per / 1e3) / 1e12
             peak, unit = tf_sus, "TFLOP/s"
-        phases[nm] = {"ms": round(per, 5), "bound": bound, "achieved": round(ach, 1),
-                      "unit": unit, "peak": peak, "frac": round(ach / peak, 4),
-                      "per_launch": amount}
-    dom = max(names, key=lambda n: phases[n]["ms"])
+        phases[nm] = {"ms": round(per, 5), "launches": int(phase_n[i]),
+                      "bound": bound, "achieved": round(ach, 1), "unit": unit,
+                      "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
+    dom = max(phases, key=lambda n: phases[n]["ms"] * phases[n]["launches"])
     d = phases[dom]
     traffic = load_traffic(dom, args.config)
     out = {
@@ -210,7 +220,7 @@ def run_gsq(args, rank, world, local_rank):
                      "peak_kind": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})",
                      "traffic": traffic},
         "phases": phases,
-        "gpu_launches": int(4 * args.steps),
+        "gpu_launches": int(sum(phase_n)),
         "clocks": clk,
         "last_loss": loss,
         "e2e": e2e,
@@ -234,8 +244,7 @@ def run_e2e(gsq, torch, cfg, W, X, rank):
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     lay = gsq.gsq_init(Wh, Xh, 128, cfg.grid, seed=rank)
-    for tau in taus:
-        lay.step(float(tau), cfg.lr)
+    lay.run(taus, cfg.lr)
     gsq._check(gsq.lib().gsq_loss_history(lay.ctx, cfg.steps - hist.size, hist.size,
                                           hist.ctypes.data), "gsq_loss_history")
     gsq.gsq_harden_pack(lay, packed, h16, None)

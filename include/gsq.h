@@ -108,6 +108,15 @@ GSQ_API int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
  */
 GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2);
 
+/*
+ * gsq_run -- n consecutive steps at temperatures taus[0..n) (host array),
+ * asynchronous.  Same results, bit for bit, as n calls of gsq_step; the
+ * backward of each step but the last also builds the next step's soft weight
+ * and Gumbel noise, so no step re-reads the logits for its soft weight.
+ */
+GSQ_API int gsq_run(gsq_ctx* ctx, const float* taus, int64_t n, float lr,
+                    float beta1, float beta2);
+
 /* gsq_last_loss -- loss (sum of squared errors) of the last step.  Syncs.
  * GSQ_ERR_NONFINITE if it was NaN / Inf; GSQ_ERR_STATE before any step. */
 GSQ_API int gsq_last_loss(gsq_ctx* ctx, double* loss);
@@ -162,10 +171,11 @@ GSQ_API const char* gsq_error_string(int status);
 
 /* ---------------------------------------------------------- measurement --
  * gsq_set_timing(ctx, on): record CUDA events on the context stream around
- * each phase of gsq_step.  gsq_phase_times(ctx, ms[4], launches[4]) returns
- * and resets the accumulated milliseconds and launch counts of phases
+ * each phase of every step.  gsq_phase_times(ctx, ms[5], launches[5])
+ * returns and resets the accumulated milliseconds and kernel launches of
  * 0 soft weight, 1 forward GEMM + loss, 2 weight-gradient GEMM,
- * 3 backward + Lion.  Syncs. */
+ * 3 backward + Lion, 4 backward + Lion that also built the next step's soft
+ * weight (gsq_run).  Syncs. */
 GSQ_API int gsq_set_timing(gsq_ctx* ctx, int on);
 GSQ_API int gsq_phase_times(gsq_ctx* ctx, double* ms, int64_t* launches);
 

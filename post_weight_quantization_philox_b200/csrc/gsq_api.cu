@@ -26,6 +26,8 @@ int num_logits(int mode) {
 
 struct Timing {
   cudaEvent_t ev[5];
+  bool soft;  // the soft-weight phase launched a kernel in this step
+  bool next;  // the backward also built the next step's soft weight
 };
 
 }  // namespace
@@ -46,7 +48,12 @@ struct gsq_ctx {
   double *partials = nullptr, *loss_hist = nullptr, *scratch = nullptr;
   unsigned* ticket = nullptr;
   int* err = nullptr;
+  float* gbuf = nullptr;  // Gumbel noise of the pending step (L x N x K)
   float *wsoft32 = nullptr, *dl = nullptr, *ds = nullptr;  // debug, lazy
+  // What and gbuf hold the soft weight and noise of step what_t at
+  // temperature what_tau (what_t < 0: nothing precomputed)
+  int64_t what_t = -1;
+  float what_tau = 0.f;
   double yref_sq = 0.0;
   CUtensorMap tm_What, tm_Xb, tm_dYt, tm_Xt;
   std::vector<void*> allocs;
@@ -256,6 +263,7 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   AL(c->dW, NK);
   AL(c->logits, c->L * NK);
   AL(c->mom, c->L * NK);
+  AL(c->gbuf, c->L * NK);
   AL(c->s, N * c->G);
   AL(c->ms, N * c->G);
   AL(c->i0, NK);
@@ -328,12 +336,12 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   // tensor maps of the persistent operands
   const int kw = split ? 2 : 1;
   CUtensorMap tmW, tmXr;
-  if (make_tmap_bf16(&c->tm_What, c->What, N, K, K, 128) ||
-      make_tmap_bf16(&c->tm_Xb, c->Xb, Tp, K, K, 256) ||
-      make_tmap_bf16(&c->tm_dYt, c->dYt, N, Tp, Tp, 128) ||
-      make_tmap_bf16(&c->tm_Xt, c->Xt, K, Tp, Tp, 256) ||
-      make_tmap_bf16(&tmW, Wop, N, kw * K, kw * K, 128) ||
-      make_tmap_bf16(&tmXr, split ? Xcat : c->Xb, Tp, kw * K, kw * K, 256))
+  if (make_tmap_bf16(&c->tm_What, c->What, N, K, K, kGemmBoxRowsA) ||
+      make_tmap_bf16(&c->tm_Xb, c->Xb, Tp, K, K, kGemmBoxRowsB) ||
+      make_tmap_bf16(&c->tm_dYt, c->dYt, N, Tp, Tp, kGemmBoxRowsA) ||
+      make_tmap_bf16(&c->tm_Xt, c->Xt, K, Tp, Tp, kGemmBoxRowsB) ||
+      make_tmap_bf16(&tmW, Wop, N, kw * K, kw * K, kGemmBoxRowsA) ||
+      make_tmap_bf16(&tmXr, split ? Xcat : c->Xb, Tp, kw * K, kw * K, kGemmBoxRowsB))
     return cleanup_fail(GSQ_ERR_CUDA);
 
   // Y_ref^T = W . bf16(X)^T (fp32 accumulate; W at its own precision)
@@ -366,11 +374,15 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
 #undef AL
 }
 
-int gsq_step(gsq_ctx* c, float tau, float lr, float beta1, float beta2) {
-  int u = usable(c);
-  if (u) return u;
-  if (!step_args_ok(tau, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
-  if (c->t >= 0xFFFFFFFFull) return GSQ_ERR_UNSUPPORTED;  // 32-bit counter word
+}  // extern "C"
+
+namespace {
+
+// One step t at temperature tau; with tau_next > 0 the backward also builds
+// the soft weight and noise of step t + 1 (which the next call then skips).
+int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
+             float beta2) {
+  if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;  // 32-bit counter word
   const StepArgs a = step_args(c, tau);
   Timing* tm = nullptr;
   if (c->timing) {
@@ -382,16 +394,53 @@ int gsq_step(gsq_ctx* c, float tau, float lr, float beta1, float beta2) {
     tm = &c->tev[c->tev_used++];
     CK(cudaEventRecord(tm->ev[0], c->st));
   }
-  CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
-  if (tm) CK(cudaEventRecord(tm->ev[1], c->st));
+  const bool soft = !(c->what_t == (int64_t)c->t && c->what_tau == tau);
+  if (soft) CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));
+  if (tm) {
+    tm->soft = soft;
+    tm->next = tau_next > 0.f;
+    CK(cudaEventRecord(tm->ev[1], c->st));
+  }
   CK(run_forward(c, c->loss_hist + (c->t % kLossRing), EPI_LOSS_DY));
   if (tm) CK(cudaEventRecord(tm->ev[2], c->st));
   CK(run_weight_grad(c));
   if (tm) CK(cudaEventRecord(tm->ev[3], c->st));
-  CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, nullptr, nullptr, c->sms,
-                          c->st));
+  CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, tau_next,
+                          c->What, nullptr, nullptr, c->sms, c->st));
   if (tm) CK(cudaEventRecord(tm->ev[4], c->st));
   c->t += 1;
+  if (tau_next > 0.f) {
+    c->what_t = (int64_t)c->t;
+    c->what_tau = tau_next;
+  } else {
+    c->what_t = -1;
+  }
+  return GSQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gsq_step(gsq_ctx* c, float tau, float lr, float beta1, float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (!step_args_ok(tau, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
+  return run_step(c, tau, 0.f, lr, beta1, beta2);
+}
+
+int gsq_run(gsq_ctx* c, const float* taus, int64_t n, float lr, float beta1,
+            float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (!taus || n <= 0) return GSQ_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < n; ++i)
+    if (!step_args_ok(taus[i], lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < n; ++i) {
+    const int rc = run_step(c, taus[i], i + 1 < n ? taus[i + 1] : 0.f, lr,
+                            beta1, beta2);
+    if (rc) return rc;
+  }
   return GSQ_OK;
 }
 
@@ -466,13 +515,14 @@ int gsq_recon_error(gsq_ctx* c, int mode, float tau, double* abs_err,
   if (!abs_err || (mode != GSQ_RECON_HARD && mode != GSQ_RECON_SOFT) ||
       (mode == GSQ_RECON_SOFT && !(tau > 0.f && std::isfinite(tau))))
     return GSQ_ERR_INVALID_ARG;
+  c->what_t = -1;  // What is overwritten below
   if (mode == GSQ_RECON_HARD) {
     CK(launch_hard_weight(c->mode, c->N, c->K, c->logits, c->s, c->i0, c->What,
                           c->st));
   } else {
     StepArgs a = step_args(c, tau);
     a.noise = 0;
-    CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
+    CK(launch_soft_weight(a, c->What, nullptr, nullptr, c->sms, c->st));
   }
   CK(run_forward(c, c->scratch, EPI_LOSS));
   int rc = check_device(c);
@@ -535,6 +585,7 @@ int gsq_import_state(gsq_ctx* c, const void* host_buf, size_t bytes) {
   CK(cudaMemcpy(c->s, p + 2 * lb, sb, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->ms, p + 2 * lb + sb, sb, cudaMemcpyHostToDevice));
   c->t = h[5];
+  c->what_t = -1;
   return GSQ_OK;
 }
 
@@ -567,16 +618,22 @@ int gsq_phase_times(gsq_ctx* c, double* ms, int64_t* launches) {
   if (u) return u;
   if (!ms) return GSQ_ERR_INVALID_ARG;
   CK(cudaStreamSynchronize(c->st));
-  double acc[4] = {0, 0, 0, 0};
-  for (size_t i = 0; i < c->tev_used; ++i)
+  double acc[5] = {0, 0, 0, 0, 0};
+  int64_t n[5] = {0, 0, 0, 0, 0};
+  for (size_t i = 0; i < c->tev_used; ++i) {
+    const Timing& te = c->tev[i];
     for (int p = 0; p < 4; ++p) {
       float x = 0.f;
-      CK(cudaEventElapsedTime(&x, c->tev[i].ev[p], c->tev[i].ev[p + 1]));
-      acc[p] += x;
+      CK(cudaEventElapsedTime(&x, te.ev[p], te.ev[p + 1]));
+      // backward launches that also built the next soft weight count apart
+      const int slot = (p == 3 && te.next) ? 4 : p;
+      acc[slot] += x;
+      if (p != 0 || te.soft) n[slot] += 1;
     }
-  for (int p = 0; p < 4; ++p) {
+  }
+  for (int p = 0; p < 5; ++p) {
     ms[p] = acc[p];
-    if (launches) launches[p] = (int64_t)c->tev_used;
+    if (launches) launches[p] = n[p];
   }
   c->tev_used = 0;
   return GSQ_OK;
@@ -636,6 +693,7 @@ int gsq_debug_set(gsq_ctx* c, int which, const void* host, size_t bytes) {
   if (!host || bytes != nb) return GSQ_ERR_INVALID_ARG;
   CK(cudaStreamSynchronize(c->st));
   CK(cudaMemcpy(p, host, nb, cudaMemcpyHostToDevice));
+  c->what_t = -1;  // any state change invalidates a precomputed soft weight
   return GSQ_OK;
 }
 
@@ -643,6 +701,7 @@ int gsq_debug_noise(gsq_ctx* c, int on) {
   int u = usable(c);
   if (u) return u;
   c->noise = on ? 1 : 0;
+  c->what_t = -1;
   return GSQ_OK;
 }
 
@@ -670,7 +729,10 @@ int gsq_debug_soft_weight(gsq_ctx* c, float tau) {
   size_t nb;
   int rc = debug_buffer(c, GSQ_DBG_WSOFT32, &p, &nb);
   if (rc) return rc;
-  CK(launch_soft_weight(step_args(c, tau), c->What, c->wsoft32, c->sms, c->st));
+  CK(launch_soft_weight(step_args(c, tau), c->What, c->gbuf, c->wsoft32, c->sms,
+                        c->st));
+  c->what_t = (int64_t)c->t;
+  c->what_tau = tau;
   return check_device(c);
 }
 
@@ -702,8 +764,13 @@ int gsq_debug_backward(gsq_ctx* c, float tau, float lr, float beta1,
   int rc = debug_buffer(c, GSQ_DBG_DL, &p, &nb);
   if (!rc) rc = debug_buffer(c, GSQ_DBG_DS, &p, &nb);
   if (rc) return rc;
-  CK(launch_backward_lion(step_args(c, tau), c->dW, lr, beta1, beta2, c->dl,
-                          c->ds, c->sms, c->st));
+  // the step's noise first (the backward takes it from the noise buffer)
+  const StepArgs a = step_args(c, tau);
+  if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
+    CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));
+  CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, 0.f, c->What,
+                          c->dl, c->ds, c->sms, c->st));
+  c->what_t = -1;
   return check_device(c);
 }
 
@@ -722,7 +789,8 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
   if (prop.major != 10) return GSQ_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap ta, tb;
-  if (make_tmap_bf16(&ta, A, M, Kc, Kc, 128) || make_tmap_bf16(&tb, B, N, Kc, Kc, 256))
+  if (make_tmap_bf16(&ta, A, M, Kc, Kc, kGemmBoxRowsA) ||
+      make_tmap_bf16(&tb, B, N, Kc, Kc, kGemmBoxRowsB))
     return GSQ_ERR_CUDA;
   int* err = nullptr;
   if (cudaMalloc(&err, 16) != cudaSuccess) {

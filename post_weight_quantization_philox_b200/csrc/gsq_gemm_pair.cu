@@ -1,0 +1,308 @@
+// gsq_gemm_pair.cu -- the GSQ GEMMs on CTA pairs (tcgen05 cta_group::2).
+//
+// C[M x N] = A[M x Kc] . B[N x Kc]^T, bf16 K-major operands, fp32 TMEM
+// accumulators, epilogues as in the single-CTA kernel (gsq_gemm_epi.cuh).
+//
+// A cluster of two CTAs on neighbouring SMs owns a 256 x 256 output tile:
+// CTA r loads rows [128 r, 128 r + 128) of the A tile and rows
+// [128 r, 128 r + 128) of the B tile (half of the tile's N) into its own
+// shared memory, in 64-wide K slabs through a 6-deep ring (32 KB per
+// stage).  One thread of the leader CTA (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, N = 256, which reads A and B from
+// both CTAs and accumulates 128 rows into each CTA's TMEM.  Compared with a
+// single CTA computing 128 x 256, each CTA moves a third fewer operand bytes
+// per MMA, and the deeper ring hides more load latency.
+//
+// Both CTAs' TMA loads count their bytes on the leader's "full" barrier; the
+// MMA thread signals each CTA's "empty" and "accumulator full" barriers with
+// one tcgen05.commit per CTA (shared::cluster addresses from mapa); the
+// epilogue warps of both CTAs release an accumulator on the leader's
+// barrier.  No cluster multicast of any load is used.  Every mbarrier wait
+// is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, drains what it
+// issued, frees TMEM and returns.
+#include "gsq_gemm_epi.cuh"
+
+namespace gsq {
+
+namespace {
+
+constexpr int PM = 256, PN = 256, HALF = 128, BK = 64;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = HALF * BK * 2;
+constexpr int B_BYTES = HALF * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * PN;
+constexpr int NUM_THREADS = 192;
+constexpr long long WAIT_LIMIT = 4000000000LL;  // clock cycles (~2 s)
+constexpr uint32_t IDESC = idesc_bf16_f32(PM, PN);
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+  double red[4];
+};
+
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctl);
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  const bool ok = mbar_wait_bounded(bar, parity, WAIT_LIMIT);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                const __grid_constant__ CUtensorMap tmB, int64_t M, int64_t N,
+                int64_t Kc, EpiParams ep) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int m_tiles = (int)((M + PM - 1) / PM);
+  const int n_tiles = (int)((N + PN - 1) / PN);
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = (int)((Kc + BK - 1) / BK);
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->tfull[b]), 1);
+      mbar_init(smem_u32(&ctl->tempty[b]), 8);  // 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(smem_u32(&ctl->done), 1);
+    ctl->abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote access
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const int mb = tile % m_tiles, nb = tile / m_tiles;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), ph ^ 1,
+                                 WAIT_LIMIT) ||
+              *(volatile int*)&ctl->abort) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&ctl->full[stage]);
+          const uint32_t fb_leader = mapa_shared(fb, 0);
+          if (leader) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          tma_load_2d_pair(sa, &tmA, fb_leader, kb * BK,
+                           mb * PM + (int)rank * HALF);
+          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, kb * BK,
+                           nb * PN + (int)rank * HALF);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+        *(volatile int*)&ctl->abort = 1;
+      }
+      // drain (leader): the last phase armed on each stage has completed,
+      // i.e. both CTAs' loads into it have landed
+      if (leader) {
+        for (int s = 0; s < STAGES; ++s) {
+          if (issued <= s) break;
+          const long long last = ((issued - 1 - s) / STAGES) * STAGES + s;
+          const uint32_t par = (uint32_t)((last / STAGES) & 1);
+          if (!mbar_wait_bounded(smem_u32(&ctl->full[s]), par, WAIT_LIMIT))
+            atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // --------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        if (!mbar_wait_bounded(smem_u32(&ctl->tempty[acc]), aph ^ 1,
+                               WAIT_LIMIT)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), ph,
+                                 WAIT_LIMIT) ||
+              *(volatile int*)&ctl->abort) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          const uint64_t ad = sdesc_kmajor_sw128(sa);
+          const uint64_t bd = sdesc_kmajor_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, IDESC,
+                           (kb > 0 || k > 0) ? 1u : 0u);
+          const uint32_t eb = smem_u32(&ctl->empty[stage]);
+          umma_commit_pair(mapa_shared(eb, 0));
+          umma_commit_pair(mapa_shared(eb, 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        const uint32_t tb = smem_u32(&ctl->tfull[acc]);
+        umma_commit_pair(mapa_shared(tb, 0));
+        umma_commit_pair(mapa_shared(tb, 1));
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      if (!ok) {
+        atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+        *(volatile int*)&ctl->abort = 1;
+      }
+      // drain: every MMA this thread issued has completed
+      umma_commit_pair(mapa_shared(smem_u32(&ctl->done), 0));
+      if (!mbar_wait_bounded(smem_u32(&ctl->done), 0, WAIT_LIMIT))
+        atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    double lsum = 0.0;
+    for (int tile = pair; tile < num_tiles; tile += npairs) {
+      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      if (!warp_wait(smem_u32(&ctl->tfull[acc]), aph) ||
+          *(volatile int*)&ctl->abort) {
+        if (lane == 0) {
+          atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+          *(volatile int*)&ctl->abort = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = (int64_t)mb * PM + (int64_t)rank * HALF + r;
+      const uint32_t tbase =
+          tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * PN);
+      float part = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < PN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), v);
+        tmem_wait_ld();
+        epilogue_chunk<EPI>(v, row, (int64_t)nb * PN + c * 32, M, N, ep, part);
+      }
+      lsum += (double)part;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+    if (EPI != EPI_STORE_F32) {
+      lsum = warp_sum_d(lsum);
+      if (lane == 0) ctl->red[q] = lsum;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (warp == 2 && lane == 0)
+        loss_finish(ctl->red[0] + ctl->red[1] + ctl->red[2] + ctl->red[3], ep);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its pair may still touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int EPI>
+cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                            int64_t M, int64_t N, int64_t Kc,
+                            const EpiParams& ep, int sm_count,
+                            cudaStream_t st) {
+  static int max_pairs = 0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs == 0) {
+    cudaError_t e = cudaFuncSetAttribute(
+        k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count / 2;
+    }
+    max_pairs = n;
+  }
+  const int64_t tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);
+  const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI>, tmA, tmB, M, N, Kc, ep);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             int64_t M, int64_t N, int64_t Kc, int mode,
+                             const EpiParams& ep, int sm_count,
+                             cudaStream_t st) {
+  switch (mode) {
+    case EPI_STORE_F32:
+      return launch_pair_epi<EPI_STORE_F32>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+    case EPI_LOSS_DY:
+      return launch_pair_epi<EPI_LOSS_DY>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+    default:
+      return launch_pair_epi<EPI_LOSS>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+  }
+}
+
+}  // namespace gsq

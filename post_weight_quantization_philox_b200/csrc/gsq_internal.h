@@ -41,11 +41,20 @@ struct EpiParams {
 int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows,
                    int64_t cols, int64_t ld, int box_rows);
 
-// C[M x N] = A[M x Kc] . B[N x Kc]^T with the epilogue selected by `mode`;
-// tmA / tmB made by make_tmap_bf16 with box rows 128 (A) and 256 (B).
+// Box rows of the tensor maps the GEMM expects for A and for B.
+constexpr int kGemmBoxRowsA = 128;
+constexpr int kGemmBoxRowsB = 128;
+
+// C[M x N] = A[M x Kc] . B[N x Kc]^T with the epilogue selected by `mode`
+// (CTA-pair tcgen05 kernel); tmA / tmB made by make_tmap_bf16 with
+// kGemmBoxRowsA / kGemmBoxRowsB rows per box.
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int64_t M, int64_t N, int64_t Kc, int mode,
                         const EpiParams& ep, int sm_count, cudaStream_t st);
+cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             int64_t M, int64_t N, int64_t Kc, int mode,
+                             const EpiParams& ep, int sm_count,
+                             cudaStream_t st);
 
 // ------------------------------------------------------- elementwise
 struct StepArgs {
@@ -72,11 +81,19 @@ cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
 cudaError_t launch_init_state(int mode, const float* W32, const int8_t* init_idx,
                               int64_t N, int64_t K, float* s, int8_t* i0,
                               float* logits, int* err, cudaStream_t st);
+// Soft weight of step a.t; keeps the step's Gumbel noise in gbuf (L planes
+// of N x K fp32) when gbuf is not null.
 cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
-                               float* wsoft32, int sm_count, cudaStream_t st);
-cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr,
-                                 float b1, float b2, float* dl_dbg,
-                                 float* ds_dbg, int sm_count, cudaStream_t st);
+                               float* gbuf, float* wsoft32, int sm_count,
+                               cudaStream_t st);
+// Backward + Lion of step a.t from dW and the noise in gbuf; with
+// tau_next > 0 also the soft weight (into What) and noise (into gbuf) of
+// step a.t + 1.
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
+                                 float* gbuf, float lr, float b1, float b2,
+                                 float tau_next, __nv_bfloat16* What,
+                                 float* dl_dbg, float* ds_dbg, int sm_count,
+                                 cudaStream_t st);
 cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
                                const float* logits, const float* s,
                                const int8_t* i0, __nv_bfloat16* What,

@@ -221,72 +221,86 @@ __device__ __forceinline__ void candidates(int lev0, float* cand) {
   }
 }
 
-// Four consecutive coordinates per thread (128-bit loads per logit plane).
+// Gumbel noise of one coordinate at step t (zeros when noise is off).
+template <int L>
+__device__ __forceinline__ void noise1(int64_t c, uint32_t t, uint32_t k0,
+                                       uint32_t k1, int noise, float (&g)[L]) {
+  float gg[5];
+  if (noise) {
+    coord_noise5((uint64_t)c, t, k0, k1, L == 5, gg);
+  } else {
+#pragma unroll
+    for (int p = 0; p < 5; ++p) gg[p] = 0.f;
+  }
+#pragma unroll
+  for (int p = 0; p < L; ++p) g[p] = gg[p];
+}
+
+// Both kernels below give one warp a group of 128 coordinates of one row;
+// lane j takes coordinates j, j+32, j+64, j+96, so every load and store of a
+// logit plane is one coalesced 128-byte access and each coordinate is
+// finished before the next one starts (few live registers).
+constexpr int kPerLane = kGroup / 32;
+
+// Soft weight (A1 + A2): w = bf16(s * v((l + g) / tau)).  When gbuf is given
+// the step's Gumbel noise is kept there (L planes) for the backward.
 template <int MODE, bool DBG>
 __global__ void __launch_bounds__(256) k_soft_weight(
     const float* __restrict__ logits, const float* __restrict__ s,
     const int8_t* __restrict__ i0, int64_t N, int64_t K, uint32_t k0,
     uint32_t k1, uint32_t t, int noise, float inv_tau,
-    __nv_bfloat16* __restrict__ What, float* __restrict__ wsoft32) {
+    __nv_bfloat16* __restrict__ What, float* __restrict__ gbuf,
+    float* __restrict__ wsoft32) {
   constexpr int L = GridT<MODE>::L;
-  const int64_t NK = N * K, G = K / kGroup, n4 = NK / 4;
-  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n4;
-       q += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t c0 = q * 4;
-    const int64_t n = c0 / K, k = c0 - n * K;
-    const float sg = __ldg(s + n * G + k / kGroup);
-    float4 lp[L];
+  const int64_t NK = N * K, G = K / kGroup;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t gi = warp; gi < N * G; gi += nwarps) {
+    const int64_t n = gi / G, g = gi - n * G;
+    const int64_t base = n * K + g * kGroup + lane;
+    const float sg = __ldg(s + gi);
 #pragma unroll
-    for (int p = 0; p < L; ++p)
-      lp[p] = __ldg(reinterpret_cast<const float4*>(logits + p * NK + c0));
-    char4 iv = make_char4(0, 0, 0, 0);
-    if (MODE == GRID_3BIT_LOCAL)
-      iv = __ldg(reinterpret_cast<const char4*>(i0 + c0));
-    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
-    float wv[4];
+    for (int j = 0; j < kPerLane; ++j) {
+      const int64_t c = base + 32 * j;
+      float l[L], gz[L], y[L], cand[5];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float l[L], g[5], y[L], cand[5];
+      for (int p = 0; p < L; ++p) l[p] = __ldg(logits + p * NK + c);
+      const int lev0 = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
+      noise1<L>(c, t, k0, k1, noise, gz);
+      candidates<MODE>(lev0, cand);
+      const float w = sg * coord_soft<MODE>(l, gz, inv_tau, cand, y);
+      What[c] = __float2bfloat16_rn(w);
+      if (gbuf) {
 #pragma unroll
-      for (int p = 0; p < L; ++p)
-        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
-      if (noise) {
-        coord_noise5((uint64_t)(c0 + j), t, k0, k1, L == 5, g);
-      } else {
-#pragma unroll
-        for (int p = 0; p < 5; ++p) g[p] = 0.f;
+        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = gz[p];
       }
-      candidates<MODE>(lev0[j], cand);
-      const float v = coord_soft<MODE>(l, g, inv_tau, cand, y);
-      wv[j] = sg * v;
+      if (DBG) wsoft32[c] = w;
     }
-    __nv_bfloat162 b01 = __floats2bfloat162_rn(wv[0], wv[1]);
-    __nv_bfloat162 b23 = __floats2bfloat162_rn(wv[2], wv[3]);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&b01);
-    pk.y = *reinterpret_cast<uint32_t*>(&b23);
-    *reinterpret_cast<uint2*>(What + c0) = pk;
-    if (DBG)
-      *reinterpret_cast<float4*>(wsoft32 + c0) =
-          make_float4(wv[0], wv[1], wv[2], wv[3]);
   }
 }
 
 // ------------------------------------------------- backward + Lion (A5)
 
-// One warp per group of 128 coordinates, four per lane.  Recomputes the
-// step's probabilities from the same Philox counters, forms
+// Takes the step's Gumbel noise from gbuf (written by the soft weight of the
+// same step), rebuilds the probabilities and forms
 //   a = s dW / tau,  dl_k = a y_k sum_j y_j (c_k - c_j)   (categorical),
 //   dl_mask1 = a (q+ - q-) p1 p0 = -dl_mask0, dl_sign+ = 2 a p1 q+ q- =
 //   -dl_sign- (ternary),  ds = sum over the group of dW v (warp shuffle),
-// then applies Lion to the logits and, on lane 0, to the group scale.
-template <int MODE, bool DBG>
-__global__ void __launch_bounds__(256) k_backward_lion(
+// then applies Lion to the logits and the group scale.  With NEXT it also
+// computes the soft weight of step t+1 from the updated logits and scale
+// (fresh Philox noise, kept in gbuf for the next backward): the same values
+// a separate soft-weight launch would produce.  All loads of the group are
+// issued first and the next step's noise (which needs none of them) is
+// computed while they are in flight.
+template <int MODE, bool DBG, bool NEXT>
+__global__ void __launch_bounds__(256, 2) k_backward_lion(
     float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ s,
     float* __restrict__ ms, const int8_t* __restrict__ i0,
-    const float* __restrict__ dW, int64_t N, int64_t K, uint32_t k0,
-    uint32_t k1, uint32_t t, int noise, float inv_tau, float lr, float b1,
-    float omb1, float b2, float omb2, float* __restrict__ dl_dbg,
+    const float* __restrict__ dW, float* __restrict__ gbuf, int64_t N,
+    int64_t K, uint32_t k0, uint32_t k1, uint32_t t_next, int noise,
+    float inv_tau, float inv_tau_next, float lr, float b1, float omb1, float b2,
+    float omb2, __nv_bfloat16* __restrict__ What, float* __restrict__ dl_dbg,
     float* __restrict__ ds_dbg) {
   constexpr int L = GridT<MODE>::L;
   const int64_t NK = N * K, G = K / kGroup;
@@ -295,40 +309,46 @@ __global__ void __launch_bounds__(256) k_backward_lion(
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t gi = warp; gi < N * G; gi += nwarps) {
     const int64_t n = gi / G, g = gi - n * G;
-    const int64_t c0 = n * K + g * kGroup + lane * 4;
+    const int64_t base = n * K + g * kGroup + lane;
     const float sg = s[gi];
-    const float4 dw4 = __ldg(reinterpret_cast<const float4*>(dW + c0));
-    float4 lp[L], mp[L];
-#pragma unroll
-    for (int p = 0; p < L; ++p) {
-      lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
-      mp[p] = *reinterpret_cast<const float4*>(mom + p * NK + c0);
-    }
-    char4 iv = make_char4(0, 0, 0, 0);
-    if (MODE == GRID_3BIT_LOCAL)
-      iv = __ldg(reinterpret_cast<const char4*>(i0 + c0));
-    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
-    const float dwv[4] = {dw4.x, dw4.y, dw4.z, dw4.w};
+    const float msg = ms[gi];
     float ds_part = 0.f;
-    float lo[L][4], mo[L][4], dlo[L][4];
+    float lnew[NEXT ? kPerLane : 1][L];
+    int lev[kPerLane];
+    float Lr[kPerLane][L], Mr[kPerLane][L], Gr[kPerLane][L], Dr[kPerLane];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float l[L], m[L], gz[5], y[L], cand[5];
+    for (int j = 0; j < kPerLane; ++j) {
+      const int64_t c = base + 32 * j;
 #pragma unroll
       for (int p = 0; p < L; ++p) {
-        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
-        m[p] = j == 0 ? mp[p].x : j == 1 ? mp[p].y : j == 2 ? mp[p].z : mp[p].w;
+        Lr[j][p] = logits[p * NK + c];
+        Mr[j][p] = mom[p * NK + c];
+        Gr[j][p] = gbuf[p * NK + c];
       }
-      if (noise) {
-        coord_noise5((uint64_t)(c0 + j), t, k0, k1, L == 5, gz);
-      } else {
+      Dr[j] = __ldg(dW + c);
+      lev[j] = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
+    }
+    float gnext[NEXT ? kPerLane : 1][L];
+    if (NEXT) {
 #pragma unroll
-        for (int p = 0; p < 5; ++p) gz[p] = 0.f;
+      for (int j = 0; j < kPerLane; ++j)
+        noise1<L>(base + 32 * j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
+    }
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+      const int64_t c = base + 32 * j;
+      float l[L], m[L], gz[L], y[L], cand[5];
+#pragma unroll
+      for (int p = 0; p < L; ++p) {
+        l[p] = Lr[j][p];
+        m[p] = Mr[j][p];
+        gz[p] = Gr[j][p];
       }
-      candidates<MODE>(lev0[j], cand);
+      const float dw = Dr[j];
+      candidates<MODE>(lev[j], cand);
       const float v = coord_soft<MODE>(l, gz, inv_tau, cand, y);
-      ds_part = fmaf(dwv[j], v, ds_part);
-      const float a = sg * dwv[j] * inv_tau;
+      ds_part = fmaf(dw, v, ds_part);
+      const float a = sg * dw * inv_tau;
       float dl[L];
       if (MODE == GRID_TERNARY) {
         const float gm = a * (y[3] - y[2]) * y[1] * y[0];
@@ -350,28 +370,34 @@ __global__ void __launch_bounds__(256) k_backward_lion(
       for (int p = 0; p < L; ++p) {
         float th = l[p], mm = m[p];
         lion_update(th, mm, dl[p], lr, b1, omb1, b2, omb2);
-        lo[p][j] = th;
-        mo[p][j] = mm;
-        dlo[p][j] = dl[p];
+        logits[p * NK + c] = th;
+        mom[p * NK + c] = mm;
+        if (NEXT) lnew[NEXT ? j : 0][p] = th;
+        if (DBG) dl_dbg[p * NK + c] = dl[p];
       }
     }
-#pragma unroll
-    for (int p = 0; p < L; ++p) {
-      *reinterpret_cast<float4*>(logits + p * NK + c0) =
-          make_float4(lo[p][0], lo[p][1], lo[p][2], lo[p][3]);
-      *reinterpret_cast<float4*>(mom + p * NK + c0) =
-          make_float4(mo[p][0], mo[p][1], mo[p][2], mo[p][3]);
-      if (DBG)
-        *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
-            make_float4(dlo[p][0], dlo[p][1], dlo[p][2], dlo[p][3]);
-    }
-    const float ds = warp_sum(ds_part);
+    // every lane takes lane 0's sum so that all lanes hold the same new scale
+    const float ds = __shfl_sync(0xffffffffu, warp_sum(ds_part), 0);
+    float s_new = sg, ms_new = msg;
+    lion_update(s_new, ms_new, ds, lr, b1, omb1, b2, omb2);
     if (lane == 0) {
-      float th = sg, mm = ms[gi];
-      lion_update(th, mm, ds, lr, b1, omb1, b2, omb2);
-      s[gi] = th;
-      ms[gi] = mm;
+      s[gi] = s_new;
+      ms[gi] = ms_new;
       if (DBG) ds_dbg[gi] = ds;
+    }
+    if (NEXT) {
+#pragma unroll
+      for (int j = 0; j < kPerLane; ++j) {
+        const int64_t c = base + 32 * j;
+        float y[L], cand[5];
+        float (&gz)[L] = gnext[NEXT ? j : 0];
+        candidates<MODE>(lev[j], cand);
+        const float w = s_new * coord_soft<MODE>(lnew[NEXT ? j : 0], gz,
+                                                 inv_tau_next, cand, y);
+        What[c] = __float2bfloat16_rn(w);
+#pragma unroll
+        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = gz[p];
+      }
     }
   }
 }
@@ -607,57 +633,78 @@ cudaError_t launch_init_state(int mode, const float* W32,
 
 template <int MODE>
 static void soft_weight_mode(const StepArgs& a, __nv_bfloat16* What,
-                             float* wsoft32, int blocks, cudaStream_t st) {
+                             float* gbuf, float* wsoft32, int blocks,
+                             cudaStream_t st) {
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
   const float inv_tau = 1.0f / a.tau;
   if (wsoft32)
     k_soft_weight<MODE, true><<<blocks, 256, 0, st>>>(
         a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        wsoft32);
+        gbuf, wsoft32);
   else
     k_soft_weight<MODE, false><<<blocks, 256, 0, st>>>(
         a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        nullptr);
+        gbuf, nullptr);
 }
 
 cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
-                               float* wsoft32, int sm_count, cudaStream_t st) {
-  const int blocks = grid_for(a.N * a.K / 4, 256, sm_count * 8);
+                               float* gbuf, float* wsoft32, int sm_count,
+                               cudaStream_t st) {
+  const int64_t groups = a.N * (a.K / kGroup);
+  const int blocks = grid_for(groups * 32, 256, sm_count * 8);
   switch (a.mode) {
-    case GRID_2BIT: soft_weight_mode<GRID_2BIT>(a, What, wsoft32, blocks, st); break;
-    case GRID_TERNARY: soft_weight_mode<GRID_TERNARY>(a, What, wsoft32, blocks, st); break;
-    default: soft_weight_mode<GRID_3BIT_LOCAL>(a, What, wsoft32, blocks, st);
+    case GRID_2BIT: soft_weight_mode<GRID_2BIT>(a, What, gbuf, wsoft32, blocks, st); break;
+    case GRID_TERNARY: soft_weight_mode<GRID_TERNARY>(a, What, gbuf, wsoft32, blocks, st); break;
+    default: soft_weight_mode<GRID_3BIT_LOCAL>(a, What, gbuf, wsoft32, blocks, st);
   }
   return cudaGetLastError();
 }
 
-template <int MODE>
-static void backward_mode(const StepArgs& a, const float* dW, float lr,
-                          float b1, float b2, float* dl_dbg, float* ds_dbg,
+template <int MODE, bool NEXT>
+static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
+                          float lr, float b1, float b2, float tau_next,
+                          __nv_bfloat16* What, float* dl_dbg, float* ds_dbg,
                           int blocks, cudaStream_t st) {
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
   const float inv_tau = 1.0f / a.tau;
+  const float inv_tau_next = NEXT ? 1.0f / tau_next : 0.f;
   const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
   if (dl_dbg)
-    k_backward_lion<MODE, true><<<blocks, 256, 0, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, a.N, a.K, k0, k1, a.t, a.noise,
-        inv_tau, lr, b1, omb1, b2, omb2, dl_dbg, ds_dbg);
+    k_backward_lion<MODE, true, NEXT><<<blocks, 256, 0, st>>>(
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
+        a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
+        dl_dbg, ds_dbg);
   else
-    k_backward_lion<MODE, false><<<blocks, 256, 0, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, a.N, a.K, k0, k1, a.t, a.noise,
-        inv_tau, lr, b1, omb1, b2, omb2, nullptr, nullptr);
+    k_backward_lion<MODE, false, NEXT><<<blocks, 256, 0, st>>>(
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
+        a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
+        nullptr, nullptr);
 }
 
-cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr,
-                                 float b1, float b2, float* dl_dbg,
-                                 float* ds_dbg, int sm_count,
+template <int MODE>
+static void backward_dispatch(const StepArgs& a, const float* dW, float* gbuf,
+                              float lr, float b1, float b2, float tau_next,
+                              __nv_bfloat16* What, float* dl_dbg,
+                              float* ds_dbg, int blocks, cudaStream_t st) {
+  if (tau_next > 0.f)
+    backward_mode<MODE, true>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+                              ds_dbg, blocks, st);
+  else
+    backward_mode<MODE, false>(a, dW, gbuf, lr, b1, b2, tau_next, What,
+                               dl_dbg, ds_dbg, blocks, st);
+}
+
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
+                                 float* gbuf, float lr, float b1, float b2,
+                                 float tau_next, __nv_bfloat16* What,
+                                 float* dl_dbg, float* ds_dbg, int sm_count,
                                  cudaStream_t st) {
   const int64_t groups = a.N * (a.K / kGroup);
   const int blocks = grid_for(groups * 32, 256, sm_count * 8);
   switch (a.mode) {
-    case GRID_2BIT: backward_mode<GRID_2BIT>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st); break;
-    case GRID_TERNARY: backward_mode<GRID_TERNARY>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st); break;
-    default: backward_mode<GRID_3BIT_LOCAL>(a, dW, lr, b1, b2, dl_dbg, ds_dbg, blocks, st);
+    case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    default: backward_dispatch<GRID_3BIT_LOCAL>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st);
   }
   return cudaGetLastError();
 }

@@ -30,7 +30,7 @@ NUM_LOGITS = {GSQ_GRID_2BIT: 4, GSQ_GRID_TERNARY: 4, GSQ_GRID_3BIT_LOCAL: 5}
 
 # every symbol include/gsq.h declares (checked by the CPU tests)
 EXPORTS = [
-    "gsq_init", "gsq_step", "gsq_last_loss", "gsq_loss_history",
+    "gsq_init", "gsq_step", "gsq_run", "gsq_last_loss", "gsq_loss_history",
     "gsq_packed_bytes", "gsq_harden_pack", "gsq_recon_error",
     "gsq_state_bytes", "gsq_export_state", "gsq_import_state", "gsq_get_step",
     "gsq_destroy", "gsq_error_string", "gsq_set_timing", "gsq_phase_times",
@@ -53,6 +53,7 @@ _pp = C.POINTER(C.c_void_p)
 _SIGS = {
     "gsq_init": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64, _p],
     "gsq_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_run": [_p, _p, _i64, _f32, _f32, _f32],
     "gsq_last_loss": [_p, C.POINTER(C.c_double)],
     "gsq_loss_history": [_p, _u64, _i64, _p],
     "gsq_packed_bytes": [_i32, _i64, _i64, C.POINTER(_sz)],
@@ -189,6 +190,13 @@ def gsq_step(layer: "Layer", tau: float, lr: float, beta1: float = 0.9,
     _check(_lib.gsq_step(layer.ctx, tau, lr, beta1, beta2), "gsq_step")
 
 
+def gsq_run(layer: "Layer", taus, lr: float, beta1: float = 0.9,
+            beta2: float = 0.99) -> None:
+    t = np.ascontiguousarray(taus, dtype=np.float32).ravel()
+    _check(_lib.gsq_run(layer.ctx, t.ctypes.data, t.size, lr, beta1, beta2),
+           "gsq_run")
+
+
 def gsq_last_loss(layer: "Layer") -> float:
     v = C.c_double()
     _check(_lib.gsq_last_loss(layer.ctx, C.byref(v)), "gsq_last_loss")
@@ -251,8 +259,8 @@ def gsq_set_timing(layer: "Layer", on: bool) -> None:
 
 
 def gsq_phase_times(layer: "Layer"):
-    ms = np.zeros(4, np.float64)
-    n = np.zeros(4, np.int64)
+    ms = np.zeros(5, np.float64)
+    n = np.zeros(5, np.int64)
     _check(_lib.gsq_phase_times(layer.ctx, ms.ctypes.data, n.ctypes.data),
            "gsq_phase_times")
     return ms, n
@@ -330,6 +338,9 @@ class Layer:
     # convenience -------------------------------------------------------
     def step(self, tau, lr, beta1=0.9, beta2=0.99):
         gsq_step(self, tau, lr, beta1, beta2)
+
+    def run(self, taus, lr, beta1=0.9, beta2=0.99):
+        gsq_run(self, taus, lr, beta1, beta2)
 
     def last_loss(self):
         return gsq_last_loss(self)

@@ -355,6 +355,31 @@ def test_first_config_full_trajectory(g, oracle_mod):
     lay.close()
 
 
+@pytest.mark.parametrize("mode,shape", [(0, (256, 512, 256)), (1, (200, 384, 200)),
+                                        (2, (136, 256, 72))])
+def test_run_equals_step_loop_bit_exact(g, mode, shape):
+    """gsq_run fuses each step's backward with the next step's soft weight;
+    the state and losses must equal those of separate gsq_step calls bit for
+    bit (same arithmetic, different kernel boundaries)."""
+    N, K, T = shape
+    cfg, W, X = make_case(mode, N, K, T)
+    taus = synth.tau_schedule(1.0, 0.05, 12)
+    a = gpu_layer(g, W, X, mode, seed=3)
+    b = gpu_layer(g, W, X, mode, seed=3)
+    la = []
+    for tau in taus:
+        a.step(float(tau), 1e-3)
+        la.append(a.last_loss())
+    b.run(taus[:5], 1e-3)
+    b.run(taus[5:], 1e-3)
+    hist = np.zeros(12)
+    g._check(g.lib().gsq_loss_history(b.ctx, 0, 12, hist.ctypes.data), "hist")
+    assert list(hist) == la
+    for which in (g.GSQ_DBG_LOGITS, g.GSQ_DBG_MOM, g.GSQ_DBG_SCALES, g.GSQ_DBG_SMOM):
+        assert np.array_equal(a.get(which), b.get(which))
+    a.close(); b.close()
+
+
 def test_checkpoint_resume_bit_exact(g):
     cfg, W, X = make_case(2, 136, 256, 72)
     taus = synth.tau_schedule(1.0, 0.1, 10)
