@@ -247,7 +247,7 @@ GSQ_API int gsq_uniforms_noalloc(int grid_mode, uint64_t seed, uint32_t t,
  * gsq_gemm_bf16_abt -- the library's tcgen05 GEMM on its own:
  * C (M x N fp32, row-major, ldc = N) = A (M x Kc bf16, row-major) .
  * B (N x Kc bf16, row-major)^T with fp32 accumulation; device pointers,
- * 16-byte aligned, Kc % 8 == 0.  Enqueued on `stream`; syncs.
+ * 16-byte aligned, Kc % 8 == 0, N % 4 == 0.  Enqueued on `stream`; syncs.
  */
 GSQ_API int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
                       int64_t N, int64_t Kc, void* stream);

@@ -55,7 +55,9 @@ struct gsq_ctx {
   int64_t what_t = -1;
   float what_tau = 0.f;
   double yref_sq = 0.0;
-  CUtensorMap tm_What, tm_Xb, tm_dYt, tm_Xt;
+  CUtensorMap tm_What, tm_Xb, tm_dYt, tm_Xt;  // GEMM operands
+  EpiMaps em_forward;  // dY^T (bf16) out, Y_ref^T in
+  EpiMaps em_wgrad;    // dW (fp32) out
   std::vector<void*> allocs;
 
   bool timing = false;
@@ -153,13 +155,9 @@ StepArgs step_args(gsq_ctx* c, float tau) {
   return a;
 }
 
-EpiParams forward_params(gsq_ctx* c, double* loss_out, bool with_dy) {
+EpiParams forward_params(gsq_ctx* c, double* loss_out) {
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
-  ep.yref = c->YrefT;
-  ep.ldy = c->Tp;
-  ep.dy = with_dy ? c->dYt : nullptr;
-  ep.lddy = c->Tp;
   ep.partials = c->partials;
   ep.ticket = c->ticket;
   ep.loss_out = loss_out;
@@ -168,18 +166,18 @@ EpiParams forward_params(gsq_ctx* c, double* loss_out, bool with_dy) {
 }
 
 cudaError_t run_forward(gsq_ctx* c, double* loss_out, int epi) {
-  EpiParams ep = forward_params(c, loss_out, epi == EPI_LOSS_DY);
-  return launch_gemm(c->tm_What, c->tm_Xb, c->N, c->Tp, c->K, epi, ep, c->sms,
+  EpiParams ep = forward_params(c, loss_out);
+  return launch_gemm(c->tm_What, c->tm_Xb, c->em_forward, c->N, c->Tp, c->K,
+                     epi, ep, c->sms,
                      c->st);
 }
 
 cudaError_t run_weight_grad(gsq_ctx* c) {
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
-  ep.out = c->dW;
-  ep.ldo = c->K;
   ep.err = c->err;
-  return launch_gemm(c->tm_dYt, c->tm_Xt, c->N, c->K, c->Tp, EPI_STORE_F32, ep,
+  return launch_gemm(c->tm_dYt, c->tm_Xt, c->em_wgrad, c->N, c->K, c->Tp,
+                     EPI_STORE_F32, ep,
                      c->sms, c->st);
 }
 
@@ -341,17 +339,22 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
       make_tmap_bf16(&c->tm_dYt, c->dYt, N, Tp, Tp, kGemmBoxRowsA) ||
       make_tmap_bf16(&c->tm_Xt, c->Xt, K, Tp, Tp, kGemmBoxRowsB) ||
       make_tmap_bf16(&tmW, Wop, N, kw * K, kw * K, kGemmBoxRowsA) ||
-      make_tmap_bf16(&tmXr, split ? Xcat : c->Xb, Tp, kw * K, kw * K, kGemmBoxRowsB))
+      make_tmap_bf16(&tmXr, split ? Xcat : c->Xb, Tp, kw * K, kw * K, kGemmBoxRowsB) ||
+      make_tmap_epi_bf16(&c->em_forward.out, c->dYt, N, Tp, Tp) ||
+      make_tmap_epi_f32(&c->em_forward.yref, c->YrefT, N, Tp, Tp) ||
+      make_tmap_epi_f32(&c->em_wgrad.out, c->dW, N, K, K))
     return cleanup_fail(GSQ_ERR_CUDA);
+  c->em_wgrad.yref = c->em_forward.yref;  // unused by the fp32-store epilogue
 
   // Y_ref^T = W . bf16(X)^T (fp32 accumulate; W at its own precision)
   {
     EpiParams ep;
     std::memset(&ep, 0, sizeof(ep));
-    ep.out = c->YrefT;
-    ep.ldo = Tp;
     ep.err = c->err;
-    ok(launch_gemm(tmW, tmXr, N, Tp, kw * K, EPI_STORE_F32, ep, c->sms, st));
+    EpiMaps em;
+    em.out = c->em_forward.yref;  // Y_ref^T is this GEMM's fp32 output
+    em.yref = c->em_forward.yref;
+    ok(launch_gemm(tmW, tmXr, em, N, Tp, kw * K, EPI_STORE_F32, ep, c->sms, st));
   }
   ok(launch_init_state(grid_mode, W32, idx_d, N, K, c->s, c->i0, c->logits,
                        c->err, st));
@@ -777,6 +780,7 @@ int gsq_debug_backward(gsq_ctx* c, float tau, float lr, float beta1,
 int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
                       int64_t N, int64_t Kc, void* stream) {
   if (!A || !B || !Cout || M <= 0 || N <= 0 || Kc <= 0 || Kc % 8 != 0 ||
+      N % 4 != 0 || (reinterpret_cast<uintptr_t>(Cout) & 15) ||
       (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(B) & 15))
     return GSQ_ERR_INVALID_ARG;
   int dev = 0;
@@ -799,12 +803,16 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
   }
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
-  ep.out = Cout;
-  ep.ldo = N;
   ep.err = err;
+  EpiMaps em;
+  if (make_tmap_epi_f32(&em.out, Cout, M, N, N)) {
+    cudaFree(err);
+    return GSQ_ERR_CUDA;
+  }
+  em.yref = em.out;
   cudaError_t e = cudaMemsetAsync(err, 0, 16, st);
   if (e == cudaSuccess)
-    e = launch_gemm(ta, tb, M, N, Kc, EPI_STORE_F32, ep, prop.multiProcessorCount, st);
+    e = launch_gemm(ta, tb, em, M, N, Kc, EPI_STORE_F32, ep, prop.multiProcessorCount, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   int h = 0;
   if (e == cudaSuccess) e = cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost);

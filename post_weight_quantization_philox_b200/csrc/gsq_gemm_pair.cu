@@ -6,12 +6,17 @@
 // A cluster of two CTAs on neighbouring SMs owns a 256 x 256 output tile:
 // CTA r loads rows [128 r, 128 r + 128) of the A tile and rows
 // [128 r, 128 r + 128) of the B tile (half of the tile's N) into its own
-// shared memory, in 64-wide K slabs through a 6-deep ring (32 KB per
+// shared memory, in 64-wide K slabs through a 5-deep ring (32 KB per
 // stage).  One thread of the leader CTA (rank 0) issues
 // tcgen05.mma.cta_group::2 with M = 256, N = 256, which reads A and B from
 // both CTAs and accumulates 128 rows into each CTA's TMEM.  Compared with a
 // single CTA computing 128 x 256, each CTA moves a third fewer operand bytes
 // per MMA, and the deeper ring hides more load latency.
+//
+// The epilogue stages each 32 x 32 piece of output in shared memory in the
+// TMA swizzle layout and writes it with one TMA store (full lines, issued
+// asynchronously), and reads Y_ref through TMA loads issued two pieces
+// ahead; per-thread row-wise global accesses slowed the main loop.
 //
 // Both CTAs' TMA loads count their bytes on the leader's "full" barrier; the
 // MMA thread signals each CTA's "empty" and "accumulator full" barriers with
@@ -27,7 +32,7 @@ namespace gsq {
 namespace {
 
 constexpr int PM = 256, PN = 256, HALF = 128, BK = 64;
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = HALF * BK * 2;
 constexpr int B_BYTES = HALF * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -42,12 +47,37 @@ struct Ctl {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
+  uint64_t ybar[4][2];  // Y_ref tile loads of each epilogue warp
   uint32_t tmem_base;
   int abort;
   double red[4];
 };
 
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctl);
+// Epilogue staging per epilogue warp (32 rows x 32 columns per unit, two
+// buffers each): fp32 out tiles 4 KB, Y_ref tiles 4 KB, bf16 dY tiles 2 KB.
+constexpr int OUT_TILE = 32 * 32 * 4;
+constexpr int DY_TILE = 32 * 32 * 2;
+template <int EPI>
+__host__ __device__ constexpr int warp_stage_bytes() {
+  return EPI == EPI_STORE_F32 ? 2 * OUT_TILE
+                              : (EPI == EPI_LOSS_DY ? 2 * OUT_TILE + 2 * DY_TILE
+                                                    : 2 * OUT_TILE);
+}
+template <int EPI>
+__host__ __device__ constexpr int smem_bytes() {
+  return STAGES * STAGE_BYTES + 4 * warp_stage_bytes<EPI>() + 1024 +
+         (int)sizeof(Ctl);
+}
+
+// shared-memory offset of 16-byte chunk j of row r in a tile written or
+// read by TMA with 128-byte rows / 128-byte swizzle, or 64-byte rows /
+// 64-byte swizzle (the tile base is 1024-byte aligned)
+__device__ __forceinline__ uint32_t swz128(int r, int j) {
+  return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ uint32_t swz64(int r, int j) {
+  return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   const bool ok = mbar_wait_bounded(bar, parity, WAIT_LIMIT);
@@ -57,12 +87,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA,
-                const __grid_constant__ CUtensorMap tmB, int64_t M, int64_t N,
+                const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmO,
+                const __grid_constant__ CUtensorMap tmY, int64_t M, int64_t N,
                 int64_t Kc, EpiParams ep) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* stage_area = smem + STAGES * STAGE_BYTES;
+  Ctl* ctl = reinterpret_cast<Ctl*>(stage_area + 4 * warp_stage_bytes<EPI>());
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -85,8 +118,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&ctl->tempty[b]), 8);  // 4 epilogue warps x 2 CTAs
     }
     mbar_init(smem_u32(&ctl->done), 1);
+    for (int w = 0; w < 4; ++w)
+      for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&ctl->ybar[w][b]), 1);
     ctl->abort = 0;
     mbar_fence_init();
+    if (EPI != EPI_LOSS) tma_prefetch_desc(&tmO);
+    if (EPI != EPI_STORE_F32) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -202,32 +239,126 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter of this warp
-    const int r = q * 32 + lane;
+    // Warp w (2..5) drains TMEM lanes [32 q, 32 q + 32), q = w % 4, in units
+    // of 32 columns: tcgen05.ld -> registers -> (Y_ref from a TMA-loaded
+    // tile) -> swizzled shared-memory tile -> one TMA store of 32 x 32.
+    const int q = warp & 3;
+    const int ew = warp - 2;
+    uint8_t* wst = stage_area + ew * warp_stage_bytes<EPI>();
+    const uint32_t out_s = smem_u32(wst);                  // 2 x OUT_TILE
+    const uint32_t y_s = smem_u32(wst);                    // 2 x OUT_TILE
+    const uint32_t dy_s = smem_u32(wst + 2 * OUT_TILE);    // 2 x DY_TILE
+    constexpr int UNITS = PN / 32;
+    const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
+    const int64_t total_units = (int64_t)my_tiles * UNITS;
+    // coordinates (x = column, y = first row) of unit u of this warp
+    auto unit_xy = [&](int64_t u, int32_t& x, int32_t& y) {
+      const int tile = pair + (int)(u / UNITS) * npairs;
+      const int mb = tile % m_tiles, nb = tile / m_tiles;
+      x = nb * PN + (int)(u % UNITS) * 32;
+      y = mb * PM + (int)rank * HALF + q * 32;
+    };
+    int64_t y_issued = 0;
+    auto issue_y = [&](int64_t u) {  // lane 0: Y_ref tile of unit u
+      int32_t x, y;
+      unit_xy(u, x, y);
+      const uint32_t bar = smem_u32(&ctl->ybar[ew][u & 1]);
+      mbar_arrive_expect_tx(bar, OUT_TILE);
+      tma_load_2d(y_s + (uint32_t)((u & 1) * OUT_TILE), &tmY, bar, x, y);
+    };
+    if (EPI != EPI_STORE_F32 && lane == 0) {
+      for (; y_issued < 2 && y_issued < total_units; ++y_issued) issue_y(y_issued);
+    }
     int acc = 0;
     uint32_t aph = 0;
     double lsum = 0.0;
-    for (int tile = pair; tile < num_tiles; tile += npairs) {
-      const int mb = tile % m_tiles, nb = tile / m_tiles;
+    int64_t u = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
       if (!warp_wait(smem_u32(&ctl->tfull[acc]), aph) ||
           *(volatile int*)&ctl->abort) {
-        if (lane == 0) {
-          atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
-          *(volatile int*)&ctl->abort = 1;
-        }
+        ok = false;
         break;
       }
       tc_fence_after();
-      const int64_t row = (int64_t)mb * PM + (int64_t)rank * HALF + r;
       const uint32_t tbase =
           tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * PN);
       float part = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < PN / 32; ++c) {
+      for (int c = 0; c < UNITS; ++c, ++u) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), v);
         tmem_wait_ld();
-        epilogue_chunk<EPI>(v, row, (int64_t)nb * PN + c * 32, M, N, ep, part);
+        int32_t x, y;
+        unit_xy(u, x, y);
+        const int b = (int)(u & 1);
+        if (EPI == EPI_STORE_F32) {
+          if (lane == 0) bulk_wait_read<1>();  // this buffer's last store read it
+          __syncwarp();
+          const uint32_t base = out_s + (uint32_t)(b * OUT_TILE);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t a = base + swz128(lane, j);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                         "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]),
+                         "r"(v[4 * j + 3])
+                         : "memory");
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmO, base, x, y);
+            bulk_commit();
+          }
+        } else {
+          // Y_ref of this unit, loaded by TMA (zero outside the matrix)
+          if (!warp_wait(smem_u32(&ctl->ybar[ew][b]), (uint32_t)((u >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          const uint32_t ybase = y_s + (uint32_t)(b * OUT_TILE);
+          float e[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 y4;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(y4.x), "=f"(y4.y), "=f"(y4.z), "=f"(y4.w)
+                         : "r"(ybase + swz128(lane, j))
+                         : "memory");
+            e[4 * j] = __uint_as_float(v[4 * j]) - y4.x;
+            e[4 * j + 1] = __uint_as_float(v[4 * j + 1]) - y4.y;
+            e[4 * j + 2] = __uint_as_float(v[4 * j + 2]) - y4.z;
+            e[4 * j + 3] = __uint_as_float(v[4 * j + 3]) - y4.w;
+          }
+          __syncwarp();  // every lane has read this Y_ref buffer
+          if (lane == 0 && y_issued < total_units && y_issued == u + 2) {
+            issue_y(y_issued);
+            ++y_issued;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) part = fmaf(e[j], e[j], part);
+          if (EPI == EPI_LOSS_DY) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            const uint32_t dbase = dy_s + (uint32_t)(b * DY_TILE);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t a = dbase + swz64(lane, j);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                           "r"(pack_bf16x2(2.f * e[8 * j], 2.f * e[8 * j + 1])),
+                           "r"(pack_bf16x2(2.f * e[8 * j + 2], 2.f * e[8 * j + 3])),
+                           "r"(pack_bf16x2(2.f * e[8 * j + 4], 2.f * e[8 * j + 5])),
+                           "r"(pack_bf16x2(2.f * e[8 * j + 6], 2.f * e[8 * j + 7]))
+                           : "memory");
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, dbase, x, y);
+              bulk_commit();
+            }
+          }
+        }
       }
       lsum += (double)part;
       tc_fence_before();
@@ -236,6 +367,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc ^= 1;
       if (acc == 0) aph ^= 1;
     }
+    if (!ok && lane == 0) {
+      atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+      *(volatile int*)&ctl->abort = 1;
+    }
+    if (lane == 0) {
+      // Y_ref loads still in flight land before the CTA exits
+      for (int64_t k = u; k < y_issued; ++k)
+        if (!mbar_wait_bounded(smem_u32(&ctl->ybar[ew][k & 1]),
+                               (uint32_t)((k >> 1) & 1), WAIT_LIMIT))
+          atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+      bulk_wait_all();  // stores complete before the CTA exits
+    }
+    __syncwarp();
     if (EPI != EPI_STORE_F32) {
       lsum = warp_sum_d(lsum);
       if (lane == 0) ctl->red[q] = lsum;
@@ -256,8 +400,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int EPI>
 cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                            int64_t M, int64_t N, int64_t Kc,
-                            const EpiParams& ep, int sm_count,
+                            const EpiMaps& maps, int64_t M, int64_t N,
+                            int64_t Kc, const EpiParams& ep, int sm_count,
                             cudaStream_t st) {
   static int max_pairs = 0;
   cudaLaunchAttribute attr[1];
@@ -267,13 +411,13 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_bytes<EPI>();
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs == 0) {
     cudaError_t e = cudaFuncSetAttribute(
-        k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<EPI>());
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
     int n = 0;
@@ -286,22 +430,23 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
   const int64_t tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
-  return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI>, tmA, tmB, M, N, Kc, ep);
+  return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI>, tmA, tmB, maps.out, maps.yref,
+                            M, N, Kc, ep);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                             int64_t M, int64_t N, int64_t Kc, int mode,
-                             const EpiParams& ep, int sm_count,
-                             cudaStream_t st) {
+                             const EpiMaps& maps, int64_t M, int64_t N,
+                             int64_t Kc, int mode, const EpiParams& ep,
+                             int sm_count, cudaStream_t st) {
   switch (mode) {
     case EPI_STORE_F32:
-      return launch_pair_epi<EPI_STORE_F32>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_STORE_F32>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
     case EPI_LOSS_DY:
-      return launch_pair_epi<EPI_LOSS_DY>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_LOSS_DY>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
     default:
-      return launch_pair_epi<EPI_LOSS>(tmA, tmB, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_LOSS>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
   }
 }
 

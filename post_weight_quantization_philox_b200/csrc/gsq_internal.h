@@ -24,22 +24,31 @@ enum EpiMode : int {
 };
 
 struct EpiParams {
-  float* out;            // EPI_STORE_F32: M x ldo
-  int64_t ldo;
-  const float* yref;     // EPI_LOSS*: M x ldy
-  int64_t ldy;
-  __nv_bfloat16* dy;     // EPI_LOSS_DY: M x lddy
-  int64_t lddy;
   double* partials;      // one slot per CTA
   unsigned* ticket;      // zero between launches
   double* loss_out;      // final loss (fp64)
   int* err;              // device error word
 };
 
+// The epilogue's tensor maps: out = C (EPI_STORE_F32, fp32 map) or dY
+// (EPI_LOSS_DY, bf16 map); yref = Y_ref (EPI_LOSS*, fp32 map).  Unused maps
+// may be any valid map.
+struct EpiMaps {
+  CUtensorMap out;
+  CUtensorMap yref;
+};
+
 // Encodes a 2-D bf16 tensor map (rows x cols, row stride ld elements) with
-// a box of box_rows x 64 elements and 128-byte swizzling.
+// a box of box_rows x 64 elements and 128-byte swizzling (GEMM operands).
 int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows,
                    int64_t cols, int64_t ld, int box_rows);
+// Tensor maps of the GEMM epilogue's 32 x 32 tiles: fp32 (128-byte rows,
+// 128-byte swizzle) for stored or read fp32 outputs, bf16 (64-byte rows,
+// 64-byte swizzle) for the bf16 output gradient.
+int make_tmap_epi_f32(CUtensorMap* map, const void* base, int64_t rows,
+                      int64_t cols, int64_t ld);
+int make_tmap_epi_bf16(CUtensorMap* map, const void* base, int64_t rows,
+                       int64_t cols, int64_t ld);
 
 // Box rows of the tensor maps the GEMM expects for A and for B.
 constexpr int kGemmBoxRowsA = 128;
@@ -49,12 +58,13 @@ constexpr int kGemmBoxRowsB = 128;
 // (CTA-pair tcgen05 kernel); tmA / tmB made by make_tmap_bf16 with
 // kGemmBoxRowsA / kGemmBoxRowsB rows per box.
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        int64_t M, int64_t N, int64_t Kc, int mode,
-                        const EpiParams& ep, int sm_count, cudaStream_t st);
+                        const EpiMaps& maps, int64_t M, int64_t N, int64_t Kc,
+                        int mode, const EpiParams& ep, int sm_count,
+                        cudaStream_t st);
 cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                             int64_t M, int64_t N, int64_t Kc, int mode,
-                             const EpiParams& ep, int sm_count,
-                             cudaStream_t st);
+                             const EpiMaps& maps, int64_t M, int64_t N,
+                             int64_t Kc, int mode, const EpiParams& ep,
+                             int sm_count, cudaStream_t st);
 
 // ------------------------------------------------------- elementwise
 struct StepArgs {
