@@ -261,25 +261,24 @@ def run_e2e(gsq, torch, cfg, W, X, rank):
 
 def cpu_baseline(cfg, budget_s=15.0, steps=None):
     """The oracle on the host cores: a row slice of the same layer (the loss
-    decomposes over rows), full K and T, timed per step."""
+    decomposes over rows), full K and T, steps timed alone (init excluded).
+    The slice is sized from one calibration step to fill about budget_s."""
     import oracle
     oracle.build()
-    threads = os.cpu_count()
-    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
     W = synth.make_weight(cfg)
     X = synth.make_calib(cfg)
-    rows = 1
-    # calibrate: one step of one row, then scale rows to the budget
-    st = oracle.init(cfg.grid, W[:rows], seed=0)
-    Y = oracle.reference_output(W[:rows], X)
-    t0 = time.perf_counter()
-    oracle.step(st, X, Y, 1.0, cfg.lr)
-    one = time.perf_counter() - t0
     nsteps = steps or 2
-    rows = int(max(1, min(cfg.N, budget_s / max(one * nsteps, 1e-6))))
+    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
+    r0 = min(8, cfg.N)
+    st = oracle.init(cfg.grid, W[:r0], seed=0)
+    Y = oracle.reference_output(W[:r0], X)
+    t0 = time.perf_counter()
+    oracle.step(st, X, Y, float(taus[0]), cfg.lr)
+    per_row = (time.perf_counter() - t0) / r0
+    rows = int(max(1, min(cfg.N, budget_s / max(per_row * nsteps, 1e-9))))
     st = oracle.init(cfg.grid, W[:rows], seed=0)
     Y = oracle.reference_output(W[:rows], X)
-    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
     t0 = time.perf_counter()
     for i in range(nsteps):
         oracle.step(st, X, Y, float(taus[i]), cfg.lr)
