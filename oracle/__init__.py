@@ -80,6 +80,8 @@ def lib():
             "gsqo_recon_error": (None, [_i32, _i32, _i64, _i64, _i64, _i32, _p,
                                         _p, _p, _p, _p, _f32, _p, _p]),
             "gsqo_gemm_abt": (None, [_i64, _i64, _i64, _p, _p, _p]),
+            "gsqo_mlp_forward_backward": (_f64, [_i64, _i64, _i64, _p, _p, _p, _p,
+                                                 _p, _i32, _p, _p, _p]),
         }
         for name, (res, args) in sigs.items():
             f = getattr(_lib, name)
@@ -321,3 +323,80 @@ def gemm_abt(A, B):
     Cm = np.zeros((M, N))
     lib().gsqo_gemm_abt(M, N, Kc, _ptr(A), _ptr(B), _ptr(Cm))
     return Cm
+
+
+# ------------------------------------------------- SwiGLU MLP joint stage
+
+MLP_WEIGHTS = ("gate", "up", "down")
+
+
+def mlp_forward_backward(Xn, R, Wg, Wu, Wd, round_bf16=True):
+    """loss, dWg, dWu, dWd of the SwiGLU MLP stage (see gsq_oracle.h)."""
+    Xn, Wg, Wu, Wd = _f32a(Xn), _f32a(Wg), _f32a(Wu), _f32a(Wd)
+    R = np.ascontiguousarray(R, np.float64)
+    T, H = Xn.shape
+    F = Wg.shape[0]
+    dWg = np.zeros((F, H), np.float32)
+    dWu = np.zeros((F, H), np.float32)
+    dWd = np.zeros((H, F), np.float32)
+    loss = lib().gsqo_mlp_forward_backward(T, H, F, _ptr(Xn), _ptr(R), _ptr(Wg),
+                                           _ptr(Wu), _ptr(Wd), int(round_bf16),
+                                           _ptr(dWg), _ptr(dWu), _ptr(dWd))
+    return loss, dWg, dWu, dWd
+
+
+def weight_seed(seed: int, which: int) -> int:
+    """Philox key of weight `which` of a block stage: the seed's high key word
+    xored with which << 16, so every weight draws its own stream."""
+    return (seed ^ (which << 48)) & 0xFFFFFFFFFFFFFFFF
+
+
+@dataclass
+class MlpState:
+    gate: State
+    up: State
+    down: State
+    t: int = 0
+
+    def weights(self):
+        return (self.gate, self.up, self.down)
+
+
+def mlp_init(mode, Wg, Wu, Wd, group=128, seed=0):
+    sts = [init(mode, W, group, seed=weight_seed(seed, i))
+           for i, W in enumerate((Wg, Wu, Wd))]
+    return MlpState(*sts)
+
+
+def mlp_step(ms: MlpState, Xn, R, tau, lr, beta1=0.9, beta2=0.99, dumps=False):
+    """One joint step: soft weights of the three weights (their own noise),
+    SwiGLU forward/backward against R, then backward + Lion per weight."""
+    wb = []
+    for st in ms.weights():
+        st.t = ms.t
+        wb.append(soft_weight(st, tau)[3])
+    loss, dWg, dWu, dWd = mlp_forward_backward(Xn, R, *wb)
+    for st, dW in zip(ms.weights(), (dWg, dWu, dWd)):
+        backward_lion(st, dW, tau, lr, beta1, beta2)
+    ms.t += 1
+    for st in ms.weights():
+        st.t = ms.t
+    if dumps:
+        return loss, dict(w=wb, dW=(dWg, dWu, dWd))
+    return loss
+
+
+def mlp_recon_error(ms: MlpState, Xn, R, emode=0, tau=1.0):
+    """||MLP(Xn) - R||^2 with the hard (emode 0) or noiseless soft (1) weights."""
+    ws = []
+    for st in ms.weights():
+        if emode == 0:
+            lev = harden(st.mode, st.logits, st.i0)
+            vals = np.array([-1.5, -0.5, 0.5, 1.5]) if st.mode == GRID_2BIT else (
+                np.array([-1.0, 0.0, 1.0]) if st.mode == GRID_TERNARY else np.arange(8) - 3.5)
+            w = np.repeat(st.s, st.group, axis=1).astype(np.float64) * vals[lev]
+            ws.append(bf16_round(w).astype(np.float32))
+        else:
+            ws.append(soft_weight(st, tau, noise=False)[3])
+    loss, _, _, _ = mlp_forward_backward(Xn, R, *ws)
+    return loss, loss / float((np.asarray(R, np.float64) ** 2).sum())

@@ -624,3 +624,93 @@ void gsqo_recon_error(int gmode, int emode, int64_t N, int64_t K, int64_t T,
     *rel_err = (y2 > 0.0) ? e2 / y2 : 0.0;
     free(wq);
 }
+
+/* --------------------------------------------------- SwiGLU MLP stage */
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* The block's MLP stage (agihunt.info summary, optimisation paragraph: the
+ * MLP is trained on the block output after the attention stages): one
+ * forward and backward pass of the SwiGLU MLP against the fixed target R. */
+double gsqo_mlp_forward_backward(int64_t T, int64_t H, int64_t F,
+                                 const float* Xn, const double* R,
+                                 const float* Wg, const float* Wu,
+                                 const float* Wd, int round, float* dWg,
+                                 float* dWu, float* dWd) {
+    double* a = (double*)malloc((size_t)(T * F) * sizeof(double));
+    double* b = (double*)malloc((size_t)(T * F) * sizeof(double));
+    double* h = (double*)malloc((size_t)(T * F) * sizeof(double));
+    double* dp = (double*)malloc((size_t)(T * H) * sizeof(double));
+    double* da = (double*)malloc((size_t)(T * F) * sizeof(double));
+    double* db = (double*)malloc((size_t)(T * F) * sizeof(double));
+    double* part = (double*)malloc((size_t)T * sizeof(double));
+    /* a, b, h */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t f = 0; f < F; ++f) {
+            double sa = 0.0, sb = 0.0;
+            for (int64_t k = 0; k < H; ++k) {
+                double x = round ? gsqo_bf16_round(Xn[t * H + k]) : (double)Xn[t * H + k];
+                sa += x * Wg[f * H + k];
+                sb += x * Wu[f * H + k];
+            }
+            a[t * F + f] = sa;
+            b[t * F + f] = sb;
+            double hv = sa * sigmoid(sa) * sb; /* silu(a) * b */
+            h[t * F + f] = round ? gsqo_bf16_round(hv) : hv;
+        }
+    /* pred, E, loss, dpred = 2E */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double row = 0.0;
+        for (int64_t n = 0; n < H; ++n) {
+            double acc = 0.0;
+            for (int64_t f = 0; f < F; ++f) acc += h[t * F + f] * Wd[n * F + f];
+            double e = acc - R[t * H + n];
+            row += e * e;
+            dp[t * H + n] = round ? gsqo_bf16_round(2.0 * e) : 2.0 * e;
+        }
+        part[t] = row;
+    }
+    double loss = 0.0;
+    for (int64_t t = 0; t < T; ++t) loss += part[t];
+    /* dh = dpred Wd; da = dh b silu'(a); db = dh silu(a) */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t f = 0; f < F; ++f) {
+            double dh = 0.0;
+            for (int64_t n = 0; n < H; ++n) dh += dp[t * H + n] * Wd[n * F + f];
+            double av = a[t * F + f], sg = sigmoid(av);
+            double dsilu = sg * (1.0 + av * (1.0 - sg));
+            double gav = dh * b[t * F + f] * dsilu;
+            double gbv = dh * av * sg;
+            da[t * F + f] = round ? gsqo_bf16_round(gav) : gav;
+            db[t * F + f] = round ? gsqo_bf16_round(gbv) : gbv;
+        }
+    /* weight gradients */
+    if (dWd) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < H; ++n)
+            for (int64_t f = 0; f < F; ++f) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + f];
+                dWd[n * F + f] = (float)acc;
+            }
+    }
+    if (dWg || dWu) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t f = 0; f < F; ++f)
+            for (int64_t k = 0; k < H; ++k) {
+                double ag = 0.0, au = 0.0;
+                for (int64_t t = 0; t < T; ++t) {
+                    double x = round ? gsqo_bf16_round(Xn[t * H + k]) : (double)Xn[t * H + k];
+                    ag += da[t * F + f] * x;
+                    au += db[t * F + f] * x;
+                }
+                if (dWg) dWg[f * H + k] = (float)ag;
+                if (dWu) dWu[f * H + k] = (float)au;
+            }
+    }
+    free(a); free(b); free(h); free(dp); free(da); free(db); free(part);
+    return loss;
+}

@@ -126,6 +126,20 @@ void gsqo_recon_error(int gmode, int emode, int64_t N, int64_t K, int64_t T,
                       const int8_t* i0, const float* X, const double* Yref,
                       float tau, double* abs_err, double* rel_err);
 
+/* SwiGLU MLP joint stage (the block's MLP trained on the block output).
+ * Xn (T x H): the normalised MLP input; R (T x H): the output the MLP must
+ * produce; Wg, Wu (F x H) and Wd (H x F): the three soft weights.
+ *   a = Xn Wg^T, b = Xn Wu^T, h = silu(a) b, pred = h Wd^T,
+ *   loss = sum (pred - R)^2, and the weight gradients dWg, dWu (F x H),
+ *   dWd (H x F) (nullable).  With round = 1 the GEMM operands that the
+ *   library keeps in bf16 (Xn, h, dpred = 2E, da, db) are rounded to bf16
+ *   as there; with round = 0 everything is exact fp64 (for the pins). */
+double gsqo_mlp_forward_backward(int64_t T, int64_t H, int64_t F,
+                                 const float* Xn, const double* R,
+                                 const float* Wg, const float* Wu,
+                                 const float* Wd, int round, float* dWg,
+                                 float* dWu, float* dWd);
+
 /* plain fp64 C = A . B^T for A (M x Kc), B (N x Kc), both row-major */
 void gsqo_gemm_abt(int64_t M, int64_t N, int64_t Kc, const float* A,
                    const float* B, double* C);

@@ -11,6 +11,7 @@ import pytest
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 sys.path.insert(0, HERE)
+import test_oracle_mlp as mlp_pins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
 
 # (name, original text, planted text, pins expected to catch it)
@@ -50,6 +51,13 @@ MUTATIONS = [
     ("pack_msb_first", "packed[n * wpr + bit / 32] |= (1u << (bit % 32));",
      "packed[n * wpr + bit / 32] |= (1u << (31 - bit % 32));",
      ["test_harden_bruteforce_and_pack_roundtrip"]),
+    ("mlp_silu_derivative", "double dsilu = sg * (1.0 + av * (1.0 - sg));",
+     "double dsilu = sg * (1.0 - av * (1.0 - sg));", ["mlp:test_mlp_matches_torch_autograd"]),
+    ("mlp_dropped_up_factor", "double gav = dh * b[t * F + f] * dsilu;",
+     "double gav = dh * dsilu;", ["mlp:test_mlp_matches_torch_autograd"]),
+    ("mlp_down_grad_transposed", "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + f];",
+     "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + (F - 1 - f)];",
+     ["mlp:test_mlp_matches_torch_autograd"]),
 ]
 
 MODES = {"test_softmax_is_library_softmax": [0, 2]}
@@ -75,7 +83,9 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
     mod = _load_mutant(tmp_path, name, old, new)
     caught = []
     for tname in catchers:
-        fn = getattr(pins, tname)
+        module = mlp_pins if tname.startswith("mlp:") else pins
+        tname = tname.split(":")[-1]
+        fn = getattr(module, tname)
         params = getattr(fn, "pytestmark", [])
         modes = MODES.get(tname)
         if modes is None:
