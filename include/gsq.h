@@ -220,6 +220,64 @@ GSQ_API int gsq_debug_weight_grad(gsq_ctx* ctx);
 GSQ_API int gsq_debug_backward(gsq_ctx* ctx, float tau, float lr, float beta1,
                        float beta2);
 
+/* ----------------------------------------------- block stage: SwiGLU MLP --
+ * The GSQ pages quantize a transformer block in stages; the last stage trains
+ * the MLP on the block output (agihunt.info summary, optimisation paragraph).
+ * gsq_mlp_* quantize the gate (F x H), up (F x H) and down (H x F)
+ * projections jointly against
+ *     loss = || D (silu(G Xn^T) * U Xn^T) - R^T ||_F^2
+ * where Xn (T x H) is the normalised MLP input and R (T x H) the output the
+ * MLP must produce (the full-precision block output minus the residual that
+ * enters the MLP).  Each weight has its own logits, scales, Lion state and
+ * Philox key (seed with weight index i xored into bits 48.. of the key);
+ * soft weights, backward + Lion, harden/pack and the grids are those of the
+ * single-layer entry points.  GEMM operands are bf16 with fp32 accumulation;
+ * h = silu(a) b, 2E, da and db are rounded to bf16 as GEMM operands.
+ *
+ * gsq_mlp_init: Xn, R, Wg, Wu, Wd host or device, dtypes GSQ_F32 / GSQ_BF16;
+ *   H and F multiples of 128 (the group), T a multiple of 64.  Syncs.
+ * gsq_mlp_step / gsq_mlp_run: as gsq_step / gsq_run for the joint loss.
+ * gsq_mlp_last_loss, gsq_mlp_recon_error (vs R; hard or noiseless soft),
+ * gsq_mlp_harden_pack(which = 0 gate, 1 up, 2 down; host or device outputs)
+ * as their single-layer counterparts.
+ * gsq_mlp_debug_get / _set: which = 0..2 with a GSQ_DBG_* weight buffer
+ *   (LOGITS, MOM, SCALES, SMOM, I0, WHAT, DW), or which = GSQ_MLP_STAGE with
+ *   a GSQ_MLP_DBG_* stage buffer (all "T" layouts are transposed: F x T or
+ *   H x T).
+ */
+typedef struct gsq_mlp gsq_mlp;
+#define GSQ_MLP_STAGE 3
+enum {
+    GSQ_MLP_DBG_AT = 0,   /* F x T fp32  a^T = G Xn^T          */
+    GSQ_MLP_DBG_BT = 1,   /* F x T fp32  b^T = U Xn^T          */
+    GSQ_MLP_DBG_HT = 2,   /* F x T bf16  h^T = silu(a^T) b^T   */
+    GSQ_MLP_DBG_DPT = 3,  /* H x T bf16  2 (pred^T - R^T)      */
+    GSQ_MLP_DBG_DHT = 4,  /* F x T fp32  dh^T = D^T dp^T       */
+    GSQ_MLP_DBG_DAT = 5,  /* F x T bf16  da^T                  */
+    GSQ_MLP_DBG_DBT = 6,  /* F x T bf16  db^T                  */
+    GSQ_MLP_DBG_RT = 7    /* H x T fp32  R^T                   */
+};
+GSQ_API int gsq_mlp_init(gsq_mlp** out, const void* Xn, int x_dtype,
+                         const void* R, int r_dtype, const void* Wg,
+                         const void* Wu, const void* Wd, int w_dtype,
+                         int64_t T, int64_t H, int64_t F, int group,
+                         int grid_mode, uint64_t seed, void* stream);
+GSQ_API int gsq_mlp_step(gsq_mlp* ctx, float tau, float lr, float beta1,
+                         float beta2);
+GSQ_API int gsq_mlp_run(gsq_mlp* ctx, const float* taus, int64_t n, float lr,
+                        float beta1, float beta2);
+GSQ_API int gsq_mlp_last_loss(gsq_mlp* ctx, double* loss);
+GSQ_API int gsq_mlp_recon_error(gsq_mlp* ctx, int mode, float tau,
+                                double* abs_err, double* rel_err);
+GSQ_API int gsq_mlp_harden_pack(gsq_mlp* ctx, int which, void* packed,
+                                uint16_t* scales_f16, float* scales_f32);
+GSQ_API int gsq_mlp_debug_get(gsq_mlp* ctx, int which, int buf, void* host,
+                              size_t bytes);
+GSQ_API int gsq_mlp_debug_set(gsq_mlp* ctx, int which, int buf,
+                              const void* host, size_t bytes);
+GSQ_API int gsq_mlp_get_step(gsq_mlp* ctx, uint64_t* t);
+GSQ_API int gsq_mlp_destroy(gsq_mlp* ctx);
+
 /*
  * gsq_uniforms_noalloc -- the L Philox uniforms of coords
  * [coord0, coord0 + count) at step t for grid_mode and seed (the values

@@ -118,5 +118,18 @@ cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
                             cudaStream_t st);
 cudaError_t launch_sumsq(const float* x, int64_t n, double* partials,
                          unsigned* ticket, double* out, cudaStream_t st);
+// SwiGLU MLP stage: h = bf16(silu(a) b); da = bf16(dh b silu'(a)),
+// db = bf16(dh silu(a)); n a multiple of 4
+cudaError_t launch_swiglu_fwd(const float* a, const float* b, int64_t n,
+                              __nv_bfloat16* h, int sm_count, cudaStream_t st);
+cudaError_t launch_swiglu_bwd(const float* a, const float* b, const float* dh,
+                              int64_t n, __nv_bfloat16* da, __nv_bfloat16* db,
+                              int sm_count, cudaStream_t st);
+// out (cols x rows) = in (rows x cols)^T
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows,
+                                  int64_t cols, __nv_bfloat16* out,
+                                  cudaStream_t st);
+cudaError_t launch_transpose_to_f32(const void* in, int in_bf16, int64_t rows,
+                                    int64_t cols, float* out, cudaStream_t st);
 
 }  // namespace gsq

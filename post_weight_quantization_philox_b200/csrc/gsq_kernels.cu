@@ -581,6 +581,93 @@ __global__ void __launch_bounds__(256) k_sumsq(const float* __restrict__ x,
   }
 }
 
+// ------------------------------------------------------ SwiGLU pieces
+// (the block's MLP stage: h = silu(a) * b and its derivatives)
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
+
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w) {
+  __nv_bfloat162 b01 = __floats2bfloat162_rn(w[0], w[1]);
+  __nv_bfloat162 b23 = __floats2bfloat162_rn(w[2], w[3]);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&b01);
+  pk.y = *reinterpret_cast<uint32_t*>(&b23);
+  *reinterpret_cast<uint2*>(dst) = pk;
+}
+
+// hT = bf16(silu(aT) * bT), elementwise over n entries
+__global__ void __launch_bounds__(256) k_swiglu_fwd(const float* __restrict__ a,
+                                                    const float* __restrict__ b,
+                                                    int64_t n,
+                                                    __nv_bfloat16* __restrict__ h) {
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n;
+       i += (int64_t)gridDim.x * blockDim.x * 4) {
+    const float4 a4 = __ldg(reinterpret_cast<const float4*>(a + i));
+    const float4 b4 = __ldg(reinterpret_cast<const float4*>(b + i));
+    const float hv[4] = {a4.x * sigmoidf_(a4.x) * b4.x, a4.y * sigmoidf_(a4.y) * b4.y,
+                         a4.z * sigmoidf_(a4.z) * b4.z, a4.w * sigmoidf_(a4.w) * b4.w};
+    store_bf16x4(h + i, hv);
+  }
+}
+
+// da = bf16(dh * b * silu'(a)), db = bf16(dh * silu(a)),
+// silu'(a) = sigma(a) (1 + a (1 - sigma(a)))
+__global__ void __launch_bounds__(256) k_swiglu_bwd(const float* __restrict__ a,
+                                                    const float* __restrict__ b,
+                                                    const float* __restrict__ dh,
+                                                    int64_t n,
+                                                    __nv_bfloat16* __restrict__ da,
+                                                    __nv_bfloat16* __restrict__ db) {
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n;
+       i += (int64_t)gridDim.x * blockDim.x * 4) {
+    const float4 a4 = __ldg(reinterpret_cast<const float4*>(a + i));
+    const float4 b4 = __ldg(reinterpret_cast<const float4*>(b + i));
+    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dh + i));
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+    float ga[4], gb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float sg = sigmoidf_(av[j]);
+      ga[j] = dv[j] * bv[j] * (sg * (1.f + av[j] * (1.f - sg)));
+      gb[j] = dv[j] * av[j] * sg;
+    }
+    store_bf16x4(da + i, ga);
+    store_bf16x4(db + i, gb);
+  }
+}
+
+// out (cols x rows) = in (rows x cols)^T, 64 x 64 tiles through shared memory
+template <typename TIn, typename TOut>
+__global__ void k_transpose(const TIn* __restrict__ in, int64_t rows,
+                            int64_t cols, TOut* __restrict__ out) {
+  __shared__ float tile[64][65];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 64 x 4
+  for (int r = ty; r < 64; r += 4) {
+    const int64_t rr = r0 + r, cc = c0 + tx;
+    float v = 0.f;
+    if (rr < rows && cc < cols) {
+      if constexpr (sizeof(TIn) == 2)
+        v = __bfloat162float(in[rr * cols + cc]);
+      else
+        v = in[rr * cols + cc];
+    }
+    tile[r][tx] = v;
+  }
+  __syncthreads();
+  for (int c = ty; c < 64; c += 4) {
+    const int64_t cc = c0 + c, rr = r0 + tx;
+    if (cc < cols && rr < rows) {
+      if constexpr (sizeof(TOut) == 2)
+        out[cc * rows + rr] = __float2bfloat16_rn(tile[tx][c]);
+      else
+        out[cc * rows + rr] = tile[tx][c];
+    }
+  }
+}
+
 int grid_for(int64_t work, int threads, int cap) {
   int64_t b = (work + threads - 1) / threads;
   if (b < 1) b = 1;
@@ -753,6 +840,38 @@ cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
     case GRID_TERNARY: k_uniforms<GRID_TERNARY><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out); break;
     default: k_uniforms<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_fwd(const float* a, const float* b, int64_t n,
+                              __nv_bfloat16* h, int sm_count, cudaStream_t st) {
+  k_swiglu_fwd<<<grid_for(n / 4, 256, sm_count * 8), 256, 0, st>>>(a, b, n, h);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_bwd(const float* a, const float* b, const float* dh,
+                              int64_t n, __nv_bfloat16* da, __nv_bfloat16* db,
+                              int sm_count, cudaStream_t st) {
+  k_swiglu_bwd<<<grid_for(n / 4, 256, sm_count * 8), 256, 0, st>>>(a, b, dh, n, da, db);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows,
+                                  int64_t cols, __nv_bfloat16* out,
+                                  cudaStream_t st) {
+  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+  k_transpose<__nv_bfloat16, __nv_bfloat16><<<grid, dim3(64, 4), 0, st>>>(in, rows, cols, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_to_f32(const void* in, int in_bf16, int64_t rows,
+                                    int64_t cols, float* out, cudaStream_t st) {
+  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+  if (in_bf16)
+    k_transpose<__nv_bfloat16, float><<<grid, dim3(64, 4), 0, st>>>(
+        (const __nv_bfloat16*)in, rows, cols, out);
+  else
+    k_transpose<float, float><<<grid, dim3(64, 4), 0, st>>>((const float*)in, rows, cols, out);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,9 @@ GSQ_NOALLOC_MAX_COORDS = 65536
 (GSQ_DBG_LOGITS, GSQ_DBG_MOM, GSQ_DBG_SCALES, GSQ_DBG_SMOM, GSQ_DBG_I0,
  GSQ_DBG_WHAT, GSQ_DBG_WSOFT32, GSQ_DBG_DW, GSQ_DBG_DYT, GSQ_DBG_YREFT,
  GSQ_DBG_DL, GSQ_DBG_DS) = range(12)
+GSQ_MLP_STAGE = 3
+(GSQ_MLP_DBG_AT, GSQ_MLP_DBG_BT, GSQ_MLP_DBG_HT, GSQ_MLP_DBG_DPT, GSQ_MLP_DBG_DHT,
+ GSQ_MLP_DBG_DAT, GSQ_MLP_DBG_DBT, GSQ_MLP_DBG_RT) = range(8)
 
 NUM_LOGITS = {GSQ_GRID_2BIT: 4, GSQ_GRID_TERNARY: 4, GSQ_GRID_3BIT_LOCAL: 5}
 
@@ -37,6 +40,9 @@ EXPORTS = [
     "gsq_debug_uniforms", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
+    "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
+    "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
+    "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
 ]
 
 
@@ -77,6 +83,17 @@ _SIGS = {
     "gsq_debug_backward": [_p, _f32, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
     "gsq_uniforms_noalloc": [_i32, _u64, _u32, _u64, _i64, _p, _p],
+    "gsq_mlp_init": [_pp, _p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i64, _i64,
+                     _i32, _i32, _u64, _p],
+    "gsq_mlp_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_mlp_run": [_p, _p, _i64, _f32, _f32, _f32],
+    "gsq_mlp_last_loss": [_p, C.POINTER(C.c_double)],
+    "gsq_mlp_recon_error": [_p, _i32, _f32, C.POINTER(C.c_double), C.POINTER(C.c_double)],
+    "gsq_mlp_harden_pack": [_p, _i32, _p, _p, _p],
+    "gsq_mlp_debug_get": [_p, _i32, _i32, _p, _sz],
+    "gsq_mlp_debug_set": [_p, _i32, _i32, _p, _sz],
+    "gsq_mlp_get_step": [_p, C.POINTER(_u64)],
+    "gsq_mlp_destroy": [_p],
 }
 
 
@@ -360,3 +377,109 @@ class Layer:
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     """bf16 bit patterns (uint16) -> float32 values (exact)."""
     return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------ block stage: SwiGLU MLP
+
+def gsq_mlp_init(Xn, R, Wg, Wu, Wd, group: int = 128,
+                 grid_mode: int = GSQ_GRID_2BIT, seed: int = 0, stream=None) -> "Mlp":
+    """Xn, R (T x H); Wg, Wu (F x H); Wd (H x F): numpy fp32 or torch fp32/bf16."""
+    xp, xdt, xk = _ptr_dtype(Xn)
+    rp, rdt, rk = _ptr_dtype(R)
+    gp, wdt, gk = _ptr_dtype(Wg)
+    up, udt, uk = _ptr_dtype(Wu)
+    dp, ddt, dk = _ptr_dtype(Wd)
+    if not (wdt == udt == ddt):
+        raise TypeError("Wg, Wu and Wd must share a dtype")
+    T, H = int(Xn.shape[0]), int(Xn.shape[1])
+    F = int(Wg.shape[0])
+    ctx = C.c_void_p()
+    _check(_lib.gsq_mlp_init(C.byref(ctx), xp, xdt, rp, rdt, gp, up, dp, wdt, T, H, F,
+                             group, grid_mode, seed & 0xFFFFFFFFFFFFFFFF,
+                             _stream_ptr(stream)), "gsq_mlp_init")
+    del xk, rk, gk, uk, dk
+    return Mlp(ctx, grid_mode, T, H, F, group)
+
+
+class Mlp:
+    """Context of the SwiGLU MLP stage (gate, up, down quantized jointly)."""
+
+    def __init__(self, ctx, mode, T, H, F, group):
+        self.ctx, self.mode, self.T, self.H, self.F, self.group = ctx, mode, T, H, F, group
+        self.L = NUM_LOGITS[mode]
+        self.shapes = ((F, H), (F, H), (H, F))
+
+    def step(self, tau, lr, beta1=0.9, beta2=0.99):
+        _check(_lib.gsq_mlp_step(self.ctx, tau, lr, beta1, beta2), "gsq_mlp_step")
+
+    def run(self, taus, lr, beta1=0.9, beta2=0.99):
+        t = np.ascontiguousarray(taus, dtype=np.float32).ravel()
+        _check(_lib.gsq_mlp_run(self.ctx, t.ctypes.data, t.size, lr, beta1, beta2),
+               "gsq_mlp_run")
+
+    def last_loss(self):
+        v = C.c_double()
+        _check(_lib.gsq_mlp_last_loss(self.ctx, C.byref(v)), "gsq_mlp_last_loss")
+        return v.value
+
+    def recon_error(self, mode=GSQ_RECON_HARD, tau=1.0):
+        a, r = C.c_double(), C.c_double()
+        _check(_lib.gsq_mlp_recon_error(self.ctx, mode, tau, C.byref(a), C.byref(r)),
+               "gsq_mlp_recon_error")
+        return a.value, r.value
+
+    def harden_pack(self, which):
+        N, K = self.shapes[which]
+        packed = np.zeros(gsq_packed_bytes(self.mode, N, K) // 4, np.uint32)
+        h16 = np.zeros((N, K // self.group), np.uint16)
+        f32 = np.zeros((N, K // self.group), np.float32)
+        _check(_lib.gsq_mlp_harden_pack(self.ctx, which, packed.ctypes.data,
+                                        h16.ctypes.data, f32.ctypes.data),
+               "gsq_mlp_harden_pack")
+        return packed, h16, f32
+
+    def _shape(self, which, buf):
+        if which < 3:
+            N, K = self.shapes[which]
+            G = K // self.group
+            return {GSQ_DBG_LOGITS: ((self.L, N, K), np.float32),
+                    GSQ_DBG_MOM: ((self.L, N, K), np.float32),
+                    GSQ_DBG_SCALES: ((N, G), np.float32), GSQ_DBG_SMOM: ((N, G), np.float32),
+                    GSQ_DBG_I0: ((N, K), np.int8), GSQ_DBG_WHAT: ((N, K), np.uint16),
+                    GSQ_DBG_DW: ((N, K), np.float32)}[buf]
+        F, H, T = self.F, self.H, self.T
+        return {GSQ_MLP_DBG_AT: ((F, T), np.float32), GSQ_MLP_DBG_BT: ((F, T), np.float32),
+                GSQ_MLP_DBG_HT: ((F, T), np.uint16), GSQ_MLP_DBG_DPT: ((H, T), np.uint16),
+                GSQ_MLP_DBG_DHT: ((F, T), np.float32), GSQ_MLP_DBG_DAT: ((F, T), np.uint16),
+                GSQ_MLP_DBG_DBT: ((F, T), np.uint16), GSQ_MLP_DBG_RT: ((H, T), np.float32)}[buf]
+
+    def get(self, which, buf):
+        shape, dt = self._shape(which, buf)
+        out = np.zeros(shape, dt)
+        _check(_lib.gsq_mlp_debug_get(self.ctx, which, buf, out.ctypes.data, out.nbytes),
+               "gsq_mlp_debug_get")
+        return out
+
+    def set(self, which, buf, arr):
+        shape, dt = self._shape(which, buf)
+        a = np.ascontiguousarray(arr, dtype=dt).reshape(shape)
+        _check(_lib.gsq_mlp_debug_set(self.ctx, which, buf, a.ctypes.data, a.nbytes),
+               "gsq_mlp_debug_set")
+
+    def get_step(self):
+        t = C.c_uint64()
+        _check(_lib.gsq_mlp_get_step(self.ctx, C.byref(t)), "gsq_mlp_get_step")
+        return t.value
+
+    def close(self):
+        if self.ctx:
+            _check(_lib.gsq_mlp_destroy(self.ctx), "gsq_mlp_destroy")
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            if self.ctx:
+                _lib.gsq_mlp_destroy(self.ctx)
+                self.ctx = None
+        except Exception:
+            pass

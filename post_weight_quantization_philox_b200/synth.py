@@ -134,3 +134,27 @@ def random_grad(shape, seed: int, scale: float = 1e-2) -> np.ndarray:
     """A seeded stand-in weight gradient for testing the backward in isolation."""
     rng = np.random.default_rng(seed)
     return (rng.normal(0.0, scale, size=shape)).astype(np.float32)
+
+
+# ------------------------------------------- block stage: SwiGLU MLP inputs
+
+# Llama-3.1-70B block MLP on 8 sequences x 2048 tokens
+MLP_STAGE = {"c5_70b_mlp": dict(T=16384, H=8192, F=28672, grid=GRID_2BIT, steps=200)}
+
+
+def make_mlp_stage(T: int, H: int, F: int, seed: int = 5005):
+    """Normalised MLP input Xn (T x H, unit RMS rows, bf16 values) and
+    N(0, 0.02^2) bf16 gate / up (F x H) and down (H x F) projections."""
+    rng = np.random.default_rng(seed)
+    X = rng.normal(0.0, 1.0, size=(T, H)).astype(np.float32)
+    X /= np.sqrt(np.mean(X.astype(np.float64) ** 2, axis=1, keepdims=True)).astype(np.float32)
+    Wg = rng.normal(0.0, 0.02, size=(F, H)).astype(np.float32)
+    Wu = rng.normal(0.0, 0.02, size=(F, H)).astype(np.float32)
+    Wd = rng.normal(0.0, 0.02, size=(H, F)).astype(np.float32)
+    return bf16_values(X), bf16_values(Wg), bf16_values(Wu), bf16_values(Wd)
+
+
+def random_target(T: int, H: int, scale: float, seed: int = 5006) -> np.ndarray:
+    """A seeded N(0, scale^2) stand-in for a block-output target."""
+    rng = np.random.default_rng(seed)
+    return rng.normal(0.0, scale, size=(T, H)).astype(np.float32)
