@@ -304,6 +304,68 @@ def load_traffic(kernel, config):
     return d.get(config, {}).get(kernel)
 
 
+def run_mlp_stage(args, rank, world, local_rank):
+    """The 70B block's MLP stage (gate/up/down quantized jointly on 16384
+    tokens): whole-stage steps through gsq_mlp_run."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    cfg = synth.MLP_STAGE["c5_70b_mlp"]
+    T, H, F = cfg["T"], cfg["H"], cfg["F"]
+    Xn, Wg, Wu, Wd = synth.make_mlp_stage(T, H, F, seed=5005 + 7919 * rank)
+    R = synth.random_target(T, H, 0.05, seed=5006 + 7919 * rank)
+    dev = lambda x: torch.from_numpy(x).to(torch.bfloat16).cuda()
+    m = gsq.gsq_mlp_init(dev(Xn), torch.from_numpy(R).cuda(), dev(Wg), dev(Wu), dev(Wd),
+                         grid_mode=cfg["grid"], seed=rank)
+    del Xn, Wg, Wu, Wd, R
+    taus = synth.tau_schedule(1.0, 0.05, cfg["steps"])
+    sched = np.array([taus[i % len(taus)] for i in range(args.warmup + args.steps)], np.float32)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    m.run(sched[:args.warmup], 1e-3)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    m.run(sched[args.warmup:], 1e-3)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    loss = m.last_loss()
+    m.close()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    per = ms / args.steps
+    coords = 3 * H * F
+    flops = 7 * 2.0 * T * H * F
+    ach = flops / (per / 1e3) / 1e12
+    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
+            "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
+            "config": {"workload": "c5_70b_mlp_stage", "T": T, "H": H, "F": F, "grid": "2bit",
+                       "weights": "gate, up, down (joint)"},
+            "roofline": {"bound": "tensor", "kernel": "whole stage step (7 GEMMs + elementwise)",
+                         "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
+                         "frac": round(ach / tf_sus, 4), "peak_kind": f"{peak_kind} (sustained bf16)",
+                         "traffic": None},
+            "gpu_launches": int(args.steps * 20), "clocks": clk, "last_loss": loss}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -337,6 +399,8 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", default=None, choices=["mlp"],
+                    help="time a block stage instead of a single layer")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
     args = ap.parse_args()
@@ -358,7 +422,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
-    out = run_gsq(args, rank, world, local_rank)
+    if args.stage == "mlp":
+        out = run_mlp_stage(args, rank, world, local_rank)
+    else:
+        out = run_gsq(args, rank, world, local_rank)
     if out:
         print(json.dumps(out))
     if world > 1:
