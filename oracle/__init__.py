@@ -82,6 +82,10 @@ def lib():
             "gsqo_gemm_abt": (None, [_i64, _i64, _i64, _p, _p, _p]),
             "gsqo_mlp_forward_backward": (_f64, [_i64, _i64, _i64, _p, _p, _p, _p,
                                                  _p, _i32, _p, _p, _p]),
+            "gsqo_attn_probs": (None, [_i64, _i64, _i64, _i64, _i64, _f64, _p, _p,
+                                       _p, _i32, _p]),
+            "gsqo_attn_vo_forward_backward": (_f64, [_i64, _i64, _i64, _i64, _i64,
+                                                     _p, _p, _p, _p, _p, _i32, _p, _p]),
         }
         for name, (res, args) in sigs.items():
             f = getattr(_lib, name)
@@ -399,4 +403,74 @@ def mlp_recon_error(ms: MlpState, Xn, R, emode=0, tau=1.0):
         else:
             ws.append(soft_weight(st, tau, noise=False)[3])
     loss, _, _, _ = mlp_forward_backward(Xn, R, *ws)
+    return loss, loss / float((np.asarray(R, np.float64) ** 2).sum())
+
+
+# ---------------------------------------------- attention V/O joint stage
+
+def attn_probs(Xa, Wq, Wk, nseq, S, nh, nkv, d=128, theta=500000.0, round_bf16=True):
+    """P[s, h, q, key] from the frozen query/key weights (see gsq_oracle.h)."""
+    Xa, Wq, Wk = _f32a(Xa), _f32a(Wq), _f32a(Wk)
+    P = np.zeros((nseq, nh, S, S), np.float32)
+    lib().gsqo_attn_probs(nseq, S, nh, nkv, d, theta, _ptr(Xa), _ptr(Wq), _ptr(Wk),
+                          int(round_bf16), _ptr(P))
+    return P
+
+
+def attn_vo_forward_backward(Xa, P, R, Wv, Wo, nseq, S, nh, nkv, d=128, round_bf16=True):
+    Xa, P, Wv, Wo = _f32a(Xa), _f32a(P), _f32a(Wv), _f32a(Wo)
+    R = np.ascontiguousarray(R, np.float64)
+    H = nh * d
+    dWv = np.zeros((nkv * d, H), np.float32)
+    dWo = np.zeros((H, H), np.float32)
+    loss = lib().gsqo_attn_vo_forward_backward(nseq, S, nh, nkv, d, _ptr(Xa), _ptr(P),
+                                                _ptr(R), _ptr(Wv), _ptr(Wo),
+                                                int(round_bf16), _ptr(dWv), _ptr(dWo))
+    return loss, dWv, dWo
+
+
+@dataclass
+class AttnState:
+    v: State
+    o: State
+    t: int = 0
+
+    def weights(self):
+        return (self.v, self.o)
+
+
+def attn_init(mode, Wv, Wo, group=128, seed=0):
+    return AttnState(init(mode, Wv, group, seed=weight_seed(seed, 0)),
+                     init(mode, Wo, group, seed=weight_seed(seed, 1)))
+
+
+def attn_step(at: AttnState, Xa, P, R, dims, tau, lr, beta1=0.9, beta2=0.99, dumps=False):
+    """One joint V/O step; dims = (nseq, S, nh, nkv, d)."""
+    wb = []
+    for st in at.weights():
+        st.t = at.t
+        wb.append(soft_weight(st, tau)[3])
+    loss, dWv, dWo = attn_vo_forward_backward(Xa, P, R, wb[0], wb[1], *dims)
+    for st, dW in zip(at.weights(), (dWv, dWo)):
+        backward_lion(st, dW, tau, lr, beta1, beta2)
+    at.t += 1
+    for st in at.weights():
+        st.t = at.t
+    if dumps:
+        return loss, dict(w=wb, dW=(dWv, dWo))
+    return loss
+
+
+def attn_recon_error(at: AttnState, Xa, P, R, dims, emode=0, tau=1.0):
+    ws = []
+    for st in at.weights():
+        if emode == 0:
+            lev = harden(st.mode, st.logits, st.i0)
+            vals = np.array([-1.5, -0.5, 0.5, 1.5]) if st.mode == GRID_2BIT else (
+                np.array([-1.0, 0.0, 1.0]) if st.mode == GRID_TERNARY else np.arange(8) - 3.5)
+            w = np.repeat(st.s, st.group, axis=1).astype(np.float64) * vals[lev]
+            ws.append(bf16_round(w).astype(np.float32))
+        else:
+            ws.append(soft_weight(st, tau, noise=False)[3])
+    loss, _, _ = attn_vo_forward_backward(Xa, P, R, ws[0], ws[1], *dims)
     return loss, loss / float((np.asarray(R, np.float64) ** 2).sum())

@@ -714,3 +714,183 @@ double gsqo_mlp_forward_backward(int64_t T, int64_t H, int64_t F,
     free(a); free(b); free(h); free(dp); free(da); free(db); free(part);
     return loss;
 }
+
+/* ------------------------------------------- attention V/O joint stage */
+
+/* The block's value/output stage (agihunt.info summary, optimisation
+ * paragraph: Q and K first, then V and O jointly): the attention
+ * probabilities come from the frozen query/key weights and stay fixed. */
+void gsqo_attn_probs(int64_t nseq, int64_t S, int64_t nh, int64_t nkv,
+                     int64_t d, double theta, const float* Xa, const float* Wq,
+                     const float* Wk, int round, float* P) {
+    const int64_t H = nh * d, Hk = nkv * d, T = nseq * S, half = d / 2;
+    const int64_t grp = nh / nkv;
+    double* Q = (double*)malloc((size_t)(T * H) * sizeof(double));
+    double* K = (double*)malloc((size_t)(T * Hk) * sizeof(double));
+    /* projections */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < H; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < H; ++k)
+                acc += (round ? gsqo_bf16_round(Xa[t * H + k]) : (double)Xa[t * H + k]) * Wq[j * H + k];
+            Q[t * H + j] = acc;
+        }
+        for (int64_t j = 0; j < Hk; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < H; ++k)
+                acc += (round ? gsqo_bf16_round(Xa[t * H + k]) : (double)Xa[t * H + k]) * Wk[j * H + k];
+            K[t * Hk + j] = acc;
+        }
+    }
+    /* rotary embedding at the position within the sequence */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const double p = (double)(t % S);
+        for (int64_t i = 0; i < half; ++i) {
+            const double ang = p * pow(theta, -2.0 * (double)i / (double)d);
+            const double cs = cos(ang), sn = sin(ang);
+            for (int64_t h = 0; h < nh; ++h) {
+                double* x = Q + t * H + h * d;
+                const double a = x[i], b = x[i + half];
+                x[i] = a * cs - b * sn;
+                x[i + half] = b * cs + a * sn;
+            }
+            for (int64_t g = 0; g < nkv; ++g) {
+                double* x = K + t * Hk + g * d;
+                const double a = x[i], b = x[i + half];
+                x[i] = a * cs - b * sn;
+                x[i + half] = b * cs + a * sn;
+            }
+        }
+        if (round) {
+            for (int64_t j = 0; j < H; ++j) Q[t * H + j] = gsqo_bf16_round(Q[t * H + j]);
+            for (int64_t j = 0; j < Hk; ++j) K[t * Hk + j] = gsqo_bf16_round(K[t * Hk + j]);
+        }
+    }
+    /* causal softmax of the scaled scores */
+    const double scale = 1.0 / sqrt((double)d);
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t s = 0; s < nseq; ++s)
+        for (int64_t h = 0; h < nh; ++h) {
+            const int64_t g = h / grp;
+            double* row = (double*)malloc((size_t)S * sizeof(double));
+            for (int64_t q = 0; q < S; ++q) {
+                const double* qv = Q + (s * S + q) * H + h * d;
+                double mx = -INFINITY;
+                for (int64_t k = 0; k <= q; ++k) {
+                    const double* kv = K + (s * S + k) * Hk + g * d;
+                    double acc = 0.0;
+                    for (int64_t j = 0; j < d; ++j) acc += qv[j] * kv[j];
+                    row[k] = acc * scale;
+                    if (row[k] > mx) mx = row[k];
+                }
+                double sum = 0.0;
+                for (int64_t k = 0; k <= q; ++k) {
+                    row[k] = exp(row[k] - mx);
+                    sum += row[k];
+                }
+                float* out = P + ((s * nh + h) * S + q) * S;
+                for (int64_t k = 0; k < S; ++k) {
+                    const double pv = k <= q ? row[k] / sum : 0.0;
+                    out[k] = (float)(round ? gsqo_bf16_round(pv) : pv);
+                }
+            }
+            free(row);
+        }
+    free(Q);
+    free(K);
+}
+
+double gsqo_attn_vo_forward_backward(int64_t nseq, int64_t S, int64_t nh,
+                                     int64_t nkv, int64_t d, const float* Xa,
+                                     const float* P, const double* R,
+                                     const float* Wv, const float* Wo,
+                                     int round, float* dWv, float* dWo) {
+    const int64_t H = nh * d, Hk = nkv * d, T = nseq * S, grp = nh / nkv;
+#define RB(x) (round ? gsqo_bf16_round(x) : (x))
+    double* V = (double*)malloc((size_t)(T * Hk) * sizeof(double));
+    double* o = (double*)malloc((size_t)(T * H) * sizeof(double));
+    double* dp = (double*)malloc((size_t)(T * H) * sizeof(double));
+    double* dO = (double*)malloc((size_t)(T * H) * sizeof(double));
+    double* dV = (double*)malloc((size_t)(T * Hk) * sizeof(double));
+    double* part = (double*)malloc((size_t)T * sizeof(double));
+    /* V = Xa Wv^T */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < Hk; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < H; ++k) acc += RB((double)Xa[t * H + k]) * Wv[j * H + k];
+            V[t * Hk + j] = RB(acc);
+        }
+    /* o_(s,h) = P_(s,h) V_(s,g) */
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t s = 0; s < nseq; ++s)
+        for (int64_t h = 0; h < nh; ++h) {
+            const int64_t g = h / grp;
+            for (int64_t q = 0; q < S; ++q)
+                for (int64_t j = 0; j < d; ++j) {
+                    double acc = 0.0;
+                    for (int64_t k = 0; k < S; ++k)
+                        acc += (double)P[((s * nh + h) * S + q) * S + k] * V[(s * S + k) * Hk + g * d + j];
+                    o[(s * S + q) * H + h * d + j] = RB(acc);
+                }
+        }
+    /* pred = o Wo^T, loss, dp = 2E */
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double row = 0.0;
+        for (int64_t n = 0; n < H; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < H; ++k) acc += o[t * H + k] * Wo[n * H + k];
+            const double e = acc - R[t * H + n];
+            row += e * e;
+            dp[t * H + n] = RB(2.0 * e);
+        }
+        part[t] = row;
+    }
+    double loss = 0.0;
+    for (int64_t t = 0; t < T; ++t) loss += part[t];
+    /* dWo = dp^T o; do = dp Wo */
+    if (dWo) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < H; ++n)
+            for (int64_t k = 0; k < H; ++k) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * o[t * H + k];
+                dWo[n * H + k] = (float)acc;
+            }
+    }
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t k = 0; k < H; ++k) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < H; ++n) acc += dp[t * H + n] * Wo[n * H + k];
+            dO[t * H + k] = RB(acc);
+        }
+    /* dV_(s,g) = sum over the group's heads of P_(s,h)^T do_(s,h) */
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t s = 0; s < nseq; ++s)
+        for (int64_t g = 0; g < nkv; ++g)
+            for (int64_t k = 0; k < S; ++k)
+                for (int64_t j = 0; j < d; ++j) {
+                    double acc = 0.0;
+                    for (int64_t h = g * grp; h < (g + 1) * grp; ++h)
+                        for (int64_t q = 0; q < S; ++q)
+                            acc += (double)P[((s * nh + h) * S + q) * S + k] * dO[(s * S + q) * H + h * d + j];
+                    dV[(s * S + k) * Hk + g * d + j] = RB(acc);
+                }
+    /* dWv = dV^T Xa */
+    if (dWv) {
+        #pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < Hk; ++j)
+            for (int64_t k = 0; k < H; ++k) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < T; ++t) acc += dV[t * Hk + j] * RB((double)Xa[t * H + k]);
+                dWv[j * H + k] = (float)acc;
+            }
+    }
+#undef RB
+    free(V); free(o); free(dp); free(dO); free(dV); free(part);
+    return loss;
+}

@@ -140,6 +140,29 @@ double gsqo_mlp_forward_backward(int64_t T, int64_t H, int64_t F,
                                  const float* Wd, int round, float* dWg,
                                  float* dWu, float* dWd);
 
+/* Attention V/O joint stage (the block's value and output projections
+ * trained together with the attention probabilities fixed).
+ *
+ * gsqo_attn_probs: P of every sequence s and head h from the attention input
+ *   Xa (T x H, T = nseq S, H = nh d) and fixed query / key weights Wq (H x H),
+ *   Wk (nkv d x H): Q = Xa Wq^T, K = Xa Wk^T, rotary embedding (rotate-half
+ *   pairs (i, i + d/2), angle p theta^(-2i/d) at position p of the sequence),
+ *   scores Q_h K_g^T / sqrt(d) with g = h / (nh / nkv), causal mask, softmax.
+ *   P layout: [s][h][q][key], fp32.  round = 1 rounds Q, K (after rotation)
+ *   and P to bf16 as the library's GEMM operands.
+ * gsqo_attn_vo_forward_backward: with V = Xa Wv^T (T x nkv d),
+ *   o_(s,h) = P_(s,h) V_(s,g), pred = o Wo^T, loss = sum (pred - R)^2, returns
+ *   the loss and dWv (nkv d x H), dWo (H x H); round = 1 rounds V, o, 2E,
+ *   do and dV to bf16 as the library's GEMM operands. */
+void gsqo_attn_probs(int64_t nseq, int64_t S, int64_t nh, int64_t nkv,
+                     int64_t d, double theta, const float* Xa, const float* Wq,
+                     const float* Wk, int round, float* P);
+double gsqo_attn_vo_forward_backward(int64_t nseq, int64_t S, int64_t nh,
+                                     int64_t nkv, int64_t d, const float* Xa,
+                                     const float* P, const double* R,
+                                     const float* Wv, const float* Wo,
+                                     int round, float* dWv, float* dWo);
+
 /* plain fp64 C = A . B^T for A (M x Kc), B (N x Kc), both row-major */
 void gsqo_gemm_abt(int64_t M, int64_t N, int64_t Kc, const float* A,
                    const float* B, double* C);

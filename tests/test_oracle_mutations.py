@@ -11,6 +11,7 @@ import pytest
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 sys.path.insert(0, HERE)
+import test_oracle_attn as attn_pins  # noqa: E402
 import test_oracle_mlp as mlp_pins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
 
@@ -55,6 +56,17 @@ MUTATIONS = [
      "double dsilu = sg * (1.0 - av * (1.0 - sg));", ["mlp:test_mlp_matches_torch_autograd"]),
     ("mlp_dropped_up_factor", "double gav = dh * b[t * F + f] * dsilu;",
      "double gav = dh * dsilu;", ["mlp:test_mlp_matches_torch_autograd"]),
+    ("attn_no_score_scale", "const double scale = 1.0 / sqrt((double)d);",
+     "const double scale = 1.0;", ["attn:test_probs_match_torch"]),
+    ("attn_rope_sign", "x[i + half] = b * cs + a * sn;\n            }\n            for (int64_t g",
+     "x[i + half] = b * cs - a * sn;\n            }\n            for (int64_t g",
+     ["attn:test_probs_match_torch", "attn:test_rotary_relative_position_property"]),
+    ("attn_causal_strict", "for (int64_t k = 0; k <= q; ++k) {\n                    const double* kv",
+     "for (int64_t k = 0; k < q + (q == 0); ++k) {\n                    const double* kv",
+     ["attn:test_probs_match_torch"]),
+    ("attn_wrong_group", "const int64_t g = h / grp;\n            for (int64_t q = 0; q < S; ++q)\n                for (int64_t j",
+     "const int64_t g = h % nkv;\n            for (int64_t q = 0; q < S; ++q)\n                for (int64_t j",
+     ["attn:test_vo_matches_torch_autograd"]),
     ("mlp_down_grad_transposed", "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + f];",
      "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + (F - 1 - f)];",
      ["mlp:test_mlp_matches_torch_autograd"]),
@@ -83,7 +95,8 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
     mod = _load_mutant(tmp_path, name, old, new)
     caught = []
     for tname in catchers:
-        module = mlp_pins if tname.startswith("mlp:") else pins
+        module = {"mlp": mlp_pins, "attn": attn_pins}.get(tname.split(":")[0], pins) \
+            if ":" in tname else pins
         tname = tname.split(":")[-1]
         fn = getattr(module, tname)
         params = getattr(fn, "pytestmark", [])
