@@ -278,6 +278,59 @@ GSQ_API int gsq_mlp_debug_set(gsq_mlp* ctx, int which, int buf,
 GSQ_API int gsq_mlp_get_step(gsq_mlp* ctx, uint64_t* t);
 GSQ_API int gsq_mlp_destroy(gsq_mlp* ctx);
 
+/* ------------------------------------------- block stage: attention V/O --
+ * The GSQ pages quantize a block's query and key projections first, then the
+ * value and output projections jointly (agihunt.info summary, optimisation
+ * paragraph).  gsq_attn_* quantize Wv (nkv d x H) and Wo (H x H) jointly
+ * against
+ *     loss = || o Wo^T - R ||_F^2,   o_(s,h) = P_(s,h) (Xa Wv^T)_(s, h / grp)
+ * with the attention probabilities P fixed: built once at init from the
+ * attention input Xa (T x H, T = n_seq seq_len, H = n_heads head_dim) and the
+ * given query / key weights Wq (H x H), Wk (nkv d x H) -- the frozen,
+ * already quantized ones -- with the rotate-half rotary embedding (pairs
+ * (i, i + d/2), angle p theta^(-2i/d) at position p within the sequence),
+ * scaled scores Q K^T / sqrt(d), a causal mask and softmax; grouped
+ * key/value heads (grp = n_heads / n_kv_heads query heads per value head).
+ * R (T x H) is the output the stage must produce (the full-precision
+ * attention output).  Q, K, P, V, o, 2E, do and dV are bf16 GEMM operands.
+ * head_dim must be 128, seq_len a multiple of 128, group 128.
+ * Entry points mirror gsq_mlp_*: which = 0 value, 1 output; stage buffers
+ * under which = GSQ_ATTN_STAGE.
+ */
+typedef struct gsq_attn gsq_attn;
+#define GSQ_ATTN_STAGE 2
+enum {
+    GSQ_ATTN_DBG_P = 0,   /* [s][h][q][key] bf16 attention probabilities */
+    GSQ_ATTN_DBG_PT = 1,  /* [s][g][key][hig][q] bf16, same values        */
+    GSQ_ATTN_DBG_VT = 2,  /* nkv d x T bf16  V^T = Wv Xa^T                */
+    GSQ_ATTN_DBG_O = 3,   /* T x H bf16 attention output o                */
+    GSQ_ATTN_DBG_DPT = 4, /* H x T bf16 2 (pred^T - R^T)                  */
+    GSQ_ATTN_DBG_DV = 5,  /* T x nkv d fp32 value gradient dV             */
+    GSQ_ATTN_DBG_RT = 6   /* H x T fp32 R^T                               */
+};
+GSQ_API int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype,
+                          const void* R, int r_dtype, const void* Wq,
+                          const void* Wk, const void* Wv, const void* Wo,
+                          int w_dtype, int64_t n_seq, int64_t seq_len,
+                          int64_t n_heads, int64_t n_kv_heads,
+                          int64_t head_dim, double rope_theta, int group,
+                          int grid_mode, uint64_t seed, void* stream);
+GSQ_API int gsq_attn_step(gsq_attn* ctx, float tau, float lr, float beta1,
+                          float beta2);
+GSQ_API int gsq_attn_run(gsq_attn* ctx, const float* taus, int64_t n,
+                         float lr, float beta1, float beta2);
+GSQ_API int gsq_attn_last_loss(gsq_attn* ctx, double* loss);
+GSQ_API int gsq_attn_recon_error(gsq_attn* ctx, int mode, float tau,
+                                 double* abs_err, double* rel_err);
+GSQ_API int gsq_attn_harden_pack(gsq_attn* ctx, int which, void* packed,
+                                 uint16_t* scales_f16, float* scales_f32);
+GSQ_API int gsq_attn_debug_get(gsq_attn* ctx, int which, int buf, void* host,
+                               size_t bytes);
+GSQ_API int gsq_attn_debug_set(gsq_attn* ctx, int which, int buf,
+                               const void* host, size_t bytes);
+GSQ_API int gsq_attn_get_step(gsq_attn* ctx, uint64_t* t);
+GSQ_API int gsq_attn_destroy(gsq_attn* ctx);
+
 /*
  * gsq_uniforms_noalloc -- the L Philox uniforms of coords
  * [coord0, coord0 + count) at step t for grid_mode and seed (the values

@@ -84,6 +84,8 @@ def lib():
                                                  _p, _i32, _p, _p, _p]),
             "gsqo_attn_probs": (None, [_i64, _i64, _i64, _i64, _i64, _f64, _p, _p,
                                        _p, _i32, _p]),
+            "gsqo_attn_prob_row": (None, [_i64, _i64, _i64, _i64, _i64, _f64, _p, _p,
+                                          _p, _i32, _i64, _i64, _i64, _p]),
             "gsqo_attn_vo_forward_backward": (_f64, [_i64, _i64, _i64, _i64, _i64,
                                                      _p, _p, _p, _p, _p, _i32, _p, _p]),
         }
@@ -415,6 +417,16 @@ def attn_probs(Xa, Wq, Wk, nseq, S, nh, nkv, d=128, theta=500000.0, round_bf16=T
     lib().gsqo_attn_probs(nseq, S, nh, nkv, d, theta, _ptr(Xa), _ptr(Wq), _ptr(Wk),
                           int(round_bf16), _ptr(P))
     return P
+
+
+def attn_prob_row(Xa, Wq, Wk, nseq, S, nh, nkv, s, h, q, d=128, theta=500000.0,
+                  round_bf16=True):
+    """P[s, h, q, :] computed on its own (d <= 256)."""
+    Xa, Wq, Wk = _f32a(Xa), _f32a(Wq), _f32a(Wk)
+    row = np.zeros(S, np.float32)
+    lib().gsqo_attn_prob_row(nseq, S, nh, nkv, d, theta, _ptr(Xa), _ptr(Wq), _ptr(Wk),
+                             int(round_bf16), s, h, q, _ptr(row))
+    return row
 
 
 def attn_vo_forward_backward(Xa, P, R, Wv, Wo, nseq, S, nh, nkv, d=128, round_bf16=True):

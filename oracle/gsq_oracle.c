@@ -894,3 +894,56 @@ double gsqo_attn_vo_forward_backward(int64_t nseq, int64_t S, int64_t nh,
     free(V); free(o); free(dp); free(dO); free(dV); free(part);
     return loss;
 }
+
+/* One query row of the attention probabilities, for sampled checks. */
+static void rotated_projection(const float* Xa, const float* W, int64_t H,
+                               int64_t t, int64_t S, int64_t col0, int64_t d,
+                               double theta, int round, double* out) {
+    const int64_t half = d / 2;
+    for (int64_t j = 0; j < d; ++j) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < H; ++k)
+            acc += (round ? gsqo_bf16_round(Xa[t * H + k]) : (double)Xa[t * H + k]) *
+                   W[(col0 + j) * H + k];
+        out[j] = acc;
+    }
+    const double p = (double)(t % S);
+    for (int64_t i = 0; i < half; ++i) {
+        const double ang = p * pow(theta, -2.0 * (double)i / (double)d);
+        const double cs = cos(ang), sn = sin(ang);
+        const double a = out[i], b = out[i + half];
+        out[i] = a * cs - b * sn;
+        out[i + half] = b * cs + a * sn;
+    }
+    if (round)
+        for (int64_t j = 0; j < d; ++j) out[j] = gsqo_bf16_round(out[j]);
+}
+
+void gsqo_attn_prob_row(int64_t nseq, int64_t S, int64_t nh, int64_t nkv,
+                        int64_t d, double theta, const float* Xa,
+                        const float* Wq, const float* Wk, int round, int64_t s,
+                        int64_t h, int64_t q, float* row) {
+    (void)nseq;
+    const int64_t H = nh * d, g = h / (nh / nkv);
+    double* qv = (double*)malloc((size_t)d * sizeof(double));
+    double* sc = (double*)malloc((size_t)S * sizeof(double));
+    rotated_projection(Xa, Wq, H, s * S + q, S, h * d, d, theta, round, qv);
+    const double scale = 1.0 / sqrt((double)d);
+    #pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k <= q; ++k) {
+        double kv[256];
+        rotated_projection(Xa, Wk, H, s * S + k, S, g * d, d, theta, round, kv);
+        double acc = 0.0;
+        for (int64_t j = 0; j < d; ++j) acc += qv[j] * kv[j];
+        sc[k] = acc * scale;
+    }
+    double mx = -INFINITY, sum = 0.0;
+    for (int64_t k = 0; k <= q; ++k) if (sc[k] > mx) mx = sc[k];
+    for (int64_t k = 0; k <= q; ++k) { sc[k] = exp(sc[k] - mx); sum += sc[k]; }
+    for (int64_t k = 0; k < S; ++k) {
+        const double pv = k <= q ? sc[k] / sum : 0.0;
+        row[k] = (float)(round ? gsqo_bf16_round(pv) : pv);
+    }
+    free(qv);
+    free(sc);
+}

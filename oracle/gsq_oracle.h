@@ -157,6 +157,12 @@ double gsqo_mlp_forward_backward(int64_t T, int64_t H, int64_t F,
 void gsqo_attn_probs(int64_t nseq, int64_t S, int64_t nh, int64_t nkv,
                      int64_t d, double theta, const float* Xa, const float* Wq,
                      const float* Wk, int round, float* P);
+/* one row P[s][h][q][:] (S entries) computed on its own, as in
+ * gsqo_attn_probs, for sampled checks of large layers */
+void gsqo_attn_prob_row(int64_t nseq, int64_t S, int64_t nh, int64_t nkv,
+                        int64_t d, double theta, const float* Xa,
+                        const float* Wq, const float* Wk, int round, int64_t s,
+                        int64_t h, int64_t q, float* row);
 double gsqo_attn_vo_forward_backward(int64_t nseq, int64_t S, int64_t nh,
                                      int64_t nkv, int64_t d, const float* Xa,
                                      const float* P, const double* R,

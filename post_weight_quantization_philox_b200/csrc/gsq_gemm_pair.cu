@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t aph = 0;
     double lsum = 0.0;
     int64_t u = 0;
+    int last_buf = -1;  // staging buffer of the newest committed store (lane 0)
     bool ok = true;
     for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
       if (!warp_wait(smem_u32(&ctl->tfull[acc]), aph) ||
@@ -293,7 +294,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         unit_xy(u, x, y);
         const int b = (int)(u & 1);
         if (EPI == EPI_STORE_F32) {
-          if (lane == 0) bulk_wait_read<1>();  // this buffer's last store read it
+          // this buffer may be rewritten once the store that last read it is
+          // done: the newest group if it used this buffer, else the one before
+          if (lane == 0) {
+            if (last_buf == b) bulk_wait_read<0>();
+            else bulk_wait_read<1>();
+          }
           __syncwarp();
           const uint32_t base = out_s + (uint32_t)(b * OUT_TILE);
 #pragma unroll
@@ -306,9 +312,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && x < N && y < M) {  // no store for a box wholly outside C
             tma_store_2d(&tmO, base, x, y);
             bulk_commit();
+            last_buf = b;
           }
         } else {
           // Y_ref of this unit, loaded by TMA (zero outside the matrix)
@@ -338,7 +345,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) part = fmaf(e[j], e[j], part);
           if (EPI == EPI_LOSS_DY) {
-            if (lane == 0) bulk_wait_read<1>();
+            if (lane == 0) {
+              if (last_buf == b) bulk_wait_read<0>();
+              else bulk_wait_read<1>();
+            }
             __syncwarp();
             const uint32_t dbase = dy_s + (uint32_t)(b * DY_TILE);
 #pragma unroll
@@ -353,9 +363,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0 && x < N && y < M) {
               tma_store_2d(&tmO, dbase, x, y);
               bulk_commit();
+              last_buf = b;
             }
           }
         }

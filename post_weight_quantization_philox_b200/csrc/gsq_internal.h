@@ -131,5 +131,21 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows,
                                   cudaStream_t st);
 cudaError_t launch_transpose_to_f32(const void* in, int in_bf16, int64_t rows,
                                     int64_t cols, float* out, cudaStream_t st);
+// attention V/O stage
+cudaError_t launch_rope(const float* x, int64_t T, int64_t cols, int64_t S, int d,
+                        double theta, __nv_bfloat16* out, int sm_count, cudaStream_t st);
+cudaError_t launch_causal_softmax(const float* scores, int64_t S, float scale,
+                                  __nv_bfloat16* P, cudaStream_t st);
+cudaError_t launch_transpose_ld(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                int64_t ld_in, __nv_bfloat16* out, int64_t ld_out,
+                                cudaStream_t st);
+cudaError_t launch_f32_to_bf16(const float* in, int64_t n, __nv_bfloat16* out,
+                               int sm_count, cudaStream_t st);
+cudaError_t launch_gather_heads(const float* og, int64_t nseq, int64_t S, int64_t nh,
+                                int64_t grp, int d, __nv_bfloat16* o, int sm_count,
+                                cudaStream_t st);
+cudaError_t launch_scatter_heads_t(const float* doT, int64_t nseq, int64_t S,
+                                   int64_t nh, int64_t grp, int d,
+                                   __nv_bfloat16* dog, int sm_count, cudaStream_t st);
 
 }  // namespace gsq

@@ -668,6 +668,126 @@ __global__ void k_transpose(const TIn* __restrict__ in, int64_t rows,
   }
 }
 
+// ------------------------------------------------ attention V/O pieces
+
+// Rotary embedding (rotate-half pairs (i, i + d/2), angle p theta^(-2i/d) at
+// the position p = t % S within the sequence; angles in double precision) of
+// an fp32 projection (T x cols, cols = heads * d), written as bf16.
+__global__ void k_rope(const float* __restrict__ x, int64_t T, int64_t cols,
+                       int64_t S, int d, double theta,
+                       __nv_bfloat16* __restrict__ out) {
+  const int half = d / 2;
+  const int64_t pairs = T * (cols / 2);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < pairs;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / (cols / 2);
+    const int64_t r = i % (cols / 2);
+    const int64_t head = r / half;
+    const int j = (int)(r % half);
+    const int64_t c0 = head * d + j, c1 = c0 + half;
+    const double ang = (double)(t % S) * pow(theta, -2.0 * (double)j / (double)d);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    const float a = x[t * cols + c0], b = x[t * cols + c1];
+    out[t * cols + c0] = __float2bfloat16_rn((float)((double)a * cs - (double)b * sn));
+    out[t * cols + c1] = __float2bfloat16_rn((float)((double)b * cs + (double)a * sn));
+  }
+}
+
+// Causal softmax of scaled scores: one block per query row q of one (s, h)
+// slice (S x S fp32); P row written as bf16 (zeros above the diagonal).
+__global__ void __launch_bounds__(256) k_causal_softmax(
+    const float* __restrict__ scores, int64_t S, float scale,
+    __nv_bfloat16* __restrict__ P) {
+  __shared__ float red[32];
+  const int64_t q = blockIdx.x;
+  const float* row = scores + q * S;
+  __nv_bfloat16* out = P + q * S;
+  float mx = -INFINITY;
+  for (int64_t k = threadIdx.x; k <= q; k += blockDim.x) mx = fmaxf(mx, row[k] * scale);
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : -INFINITY;
+    v = warp_max(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  mx = red[0];
+  __syncthreads();
+  float sum = 0.f;
+  for (int64_t k = threadIdx.x; k <= q; k += blockDim.x) sum += expf(row[k] * scale - mx);
+  sum = warp_sum(sum);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float inv = 1.f / red[0];
+  for (int64_t k = threadIdx.x; k < S; k += blockDim.x)
+    out[k] = __float2bfloat16_rn(k <= q ? expf(row[k] * scale - mx) * inv : 0.f);
+}
+
+// out[c * ld_out + r] = in[r * ld_in + c] for an rows x cols bf16 block
+__global__ void k_transpose_ld(const __nv_bfloat16* __restrict__ in, int64_t rows,
+                               int64_t cols, int64_t ld_in,
+                               __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 64 x 4
+  for (int r = ty; r < 64; r += 4) {
+    const int64_t rr = r0 + r, cc = c0 + tx;
+    tile[r][tx] = (rr < rows && cc < cols) ? in[rr * ld_in + cc] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  for (int c = ty; c < 64; c += 4) {
+    const int64_t cc = c0 + c, rr = r0 + tx;
+    if (cc < cols && rr < rows) out[cc * ld_out + rr] = tile[tx][c];
+  }
+}
+
+__global__ void k_f32_to_bf16(const float* __restrict__ in, int64_t n,
+                              __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(in[i]);
+}
+
+// o (T x nh d, bf16) from the per-group stacked attention outputs
+// og[s][g][hig][q][j] (fp32), h = g grp + hig
+__global__ void k_gather_heads(const float* __restrict__ og, int64_t nseq,
+                               int64_t S, int64_t nh, int64_t grp, int d,
+                               __nv_bfloat16* __restrict__ o) {
+  const int64_t H = nh * d, n = nseq * S * H;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / H, c = i % H;
+    const int64_t s = t / S, q = t % S, h = c / d, j = c % d;
+    const int64_t g = h / grp, hig = h % grp;
+    const int64_t nkv = nh / grp;
+    o[i] = __float2bfloat16_rn(og[(((s * nkv + g) * grp + hig) * S + q) * d + j]);
+  }
+}
+
+// dog[s][g][j][hig][q] (bf16) from do^T (nh d x T, fp32): the output
+// gradient of each group's heads, laid out as one K-major operand per (s, g)
+__global__ void k_scatter_heads_t(const float* __restrict__ doT, int64_t nseq,
+                                  int64_t S, int64_t nh, int64_t grp, int d,
+                                  __nv_bfloat16* __restrict__ dog) {
+  const int64_t T = nseq * S, H = nh * d, n = H * T;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / T, t = i % T;  // row = h d + j
+    const int64_t h = row / d, j = row % d, s = t / S, q = t % S;
+    const int64_t g = h / grp, hig = h % grp, nkv = nh / grp;
+    dog[(((s * nkv + g) * d + j) * grp + hig) * S + q] = __float2bfloat16_rn(doT[i]);
+  }
+}
+
 int grid_for(int64_t work, int threads, int cap) {
   int64_t b = (work + threads - 1) / threads;
   if (b < 1) b = 1;
@@ -872,6 +992,48 @@ cudaError_t launch_transpose_to_f32(const void* in, int in_bf16, int64_t rows,
         (const __nv_bfloat16*)in, rows, cols, out);
   else
     k_transpose<float, float><<<grid, dim3(64, 4), 0, st>>>((const float*)in, rows, cols, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope(const float* x, int64_t T, int64_t cols, int64_t S, int d,
+                        double theta, __nv_bfloat16* out, int sm_count, cudaStream_t st) {
+  k_rope<<<grid_for(T * cols / 2, 256, sm_count * 8), 256, 0, st>>>(x, T, cols, S, d, theta, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_causal_softmax(const float* scores, int64_t S, float scale,
+                                  __nv_bfloat16* P, cudaStream_t st) {
+  k_causal_softmax<<<(unsigned)S, 256, 0, st>>>(scores, S, scale, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_ld(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                                int64_t ld_in, __nv_bfloat16* out, int64_t ld_out,
+                                cudaStream_t st) {
+  dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+  k_transpose_ld<<<grid, dim3(64, 4), 0, st>>>(in, rows, cols, ld_in, out, ld_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* in, int64_t n, __nv_bfloat16* out,
+                               int sm_count, cudaStream_t st) {
+  k_f32_to_bf16<<<grid_for(n, 256, sm_count * 8), 256, 0, st>>>(in, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_heads(const float* og, int64_t nseq, int64_t S, int64_t nh,
+                                int64_t grp, int d, __nv_bfloat16* o, int sm_count,
+                                cudaStream_t st) {
+  k_gather_heads<<<grid_for(nseq * S * nh * d, 256, sm_count * 8), 256, 0, st>>>(
+      og, nseq, S, nh, grp, d, o);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_heads_t(const float* doT, int64_t nseq, int64_t S,
+                                   int64_t nh, int64_t grp, int d,
+                                   __nv_bfloat16* dog, int sm_count, cudaStream_t st) {
+  k_scatter_heads_t<<<grid_for(nseq * S * nh * d, 256, sm_count * 8), 256, 0, st>>>(
+      doT, nseq, S, nh, grp, d, dog);
   return cudaGetLastError();
 }
 

@@ -26,6 +26,9 @@ GSQ_NOALLOC_MAX_COORDS = 65536
  GSQ_DBG_WHAT, GSQ_DBG_WSOFT32, GSQ_DBG_DW, GSQ_DBG_DYT, GSQ_DBG_YREFT,
  GSQ_DBG_DL, GSQ_DBG_DS) = range(12)
 GSQ_MLP_STAGE = 3
+GSQ_ATTN_STAGE = 2
+(GSQ_ATTN_DBG_P, GSQ_ATTN_DBG_PT, GSQ_ATTN_DBG_VT, GSQ_ATTN_DBG_O, GSQ_ATTN_DBG_DPT,
+ GSQ_ATTN_DBG_DV, GSQ_ATTN_DBG_RT) = range(7)
 (GSQ_MLP_DBG_AT, GSQ_MLP_DBG_BT, GSQ_MLP_DBG_HT, GSQ_MLP_DBG_DPT, GSQ_MLP_DBG_DHT,
  GSQ_MLP_DBG_DAT, GSQ_MLP_DBG_DBT, GSQ_MLP_DBG_RT) = range(8)
 
@@ -43,6 +46,9 @@ EXPORTS = [
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
+    "gsq_attn_init", "gsq_attn_step", "gsq_attn_run", "gsq_attn_last_loss",
+    "gsq_attn_recon_error", "gsq_attn_harden_pack", "gsq_attn_debug_get",
+    "gsq_attn_debug_set", "gsq_attn_get_step", "gsq_attn_destroy",
 ]
 
 
@@ -94,6 +100,17 @@ _SIGS = {
     "gsq_mlp_debug_set": [_p, _i32, _i32, _p, _sz],
     "gsq_mlp_get_step": [_p, C.POINTER(_u64)],
     "gsq_mlp_destroy": [_p],
+    "gsq_attn_init": [_pp, _p, _i32, _p, _i32, _p, _p, _p, _p, _i32, _i64, _i64, _i64,
+                      _i64, _i64, C.c_double, _i32, _i32, _u64, _p],
+    "gsq_attn_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_attn_run": [_p, _p, _i64, _f32, _f32, _f32],
+    "gsq_attn_last_loss": [_p, C.POINTER(C.c_double)],
+    "gsq_attn_recon_error": [_p, _i32, _f32, C.POINTER(C.c_double), C.POINTER(C.c_double)],
+    "gsq_attn_harden_pack": [_p, _i32, _p, _p, _p],
+    "gsq_attn_debug_get": [_p, _i32, _i32, _p, _sz],
+    "gsq_attn_debug_set": [_p, _i32, _i32, _p, _sz],
+    "gsq_attn_get_step": [_p, C.POINTER(_u64)],
+    "gsq_attn_destroy": [_p],
 }
 
 
@@ -480,6 +497,110 @@ class Mlp:
         try:
             if self.ctx:
                 _lib.gsq_mlp_destroy(self.ctx)
+                self.ctx = None
+        except Exception:
+            pass
+
+
+# ----------------------------------------- block stage: attention V/O
+
+def gsq_attn_init(Xa, R, Wq, Wk, Wv, Wo, n_seq, seq_len, n_heads, n_kv_heads,
+                  head_dim=128, rope_theta=500000.0, group=128,
+                  grid_mode=GSQ_GRID_2BIT, seed=0, stream=None) -> "Attn":
+    """Xa, R (T x H); Wq, Wo (H x H); Wk, Wv (n_kv_heads head_dim x H)."""
+    xp, xdt, xk = _ptr_dtype(Xa)
+    rp, rdt, rk = _ptr_dtype(R)
+    ws = [_ptr_dtype(W) for W in (Wq, Wk, Wv, Wo)]
+    if len({w[1] for w in ws}) != 1:
+        raise TypeError("Wq, Wk, Wv and Wo must share a dtype")
+    ctx = C.c_void_p()
+    _check(_lib.gsq_attn_init(C.byref(ctx), xp, xdt, rp, rdt, ws[0][0], ws[1][0], ws[2][0],
+                              ws[3][0], ws[0][1], n_seq, seq_len, n_heads, n_kv_heads,
+                              head_dim, rope_theta, group, grid_mode,
+                              seed & 0xFFFFFFFFFFFFFFFF, _stream_ptr(stream)),
+           "gsq_attn_init")
+    del xk, rk, ws
+    return Attn(ctx, grid_mode, n_seq, seq_len, n_heads, n_kv_heads, head_dim, group)
+
+
+class Attn:
+    """Context of the attention V/O stage (value and output quantized jointly)."""
+
+    def __init__(self, ctx, mode, nseq, S, nh, nkv, d, group):
+        self.ctx, self.mode, self.group = ctx, mode, group
+        self.nseq, self.S, self.nh, self.nkv, self.d = nseq, S, nh, nkv, d
+        self.T, self.H, self.Hk = nseq * S, nh * d, nkv * d
+        self.L = NUM_LOGITS[mode]
+        self.shapes = ((self.Hk, self.H), (self.H, self.H))
+
+    def step(self, tau, lr, beta1=0.9, beta2=0.99):
+        _check(_lib.gsq_attn_step(self.ctx, tau, lr, beta1, beta2), "gsq_attn_step")
+
+    def run(self, taus, lr, beta1=0.9, beta2=0.99):
+        t = np.ascontiguousarray(taus, dtype=np.float32).ravel()
+        _check(_lib.gsq_attn_run(self.ctx, t.ctypes.data, t.size, lr, beta1, beta2),
+               "gsq_attn_run")
+
+    def last_loss(self):
+        v = C.c_double()
+        _check(_lib.gsq_attn_last_loss(self.ctx, C.byref(v)), "gsq_attn_last_loss")
+        return v.value
+
+    def recon_error(self, mode=GSQ_RECON_HARD, tau=1.0):
+        a, r = C.c_double(), C.c_double()
+        _check(_lib.gsq_attn_recon_error(self.ctx, mode, tau, C.byref(a), C.byref(r)),
+               "gsq_attn_recon_error")
+        return a.value, r.value
+
+    def harden_pack(self, which):
+        N, K = self.shapes[which]
+        packed = np.zeros(gsq_packed_bytes(self.mode, N, K) // 4, np.uint32)
+        h16 = np.zeros((N, K // self.group), np.uint16)
+        f32 = np.zeros((N, K // self.group), np.float32)
+        _check(_lib.gsq_attn_harden_pack(self.ctx, which, packed.ctypes.data,
+                                         h16.ctypes.data, f32.ctypes.data),
+               "gsq_attn_harden_pack")
+        return packed, h16, f32
+
+    def _shape(self, which, buf):
+        if which < 2:
+            N, K = self.shapes[which]
+            G = K // self.group
+            return {GSQ_DBG_LOGITS: ((self.L, N, K), np.float32),
+                    GSQ_DBG_MOM: ((self.L, N, K), np.float32),
+                    GSQ_DBG_SCALES: ((N, G), np.float32), GSQ_DBG_SMOM: ((N, G), np.float32),
+                    GSQ_DBG_I0: ((N, K), np.int8), GSQ_DBG_WHAT: ((N, K), np.uint16),
+                    GSQ_DBG_DW: ((N, K), np.float32)}[buf]
+        P = (self.nseq, self.nh, self.S, self.S)
+        return {GSQ_ATTN_DBG_P: (P, np.uint16), GSQ_ATTN_DBG_PT: (P, np.uint16),
+                GSQ_ATTN_DBG_VT: ((self.Hk, self.T), np.uint16),
+                GSQ_ATTN_DBG_O: ((self.T, self.H), np.uint16),
+                GSQ_ATTN_DBG_DPT: ((self.H, self.T), np.uint16),
+                GSQ_ATTN_DBG_DV: ((self.T, self.Hk), np.float32),
+                GSQ_ATTN_DBG_RT: ((self.H, self.T), np.float32)}[buf]
+
+    def get(self, which, buf):
+        shape, dt = self._shape(which, buf)
+        out = np.zeros(shape, dt)
+        _check(_lib.gsq_attn_debug_get(self.ctx, which, buf, out.ctypes.data, out.nbytes),
+               "gsq_attn_debug_get")
+        return out
+
+    def set(self, which, buf, arr):
+        shape, dt = self._shape(which, buf)
+        a = np.ascontiguousarray(arr, dtype=dt).reshape(shape)
+        _check(_lib.gsq_attn_debug_set(self.ctx, which, buf, a.ctypes.data, a.nbytes),
+               "gsq_attn_debug_set")
+
+    def close(self):
+        if self.ctx:
+            _check(_lib.gsq_attn_destroy(self.ctx), "gsq_attn_destroy")
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            if self.ctx:
+                _lib.gsq_attn_destroy(self.ctx)
                 self.ctx = None
         except Exception:
             pass

@@ -158,3 +158,23 @@ def random_target(T: int, H: int, scale: float, seed: int = 5006) -> np.ndarray:
     """A seeded N(0, scale^2) stand-in for a block-output target."""
     rng = np.random.default_rng(seed)
     return rng.normal(0.0, scale, size=(T, H)).astype(np.float32)
+
+
+# ----------------------------------------- block stage: attention V/O inputs
+
+# Llama-3.1-70B attention: 64 query heads, 8 key/value heads of 128, 8 x 2048
+ATTN_STAGE = {"c5_70b_attn": dict(nseq=8, S=2048, nh=64, nkv=8, d=128, grid=GRID_2BIT,
+                                  steps=200)}
+
+
+def make_attn_stage(nseq: int, S: int, nh: int, nkv: int, d: int = 128, seed: int = 6006):
+    """Normalised attention input Xa (nseq S x nh d, unit RMS rows) and
+    N(0, 0.02^2) query (H x H), key and value (nkv d x H) and output (H x H)
+    projections, all bf16 values."""
+    rng = np.random.default_rng(seed)
+    H, Hk = nh * d, nkv * d
+    X = rng.normal(0.0, 1.0, size=(nseq * S, H)).astype(np.float32)
+    X /= np.sqrt(np.mean(X.astype(np.float64) ** 2, axis=1, keepdims=True)).astype(np.float32)
+    Ws = [rng.normal(0.0, 0.02, size=shape).astype(np.float32)
+          for shape in ((H, H), (Hk, H), (Hk, H), (H, H))]
+    return (bf16_values(X), *[bf16_values(W) for W in Ws])

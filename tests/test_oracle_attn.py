@@ -145,3 +145,12 @@ def test_vo_zero_loss_on_own_output(oracle_mod):
     R = o @ Wo.T.astype(np.float64)
     loss, dWv, dWo = oracle_mod.attn_vo_forward_backward(Xa, P, R, Wv, Wo, **DIMS, round_bf16=False)
     assert loss < 1e-18 and np.abs(dWv).max() < 1e-9 and np.abs(dWo).max() < 1e-9
+
+
+def test_single_row_equals_full_probabilities(oracle_mod):
+    Xa, Wq, Wk, _, _ = _inputs(seed=8)
+    P = oracle_mod.attn_probs(Xa, Wq, Wk, **DIMS)
+    for s, h, q in [(0, 0, 0), (1, 3, 9), (0, 2, 15)]:
+        row = oracle_mod.attn_prob_row(Xa, Wq, Wk, DIMS["nseq"], DIMS["S"], DIMS["nh"],
+                                       DIMS["nkv"], s, h, q)
+        assert np.array_equal(row, P[s, h, q])
