@@ -56,8 +56,10 @@ MUTATIONS = [
      "double dsilu = sg * (1.0 - av * (1.0 - sg));", ["mlp:test_mlp_matches_torch_autograd"]),
     ("mlp_dropped_up_factor", "double gav = dh * b[t * F + f] * dsilu;",
      "double gav = dh * dsilu;", ["mlp:test_mlp_matches_torch_autograd"]),
-    ("attn_no_score_scale", "const double scale = 1.0 / sqrt((double)d);",
-     "const double scale = 1.0;", ["attn:test_probs_match_torch"]),
+    ("attn_no_score_scale",
+     "const double scale = 1.0 / sqrt((double)d);\n    #pragma omp parallel for collapse(2)",
+     "const double scale = 1.0;\n    #pragma omp parallel for collapse(2)",
+     ["attn:test_probs_match_torch"]),
     ("attn_rope_sign", "x[i + half] = b * cs + a * sn;\n            }\n            for (int64_t g",
      "x[i + half] = b * cs - a * sn;\n            }\n            for (int64_t g",
      ["attn:test_probs_match_torch", "attn:test_rotary_relative_position_property"]),
