@@ -366,6 +366,74 @@ def run_mlp_stage(args, rank, world, local_rank):
             "gpu_launches": int(args.steps * 20), "clocks": clk, "last_loss": loss}
 
 
+def run_attn_stage(args, rank, world, local_rank):
+    """The 70B block's attention V/O stage (value and output quantized
+    jointly, 64/8 heads x 128, 8 x 2048 tokens) through gsq_attn_run."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    cfg = synth.ATTN_STAGE["c5_70b_attn"]
+    dims = dict(nseq=cfg["nseq"], S=cfg["S"], nh=cfg["nh"], nkv=cfg["nkv"], d=cfg["d"])
+    Xa, Wq, Wk, Wv, Wo = synth.make_attn_stage(**dims, seed=6006 + 7919 * rank)
+    T, H = Xa.shape
+    R = synth.random_target(T, H, 0.05, seed=6007 + 7919 * rank)
+    dev = lambda x: torch.from_numpy(x).to(torch.bfloat16).cuda()
+    a = gsq.gsq_attn_init(dev(Xa), torch.from_numpy(R).cuda(), dev(Wq), dev(Wk), dev(Wv),
+                          dev(Wo), dims["nseq"], dims["S"], dims["nh"], dims["nkv"],
+                          dims["d"], grid_mode=cfg["grid"], seed=rank)
+    del Xa, Wq, Wk, Wv, Wo, R
+    taus = synth.tau_schedule(1.0, 0.05, cfg["steps"])
+    sched = np.array([taus[i % len(taus)] for i in range(args.warmup + args.steps)], np.float32)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    a.run(sched[:args.warmup], 1e-3)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    a.run(sched[args.warmup:], 1e-3)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    loss = a.last_loss()
+    a.close()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    per = ms / args.steps
+    S, nh, nkv, d = dims["S"], dims["nh"], dims["nkv"], dims["d"]
+    Hk = nkv * d
+    coords = Hk * H + H * H
+    # useful flops per step: V, P.V, pred, dWo, do, P^T.do, dWv
+    flops = 2.0 * (2 * T * H * Hk + 3 * T * H * H + 2 * dims["nseq"] * nh * S * S * d)
+    ach = flops / (per / 1e3) / 1e12
+    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
+            "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
+            "config": {"workload": "c5_70b_attn_vo_stage", **dims, "grid": "2bit",
+                       "weights": "value, output (joint)"},
+            "roofline": {"bound": "tensor", "kernel": "whole stage step (GEMMs + elementwise)",
+                         "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
+                         "frac": round(ach / tf_sus, 4), "peak_kind": f"{peak_kind} (sustained bf16)",
+                         "traffic": None},
+            "gpu_launches": int(args.steps * (14 + 2 * dims["nseq"] * nkv)), "clocks": clk,
+            "last_loss": loss}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -399,7 +467,7 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["mlp"],
+    ap.add_argument("--stage", default=None, choices=["mlp", "attn"],
                     help="time a block stage instead of a single layer")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
@@ -424,6 +492,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     if args.stage == "mlp":
         out = run_mlp_stage(args, rank, world, local_rank)
+    elif args.stage == "attn":
+        out = run_attn_stage(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:
