@@ -417,8 +417,9 @@ def run_attn_stage(args, rank, world, local_rank):
     S, nh, nkv, d = dims["S"], dims["nh"], dims["nkv"], dims["d"]
     Hk = nkv * d
     coords = Hk * H + H * H
-    # useful flops per step: V, P.V, pred, dWo, do, P^T.do, dWv
-    flops = 2.0 * (2 * T * H * Hk + 3 * T * H * H + 2 * dims["nseq"] * nh * S * S * d)
+    # useful flops per step: V, P.V, pred, dWo, do, P^T.do, dWv; the two
+    # products with the causal P count its nonzero half only
+    flops = 2.0 * (2 * T * H * Hk + 3 * T * H * H) + 2 * 2.0 * dims["nseq"] * nh * d * S * (S + 1) / 2
     ach = flops / (per / 1e3) / 1e12
     return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
@@ -430,7 +431,7 @@ def run_attn_stage(args, rank, world, local_rank):
                          "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
                          "frac": round(ach / tf_sus, 4), "peak_kind": f"{peak_kind} (sustained bf16)",
                          "traffic": None},
-            "gpu_launches": int(args.steps * (14 + 2 * dims["nseq"] * nkv)), "clocks": clk,
+            "gpu_launches": int(args.steps * 17 + 2), "clocks": clk,
             "last_loss": loss}
 
 

@@ -17,6 +17,11 @@
 //   dWo = dp^T . o ;  do^T = Wo^T dp^T
 //   dV_(s,g) = P^T_(s,g) . do_(s, g's heads)         (S x d, K = grp S)
 //   dWv = dV^T . Xa ; backward + Lion for Wv and Wo.
+// The per-(s, g) products run as one batched launch each, on 256 x 128
+// tiles (N = d = 128).  When S is a multiple of 256 they skip the zero half
+// of the causal P: o tiles of queries [q0, q0 + 256) contract over keys
+// [0, q0 + 256) only, dV tiles of keys [k0, k0 + 256) over queries [k0, S) of
+// each head.
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -47,8 +52,9 @@ struct gsq_attn {
   float what_tau = 0.f;
   CUtensorMap tmB_Xa, tmB_o, tmB_oT, tmB_dp, tmB_XaT, tmA_dpT, tmA_WoT, tmA_dVT;
   EpiMaps em_VT, em_pred, em_doT;
-  std::vector<CUtensorMap> tmA_P, tmB_VT, tmA_PT, tmB_dog;  // per (s, g)
-  std::vector<EpiMaps> em_og, em_dV;                          // per (s, g)
+  // all (s, g) problems of a step in one launch each (GemmSched)
+  CUtensorMap tmA_P, tmB_VT, tm_og, tmA_PT, tmB_dog, tm_dV;
+  GemmSched sc_pv, sc_dv;
   std::vector<void*> allocs;
 };
 
@@ -129,12 +135,9 @@ cudaError_t forward(gsq_attn* c, double* loss_out, bool with_dp) {
                        c->sms, c->st)) != cudaSuccess) return e;
   if ((e = launch_f32_to_bf16(c->VT32, Hk * T, c->VT, c->sms, c->st)) != cudaSuccess)
     return e;
-  for (int64_t s = 0; s < c->nseq; ++s)
-    for (int64_t g = 0; g < c->nkv; ++g) {
-      const size_t i = (size_t)(s * c->nkv + g);
-      if ((e = launch_gemm(c->tmA_P[i], c->tmB_VT[i], c->em_og[i], c->grp * S, c->d, S,
-                           EPI_STORE_F32, ep, c->sms, c->st)) != cudaSuccess) return e;
-    }
+  if ((e = launch_gemm_batched(c->tmA_P, c->tmB_VT, c->tm_og, c->grp * S, c->d, S, 128,
+                               c->sc_pv, ep, c->sms, c->st)) != cudaSuccess)
+    return e;
   if ((e = launch_gather_heads(c->og, c->nseq, S, c->nh, c->grp, (int)c->d, c->o,
                                c->sms, c->st)) != cudaSuccess) return e;
   if ((e = launch_transpose_bf16(c->o, T, H, c->oT, c->st)) != cudaSuccess) return e;
@@ -162,12 +165,8 @@ int run_step(gsq_attn* c, float tau, float tau_next, float lr, float b1, float b
   CKA(launch_scatter_heads_t(c->doT32, c->nseq, S, c->nh, c->grp, (int)c->d, c->dog,
                              c->sms, c->st));
   // dV_(s,g) = P^T_(s,g) . do_(s, g's heads)
-  for (int64_t s = 0; s < c->nseq; ++s)
-    for (int64_t g = 0; g < c->nkv; ++g) {
-      const size_t i = (size_t)(s * c->nkv + g);
-      CKA(launch_gemm(c->tmA_PT[i], c->tmB_dog[i], c->em_dV[i], S, c->d, c->grp * S,
-                      EPI_STORE_F32, ep, c->sms, c->st));
-    }
+  CKA(launch_gemm_batched(c->tmA_PT, c->tmB_dog, c->tm_dV, S, c->d, c->grp * S, 128,
+                          c->sc_dv, ep, c->sms, c->st));
   // dWv = dV^T . Xa
   CKA(launch_f32_to_bf16(c->dV32, T * Hk, c->dVb, c->sms, c->st));
   CKA(launch_transpose_bf16(c->dVb, T, Hk, c->dVT, c->st));
@@ -397,34 +396,47 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
     bad |= make_tmap_epi_bf16(&c->em_pred.out, c->dpT, H, T, T) != 0;
     bad |= make_tmap_epi_f32(&c->em_pred.yref, c->RT, H, T, T) != 0;
   }
-  const size_t nsg = (size_t)(c->nseq * c->nkv);
-  c->tmA_P.resize(nsg);
-  c->tmB_VT.resize(nsg);
-  c->tmA_PT.resize(nsg);
-  c->tmB_dog.resize(nsg);
-  c->em_og.resize(nsg);
-  c->em_dV.resize(nsg);
-  for (int64_t s = 0; s < c->nseq; ++s)
-    for (int64_t g = 0; g < c->nkv; ++g) {
-      const size_t i = (size_t)(s * c->nkv + g);
-      CUtensorMap m;
-      // the group's grp heads of P, stacked: (grp S) x S
-      bad |= make_tmap_bf16(&c->tmA_P[i], c->P + (s * c->nh + g * grp) * S * S, grp * S, S,
-                            S, kGemmBoxRowsA) != 0;
-      // V_(s,g)^T: d x S slice of V^T
-      bad |= make_tmap_bf16(&c->tmB_VT[i], c->VT + (g * d) * T + s * S, d, S, T,
-                            kGemmBoxRowsB) != 0;
-      bad |= make_tmap_epi_f32(&m, c->og + (s * c->nkv + g) * grp * S * d, grp * S, d, d) != 0;
-      c->em_og[i] = out_only(m);
-      // P^T_(s,g): S x (grp S)
-      bad |= make_tmap_bf16(&c->tmA_PT[i], c->PT + (s * c->nkv + g) * S * grp * S, S, grp * S,
-                            grp * S, kGemmBoxRowsA) != 0;
-      // do_(s, g's heads) as d x (grp S)
-      bad |= make_tmap_bf16(&c->tmB_dog[i], c->dog + (s * c->nkv + g) * d * grp * S, d,
-                            grp * S, grp * S, kGemmBoxRowsB) != 0;
-      bad |= make_tmap_epi_f32(&m, c->dV32 + s * S * Hk + g * d, S, d, Hk) != 0;
-      c->em_dV[i] = out_only(m);
-    }
+  {
+    // P as (nseq nh S) x S: problem (s, g) is the grp S rows of g's heads
+    bad |= make_tmap_bf16(&c->tmA_P, c->P, c->nseq * c->nh * S, S, S, kGemmBoxRowsA) != 0;
+    // V^T (Hk x T): problem (s, g) is rows g d.., columns s S..
+    bad |= make_tmap_bf16(&c->tmB_VT, c->VT, Hk, T, T, kGemmBoxRowsBNarrow) != 0;
+    // attention outputs per (s, g): (grp S) x d, stacked
+    bad |= make_tmap_epi_f32(&c->tm_og, c->og, c->nseq * c->nh * S, d, d) != 0;
+    // P^T as (nseq nkv S) x (grp S)
+    bad |= make_tmap_bf16(&c->tmA_PT, c->PT, c->nseq * c->nkv * S, grp * S, grp * S,
+                          kGemmBoxRowsA) != 0;
+    // do per (s, g) as d x (grp S), stacked
+    bad |= make_tmap_bf16(&c->tmB_dog, c->dog, c->nseq * c->nkv * d, grp * S, grp * S,
+                          kGemmBoxRowsBNarrow) != 0;
+    // dV (T x Hk): problem (s, g) is rows s S.., columns g d..
+    bad |= make_tmap_epi_f32(&c->tm_dV, c->dV32, T, Hk, Hk) != 0;
+    // problem p = s nkv + g; causal K ranges when a period holds whole tiles
+    const bool causal = S % 256 == 0;
+    GemmSched& a = c->sc_pv;
+    a.count = (int)(c->nseq * c->nkv);
+    a.inner = (int)c->nkv;
+    a.a_row[0] = c->nh * S;
+    a.a_row[1] = grp * S;
+    a.b_row[1] = d;
+    a.b_k[0] = S;
+    a.o_row[0] = c->nh * S;
+    a.o_row[1] = grp * S;
+    a.causal = causal ? 1 : 0;
+    a.seg = S;
+    GemmSched& b = c->sc_dv;
+    b.count = (int)(c->nseq * c->nkv);
+    b.inner = (int)c->nkv;
+    b.a_row[0] = c->nkv * S;
+    b.a_row[1] = S;
+    b.b_row[0] = c->nkv * d;
+    b.b_row[1] = d;
+    b.o_row[0] = S;
+    b.o_col[1] = d;
+    b.causal = causal ? 2 : 0;
+    b.seg = S;
+    b.nseg = (int)grp;
+  }
   if (bad) return cleanup_fail(GSQ_ERR_CUDA);
 
   // attention probabilities from the frozen Q and K projections

@@ -31,16 +31,26 @@ namespace gsq {
 
 namespace {
 
-constexpr int PM = 256, PN = 256, HALF = 128, BK = 64;
-constexpr int STAGES = 5;
+constexpr int PM = 256, HALF = 128, BK = 64;
 constexpr int A_BYTES = HALF * BK * 2;
-constexpr int B_BYTES = HALF * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int TMEM_COLS = 2 * PN;
 constexpr int NUM_THREADS = 192;
 constexpr long long WAIT_LIMIT = 4000000000LL;  // clock cycles (~2 s)
-constexpr uint32_t IDESC = idesc_bf16_f32(PM, PN);
 
+// Output tile width BN (256, or 128 for N = 128 problems): each CTA loads
+// BN / 2 rows of B per stage; two BN-column TMEM accumulators per CTA.
+template <int BN>
+struct Cfg {
+  static constexpr int PN = BN;
+  static constexpr int HALFN = BN / 2;
+  static constexpr int STAGES = BN == 256 ? 5 : 6;
+  static constexpr int B_BYTES = HALFN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(PM, BN);
+  static constexpr int UNITS = BN / 32;
+};
+
+template <int STAGES>
 struct Ctl {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -63,10 +73,75 @@ __host__ __device__ constexpr int warp_stage_bytes() {
                               : (EPI == EPI_LOSS_DY ? 2 * OUT_TILE + 2 * DY_TILE
                                                     : 2 * OUT_TILE);
 }
-template <int EPI>
+template <int EPI, int BN>
 __host__ __device__ constexpr int smem_bytes() {
-  return STAGES * STAGE_BYTES + 4 * warp_stage_bytes<EPI>() + 1024 +
-         (int)sizeof(Ctl);
+  return Cfg<BN>::STAGES * Cfg<BN>::STAGE_BYTES + 4 * warp_stage_bytes<EPI>() + 1024 +
+         (int)sizeof(Ctl<Cfg<BN>::STAGES>);
+}
+
+// Where tile `tile` of a launch sits: problem offsets, tile origin, and its
+// K range (see GemmSched).
+struct TileAt {
+  int64_t a_row, a_k, b_row, b_k, o_row, o_col;  // origin of the problem
+  int64_t m0, n0;  // tile origin inside the problem
+  int64_t r0;      // causal: tile rows' position inside their period
+  int nk;          // K blocks of 64
+  int kps;         // causal = 2: K blocks per period
+};
+
+template <int BN>
+__device__ __forceinline__ TileAt tile_at(int tile, int m_tiles, int n_tiles,
+                                          int64_t Kc, const GemmSched& sc) {
+  TileAt t;
+  int mb, nb, p;
+  t.r0 = 0;
+  t.kps = 0;
+  if (sc.causal == 0) {
+    mb = tile % m_tiles;
+    const int r = tile / m_tiles;
+    nb = r % n_tiles;
+    p = r / n_tiles;
+    t.nk = (int)((Kc + BK - 1) / BK);
+  } else {
+    // the period position is the slowest index, longest K first
+    const int rbs = (int)(sc.seg / PM);
+    const int hs = m_tiles / rbs;
+    const int per = sc.count * n_tiles * hs;
+    const int j = tile / per;
+    int rest = tile - j * per;
+    const int hseg = rest % hs;
+    rest /= hs;
+    nb = rest % n_tiles;
+    p = rest / n_tiles;
+    const int rb = sc.causal == 1 ? rbs - 1 - j : j;
+    mb = hseg * rbs + rb;
+    t.r0 = (int64_t)rb * PM;
+    if (sc.causal == 1) {
+      const int64_t kend = t.r0 + PM < Kc ? t.r0 + PM : Kc;
+      t.nk = (int)((kend + BK - 1) / BK);
+    } else {
+      t.kps = (int)((sc.seg - t.r0) / BK);
+      t.nk = sc.nseg * t.kps;
+    }
+  }
+  const int64_t p1 = p / sc.inner, p2 = p - p1 * sc.inner;
+  t.a_row = sc.a_row[0] * p1 + sc.a_row[1] * p2;
+  t.a_k = sc.a_k[0] * p1 + sc.a_k[1] * p2;
+  t.b_row = sc.b_row[0] * p1 + sc.b_row[1] * p2;
+  t.b_k = sc.b_k[0] * p1 + sc.b_k[1] * p2;
+  t.o_row = sc.o_row[0] * p1 + sc.o_row[1] * p2;
+  t.o_col = sc.o_col[0] * p1 + sc.o_col[1] * p2;
+  t.m0 = (int64_t)mb * PM;
+  t.n0 = (int64_t)nb * BN;
+  return t;
+}
+
+// K coordinate (inside the problem) of K block kb of a tile
+__device__ __forceinline__ int64_t tile_k(const TileAt& t, int kb,
+                                          const GemmSched& sc) {
+  if (sc.causal != 2) return (int64_t)kb * BK;
+  const int sgi = kb / t.kps;
+  return sgi * sc.seg + t.r0 + (int64_t)(kb - sgi * t.kps) * BK;
 }
 
 // shared-memory offset of 16-byte chunk j of row r in a tile written or
@@ -84,26 +159,28 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int EPI>
+template <int EPI, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmO,
                 const __grid_constant__ CUtensorMap tmY, int64_t M, int64_t N,
-                int64_t Kc, EpiParams ep) {
+                int64_t Kc, EpiParams ep, const __grid_constant__ GemmSched sc) {
+  using C = Cfg<BN>;
+  constexpr int PN = C::PN, STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
+  constexpr int TMEM_COLS = C::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_area = smem + STAGES * STAGE_BYTES;
-  Ctl* ctl = reinterpret_cast<Ctl*>(stage_area + 4 * warp_stage_bytes<EPI>());
+  auto* ctl = reinterpret_cast<Ctl<STAGES>*>(stage_area + 4 * warp_stage_bytes<EPI>());
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int m_tiles = (int)((M + PM - 1) / PM);
   const int n_tiles = (int)((N + PN - 1) / PN);
-  const int num_tiles = m_tiles * n_tiles;
-  const int num_kb = (int)((Kc + BK - 1) / BK);
+  const int num_tiles = m_tiles * n_tiles * sc.count;
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0 && lane == 0) {
@@ -143,8 +220,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       long long issued = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        const int mb = tile % m_tiles, nb = tile / m_tiles;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const TileAt ta = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
+        const int32_t ya = (int32_t)(ta.a_row + ta.m0 + (int)rank * HALF);
+        const int32_t yb = (int32_t)(ta.b_row + ta.n0 + (int)rank * C::HALFN);
+        for (int kb = 0; kb < ta.nk; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), ph ^ 1,
                                  WAIT_LIMIT) ||
               *(volatile int*)&ctl->abort) {
@@ -155,10 +234,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb_leader = mapa_shared(fb, 0);
           if (leader) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
           const uint32_t sa = sbase + stage * STAGE_BYTES;
-          tma_load_2d_pair(sa, &tmA, fb_leader, kb * BK,
-                           mb * PM + (int)rank * HALF);
-          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, kb * BK,
-                           nb * PN + (int)rank * HALF);
+          const int64_t kx = tile_k(ta, kb, sc);
+          tma_load_2d_pair(sa, &tmA, fb_leader, (int32_t)(ta.a_k + kx), ya);
+          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, (int32_t)(ta.b_k + kx), yb);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -198,7 +276,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int nk = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc).nk;
+        for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), ph,
                                  WAIT_LIMIT) ||
               *(volatile int*)&ctl->abort) {
@@ -211,7 +290,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t bd = sdesc_kmajor_sw128(sa + A_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, IDESC,
+            umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, C::IDESC,
                            (kb > 0 || k > 0) ? 1u : 0u);
           const uint32_t eb = smem_u32(&ctl->empty[stage]);
           umma_commit_pair(mapa_shared(eb, 0));
@@ -248,15 +327,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t out_s = smem_u32(wst);                  // 2 x OUT_TILE
     const uint32_t y_s = smem_u32(wst);                    // 2 x OUT_TILE
     const uint32_t dy_s = smem_u32(wst + 2 * OUT_TILE);    // 2 x DY_TILE
-    constexpr int UNITS = PN / 32;
+    constexpr int UNITS = C::UNITS;
     const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
     const int64_t total_units = (int64_t)my_tiles * UNITS;
-    // coordinates (x = column, y = first row) of unit u of this warp
+    // coordinates (x = column, y = first row) of unit u of this warp; false
+    // when the unit lies wholly outside its problem's M x N
     auto unit_xy = [&](int64_t u, int32_t& x, int32_t& y) {
       const int tile = pair + (int)(u / UNITS) * npairs;
-      const int mb = tile % m_tiles, nb = tile / m_tiles;
-      x = nb * PN + (int)(u % UNITS) * 32;
-      y = mb * PM + (int)rank * HALF + q * 32;
+      const TileAt ta = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
+      const int64_t lx = ta.n0 + (int)(u % UNITS) * 32;
+      const int64_t ly = ta.m0 + (int)rank * HALF + q * 32;
+      x = (int32_t)(ta.o_col + lx);
+      y = (int32_t)(ta.o_row + ly);
+      return lx < N && ly < M;
     };
     int64_t y_issued = 0;
     auto issue_y = [&](int64_t u) {  // lane 0: Y_ref tile of unit u
@@ -291,7 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), v);
         tmem_wait_ld();
         int32_t x, y;
-        unit_xy(u, x, y);
+        const bool inside = unit_xy(u, x, y);
         const int b = (int)(u & 1);
         if (EPI == EPI_STORE_F32) {
           // this buffer may be rewritten once the store that last read it is
@@ -312,7 +395,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0 && x < N && y < M) {  // no store for a box wholly outside C
+          if (lane == 0 && inside) {  // no store for a box wholly outside C
             tma_store_2d(&tmO, base, x, y);
             bulk_commit();
             last_buf = b;
@@ -363,7 +446,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             fence_async_smem();
             __syncwarp();
-            if (lane == 0 && x < N && y < M) {
+            if (lane == 0 && inside) {
               tma_store_2d(&tmO, dbase, x, y);
               bulk_commit();
               last_buf = b;
@@ -409,11 +492,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
                             const EpiMaps& maps, int64_t M, int64_t N,
-                            int64_t Kc, const EpiParams& ep, int sm_count,
-                            cudaStream_t st) {
+                            int64_t Kc, const GemmSched& sc, const EpiParams& ep,
+                            int sm_count, cudaStream_t st) {
   static int max_pairs = 0;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -422,27 +505,30 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
   attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<EPI>();
+  cfg.dynamicSmemBytes = smem_bytes<EPI, BN>();
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (max_pairs == 0) {
-    cudaError_t e = cudaFuncSetAttribute(
-        k_gemm_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<EPI>());
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes<EPI, BN>());
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI>, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI, BN>, &cfg) != cudaSuccess ||
+        n <= 0) {
       cudaGetLastError();
       n = sm_count / 2;
     }
     max_pairs = n;
   }
-  const int64_t tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);
+  const int64_t tiles =
+      ((M + PM - 1) / PM) * ((N + BN - 1) / BN) * (int64_t)sc.count;
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
-  return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI>, tmA, tmB, maps.out, maps.yref,
-                            M, N, Kc, ep);
+  return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI, BN>, tmA, tmB, maps.out, maps.yref,
+                            M, N, Kc, ep, sc);
 }
 
 }  // namespace
@@ -451,14 +537,42 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const EpiMaps& maps, int64_t M, int64_t N,
                              int64_t Kc, int mode, const EpiParams& ep,
                              int sm_count, cudaStream_t st) {
+  const GemmSched one;
   switch (mode) {
     case EPI_STORE_F32:
-      return launch_pair_epi<EPI_STORE_F32>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_STORE_F32, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
+                                                 sm_count, st);
     case EPI_LOSS_DY:
-      return launch_pair_epi<EPI_LOSS_DY>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_LOSS_DY, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
+                                               sm_count, st);
     default:
-      return launch_pair_epi<EPI_LOSS>(tmA, tmB, maps, M, N, Kc, ep, sm_count, st);
+      return launch_pair_epi<EPI_LOSS, 256>(tmA, tmB, maps, M, N, Kc, one, ep, sm_count,
+                                            st);
   }
+}
+
+cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmOut, int64_t M, int64_t N,
+                                int64_t Kc, int bn, const GemmSched& sc,
+                                const EpiParams& ep, int sm_count, cudaStream_t st) {
+  if (sc.count < 1 || sc.inner < 1 || M <= 0 || N <= 0 || Kc <= 0 || Kc % BK)
+    return cudaErrorInvalidValue;
+  if (sc.causal) {
+    if (sc.seg <= 0 || sc.seg % PM || sc.nseg < 1) return cudaErrorInvalidValue;
+    if (sc.causal == 1 && M % sc.seg) return cudaErrorInvalidValue;
+    if (sc.causal == 2 && (M != sc.seg || Kc != sc.seg * sc.nseg)) return cudaErrorInvalidValue;
+    if (sc.causal > 2) return cudaErrorInvalidValue;
+  }
+  EpiMaps maps;
+  maps.out = tmOut;
+  maps.yref = tmOut;
+  if (bn == 128)
+    return launch_pair_epi<EPI_STORE_F32, 128>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
+                                               st);
+  if (bn == 256)
+    return launch_pair_epi<EPI_STORE_F32, 256>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
+                                               st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace gsq

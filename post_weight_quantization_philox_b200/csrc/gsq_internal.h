@@ -66,6 +66,37 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                              int64_t Kc, int mode, const EpiParams& ep,
                              int sm_count, cudaStream_t st);
 
+// Many equal GEMMs in one launch.  Problem p = p1 * inner + p2 (p < count)
+// is C_p[M x N] = A_p[M x Kc] . B_p[N x Kc]^T, where the operands and the
+// output are windows of the tensor maps whose origin is
+//   rows: x[0] * p1 + x[1] * p2,   K / columns: likewise
+// for x = a_row / a_k (A), b_row / b_k (B), o_row / o_col (output).
+// causal = 1 (lower-triangular A): the rows of A repeat in periods of `seg`
+// rows, and an output tile whose rows sit at [r0, r0 + 256) of a period
+// contracts over K in [0, r0 + 256) only (A is zero beyond).
+// causal = 2 (transposed): K is `nseg` periods of `seg`, and a tile whose rows
+// sit at [r0, r0 + 256) of a period of M contracts over [r0, seg) of each
+// K period only.  Tiles with the longest K run first.
+// Only the fp32 store epilogue; Kc and, with causal, seg are multiples of 64
+// and seg of 256.
+struct GemmSched {
+  int count = 1, inner = 1;
+  int64_t a_row[2] = {0, 0}, a_k[2] = {0, 0};
+  int64_t b_row[2] = {0, 0}, b_k[2] = {0, 0};
+  int64_t o_row[2] = {0, 0}, o_col[2] = {0, 0};
+  int causal = 0;
+  int64_t seg = 0;
+  int nseg = 1;
+};
+// Box rows of the B tensor map for the 128-wide output tiles (bn = 128).
+constexpr int kGemmBoxRowsBNarrow = 64;
+// bn = 256 (B map with kGemmBoxRowsB rows per box) or 128 (B map with
+// kGemmBoxRowsBNarrow rows per box, for N = 128 problems).
+cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                const CUtensorMap& tmOut, int64_t M, int64_t N,
+                                int64_t Kc, int bn, const GemmSched& sc,
+                                const EpiParams& ep, int sm_count, cudaStream_t st);
+
 // ------------------------------------------------------- elementwise
 struct StepArgs {
   int mode;

@@ -96,6 +96,29 @@ def test_one_step(g, oracle_mod, mode):
     a.close()
 
 
+DIMS_CAUSAL = dict(nseq=2, S=512, nh=4, nkv=2, d=128)
+
+
+def test_one_step_causal_tiles(g, oracle_mod):
+    """S a multiple of 256: the batched products skip the zero half of P."""
+    dims = DIMS_CAUSAL
+    Xa, Wq, Wk, Wv, Wo = case(seed=7, **dims)
+    R = fp_target(oracle_mod, Xa, Wq, Wk, Wv, Wo, dims)
+    a = make(g, Xa, R, Wq, Wk, Wv, Wo, mode=0, seed=9, dims=dims)
+    at = oracle_mod.attn_init(0, Wv, Wo, seed=9)
+    P = oracle_mod.attn_probs(Xa, Wq, Wk, **dims)
+    tau, lr = 0.7, 1e-3
+    a.step(tau, lr)
+    loss, d = oracle_mod.attn_step(at, Xa, P, R.astype(np.float64), tuple(dims.values()),
+                                   tau, lr, dumps=True)
+    assert abs(a.last_loss() - loss) <= 1e-2 * loss
+    for i in range(2):
+        dW = a.get(i, g.GSQ_DBG_DW)
+        assert np.linalg.norm(dW - d["dW"][i]) / np.linalg.norm(d["dW"][i]) < 2e-2
+        assert (a.get(i, g.GSQ_DBG_LOGITS) == at.weights()[i].logits).mean() > 0.99
+    a.close()
+
+
 def test_trajectory(g, oracle_mod):
     Xa, Wq, Wk, Wv, Wo = case(seed=2)
     R = fp_target(oracle_mod, Xa, Wq, Wk, Wv, Wo, DIMS)
@@ -139,28 +162,67 @@ def test_run_equals_step_loop_bit_exact(g, oracle_mod):
 
 def test_full_70b_shape(g, oracle_mod):
     """The 70B attention shape (64 query / 8 value heads of 128, 8 x 2048
-    tokens): sampled probability rows against the oracle, finite losses, and
-    the value-gradient identity on sampled entries."""
+    tokens) in the bench's launch configuration: sampled probability rows
+    against the oracle; after one step, sampled entries of V, of the
+    attention outputs o = P V and of the value gradient dV = sum P^T do
+    recomputed on the host from the step's own bf16 operands; a short run
+    with finite losses."""
     import torch
     cfg = synth.ATTN_STAGE["c5_70b_attn"]
     dims = dict(nseq=cfg["nseq"], S=cfg["S"], nh=cfg["nh"], nkv=cfg["nkv"], d=cfg["d"])
+    nseq, S, nh, nkv, d = (dims[k] for k in ("nseq", "S", "nh", "nkv", "d"))
+    grp = nh // nkv
     Xa, Wq, Wk, Wv, Wo = synth.make_attn_stage(**dims)
     T, H = Xa.shape
     R = synth.random_target(T, H, 0.05)
     dev = lambda x: torch.from_numpy(x).cuda().to(torch.bfloat16)
     a = g.gsq_attn_init(dev(Xa), torch.from_numpy(R).cuda(), dev(Wq), dev(Wk), dev(Wv),
-                        dev(Wo), dims["nseq"], dims["S"], dims["nh"], dims["nkv"], dims["d"],
-                        grid_mode=cfg["grid"], seed=0)
+                        dev(Wo), nseq, S, nh, nkv, d, grid_mode=cfg["grid"], seed=0)
     P = a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_P)
     for s, h, q in [(0, 0, 5), (3, 17, 1000), (7, 63, 2047)]:
         row = bits_to_f32(P[s, h, q]).astype(np.float64)
-        ref = oracle_mod.attn_prob_row(Xa, Wq, Wk, dims["nseq"], dims["S"], dims["nh"],
-                                       dims["nkv"], s, h, q).astype(np.float64)
+        ref = oracle_mod.attn_prob_row(Xa, Wq, Wk, nseq, S, nh, nkv, s, h, q).astype(np.float64)
         assert np.all(row[q + 1:] == 0)
         assert np.abs(row - ref).max() < 2e-2
         assert abs(row.sum() - 1.0) < 2e-2
+    s_chk = 5
+    Ps = bits_to_f32(P[s_chk]).astype(np.float64)  # nh x S x S
     del P
+    a.step(1.0, 1e-3)
+    assert np.isfinite(a.last_loss()) and a.last_loss() > 0
+    rows = slice(s_chk * S, (s_chk + 1) * S)
+    VT = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_VT)).astype(np.float64)  # Hk x T
+    Wv_hat = bits_to_f32(a.get(0, g.GSQ_DBG_WHAT)).astype(np.float64)
+    # V = bf16(Xa Wv^T): sampled rows within one bf16 rounding
+    for j in (0, 517, nkv * d - 1):
+        ref = Xa[rows].astype(np.float64) @ Wv_hat[j]
+        mag = np.abs(Xa[rows].astype(np.float64)) @ np.abs(Wv_hat[j])
+        assert np.all(np.abs(VT[j, rows] - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5 * mag)
+    # o = P V for sampled (head, query) rows of one sequence
+    O = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_O)).astype(np.float64)  # T x H
+    for h, q in [(0, 0), (9, 255), (9, 256), (40, 1500), (63, 2047)]:
+        gq = h // grp
+        ref = Ps[h, q] @ VT[gq * d:(gq + 1) * d, rows].T
+        mag = Ps[h, q] @ np.abs(VT[gq * d:(gq + 1) * d, rows]).T
+        got = O[s_chk * S + q, h * d:(h + 1) * d]
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5 * mag), (h, q)
+    del O
+    # dV = sum over the group's heads of P^T do, do = bf16(dp Wo) (sampled keys)
+    dpT = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DPT))  # H x T
+    Wo_hat = bits_to_f32(a.get(1, g.GSQ_DBG_WHAT))
+    dV = a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DV).reshape(T, nkv * d)
+    gk = 3
+    dp_s = torch.from_numpy(np.ascontiguousarray(dpT[:, rows].T)).double()
+    do = (dp_s @ torch.from_numpy(Wo_hat[:, gk * grp * d:(gk + 1) * grp * d]).double())
+    do = do.float().to(torch.bfloat16).double().numpy()  # S x (grp d)
+    for key in (0, 255, 256, 1024, 2047):
+        ref = np.zeros(d)
+        for hig in range(grp):
+            h = gk * grp + hig
+            ref += Ps[h, :, key] @ do[:, hig * d:(hig + 1) * d]
+        got = dV[s_chk * S + key, gk * d:(gk + 1) * d].astype(np.float64)
+        assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref) + 1e-12, key
     taus = synth.tau_schedule(1.0, 0.05, cfg["steps"])
-    a.run(taus[:2], 1e-3)
+    a.run(taus[1:3], 1e-3)
     assert np.isfinite(a.last_loss()) and a.last_loss() > 0
     a.close()
