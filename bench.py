@@ -291,17 +291,25 @@ def cpu_baseline(cfg, budget_s=15.0, steps=None):
 def load_traffic(kernel, config):
     """DRAM bytes per launch from the committed ncu summary, or None when the
     kernels changed since those counters were taken."""
-    import glob
-    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    src = sorted(glob.glob(os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc", "*")))
-    h = hashlib.sha256(b"".join(open(f, "rb").read() for f in src)).hexdigest()[:16]
-    if d.get("_csrc_sha256_16") != h:
+    if d.get("_kernel_sources_sha256_16") != kernel_sources_hash():
         return None
     return d.get(config, {}).get(kernel)
+
+
+# the sources that define the single-layer step's kernels and their launches
+STEP_KERNEL_SOURCES = ("gsq_api.cu", "gsq_device.cuh", "gsq_gemm.cu", "gsq_gemm_epi.cuh",
+                       "gsq_gemm_pair.cu", "gsq_internal.h", "gsq_kernels.cu")
+
+
+def kernel_sources_hash():
+    import hashlib
+    csrc = os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc")
+    blob = b"".join(open(os.path.join(csrc, f), "rb").read() for f in STEP_KERNEL_SOURCES)
+    return hashlib.sha256(blob).hexdigest()[:16]
 
 
 def run_mlp_stage(args, rank, world, local_rank):

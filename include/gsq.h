@@ -305,7 +305,7 @@ enum {
     GSQ_ATTN_DBG_VT = 2,  /* nkv d x T bf16  V^T = Wv Xa^T                */
     GSQ_ATTN_DBG_O = 3,   /* T x H bf16 attention output o                */
     GSQ_ATTN_DBG_DPT = 4, /* H x T bf16 2 (pred^T - R^T)                  */
-    GSQ_ATTN_DBG_DV = 5,  /* T x nkv d fp32 value gradient dV             */
+    GSQ_ATTN_DBG_DV = 5,  /* T x nkv d bf16 value gradient dV             */
     GSQ_ATTN_DBG_RT = 6   /* H x T fp32 R^T                               */
 };
 GSQ_API int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype,

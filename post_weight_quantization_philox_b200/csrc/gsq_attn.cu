@@ -11,11 +11,13 @@
 //   P^T[s][g][key][hig][q] (hig = h - g grp), i.e. one K-major operand per
 //   (s, g) for the value gradient.
 // Per step t (CTA-pair tcgen05 GEMMs, all A . B^T with K-major operands):
-//   V^T = Wv Xa^T                                  (Hk x T)
-//   o_(s,g-heads) = P_(s, g's heads) . V_(s,g)      (grp S x d per (s, g))
+//   V^T = bf16(Wv Xa^T)                               (Hk x T)
+//   o_(s,g-heads) = bf16(P_(s, g's heads) . V_(s,g))   (grp S x d per (s, g),
+//                   written straight into o, T x H)
 //   pred^T = Wo o^T; E = pred^T - R^T; loss; dp^T = bf16(2E)
-//   dWo = dp^T . o ;  do^T = Wo^T dp^T
-//   dV_(s,g) = P^T_(s,g) . do_(s, g's heads)         (S x d, K = grp S)
+//   dWo = dp^T . o ;  do^T = bf16(Wo^T dp^T)           (H x T)
+//   dV_(s,g) = bf16(P^T_(s,g) . do_(s, g's heads))     (S x d, K = grp S: one
+//              K segment per head, read from do^T in place)
 //   dWv = dV^T . Xa ; backward + Lion for Wv and Wo.
 // The per-(s, g) products run as one batched launch each, on 256 x 128
 // tiles (N = d = 128).  When S is a multiple of 256 they skip the zero half
@@ -42,8 +44,8 @@ struct gsq_attn {
   StageWeight w[2];  // value (Hk x H), output (H x H)
   __nv_bfloat16 *Xa = nullptr, *XaT = nullptr, *P = nullptr, *PT = nullptr;
   __nv_bfloat16 *VT = nullptr, *o = nullptr, *oT = nullptr, *dpT = nullptr, *dp = nullptr;
-  __nv_bfloat16 *WoT = nullptr, *dog = nullptr, *dVb = nullptr, *dVT = nullptr;
-  float *RT = nullptr, *VT32 = nullptr, *og = nullptr, *doT32 = nullptr, *dV32 = nullptr;
+  __nv_bfloat16 *WoT = nullptr, *doT = nullptr, *dVb = nullptr, *dVT = nullptr;
+  float* RT = nullptr;
   double *partials = nullptr, *loss_hist = nullptr, *scratch = nullptr;
   unsigned* ticket = nullptr;
   int* err = nullptr;
@@ -53,7 +55,7 @@ struct gsq_attn {
   CUtensorMap tmB_Xa, tmB_o, tmB_oT, tmB_dp, tmB_XaT, tmA_dpT, tmA_WoT, tmA_dVT;
   EpiMaps em_VT, em_pred, em_doT;
   // all (s, g) problems of a step in one launch each (GemmSched)
-  CUtensorMap tmA_P, tmB_VT, tm_og, tmA_PT, tmB_dog, tm_dV;
+  CUtensorMap tmA_P, tmB_VT, tm_o, tmA_PT, tmB_doT, tm_dV;
   GemmSched sc_pv, sc_dv;
   std::vector<void*> allocs;
 };
@@ -131,15 +133,11 @@ cudaError_t forward(gsq_attn* c, double* loss_out, bool with_dp) {
   const int64_t T = c->T, H = c->H, Hk = c->Hk, S = c->S;
   cudaError_t e;
   EpiParams ep = epi(c, loss_out);
-  if ((e = launch_gemm(c->w[0].tmA, c->tmB_Xa, c->em_VT, Hk, T, H, EPI_STORE_F32, ep,
+  if ((e = launch_gemm(c->w[0].tmA, c->tmB_Xa, c->em_VT, Hk, T, H, EPI_STORE_BF16, ep,
                        c->sms, c->st)) != cudaSuccess) return e;
-  if ((e = launch_f32_to_bf16(c->VT32, Hk * T, c->VT, c->sms, c->st)) != cudaSuccess)
+  if ((e = launch_gemm_batched(c->tmA_P, c->tmB_VT, c->tm_o, c->grp * S, c->d, S, 128,
+                               c->sc_pv, EPI_STORE_BF16, ep, c->sms, c->st)) != cudaSuccess)
     return e;
-  if ((e = launch_gemm_batched(c->tmA_P, c->tmB_VT, c->tm_og, c->grp * S, c->d, S, 128,
-                               c->sc_pv, ep, c->sms, c->st)) != cudaSuccess)
-    return e;
-  if ((e = launch_gather_heads(c->og, c->nseq, S, c->nh, c->grp, (int)c->d, c->o,
-                               c->sms, c->st)) != cudaSuccess) return e;
   if ((e = launch_transpose_bf16(c->o, T, H, c->oT, c->st)) != cudaSuccess) return e;
   return launch_gemm(c->w[1].tmA, c->tmB_o, c->em_pred, H, T, H,
                      with_dp ? EPI_LOSS_DY : EPI_LOSS, ep, c->sms, c->st);
@@ -160,15 +158,12 @@ int run_step(gsq_attn* c, float tau, float tau_next, float lr, float b1, float b
   // do^T = Wo^T . dp^T
   CKA(launch_transpose_bf16(c->w[1].What, H, H, c->WoT, c->st));
   CKA(launch_transpose_bf16(c->dpT, H, T, c->dp, c->st));
-  CKA(launch_gemm(c->tmA_WoT, c->tmB_dp, c->em_doT, H, T, H, EPI_STORE_F32, ep, c->sms,
+  CKA(launch_gemm(c->tmA_WoT, c->tmB_dp, c->em_doT, H, T, H, EPI_STORE_BF16, ep, c->sms,
                   c->st));
-  CKA(launch_scatter_heads_t(c->doT32, c->nseq, S, c->nh, c->grp, (int)c->d, c->dog,
-                             c->sms, c->st));
   // dV_(s,g) = P^T_(s,g) . do_(s, g's heads)
-  CKA(launch_gemm_batched(c->tmA_PT, c->tmB_dog, c->tm_dV, S, c->d, c->grp * S, 128,
-                          c->sc_dv, ep, c->sms, c->st));
+  CKA(launch_gemm_batched(c->tmA_PT, c->tmB_doT, c->tm_dV, S, c->d, c->grp * S, 128,
+                          c->sc_dv, EPI_STORE_BF16, ep, c->sms, c->st));
   // dWv = dV^T . Xa
-  CKA(launch_f32_to_bf16(c->dV32, T * Hk, c->dVb, c->sms, c->st));
   CKA(launch_transpose_bf16(c->dVb, T, Hk, c->dVT, c->st));
   CKA(launch_gemm(c->tmA_dVT, c->tmB_XaT, c->w[0].em_dW, Hk, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
@@ -197,7 +192,7 @@ int attn_buffer(gsq_attn* c, int which, int buf, void** p, size_t* bytes) {
     case GSQ_ATTN_DBG_VT: *p = c->VT; *bytes = TK * 2; return GSQ_OK;
     case GSQ_ATTN_DBG_O: *p = c->o; *bytes = TH * 2; return GSQ_OK;
     case GSQ_ATTN_DBG_DPT: *p = c->dpT; *bytes = TH * 2; return GSQ_OK;
-    case GSQ_ATTN_DBG_DV: *p = c->dV32; *bytes = TK * 4; return GSQ_OK;
+    case GSQ_ATTN_DBG_DV: *p = c->dVb; *bytes = TK * 2; return GSQ_OK;
     case GSQ_ATTN_DBG_RT: *p = c->RT; *bytes = TH * 4; return GSQ_OK;
     default: return GSQ_ERR_INVALID_ARG;
   }
@@ -273,17 +268,13 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
   ALA(c->RT, H * T);
   ALA(c->P, PS);
   ALA(c->PT, PS);
-  ALA(c->VT32, Hk * T);
   ALA(c->VT, Hk * T);
-  ALA(c->og, T * H);
   ALA(c->o, T * H);
   ALA(c->oT, H * T);
   ALA(c->dpT, H * T);
   ALA(c->dp, T * H);
   ALA(c->WoT, H * H);
-  ALA(c->doT32, H * T);
-  ALA(c->dog, T * H);
-  ALA(c->dV32, T * Hk);
+  ALA(c->doT, H * T);
   ALA(c->dVb, T * Hk);
   ALA(c->dVT, Hk * T);
   ALA(c->partials, kStagePartials);
@@ -389,9 +380,9 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
   bad |= make_tmap_bf16(&c->tmA_dVT, c->dVT, Hk, T, T, kGemmBoxRowsA) != 0;
   {
     CUtensorMap m;
-    bad |= make_tmap_epi_f32(&m, c->VT32, Hk, T, T) != 0;
+    bad |= make_tmap_epi_bf16(&m, c->VT, Hk, T, T) != 0;
     c->em_VT = out_only(m);
-    bad |= make_tmap_epi_f32(&m, c->doT32, H, T, T) != 0;
+    bad |= make_tmap_epi_bf16(&m, c->doT, H, T, T) != 0;
     c->em_doT = out_only(m);
     bad |= make_tmap_epi_bf16(&c->em_pred.out, c->dpT, H, T, T) != 0;
     bad |= make_tmap_epi_f32(&c->em_pred.yref, c->RT, H, T, T) != 0;
@@ -401,16 +392,17 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
     bad |= make_tmap_bf16(&c->tmA_P, c->P, c->nseq * c->nh * S, S, S, kGemmBoxRowsA) != 0;
     // V^T (Hk x T): problem (s, g) is rows g d.., columns s S..
     bad |= make_tmap_bf16(&c->tmB_VT, c->VT, Hk, T, T, kGemmBoxRowsBNarrow) != 0;
-    // attention outputs per (s, g): (grp S) x d, stacked
-    bad |= make_tmap_epi_f32(&c->tm_og, c->og, c->nseq * c->nh * S, d, d) != 0;
+    // o (T x H): problem (s, g) rows (hig, q) land at row s S + q, columns
+    // (g grp + hig) d..
+    bad |= make_tmap_epi_bf16(&c->tm_o, c->o, T, H, H) != 0;
     // P^T as (nseq nkv S) x (grp S)
     bad |= make_tmap_bf16(&c->tmA_PT, c->PT, c->nseq * c->nkv * S, grp * S, grp * S,
                           kGemmBoxRowsA) != 0;
-    // do per (s, g) as d x (grp S), stacked
-    bad |= make_tmap_bf16(&c->tmB_dog, c->dog, c->nseq * c->nkv * d, grp * S, grp * S,
-                          kGemmBoxRowsBNarrow) != 0;
+    // do^T (H x T): K segment hig of problem (s, g) is rows (g grp + hig) d..,
+    // columns s S..
+    bad |= make_tmap_bf16(&c->tmB_doT, c->doT, H, T, T, kGemmBoxRowsBNarrow) != 0;
     // dV (T x Hk): problem (s, g) is rows s S.., columns g d..
-    bad |= make_tmap_epi_f32(&c->tm_dV, c->dV32, T, Hk, Hk) != 0;
+    bad |= make_tmap_epi_bf16(&c->tm_dV, c->dVb, T, Hk, Hk) != 0;
     // problem p = s nkv + g; causal K ranges when a period holds whole tiles
     const bool causal = S % 256 == 0;
     GemmSched& a = c->sc_pv;
@@ -420,8 +412,10 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
     a.a_row[1] = grp * S;
     a.b_row[1] = d;
     a.b_k[0] = S;
-    a.o_row[0] = c->nh * S;
-    a.o_row[1] = grp * S;
+    a.o_row[0] = S;
+    a.o_col[1] = grp * d;
+    a.o_fold = S;
+    a.o_fold_col = d;
     a.causal = causal ? 1 : 0;
     a.seg = S;
     GemmSched& b = c->sc_dv;
@@ -429,13 +423,15 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
     b.inner = (int)c->nkv;
     b.a_row[0] = c->nkv * S;
     b.a_row[1] = S;
-    b.b_row[0] = c->nkv * d;
-    b.b_row[1] = d;
+    b.b_row[1] = grp * d;
+    b.b_k[0] = S;
     b.o_row[0] = S;
     b.o_col[1] = d;
     b.causal = causal ? 2 : 0;
     b.seg = S;
     b.nseg = (int)grp;
+    b.a_seg_k = S;
+    b.b_seg_row = d;
   }
   if (bad) return cleanup_fail(GSQ_ERR_CUDA);
 

@@ -69,9 +69,9 @@ constexpr int OUT_TILE = 32 * 32 * 4;
 constexpr int DY_TILE = 32 * 32 * 2;
 template <int EPI>
 __host__ __device__ constexpr int warp_stage_bytes() {
-  return EPI == EPI_STORE_F32 ? 2 * OUT_TILE
-                              : (EPI == EPI_LOSS_DY ? 2 * OUT_TILE + 2 * DY_TILE
-                                                    : 2 * OUT_TILE);
+  return EPI == EPI_STORE_BF16 ? 2 * DY_TILE
+                               : (EPI == EPI_LOSS_DY ? 2 * OUT_TILE + 2 * DY_TILE
+                                                     : 2 * OUT_TILE);
 }
 template <int EPI, int BN>
 __host__ __device__ constexpr int smem_bytes() {
@@ -102,6 +102,7 @@ __device__ __forceinline__ TileAt tile_at(int tile, int m_tiles, int n_tiles,
     nb = r % n_tiles;
     p = r / n_tiles;
     t.nk = (int)((Kc + BK - 1) / BK);
+    if (sc.nseg > 1) t.kps = (int)(sc.seg / BK);
   } else {
     // the period position is the slowest index, longest K first
     const int rbs = (int)(sc.seg / PM);
@@ -136,12 +137,26 @@ __device__ __forceinline__ TileAt tile_at(int tile, int m_tiles, int n_tiles,
   return t;
 }
 
-// K coordinate (inside the problem) of K block kb of a tile
-__device__ __forceinline__ int64_t tile_k(const TileAt& t, int kb,
-                                          const GemmSched& sc) {
-  if (sc.causal != 2) return (int64_t)kb * BK;
+// TMA coordinates of K block kb of a tile: A and B column (K) and the row
+// offset each operand adds for its K segment
+struct KAt {
+  int64_t ak, bk, arow, brow;
+};
+__device__ __forceinline__ KAt tile_k(const TileAt& t, int kb, const GemmSched& sc) {
+  KAt k;
+  if (sc.causal != 2 && sc.nseg <= 1) {
+    k.ak = t.a_k + (int64_t)kb * BK;
+    k.bk = t.b_k + (int64_t)kb * BK;
+    k.arow = k.brow = 0;
+    return k;
+  }
   const int sgi = kb / t.kps;
-  return sgi * sc.seg + t.r0 + (int64_t)(kb - sgi * t.kps) * BK;
+  const int64_t within = t.r0 + (int64_t)(kb - sgi * t.kps) * BK;
+  k.ak = t.a_k + sgi * sc.a_seg_k + within;
+  k.bk = t.b_k + sgi * sc.b_seg_k + within;
+  k.arow = sgi * sc.a_seg_row;
+  k.brow = sgi * sc.b_seg_row;
+  return k;
 }
 
 // shared-memory offset of 16-byte chunk j of row r in a tile written or
@@ -200,7 +215,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ctl->abort = 0;
     mbar_fence_init();
     if (EPI != EPI_LOSS) tma_prefetch_desc(&tmO);
-    if (EPI != EPI_STORE_F32) tma_prefetch_desc(&tmY);
+    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -234,9 +249,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb_leader = mapa_shared(fb, 0);
           if (leader) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
           const uint32_t sa = sbase + stage * STAGE_BYTES;
-          const int64_t kx = tile_k(ta, kb, sc);
-          tma_load_2d_pair(sa, &tmA, fb_leader, (int32_t)(ta.a_k + kx), ya);
-          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, (int32_t)(ta.b_k + kx), yb);
+          const KAt kx = tile_k(ta, kb, sc);
+          tma_load_2d_pair(sa, &tmA, fb_leader, (int32_t)kx.ak, ya + (int32_t)kx.arow);
+          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, (int32_t)kx.bk,
+                           yb + (int32_t)kx.brow);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -337,8 +353,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const TileAt ta = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
       const int64_t lx = ta.n0 + (int)(u % UNITS) * 32;
       const int64_t ly = ta.m0 + (int)rank * HALF + q * 32;
-      x = (int32_t)(ta.o_col + lx);
-      y = (int32_t)(ta.o_row + ly);
+      if (sc.o_fold > 0) {
+        const int64_t f = ly / sc.o_fold;
+        x = (int32_t)(ta.o_col + f * sc.o_fold_col + lx);
+        y = (int32_t)(ta.o_row + (ly - f * sc.o_fold));
+      } else {
+        x = (int32_t)(ta.o_col + lx);
+        y = (int32_t)(ta.o_row + ly);
+      }
       return lx < N && ly < M;
     };
     int64_t y_issued = 0;
@@ -349,7 +371,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive_expect_tx(bar, OUT_TILE);
       tma_load_2d(y_s + (uint32_t)((u & 1) * OUT_TILE), &tmY, bar, x, y);
     };
-    if (EPI != EPI_STORE_F32 && lane == 0) {
+    if ((EPI == EPI_LOSS_DY || EPI == EPI_LOSS) && lane == 0) {
       for (; y_issued < 2 && y_issued < total_units; ++y_issued) issue_y(y_issued);
     }
     int acc = 0;
@@ -376,7 +398,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int32_t x, y;
         const bool inside = unit_xy(u, x, y);
         const int b = (int)(u & 1);
-        if (EPI == EPI_STORE_F32) {
+        if (EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
           // this buffer may be rewritten once the store that last read it is
           // done: the newest group if it used this buffer, else the one before
           if (lane == 0) {
@@ -384,14 +406,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else bulk_wait_read<1>();
           }
           __syncwarp();
-          const uint32_t base = out_s + (uint32_t)(b * OUT_TILE);
+          const uint32_t base =
+              out_s + (uint32_t)(b * (EPI == EPI_STORE_F32 ? OUT_TILE : DY_TILE));
+          if (EPI == EPI_STORE_F32) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t a = base + swz128(lane, j);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
-                         "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]),
-                         "r"(v[4 * j + 3])
-                         : "memory");
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t a = base + swz128(lane, j);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                           "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]),
+                           "r"(v[4 * j + 3])
+                           : "memory");
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t a = base + swz64(lane, j);
+              const float* f = reinterpret_cast<const float*>(v) + 8 * j;
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                           "r"(pack_bf16x2(f[0], f[1])), "r"(pack_bf16x2(f[2], f[3])),
+                           "r"(pack_bf16x2(f[4], f[5])), "r"(pack_bf16x2(f[6], f[7]))
+                           : "memory");
+            }
           }
           fence_async_smem();
           __syncwarp();
@@ -474,7 +509,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bulk_wait_all();  // stores complete before the CTA exits
     }
     __syncwarp();
-    if (EPI != EPI_STORE_F32) {
+    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS) {
       lsum = warp_sum_d(lsum);
       if (lane == 0) ctl->red[q] = lsum;
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -545,6 +580,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
     case EPI_LOSS_DY:
       return launch_pair_epi<EPI_LOSS_DY, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
                                                sm_count, st);
+    case EPI_STORE_BF16:
+      return launch_pair_epi<EPI_STORE_BF16, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
+                                                  sm_count, st);
     default:
       return launch_pair_epi<EPI_LOSS, 256>(tmA, tmB, maps, M, N, Kc, one, ep, sm_count,
                                             st);
@@ -553,25 +591,36 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
 
 cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmOut, int64_t M, int64_t N,
-                                int64_t Kc, int bn, const GemmSched& sc,
+                                int64_t Kc, int bn, const GemmSched& sc, int mode,
                                 const EpiParams& ep, int sm_count, cudaStream_t st) {
   if (sc.count < 1 || sc.inner < 1 || M <= 0 || N <= 0 || Kc <= 0 || Kc % BK)
     return cudaErrorInvalidValue;
+  if (sc.causal < 0 || sc.causal > 2 || sc.nseg < 1) return cudaErrorInvalidValue;
+  if (sc.nseg > 1 || sc.causal == 2) {
+    if (sc.seg <= 0 || sc.seg % BK || Kc != sc.seg * sc.nseg) return cudaErrorInvalidValue;
+    if (sc.causal == 1) return cudaErrorInvalidValue;
+  }
   if (sc.causal) {
-    if (sc.seg <= 0 || sc.seg % PM || sc.nseg < 1) return cudaErrorInvalidValue;
+    if (sc.seg <= 0 || sc.seg % PM) return cudaErrorInvalidValue;
     if (sc.causal == 1 && M % sc.seg) return cudaErrorInvalidValue;
-    if (sc.causal == 2 && (M != sc.seg || Kc != sc.seg * sc.nseg)) return cudaErrorInvalidValue;
-    if (sc.causal > 2) return cudaErrorInvalidValue;
+    if (sc.causal == 2 && M != sc.seg) return cudaErrorInvalidValue;
   }
   EpiMaps maps;
   maps.out = tmOut;
   maps.yref = tmOut;
-  if (bn == 128)
+  if (sc.o_fold < 0 || (sc.o_fold > 0 && sc.o_fold % 32)) return cudaErrorInvalidValue;
+  if (mode == EPI_STORE_F32 && bn == 128)
     return launch_pair_epi<EPI_STORE_F32, 128>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
                                                st);
-  if (bn == 256)
+  if (mode == EPI_STORE_F32 && bn == 256)
     return launch_pair_epi<EPI_STORE_F32, 256>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
                                                st);
+  if (mode == EPI_STORE_BF16 && bn == 128)
+    return launch_pair_epi<EPI_STORE_BF16, 128>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
+                                                st);
+  if (mode == EPI_STORE_BF16 && bn == 256)
+    return launch_pair_epi<EPI_STORE_BF16, 256>(tmA, tmB, maps, M, N, Kc, sc, ep, sm_count,
+                                                st);
   return cudaErrorInvalidValue;
 }
 

@@ -20,7 +20,8 @@ enum : int {
 enum EpiMode : int {
   EPI_STORE_F32 = 0,  // C = acc (fp32 store)
   EPI_LOSS_DY = 1,    // E = acc - Yref; loss += sum E^2; dY = bf16(2E)
-  EPI_LOSS = 2        // E = acc - Yref; loss += sum E^2
+  EPI_LOSS = 2,       // E = acc - Yref; loss += sum E^2
+  EPI_STORE_BF16 = 3  // C = bf16(acc)
 };
 
 struct EpiParams {
@@ -30,9 +31,9 @@ struct EpiParams {
   int* err;              // device error word
 };
 
-// The epilogue's tensor maps: out = C (EPI_STORE_F32, fp32 map) or dY
-// (EPI_LOSS_DY, bf16 map); yref = Y_ref (EPI_LOSS*, fp32 map).  Unused maps
-// may be any valid map.
+// The epilogue's tensor maps: out = C (EPI_STORE_F32, fp32 map; EPI_STORE_BF16,
+// bf16 map) or dY (EPI_LOSS_DY, bf16 map); yref = Y_ref (EPI_LOSS*, fp32 map).
+// Unused maps may be any valid map.
 struct EpiMaps {
   CUtensorMap out;
   CUtensorMap yref;
@@ -74,11 +75,16 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
 // causal = 1 (lower-triangular A): the rows of A repeat in periods of `seg`
 // rows, and an output tile whose rows sit at [r0, r0 + 256) of a period
 // contracts over K in [0, r0 + 256) only (A is zero beyond).
-// causal = 2 (transposed): K is `nseg` periods of `seg`, and a tile whose rows
-// sit at [r0, r0 + 256) of a period of M contracts over [r0, seg) of each
-// K period only.  Tiles with the longest K run first.
-// Only the fp32 store epilogue; Kc and, with causal, seg are multiples of 64
-// and seg of 256.
+// nseg > 1: K is `nseg` segments of `seg` columns (Kc = nseg seg); segment i
+// of A starts at K column i a_seg_k and row offset i a_seg_row, of B at
+// i b_seg_k and i b_seg_row.
+// causal = 2 (transposed, with segments): a tile whose rows sit at
+// [r0, r0 + 256) of M (M = seg) contracts over [r0, seg) of each segment
+// only.  With causal, tiles with the longest K run first.
+// o_fold > 0: local output row ly goes to row ly % o_fold, column offset
+// (ly / o_fold) o_fold_col (rows of stacked heads placed side by side).
+// Store epilogues only; Kc and, with causal, seg are multiples of 64 and seg
+// of 256.
 struct GemmSched {
   int count = 1, inner = 1;
   int64_t a_row[2] = {0, 0}, a_k[2] = {0, 0};
@@ -87,14 +93,17 @@ struct GemmSched {
   int causal = 0;
   int64_t seg = 0;
   int nseg = 1;
+  int64_t a_seg_k = 0, a_seg_row = 0, b_seg_k = 0, b_seg_row = 0;
+  int64_t o_fold = 0, o_fold_col = 0;
 };
 // Box rows of the B tensor map for the 128-wide output tiles (bn = 128).
 constexpr int kGemmBoxRowsBNarrow = 64;
 // bn = 256 (B map with kGemmBoxRowsB rows per box) or 128 (B map with
 // kGemmBoxRowsBNarrow rows per box, for N = 128 problems).
+// mode: EPI_STORE_F32 (tmOut an fp32 epilogue map) or EPI_STORE_BF16 (bf16).
 cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmOut, int64_t M, int64_t N,
-                                int64_t Kc, int bn, const GemmSched& sc,
+                                int64_t Kc, int bn, const GemmSched& sc, int mode,
                                 const EpiParams& ep, int sm_count, cudaStream_t st);
 
 // ------------------------------------------------------- elementwise
@@ -172,11 +181,5 @@ cudaError_t launch_transpose_ld(const __nv_bfloat16* in, int64_t rows, int64_t c
                                 cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* in, int64_t n, __nv_bfloat16* out,
                                int sm_count, cudaStream_t st);
-cudaError_t launch_gather_heads(const float* og, int64_t nseq, int64_t S, int64_t nh,
-                                int64_t grp, int d, __nv_bfloat16* o, int sm_count,
-                                cudaStream_t st);
-cudaError_t launch_scatter_heads_t(const float* doT, int64_t nseq, int64_t S,
-                                   int64_t nh, int64_t grp, int d,
-                                   __nv_bfloat16* dog, int sm_count, cudaStream_t st);
 
 }  // namespace gsq

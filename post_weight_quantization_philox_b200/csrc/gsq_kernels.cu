@@ -750,42 +750,58 @@ __global__ void k_transpose_ld(const __nv_bfloat16* __restrict__ in, int64_t row
   }
 }
 
+// The same transpose with 16-byte accesses (rows, cols, ld_in, ld_out and
+// both pointers multiples of 8 elements / 16 bytes): a 64 x 64 tile per
+// iteration, held in shared memory as 32-bit words (two neighbouring
+// columns); an output word pairs rows 2p and 2p + 1 of one column, taken
+// from two words with one byte permute.  Each lane writes 32 contiguous
+// output bytes (16 rows of one column).
+__global__ void __launch_bounds__(256) k_transpose_b16v(
+    const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t cols,
+    int64_t ld_in, __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  __shared__ uint32_t tile[64][33];
+  const int tid = threadIdx.x;
+  const int64_t tr = (rows + 63) / 64, tc = (cols + 63) / 64;
+  for (int64_t t = blockIdx.x; t < tr * tc; t += gridDim.x) {
+    const int64_t r0 = (t / tc) * 64, c0 = (t % tc) * 64;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int id = tid + 256 * i, r = id >> 3, ch = id & 7;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r0 + r < rows && c0 + ch * 8 < cols)
+        v = __ldg(reinterpret_cast<const uint4*>(in + (r0 + r) * ld_in + c0 + ch * 8));
+      tile[r][ch * 4] = v.x;
+      tile[r][ch * 4 + 1] = v.y;
+      tile[r][ch * 4 + 2] = v.z;
+      tile[r][ch * 4 + 3] = v.w;
+    }
+    __syncthreads();
+    {
+      const int c = tid & 63, q = tid >> 6;  // output row c0 + c, rows 16 q ..
+      const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;  // high or low halves
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int r = 16 * q + 2 * k;
+        w[k] = __byte_perm(tile[r][c >> 1], tile[r + 1][c >> 1], sel);
+      }
+      if (c0 + c < cols) {
+        __nv_bfloat16* o = out + (c0 + c) * ld_out + r0 + 16 * q;
+        if (r0 + 16 * q < rows)
+          *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (r0 + 16 * q + 8 < rows)
+          *reinterpret_cast<uint4*>(o + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void k_f32_to_bf16(const float* __restrict__ in, int64_t n,
                               __nv_bfloat16* __restrict__ out) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
     out[i] = __float2bfloat16_rn(in[i]);
-}
-
-// o (T x nh d, bf16) from the per-group stacked attention outputs
-// og[s][g][hig][q][j] (fp32), h = g grp + hig
-__global__ void k_gather_heads(const float* __restrict__ og, int64_t nseq,
-                               int64_t S, int64_t nh, int64_t grp, int d,
-                               __nv_bfloat16* __restrict__ o) {
-  const int64_t H = nh * d, n = nseq * S * H;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / H, c = i % H;
-    const int64_t s = t / S, q = t % S, h = c / d, j = c % d;
-    const int64_t g = h / grp, hig = h % grp;
-    const int64_t nkv = nh / grp;
-    o[i] = __float2bfloat16_rn(og[(((s * nkv + g) * grp + hig) * S + q) * d + j]);
-  }
-}
-
-// dog[s][g][j][hig][q] (bf16) from do^T (nh d x T, fp32): the output
-// gradient of each group's heads, laid out as one K-major operand per (s, g)
-__global__ void k_scatter_heads_t(const float* __restrict__ doT, int64_t nseq,
-                                  int64_t S, int64_t nh, int64_t grp, int d,
-                                  __nv_bfloat16* __restrict__ dog) {
-  const int64_t T = nseq * S, H = nh * d, n = H * T;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / T, t = i % T;  // row = h d + j
-    const int64_t h = row / d, j = row % d, s = t / S, q = t % S;
-    const int64_t g = h / grp, hig = h % grp, nkv = nh / grp;
-    dog[(((s * nkv + g) * d + j) * grp + hig) * S + q] = __float2bfloat16_rn(doT[i]);
-  }
 }
 
 int grid_for(int64_t work, int threads, int cap) {
@@ -976,9 +992,32 @@ cudaError_t launch_swiglu_bwd(const float* a, const float* b, const float* dh,
   return cudaGetLastError();
 }
 
+namespace {
+bool b16v_ok(const void* in, int64_t rows, int64_t cols, int64_t ld_in,
+             const void* out, int64_t ld_out) {
+  return rows % 8 == 0 && cols % 8 == 0 && ld_in % 8 == 0 && ld_out % 8 == 0 &&
+         (reinterpret_cast<uintptr_t>(in) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+}
+cudaError_t launch_b16v(const __nv_bfloat16* in, int64_t rows, int64_t cols,
+                        int64_t ld_in, __nv_bfloat16* out, int64_t ld_out,
+                        cudaStream_t st) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = ((rows + 63) / 64) * ((cols + 63) / 64);
+  const int64_t cap = (int64_t)sms * 8;
+  k_transpose_b16v<<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, st>>>(in, rows, cols,
+                                                                         ld_in, out, ld_out);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows,
                                   int64_t cols, __nv_bfloat16* out,
                                   cudaStream_t st) {
+  if (rows > 0 && cols > 0 && b16v_ok(in, rows, cols, cols, out, rows))
+    return launch_b16v(in, rows, cols, cols, out, rows, st);
   dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
   k_transpose<__nv_bfloat16, __nv_bfloat16><<<grid, dim3(64, 4), 0, st>>>(in, rows, cols, out);
   return cudaGetLastError();
@@ -1010,6 +1049,8 @@ cudaError_t launch_causal_softmax(const float* scores, int64_t S, float scale,
 cudaError_t launch_transpose_ld(const __nv_bfloat16* in, int64_t rows, int64_t cols,
                                 int64_t ld_in, __nv_bfloat16* out, int64_t ld_out,
                                 cudaStream_t st) {
+  if (rows > 0 && cols > 0 && b16v_ok(in, rows, cols, ld_in, out, ld_out))
+    return launch_b16v(in, rows, cols, ld_in, out, ld_out, st);
   dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
   k_transpose_ld<<<grid, dim3(64, 4), 0, st>>>(in, rows, cols, ld_in, out, ld_out);
   return cudaGetLastError();
@@ -1018,22 +1059,6 @@ cudaError_t launch_transpose_ld(const __nv_bfloat16* in, int64_t rows, int64_t c
 cudaError_t launch_f32_to_bf16(const float* in, int64_t n, __nv_bfloat16* out,
                                int sm_count, cudaStream_t st) {
   k_f32_to_bf16<<<grid_for(n, 256, sm_count * 8), 256, 0, st>>>(in, n, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_heads(const float* og, int64_t nseq, int64_t S, int64_t nh,
-                                int64_t grp, int d, __nv_bfloat16* o, int sm_count,
-                                cudaStream_t st) {
-  k_gather_heads<<<grid_for(nseq * S * nh * d, 256, sm_count * 8), 256, 0, st>>>(
-      og, nseq, S, nh, grp, d, o);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_scatter_heads_t(const float* doT, int64_t nseq, int64_t S,
-                                   int64_t nh, int64_t grp, int d,
-                                   __nv_bfloat16* dog, int sm_count, cudaStream_t st) {
-  k_scatter_heads_t<<<grid_for(nseq * S * nh * d, 256, sm_count * 8), 256, 0, st>>>(
-      doT, nseq, S, nh, grp, d, dog);
   return cudaGetLastError();
 }
 

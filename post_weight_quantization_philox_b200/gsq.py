@@ -576,7 +576,7 @@ class Attn:
                 GSQ_ATTN_DBG_VT: ((self.Hk, self.T), np.uint16),
                 GSQ_ATTN_DBG_O: ((self.T, self.H), np.uint16),
                 GSQ_ATTN_DBG_DPT: ((self.H, self.T), np.uint16),
-                GSQ_ATTN_DBG_DV: ((self.T, self.Hk), np.float32),
+                GSQ_ATTN_DBG_DV: ((self.T, self.Hk), np.uint16),
                 GSQ_ATTN_DBG_RT: ((self.H, self.T), np.float32)}[buf]
 
     def get(self, which, buf):

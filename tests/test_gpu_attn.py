@@ -210,7 +210,7 @@ def test_full_70b_shape(g, oracle_mod):
     # dV = sum over the group's heads of P^T do, do = bf16(dp Wo) (sampled keys)
     dpT = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DPT))  # H x T
     Wo_hat = bits_to_f32(a.get(1, g.GSQ_DBG_WHAT))
-    dV = a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DV).reshape(T, nkv * d)
+    dV = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DV)).reshape(T, nkv * d)
     gk = 3
     dp_s = torch.from_numpy(np.ascontiguousarray(dpT[:, rows].T)).double()
     do = (dp_s @ torch.from_numpy(Wo_hat[:, gk * grp * d:(gk + 1) * grp * d]).double())
