@@ -236,6 +236,15 @@ __device__ __forceinline__ void noise1(int64_t c, uint32_t t, uint32_t k0,
   for (int p = 0; p < L; ++p) g[p] = gg[p];
 }
 
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w) {
+  __nv_bfloat162 b01 = __floats2bfloat162_rn(w[0], w[1]);
+  __nv_bfloat162 b23 = __floats2bfloat162_rn(w[2], w[3]);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&b01);
+  pk.y = *reinterpret_cast<uint32_t*>(&b23);
+  *reinterpret_cast<uint2*>(dst) = pk;
+}
+
 // Both kernels below give one warp a group of 128 coordinates of one row;
 // lane j takes coordinates j, j+32, j+64, j+96, so every load and store of a
 // logit plane is one coalesced 128-byte access and each coordinate is
@@ -293,56 +302,96 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 // a separate soft-weight launch would produce.  All loads of the group are
 // issued first and the next step's noise (which needs none of them) is
 // computed while they are in flight.
+// Backward + Lion (A5), optionally fused with the next step's A1 + A2.  One
+// warp per 128-group; lane j owns the four consecutive coordinates 4j..4j+3.
+// The warp's next group is staged into shared memory with per-lane 16-byte
+// async copies (each lane copies exactly the pieces it will read) while the
+// current group is computed, so the loads of one group overlap the
+// arithmetic of the previous one.  Every global access is 16 bytes wide.
+template <int MODE>
+struct BwdCfg {
+  static constexpr int L = GridT<MODE>::L;
+  static constexpr int PLANES = 1 + 3 * L;  // dW, logits, momenta, noise
+  static constexpr int BUF = PLANES * 512 + (MODE == GRID_3BIT_LOCAL ? 128 : 0);
+  static constexpr int WARPS = L == 5 ? 4 : 8;  // warps per CTA
+  static constexpr int CTAS = L == 5 ? 3 : 2;   // CTAs per SM
+  static constexpr int SMEM = WARPS * 2 * BUF;
+};
+
 template <int MODE, bool DBG, bool NEXT>
-__global__ void __launch_bounds__(256, 2) k_backward_lion(
-    float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ s,
-    float* __restrict__ ms, const int8_t* __restrict__ i0,
-    const float* __restrict__ dW, float* __restrict__ gbuf, int64_t N,
-    int64_t K, uint32_t k0, uint32_t k1, uint32_t t_next, int noise,
-    float inv_tau, float inv_tau_next, float lr, float b1, float omb1, float b2,
-    float omb2, __nv_bfloat16* __restrict__ What, float* __restrict__ dl_dbg,
-    float* __restrict__ ds_dbg) {
-  constexpr int L = GridT<MODE>::L;
-  const int64_t NK = N * K, G = K / kGroup;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t gi = warp; gi < N * G; gi += nwarps) {
-    const int64_t n = gi / G, g = gi - n * G;
-    const int64_t base = n * K + g * kGroup + lane;
+__global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
+    k_backward_lion(float* __restrict__ logits, float* __restrict__ mom,
+                    float* __restrict__ s, float* __restrict__ ms,
+                    const int8_t* __restrict__ i0, const float* __restrict__ dW,
+                    float* __restrict__ gbuf, int64_t N, int64_t K, uint32_t k0,
+                    uint32_t k1, uint32_t t_next, int noise, float inv_tau,
+                    float inv_tau_next, float lr, float b1, float omb1, float b2,
+                    float omb2, __nv_bfloat16* __restrict__ What,
+                    float* __restrict__ dl_dbg, float* __restrict__ ds_dbg) {
+  using C = BwdCfg<MODE>;
+  constexpr int L = C::L;
+  extern __shared__ __align__(16) uint8_t bwd_smem[];
+  const int64_t NK = N * K, G = K / kGroup, groups = N * G;
+  const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
+  const int64_t warp = (int64_t)blockIdx.x * C::WARPS + wic;
+  const int64_t nwarps = (int64_t)gridDim.x * C::WARPS;
+  const uint32_t wbuf = smem_u32(bwd_smem) + (uint32_t)(wic * 2 * C::BUF);
+  // shared-memory plane order: dW, logits 0..L-1, momenta, noise, (i0)
+  auto prefetch = [&](int64_t gi, int buf) {
+    const int64_t c = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
+    const uint32_t d = wbuf + (uint32_t)(buf * C::BUF + 16 * lane);
+    cp_async16(d, dW + c);
+#pragma unroll
+    for (int p = 0; p < L; ++p) {
+      cp_async16(d + (uint32_t)((1 + p) * 512), logits + p * NK + c);
+      cp_async16(d + (uint32_t)((1 + L + p) * 512), mom + p * NK + c);
+      cp_async16(d + (uint32_t)((1 + 2 * L + p) * 512), gbuf + p * NK + c);
+    }
+    if (MODE == GRID_3BIT_LOCAL)
+      cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::PLANES * 512 + 4 * lane), i0 + c);
+  };
+  int64_t gi = warp;
+  if (gi < groups) prefetch(gi, 0);
+  cp_async_commit();
+  for (int buf = 0; gi < groups; gi += nwarps, buf ^= 1) {
+    if (gi + nwarps < groups) prefetch(gi + nwarps, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();  // this lane's copies of group gi have landed
+    const uint8_t* sb = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
+    const int64_t c0 = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
     const float sg = s[gi];
     const float msg = ms[gi];
-    float ds_part = 0.f;
-    float lnew[NEXT ? kPerLane : 1][L];
-    int lev[kPerLane];
-    float Lr[kPerLane][L], Mr[kPerLane][L], Gr[kPerLane][L], Dr[kPerLane];
+    float Dr[4], Lr[L][4], Mr[L][4], Gr[L][4];
+    *reinterpret_cast<float4*>(Dr) = *reinterpret_cast<const float4*>(sb);
 #pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-      const int64_t c = base + 32 * j;
-#pragma unroll
-      for (int p = 0; p < L; ++p) {
-        Lr[j][p] = logits[p * NK + c];
-        Mr[j][p] = mom[p * NK + c];
-        Gr[j][p] = gbuf[p * NK + c];
-      }
-      Dr[j] = __ldg(dW + c);
-      lev[j] = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
+    for (int p = 0; p < L; ++p) {
+      *reinterpret_cast<float4*>(Lr[p]) = *reinterpret_cast<const float4*>(sb + (1 + p) * 512);
+      *reinterpret_cast<float4*>(Mr[p]) =
+          *reinterpret_cast<const float4*>(sb + (1 + L + p) * 512);
+      *reinterpret_cast<float4*>(Gr[p]) =
+          *reinterpret_cast<const float4*>(sb + (1 + 2 * L + p) * 512);
     }
-    float gnext[NEXT ? kPerLane : 1][L];
+    int lev[4] = {0, 0, 0, 0};
+    if (MODE == GRID_3BIT_LOCAL) {
+      const uint32_t b4 = *reinterpret_cast<const uint32_t*>(
+          bwd_smem + wic * 2 * C::BUF + buf * C::BUF + C::PLANES * 512 + 4 * lane);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) lev[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
+    }
+    float gnext[NEXT ? 4 : 1][L];
     if (NEXT) {
 #pragma unroll
-      for (int j = 0; j < kPerLane; ++j)
-        noise1<L>(base + 32 * j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
+      for (int j = 0; j < 4; ++j) noise1<L>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
     }
+    float ds_part = 0.f;
+    float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
 #pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-      const int64_t c = base + 32 * j;
-      float l[L], m[L], gz[L], y[L], cand[5];
+    for (int j = 0; j < 4; ++j) {
+      float l[L], gz[L], y[L], cand[5];
 #pragma unroll
       for (int p = 0; p < L; ++p) {
-        l[p] = Lr[j][p];
-        m[p] = Mr[j][p];
-        gz[p] = Gr[j][p];
+        l[p] = Lr[p][j];
+        gz[p] = Gr[p][j];
       }
       const float dw = Dr[j];
       candidates<MODE>(lev[j], cand);
@@ -368,13 +417,20 @@ __global__ void __launch_bounds__(256, 2) k_backward_lion(
       }
 #pragma unroll
       for (int p = 0; p < L; ++p) {
-        float th = l[p], mm = m[p];
+        float th = l[p], mm = Mr[p][j];
         lion_update(th, mm, dl[p], lr, b1, omb1, b2, omb2);
-        logits[p * NK + c] = th;
-        mom[p * NK + c] = mm;
-        if (NEXT) lnew[NEXT ? j : 0][p] = th;
-        if (DBG) dl_dbg[p * NK + c] = dl[p];
+        Lo[p][j] = th;
+        Mo[p][j] = mm;
+        if (DBG) Do[DBG ? p : 0][j] = dl[p];
       }
+    }
+#pragma unroll
+    for (int p = 0; p < L; ++p) {
+      *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(Lo[p]);
+      *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(Mo[p]);
+      if (DBG)
+        *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
+            *reinterpret_cast<float4*>(Do[DBG ? p : 0]);
     }
     // every lane takes lane 0's sum so that all lanes hold the same new scale
     const float ds = __shfl_sync(0xffffffffu, warp_sum(ds_part), 0);
@@ -386,20 +442,25 @@ __global__ void __launch_bounds__(256, 2) k_backward_lion(
       if (DBG) ds_dbg[gi] = ds;
     }
     if (NEXT) {
+      float w[4];
 #pragma unroll
-      for (int j = 0; j < kPerLane; ++j) {
-        const int64_t c = base + 32 * j;
-        float y[L], cand[5];
-        float (&gz)[L] = gnext[NEXT ? j : 0];
+      for (int j = 0; j < 4; ++j) {
+        float l[L], y[L], cand[5];
+#pragma unroll
+        for (int p = 0; p < L; ++p) l[p] = Lo[p][j];
         candidates<MODE>(lev[j], cand);
-        const float w = s_new * coord_soft<MODE>(lnew[NEXT ? j : 0], gz,
-                                                 inv_tau_next, cand, y);
-        What[c] = __float2bfloat16_rn(w);
+        w[j] = s_new * coord_soft<MODE>(l, gnext[NEXT ? j : 0], inv_tau_next, cand, y);
+      }
+      store_bf16x4(What + c0, w);
 #pragma unroll
-        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = gz[p];
+      for (int p = 0; p < L; ++p) {
+        float4 g4 = make_float4(gnext[NEXT ? 0 : 0][p], gnext[NEXT ? 1 : 0][p],
+                                gnext[NEXT ? 2 : 0][p], gnext[NEXT ? 3 : 0][p]);
+        *reinterpret_cast<float4*>(gbuf + p * NK + c0) = g4;
       }
     }
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------- harden + pack (A6)
@@ -586,14 +647,6 @@ __global__ void __launch_bounds__(256) k_sumsq(const float* __restrict__ x,
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + expf(-x)); }
 
-__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w) {
-  __nv_bfloat162 b01 = __floats2bfloat162_rn(w[0], w[1]);
-  __nv_bfloat162 b23 = __floats2bfloat162_rn(w[2], w[3]);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&b01);
-  pk.y = *reinterpret_cast<uint32_t*>(&b23);
-  *reinterpret_cast<uint2*>(dst) = pk;
-}
 
 // hT = bf16(silu(aT) * bT), elementwise over n entries
 __global__ void __launch_bounds__(256) k_swiglu_fwd(const float* __restrict__ a,
@@ -892,16 +945,26 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   const float inv_tau = 1.0f / a.tau;
   const float inv_tau_next = NEXT ? 1.0f / tau_next : 0.f;
   const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
-  if (dl_dbg)
-    k_backward_lion<MODE, true, NEXT><<<blocks, 256, 0, st>>>(
+  using C = BwdCfg<MODE>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaFuncSetAttribute(k_backward_lion<MODE, true, NEXT>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaFuncSetAttribute(k_backward_lion<MODE, false, NEXT>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr_set = true;
+  }
+  if (dl_dbg) {
+    k_backward_lion<MODE, true, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
         a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         dl_dbg, ds_dbg);
-  else
-    k_backward_lion<MODE, false, NEXT><<<blocks, 256, 0, st>>>(
+  } else {
+    k_backward_lion<MODE, false, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
         a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         nullptr, nullptr);
+  }
 }
 
 template <int MODE>
@@ -923,7 +986,15 @@ cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
                                  float* dl_dbg, float* ds_dbg, int sm_count,
                                  cudaStream_t st) {
   const int64_t groups = a.N * (a.K / kGroup);
-  const int blocks = grid_for(groups * 32, 256, sm_count * 8);
+  // persistent: as many CTAs as fit on the SMs at once, fewer for small layers
+  auto blocks_for = [&](int warps, int ctas) {
+    const int64_t need = (groups + warps - 1) / warps;
+    const int64_t cap = (int64_t)sm_count * ctas;
+    return (int)(need < cap ? need : cap);
+  };
+  const int blocks = a.mode == GRID_3BIT_LOCAL
+                         ? blocks_for(BwdCfg<GRID_3BIT_LOCAL>::WARPS, BwdCfg<GRID_3BIT_LOCAL>::CTAS)
+                         : blocks_for(BwdCfg<GRID_2BIT>::WARPS, BwdCfg<GRID_2BIT>::CTAS);
   switch (a.mode) {
     case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
     case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
