@@ -80,6 +80,11 @@ def lib():
             "gsqo_recon_error": (None, [_i32, _i32, _i64, _i64, _i64, _i32, _p,
                                         _p, _p, _p, _p, _f32, _p, _p]),
             "gsqo_gemm_abt": (None, [_i64, _i64, _i64, _p, _p, _p]),
+            "gsqo_scale_backward_lion": (None, [_i32, _i64, _i64, _i32, _p, _p, _p,
+                                                _p, _p, _f32, _f32, _f32, _p]),
+            "gsqo_scale_step": (_i32, [_i32, _i64, _i64, _i64, _i32, _p, _p, _p,
+                                       _p, _p, _p, _f32, _f32, _f32, _p, _p, _p,
+                                       _p]),
             "gsqo_mlp_forward_backward": (_f64, [_i64, _i64, _i64, _p, _p, _p, _p,
                                                  _p, _i32, _p, _p, _p]),
             "gsqo_attn_probs": (None, [_i64, _i64, _i64, _i64, _i64, _f64, _p, _p,
@@ -280,6 +285,40 @@ def backward_lion(st: State, dW, tau, lr, beta1=0.9, beta2=0.99):
     if rc != 0:
         raise RuntimeError(f"gsqo_backward_lion failed ({rc})")
     return dl, ds
+
+
+def scale_backward_lion(st: State, dW, lr, beta1=0.9, beta2=0.99):
+    """Scale-only A5 from a given dW: the assignments frozen at the hard
+    choice of st.logits, Lion on st.s / st.ms in place; returns ds."""
+    L, N, K = st.logits.shape
+    dW = _f32a(dW)
+    ds = np.zeros_like(st.s)
+    lib().gsqo_scale_backward_lion(st.mode, N, K, st.group, _ptr(st.logits),
+                                   _ptr(st.i0), _ptr(st.s), _ptr(st.ms), _ptr(dW),
+                                   lr, beta1, beta2, _ptr(ds))
+    return ds
+
+
+def scale_step(st: State, X, Yref, lr: float, beta1: float = 0.9, beta2: float = 0.99,
+               dumps: bool = False):
+    """One scale-only step in place (logits untouched, t unchanged); returns
+    the loss (and the hard weight, dW and ds if dumps)."""
+    X = _f32a(X)
+    Yref = np.ascontiguousarray(Yref, np.float64)
+    L, N, K = st.logits.shape
+    T = X.shape[0]
+    d = {}
+    if dumps:
+        d = dict(w=np.zeros((N, K), np.float32), dW=np.zeros((N, K), np.float32),
+                 ds=np.zeros_like(st.s))
+    loss = C.c_double(0.0)
+    rc = lib().gsqo_scale_step(st.mode, N, K, T, st.group, _ptr(st.logits), _ptr(st.i0),
+                               _ptr(st.s), _ptr(st.ms), _ptr(X), _ptr(Yref), lr, beta1,
+                               beta2, C.byref(loss), _ptr(d.get("w")), _ptr(d.get("dW")),
+                               _ptr(d.get("ds")))
+    if rc != 0:
+        raise RuntimeError(f"gsqo_scale_step failed ({rc})")
+    return (loss.value, d) if dumps else loss.value
 
 
 def harden(mode, logits, i0):

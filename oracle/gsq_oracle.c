@@ -596,6 +596,70 @@ void gsqo_unpack(int mode, int64_t N, int64_t K, const uint32_t* packed,
         }
 }
 
+/* ----------------------------------------------------- scale-only step */
+
+/* Scale-only training (agihunt.info summary, optimisation paragraph: the
+ * 2-bit models get one more round that changes only the group scales),
+ * restated for the layer objective: the assignments stay at the hard choice
+ * of the current logits (gsqo_harden), the weight is w = bf16(s_g c_level),
+ * and only s moves:
+ *   ds_g = sum over the group of dW_i c_level(i)   (fp64 sum, in k order)
+ * followed by Lion on s with its momentum ms.  Given dW. */
+void gsqo_scale_backward_lion(int mode, int64_t N, int64_t K, int group,
+                              const float* logits, const int8_t* i0, float* s,
+                              float* ms, const float* dW, float lr, float beta1,
+                              float beta2, float* ds_dump) {
+    int64_t NK = N * K, G = K / group;
+    uint8_t* lev = (uint8_t*)malloc((size_t)NK);
+    float* ds = (float*)malloc((size_t)(N * G) * sizeof(float));
+    gsqo_harden(mode, N, K, logits, i0, lev);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            double acc = 0.0;
+            for (int64_t k = g * group; k < (g + 1) * group; ++k)
+                acc += (double)dW[n * K + k] * gsqo_level_value(mode, lev[n * K + k]);
+            ds[n * G + g] = (float)acc;
+        }
+    if (ds_dump) memcpy(ds_dump, ds, (size_t)(N * G) * sizeof(float));
+    gsqo_lion(N * G, s, ms, ds, lr, beta1, beta2);
+    free(lev);
+    free(ds);
+}
+
+/* One scale-only step: hard weight, loss and output gradient (gsqo_forward),
+ * weight gradient (gsqo_weight_grad), then gsqo_scale_backward_lion. */
+int gsqo_scale_step(int mode, int64_t N, int64_t K, int64_t T, int group,
+                    const float* logits, const int8_t* i0, float* s, float* ms,
+                    const float* X, const double* Yref, float lr, float beta1,
+                    float beta2, double* loss, float* w_dump, float* dW_dump,
+                    float* ds_dump) {
+    if (gsqo_num_logits(mode) < 0 || K % group != 0) return -1;
+    int64_t NK = N * K, G = K / group;
+    uint8_t* lev = (uint8_t*)malloc((size_t)NK);
+    float* wq = (float*)malloc((size_t)NK * sizeof(float));
+    float* dY = (float*)malloc((size_t)(T * N) * sizeof(float));
+    float* dW = (float*)malloc((size_t)NK * sizeof(float));
+    if (!lev || !wq || !dY || !dW) {
+        free(lev); free(wq); free(dY); free(dW);
+        return -3;
+    }
+    gsqo_harden(mode, N, K, logits, i0, lev);
+    for (int64_t c = 0; c < NK; ++c) {
+        int64_t n = c / K, k = c % K;
+        double w = (double)s[n * G + k / group] * gsqo_level_value(mode, lev[c]);
+        wq[c] = (float)gsqo_bf16_round(w);
+    }
+    double l = gsqo_forward(N, K, T, X, wq, Yref, dY);
+    gsqo_weight_grad(N, K, T, dY, X, dW);
+    gsqo_scale_backward_lion(mode, N, K, group, logits, i0, s, ms, dW, lr, beta1,
+                             beta2, ds_dump);
+    if (loss) *loss = l;
+    if (w_dump) memcpy(w_dump, wq, (size_t)NK * sizeof(float));
+    if (dW_dump) memcpy(dW_dump, dW, (size_t)NK * sizeof(float));
+    free(lev); free(wq); free(dY); free(dW);
+    return 0;
+}
+
 /* ------------------------------------------------------------ recon error */
 
 void gsqo_recon_error(int gmode, int emode, int64_t N, int64_t K, int64_t T,

@@ -126,6 +126,20 @@ void gsqo_recon_error(int gmode, int emode, int64_t N, int64_t K, int64_t T,
                       const int8_t* i0, const float* X, const double* Yref,
                       float tau, double* abs_err, double* rel_err);
 
+/* Scale-only step (the assignments frozen at the hard choice of the logits,
+ * only the group scales trained; agihunt.info summary, optimisation
+ * paragraph): w = bf16(s c_level); loss, dY, dW as in gsqo_step; ds_g =
+ * sum dW_i c_level(i); Lion on s, ms.  The _backward_lion form takes dW. */
+void gsqo_scale_backward_lion(int mode, int64_t N, int64_t K, int group,
+                              const float* logits, const int8_t* i0, float* s,
+                              float* ms, const float* dW, float lr, float beta1,
+                              float beta2, float* ds_dump);
+int gsqo_scale_step(int mode, int64_t N, int64_t K, int64_t T, int group,
+                    const float* logits, const int8_t* i0, float* s, float* ms,
+                    const float* X, const double* Yref, float lr, float beta1,
+                    float beta2, double* loss, float* w_dump, float* dW_dump,
+                    float* ds_dump);
+
 /* SwiGLU MLP joint stage (the block's MLP trained on the block output).
  * Xn (T x H): the normalised MLP input; R (T x H): the output the MLP must
  * produce; Wg, Wu (F x H) and Wd (H x F): the three soft weights.

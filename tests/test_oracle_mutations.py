@@ -14,6 +14,7 @@ sys.path.insert(0, HERE)
 import test_oracle_attn as attn_pins  # noqa: E402
 import test_oracle_mlp as mlp_pins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
+import test_oracle_scale as scale_pins  # noqa: E402
 
 # (name, original text, planted text, pins expected to catch it)
 MUTATIONS = [
@@ -72,6 +73,14 @@ MUTATIONS = [
     ("mlp_down_grad_transposed", "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + f];",
      "for (int64_t t = 0; t < T; ++t) acc += dp[t * H + n] * h[t * F + (F - 1 - f)];",
      ["mlp:test_mlp_matches_torch_autograd"]),
+    ("scale_grad_uses_level_index",
+     "acc += (double)dW[n * K + k] * gsqo_level_value(mode, lev[n * K + k]);",
+     "acc += (double)dW[n * K + k] * (double)lev[n * K + k];",
+     ["scale:test_scale_grad_central_differences"]),
+    ("scale_weight_unscaled",
+     "double w = (double)s[n * G + k / group] * gsqo_level_value(mode, lev[c]);\n        wq[c]",
+     "double w = gsqo_level_value(mode, lev[c]);\n        wq[c]",
+     ["scale:test_scale_grad_central_differences", "scale:test_scale_step_on_grid_weight_is_a_fixed_point"]),
 ]
 
 MODES = {"test_softmax_is_library_softmax": [0, 2]}
@@ -97,7 +106,8 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
     mod = _load_mutant(tmp_path, name, old, new)
     caught = []
     for tname in catchers:
-        module = {"mlp": mlp_pins, "attn": attn_pins}.get(tname.split(":")[0], pins) \
+        module = {"mlp": mlp_pins, "attn": attn_pins, "scale": scale_pins}.get(
+            tname.split(":")[0], pins) \
             if ":" in tname else pins
         tname = tname.split(":")[-1]
         fn = getattr(module, tname)
