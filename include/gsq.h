@@ -119,6 +119,23 @@ GSQ_API int gsq_run(gsq_ctx* ctx, const float* taus, int64_t n, float lr,
 
 /* gsq_last_loss -- loss (sum of squared errors) of the last step.  Syncs.
  * GSQ_ERR_NONFINITE if it was NaN / Inf; GSQ_ERR_STATE before any step. */
+/* Scale-only step (agihunt.info summary, optimisation paragraph: the 2-bit
+ * models get one more round that changes only the group scales), on the
+ * layer objective of gsq_step:
+ *   codes   = hard choice of the current logits (argmax, first maximum, no
+ *             noise; computed once and kept until the logits change),
+ *   w       = bf16(s_g c_code)                  (N x K),
+ *   loss, dY^T, dW as in gsq_step,
+ *   ds_g    = sum over group g of dW_i c_code(i),
+ *   Lion on s with momentum ms (as in gsq_step).
+ * Logits, their momenta and i0 are left as they are.  The step counter t
+ * advances and the loss goes to the same history as gsq_step's.  Enqueued
+ * on the context's stream without a host sync.
+ * Errors: GSQ_ERR_INVALID_ARG for lr < 0 or beta outside [0, 1);
+ * GSQ_ERR_STATE after an earlier failure. */
+GSQ_API int gsq_scale_step(gsq_ctx* ctx, float lr, float beta1, float beta2);
+/* n scale-only steps (n > 0) */
+GSQ_API int gsq_scale_run(gsq_ctx* ctx, int64_t n, float lr, float beta1, float beta2);
 GSQ_API int gsq_last_loss(gsq_ctx* ctx, double* loss);
 
 /* gsq_loss_history -- losses of steps [t0, t0 + n) (the last 4096 steps are
@@ -219,6 +236,8 @@ GSQ_API int gsq_debug_forward(gsq_ctx* ctx, double* loss);
 GSQ_API int gsq_debug_weight_grad(gsq_ctx* ctx);
 GSQ_API int gsq_debug_backward(gsq_ctx* ctx, float tau, float lr, float beta1,
                        float beta2);
+/* scale-only backward + Lion from the current dW (fills GSQ_DBG_DS) */
+GSQ_API int gsq_debug_scale_backward(gsq_ctx* ctx, float lr, float beta1, float beta2);
 
 /* ----------------------------------------------- block stage: SwiGLU MLP --
  * The GSQ pages quantize a transformer block in stages; the last stage trains

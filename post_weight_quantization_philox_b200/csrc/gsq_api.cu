@@ -54,6 +54,9 @@ struct gsq_ctx {
   // temperature what_tau (what_t < 0: nothing precomputed)
   int64_t what_t = -1;
   float what_tau = 0.f;
+  // level codes of the hard choice of the current logits (scale-only steps)
+  int8_t* hcode = nullptr;
+  bool hcode_valid = false;
   double yref_sq = 0.0;
   CUtensorMap tm_What, tm_Xb, tm_dYt, tm_Xt;  // GEMM operands
   EpiMaps em_forward;  // dY^T (bf16) out, Y_ref^T in
@@ -265,6 +268,7 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   AL(c->s, N * c->G);
   AL(c->ms, N * c->G);
   AL(c->i0, NK);
+  AL(c->hcode, NK);
   AL(c->partials, kMaxPartials);
   AL(c->loss_hist, kLossRing);
   AL(c->scratch, 4);
@@ -412,6 +416,7 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
                           c->What, nullptr, nullptr, c->sms, c->st));
   if (tm) CK(cudaEventRecord(tm->ev[4], c->st));
   c->t += 1;
+  c->hcode_valid = false;  // the logits moved
   if (tau_next > 0.f) {
     c->what_t = (int64_t)c->t;
     c->what_tau = tau_next;
@@ -421,9 +426,50 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
   return GSQ_OK;
 }
 
+// codes of the hard choice of the current logits, computed once per logits
+cudaError_t ensure_hard_codes(gsq_ctx* c) {
+  if (c->hcode_valid) return cudaSuccess;
+  cudaError_t e = launch_hard_codes(c->mode, c->N, c->K, c->logits, c->i0, c->hcode, c->st);
+  if (e == cudaSuccess) c->hcode_valid = true;
+  return e;
+}
+
+// One scale-only step: hard weight from the frozen codes and the current
+// scales, forward + loss, weight gradient, scale gradient + Lion on s.
+int run_scale_step(gsq_ctx* c, float lr, float beta1, float beta2) {
+  if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;
+  CK(ensure_hard_codes(c));
+  CK(launch_code_weight(c->mode, c->N, c->K, c->hcode, c->s, c->What, c->st));
+  CK(run_forward(c, c->loss_hist + (c->t % kLossRing), EPI_LOSS_DY));
+  CK(run_weight_grad(c));
+  CK(launch_scale_lion(c->mode, c->N, c->K, c->hcode, c->dW, c->s, c->ms, lr, beta1, beta2,
+                       nullptr, c->sms, c->st));
+  c->t += 1;
+  c->what_t = -1;
+  return GSQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int gsq_scale_step(gsq_ctx* c, float lr, float beta1, float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (!step_args_ok(1.0f, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
+  return run_scale_step(c, lr, beta1, beta2);
+}
+
+int gsq_scale_run(gsq_ctx* c, int64_t n, float lr, float beta1, float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (n <= 0 || !step_args_ok(1.0f, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < n; ++i) {
+    const int rc = run_scale_step(c, lr, beta1, beta2);
+    if (rc) return rc;
+  }
+  return GSQ_OK;
+}
 
 int gsq_step(gsq_ctx* c, float tau, float lr, float beta1, float beta2) {
   int u = usable(c);
@@ -589,6 +635,7 @@ int gsq_import_state(gsq_ctx* c, const void* host_buf, size_t bytes) {
   CK(cudaMemcpy(c->ms, p + 2 * lb + sb, sb, cudaMemcpyHostToDevice));
   c->t = h[5];
   c->what_t = -1;
+  c->hcode_valid = false;
   return GSQ_OK;
 }
 
@@ -697,6 +744,7 @@ int gsq_debug_set(gsq_ctx* c, int which, const void* host, size_t bytes) {
   CK(cudaStreamSynchronize(c->st));
   CK(cudaMemcpy(p, host, nb, cudaMemcpyHostToDevice));
   c->what_t = -1;  // any state change invalidates a precomputed soft weight
+  c->hcode_valid = false;  // and the hard codes
   return GSQ_OK;
 }
 
@@ -774,6 +822,21 @@ int gsq_debug_backward(gsq_ctx* c, float tau, float lr, float beta1,
   CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, 0.f, c->What,
                           c->dl, c->ds, c->sms, c->st));
   c->what_t = -1;
+  c->hcode_valid = false;
+  return check_device(c);
+}
+
+int gsq_debug_scale_backward(gsq_ctx* c, float lr, float beta1, float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (!step_args_ok(1.0f, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
+  void* p;
+  size_t nb;
+  int rc = debug_buffer(c, GSQ_DBG_DS, &p, &nb);
+  if (rc) return rc;
+  CK(ensure_hard_codes(c));
+  CK(launch_scale_lion(c->mode, c->N, c->K, c->hcode, c->dW, c->s, c->ms, lr, beta1, beta2,
+                       c->ds, c->sms, c->st));
   return check_device(c);
 }
 

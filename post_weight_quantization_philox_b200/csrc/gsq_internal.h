@@ -151,6 +151,15 @@ cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
 cudaError_t launch_harden_pack(int mode, int64_t N, int64_t K,
                                const float* logits, const int8_t* i0,
                                uint32_t* packed, cudaStream_t st);
+// scale-only step: int8 level codes of the hard choice; w = bf16(s c_code);
+// ds_g = sum dW c_code and Lion on s (ds into ds_dbg when not null)
+cudaError_t launch_hard_codes(int mode, int64_t N, int64_t K, const float* logits,
+                              const int8_t* i0, int8_t* code, cudaStream_t st);
+cudaError_t launch_code_weight(int mode, int64_t N, int64_t K, const int8_t* code,
+                               const float* s, __nv_bfloat16* What, cudaStream_t st);
+cudaError_t launch_scale_lion(int mode, int64_t N, int64_t K, const int8_t* code,
+                              const float* dW, float* s, float* ms, float lr, float b1,
+                              float b2, float* ds_dbg, int sm_count, cudaStream_t st);
 cudaError_t launch_export_scales(const float* s, int64_t n, uint16_t* f16,
                                  float* f32, cudaStream_t st);
 cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,

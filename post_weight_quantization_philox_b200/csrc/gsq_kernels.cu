@@ -481,6 +481,90 @@ __device__ __forceinline__ int hard_level(const float* l, int lev0) {
   return best;
 }
 
+// ------------------------------------------------- scale-only step
+
+// Level codes of the hard choice (argmax of the logits, no noise), four
+// coordinates per thread.
+template <int MODE>
+__global__ void __launch_bounds__(256) k_hard_codes(const float* __restrict__ logits,
+                                                    const int8_t* __restrict__ i0,
+                                                    int64_t NK, int8_t* __restrict__ code) {
+  constexpr int L = GridT<MODE>::L;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < NK / 4;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c0 = q * 4;
+    float4 lp[L];
+#pragma unroll
+    for (int p = 0; p < L; ++p) lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
+    char4 iv = make_char4(0, 0, 0, 0);
+    if (MODE == GRID_3BIT_LOCAL) iv = *reinterpret_cast<const char4*>(i0 + c0);
+    const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
+    int out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[L];
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
+      out[j] = hard_level<MODE>(l, lev0[j]);
+    }
+    *reinterpret_cast<char4*>(code + c0) =
+        make_char4((signed char)out[0], (signed char)out[1], (signed char)out[2],
+                   (signed char)out[3]);
+  }
+}
+
+// w = bf16(s_g c_code), four coordinates per thread
+template <int MODE>
+__global__ void __launch_bounds__(256) k_code_weight(const int8_t* __restrict__ code,
+                                                     const float* __restrict__ s, int64_t N,
+                                                     int64_t K, __nv_bfloat16* __restrict__ What) {
+  const int64_t NK = N * K, G = K / kGroup;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < NK / 4;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c0 = q * 4, n = c0 / K, k = c0 - n * K;
+    const float sg = __ldg(s + n * G + k / kGroup);
+    const char4 cv = *reinterpret_cast<const char4*>(code + c0);
+    const float w[4] = {sg * GridT<MODE>::level(cv.x), sg * GridT<MODE>::level(cv.y),
+                        sg * GridT<MODE>::level(cv.z), sg * GridT<MODE>::level(cv.w)};
+    store_bf16x4(What + c0, w);
+  }
+}
+
+// Scale-only backward + Lion: ds_g = sum over the group of dW_i c_code(i)
+// (one warp per group, four consecutive coordinates per lane, warp-shuffle
+// sum), then Lion on s and its momentum.
+template <int MODE>
+__global__ void __launch_bounds__(256) k_scale_lion(const int8_t* __restrict__ code,
+                                                    const float* __restrict__ dW,
+                                                    float* __restrict__ s,
+                                                    float* __restrict__ ms, int64_t N,
+                                                    int64_t K, float lr, float b1, float omb1,
+                                                    float b2, float omb2,
+                                                    float* __restrict__ ds_dbg) {
+  const int64_t G = K / kGroup;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t gi = warp; gi < N * G; gi += nwarps) {
+    const int64_t c0 = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
+    const float4 d4 = __ldg(reinterpret_cast<const float4*>(dW + c0));
+    const char4 cv = *reinterpret_cast<const char4*>(code + c0);
+    float part = d4.x * GridT<MODE>::level(cv.x);
+    part = fmaf(d4.y, GridT<MODE>::level(cv.y), part);
+    part = fmaf(d4.z, GridT<MODE>::level(cv.z), part);
+    part = fmaf(d4.w, GridT<MODE>::level(cv.w), part);
+    const float ds = __shfl_sync(0xffffffffu, warp_sum(part), 0);
+    if (lane == 0) {
+      float sv = s[gi], mv = ms[gi];
+      lion_update(sv, mv, ds, lr, b1, omb1, b2, omb2);
+      s[gi] = sv;
+      ms[gi] = mv;
+      if (ds_dbg) ds_dbg[gi] = ds;
+    }
+  }
+}
+
 // 2-bit / ternary: 16 codes -> one 32-bit word per thread.
 // 3-bit: 32 codes -> three 32-bit words per thread.  Codes never straddle
 // rows because K is a multiple of 128.
@@ -1012,6 +1096,50 @@ cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
     case GRID_2BIT: k_hard_weight<GRID_2BIT><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
     case GRID_TERNARY: k_hard_weight<GRID_TERNARY><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
     default: k_hard_weight<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hard_codes(int mode, int64_t N, int64_t K, const float* logits,
+                              const int8_t* i0, int8_t* code, cudaStream_t st) {
+  const int blocks = grid_for(N * K / 4, 256, 4096);
+  switch (mode) {
+    case GRID_2BIT: k_hard_codes<GRID_2BIT><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
+    case GRID_TERNARY: k_hard_codes<GRID_TERNARY><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
+    default: k_hard_codes<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(logits, i0, N * K, code);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_code_weight(int mode, int64_t N, int64_t K, const int8_t* code,
+                               const float* s, __nv_bfloat16* What, cudaStream_t st) {
+  const int blocks = grid_for(N * K / 4, 256, 4096);
+  switch (mode) {
+    case GRID_2BIT: k_code_weight<GRID_2BIT><<<blocks, 256, 0, st>>>(code, s, N, K, What); break;
+    case GRID_TERNARY: k_code_weight<GRID_TERNARY><<<blocks, 256, 0, st>>>(code, s, N, K, What); break;
+    default: k_code_weight<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(code, s, N, K, What);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_lion(int mode, int64_t N, int64_t K, const int8_t* code,
+                              const float* dW, float* s, float* ms, float lr, float b1,
+                              float b2, float* ds_dbg, int sm_count, cudaStream_t st) {
+  const int64_t groups = N * (K / kGroup);
+  const int blocks = grid_for(groups * 32, 256, sm_count * 8);
+  const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
+  switch (mode) {
+    case GRID_2BIT:
+      k_scale_lion<GRID_2BIT><<<blocks, 256, 0, st>>>(code, dW, s, ms, N, K, lr, b1, omb1, b2,
+                                                     omb2, ds_dbg);
+      break;
+    case GRID_TERNARY:
+      k_scale_lion<GRID_TERNARY><<<blocks, 256, 0, st>>>(code, dW, s, ms, N, K, lr, b1, omb1,
+                                                        b2, omb2, ds_dbg);
+      break;
+    default:
+      k_scale_lion<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(code, dW, s, ms, N, K, lr, b1,
+                                                           omb1, b2, omb2, ds_dbg);
   }
   return cudaGetLastError();
 }

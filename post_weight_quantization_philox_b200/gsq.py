@@ -43,6 +43,7 @@ EXPORTS = [
     "gsq_debug_uniforms", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
+    "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
@@ -87,6 +88,9 @@ _SIGS = {
     "gsq_debug_forward": [_p, C.POINTER(C.c_double)],
     "gsq_debug_weight_grad": [_p],
     "gsq_debug_backward": [_p, _f32, _f32, _f32, _f32],
+    "gsq_scale_step": [_p, _f32, _f32, _f32],
+    "gsq_scale_run": [_p, _i64, _f32, _f32, _f32],
+    "gsq_debug_scale_backward": [_p, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
     "gsq_uniforms_noalloc": [_i32, _u64, _u32, _u64, _i64, _p, _p],
     "gsq_mlp_init": [_pp, _p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i64, _i64,
@@ -222,6 +226,15 @@ def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
 def gsq_step(layer: "Layer", tau: float, lr: float, beta1: float = 0.9,
              beta2: float = 0.99) -> None:
     _check(_lib.gsq_step(layer.ctx, tau, lr, beta1, beta2), "gsq_step")
+
+
+def gsq_scale_step(layer: "Layer", lr: float, beta1: float = 0.9, beta2: float = 0.99) -> None:
+    _check(_lib.gsq_scale_step(layer.ctx, lr, beta1, beta2), "gsq_scale_step")
+
+
+def gsq_scale_run(layer: "Layer", n: int, lr: float, beta1: float = 0.9,
+                  beta2: float = 0.99) -> None:
+    _check(_lib.gsq_scale_run(layer.ctx, n, lr, beta1, beta2), "gsq_scale_run")
 
 
 def gsq_run(layer: "Layer", taus, lr: float, beta1: float = 0.9,
@@ -369,9 +382,19 @@ class Layer:
         _check(_lib.gsq_debug_backward(self.ctx, tau, lr, beta1, beta2),
                "gsq_debug_backward")
 
+    def debug_scale_backward(self, lr, beta1=0.9, beta2=0.99):
+        _check(_lib.gsq_debug_scale_backward(self.ctx, lr, beta1, beta2),
+               "gsq_debug_scale_backward")
+
     # convenience -------------------------------------------------------
     def step(self, tau, lr, beta1=0.9, beta2=0.99):
         gsq_step(self, tau, lr, beta1, beta2)
+
+    def scale_step(self, lr, beta1=0.9, beta2=0.99):
+        gsq_scale_step(self, lr, beta1, beta2)
+
+    def scale_run(self, n, lr, beta1=0.9, beta2=0.99):
+        gsq_scale_run(self, n, lr, beta1, beta2)
 
     def run(self, taus, lr, beta1=0.9, beta2=0.99):
         gsq_run(self, taus, lr, beta1, beta2)
