@@ -443,6 +443,65 @@ def run_attn_stage(args, rank, world, local_rank):
             "last_loss": loss}
 
 
+def run_scale_stage(args, rank, world, local_rank):
+    """Scale-only steps (assignments frozen at the hard choice, group scales
+    trained) on the --config layer, after a short GSQ warm start."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    cfg = synth.CONFIGS[args.config]
+    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
+    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    lay = gsq.gsq_init(torch.from_numpy(W).to(torch.bfloat16).cuda(),
+                       torch.from_numpy(X).to(torch.bfloat16).cuda(), 128, cfg.grid, seed=rank)
+    lay.run(synth.tau_schedule(cfg.tau0, cfg.tau1, 20), cfg.lr)  # assignments to freeze
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    lay.scale_run(args.warmup, cfg.lr)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    lay.scale_run(args.steps, cfg.lr)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    loss = lay.last_loss()
+    lay.close()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    per = ms / args.steps
+    flops = 4.0 * cfg.N * cfg.T * cfg.K  # forward + weight-gradient GEMMs
+    ach = flops / (per / 1e3) / 1e12
+    coords = cfg.N * cfg.K
+    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
+            "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
+            "config": {"workload": cfg.name + "_scale_only", "N": cfg.N, "K": cfg.K,
+                       "T": cfg.T, "grid": ["2bit", "ternary", "3bit_local"][cfg.grid],
+                       "step": "scale-only (hard codes frozen)"},
+            "roofline": {"bound": "tensor", "kernel": "whole scale-only step (2 GEMMs + 8 B/coord)",
+                         "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
+                         "frac": round(ach / tf_sus, 4),
+                         "peak_kind": f"{peak_kind} (sustained bf16)", "traffic": None},
+            "gpu_launches": int(args.steps * 4), "clocks": clk, "last_loss": loss}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -476,7 +535,7 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["mlp", "attn"],
+    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale"],
                     help="time a block stage instead of a single layer")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
@@ -503,6 +562,8 @@ def main():
         out = run_mlp_stage(args, rank, world, local_rank)
     elif args.stage == "attn":
         out = run_attn_stage(args, rank, world, local_rank)
+    elif args.stage == "scale":
+        out = run_scale_stage(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:
