@@ -19,6 +19,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
+from . import gptq  # noqa: F401  (GPTQ initial assignment, plain numpy)
+
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "gsq_oracle.c")
 LIB = os.path.join(HERE, "libgsq_oracle.so")

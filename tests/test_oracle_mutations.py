@@ -14,6 +14,7 @@ sys.path.insert(0, HERE)
 import test_oracle_attn as attn_pins  # noqa: E402
 import test_oracle_mlp as mlp_pins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
+import test_oracle_gptq as gptq_pins  # noqa: E402
 import test_oracle_scale as scale_pins  # noqa: E402
 
 # (name, original text, planted text, pins expected to catch it)
@@ -81,6 +82,14 @@ MUTATIONS = [
      "double w = (double)s[n * G + k / group] * gsqo_level_value(mode, lev[c]);\n        wq[c]",
      "double w = gsqo_level_value(mode, lev[c]);\n        wq[c]",
      ["scale:test_scale_grad_central_differences", "scale:test_scale_step_on_grid_weight_is_a_fixed_point"]),
+    ("gptq_update_transposed", "W[:, j + 1:] -= np.outer(e, U[j, j + 1:])",
+     "W[:, j + 1:] -= np.outer(e, U[j + 1:, j])",
+     ["gptq:test_first_column_update_is_damped_least_squares", "gptq:test_loss_identity_over_the_loop"]),
+    ("gptq_no_diagonal_division", "e = (W[:, j] - q) / U[j, j]", "e = (W[:, j] - q)",
+     ["gptq:test_first_column_update_is_damped_least_squares", "gptq:test_loss_identity_over_the_loop"]),
+    ("gptq_scale_from_group_start_only", "absmax = np.abs(W[:, j:j + group]).max(axis=1)",
+     "absmax = np.abs(W[:, j:j + 1]).max(axis=1)",
+     ["gptq:test_diagonal_hessian_is_round_to_nearest"]),
 ]
 
 MODES = {"test_softmax_is_library_softmax": [0, 2]}
@@ -90,10 +99,12 @@ def _load_mutant(tmp_path, name, old, new):
     dst = tmp_path / f"oracle_{name}"
     shutil.copytree(os.path.join(ROOT, "oracle"), dst,
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
-    src = (dst / "gsq_oracle.c").read_text()
+    target = "gptq.py" if name.startswith("gptq_") else "gsq_oracle.c"
+    src = (dst / target).read_text()
     assert src.count(old) == 1, f"mutation anchor not unique: {name}"
-    (dst / "gsq_oracle.c").write_text(src.replace(old, new))
-    spec = importlib.util.spec_from_file_location(f"oracle_{name}", dst / "__init__.py")
+    (dst / target).write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", dst / "__init__.py",
+                                                  submodule_search_locations=[str(dst)])
     mod = importlib.util.module_from_spec(spec)
     sys.modules[spec.name] = mod
     spec.loader.exec_module(mod)
@@ -106,7 +117,8 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
     mod = _load_mutant(tmp_path, name, old, new)
     caught = []
     for tname in catchers:
-        module = {"mlp": mlp_pins, "attn": attn_pins, "scale": scale_pins}.get(
+        module = {"mlp": mlp_pins, "attn": attn_pins, "scale": scale_pins,
+                  "gptq": gptq_pins}.get(
             tname.split(":")[0], pins) \
             if ":" in tname else pins
         tname = tname.split(":")[-1]
