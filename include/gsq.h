@@ -98,6 +98,36 @@ GSQ_API int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
              int grid_mode, const int8_t* init_idx, uint64_t seed,
              void* stream);
 
+/* GPTQ initial assignment (agihunt.info summary, optimisation paragraph: GSQ
+ * starts from GPTQ; the algorithm of Frantar et al., "GPTQ: Accurate
+ * Post-Training Quantization for Generative Pre-trained Transformers",
+ * ICLR 2023), for the symmetric group-128 grids of grid_mode:
+ *   H = bf16(X)^T bf16(X); dead inputs (H_ii = 0): H_ii = 1, W[:, i] = 0;
+ *   H += damp mean(diag H) I; U = upper Cholesky factor of H^-1;
+ *   columns in input order: at the first column of each group the scale is
+ *   absmax / c_max of the (updated) group; the column is rounded to the
+ *   nearest level (first on ties) and its error (w - s c) / U_jj is pushed
+ *   onto the later columns through row j of U.
+ * Computed in fp32 on the GPU (Hessian on the tensor cores).
+ * W (N x K) and X (T x K): fp32 or bf16 (w_dtype, x_dtype), host or device,
+ * read only.  levels (N x K int8 level indices, the init_idx of gsq_init)
+ * and scales (N x K/group fp32): caller-owned, host or device.  damp >= 0
+ * (GPTQ's default 0.01).  Synchronises the stream; allocates and frees its
+ * own workspace (about 8 K^2 + 8 N K bytes).
+ * Errors: GSQ_ERR_INVALID_ARG for bad sizes / pointers / dtypes / damp or
+ * K > 65536; GSQ_ERR_UNSUPPORTED for group != 128 or a non-sm_100 device;
+ * GSQ_ERR_NONFINITE if the damped Hessian is not positive definite in fp32
+ * or an input is not finite; GSQ_ERR_OOM. */
+GSQ_API int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N,
+                     int64_t K, int64_t T, int group, int grid_mode, float damp,
+                     int8_t* levels, float* scales, void* stream);
+/* gsq_init from the GPTQ assignment: the initial levels (init_idx) and the
+ * group scales both come from gsq_gptq (instead of round-to-nearest with
+ * absmax scales); everything else as gsq_init.  Synchronises the stream. */
+GSQ_API int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+                          int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+                          int grid_mode, float damp, uint64_t seed, void* stream);
+
 /*
  * gsq_step -- one reconstruction step at temperature tau (asynchronous):
  * soft weight (noise of step t), forward GEMM with fused loss and dY,

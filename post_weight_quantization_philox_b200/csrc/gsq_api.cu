@@ -207,6 +207,39 @@ const char* gsq_error_string(int status) {
   }
 }
 
+int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void* X, int x_dtype,
+                  int64_t N, int64_t K, int64_t T, int group, int grid_mode, float damp,
+                  uint64_t seed, void* stream) {
+  if (!out) return GSQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (N <= 0 || K <= 0 || group <= 0 || K % group != 0) return GSQ_ERR_INVALID_ARG;
+  int8_t* lev = nullptr;
+  float* sc = nullptr;
+  if (cudaMalloc(&lev, (size_t)N * K) != cudaSuccess ||
+      cudaMalloc(&sc, (size_t)N * (K / group) * 4) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(lev);
+    return GSQ_ERR_OOM;
+  }
+  int rc = gsq_gptq(W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, damp, lev, sc, stream);
+  if (!rc) rc = gsq_init(out, W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, lev, seed,
+                         stream);
+  if (!rc) {
+    gsq_ctx* c = *out;
+    if (cudaMemcpyAsync(c->s, sc, (size_t)N * c->G * 4, cudaMemcpyDeviceToDevice, c->st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(c->st) != cudaSuccess) {
+      cudaGetLastError();
+      gsq_destroy(c);
+      *out = nullptr;
+      rc = GSQ_ERR_CUDA;
+    }
+  }
+  cudaFree(lev);
+  cudaFree(sc);
+  return rc;
+}
+
 int gsq_packed_bytes(int grid_mode, int64_t N, int64_t K, size_t* bytes) {
   if (!bytes || N <= 0 || K <= 0 || K % kGroup != 0 || num_logits(grid_mode) < 0)
     return GSQ_ERR_INVALID_ARG;

@@ -1,0 +1,489 @@
+// gsq_gptq.cu -- GPTQ initial assignment for the GSQ grids on the GPU.
+//
+// GSQ starts its logits from a GPTQ solution (agihunt.info summary,
+// optimisation paragraph).  GPTQ is the algorithm of Frantar, Ashkboos,
+// Hoefler and Alistarh ("GPTQ: Accurate Post-Training Quantization for
+// Generative Pre-trained Transformers", ICLR 2023): columns are quantized in
+// input order and each column's rounding error is pushed onto the columns
+// not yet quantized through U, the upper Cholesky factor of H^-1
+// (H^-1 = U^T U, H = X^T X damped).  Here, for the symmetric group-128 GSQ
+// grids, in fp32:
+//
+//   H      = Xt Xt^T on the tensor cores (bf16 operands, fp32 accumulation)
+//   dead inputs (H_ii = 0): H_ii = 1, W[:, i] = 0; H_ii += damp mean(diag H)
+//   U      = J L^-1 J with L L^T = J H J (J reverses the index order), so
+//            U^T U = J (J H J)^-1 J = H^-1 and U is upper triangular;
+//            L from a blocked right-looking Cholesky (64 x 64 diagonal
+//            blocks in one CTA, a row-wise triangular solve for the panel,
+//            a SIMT fp32 GEMM for the trailing update), L^-1 by block
+//            forward substitution with the same two kernels
+//   per group of 128 columns: one thread per row carries the row's 128
+//            weights in shared memory, sets the group scale absmax / c_max
+//            from the updated weights, rounds each column to the nearest
+//            level (first on ties) and feeds its error
+//            e_j = (w_j - s c) / U_jj forward within the group; the error
+//            block E (128 x N) then updates every later column at once:
+//            W[:, j1:] -= E^T U[j0:j1, j1:]   (SIMT fp32 GEMM)
+//
+// This runs once per layer before the reconstruction steps; none of it is on
+// the per-step path.
+#include <cmath>
+#include <vector>
+
+#include "../../include/gsq.h"
+#include "gsq_device.cuh"
+#include "gsq_internal.h"
+#include "gsq_stage.h"
+
+namespace gsq {
+namespace {
+
+constexpr int kNb = 64;     // Cholesky / inverse block
+constexpr int kCols = 128;  // GPTQ column block (= the quantization group)
+
+int grid_cap(int64_t work, int threads, int cap) {
+  const int64_t b = (work + threads - 1) / threads;
+  return (int)(b < 1 ? 1 : (b > cap ? cap : b));
+}
+
+// dead inputs (H_ii = 0 -> 1, flagged), then H_ii += damp * mean(diag H);
+// one block
+__global__ void k_gptq_damp(float* __restrict__ H, int64_t K, float damp,
+                            int* __restrict__ dead) {
+  __shared__ double red[32];
+  double sum = 0.0;
+  for (int64_t i = threadIdx.x; i < K; i += blockDim.x) {
+    float d = H[i * K + i];
+    const int z = d == 0.f;
+    dead[i] = z;
+    if (z) {
+      d = 1.f;
+      H[i * K + i] = 1.f;
+    }
+    sum += (double)d;
+  }
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    double v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float add = (float)((double)damp * red[0] / (double)K);
+  for (int64_t i = threadIdx.x; i < K; i += blockDim.x) H[i * K + i] += add;
+}
+
+__global__ void k_zero_dead_cols(float* __restrict__ W, int64_t N, int64_t K,
+                                 const int* __restrict__ dead) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < N * K;
+       i += (int64_t)gridDim.x * blockDim.x)
+    if (dead[i % K]) W[i] = 0.f;
+}
+
+// dst[i][j] = src[K-1-i][K-1-j]
+__global__ void k_reverse(const float* __restrict__ src, float* __restrict__ dst, int64_t K) {
+  const int64_t KK = K * K;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < KK;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = src[KK - 1 - i];
+}
+
+// Lower Cholesky factor of the 64 x 64 diagonal block at (k0, k0), in place
+// (lower triangle only).  A pivot that is not positive is recorded and
+// replaced by 1 so that nothing downstream turns into NaN.
+__global__ void __launch_bounds__(256) k_potrf64(float* __restrict__ A, int64_t K, int64_t k0,
+                                                 int* __restrict__ err) {
+  __shared__ float a[kNb][kNb + 1];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
+    const int r = e / kNb, c = e % kNb;
+    a[r][c] = c <= r ? A[(k0 + r) * K + k0 + c] : 0.f;
+  }
+  __syncthreads();
+  for (int c = 0; c < kNb; ++c) {
+    if (tid == 0) {
+      float d = a[c][c];
+      if (!(d > 0.f) || !isfinite(d)) {
+        atomicCAS(err, 0, DEV_ERR_NONFINITE);
+        d = 1.f;
+      }
+      a[c][c] = sqrtf(d);
+    }
+    __syncthreads();
+    const float piv = a[c][c];
+    for (int r = c + 1 + tid; r < kNb; r += blockDim.x) a[r][c] /= piv;
+    __syncthreads();
+    for (int e = tid; e < kNb * kNb; e += blockDim.x) {
+      const int r = e / kNb, s = e % kNb;
+      if (s > c && s <= r) a[r][s] -= a[r][c] * a[s][c];
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
+    const int r = e / kNb, c = e % kNb;
+    if (c <= r) A[(k0 + r) * K + k0 + c] = a[r][c];
+  }
+}
+
+// For each of `rows` vectors x (element c at X[r rs + c cs]) solve
+// x L^T = b in place, L the 64 x 64 lower triangle at L (leading dim ldl):
+// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector.
+__global__ void __launch_bounds__(64) k_trsm64(float* __restrict__ X, int64_t rows, int64_t rs,
+                                               int64_t cs, const float* __restrict__ L,
+                                               int64_t ldl) {
+  __shared__ float ls[kNb][kNb];
+  __shared__ float xs[kNb][64];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
+    const int r = e / kNb, c = e % kNb;
+    ls[r][c] = c <= r ? L[r * ldl + c] : 0.f;
+  }
+  const int64_t r = (int64_t)blockIdx.x * 64 + tid;
+  if (r < rows)
+    for (int c = 0; c < kNb; ++c) xs[c][tid] = X[r * rs + c * cs];
+  __syncthreads();
+  if (r >= rows) return;
+  for (int c = 0; c < kNb; ++c) {
+    float acc = xs[c][tid];
+    for (int s = 0; s < c; ++s) acc = fmaf(-xs[s][tid], ls[c][s], acc);
+    xs[c][tid] = acc / ls[c][c];
+  }
+  for (int c = 0; c < kNb; ++c) X[r * rs + c * cs] = xs[c][tid];
+}
+
+// C[m][n] -= sum_k A(m, k) B(k, n) with A(m, k) = A[m a_rs + k a_cs] and
+// B(k, n) = B[k b_rs + n b_cs]; C has leading dimension ldc.  64 x 64 tiles,
+// 16-deep K slices in shared memory, 4 x 4 outputs per thread.  With lower,
+// tiles wholly above the diagonal (n0 > m0 + 63) are skipped.
+struct SubGemm {
+  int64_t M, N, Kd;
+  const float* A;
+  int64_t a_rs, a_cs;
+  const float* B;
+  int64_t b_rs, b_cs;
+  float* C;
+  int64_t ldc;
+  int lower;
+};
+
+__global__ void __launch_bounds__(256) k_gemm_sub(const SubGemm g) {
+  __shared__ float as[16][64 + 4];
+  __shared__ float bs[16][64 + 4];
+  const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
+  if (g.lower && n0 > m0 + 63) return;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  float acc[4][4] = {};
+  for (int64_t k0 = 0; k0 < g.Kd; k0 += 16) {
+    for (int e = tid; e < 16 * 64; e += 256) {
+      const int kk = e / 64, mm = e % 64;
+      const int64_t m = m0 + mm, k = k0 + kk;
+      as[kk][mm] = (m < g.M && k < g.Kd) ? g.A[m * g.a_rs + k * g.a_cs] : 0.f;
+      const int64_t n = n0 + mm;
+      bs[kk][mm] = (n < g.N && k < g.Kd) ? g.B[k * g.b_rs + n * g.b_cs] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = as[kk][ty * 4 + i];
+        bv[i] = bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+      if (m < g.M && n < g.N) g.C[m * g.ldc + n] -= acc[i][j];
+    }
+}
+
+__global__ void k_unit_diag_block(float* __restrict__ M, int64_t K, int64_t r0) {
+  if (threadIdx.x < kNb) M[(r0 + threadIdx.x) * K + r0 + threadIdx.x] = 1.f;
+}
+
+// Nearest level of w / s (first level on ties; s = 0 gives w / s := 0), in fp32.
+template <int MODE>
+__device__ __forceinline__ int gptq_round(float w, float s) {
+  using Gr = GridT<MODE>;
+  const float q = s > 0.f ? w / s : 0.f;
+  int best = 0;
+  float bd = fabsf(q - Gr::level(0));
+#pragma unroll
+  for (int k = 1; k < Gr::LEVELS; ++k) {
+    const float d = fabsf(q - Gr::level(k));
+    if (d < bd) {
+      bd = d;
+      best = k;
+    }
+  }
+  return best;
+}
+
+// One block of 128 columns [j0, j0 + 128) for 128 rows per CTA (one thread
+// per row).  The block's rows of W and the 128 x 128 block of U sit in
+// shared memory (padded rows: conflict-free column access); the row's group
+// scale is set from the updated weights at the block start; every column is
+// rounded, its error fed forward inside the block; the levels go out through
+// shared memory with coalesced stores, the errors as E[j][n].
+constexpr int kColsSmem = 2 * kCols * (kCols + 1) * 4 + kCols * (kCols + 4);
+
+template <int MODE>
+__global__ void __launch_bounds__(kCols) k_gptq_cols(const float* __restrict__ W, int64_t N,
+                                                    int64_t K, const float* __restrict__ U,
+                                                    int64_t j0, int8_t* __restrict__ levels,
+                                                    float* __restrict__ scales,
+                                                    float* __restrict__ E) {
+  using Gr = GridT<MODE>;
+  extern __shared__ __align__(16) uint8_t gsm[];
+  float (*us)[kCols + 1] = reinterpret_cast<float (*)[kCols + 1]>(gsm);
+  float (*ws)[kCols + 1] = reinterpret_cast<float (*)[kCols + 1]>(gsm + kCols * (kCols + 1) * 4);
+  int8_t (*lv)[kCols + 4] = reinterpret_cast<int8_t (*)[kCols + 4]>(gsm + 2 * kCols * (kCols + 1) * 4);
+  const int tid = threadIdx.x;
+  const int64_t n0 = (int64_t)blockIdx.x * kCols;
+  for (int r = 0; r < kCols; ++r) {
+    us[r][tid] = tid >= r ? U[(j0 + r) * K + j0 + tid] : 0.f;
+    ws[tid][r] = n0 + r < N ? W[(n0 + r) * K + j0 + tid] : 0.f;
+  }
+  __syncthreads();
+  const int64_t n = n0 + tid;
+  if (n < N) {
+    float amax = 0.f;
+    for (int c = 0; c < kCols; ++c) amax = fmaxf(amax, fabsf(ws[c][tid]));
+    const float s = amax / Gr::CMAX;
+    scales[n * (K / kCols) + j0 / kCols] = s;
+    for (int j = 0; j < kCols; ++j) {
+      const float w = ws[j][tid];
+      const int lev = gptq_round<MODE>(w, s);
+      const float e = (w - s * Gr::level(lev)) / us[j][j];
+      lv[tid][j] = (int8_t)lev;
+      E[j * N + n] = e;
+      for (int c = j + 1; c < kCols; ++c) ws[c][tid] = fmaf(-e, us[j][c], ws[c][tid]);
+    }
+  }
+  __syncthreads();
+  for (int r = 0; r < kCols; ++r)
+    if (n0 + r < N) levels[(n0 + r) * K + j0 + tid] = lv[r][tid];
+}
+
+}  // namespace
+
+namespace {
+
+template <int MODE>
+cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_t* levels,
+                         float* scales, float* E, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gptq_cols<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kColsSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const unsigned rb = (unsigned)((N + kCols - 1) / kCols);
+  for (int64_t j0 = 0; j0 < K; j0 += kCols) {
+    k_gptq_cols<MODE><<<rb, kCols, kColsSmem, st>>>(W32, N, K, U, j0, levels, scales, E);
+    const int64_t j1 = j0 + kCols, rest = K - j1;
+    if (rest > 0) {
+      // W[:, j1:] -= E^T U[j0:j1, j1:]
+      const SubGemm g{N, rest, kCols, E, 1, N, U + j0 * K + j1, K, 1, W32 + j1, K, 0};
+      k_gemm_sub<<<dim3((unsigned)((rest + 63) / 64), (unsigned)((N + 63) / 64)), 256, 0, st>>>(g);
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// GPTQ on device inputs; levels (N x K int8) and scales (N x K/128 fp32) are
+// device buffers.  Allocates its workspace, synchronises the stream, frees.
+int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype, int64_t N,
+             int64_t K, int64_t T, float damp, int8_t* levels, float* scales, int sm_count,
+             cudaStream_t st) {
+  const int64_t Tp = (T + 63) / 64 * 64, NK = N * K, KK = K * K;
+  std::vector<void*> bufs;
+  bool oom = false;
+  auto alloc = [&](size_t bytes) -> void* {
+    void* p = nullptr;
+    if (oom || cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      oom = true;
+      return nullptr;
+    }
+    bufs.push_back(p);
+    return p;
+  };
+  float* W32 = (float*)alloc((size_t)NK * 4);
+  __nv_bfloat16* Wop = (__nv_bfloat16*)alloc((size_t)NK * 2);
+  __nv_bfloat16* Xb = (__nv_bfloat16*)alloc((size_t)Tp * K * 2);
+  __nv_bfloat16* Xt = (__nv_bfloat16*)alloc((size_t)K * Tp * 2);
+  float* B1 = (float*)alloc((size_t)KK * 4);
+  float* B2 = (float*)alloc((size_t)KK * 4);
+  int* dead = (int*)alloc((size_t)K * 4);
+  float* E = (float*)alloc((size_t)kCols * N * 4);
+  int* err = (int*)alloc(64);
+  double* partials = (double*)alloc(4096 * 8);
+  unsigned* ticket = (unsigned*)alloc(16);
+  auto finish = [&](int status) {
+    cudaStreamSynchronize(st);
+    cudaGetLastError();
+    for (void* p : bufs) cudaFree(p);
+    return status;
+  };
+  if (oom) return finish(GSQ_ERR_OOM);
+
+  cudaError_t e = cudaSuccess;
+  auto ok = [&](cudaError_t x) {
+    if (e == cudaSuccess) e = x;
+    return e == cudaSuccess;
+  };
+  ok(cudaMemsetAsync(err, 0, 64, st));
+  ok(cudaMemsetAsync(ticket, 0, 16, st));
+  ok(cudaMemsetAsync(Xt, 0, (size_t)K * Tp * 2, st));
+  ok(cudaMemsetAsync(Xb, 0, (size_t)Tp * K * 2, st));
+  ok(launch_convert_x(Xd, x_dtype, T, K, Tp, Xb, Xt, nullptr, err, st));
+  ok(launch_convert_w(Wd, w_dtype, N, K, W32, Wop, 0, err, st));
+
+  // H = Xt Xt^T (fp32) into B1
+  CUtensorMap ta, tb;
+  EpiMaps em;
+  if (make_tmap_bf16(&ta, Xt, K, Tp, Tp, kGemmBoxRowsA) ||
+      make_tmap_bf16(&tb, Xt, K, Tp, Tp, kGemmBoxRowsB) ||
+      make_tmap_epi_f32(&em.out, B1, K, K, K))
+    return finish(GSQ_ERR_CUDA);
+  em.yref = em.out;
+  EpiParams ep;
+  ep.partials = partials;
+  ep.ticket = ticket;
+  ep.loss_out = nullptr;
+  ep.err = err;
+  ok(launch_gemm(ta, tb, em, K, K, Tp, EPI_STORE_F32, ep, sm_count, st));
+  k_gptq_damp<<<1, 1024, 0, st>>>(B1, K, damp, dead);
+  k_zero_dead_cols<<<grid_cap(NK, 256, sm_count * 8), 256, 0, st>>>(W32, N, K, dead);
+  ok(cudaGetLastError());
+
+  // A = J H J into B2, lower Cholesky in place
+  const int rgrid = grid_cap(KK, 256, sm_count * 8);
+  k_reverse<<<rgrid, 256, 0, st>>>(B1, B2, K);
+  float* A = B2;
+  for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
+    k_potrf64<<<1, 256, 0, st>>>(A, K, k0, err);
+    const int64_t rest = K - k0 - kNb;
+    if (rest > 0) {
+      float* P = A + (k0 + kNb) * K + k0;
+      k_trsm64<<<(unsigned)((rest + 63) / 64), 64, 0, st>>>(P, rest, K, 1, A + k0 * K + k0, K);
+      const SubGemm g{rest, rest, kNb, P, K, 1, P, 1, K, P + kNb, K, 1};
+      const unsigned t = (unsigned)((rest + 63) / 64);
+      k_gemm_sub<<<dim3(t, t), 256, 0, st>>>(g);
+    }
+    ok(cudaGetLastError());
+  }
+  // M = L^-1 into B1 by block forward substitution
+  float* M = B1;
+  ok(cudaMemsetAsync(M, 0, (size_t)KK * 4, st));
+  for (int64_t r0 = 0; r0 < K && e == cudaSuccess; r0 += kNb) {
+    const int64_t c1 = r0 + kNb;
+    k_unit_diag_block<<<1, kNb, 0, st>>>(M, K, r0);
+    if (r0 > 0) {
+      const SubGemm g{kNb, c1, r0, A + r0 * K, K, 1, M, K, 1, M + r0 * K, K, 0};
+      k_gemm_sub<<<dim3((unsigned)((c1 + 63) / 64), 1), 256, 0, st>>>(g);
+    }
+    k_trsm64<<<(unsigned)((c1 + 63) / 64), 64, 0, st>>>(M + r0 * K, c1, 1, K, A + r0 * K + r0, K);
+    ok(cudaGetLastError());
+  }
+  // U = J M J into B2
+  k_reverse<<<rgrid, 256, 0, st>>>(M, B2, K);
+  ok(cudaGetLastError());
+  const float* U = B2;
+  if (e == cudaSuccess) {
+    switch (mode) {
+      case GRID_2BIT: ok(gptq_columns<GRID_2BIT>(W32, N, K, U, levels, scales, E, st)); break;
+      case GRID_TERNARY: ok(gptq_columns<GRID_TERNARY>(W32, N, K, U, levels, scales, E, st)); break;
+      default: ok(gptq_columns<GRID_3BIT_LOCAL>(W32, N, K, U, levels, scales, E, st));
+    }
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  int h = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess)
+    return finish(e == cudaErrorMemoryAllocation ? GSQ_ERR_OOM : GSQ_ERR_CUDA);
+  if (h == DEV_ERR_NONFINITE) return finish(GSQ_ERR_NONFINITE);
+  if (h == DEV_ERR_TIMEOUT) return finish(GSQ_ERR_TIMEOUT);
+  if (h != DEV_OK) return finish(GSQ_ERR_CUDA);
+  return finish(GSQ_OK);
+}
+
+}  // namespace gsq
+
+extern "C" {
+
+int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, int64_t K,
+             int64_t T, int group, int grid_mode, float damp, int8_t* levels, float* scales,
+             void* stream) {
+  using namespace gsq;
+  if (!W || !X || !levels || !scales || N <= 0 || K <= 0 || T <= 0 || group <= 0 ||
+      (w_dtype != GSQ_F32 && w_dtype != GSQ_BF16) ||
+      (x_dtype != GSQ_F32 && x_dtype != GSQ_BF16) || stage_num_logits(grid_mode) < 0 ||
+      K % group != 0 || !(damp >= 0.f) || !std::isfinite(damp) || N > ((int64_t)1 << 31) ||
+      T > ((int64_t)1 << 31) || K > 65536)
+    return GSQ_ERR_INVALID_ARG;
+  if (group != kStageGroup) return GSQ_ERR_UNSUPPORTED;
+  int dev = 0;
+  cudaDeviceProp prop;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GSQ_ERR_CUDA;
+  }
+  if (prop.major != 10) return GSQ_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t wbytes = (size_t)N * K * (w_dtype == GSQ_F32 ? 4 : 2);
+  const size_t xbytes = (size_t)T * K * (x_dtype == GSQ_F32 ? 4 : 2);
+  const size_t lbytes = (size_t)N * K, sbytes = (size_t)N * (K / group) * 4;
+  std::vector<void*> tmp;
+  auto dev_copy = [&](const void* p, size_t bytes, void** out) -> int {
+    if (stage_is_device_ptr(p)) {
+      *out = const_cast<void*>(p);
+      return GSQ_OK;
+    }
+    if (cudaMalloc(out, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return GSQ_ERR_OOM;
+    }
+    tmp.push_back(*out);
+    return GSQ_OK;
+  };
+  void *Wd = nullptr, *Xd = nullptr, *Ld = nullptr, *Sd = nullptr;
+  int rc = dev_copy(W, wbytes, &Wd);
+  if (!rc) rc = dev_copy(X, xbytes, &Xd);
+  if (!rc) rc = dev_copy(levels, lbytes, &Ld);
+  if (!rc) rc = dev_copy(scales, sbytes, &Sd);
+  cudaError_t e = cudaSuccess;
+  if (!rc && Wd != W) e = cudaMemcpyAsync(Wd, W, wbytes, cudaMemcpyDefault, st);
+  if (!rc && e == cudaSuccess && Xd != X) e = cudaMemcpyAsync(Xd, X, xbytes, cudaMemcpyDefault, st);
+  if (!rc && e != cudaSuccess) rc = GSQ_ERR_CUDA;
+  if (!rc)
+    rc = gptq_run(grid_mode, Wd, w_dtype, Xd, x_dtype, N, K, T, damp, (int8_t*)Ld, (float*)Sd,
+                  prop.multiProcessorCount, st);
+  if (!rc && Ld != levels &&
+      cudaMemcpy(levels, Ld, lbytes, cudaMemcpyDeviceToHost) != cudaSuccess)
+    rc = GSQ_ERR_CUDA;
+  if (!rc && Sd != scales &&
+      cudaMemcpy(scales, Sd, sbytes, cudaMemcpyDeviceToHost) != cudaSuccess)
+    rc = GSQ_ERR_CUDA;
+  cudaStreamSynchronize(st);
+  cudaGetLastError();
+  for (void* p : tmp) cudaFree(p);
+  return rc;
+}
+
+}  // extern "C"

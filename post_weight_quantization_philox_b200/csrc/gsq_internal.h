@@ -106,6 +106,13 @@ cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 int64_t Kc, int bn, const GemmSched& sc, int mode,
                                 const EpiParams& ep, int sm_count, cudaStream_t st);
 
+// GPTQ initial assignment (gsq_gptq.cu) on device inputs: levels (N x K
+// int8 level indices) and scales (N x K/128) into device buffers; returns a
+// GSQ status and leaves the stream synchronised.
+int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype, int64_t N,
+             int64_t K, int64_t T, float damp, int8_t* levels, float* scales, int sm_count,
+             cudaStream_t st);
+
 // ------------------------------------------------------- elementwise
 struct StepArgs {
   int mode;

@@ -44,6 +44,7 @@ EXPORTS = [
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
+    "gsq_gptq", "gsq_init_gptq",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
@@ -89,6 +90,8 @@ _SIGS = {
     "gsq_debug_weight_grad": [_p],
     "gsq_debug_backward": [_p, _f32, _f32, _f32, _f32],
     "gsq_scale_step": [_p, _f32, _f32, _f32],
+    "gsq_gptq": [_p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _p, _p, _p],
+    "gsq_init_gptq": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _u64, _p],
     "gsq_scale_run": [_p, _i64, _f32, _f32, _f32],
     "gsq_debug_scale_backward": [_p, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
@@ -220,6 +223,41 @@ def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
                          grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
            "gsq_init")
     del wk, xk, ik
+    return Layer(ctx, grid_mode, N, K, T, group)
+
+
+def gsq_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT, damp: float = 0.01,
+             stream=None):
+    """GPTQ initial levels (N x K int8) and group scales (N x K/group fp32),
+    returned as host numpy arrays.  W, X as for gsq_init."""
+    wp, wdt, wk = _ptr_dtype(W)
+    xp, xdt, xk = _ptr_dtype(X)
+    N, K = int(W.shape[0]), int(W.shape[1])
+    T = int(X.shape[0])
+    if int(X.shape[1]) != K:
+        raise ValueError("X and W disagree on K")
+    lev = np.zeros((N, K), np.int8)
+    sc = np.zeros((N, K // group), np.float32)
+    _check(_lib.gsq_gptq(wp, wdt, xp, xdt, N, K, T, group, grid_mode, damp,
+                         lev.ctypes.data, sc.ctypes.data, _stream_ptr(stream)), "gsq_gptq")
+    del wk, xk
+    return lev, sc
+
+
+def gsq_init_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
+                  damp: float = 0.01, seed: int = 0, stream=None) -> "Layer":
+    """gsq_init with the GPTQ levels and scales as the starting point."""
+    wp, wdt, wk = _ptr_dtype(W)
+    xp, xdt, xk = _ptr_dtype(X)
+    N, K = int(W.shape[0]), int(W.shape[1])
+    T = int(X.shape[0])
+    if int(X.shape[1]) != K:
+        raise ValueError("X and W disagree on K")
+    ctx = C.c_void_p()
+    _check(_lib.gsq_init_gptq(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group, grid_mode,
+                              damp, seed & 0xFFFFFFFFFFFFFFFF, _stream_ptr(stream)),
+           "gsq_init_gptq")
+    del wk, xk
     return Layer(ctx, grid_mode, N, K, T, group)
 
 

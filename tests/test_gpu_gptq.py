@@ -1,0 +1,157 @@
+"""Parity of the GPU GPTQ initial assignment (gsq_gptq, gsq_init_gptq) with
+the oracle's fp64 GPTQ.  Needs a B200.
+
+GPTQ is sequential: each column's rounding decision moves the later columns,
+so an fp32 decision that lands on the other side of a rounding tie than the
+fp64 one sends the rest of the row down another, equally valid, greedy
+branch.  Parity is therefore: the share of identical levels; the GPTQ
+objective (W - Q) H (W - Q)^T of every row within 2% of the oracle's, except
+rows whose first differing column is a tie in the oracle's own trajectory
+(checked by replaying the oracle up to that column), which must be rare.
+Where no error is fed forward (a diagonal Hessian) the result is
+round-to-nearest and must be bit-exact."""
+import numpy as np
+import pytest
+
+from post_weight_quantization_philox_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    return gsq
+
+
+def correlated(T, K, seed, outliers=0):
+    rng = np.random.default_rng(seed)
+    X = rng.normal(0, 1, (T, K // 8)) @ rng.normal(0, 1, (K // 8, K))
+    X += 0.3 * rng.normal(0, 1, (T, K))
+    if outliers:
+        X[:, rng.permutation(K)[:outliers]] *= 10.0
+    return synth.bf16_values(X)
+
+
+def objective(oracle_mod, mode, W, lev, s, H):
+    Q = oracle_mod.gptq.quantized(mode, lev, s)
+    D = Q - W.astype(np.float64)
+    return np.einsum("nk,kl,nl->n", D, H, D)
+
+
+def tie_at_first_difference(oracle_mod, mode, w_row, X, lev_row, ref_row):
+    """True when the first column where the GPU and the oracle chose different
+    levels is a rounding tie in the oracle's own trajectory (w / s within 1e-4
+    of a midpoint between two levels): both choices are then valid GPTQ
+    results and the greedy loop continues on different branches."""
+    G = oracle_mod.gptq
+    j = int(np.argmax(lev_row != ref_row))
+    _, s, _, Wa, _ = G.gptq(mode, w_row[None, :], X, cols=j)
+    w = Wa[0, j]
+    if j % 128 == 0:  # the group's scale is set when its first column is reached
+        sc = np.float32(np.abs(Wa[0, j:j + 128]).max()) / np.float32(G.LEVELS[mode].max())
+    else:
+        sc = s[0, j // 128]
+    mids = (G.LEVELS[mode][1:] + G.LEVELS[mode][:-1]) / 2
+    return np.min(np.abs(w / float(sc) - mids)) < 1e-4
+
+
+def check_rows(oracle_mod, mode, W, X, lev, s, rl, rs, H, max_ties):
+    ours = objective(oracle_mod, mode, W, lev, s, H)
+    ref = objective(oracle_mod, mode, W, rl, rs, H)
+    off = np.nonzero(np.abs(ours - ref) > 0.02 * ref)[0]
+    for i in off:
+        assert tie_at_first_difference(oracle_mod, mode, W[i], X, lev[i], rl[i]), i
+    assert len(off) <= max_ties, off
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_gptq_matches_oracle(g, oracle_mod, mode):
+    N, K, T = 192, 512, 640
+    X = correlated(T, K, 1 + mode, outliers=5)
+    W = np.random.default_rng(11 + mode).normal(0, 0.02, (N, K)).astype(np.float32)
+    lev, s = g.gsq_gptq(W, X, grid_mode=mode)
+    rl, rs, _, _, H = oracle_mod.gptq.gptq(mode, W, X)
+    assert (lev == rl).mean() > 0.97
+    check_rows(oracle_mod, mode, W, X, lev, s, rl, rs, H, max_ties=N // 50 + 1)
+    # the first group's scale sees no fed-forward error before it
+    assert np.allclose(s[:, 0], rs[:, 0], rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("mode", [0, 2])
+def test_diagonal_hessian_is_the_round_to_nearest_init(g, mode):
+    """Orthogonal input columns: GPTQ feeds nothing forward, so it must give
+    the same levels and scales as gsq_init's round-to-nearest, bit for bit."""
+    K = 256
+    h = np.array([[1.0]])
+    while h.shape[0] < K:
+        h = np.block([[h, h], [h, -h]])
+    X = (h * 0.5).astype(np.float32)
+    W = np.random.default_rng(3).normal(0, 0.02, (128, K)).astype(np.float32)
+    lev, s = g.gsq_gptq(W, X, grid_mode=mode)
+    lay = g.gsq_init(W, X, 128, mode)
+    assert np.array_equal(s, lay.get(g.GSQ_DBG_SCALES))
+    if mode == 2:
+        ref = lay.get(g.GSQ_DBG_I0)
+    else:
+        ref = np.argmax(lay.get(g.GSQ_DBG_LOGITS), axis=0)
+    assert np.array_equal(lev.astype(np.int64), ref.astype(np.int64))
+    lay.close()
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_init_gptq_context(g, oracle_mod, mode):
+    """The context starts from the GPTQ levels and scales, and its initial hard
+    reconstruction error is below that of the round-to-nearest start."""
+    N, K, T = 256, 512, 512
+    X = correlated(T, K, 7)
+    W = np.random.default_rng(8).normal(0, 0.02, (N, K)).astype(np.float32)
+    lev, s = g.gsq_gptq(W, X, grid_mode=mode)
+    a = g.gsq_init_gptq(W, X, grid_mode=mode, seed=1)
+    b = g.gsq_init(W, X, 128, mode, seed=1)
+    assert np.array_equal(a.get(g.GSQ_DBG_SCALES), s)
+    if mode == 2:
+        assert np.array_equal(a.get(g.GSQ_DBG_I0), lev)
+    elif mode == 0:
+        assert np.array_equal(np.argmax(a.get(g.GSQ_DBG_LOGITS), axis=0), lev)
+    ra = g.gsq_recon_error(a, g.GSQ_RECON_HARD)[1]
+    rb = g.gsq_recon_error(b, g.GSQ_RECON_HARD)[1]
+    assert ra < 0.9 * rb
+    for tau in synth.tau_schedule(1.0, 0.1, 5):
+        a.step(float(tau), 1e-3)
+    assert np.isfinite(a.last_loss())
+    a.close(); b.close()
+
+
+def test_dead_inputs_and_bad_arguments(g):
+    K = 256
+    X = correlated(300, K, 9)
+    X[:, [1, 200]] = 0.0
+    W = np.random.default_rng(10).normal(0, 0.02, (64, K)).astype(np.float32)
+    lev, s = g.gsq_gptq(W, X)
+    assert np.all(np.isfinite(s)) and lev.min() >= 0 and lev.max() <= 3
+    with pytest.raises(g.GSQError):
+        g.gsq_gptq(W, X, damp=-1.0)
+    with pytest.raises(g.GSQError):
+        g.gsq_gptq(W, X, group=64)
+    with pytest.raises(g.GSQError):
+        g.gsq_gptq(W[:, :200], X[:, :200])
+
+
+def test_full_size_q_proj_row_slices(g, oracle_mod):
+    """The q_proj-shaped layer (4096 x 4096, T 4096): GPU GPTQ on the whole
+    layer, the oracle on a few rows (rows are independent given H)."""
+    import torch
+    cfg = synth.CONFIGS["c2_qproj_4096x4096"]
+    W, X = synth.make_weight(cfg), synth.make_calib(cfg)
+    lev, s = g.gsq_gptq(torch.from_numpy(W).cuda().to(torch.bfloat16),
+                        torch.from_numpy(X).cuda().to(torch.bfloat16), grid_mode=0)
+    rows = [0, 1, 2049, 4095]
+    rl, rs, _, _, H = oracle_mod.gptq.gptq(0, W[rows], X)
+    assert (lev[rows] == rl).mean() > 0.97
+    check_rows(oracle_mod, 0, W[rows], X, lev[rows], s[rows], rl, rs, H, max_ties=1)
