@@ -502,6 +502,78 @@ def run_scale_stage(args, rank, world, local_rank):
             "gpu_launches": int(args.steps * 4), "clocks": clk, "last_loss": loss}
 
 
+def gptq_simt_flops(N: int, K: int) -> float:
+    """fp32 SIMT flops of one GPTQ call: Cholesky of the damped K x K
+    Hessian (K^3 / 3), inverse of its triangular factor (K^3 / 3), the
+    trailing-column error updates (N K^2 in total) and the in-group feedback
+    (N K 128)."""
+    return 2.0 * K ** 3 / 3.0 + float(N) * K * K + float(N) * K * 128
+
+
+def run_gptq_stage(args, rank, world, local_rank):
+    """GPTQ initial assignment (Hessian, Cholesky, inverse, column-wise error
+    feedback) of the --config layer, device inputs and outputs."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    cfg = synth.CONFIGS[args.config]
+    W = torch.from_numpy(synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank))
+    X = torch.from_numpy(synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank))
+    dt = torch.bfloat16 if cfg.w_bf16 else torch.float32
+    W, X = W.to(dt).cuda(), X.to(dt).cuda()
+    lev = torch.empty((cfg.N, cfg.K), dtype=torch.int8, device="cuda")
+    sc = torch.empty((cfg.N, cfg.K // 128), dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        gsq.gsq_gptq(W, X, 128, cfg.grid, levels=lev, scales=sc)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        gsq.gsq_gptq(W, X, 128, cfg.grid, levels=lev, scales=sc)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    per = ms / args.steps
+    props = torch.cuda.get_device_properties(local_rank)
+    sm_mhz = clk.get("sm_mhz") or 1965.0
+    # fp32 FMA peak: 128 lanes per SM, 2 flops per FMA, at the sampled clock
+    alu_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    flops = gptq_simt_flops(cfg.N, cfg.K)
+    ach = flops / (per / 1e3) / 1e12
+    coords = cfg.N * cfg.K
+    return {"metric": METRIC, "value": world * coords / (per / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
+            "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp32 (Hessian: bf16 operands, fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": cfg.name + "_gptq_init", "N": cfg.N, "K": cfg.K,
+                       "T": cfg.T, "grid": ["2bit", "ternary", "3bit_local"][cfg.grid],
+                       "step": "one GPTQ call (workspace allocated and freed inside)"},
+            "roofline": {"bound": "alu", "kernel": "whole GPTQ call (SIMT fp32 flops)",
+                         "achieved": round(ach, 2), "peak": round(alu_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(ach / alu_peak, 4),
+                         "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x sampled SM clock",
+                         "traffic": None},
+            "clocks": clk}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -535,7 +607,7 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale"],
+    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq"],
                     help="time a block stage instead of a single layer")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
@@ -564,6 +636,8 @@ def main():
         out = run_attn_stage(args, rank, world, local_rank)
     elif args.stage == "scale":
         out = run_scale_stage(args, rank, world, local_rank)
+    elif args.stage == "gptq":
+        out = run_gptq_stage(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:

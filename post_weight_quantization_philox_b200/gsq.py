@@ -227,21 +227,29 @@ def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
 
 
 def gsq_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT, damp: float = 0.01,
-             stream=None):
-    """GPTQ initial levels (N x K int8) and group scales (N x K/group fp32),
-    returned as host numpy arrays.  W, X as for gsq_init."""
+             stream=None, levels=None, scales=None):
+    """GPTQ initial levels (N x K int8) and group scales (N x K/group fp32).
+    W, X as for gsq_init.  Returned as host numpy arrays, or written into
+    `levels` / `scales` (contiguous int8 / fp32 torch tensors or numpy arrays
+    of those shapes, host or device) when both are given."""
     wp, wdt, wk = _ptr_dtype(W)
     xp, xdt, xk = _ptr_dtype(X)
     N, K = int(W.shape[0]), int(W.shape[1])
     T = int(X.shape[0])
     if int(X.shape[1]) != K:
         raise ValueError("X and W disagree on K")
-    lev = np.zeros((N, K), np.int8)
-    sc = np.zeros((N, K // group), np.float32)
+    if (levels is None) != (scales is None):
+        raise ValueError("give both levels and scales, or neither")
+    if levels is None:
+        levels = np.zeros((N, K), np.int8)
+        scales = np.zeros((N, K // group), np.float32)
+    if tuple(levels.shape) != (N, K) or tuple(scales.shape) != (N, K // group):
+        raise ValueError("levels / scales have the wrong shape")
     _check(_lib.gsq_gptq(wp, wdt, xp, xdt, N, K, T, group, grid_mode, damp,
-                         lev.ctypes.data, sc.ctypes.data, _stream_ptr(stream)), "gsq_gptq")
+                         _host_ptr(levels), _host_ptr(scales), _stream_ptr(stream)),
+           "gsq_gptq")
     del wk, xk
-    return lev, sc
+    return levels, scales
 
 
 def gsq_init_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
