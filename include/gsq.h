@@ -380,6 +380,79 @@ GSQ_API int gsq_attn_debug_set(gsq_attn* ctx, int which, int buf,
 GSQ_API int gsq_attn_get_step(gsq_attn* ctx, uint64_t* t);
 GSQ_API int gsq_attn_destroy(gsq_attn* ctx);
 
+/* ------------------------------------------- staged block pipeline ------
+ * GSQ quantizes the blocks of a model one after another: every block is
+ * reconstructed from the output of the already quantized blocks before it,
+ * and inside a block the query and key projections come first (each on its
+ * own output), then the value and output projections together, then the MLP
+ * on the block output (agihunt.info summary, optimisation paragraph).
+ *
+ * The block is a pre-norm Llama block on an fp32 residual stream x (T x H,
+ * T = n_seq seq_len tokens, H = n_heads head_dim):
+ *   xa = bf16(RMSNorm(x)),  h = x + Attn(xa),  xm = bf16(RMSNorm(h)),
+ *   y  = h + bf16(silu(xm Wg^T) * (xm Wu^T)) Wd^T,
+ * RMSNorm(v) = v / sqrt(mean(v^2) + rms_eps) (unit gain); Attn as in
+ * gsq_attn_* (rotate-half rotary embedding with rope_theta, causal softmax of
+ * Q K^T / sqrt(d), grouped key/value heads), then the output projection.
+ * GEMMs take bf16 operands with fp32 accumulation; V, the attention output o
+ * and silu(a) b are rounded to bf16 as GEMM operands.
+ *
+ * Weights W[7] in the order query (H x H), key (Hk x H), value (Hk x H),
+ * output (H x H), gate (ffn x H), up (ffn x H), down (H x ffn), Hk =
+ * n_kv_heads head_dim; bf16, row-major, host or device, read only.
+ * head_dim must be 128, seq_len a multiple of 128 (at most 65536), ffn a
+ * multiple of 128, n_heads a multiple of n_kv_heads.
+ *
+ * gsq_dequant -- the bf16 weight of a packed code stream (the output of
+ *   gsq_harden_pack): W[n][k] = bf16(scales_f32[n][k / 128] c(code)) with c
+ *   the grid's unit level of the code (2-bit code - 1.5, ternary code - 1,
+ *   3-bit code - 3.5).  packed: gsq_packed_bytes bytes; scales_f32: N x K/128;
+ *   W_bf16: N x K; each host or device.  Syncs.
+ *
+ * gsq_block_forward -- y (and h, nullable) of the block above for input x
+ *   (T x H fp32, host or device) and weights W[7]; outputs T x H fp32, host
+ *   or device.  Allocates its own scratch.  Syncs.
+ *
+ * gsq_block_quantize -- GSQ's staged reconstruction of one block:
+ *   1. the full-precision block on x_in: the attention output attn_fp and y_fp;
+ *   2. stage 0 (query) and stage 1 (key): a gsq_init context on xa with the
+ *      full-precision weight's own output as target, gsq_run over taus[j];
+ *   3. stage 2: gsq_attn_* with the probabilities of the quantized query and
+ *      key weights, target attn_fp, over taus[2];
+ *   4. h_q = x_in + Attn_q(xa); stage 3: gsq_mlp_* on bf16(RMSNorm(h_q))
+ *      with target y_fp - h_q (the MLP is trained on the block output), over
+ *      taus[3];
+ *   5. x_out = h_q + MLP_q(bf16(RMSNorm(h_q))), the next block's input.
+ *   Each stage's weights are hardened (argmax, packed, dequantized) before
+ *   the next stage uses them.  Stage j draws its noise with Philox key
+ *   seed ^ (j << 56) (joint stages further ^ (i << 48) for weight i).
+ *   taus[j]: n_steps[j] temperatures (host arrays; n_steps[j] >= 0);
+ *   lr, beta1, beta2 as gsq_step.  Outputs: x_out (T x H fp32, host or
+ *   device); per weight i (arrays and entries nullable) packed[i]
+ *   (gsq_packed_bytes bytes), scales_f16[i] / scales_f32[i] (rows x cols/128);
+ *   stats (nullable, 4 x 5 doubles): per stage the first and the last step's
+ *   loss, the final hard reconstruction error (abs, rel) and the milliseconds
+ *   of its steps (CUDA events).  Every context and scratch buffer is freed
+ *   before the call returns.  Syncs.
+ * Errors: GSQ_ERR_INVALID_ARG, GSQ_ERR_UNSUPPORTED (shape limits above,
+ * group != 128), GSQ_ERR_OOM, GSQ_ERR_NONFINITE, GSQ_ERR_TIMEOUT,
+ * GSQ_ERR_CUDA, or a stage's own status.
+ */
+GSQ_API int gsq_dequant(int grid_mode, const void* packed, const float* scales_f32, int64_t N,
+                        int64_t K, int group, void* W_bf16, void* stream);
+GSQ_API int gsq_block_forward(const float* x, const void* const* W, int64_t n_seq,
+                              int64_t seq_len, int64_t n_heads, int64_t n_kv_heads,
+                              int64_t head_dim, int64_t ffn, double rope_theta,
+                              float rms_eps, float* h_out, float* y_out, void* stream);
+GSQ_API int gsq_block_quantize(const float* x_in, const void* const* W, int64_t n_seq,
+                               int64_t seq_len, int64_t n_heads, int64_t n_kv_heads,
+                               int64_t head_dim, int64_t ffn, double rope_theta,
+                               float rms_eps, int group, int grid_mode,
+                               const float* const* taus, const int64_t* n_steps, float lr,
+                               float beta1, float beta2, uint64_t seed, float* x_out,
+                               void* const* packed, uint16_t* const* scales_f16,
+                               float* const* scales_f32, double* stats, void* stream);
+
 /*
  * gsq_uniforms_noalloc -- the L Philox uniforms of coords
  * [coord0, coord0 + count) at step t for grid_mode and seed (the values

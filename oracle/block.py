@@ -130,6 +130,34 @@ def block_forward(x, W: dict, dm: BlockDims, theta=ROPE_THETA, eps=RMS_EPS,
     return {"xa": xa, "attn": attn, "h": h, "xm": xm, "mlp": mlp, "y": h + mlp}
 
 
+def block_forward_rows(x, W: dict, dm: BlockDims, s: int, positions, theta=ROPE_THETA,
+                       eps=RMS_EPS, round_bf16=True) -> np.ndarray:
+    """y of the block at `positions` of sequence s, computed from rows
+    0..max(positions) of that sequence only (causal attention needs nothing
+    later): for checking samples of layers too large for block_forward."""
+    from . import attn_prob_row
+    positions = list(positions)
+    last = max(positions) + 1
+    rows = np.asarray(x[s * dm.S:s * dm.S + last], np.float64)
+    xa = _r(rmsnorm(rows, eps), round_bf16)
+    V = _r(xa @ np.asarray(W["v"], np.float64).T, round_bf16)
+    grp = dm.nh // dm.nkv
+    xa32 = np.ascontiguousarray(xa, np.float32)
+    o = np.zeros((len(positions), dm.H))
+    for i, p in enumerate(positions):
+        for h in range(dm.nh):
+            g = h // grp
+            # the probability row of query p only needs keys 0..p of this sequence
+            prow = attn_prob_row(xa32, W["q"], W["k"], 1, last, dm.nh, dm.nkv, 0, h, p, dm.d,
+                                 theta, round_bf16)
+            o[i, h * dm.d:(h + 1) * dm.d] = (prow[:p + 1].astype(np.float64)
+                                             @ V[:p + 1, g * dm.d:(g + 1) * dm.d])
+    o = _r(o, round_bf16)
+    hrows = rows[positions] + o @ np.asarray(W["o"], np.float64).T
+    xm = _r(rmsnorm(hrows, eps), round_bf16)
+    return hrows + mlp_out(xm, W["gate"], W["up"], W["down"], round_bf16)
+
+
 LEVEL_VALUES = {GRID_2BIT: np.array([-1.5, -0.5, 0.5, 1.5]),
                 GRID_TERNARY: np.array([-1.0, 0.0, 1.0]),
                 2: np.arange(8) - 3.5}

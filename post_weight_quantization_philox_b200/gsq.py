@@ -51,6 +51,7 @@ EXPORTS = [
     "gsq_attn_init", "gsq_attn_step", "gsq_attn_run", "gsq_attn_last_loss",
     "gsq_attn_recon_error", "gsq_attn_harden_pack", "gsq_attn_debug_get",
     "gsq_attn_debug_set", "gsq_attn_get_step", "gsq_attn_destroy",
+    "gsq_dequant", "gsq_block_forward", "gsq_block_quantize",
 ]
 
 
@@ -118,6 +119,12 @@ _SIGS = {
     "gsq_attn_debug_set": [_p, _i32, _i32, _p, _sz],
     "gsq_attn_get_step": [_p, C.POINTER(_u64)],
     "gsq_attn_destroy": [_p],
+    "gsq_dequant": [_i32, _p, _p, _i64, _i64, _i32, _p, _p],
+    "gsq_block_forward": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, C.c_double, _f32,
+                          _p, _p, _p],
+    "gsq_block_quantize": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, C.c_double, _f32,
+                           _i32, _i32, _p, _p, _f32, _f32, _f32, _u64, _p, _p, _p, _p, _p,
+                           _p],
 }
 
 
@@ -673,3 +680,125 @@ class Attn:
                 self.ctx = None
         except Exception:
             pass
+
+
+# ------------------------------------------------------ staged block pipeline
+
+BLOCK_WEIGHTS = ("q", "k", "v", "o", "gate", "up", "down")
+BLOCK_STAGES = ("q", "k", "vo", "mlp")
+
+
+def block_weight_shapes(n_heads, n_kv_heads, head_dim, ffn):
+    H, Hk = n_heads * head_dim, n_kv_heads * head_dim
+    return {"q": (H, H), "k": (Hk, H), "v": (Hk, H), "o": (H, H),
+            "gate": (ffn, H), "up": (ffn, H), "down": (H, ffn)}
+
+
+def _block_shapes_ok(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn):
+    """The C entry points see raw pointers: check every extent here."""
+    shapes = block_weight_shapes(n_heads, n_kv_heads, head_dim, ffn)
+    if tuple(x.shape) != (n_seq * seq_len, n_heads * head_dim):
+        raise ValueError(f"x has shape {tuple(x.shape)}, expected "
+                         f"{(n_seq * seq_len, n_heads * head_dim)}")
+    for name in BLOCK_WEIGHTS:
+        if tuple(W[name].shape) != shapes[name]:
+            raise ValueError(f"weight {name} has shape {tuple(W[name].shape)}, "
+                             f"expected {shapes[name]}")
+
+
+def _bf16_weights(W):
+    """Keep-alive list and a C array of the seven bf16 weight pointers."""
+    import torch
+    keep = []
+    for name in BLOCK_WEIGHTS:
+        w = W[name]
+        if not isinstance(w, torch.Tensor):
+            w = torch.from_numpy(np.ascontiguousarray(w, np.float32))
+        w = w.to(torch.bfloat16).contiguous()
+        keep.append(w)
+    arr = (C.c_void_p * 7)(*[w.data_ptr() for w in keep])
+    return keep, arr
+
+
+def _f32_tensor(x):
+    import torch
+    if not isinstance(x, torch.Tensor):
+        x = torch.from_numpy(np.ascontiguousarray(x, np.float32))
+    return x.to(torch.float32).contiguous()
+
+
+def gsq_dequant(grid_mode, packed, scales_f32, N, K, group=128, out=None, stream=None):
+    """bf16 weight (N x K) of a packed code stream and its fp32 group scales.
+    Returns `out` (a torch bf16 tensor, host or device) or a new device tensor."""
+    import torch
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    if (tuple(out.shape) != (N, K) or out.dtype != torch.bfloat16
+            or int(np.prod(scales_f32.shape)) != N * (K // group)
+            or int(packed.nbytes if hasattr(packed, "nbytes") else
+                   packed.numel() * packed.element_size()) != gsq_packed_bytes(grid_mode, N, K)):
+        raise ValueError("gsq_dequant: buffer sizes do not match N x K")
+    _check(_lib.gsq_dequant(grid_mode, _host_ptr(packed), _host_ptr(scales_f32), N, K, group,
+                            out.data_ptr(), _stream_ptr(stream)), "gsq_dequant")
+    return out
+
+
+def gsq_block_forward(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn,
+                      rope_theta=500000.0, rms_eps=1e-5, stream=None):
+    """(h, y) of the pre-norm block on the fp32 residual stream x (T x H) with
+    bf16 weights W (dict of the seven projections); device tensors."""
+    import torch
+    x = _f32_tensor(x)
+    _block_shapes_ok(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn)
+    keep, arr = _bf16_weights(W)
+    T, H = int(x.shape[0]), int(x.shape[1])
+    dev = x.device if x.is_cuda else torch.device("cuda")
+    h = torch.empty((T, H), dtype=torch.float32, device=dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+    _check(_lib.gsq_block_forward(x.data_ptr(), arr, n_seq, seq_len, n_heads, n_kv_heads,
+                                  head_dim, ffn, rope_theta, rms_eps, h.data_ptr(),
+                                  y.data_ptr(), _stream_ptr(stream)), "gsq_block_forward")
+    del keep
+    return h, y
+
+
+def gsq_block_quantize(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn, taus,
+                       lr, beta1=0.9, beta2=0.99, seed=0, grid_mode=GSQ_GRID_2BIT,
+                       group=128, rope_theta=500000.0, rms_eps=1e-5, stream=None):
+    """GSQ's staged reconstruction of one block (Q, K, then V/O, then the MLP
+    on the block output).  taus: four temperature schedules (one per stage).
+    Returns a dict: x_out (device fp32, the next block's input), packed and
+    scales_f32 per weight (device tensors), stats per stage (first loss, last
+    loss, hard abs / rel error, ms)."""
+    import torch
+    x = _f32_tensor(x)
+    _block_shapes_ok(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn)
+    keep, arr = _bf16_weights(W)
+    T, H = int(x.shape[0]), int(x.shape[1])
+    dev = x.device if x.is_cuda else torch.device("cuda")
+    shapes = block_weight_shapes(n_heads, n_kv_heads, head_dim, ffn)
+    x_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    packed, scales = {}, {}
+    for name in BLOCK_WEIGHTS:
+        N, K = shapes[name]
+        packed[name] = torch.empty(gsq_packed_bytes(grid_mode, N, K) // 4, dtype=torch.int32,
+                                   device=dev)
+        scales[name] = torch.empty((N, K // group), dtype=torch.float32, device=dev)
+    tau_arr = [np.ascontiguousarray(t, np.float32) for t in taus]
+    if len(tau_arr) != 4:
+        raise ValueError("taus: one schedule per stage (4)")
+    tp = (C.c_void_p * 4)(*[t.ctypes.data if t.size else None for t in tau_arr])
+    ns = (C.c_int64 * 4)(*[int(t.size) for t in tau_arr])
+    pk = (C.c_void_p * 7)(*[packed[n].data_ptr() for n in BLOCK_WEIGHTS])
+    sc = (C.c_void_p * 7)(*[scales[n].data_ptr() for n in BLOCK_WEIGHTS])
+    stats = np.zeros(20, np.float64)
+    _check(_lib.gsq_block_quantize(x.data_ptr(), arr, n_seq, seq_len, n_heads, n_kv_heads,
+                                   head_dim, ffn, rope_theta, rms_eps, group, grid_mode, tp,
+                                   ns, lr, beta1, beta2, seed & 0xFFFFFFFFFFFFFFFF,
+                                   x_out.data_ptr(), pk, None, sc, stats.ctypes.data,
+                                   _stream_ptr(stream)), "gsq_block_quantize")
+    del keep, tau_arr
+    st = {name: dict(first_loss=stats[5 * j], last_loss=stats[5 * j + 1],
+                     recon=(stats[5 * j + 2], stats[5 * j + 3]), ms=stats[5 * j + 4])
+          for j, name in enumerate(BLOCK_STAGES)}
+    return {"x_out": x_out, "packed": packed, "scales": scales, "stats": st}

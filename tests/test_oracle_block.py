@@ -7,6 +7,8 @@ output (agihunt.info summary, optimisation paragraph).  CPU only.
   rotation for the rotary embedding, torch's scaled-dot-product attention
   with a causal mask, grouped heads by repetition);
 * causality and independence of sequences, exactly;
+* output rows computed alone (for sampled checks of large layers) equal the
+  rows of the full forward;
 * weights already on the grid with lr = 0: every stage ends with zero hard
   error and the quantized block reproduces the full-precision block;
 * the V/O stage's hard loss equals the error of the quantized attention
@@ -108,6 +110,16 @@ def pin_causal_and_sequences_independent(B):
     assert not np.array_equal(y[dm.S + 3:], y3[dm.S + 3:])
 
 
+def pin_rows_alone_equal_full_forward(B):
+    dm = B.BlockDims(**SMALL)
+    W = weights(B, dm, 12, scale=0.2)
+    x = np.random.default_rng(13).normal(0, 1, (dm.T, dm.H))
+    y = B.block_forward(x, W, dm)["y"]
+    for s, pos in ((0, [0, 3]), (1, [7, 2, 5])):
+        rows = B.block_forward_rows(x, W, dm, s, pos)
+        assert np.allclose(rows, y[[s * dm.S + p for p in pos]], rtol=0, atol=1e-12), (s, pos)
+
+
 def on_grid_weights(B, dm, seed):
     """Weights on the 2-bit grid with scale 2^-6 and a +-1.5 level in every
     group, so round-to-nearest from absmax / 1.5 recovers them exactly."""
@@ -188,6 +200,10 @@ def test_causal_and_sequences_independent(B):
     pin_causal_and_sequences_independent(B)
 
 
+def test_rows_computed_alone_equal_full_forward(B):
+    pin_rows_alone_equal_full_forward(B)
+
+
 def test_on_grid_block_reproduced_exactly(B):
     pin_on_grid_block_reproduced(B)
 
@@ -231,6 +247,9 @@ MUTATIONS = [
      lambda B: pin_stage_losses_are_block_errors(B, make_stack(B))),
     ("prefix_full_precision", '        x = r["x_out"]', '        x = r["y_fp"]',
      lambda B: pin_stack_is_quantized_prefix_forward(B, make_stack(B))),
+    ("rows_value_head_group", "V[:p + 1, g * dm.d:(g + 1) * dm.d]",
+     "V[:p + 1, h % dm.nkv * dm.d:(h % dm.nkv + 1) * dm.d]",
+     lambda B: pin_rows_alone_equal_full_forward(B)),
     ("mlp_input_unnormalised", "xm = f32(bf16_round(rmsnorm(h, eps)))",
      "xm = f32(bf16_round(h))", lambda B: pin_on_grid_block_reproduced(B)),
 ]
