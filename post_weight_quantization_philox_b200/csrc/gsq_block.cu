@@ -257,10 +257,13 @@ struct Arena {
   }
 };
 
-// a device copy of a caller buffer when it is host memory
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// a device copy of a caller buffer when it is host memory or not 16-byte
+// aligned (the kernels use 16-byte vector accesses and TMA)
 const void* device_view(Arena& A, const void* p, size_t bytes) {
   if (A.status != GSQ_OK) return nullptr;
-  if (stage_is_device_ptr(p)) return p;
+  if (stage_is_device_ptr(p) && aligned16(p)) return p;
   void* d = A.get<char>(bytes);
   if (d) A.ok(cudaMemcpyAsync(d, p, bytes, cudaMemcpyDefault, A.st));
   return d;
@@ -447,7 +450,7 @@ int gsq_dequant(int grid_mode, const void* packed, const float* scales_f32, int6
   const void* pd = device_view(A, packed, pbytes);
   const void* sd = device_view(A, scales_f32, (size_t)N * (K / group) * 4);
   void* wd = W_bf16;
-  const bool out_dev = stage_is_device_ptr(W_bf16);
+  const bool out_dev = stage_is_device_ptr(W_bf16) && aligned16(W_bf16);
   if (!out_dev) wd = A.get<__nv_bfloat16>(N * K);
   if (A.status != GSQ_OK) return A.status;
   A.ok(launch_dequant(grid_mode, static_cast<const uint32_t*>(pd), static_cast<const float*>(sd),
