@@ -502,6 +502,94 @@ def run_scale_stage(args, rank, world, local_rank):
             "gpu_launches": int(args.steps * 4), "clocks": clk, "last_loss": loss}
 
 
+# Llama-3.1-70B block on 8 sequences x 2048 tokens
+BLOCK_70B = dict(nseq=8, S=2048, nh=64, nkv=8, d=128, F=28672)
+
+
+def block_step_flops(nseq, S, nh, nkv, d, F):
+    """GEMM flops of one step of each stage (Q, K, V/O, MLP) of the block."""
+    T, H, Hk = nseq * S, nh * d, nkv * d
+    q = 4.0 * T * H * H
+    k = 4.0 * T * H * Hk
+    vo = 2.0 * (2 * T * H * Hk + 3 * T * H * H) + 2 * 2.0 * nseq * nh * d * S * (S + 1) / 2
+    mlp = 7 * 2.0 * T * H * F
+    return [q, k, vo, mlp]
+
+
+def run_block_pipeline(args, rank, world, local_rank):
+    """GSQ's staged reconstruction of one 70B-shaped block (Q, K, V/O, MLP on
+    the block output, then the quantized output for the next block) through
+    gsq_block_quantize, --steps steps per stage; the timed region is the
+    whole call (full-precision forward, four stage contexts, hardening,
+    propagation)."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    dm = BLOCK_70B
+    T, H, Hk, F = dm["nseq"] * dm["S"], dm["nh"] * dm["d"], dm["nkv"] * dm["d"], dm["F"]
+    # seeded synthetic block: x ~ N(0, 1) residual stream, weights N(0, 0.02^2)
+    gen = torch.Generator(device="cuda").manual_seed(7007 + 7919 * rank)
+    x = torch.randn((T, H), generator=gen, device="cuda")
+    shapes = gsq.block_weight_shapes(dm["nh"], dm["nkv"], dm["d"], F)
+    W = {n: (torch.randn(shp, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+         for n, shp in shapes.items()}
+    dims = (dm["nseq"], dm["S"], dm["nh"], dm["nkv"], dm["d"], F)
+    warm = [synth.tau_schedule(1.0, 0.05, args.warmup)] * 4
+    gsq.gsq_block_quantize(x, W, *dims, warm, 1e-3, seed=rank)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    taus = [synth.tau_schedule(1.0, 0.05, args.steps)] * 4
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    r = gsq.gsq_block_quantize(x, W, *dims, taus, 1e-3, seed=rank)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    coords = sum(a * b for a, b in shapes.values())
+    flops = block_step_flops(*dims)
+    stage_ms = [r["stats"][s]["ms"] for s in gsq.BLOCK_STAGES]
+    steps_ms = sum(stage_ms)
+    ach = sum(flops) * args.steps / (ms / 1e3) / 1e12
+    per_stage = {s: {"ms_per_step": m / args.steps,
+                     "tflops": round(f * args.steps / (m / 1e3) / 1e12, 1) if m > 0 else None}
+                 for s, m, f in zip(gsq.BLOCK_STAGES, stage_ms, flops)}
+    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "steps_per_s": 1e3 * args.steps / ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 GEMM operands, fp32 state and residual stream", "data":
+            "synthetic (seeded torch generator: x ~ N(0,1), weights ~ N(0,0.02^2) bf16)",
+            "config": {"workload": "c5_70b_block_pipeline", **dm, "grid": "2bit",
+                       "steps_per_stage": args.steps,
+                       "step": "one step of every stage; timed: the whole block call"},
+            "roofline": {"bound": "tensor", "kernel": "whole block call (stage GEMM flops)",
+                         "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
+                         "frac": round(ach / tf_sus, 4),
+                         "peak_kind": f"{peak_kind} (sustained bf16)", "traffic": None},
+            "stages": per_stage, "stage_steps_share": round(steps_ms / ms, 4),
+            "stage_stats": {s: {k: v for k, v in r["stats"][s].items() if k != "ms"}
+                            for s in gsq.BLOCK_STAGES},
+            "clocks": clk}
+
+
 def gptq_simt_flops(N: int, K: int) -> float:
     """fp32 SIMT flops of one GPTQ call: Cholesky of the damped K x K
     Hessian (K^3 / 3), inverse of its triangular factor (K^3 / 3), the
@@ -607,7 +695,7 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq"],
+    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq", "block"],
                     help="time a block stage instead of a single layer")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
@@ -638,6 +726,8 @@ def main():
         out = run_scale_stage(args, rank, world, local_rank)
     elif args.stage == "gptq":
         out = run_gptq_stage(args, rank, world, local_rank)
+    elif args.stage == "block":
+        out = run_block_pipeline(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:

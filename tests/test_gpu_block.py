@@ -7,9 +7,15 @@ prefix's output; inside a block Q and K, then V with O, then the MLP on the
 block output (agihunt.info summary, optimisation paragraph).
 
 Tolerances: dequantization bit-exact (the same fp32 product and rounding as
-the stages' hard weight); the block forward normwise 2e-3 on each sublayer's
-contribution (bf16 operands, fp32 accumulation on the GPU against fp64 with
-the same bf16 roundings in the oracle); the pipeline's first-step losses of
+the stages' hard weight); the block forward 2^-7 relative on each sublayer's
+contribution, per row and normwise.  Both sides round the same GEMM operands
+to bf16 (xa, Q, K, P, V, o, xm, silu(a) b), but the GPU accumulates in fp32
+and the oracle in fp64, so an operand that sits near a rounding boundary can
+land one bf16 unit (2^-8 relative) apart; a sublayer whose operands all
+moved by one unit would be off by about 2^-8, and the bound allows twice
+that.  (Measured: attention rows 1e-6 without such a flip, up to 3e-3 with;
+MLP rows about 1e-3, where the attention's difference moves the bf16
+rounding of RMSNorm(h).)  The pipeline's first-step losses of
 every stage 1e-2 (the loss contract), final hard errors within 2%, and the
 block output equal to the oracle's block forward with the GPU's own hard
 weights at the forward tolerance."""
@@ -20,7 +26,7 @@ from post_weight_quantization_philox_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-FWD_TOL = 2e-3
+FWD_TOL = 2.0 ** -7
 
 
 @pytest.fixture(scope="module")
@@ -93,6 +99,14 @@ def test_block_forward_matches_oracle(g, B):
     xs = np.float32(x).astype(np.float64)
     assert rel(h - xs, f["h"] - xs) < FWD_TOL
     assert rel(y - h, f["y"] - f["h"]) < FWD_TOL
+    rows_a = (np.linalg.norm((h - xs) - (f["h"] - xs), axis=1)
+              / np.linalg.norm(f["h"] - xs, axis=1))
+    rows_m = (np.linalg.norm((y - h) - (f["y"] - f["h"]), axis=1)
+              / np.linalg.norm(f["y"] - f["h"], axis=1))
+    assert rows_a.max() < FWD_TOL and rows_m.max() < FWD_TOL
+    # the first query of every sequence attends to itself only: no
+    # probability rounding, so the attention rows agree to fp32 accumulation
+    assert rows_a[0] < 1e-4 and rows_a[dm.S] < 1e-4
 
 
 def test_block_forward_full_70b_shape_sampled_rows(g, B):
