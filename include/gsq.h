@@ -141,12 +141,8 @@ GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2
 /*
  * gsq_run -- n consecutive steps at temperatures taus[0..n) (host array),
  * asynchronous.  Same results, bit for bit, as n calls of gsq_step; the
- * backward of each step but the last also builds the next step's soft
- * weight, so no step re-reads the logits for its soft weight.  The next
- * step's Gumbel noise is drawn on a second stream of the context while the
- * current step's GEMMs run (the given stream waits for it through an event
- * before the backward), so work on the given stream still completes in
- * order.
+ * backward of each step but the last also builds the next step's soft weight
+ * and Gumbel noise, so no step re-reads the logits for its soft weight.
  */
 GSQ_API int gsq_run(gsq_ctx* ctx, const float* taus, int64_t n, float lr,
                     float beta1, float beta2);
@@ -226,8 +222,7 @@ GSQ_API const char* gsq_error_string(int status);
  * returns and resets the accumulated milliseconds and kernel launches of
  * 0 soft weight, 1 forward GEMM + loss, 2 weight-gradient GEMM,
  * 3 backward + Lion, 4 backward + Lion that also built the next step's soft
- * weight (gsq_run; its launches include the kernel that drew that step's
- * noise on a side stream during the GEMMs).  Syncs. */
+ * weight (gsq_run).  Syncs. */
 GSQ_API int gsq_set_timing(gsq_ctx* ctx, int on);
 GSQ_API int gsq_phase_times(gsq_ctx* ctx, double* ms, int64_t* launches);
 

@@ -6,7 +6,6 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
-#include <utility>
 #include <vector>
 
 #include "../../include/gsq.h"
@@ -50,11 +49,6 @@ struct gsq_ctx {
   unsigned* ticket = nullptr;
   int* err = nullptr;
   float* gbuf = nullptr;  // Gumbel noise of the pending step (L x N x K)
-  // gsq_run draws the noise of step t + 1 into gbuf2 on the side stream nst
-  // while the GEMMs of step t run on st; the two buffers then swap.
-  float* gbuf2 = nullptr;
-  cudaStream_t nst = nullptr;
-  cudaEvent_t ev_free = nullptr, ev_ready = nullptr;
   float *wsoft32 = nullptr, *dl = nullptr, *ds = nullptr;  // debug, lazy
   // What and gbuf hold the soft weight and noise of step what_t at
   // temperature what_tau (what_t < 0: nothing precomputed)
@@ -107,14 +101,6 @@ int dalloc(gsq_ctx* c, T** p, size_t count) {
 }
 
 void free_all(gsq_ctx* c) {
-  if (c->nst) {
-    cudaStreamSynchronize(c->nst);
-    cudaStreamDestroy(c->nst);
-    c->nst = nullptr;
-  }
-  if (c->ev_free) cudaEventDestroy(c->ev_free);
-  if (c->ev_ready) cudaEventDestroy(c->ev_ready);
-  c->ev_free = c->ev_ready = nullptr;
   for (void* p : c->allocs) cudaFree(p);
   c->allocs.clear();
   for (auto& te : c->tev)
@@ -312,7 +298,6 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   AL(c->logits, c->L * NK);
   AL(c->mom, c->L * NK);
   AL(c->gbuf, c->L * NK);
-  AL(c->gbuf2, c->L * NK);
   AL(c->s, N * c->G);
   AL(c->ms, N * c->G);
   AL(c->i0, NK);
@@ -361,12 +346,6 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
     return status;
   };
   if (rc != GSQ_OK) return cleanup_fail(rc);
-  if (cudaStreamCreateWithFlags(&c->nst, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaEventCreateWithFlags(&c->ev_free, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&c->ev_ready, cudaEventDisableTiming) != cudaSuccess) {
-    cudaGetLastError();
-    return cleanup_fail(GSQ_ERR_CUDA);
-  }
 
   cudaStream_t st = c->st;
   cudaError_t e = cudaSuccess;
@@ -455,18 +434,6 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
     tm = &c->tev[c->tev_used++];
     CK(cudaEventRecord(tm->ev[0], c->st));
   }
-  const bool fused = tau_next > 0.f;
-  if (fused) {
-    // the noise of step t + 1 (it depends on nothing but the counter) goes
-    // into gbuf2 on the side stream once the last reader of gbuf2 -- the
-    // backward of step t - 1, already enqueued on st -- is done; it then
-    // runs beside this step's GEMMs (a small grid leaves room for them)
-    CK(cudaEventRecord(c->ev_free, c->st));
-    CK(cudaStreamWaitEvent(c->nst, c->ev_free, 0));
-    CK(launch_noise(c->mode, c->N, c->K, c->seed, (uint32_t)(c->t + 1), c->noise, c->gbuf2,
-                    2 * c->sms, c->nst));
-    CK(cudaEventRecord(c->ev_ready, c->nst));
-  }
   const bool soft = !(c->what_t == (int64_t)c->t && c->what_tau == tau);
   if (soft) CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));
   if (tm) {
@@ -478,12 +445,9 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
   if (tm) CK(cudaEventRecord(tm->ev[2], c->st));
   CK(run_weight_grad(c));
   if (tm) CK(cudaEventRecord(tm->ev[3], c->st));
-  if (fused) CK(cudaStreamWaitEvent(c->st, c->ev_ready, 0));
   CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, tau_next,
-                          c->What, nullptr, nullptr, c->sms, c->st,
-                          fused ? c->gbuf2 : nullptr));
+                          c->What, nullptr, nullptr, c->sms, c->st));
   if (tm) CK(cudaEventRecord(tm->ev[4], c->st));
-  if (fused) std::swap(c->gbuf, c->gbuf2);  // step t + 1's noise is now current
   c->t += 1;
   c->hcode_valid = false;  // the logits moved
   if (tau_next > 0.f) {
@@ -747,8 +711,7 @@ int gsq_phase_times(gsq_ctx* c, double* ms, int64_t* launches) {
       // backward launches that also built the next soft weight count apart
       const int slot = (p == 3 && te.next) ? 4 : p;
       acc[slot] += x;
-      // a fused backward step also launched the side-stream noise kernel
-      if (p != 0 || te.soft) n[slot] += slot == 4 ? 2 : 1;
+      if (p != 0 || te.soft) n[slot] += 1;
     }
   }
   for (int p = 0; p < 5; ++p) {

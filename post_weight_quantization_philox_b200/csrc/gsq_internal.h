@@ -144,18 +144,13 @@ cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
                                float* gbuf, float* wsoft32, int sm_count,
                                cudaStream_t st);
 // Backward + Lion of step a.t from dW and the noise in gbuf; with
-// tau_next > 0 also the soft weight of step a.t + 1 (into What), with that
-// step's noise read from gnext when given (drawn by launch_noise), else
-// drawn here and written over gbuf.
+// tau_next > 0 also the soft weight (into What) and noise (into gbuf) of
+// step a.t + 1.
 cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
                                  float* gbuf, float lr, float b1, float b2,
                                  float tau_next, __nv_bfloat16* What,
                                  float* dl_dbg, float* ds_dbg, int sm_count,
-                                 cudaStream_t st, const float* gnext = nullptr);
-// Gumbel noise of step t (L planes of N x K) into gout; `blocks` CTAs of 256
-// threads, grid-stride (small grids leave room for concurrent kernels).
-cudaError_t launch_noise(int mode, int64_t N, int64_t K, uint64_t seed, uint32_t t,
-                         int noise, float* gout, int blocks, cudaStream_t st);
+                                 cudaStream_t st);
 cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
                                const float* logits, const float* s,
                                const int8_t* i0, __nv_bfloat16* What,

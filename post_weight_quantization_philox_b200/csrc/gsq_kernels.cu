@@ -318,16 +318,12 @@ struct BwdCfg {
   static constexpr int SMEM = WARPS * 2 * BUF;
 };
 
-// NEXT: 0 = backward only; 1 = also the next step's soft weight, its noise
-// drawn here and written over this step's in gbuf; 2 = also the next step's
-// soft weight, its noise read from gnext (drawn beforehand by k_noise).
-template <int MODE, bool DBG, int NEXT>
+template <int MODE, bool DBG, bool NEXT>
 __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
     k_backward_lion(float* __restrict__ logits, float* __restrict__ mom,
                     float* __restrict__ s, float* __restrict__ ms,
                     const int8_t* __restrict__ i0, const float* __restrict__ dW,
-                    float* __restrict__ gbuf, const float* __restrict__ gnext_in,
-                    int64_t N, int64_t K, uint32_t k0,
+                    float* __restrict__ gbuf, int64_t N, int64_t K, uint32_t k0,
                     uint32_t k1, uint32_t t_next, int noise, float inv_tau,
                     float inv_tau_next, float lr, float b1, float omb1, float b2,
                     float omb2, __nv_bfloat16* __restrict__ What,
@@ -383,18 +379,9 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
       for (int j = 0; j < 4; ++j) lev[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
     float gnext[NEXT ? 4 : 1][L];
-    if (NEXT == 1) {
+    if (NEXT) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) noise1<L>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
-    } else if (NEXT == 2) {
-#pragma unroll
-      for (int p = 0; p < L; ++p) {
-        const float4 g4 = __ldg(reinterpret_cast<const float4*>(gnext_in + p * NK + c0));
-        gnext[0][p] = g4.x;
-        gnext[NEXT ? 1 : 0][p] = g4.y;
-        gnext[NEXT ? 2 : 0][p] = g4.z;
-        gnext[NEXT ? 3 : 0][p] = g4.w;
-      }
     }
     float ds_part = 0.f;
     float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
@@ -465,13 +452,11 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
         w[j] = s_new * coord_soft<MODE>(l, gnext[NEXT ? j : 0], inv_tau_next, cand, y);
       }
       store_bf16x4(What + c0, w);
-      if (NEXT == 1) {
 #pragma unroll
-        for (int p = 0; p < L; ++p) {
-          float4 g4 = make_float4(gnext[NEXT ? 0 : 0][p], gnext[NEXT ? 1 : 0][p],
-                                  gnext[NEXT ? 2 : 0][p], gnext[NEXT ? 3 : 0][p]);
-          *reinterpret_cast<float4*>(gbuf + p * NK + c0) = g4;
-        }
+      for (int p = 0; p < L; ++p) {
+        float4 g4 = make_float4(gnext[NEXT ? 0 : 0][p], gnext[NEXT ? 1 : 0][p],
+                                gnext[NEXT ? 2 : 0][p], gnext[NEXT ? 3 : 0][p]);
+        *reinterpret_cast<float4*>(gbuf + p * NK + c0) = g4;
       }
     }
   }
@@ -1035,9 +1020,9 @@ cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
   return cudaGetLastError();
 }
 
-template <int MODE, int NEXT>
+template <int MODE, bool NEXT>
 static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
-                          const float* gnext, float lr, float b1, float b2, float tau_next,
+                          float lr, float b1, float b2, float tau_next,
                           __nv_bfloat16* What, float* dl_dbg, float* ds_dbg,
                           int blocks, cudaStream_t st) {
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
@@ -1055,12 +1040,12 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   }
   if (dl_dbg) {
     k_backward_lion<MODE, true, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, gnext, a.N, a.K, k0, k1,
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         dl_dbg, ds_dbg);
   } else {
     k_backward_lion<MODE, false, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, gnext, a.N, a.K, k0, k1,
+        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         nullptr, nullptr);
   }
@@ -1068,25 +1053,22 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
 
 template <int MODE>
 static void backward_dispatch(const StepArgs& a, const float* dW, float* gbuf,
-                              const float* gnext, float lr, float b1, float b2,
-                              float tau_next, __nv_bfloat16* What, float* dl_dbg,
+                              float lr, float b1, float b2, float tau_next,
+                              __nv_bfloat16* What, float* dl_dbg,
                               float* ds_dbg, int blocks, cudaStream_t st) {
-  if (tau_next > 0.f && gnext)
-    backward_mode<MODE, 2>(a, dW, gbuf, gnext, lr, b1, b2, tau_next, What, dl_dbg,
-                           ds_dbg, blocks, st);
-  else if (tau_next > 0.f)
-    backward_mode<MODE, 1>(a, dW, gbuf, nullptr, lr, b1, b2, tau_next, What, dl_dbg,
-                           ds_dbg, blocks, st);
+  if (tau_next > 0.f)
+    backward_mode<MODE, true>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+                              ds_dbg, blocks, st);
   else
-    backward_mode<MODE, 0>(a, dW, gbuf, nullptr, lr, b1, b2, tau_next, What, dl_dbg,
-                           ds_dbg, blocks, st);
+    backward_mode<MODE, false>(a, dW, gbuf, lr, b1, b2, tau_next, What,
+                               dl_dbg, ds_dbg, blocks, st);
 }
 
 cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
                                  float* gbuf, float lr, float b1, float b2,
                                  float tau_next, __nv_bfloat16* What,
                                  float* dl_dbg, float* ds_dbg, int sm_count,
-                                 cudaStream_t st, const float* gnext) {
+                                 cudaStream_t st) {
   const int64_t groups = a.N * (a.K / kGroup);
   // persistent: as many CTAs as fit on the SMs at once, fewer for small layers
   auto blocks_for = [&](int warps, int ctas) {
@@ -1098,42 +1080,9 @@ cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
                          ? blocks_for(BwdCfg<GRID_3BIT_LOCAL>::WARPS, BwdCfg<GRID_3BIT_LOCAL>::CTAS)
                          : blocks_for(BwdCfg<GRID_2BIT>::WARPS, BwdCfg<GRID_2BIT>::CTAS);
   switch (a.mode) {
-    case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, gbuf, gnext, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
-    case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, gbuf, gnext, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
-    default: backward_dispatch<GRID_3BIT_LOCAL>(a, dW, gbuf, gnext, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st);
-  }
-  return cudaGetLastError();
-}
-
-// Gumbel noise of step t for every coordinate into gout (L planes of N x K):
-// one thread per four consecutive coordinates, 16-byte stores.  Used to draw
-// the next step's noise on a second stream while the GEMMs of the current
-// step run, so the fused backward only reads it.
-template <int MODE>
-__global__ void __launch_bounds__(256) k_noise(int64_t NK, uint32_t k0, uint32_t k1,
-                                               uint32_t t, int noise,
-                                               float* __restrict__ gout) {
-  constexpr int L = GridT<MODE>::L;
-  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < NK / 4;
-       q += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t c0 = q * 4;
-    float g[4][L];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) noise1<L>(c0 + j, t, k0, k1, noise, g[j]);
-#pragma unroll
-    for (int p = 0; p < L; ++p)
-      __stcs(reinterpret_cast<float4*>(gout + p * NK + c0),
-             make_float4(g[0][p], g[1][p], g[2][p], g[3][p]));
-  }
-}
-
-cudaError_t launch_noise(int mode, int64_t N, int64_t K, uint64_t seed, uint32_t t,
-                         int noise, float* gout, int blocks, cudaStream_t st) {
-  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
-  switch (mode) {
-    case GRID_2BIT: k_noise<GRID_2BIT><<<blocks, 256, 0, st>>>(N * K, k0, k1, t, noise, gout); break;
-    case GRID_TERNARY: k_noise<GRID_TERNARY><<<blocks, 256, 0, st>>>(N * K, k0, k1, t, noise, gout); break;
-    default: k_noise<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(N * K, k0, k1, t, noise, gout);
+    case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    default: backward_dispatch<GRID_3BIT_LOCAL>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st);
   }
   return cudaGetLastError();
 }
