@@ -69,6 +69,8 @@ def lib():
             "gsqo_backward": (None, [_i32, _i64, _i64, _i32, _p, _p, _p, _p, _p,
                                      _f32, _p, _p]),
             "gsqo_lion": (None, [_i64, _p, _p, _p, _f32, _f32, _f32]),
+            "gsqo_bf16_sr": (_f32, [_f32, _u32]),
+            "gsqo_state16_store": (None, [_i32, _i64, _i64, _i64, _u64, _u32, _p, _p]),
             "gsqo_step": (_i32, [_i32, _i64, _i64, _i64, _i64, _i32, _p, _p, _p,
                                  _p, _p, _p, _p, _u64, _u32, _f32, _f32, _f32,
                                  _f32, _i32, _p, _p, _p, _p, _p, _p]),
@@ -162,15 +164,31 @@ class State:
     seed: int = 0
     t: int = 0
     noise: bool = True
+    # bf16 logits and momenta (the reduced-memory mode): after each Lion
+    # update the logits are rounded stochastically and the momenta to nearest
+    state16: bool = False
 
     def copy(self) -> "State":
         return State(self.mode, self.N, self.K, self.group, self.logits.copy(),
                      self.mom.copy(), self.s.copy(), self.ms.copy(),
-                     self.i0.copy(), self.row0, self.seed, self.t, self.noise)
+                     self.i0.copy(), self.row0, self.seed, self.t, self.noise,
+                     self.state16)
+
+
+def bf16_sr(x: float, r9: int) -> float:
+    """Stochastic rounding of an fp32 value to bf16 with a 9-bit threshold."""
+    return lib().gsqo_bf16_sr(x, r9)
+
+
+def state16_store(st: "State", t_next: int) -> None:
+    """Rounds st.logits (stochastically) and st.mom (to nearest) to bf16 in
+    place, thresholds from the Philox words of step t_next."""
+    lib().gsqo_state16_store(st.mode, st.row0, st.N, st.K, st.seed, t_next,
+                             _ptr(st.logits), _ptr(st.mom))
 
 
 def init(mode: int, W, group: int = 128, init_idx=None, seed: int = 0,
-         row0: int = 0) -> State:
+         row0: int = 0, state16: bool = False) -> State:
     W = _f32a(W)
     N, K = W.shape
     L = NUM_LOGITS[mode]
@@ -184,6 +202,7 @@ def init(mode: int, W, group: int = 128, init_idx=None, seed: int = 0,
                          _ptr(st.i0), _ptr(st.logits), _ptr(st.mom), _ptr(st.ms))
     if rc != 0:
         raise ValueError(f"gsqo_init failed ({rc})")
+    st.state16 = state16  # the initial logits (0, +2) and momenta (0) are bf16 values
     return st
 
 
@@ -269,6 +288,8 @@ def step(st: State, X, Yref, tau: float, lr: float, beta1: float = 0.9,
                          _ptr(d.get("dl")), _ptr(d.get("ds")))
     if rc != 0:
         raise RuntimeError(f"gsqo_step failed ({rc})")
+    if st.state16:
+        state16_store(st, st.t + 1)
     st.t += 1
     return (loss.value, d) if dumps else loss.value
 
@@ -286,6 +307,8 @@ def backward_lion(st: State, dW, tau, lr, beta1=0.9, beta2=0.99):
                                   _ptr(dl), _ptr(ds))
     if rc != 0:
         raise RuntimeError(f"gsqo_backward_lion failed ({rc})")
+    if st.state16:
+        state16_store(st, st.t + 1)
     return dl, ds
 
 

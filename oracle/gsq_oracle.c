@@ -527,6 +527,49 @@ int gsqo_step(int mode, int64_t row0, int64_t N, int64_t K, int64_t T,
     return rc;
 }
 
+/* --------------------------------------------- bf16 logit / momentum state */
+
+/* Stochastic rounding of an fp32 value to bf16 with a 9-bit threshold r:
+ * r << 7 is added to the fp32 bit pattern and the low 16 bits are dropped,
+ * so the magnitude rounds up with probability (low 16 bits) / 2^16, to 2^-9
+ * of a bf16 unit.  Exactly representable values are returned unchanged. */
+float gsqo_bf16_sr(float x, uint32_t r9) {
+    uint32_t b;
+    memcpy(&b, &x, sizeof(b));
+    b += (r9 & 0x1FFu) << 7;
+    b &= 0xFFFF0000u;
+    float y;
+    memcpy(&y, &b, sizeof(y));
+    return y;
+}
+
+/* After the fp32 Lion update of step t: logits to bf16 by stochastic
+ * rounding, the threshold of logit p of a coordinate being the low 9 bits of
+ * the Philox word that gives that coordinate and logit its noise at step
+ * t + 1 (the words of coord_uniforms); momenta to the nearest bf16 (ties to
+ * even).  Rows row0.. of the layer (global coordinate (row0 + n) K + k). */
+void gsqo_state16_store(int mode, int64_t row0, int64_t N, int64_t K,
+                        uint64_t seed, uint32_t t_next, float* logits,
+                        float* mom) {
+    const int L = gsqo_num_logits(mode);
+    const int64_t NK = N * K;
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    for (int64_t i = 0; i < NK; ++i) {
+        const uint64_t coord = (uint64_t)(row0 * K + i);
+        uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next, 0u};
+        uint32_t w[8];
+        gsqo_philox4x32_10(ctr, key, w);
+        if (L == 5) {
+            ctr[3] = 1u;
+            gsqo_philox4x32_10(ctr, key, w + 4);
+        }
+        for (int p = 0; p < L; ++p) {
+            logits[p * NK + i] = gsqo_bf16_sr(logits[p * NK + i], w[p]);
+            mom[p * NK + i] = (float)gsqo_bf16_round((double)mom[p * NK + i]);
+        }
+    }
+}
+
 /* ---------------------------------------------------------- harden, pack */
 
 static int argmax_first(const float* l, int n) {

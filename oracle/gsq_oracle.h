@@ -108,6 +108,15 @@ int gsqo_backward_lion(int mode, int64_t row0, int64_t N, int64_t K, int group,
                        float beta2, int noise_on, float* dl_dump,
                        float* ds_dump);
 
+/* bf16 state (the reduced-memory mode): stochastic rounding with a 9-bit
+ * threshold, and the rounding of logits (stochastic, thresholds from the
+ * low 9 bits of the step-(t+1) Philox words) and momenta (nearest) after
+ * the fp32 Lion update of step t */
+float gsqo_bf16_sr(float x, uint32_t r9);
+void gsqo_state16_store(int mode, int64_t row0, int64_t N, int64_t K,
+                        uint64_t seed, uint32_t t_next, float* logits,
+                        float* mom);
+
 /* A6: hard level per coordinate (argmax of logits, first max, no noise) */
 void gsqo_harden(int mode, int64_t N, int64_t K, const float* logits,
                  const int8_t* i0, uint8_t* level);

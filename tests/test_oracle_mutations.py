@@ -16,6 +16,7 @@ import test_oracle_mlp as mlp_pins  # noqa: E402
 import test_oracle_pins as pins  # noqa: E402
 import test_oracle_gptq as gptq_pins  # noqa: E402
 import test_oracle_scale as scale_pins  # noqa: E402
+import test_oracle_state16 as state16_pins  # noqa: E402
 
 # (name, original text, planted text, pins expected to catch it)
 MUTATIONS = [
@@ -82,6 +83,20 @@ MUTATIONS = [
      "double w = (double)s[n * G + k / group] * gsqo_level_value(mode, lev[c]);\n        wq[c]",
      "double w = gsqo_level_value(mode, lev[c]);\n        wq[c]",
      ["scale:test_scale_grad_central_differences", "scale:test_scale_step_on_grid_weight_is_a_fixed_point"]),
+    ("state16_logits_to_nearest", "logits[p * NK + i] = gsqo_bf16_sr(logits[p * NK + i], w[p]);",
+     "logits[p * NK + i] = (float)gsqo_bf16_round((double)logits[p * NK + i]);",
+     ["state16:test_rounding_follows_fp32_lion_on_average",
+      "state16:test_thresholds_are_next_step_philox_words"]),
+    ("state16_thresholds_this_step",
+     "uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next, 0u};",
+     "uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next - 1u, 0u};",
+     ["state16:test_thresholds_are_next_step_philox_words"]),
+    ("state16_threshold_scale", "b += (r9 & 0x1FFu) << 7;", "b += (r9 & 0x1FFu) << 6;",
+     ["state16:test_stochastic_rounding_brackets_and_is_unbiased"]),
+    ("state16_momenta_truncated",
+     "mom[p * NK + i] = (float)gsqo_bf16_round((double)mom[p * NK + i]);",
+     "mom[p * NK + i] = gsqo_bf16_sr(mom[p * NK + i], 0u);",
+     ["state16:test_momenta_round_to_nearest"]),
     ("gptq_update_transposed", "W[:, j + 1:] -= np.outer(e, U[j, j + 1:])",
      "W[:, j + 1:] -= np.outer(e, U[j + 1:, j])",
      ["gptq:test_first_column_update_is_damped_least_squares", "gptq:test_loss_identity_over_the_loop"]),
@@ -118,7 +133,7 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new, catchers):
     caught = []
     for tname in catchers:
         module = {"mlp": mlp_pins, "attn": attn_pins, "scale": scale_pins,
-                  "gptq": gptq_pins}.get(
+                  "gptq": gptq_pins, "state16": state16_pins}.get(
             tname.split(":")[0], pins) \
             if ":" in tname else pins
         tname = tname.split(":")[-1]
