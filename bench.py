@@ -95,11 +95,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def phase_bytes_flops(cfg, layer):
-    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch.
+def phase_bytes_flops(cfg, layer, es=4):
+    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch; es is
+    the bytes of one logit / momentum element (4, or 2 in the bf16 state).
 
     soft weight:        read L logit planes + scale (+ initial level),
-                        write bf16 weight and the L noise planes;
+                        write bf16 weight and the L fp32 noise planes;
     backward + Lion:    read dW, logits, momenta, noise (+ initial level),
                         write logits and momenta, 16 B per group of scales;
     ... + next soft:    also write the next bf16 weight and noise planes."""
@@ -107,9 +108,9 @@ def phase_bytes_flops(cfg, layer):
     L = layer.L
     extra = 1 if cfg.grid == synth.GRID_3BIT_LOCAL else 0  # initial level (int8)
     groups = cfg.N * (cfg.K // 128)
-    soft = NK * (8 * L + 2 + extra) + groups * 4
-    back = NK * (4 + 20 * L + extra) + groups * 16
-    back_next = NK * (6 + 24 * L + extra) + groups * 16
+    soft = NK * (es * L + 4 * L + 2 + extra) + groups * 4
+    back = NK * (4 + 4 * es * L + 4 * L + extra) + groups * 16
+    back_next = NK * (6 + 4 * es * L + 8 * L + extra) + groups * 16
     gemm = 2.0 * cfg.N * cfg.T * cfg.K
     return {"soft_weight": ("hbm", soft), "forward_gemm": ("tensor", gemm),
             "weight_grad_gemm": ("tensor", gemm), "backward_lion": ("hbm", back),
@@ -134,7 +135,8 @@ def run_gsq(args, rank, world, local_rank):
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
     stream = torch.cuda.current_stream()
-    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=rank)
+    state16 = args.state == "bf16"
+    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=rank, state_bf16=state16)
     taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
     nt = len(taus)
 
@@ -186,7 +188,8 @@ def run_gsq(args, rank, world, local_rank):
     value = world * coords * steps_per_s
     names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion",
              "backward_lion_next_soft"]
-    work = phase_bytes_flops(cfg, lay)
+    es = 2 if state16 else 4
+    work = phase_bytes_flops(cfg, lay, es)
     phases = {}
     for i, nm in enumerate(names):
         if phase_n[i] == 0:
@@ -204,17 +207,21 @@ def run_gsq(args, rank, world, local_rank):
                       "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
     dom = max(phases, key=lambda n: phases[n]["ms"] * phases[n]["launches"])
     d = phases[dom]
-    traffic = load_traffic(dom, args.config)
+    traffic = load_traffic(dom, args.config + ("_bf16_state" if state16 else ""))
+    state_mb = 2 * lay.L * coords * es / 1e6
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "steps_per_s": steps_per_s, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state",
+        "vs_baseline": None,
+        "dtype": ("bf16 GEMM operands, bf16 logit/momentum state (stochastic rounding)"
+                  if state16 else "bf16 GEMM operands, fp32 state"),
         "data": "synthetic (seeded; W ~ N(0,0.02^2) bf16, X ~ N(0,1) bf16 with 1% outlier channels x20)",
-        "config": {"workload": cfg.name, "N": cfg.N, "K": cfg.K, "T": cfg.T,
+        "config": {"workload": cfg.name + ("_bf16_state" if state16 else ""),
+                   "N": cfg.N, "K": cfg.K, "T": cfg.T,
                    "grid": ["2bit", "ternary", "3bit_local"][cfg.grid], "group": 128,
                    "parallelism": f"independent layer per GPU x{world}",
-                   "l2": "state (logits + Lion momenta, 537 MB) larger than L2; no flush"},
+                   "l2": f"state (logits + Lion momenta, {state_mb:.0f} MB) larger than L2; no flush"},
         "roofline": {"bound": d["bound"], "kernel": dom, "achieved": d["achieved"],
                      "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
                      "peak_kind": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})",
@@ -697,6 +704,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq", "block"],
                     help="time a block stage instead of a single layer")
+    ap.add_argument("--state", default="fp32", choices=["fp32", "bf16"],
+                    help="logit / momentum storage of the single-layer step")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
     args = ap.parse_args()

@@ -98,6 +98,25 @@ GSQ_API int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
              int grid_mode, const int8_t* init_idx, uint64_t seed,
              void* stream);
 
+/* gsq_init_bf16_state -- gsq_init with the logits and their Lion momenta
+ * stored as bf16 instead of fp32: half the state memory (the pages put the
+ * logits alone at 2-5x the weight memory, agihunt.info summary, limitations
+ * paragraph) and 32 fewer bytes per coordinate moved by every step's fused
+ * backward for the 2-bit and ternary grids (40 for 3-bit).  Each step still
+ * computes in fp32; after the Lion update the logits are rounded to bf16
+ * stochastically (the fp32 bit pattern plus t << 7, truncated to its top 16
+ * bits, where the 9-bit threshold t is the low 9 bits of the Philox word
+ * that gives the same coordinate and logit its noise at the next step), so
+ * a step smaller than half a bf16 unit still moves a logit in expectation;
+ * the momenta are rounded to the nearest bf16.  Scales and their momenta
+ * stay fp32.  Arguments and errors as gsq_init.  In this mode
+ * GSQ_DBG_LOGITS / GSQ_DBG_MOM and the checkpoint's logit and momentum
+ * sections hold bf16 (2 bytes per element). */
+GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+                                int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+                                int grid_mode, const int8_t* init_idx, uint64_t seed,
+                                void* stream);
+
 /* GPTQ initial assignment (agihunt.info summary, optimisation paragraph: GSQ
  * starts from GPTQ; the algorithm of Frantar et al., "GPTQ: Accurate
  * Post-Training Quantization for Generative Pre-trained Transformers",

@@ -34,6 +34,9 @@ struct Timing {
 
 struct gsq_ctx {
   int mode = 0, L = 0, group = kGroup;
+  // logits and Lion momenta stored as bf16 (the reduced-memory state); the
+  // pointers below keep their float type and the launchers reinterpret them
+  int state16 = 0;
   int64_t N = 0, K = 0, T = 0, Tp = 0, G = 0;
   uint64_t seed = 0, t = 0;
   int noise = 1;
@@ -155,7 +158,13 @@ StepArgs step_args(gsq_ctx* c, float tau) {
   a.t = (uint32_t)c->t;
   a.noise = c->noise;
   a.tau = tau;
+  a.state16 = c->state16;
   return a;
+}
+
+// bytes of one full logit (or momentum) state: L x N x K elements
+size_t state_plane_bytes(const gsq_ctx* c) {
+  return (size_t)c->L * c->N * c->K * (c->state16 ? 2 : 4);
 }
 
 EpiParams forward_params(gsq_ctx* c, double* loss_out) {
@@ -248,10 +257,14 @@ int gsq_packed_bytes(int grid_mode, int64_t N, int64_t K, size_t* bytes) {
   return GSQ_OK;
 }
 
-int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
-             int x_dtype, int64_t N, int64_t K, int64_t T, int group,
-             int grid_mode, const int8_t* init_idx, uint64_t seed,
-             void* stream) {
+}  // extern "C"
+
+namespace {
+
+int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+              int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+              int grid_mode, const int8_t* init_idx, uint64_t seed,
+              void* stream, int state16) {
   if (!out) return GSQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (!W || !X || N <= 0 || K <= 0 || T <= 0 || group <= 0 ||
@@ -274,6 +287,7 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   if (!c) return GSQ_ERR_OOM;
   c->mode = grid_mode;
   c->L = num_logits(grid_mode);
+  c->state16 = state16 ? 1 : 0;
   c->N = N;
   c->K = K;
   c->T = T;
@@ -295,8 +309,9 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   AL(c->dYt, N * Tp);
   AL(c->YrefT, N * Tp);
   AL(c->dW, NK);
-  AL(c->logits, c->L * NK);
-  AL(c->mom, c->L * NK);
+  // bf16 state: half as many 4-byte words
+  AL(c->logits, state16 ? (c->L * NK + 1) / 2 : c->L * NK);
+  AL(c->mom, state16 ? (c->L * NK + 1) / 2 : c->L * NK);
   AL(c->gbuf, c->L * NK);
   AL(c->s, N * c->G);
   AL(c->ms, N * c->G);
@@ -360,7 +375,7 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   ok(cudaMemsetAsync(c->err, 0, 4 * sizeof(int), st));
   ok(cudaMemsetAsync(c->ticket, 0, 4 * sizeof(unsigned), st));
   ok(cudaMemsetAsync(c->loss_hist, 0, kLossRing * sizeof(double), st));
-  ok(cudaMemsetAsync(c->mom, 0, (size_t)c->L * NK * 4, st));
+  ok(cudaMemsetAsync(c->mom, 0, state_plane_bytes(c), st));
   ok(cudaMemsetAsync(c->ms, 0, (size_t)N * c->G * 4, st));
   ok(cudaMemsetAsync(c->dW, 0, (size_t)NK * 4, st));
   ok(cudaMemsetAsync(c->dYt, 0, (size_t)N * Tp * 2, st));
@@ -394,7 +409,7 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
     ok(launch_gemm(tmW, tmXr, em, N, Tp, kw * K, EPI_STORE_F32, ep, c->sms, st));
   }
   ok(launch_init_state(grid_mode, W32, idx_d, N, K, c->s, c->i0, c->logits,
-                       c->err, st));
+                       c->err, st, c->state16));
   ok(launch_sumsq(c->YrefT, N * Tp, c->partials, c->ticket, c->scratch, st));
   if (e != cudaSuccess) return cleanup_fail(cuda_status(e));
   e = cudaStreamSynchronize(st);
@@ -412,6 +427,26 @@ int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   *out = c;
   return GSQ_OK;
 #undef AL
+}
+
+}  // namespace
+
+extern "C" {
+
+int gsq_init(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+             int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+             int grid_mode, const int8_t* init_idx, uint64_t seed,
+             void* stream) {
+  return init_impl(out, W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, init_idx, seed,
+                   stream, 0);
+}
+
+int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+                        int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+                        int grid_mode, const int8_t* init_idx, uint64_t seed,
+                        void* stream) {
+  return init_impl(out, W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, init_idx, seed,
+                   stream, 1);
 }
 
 }  // extern "C"
@@ -462,7 +497,8 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
 // codes of the hard choice of the current logits, computed once per logits
 cudaError_t ensure_hard_codes(gsq_ctx* c) {
   if (c->hcode_valid) return cudaSuccess;
-  cudaError_t e = launch_hard_codes(c->mode, c->N, c->K, c->logits, c->i0, c->hcode, c->st);
+  cudaError_t e = launch_hard_codes(c->mode, c->N, c->K, c->logits, c->i0, c->hcode, c->st,
+                                    c->state16);
   if (e == cudaSuccess) c->hcode_valid = true;
   return e;
 }
@@ -574,7 +610,8 @@ int gsq_harden_pack(gsq_ctx* c, void* packed, uint16_t* scales_f16,
   uint16_t* h16 = scales_f16 ? (hd ? scales_f16 : reinterpret_cast<uint16_t*>(sp)) : nullptr;
   if (scales_f16 && !hd) sp += (ng * 2 + 15) / 16 * 16;
   float* f32 = scales_f32 ? (fd ? scales_f32 : reinterpret_cast<float*>(sp)) : nullptr;
-  cudaError_t e = launch_harden_pack(c->mode, c->N, c->K, c->logits, c->i0, pk, c->st);
+  cudaError_t e = launch_harden_pack(c->mode, c->N, c->K, c->logits, c->i0, pk, c->st,
+                                     c->state16);
   if (e == cudaSuccess && (h16 || f32))
     e = launch_export_scales(c->s, ng, h16, f32, c->st);
   if (e == cudaSuccess && !pd)
@@ -599,8 +636,8 @@ int gsq_recon_error(gsq_ctx* c, int mode, float tau, double* abs_err,
     return GSQ_ERR_INVALID_ARG;
   c->what_t = -1;  // What is overwritten below
   if (mode == GSQ_RECON_HARD) {
-    CK(launch_hard_weight(c->mode, c->N, c->K, c->logits, c->s, c->i0, c->What,
-                          c->st));
+    CK(launch_hard_weight(c->mode, c->N, c->K, c->logits, c->s, c->i0, c->What, c->st,
+                          c->state16));
   } else {
     StepArgs a = step_args(c, tau);
     a.noise = 0;
@@ -618,8 +655,7 @@ int gsq_recon_error(gsq_ctx* c, int mode, float tau, double* abs_err,
 
 int gsq_state_bytes(gsq_ctx* c, size_t* bytes) {
   if (!c || !bytes) return GSQ_ERR_INVALID_ARG;
-  *bytes = 8 * sizeof(uint64_t) + (size_t)c->L * c->N * c->K * 4 * 2 +
-           (size_t)c->N * c->G * 4 * 2;
+  *bytes = 8 * sizeof(uint64_t) + state_plane_bytes(c) * 2 + (size_t)c->N * c->G * 4 * 2;
   return GSQ_OK;
 }
 
@@ -639,9 +675,9 @@ int gsq_export_state(gsq_ctx* c, void* host_buf, size_t bytes) {
   h[4] = (uint64_t)c->group;
   h[5] = c->t;
   h[6] = c->seed;
-  h[7] = 0;
+  h[7] = (uint64_t)c->state16;
   char* p = static_cast<char*>(host_buf) + 8 * sizeof(uint64_t);
-  const size_t lb = (size_t)c->L * c->N * c->K * 4, sb = (size_t)c->N * c->G * 4;
+  const size_t lb = state_plane_bytes(c), sb = (size_t)c->N * c->G * 4;
   CK(cudaMemcpy(p, c->logits, lb, cudaMemcpyDeviceToHost));
   CK(cudaMemcpy(p + lb, c->mom, lb, cudaMemcpyDeviceToHost));
   CK(cudaMemcpy(p + 2 * lb, c->s, sb, cudaMemcpyDeviceToHost));
@@ -657,11 +693,12 @@ int gsq_import_state(gsq_ctx* c, const void* host_buf, size_t bytes) {
   if (!host_buf || bytes != need) return GSQ_ERR_INVALID_ARG;
   const uint64_t* h = static_cast<const uint64_t*>(host_buf);
   if (h[0] != kStateMagic || h[1] != (uint64_t)c->mode || h[2] != (uint64_t)c->N ||
-      h[3] != (uint64_t)c->K || h[4] != (uint64_t)c->group || h[6] != c->seed)
+      h[3] != (uint64_t)c->K || h[4] != (uint64_t)c->group || h[6] != c->seed ||
+      h[7] != (uint64_t)c->state16)
     return GSQ_ERR_INVALID_ARG;
   CK(cudaStreamSynchronize(c->st));
   const char* p = static_cast<const char*>(host_buf) + 8 * sizeof(uint64_t);
-  const size_t lb = (size_t)c->L * c->N * c->K * 4, sb = (size_t)c->N * c->G * 4;
+  const size_t lb = state_plane_bytes(c), sb = (size_t)c->N * c->G * 4;
   CK(cudaMemcpy(c->logits, p, lb, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->mom, p + lb, lb, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->s, p + 2 * lb, sb, cudaMemcpyHostToDevice));
@@ -729,8 +766,8 @@ static int debug_buffer(gsq_ctx* c, int which, void** p, size_t* bytes) {
                NG = (size_t)c->N * c->G;
   int rc = GSQ_OK;
   switch (which) {
-    case GSQ_DBG_LOGITS: *p = c->logits; *bytes = LNK * 4; break;
-    case GSQ_DBG_MOM: *p = c->mom; *bytes = LNK * 4; break;
+    case GSQ_DBG_LOGITS: *p = c->logits; *bytes = state_plane_bytes(c); break;
+    case GSQ_DBG_MOM: *p = c->mom; *bytes = state_plane_bytes(c); break;
     case GSQ_DBG_SCALES: *p = c->s; *bytes = NG * 4; break;
     case GSQ_DBG_SMOM: *p = c->ms; *bytes = NG * 4; break;
     case GSQ_DBG_I0: *p = c->i0; *bytes = NK; break;

@@ -116,6 +116,7 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
 // ------------------------------------------------------- elementwise
 struct StepArgs {
   int mode;
+  int state16 = 0;  // logits / momenta planes hold bf16 (reduced-memory state)
   int64_t N, K, G;
   const float* logits;   // L x N x K
   float* logits_w;       // same buffer, written by the backward
@@ -135,9 +136,11 @@ cudaError_t launch_convert_x(const void* X, int dtype, int64_t T, int64_t K,
 cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
                              float* W32, __nv_bfloat16* Wop, int split,
                              int* err, cudaStream_t st);
+// state16: the logit planes hold bf16 (the pointers keep their float type;
+// the launchers reinterpret them)
 cudaError_t launch_init_state(int mode, const float* W32, const int8_t* init_idx,
                               int64_t N, int64_t K, float* s, int8_t* i0,
-                              float* logits, int* err, cudaStream_t st);
+                              float* logits, int* err, cudaStream_t st, int state16 = 0);
 // Soft weight of step a.t; keeps the step's Gumbel noise in gbuf (L planes
 // of N x K fp32) when gbuf is not null.
 cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
@@ -154,14 +157,15 @@ cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
 cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
                                const float* logits, const float* s,
                                const int8_t* i0, __nv_bfloat16* What,
-                               cudaStream_t st);
+                               cudaStream_t st, int state16 = 0);
 cudaError_t launch_harden_pack(int mode, int64_t N, int64_t K,
                                const float* logits, const int8_t* i0,
-                               uint32_t* packed, cudaStream_t st);
+                               uint32_t* packed, cudaStream_t st, int state16 = 0);
 // scale-only step: int8 level codes of the hard choice; w = bf16(s c_code);
 // ds_g = sum dW c_code and Lion on s (ds into ds_dbg when not null)
 cudaError_t launch_hard_codes(int mode, int64_t N, int64_t K, const float* logits,
-                              const int8_t* i0, int8_t* code, cudaStream_t st);
+                              const int8_t* i0, int8_t* code, cudaStream_t st,
+                              int state16 = 0);
 cudaError_t launch_code_weight(int mode, int64_t N, int64_t K, const int8_t* code,
                                const float* s, __nv_bfloat16* What, cudaStream_t st);
 cudaError_t launch_scale_lion(int mode, int64_t N, int64_t K, const int8_t* code,

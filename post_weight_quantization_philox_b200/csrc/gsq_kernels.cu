@@ -15,6 +15,41 @@ namespace {
 
 constexpr int kGroup = 128;
 
+// Logit and Lion-momentum planes hold fp32, or bf16 in the reduced-memory
+// state mode; St<TS> loads them as fp32 and stores fp32 values.
+template <typename TS>
+struct St;
+template <>
+struct St<float> {
+  __device__ static float ld(const float* p) { return __ldg(p); }
+  __device__ static float4 ld4(const float* p) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+  }
+  __device__ static void st(float* p, float v) { *p = v; }
+};
+template <>
+struct St<__nv_bfloat16> {
+  __device__ static float ld(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
+  __device__ static float4 ld4(const __nv_bfloat16* p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+  }
+  // every value stored through here is already a bf16 value
+  __device__ static void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+// bf16 by stochastic rounding with a 9-bit threshold r: r << 7 is added to
+// the fp32 bit pattern and the low half dropped (the magnitude rounds up
+// with probability low16 / 2^16, to 2^-9 of a bf16 unit); returned as the
+// fp32 value of the bf16 result.
+__device__ __forceinline__ float bf16_sr(float x, uint32_t r) {
+  return __uint_as_float((__float_as_uint(x) + ((r & 0x1FFu) << 7)) & 0xFFFF0000u);
+}
+__device__ __forceinline__ float bf16_rn(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 __device__ __forceinline__ void set_err(int* err, int code) {
   atomicCAS(err, 0, code);
 }
@@ -91,12 +126,12 @@ __global__ void k_convert_w(const void* __restrict__ W, int dtype, int64_t N,
 // One warp per group of 128: s = absmax / c_max; initial level by
 // round-to-nearest of w / s (first level on ties, s = 0 -> w / s := 0) or
 // from init_idx; logits +2 on the initial slot.  All comparisons in fp32.
-template <int MODE>
+template <int MODE, typename TS>
 __global__ void k_init_state(const float* __restrict__ W32,
                              const int8_t* __restrict__ init_idx, int64_t N,
                              int64_t K, float* __restrict__ s,
                              int8_t* __restrict__ i0,
-                             float* __restrict__ logits, int* err) {
+                             TS* __restrict__ logits, int* err) {
   using Gr = GridT<MODE>;
   const int64_t G = K / kGroup, NK = N * K;
   const int lane = threadIdx.x & 31;
@@ -156,7 +191,7 @@ __global__ void k_init_state(const float* __restrict__ W32,
         lg[plus ? 3 : 2] = 2.f;
       }
 #pragma unroll
-      for (int p = 0; p < Gr::L; ++p) logits[p * NK + c] = lg[p];
+      for (int p = 0; p < Gr::L; ++p) St<TS>::st(logits + p * NK + c, lg[p]);
     }
   }
 }
@@ -253,9 +288,9 @@ constexpr int kPerLane = kGroup / 32;
 
 // Soft weight (A1 + A2): w = bf16(s * v((l + g) / tau)).  When gbuf is given
 // the step's Gumbel noise is kept there (L planes) for the backward.
-template <int MODE, bool DBG>
+template <int MODE, bool DBG, typename TS>
 __global__ void __launch_bounds__(256) k_soft_weight(
-    const float* __restrict__ logits, const float* __restrict__ s,
+    const TS* __restrict__ logits, const float* __restrict__ s,
     const int8_t* __restrict__ i0, int64_t N, int64_t K, uint32_t k0,
     uint32_t k1, uint32_t t, int noise, float inv_tau,
     __nv_bfloat16* __restrict__ What, float* __restrict__ gbuf,
@@ -274,7 +309,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
       const int64_t c = base + 32 * j;
       float l[L], gz[L], y[L], cand[5];
 #pragma unroll
-      for (int p = 0; p < L; ++p) l[p] = __ldg(logits + p * NK + c);
+      for (int p = 0; p < L; ++p) l[p] = St<TS>::ld(logits + p * NK + c);
       const int lev0 = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
       noise1<L>(c, t, k0, k1, noise, gz);
       candidates<MODE>(lev0, cand);
@@ -308,19 +343,27 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 // async copies (each lane copies exactly the pieces it will read) while the
 // current group is computed, so the loads of one group overlap the
 // arithmetic of the previous one.  Every global access is 16 bytes wide.
-template <int MODE>
+template <int MODE, typename TS = float>
 struct BwdCfg {
   static constexpr int L = GridT<MODE>::L;
-  static constexpr int PLANES = 1 + 3 * L;  // dW, logits, momenta, noise
-  static constexpr int BUF = PLANES * 512 + (MODE == GRID_3BIT_LOCAL ? 128 : 0);
+  // per-warp staging of one group: dW, logits, momenta, noise (, i0); the
+  // logit and momentum planes take 128 sizeof(TS) bytes each
+  static constexpr int SP = 128 * (int)sizeof(TS);
+  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * SP, OFF_G = OFF_M + L * SP;
+  static constexpr int OFF_I = OFF_G + L * 512;
+  static constexpr int BUF = OFF_I + (MODE == GRID_3BIT_LOCAL ? 128 : 0);
   static constexpr int WARPS = L == 5 ? 4 : 8;  // warps per CTA
   static constexpr int CTAS = L == 5 ? 3 : 2;   // CTAs per SM
   static constexpr int SMEM = WARPS * 2 * BUF;
 };
 
-template <int MODE, bool DBG, bool NEXT>
-__global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
-    k_backward_lion(float* __restrict__ logits, float* __restrict__ mom,
+// With TS = bf16 (the reduced-memory state) the updated logits are rounded
+// stochastically, thresholds from the low 9 bits of the Philox words of
+// step t + 1 (the words of the next step's noise), and the momenta to
+// nearest.
+template <int MODE, bool DBG, bool NEXT, typename TS>
+__global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>::CTAS)
+    k_backward_lion(TS* __restrict__ logits, TS* __restrict__ mom,
                     float* __restrict__ s, float* __restrict__ ms,
                     const int8_t* __restrict__ i0, const float* __restrict__ dW,
                     float* __restrict__ gbuf, int64_t N, int64_t K, uint32_t k0,
@@ -328,8 +371,9 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
                     float inv_tau_next, float lr, float b1, float omb1, float b2,
                     float omb2, __nv_bfloat16* __restrict__ What,
                     float* __restrict__ dl_dbg, float* __restrict__ ds_dbg) {
-  using C = BwdCfg<MODE>;
+  using C = BwdCfg<MODE, TS>;
   constexpr int L = C::L;
+  constexpr bool S16 = sizeof(TS) == 2;
   extern __shared__ __align__(16) uint8_t bwd_smem[];
   const int64_t NK = N * K, G = K / kGroup, groups = N * G;
   const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
@@ -341,14 +385,20 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
     const int64_t c = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
     const uint32_t d = wbuf + (uint32_t)(buf * C::BUF + 16 * lane);
     cp_async16(d, dW + c);
+    const uint32_t ds_ = wbuf + (uint32_t)(buf * C::BUF + (S16 ? 8 : 16) * lane);
 #pragma unroll
     for (int p = 0; p < L; ++p) {
-      cp_async16(d + (uint32_t)((1 + p) * 512), logits + p * NK + c);
-      cp_async16(d + (uint32_t)((1 + L + p) * 512), mom + p * NK + c);
-      cp_async16(d + (uint32_t)((1 + 2 * L + p) * 512), gbuf + p * NK + c);
+      if (S16) {
+        cp_async8(ds_ + (uint32_t)(C::OFF_L + p * C::SP), logits + p * NK + c);
+        cp_async8(ds_ + (uint32_t)(C::OFF_M + p * C::SP), mom + p * NK + c);
+      } else {
+        cp_async16(ds_ + (uint32_t)(C::OFF_L + p * C::SP), logits + p * NK + c);
+        cp_async16(ds_ + (uint32_t)(C::OFF_M + p * C::SP), mom + p * NK + c);
+      }
+      cp_async16(d + (uint32_t)(C::OFF_G + p * 512), gbuf + p * NK + c);
     }
     if (MODE == GRID_3BIT_LOCAL)
-      cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::PLANES * 512 + 4 * lane), i0 + c);
+      cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::OFF_I + 4 * lane), i0 + c);
   };
   int64_t gi = warp;
   if (gi < groups) prefetch(gi, 0);
@@ -358,6 +408,7 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
     cp_async_commit();
     cp_async_wait<1>();  // this lane's copies of group gi have landed
     const uint8_t* sb = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
+    const uint8_t* sb_s = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + (S16 ? 8 : 16) * lane;
     const int64_t c0 = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
     const float sg = s[gi];
     const float msg = ms[gi];
@@ -365,21 +416,49 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
     *reinterpret_cast<float4*>(Dr) = *reinterpret_cast<const float4*>(sb);
 #pragma unroll
     for (int p = 0; p < L; ++p) {
-      *reinterpret_cast<float4*>(Lr[p]) = *reinterpret_cast<const float4*>(sb + (1 + p) * 512);
-      *reinterpret_cast<float4*>(Mr[p]) =
-          *reinterpret_cast<const float4*>(sb + (1 + L + p) * 512);
+      if (S16) {
+        const uint2 lu = *reinterpret_cast<const uint2*>(sb_s + C::OFF_L + p * C::SP);
+        const uint2 mu = *reinterpret_cast<const uint2*>(sb_s + C::OFF_M + p * C::SP);
+        Lr[p][0] = __uint_as_float(lu.x << 16);
+        Lr[p][1] = __uint_as_float(lu.x & 0xFFFF0000u);
+        Lr[p][2] = __uint_as_float(lu.y << 16);
+        Lr[p][3] = __uint_as_float(lu.y & 0xFFFF0000u);
+        Mr[p][0] = __uint_as_float(mu.x << 16);
+        Mr[p][1] = __uint_as_float(mu.x & 0xFFFF0000u);
+        Mr[p][2] = __uint_as_float(mu.y << 16);
+        Mr[p][3] = __uint_as_float(mu.y & 0xFFFF0000u);
+      } else {
+        *reinterpret_cast<float4*>(Lr[p]) =
+            *reinterpret_cast<const float4*>(sb + C::OFF_L + p * C::SP);
+        *reinterpret_cast<float4*>(Mr[p]) =
+            *reinterpret_cast<const float4*>(sb + C::OFF_M + p * C::SP);
+      }
       *reinterpret_cast<float4*>(Gr[p]) =
-          *reinterpret_cast<const float4*>(sb + (1 + 2 * L + p) * 512);
+          *reinterpret_cast<const float4*>(sb + C::OFF_G + p * 512);
     }
     int lev[4] = {0, 0, 0, 0};
     if (MODE == GRID_3BIT_LOCAL) {
       const uint32_t b4 = *reinterpret_cast<const uint32_t*>(
-          bwd_smem + wic * 2 * C::BUF + buf * C::BUF + C::PLANES * 512 + 4 * lane);
+          bwd_smem + wic * 2 * C::BUF + buf * C::BUF + C::OFF_I + 4 * lane);
 #pragma unroll
       for (int j = 0; j < 4; ++j) lev[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
     float gnext[NEXT ? 4 : 1][L];
-    if (NEXT) {
+    uint32_t rsr[S16 ? 4 : 1][L];  // stochastic-rounding thresholds (bf16 state)
+    if (S16) {
+      // the Philox words of step t + 1 give the next step's noise (NEXT) and
+      // the rounding thresholds of this step's update
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t wd[5];
+        coord_words5((uint64_t)(c0 + j), t_next, k0, k1, L == 5, wd);
+#pragma unroll
+        for (int p = 0; p < L; ++p) {
+          rsr[S16 ? j : 0][p] = wd[p];
+          if (NEXT) gnext[NEXT ? j : 0][p] = noise ? gumbel(word_to_unit(wd[p])) : 0.f;
+        }
+      }
+    } else if (NEXT) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) noise1<L>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
     }
@@ -419,6 +498,10 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
       for (int p = 0; p < L; ++p) {
         float th = l[p], mm = Mr[p][j];
         lion_update(th, mm, dl[p], lr, b1, omb1, b2, omb2);
+        if (S16) {
+          th = bf16_sr(th, rsr[S16 ? j : 0][p]);
+          mm = bf16_rn(mm);
+        }
         Lo[p][j] = th;
         Mo[p][j] = mm;
         if (DBG) Do[DBG ? p : 0][j] = dl[p];
@@ -426,8 +509,18 @@ __global__ void __launch_bounds__(BwdCfg<MODE>::WARPS * 32, BwdCfg<MODE>::CTAS)
     }
 #pragma unroll
     for (int p = 0; p < L; ++p) {
-      *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(Lo[p]);
-      *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(Mo[p]);
+      if (S16) {
+        // the values are bf16 already: keep their top halves
+        *reinterpret_cast<uint2*>(logits + p * NK + c0) =
+            make_uint2((__float_as_uint(Lo[p][0]) >> 16) | (__float_as_uint(Lo[p][1]) & 0xFFFF0000u),
+                       (__float_as_uint(Lo[p][2]) >> 16) | (__float_as_uint(Lo[p][3]) & 0xFFFF0000u));
+        *reinterpret_cast<uint2*>(mom + p * NK + c0) =
+            make_uint2((__float_as_uint(Mo[p][0]) >> 16) | (__float_as_uint(Mo[p][1]) & 0xFFFF0000u),
+                       (__float_as_uint(Mo[p][2]) >> 16) | (__float_as_uint(Mo[p][3]) & 0xFFFF0000u));
+      } else {
+        *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(Lo[p]);
+        *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(Mo[p]);
+      }
       if (DBG)
         *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
             *reinterpret_cast<float4*>(Do[DBG ? p : 0]);
@@ -485,8 +578,8 @@ __device__ __forceinline__ int hard_level(const float* l, int lev0) {
 
 // Level codes of the hard choice (argmax of the logits, no noise), four
 // coordinates per thread.
-template <int MODE>
-__global__ void __launch_bounds__(256) k_hard_codes(const float* __restrict__ logits,
+template <int MODE, typename TS>
+__global__ void __launch_bounds__(256) k_hard_codes(const TS* __restrict__ logits,
                                                     const int8_t* __restrict__ i0,
                                                     int64_t NK, int8_t* __restrict__ code) {
   constexpr int L = GridT<MODE>::L;
@@ -495,7 +588,7 @@ __global__ void __launch_bounds__(256) k_hard_codes(const float* __restrict__ lo
     const int64_t c0 = q * 4;
     float4 lp[L];
 #pragma unroll
-    for (int p = 0; p < L; ++p) lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
+    for (int p = 0; p < L; ++p) lp[p] = St<TS>::ld4(logits + p * NK + c0);
     char4 iv = make_char4(0, 0, 0, 0);
     if (MODE == GRID_3BIT_LOCAL) iv = *reinterpret_cast<const char4*>(i0 + c0);
     const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
@@ -568,9 +661,9 @@ __global__ void __launch_bounds__(256) k_scale_lion(const int8_t* __restrict__ c
 // 2-bit / ternary: 16 codes -> one 32-bit word per thread.
 // 3-bit: 32 codes -> three 32-bit words per thread.  Codes never straddle
 // rows because K is a multiple of 128.
-template <int MODE>
+template <int MODE, typename TS>
 __global__ void __launch_bounds__(256) k_harden_pack(
-    const float* __restrict__ logits, const int8_t* __restrict__ i0,
+    const TS* __restrict__ logits, const int8_t* __restrict__ i0,
     int64_t N, int64_t K, uint32_t* __restrict__ packed) {
   constexpr int L = GridT<MODE>::L;
   constexpr int CPT = (MODE == GRID_3BIT_LOCAL) ? 32 : 16;  // codes / thread
@@ -584,7 +677,7 @@ __global__ void __launch_bounds__(256) k_harden_pack(
       float4 lp[L];
 #pragma unroll
       for (int p = 0; p < L; ++p)
-        lp[p] = __ldg(reinterpret_cast<const float4*>(logits + p * NK + c0 + j4 * 4));
+        lp[p] = St<TS>::ld4(logits + p * NK + c0 + j4 * 4);
       char4 iv = make_char4(0, 0, 0, 0);
       if (MODE == GRID_3BIT_LOCAL)
         iv = __ldg(reinterpret_cast<const char4*>(i0 + c0 + j4 * 4));
@@ -617,9 +710,9 @@ __global__ void __launch_bounds__(256) k_harden_pack(
 }
 
 // bf16(s * level) of the hard choice, four coordinates per thread
-template <int MODE>
+template <int MODE, typename TS>
 __global__ void __launch_bounds__(256) k_hard_weight(
-    const float* __restrict__ logits, const float* __restrict__ s,
+    const TS* __restrict__ logits, const float* __restrict__ s,
     const int8_t* __restrict__ i0, int64_t N, int64_t K,
     __nv_bfloat16* __restrict__ What) {
   constexpr int L = GridT<MODE>::L;
@@ -631,8 +724,7 @@ __global__ void __launch_bounds__(256) k_hard_weight(
     const float sg = s[n * G + k / kGroup];
     float4 lp[L];
 #pragma unroll
-    for (int p = 0; p < L; ++p)
-      lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
+    for (int p = 0; p < L; ++p) lp[p] = St<TS>::ld4(logits + p * NK + c0);
     char4 iv = make_char4(0, 0, 0, 0);
     if (MODE == GRID_3BIT_LOCAL) iv = *reinterpret_cast<const char4*>(i0 + c0);
     const int lev0[4] = {iv.x, iv.y, iv.z, iv.w};
@@ -972,39 +1064,57 @@ cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
 cudaError_t launch_init_state(int mode, const float* W32,
                               const int8_t* init_idx, int64_t N, int64_t K,
                               float* s, int8_t* i0, float* logits, int* err,
-                              cudaStream_t st) {
+                              cudaStream_t st, int state16) {
   const int64_t groups = N * (K / kGroup);
   const int blocks = grid_for(groups * 32, 256, 8192);
-  switch (mode) {
-    case GRID_2BIT:
-      k_init_state<GRID_2BIT><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s,
-                                                       i0, logits, err);
+  __nv_bfloat16* l16 = reinterpret_cast<__nv_bfloat16*>(logits);
+  switch (mode * 2 + (state16 ? 1 : 0)) {
+    case GRID_2BIT * 2:
+      k_init_state<GRID_2BIT, float><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, logits, err);
       break;
-    case GRID_TERNARY:
-      k_init_state<GRID_TERNARY><<<blocks, 256, 0, st>>>(W32, init_idx, N, K,
-                                                          s, i0, logits, err);
+    case GRID_2BIT * 2 + 1:
+      k_init_state<GRID_2BIT, __nv_bfloat16><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, l16, err);
+      break;
+    case GRID_TERNARY * 2:
+      k_init_state<GRID_TERNARY, float><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, logits, err);
+      break;
+    case GRID_TERNARY * 2 + 1:
+      k_init_state<GRID_TERNARY, __nv_bfloat16><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, l16, err);
+      break;
+    case GRID_3BIT_LOCAL * 2:
+      k_init_state<GRID_3BIT_LOCAL, float><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, logits, err);
       break;
     default:
-      k_init_state<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(
-          W32, init_idx, N, K, s, i0, logits, err);
+      k_init_state<GRID_3BIT_LOCAL, __nv_bfloat16><<<blocks, 256, 0, st>>>(W32, init_idx, N, K, s, i0, l16, err);
   }
   return cudaGetLastError();
+}
+
+template <int MODE, typename TS>
+static void soft_weight_ts(const StepArgs& a, __nv_bfloat16* What,
+                           float* gbuf, float* wsoft32, int blocks,
+                           cudaStream_t st) {
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+  const float inv_tau = 1.0f / a.tau;
+  const TS* lg = reinterpret_cast<const TS*>(a.logits);
+  if (wsoft32)
+    k_soft_weight<MODE, true, TS><<<blocks, 256, 0, st>>>(
+        lg, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
+        gbuf, wsoft32);
+  else
+    k_soft_weight<MODE, false, TS><<<blocks, 256, 0, st>>>(
+        lg, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
+        gbuf, nullptr);
 }
 
 template <int MODE>
 static void soft_weight_mode(const StepArgs& a, __nv_bfloat16* What,
                              float* gbuf, float* wsoft32, int blocks,
                              cudaStream_t st) {
-  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
-  const float inv_tau = 1.0f / a.tau;
-  if (wsoft32)
-    k_soft_weight<MODE, true><<<blocks, 256, 0, st>>>(
-        a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        gbuf, wsoft32);
+  if (a.state16)
+    soft_weight_ts<MODE, __nv_bfloat16>(a, What, gbuf, wsoft32, blocks, st);
   else
-    k_soft_weight<MODE, false><<<blocks, 256, 0, st>>>(
-        a.logits, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        gbuf, nullptr);
+    soft_weight_ts<MODE, float>(a, What, gbuf, wsoft32, blocks, st);
 }
 
 cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
@@ -1020,7 +1130,7 @@ cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
   return cudaGetLastError();
 }
 
-template <int MODE, bool NEXT>
+template <int MODE, bool NEXT, typename TS>
 static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
                           float lr, float b1, float b2, float tau_next,
                           __nv_bfloat16* What, float* dl_dbg, float* ds_dbg,
@@ -1029,23 +1139,25 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   const float inv_tau = 1.0f / a.tau;
   const float inv_tau_next = NEXT ? 1.0f / tau_next : 0.f;
   const float omb1 = 1.0f - b1, omb2 = 1.0f - b2;
-  using C = BwdCfg<MODE>;
+  using C = BwdCfg<MODE, TS>;
+  TS* lg = reinterpret_cast<TS*>(a.logits_w);
+  TS* mm = reinterpret_cast<TS*>(a.mom);
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaFuncSetAttribute(k_backward_lion<MODE, true, NEXT>,
+    cudaFuncSetAttribute(k_backward_lion<MODE, true, NEXT, TS>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    cudaFuncSetAttribute(k_backward_lion<MODE, false, NEXT>,
+    cudaFuncSetAttribute(k_backward_lion<MODE, false, NEXT, TS>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     attr_set = true;
   }
   if (dl_dbg) {
-    k_backward_lion<MODE, true, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
+    k_backward_lion<MODE, true, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
+        lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         dl_dbg, ds_dbg);
   } else {
-    k_backward_lion<MODE, false, NEXT><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        a.logits_w, a.mom, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
+    k_backward_lion<MODE, false, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
+        lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         nullptr, nullptr);
   }
@@ -1056,12 +1168,22 @@ static void backward_dispatch(const StepArgs& a, const float* dW, float* gbuf,
                               float lr, float b1, float b2, float tau_next,
                               __nv_bfloat16* What, float* dl_dbg,
                               float* ds_dbg, int blocks, cudaStream_t st) {
-  if (tau_next > 0.f)
-    backward_mode<MODE, true>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
-                              ds_dbg, blocks, st);
-  else
-    backward_mode<MODE, false>(a, dW, gbuf, lr, b1, b2, tau_next, What,
-                               dl_dbg, ds_dbg, blocks, st);
+  const bool next = tau_next > 0.f;
+  if (a.state16) {
+    if (next)
+      backward_mode<MODE, true, __nv_bfloat16>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+                                               ds_dbg, blocks, st);
+    else
+      backward_mode<MODE, false, __nv_bfloat16>(a, dW, gbuf, lr, b1, b2, tau_next, What,
+                                                dl_dbg, ds_dbg, blocks, st);
+  } else {
+    if (next)
+      backward_mode<MODE, true, float>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg,
+                                       blocks, st);
+    else
+      backward_mode<MODE, false, float>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+                                        ds_dbg, blocks, st);
+  }
 }
 
 cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
@@ -1090,23 +1212,31 @@ cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
 cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,
                                const float* logits, const float* s,
                                const int8_t* i0, __nv_bfloat16* What,
-                               cudaStream_t st) {
+                               cudaStream_t st, int state16) {
   const int blocks = grid_for(N * K / 4, 256, 4096);
-  switch (mode) {
-    case GRID_2BIT: k_hard_weight<GRID_2BIT><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
-    case GRID_TERNARY: k_hard_weight<GRID_TERNARY><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
-    default: k_hard_weight<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What);
+  const __nv_bfloat16* l16 = reinterpret_cast<const __nv_bfloat16*>(logits);
+  switch (mode * 2 + (state16 ? 1 : 0)) {
+    case GRID_2BIT * 2: k_hard_weight<GRID_2BIT, float><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
+    case GRID_2BIT * 2 + 1: k_hard_weight<GRID_2BIT, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, s, i0, N, K, What); break;
+    case GRID_TERNARY * 2: k_hard_weight<GRID_TERNARY, float><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
+    case GRID_TERNARY * 2 + 1: k_hard_weight<GRID_TERNARY, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, s, i0, N, K, What); break;
+    case GRID_3BIT_LOCAL * 2: k_hard_weight<GRID_3BIT_LOCAL, float><<<blocks, 256, 0, st>>>(logits, s, i0, N, K, What); break;
+    default: k_hard_weight<GRID_3BIT_LOCAL, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, s, i0, N, K, What);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_hard_codes(int mode, int64_t N, int64_t K, const float* logits,
-                              const int8_t* i0, int8_t* code, cudaStream_t st) {
+                              const int8_t* i0, int8_t* code, cudaStream_t st, int state16) {
   const int blocks = grid_for(N * K / 4, 256, 4096);
-  switch (mode) {
-    case GRID_2BIT: k_hard_codes<GRID_2BIT><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
-    case GRID_TERNARY: k_hard_codes<GRID_TERNARY><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
-    default: k_hard_codes<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(logits, i0, N * K, code);
+  const __nv_bfloat16* l16 = reinterpret_cast<const __nv_bfloat16*>(logits);
+  switch (mode * 2 + (state16 ? 1 : 0)) {
+    case GRID_2BIT * 2: k_hard_codes<GRID_2BIT, float><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
+    case GRID_2BIT * 2 + 1: k_hard_codes<GRID_2BIT, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, i0, N * K, code); break;
+    case GRID_TERNARY * 2: k_hard_codes<GRID_TERNARY, float><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
+    case GRID_TERNARY * 2 + 1: k_hard_codes<GRID_TERNARY, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, i0, N * K, code); break;
+    case GRID_3BIT_LOCAL * 2: k_hard_codes<GRID_3BIT_LOCAL, float><<<blocks, 256, 0, st>>>(logits, i0, N * K, code); break;
+    default: k_hard_codes<GRID_3BIT_LOCAL, __nv_bfloat16><<<blocks, 256, 0, st>>>(l16, i0, N * K, code);
   }
   return cudaGetLastError();
 }
@@ -1146,16 +1276,16 @@ cudaError_t launch_scale_lion(int mode, int64_t N, int64_t K, const int8_t* code
 
 cudaError_t launch_harden_pack(int mode, int64_t N, int64_t K,
                                const float* logits, const int8_t* i0,
-                               uint32_t* packed, cudaStream_t st) {
-  switch (mode) {
-    case GRID_2BIT:
-      k_harden_pack<GRID_2BIT><<<grid_for(N * K / 16, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
-      break;
-    case GRID_TERNARY:
-      k_harden_pack<GRID_TERNARY><<<grid_for(N * K / 16, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
-      break;
-    default:
-      k_harden_pack<GRID_3BIT_LOCAL><<<grid_for(N * K / 32, 256, 4096), 256, 0, st>>>(logits, i0, N, K, packed);
+                               uint32_t* packed, cudaStream_t st, int state16) {
+  const __nv_bfloat16* l16 = reinterpret_cast<const __nv_bfloat16*>(logits);
+  const int b16 = grid_for(N * K / 16, 256, 4096), b32 = grid_for(N * K / 32, 256, 4096);
+  switch (mode * 2 + (state16 ? 1 : 0)) {
+    case GRID_2BIT * 2: k_harden_pack<GRID_2BIT, float><<<b16, 256, 0, st>>>(logits, i0, N, K, packed); break;
+    case GRID_2BIT * 2 + 1: k_harden_pack<GRID_2BIT, __nv_bfloat16><<<b16, 256, 0, st>>>(l16, i0, N, K, packed); break;
+    case GRID_TERNARY * 2: k_harden_pack<GRID_TERNARY, float><<<b16, 256, 0, st>>>(logits, i0, N, K, packed); break;
+    case GRID_TERNARY * 2 + 1: k_harden_pack<GRID_TERNARY, __nv_bfloat16><<<b16, 256, 0, st>>>(l16, i0, N, K, packed); break;
+    case GRID_3BIT_LOCAL * 2: k_harden_pack<GRID_3BIT_LOCAL, float><<<b32, 256, 0, st>>>(logits, i0, N, K, packed); break;
+    default: k_harden_pack<GRID_3BIT_LOCAL, __nv_bfloat16><<<b32, 256, 0, st>>>(l16, i0, N, K, packed);
   }
   return cudaGetLastError();
 }

@@ -44,7 +44,7 @@ EXPORTS = [
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
-    "gsq_gptq", "gsq_init_gptq",
+    "gsq_gptq", "gsq_init_gptq", "gsq_init_bf16_state",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
@@ -93,6 +93,8 @@ _SIGS = {
     "gsq_scale_step": [_p, _f32, _f32, _f32],
     "gsq_gptq": [_p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _p, _p, _p],
     "gsq_init_gptq": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _u64, _p],
+    "gsq_init_bf16_state": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64,
+                            _p],
     "gsq_scale_run": [_p, _i64, _f32, _f32, _f32],
     "gsq_debug_scale_backward": [_p, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
@@ -204,8 +206,9 @@ def gsq_packed_bytes(grid_mode: int, N: int, K: int) -> int:
 
 
 def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
-             init_idx=None, seed: int = 0, stream=None) -> "Layer":
-    """W (N x K) and X (T x K): numpy fp32 or torch fp32/bf16, host or device."""
+             init_idx=None, seed: int = 0, stream=None, state_bf16: bool = False) -> "Layer":
+    """W (N x K) and X (T x K): numpy fp32 or torch fp32/bf16, host or device.
+    state_bf16 selects gsq_init_bf16_state (bf16 logits and momenta)."""
     wp, wdt, wk = _ptr_dtype(W)
     xp, xdt, xk = _ptr_dtype(X)
     N, K = int(W.shape[0]), int(W.shape[1])
@@ -226,11 +229,12 @@ def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
             ip = ik.ctypes.data
     ctx = C.c_void_p()
     st = _stream_ptr(stream)
-    _check(_lib.gsq_init(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group,
-                         grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
-           "gsq_init")
+    fn = _lib.gsq_init_bf16_state if state_bf16 else _lib.gsq_init
+    _check(fn(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group,
+              grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
+           "gsq_init_bf16_state" if state_bf16 else "gsq_init")
     del wk, xk, ik
-    return Layer(ctx, grid_mode, N, K, T, group)
+    return Layer(ctx, grid_mode, N, K, T, group, state16=state_bf16)
 
 
 def gsq_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT, damp: float = 0.01,
@@ -378,8 +382,9 @@ def gsq_gemm_bf16_abt(A, B, Cout, stream=None) -> None:
 class Layer:
     """A GSQ context for one linear layer (owner of the C handle)."""
 
-    def __init__(self, ctx, mode, N, K, T, group):
+    def __init__(self, ctx, mode, N, K, T, group, state16=False):
         self.ctx, self.mode, self.N, self.K, self.T, self.group = ctx, mode, N, K, T, group
+        self.state16 = bool(state16)
         self.G = K // group
         self.L = NUM_LOGITS[mode]
         self.Tp = (T + 63) // 64 * 64
@@ -396,6 +401,8 @@ class Layer:
 
     def _shape(self, which):
         spec, dt = self._SHAPES[which]
+        if self.state16 and which in (GSQ_DBG_LOGITS, GSQ_DBG_MOM):
+            dt = np.uint16  # bf16 bit patterns
         return tuple(getattr(self, d) for d in spec.split(",")), dt
 
     def get(self, which) -> np.ndarray:
