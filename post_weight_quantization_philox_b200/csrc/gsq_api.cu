@@ -51,9 +51,9 @@ struct gsq_ctx {
   double *partials = nullptr, *loss_hist = nullptr, *scratch = nullptr;
   unsigned* ticket = nullptr;
   int* err = nullptr;
-  float* gbuf = nullptr;  // Gumbel noise of the pending step (L x N x K)
+  float* gbuf = nullptr;  // probabilities of the pending step (L x N x K)
   float *wsoft32 = nullptr, *dl = nullptr, *ds = nullptr;  // debug, lazy
-  // What and gbuf hold the soft weight and noise of step what_t at
+  // What and gbuf hold the soft weight and probabilities of step what_t at
   // temperature what_tau (what_t < 0: nothing precomputed)
   int64_t what_t = -1;
   float what_tau = 0.f;
@@ -454,7 +454,8 @@ int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const void* X
 namespace {
 
 // One step t at temperature tau; with tau_next > 0 the backward also builds
-// the soft weight and noise of step t + 1 (which the next call then skips).
+// the soft weight and probabilities of step t + 1 (which the next call then
+// skips).
 int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
              float beta2) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;  // 32-bit counter word
@@ -885,7 +886,7 @@ int gsq_debug_backward(gsq_ctx* c, float tau, float lr, float beta1,
   int rc = debug_buffer(c, GSQ_DBG_DL, &p, &nb);
   if (!rc) rc = debug_buffer(c, GSQ_DBG_DS, &p, &nb);
   if (rc) return rc;
-  // the step's noise first (the backward takes it from the noise buffer)
+  // the step's soft weight first (the backward takes its probabilities)
   const StepArgs a = step_args(c, tau);
   if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
     CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));

@@ -242,6 +242,17 @@ __device__ __forceinline__ float coord_soft(const float* l, const float* g,
   }
 }
 
+// The unit value v from probabilities y, with the same operations in the same
+// order as coord_soft, so it equals the v coord_soft returned for them.
+template <int MODE>
+__device__ __forceinline__ float value_of(const float* y, const float* cand) {
+  if (MODE == GRID_TERNARY) return y[1] * (y[3] - y[2]);
+  float v = 0.f;
+#pragma unroll
+  for (int k = 0; k < GridT<MODE>::L; ++k) v = fmaf(y[k], cand[k], v);
+  return v;
+}
+
 template <int MODE>
 __device__ __forceinline__ void candidates(int lev0, float* cand) {
   if (MODE == GRID_2BIT) {
@@ -287,7 +298,9 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w)
 constexpr int kPerLane = kGroup / 32;
 
 // Soft weight (A1 + A2): w = bf16(s * v((l + g) / tau)).  When gbuf is given
-// the step's Gumbel noise is kept there (L planes) for the backward.
+// the step's probabilities y = softmax((l + g) / tau) are kept there (L
+// planes) for the backward, which then needs neither the noise nor a second
+// softmax.
 template <int MODE, bool DBG, typename TS>
 __global__ void __launch_bounds__(256) k_soft_weight(
     const TS* __restrict__ logits, const float* __restrict__ s,
@@ -317,7 +330,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
       What[c] = __float2bfloat16_rn(w);
       if (gbuf) {
 #pragma unroll
-        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = gz[p];
+        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = y[p];
       }
       if (DBG) wsoft32[c] = w;
     }
@@ -326,15 +339,15 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 
 // ------------------------------------------------- backward + Lion (A5)
 
-// Takes the step's Gumbel noise from gbuf (written by the soft weight of the
-// same step), rebuilds the probabilities and forms
+// Takes the step's probabilities y from gbuf (written by the soft weight of
+// the same step, from the pre-update logits and the step's noise) and forms
 //   a = s dW / tau,  dl_k = a y_k sum_j y_j (c_k - c_j)   (categorical),
 //   dl_mask1 = a (q+ - q-) p1 p0 = -dl_mask0, dl_sign+ = 2 a p1 q+ q- =
 //   -dl_sign- (ternary),  ds = sum over the group of dW v (warp shuffle),
 // then applies Lion to the logits and the group scale.  With NEXT it also
 // computes the soft weight of step t+1 from the updated logits and scale
-// (fresh Philox noise, kept in gbuf for the next backward): the same values
-// a separate soft-weight launch would produce.  All loads of the group are
+// (fresh Philox noise; its probabilities go to gbuf for the next backward):
+// the same values a separate soft-weight launch would produce.  All loads of the group are
 // issued first and the next step's noise (which needs none of them) is
 // computed while they are in flight.
 // Backward + Lion (A5), optionally fused with the next step's A1 + A2.  One
@@ -346,7 +359,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 template <int MODE, typename TS = float>
 struct BwdCfg {
   static constexpr int L = GridT<MODE>::L;
-  // per-warp staging of one group: dW, logits, momenta, noise (, i0); the
+  // per-warp staging of one group: dW, logits, momenta, probabilities (, i0); the
   // logit and momentum planes take 128 sizeof(TS) bytes each
   static constexpr int SP = 128 * (int)sizeof(TS);
   static constexpr int OFF_L = 512, OFF_M = OFF_L + L * SP, OFF_G = OFF_M + L * SP;
@@ -466,15 +479,15 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float l[L], gz[L], y[L], cand[5];
+      float l[L], y[L], cand[5];
 #pragma unroll
       for (int p = 0; p < L; ++p) {
         l[p] = Lr[p][j];
-        gz[p] = Gr[p][j];
+        y[p] = Gr[p][j];  // this step's probabilities, kept by its soft weight
       }
       const float dw = Dr[j];
       candidates<MODE>(lev[j], cand);
-      const float v = coord_soft<MODE>(l, gz, inv_tau, cand, y);
+      const float v = value_of<MODE>(y, cand);
       ds_part = fmaf(dw, v, ds_part);
       const float a = sg * dw * inv_tau;
       float dl[L];
@@ -535,21 +548,21 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
       if (DBG) ds_dbg[gi] = ds;
     }
     if (NEXT) {
-      float w[4];
+      float w[4], yn[4][L];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float l[L], y[L], cand[5];
+        float l[L], cand[5];
 #pragma unroll
         for (int p = 0; p < L; ++p) l[p] = Lo[p][j];
         candidates<MODE>(lev[j], cand);
-        w[j] = s_new * coord_soft<MODE>(l, gnext[NEXT ? j : 0], inv_tau_next, cand, y);
+        w[j] = s_new * coord_soft<MODE>(l, gnext[NEXT ? j : 0], inv_tau_next, cand, yn[j]);
       }
       store_bf16x4(What + c0, w);
 #pragma unroll
       for (int p = 0; p < L; ++p) {
-        float4 g4 = make_float4(gnext[NEXT ? 0 : 0][p], gnext[NEXT ? 1 : 0][p],
-                                gnext[NEXT ? 2 : 0][p], gnext[NEXT ? 3 : 0][p]);
-        *reinterpret_cast<float4*>(gbuf + p * NK + c0) = g4;
+        // the next step's probabilities, for its backward
+        float4 y4 = make_float4(yn[0][p], yn[1][p], yn[2][p], yn[3][p]);
+        *reinterpret_cast<float4*>(gbuf + p * NK + c0) = y4;
       }
     }
   }
