@@ -472,6 +472,93 @@ GSQ_API int gsq_block_quantize(const float* x_in, const void* const* W, int64_t 
                                void* const* packed, uint16_t* const* scales_f16,
                                float* const* scales_f32, double* stats, void* stream);
 
+/* ------------------------------------------------ GGUF K-Quant formats --
+ * GSQ on llama.cpp's K-Quant formats: start from an existing K-Quant (e.g. a
+ * released GGUF checkpoint), optimise with the GSQ step, and project the
+ * result back into the same format (agihunt.info summary, optimisation and
+ * results paragraphs: Qwen3-8B Q2_K and Q3_K_M, format unchanged).
+ *
+ * Formats (super-blocks of 256 consecutive weights of a row, 16 sub-blocks of
+ * 16; K % 256 == 0):
+ *   GSQ_KQ_Q2_K  w = d sc_j q - dmin m_j, q 0..3, sc_j, m_j 0..15, d, dmin
+ *                fp16; 84 bytes per super-block
+ *   GSQ_KQ_Q3_K  w = d sc_j q, q -4..3, sc_j -32..31, d fp16; 110 bytes
+ * in the GGUF block encodings of Q2_K / Q3_K (blocks in row-major order of
+ * the super-blocks).
+ * State: per coordinate logits over q (Q2_K: 4; Q3_K: 5 local shifts
+ * -2..+2 around the start code, clamped to [-4, 3]), +2 on the start code;
+ * per sub-block continuous a_j (and b_j for Q2_K), starting at d sc_j and
+ * dmin m_j.  A step: soft weight w = bf16(a_j sum_k y_k c_k - b_j) with
+ * Philox Gumbel noise (the 2-bit grid's words for Q2_K, the 3-bit local
+ * grid's for Q3_K), the layer loss ||X w^T - X W^T||^2 and dW as gsq_step,
+ * dl_k = (a_j dw / tau) y_k sum_m y_m (c_k - c_m), da_j = sum dw v,
+ * db_j = -sum dw, Lion on all of them.  Export (the projection back): hard
+ * codes by argmax (first maximum); d = fp16(max_j a_j / 15), sc_j =
+ * rint(a_j / d) in 0..15 (a_j, b_j clamped at 0), dmin and m_j likewise
+ * (Q2_K); d = fp16(max_j |a_j| / 31), sc_j = rint(a_j / d) in -32..31 (Q3_K).
+ *
+ * gsq_kq_block_bytes: bytes of the N x K weight in the format.
+ * gsq_kq_init: W (N x K), X (T x K) fp32/bf16, host or device; start_blocks
+ *   (nullable, host or device) the starting K-Quant; NULL starts from the
+ *   min-max K-Quant of W: per sub-block a = (max w - min(0, min w)) / 3 and
+ *   b = -min(0, min w) (Q2_K) or a = -w_e / 4 with w_e the largest-magnitude
+ *   weight (Q3_K), projected as above, each weight's code its nearest level
+ *   (first on ties).  Syncs.
+ * gsq_kq_step / gsq_kq_run / gsq_kq_last_loss: as gsq_step / gsq_run /
+ *   gsq_last_loss (gsq_kq_run is a loop of steps).
+ * gsq_kq_export: the projected blocks (host or device).  Syncs.
+ * gsq_kq_start_blocks: the starting blocks.  Syncs.
+ * gsq_kq_recon_error: abs = ||bf16(X) Wq^T - Y_ref||^2 and rel = abs /
+ *   ||Y_ref||^2 of the exported (which = 0) or starting (1) blocks.  Syncs.
+ * gsq_kq_dequant: bf16 weight (N x K) of blocks, w = bf16((d sc_j) q -
+ *   dmin m_j) with each product and the difference rounded in fp32.  Syncs.
+ * gsq_kq_debug_get / _set (GSQ_KQ_DBG_*), gsq_kq_debug_soft_weight (fills
+ *   GSQ_KQ_DBG_WSOFT32), gsq_kq_debug_backward (soft weight of the current
+ *   step, then backward + Lion from the current dW, filling DL, DA, DB),
+ *   gsq_kq_debug_noise: test entry points as their single-layer
+ *   counterparts.
+ * Errors: GSQ_ERR_INVALID_ARG (sizes, K % 256, format, null pointers),
+ * GSQ_ERR_UNSUPPORTED (no sm_100 device), GSQ_ERR_OOM, GSQ_ERR_NONFINITE,
+ * GSQ_ERR_STATE, GSQ_ERR_CUDA.
+ */
+enum { GSQ_KQ_Q2_K = 0, GSQ_KQ_Q3_K = 1 };
+enum {
+  GSQ_KQ_DBG_LOGITS = 0, /* L x N x K fp32 */
+  GSQ_KQ_DBG_MOM = 1,    /* L x N x K fp32 */
+  GSQ_KQ_DBG_A = 2,      /* N x K/16 fp32 sub-block scale a_j */
+  GSQ_KQ_DBG_MA = 3,
+  GSQ_KQ_DBG_B = 4,      /* N x K/16 fp32 sub-block offset b_j (Q2_K) */
+  GSQ_KQ_DBG_MB = 5,
+  GSQ_KQ_DBG_Q0 = 6,     /* N x K int8 start codes */
+  GSQ_KQ_DBG_WHAT = 7,   /* N x K bf16 soft weight */
+  GSQ_KQ_DBG_DW = 8,     /* N x K fp32 weight gradient */
+  GSQ_KQ_DBG_DL = 9,     /* L x N x K fp32 logit gradient */
+  GSQ_KQ_DBG_DA = 10,    /* N x K/16 fp32 */
+  GSQ_KQ_DBG_DB = 11,    /* N x K/16 fp32 */
+  GSQ_KQ_DBG_WSOFT32 = 12 /* N x K fp32 soft weight before rounding */
+};
+typedef struct gsq_kq gsq_kq;
+GSQ_API int gsq_kq_block_bytes(int format, int64_t N, int64_t K, size_t* bytes);
+GSQ_API int gsq_kq_init(gsq_kq** out, const void* W, int w_dtype, const void* X, int x_dtype,
+                        int64_t N, int64_t K, int64_t T, int format, const void* start_blocks,
+                        uint64_t seed, void* stream);
+GSQ_API int gsq_kq_step(gsq_kq* ctx, float tau, float lr, float beta1, float beta2);
+GSQ_API int gsq_kq_run(gsq_kq* ctx, const float* taus, int64_t n, float lr, float beta1,
+                       float beta2);
+GSQ_API int gsq_kq_last_loss(gsq_kq* ctx, double* loss);
+GSQ_API int gsq_kq_export(gsq_kq* ctx, void* blocks);
+GSQ_API int gsq_kq_start_blocks(gsq_kq* ctx, void* blocks);
+GSQ_API int gsq_kq_recon_error(gsq_kq* ctx, int which, double* abs_err, double* rel_err);
+GSQ_API int gsq_kq_dequant(int format, const void* blocks, int64_t N, int64_t K, void* W_bf16,
+                           void* stream);
+GSQ_API int gsq_kq_debug_get(gsq_kq* ctx, int which, void* host, size_t bytes);
+GSQ_API int gsq_kq_debug_set(gsq_kq* ctx, int which, const void* host, size_t bytes);
+GSQ_API int gsq_kq_debug_soft_weight(gsq_kq* ctx, float tau);
+GSQ_API int gsq_kq_debug_backward(gsq_kq* ctx, float tau, float lr, float beta1, float beta2);
+GSQ_API int gsq_kq_debug_noise(gsq_kq* ctx, int on);
+GSQ_API int gsq_kq_get_step(gsq_kq* ctx, uint64_t* t);
+GSQ_API int gsq_kq_destroy(gsq_kq* ctx);
+
 /*
  * gsq_uniforms_noalloc -- the L Philox uniforms of coords
  * [coord0, coord0 + count) at step t for grid_mode and seed (the values

@@ -219,9 +219,10 @@ class KqState:
     q0: np.ndarray       # (N, K) int64: start codes
     seed: int = 0
     t: int = 0
+    row0: int = 0        # first row of the layer (noise is keyed by the global coordinate)
 
 
-def init_state(fmt: int, blocks, N: int, K: int, seed: int = 0) -> KqState:
+def init_state(fmt: int, blocks, N: int, K: int, seed: int = 0, row0: int = 0) -> KqState:
     q, sc, m, d, dm = decode(fmt, blocks)
     a = (d[:, None] * sc.astype(F32)).astype(F32).reshape(N, K // 16)
     b = (dm[:, None] * m.astype(F32)).astype(F32).reshape(N, K // 16)
@@ -234,7 +235,7 @@ def init_state(fmt: int, blocks, N: int, K: int, seed: int = 0) -> KqState:
     else:
         logits[2] = 2.0
     return KqState(fmt, N, K, logits, np.zeros_like(logits), a, np.zeros_like(a), b,
-                   np.zeros_like(b), q, seed)
+                   np.zeros_like(b), q, seed, 0, row0)
 
 
 def candidates(st: KqState) -> np.ndarray:
@@ -247,7 +248,7 @@ def candidates(st: KqState) -> np.ndarray:
 
 def noise(st: KqState, t: int) -> np.ndarray:
     mode = GRID_2BIT if st.fmt == Q2_K else GRID_3BIT_LOCAL
-    u = uniforms(mode, st.seed, t, 0, st.N * st.K).astype(np.float64)
+    u = uniforms(mode, st.seed, t, st.row0 * st.K, st.N * st.K).astype(np.float64)
     return (-np.log(-np.log(u))).T.reshape(-1, st.N, st.K)
 
 

@@ -52,6 +52,10 @@ EXPORTS = [
     "gsq_attn_recon_error", "gsq_attn_harden_pack", "gsq_attn_debug_get",
     "gsq_attn_debug_set", "gsq_attn_get_step", "gsq_attn_destroy",
     "gsq_dequant", "gsq_block_forward", "gsq_block_quantize",
+    "gsq_kq_block_bytes", "gsq_kq_init", "gsq_kq_step", "gsq_kq_run", "gsq_kq_last_loss",
+    "gsq_kq_export", "gsq_kq_start_blocks", "gsq_kq_recon_error", "gsq_kq_dequant",
+    "gsq_kq_debug_get", "gsq_kq_debug_set", "gsq_kq_debug_soft_weight",
+    "gsq_kq_debug_backward", "gsq_kq_debug_noise", "gsq_kq_get_step", "gsq_kq_destroy",
 ]
 
 
@@ -122,6 +126,22 @@ _SIGS = {
     "gsq_attn_get_step": [_p, C.POINTER(_u64)],
     "gsq_attn_destroy": [_p],
     "gsq_dequant": [_i32, _p, _p, _i64, _i64, _i32, _p, _p],
+    "gsq_kq_block_bytes": [_i32, _i64, _i64, C.POINTER(_sz)],
+    "gsq_kq_init": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _p, _u64, _p],
+    "gsq_kq_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_kq_run": [_p, _p, _i64, _f32, _f32, _f32],
+    "gsq_kq_last_loss": [_p, C.POINTER(C.c_double)],
+    "gsq_kq_export": [_p, _p],
+    "gsq_kq_start_blocks": [_p, _p],
+    "gsq_kq_recon_error": [_p, _i32, C.POINTER(C.c_double), C.POINTER(C.c_double)],
+    "gsq_kq_dequant": [_i32, _p, _i64, _i64, _p, _p],
+    "gsq_kq_debug_get": [_p, _i32, _p, _sz],
+    "gsq_kq_debug_set": [_p, _i32, _p, _sz],
+    "gsq_kq_debug_soft_weight": [_p, _f32],
+    "gsq_kq_debug_backward": [_p, _f32, _f32, _f32, _f32],
+    "gsq_kq_debug_noise": [_p, _i32],
+    "gsq_kq_get_step": [_p, C.POINTER(_u64)],
+    "gsq_kq_destroy": [_p],
     "gsq_block_forward": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, C.c_double, _f32,
                           _p, _p, _p],
     "gsq_block_quantize": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, C.c_double, _f32,
@@ -809,3 +829,140 @@ def gsq_block_quantize(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn,
                      recon=(stats[5 * j + 2], stats[5 * j + 3]), ms=stats[5 * j + 4])
           for j, name in enumerate(BLOCK_STAGES)}
     return {"x_out": x_out, "packed": packed, "scales": scales, "stats": st}
+
+
+# ------------------------------------------------------- GGUF K-Quant formats
+
+GSQ_KQ_Q2_K, GSQ_KQ_Q3_K = 0, 1
+(GSQ_KQ_DBG_LOGITS, GSQ_KQ_DBG_MOM, GSQ_KQ_DBG_A, GSQ_KQ_DBG_MA, GSQ_KQ_DBG_B, GSQ_KQ_DBG_MB,
+ GSQ_KQ_DBG_Q0, GSQ_KQ_DBG_WHAT, GSQ_KQ_DBG_DW, GSQ_KQ_DBG_DL, GSQ_KQ_DBG_DA, GSQ_KQ_DBG_DB,
+ GSQ_KQ_DBG_WSOFT32) = range(13)
+
+
+def gsq_kq_block_bytes(fmt: int, N: int, K: int) -> int:
+    b = C.c_size_t()
+    _check(_lib.gsq_kq_block_bytes(fmt, N, K, C.byref(b)), "gsq_kq_block_bytes")
+    return b.value
+
+
+def gsq_kq_init(W, X, fmt: int = GSQ_KQ_Q2_K, start_blocks=None, seed: int = 0,
+                stream=None) -> "KqLayer":
+    """GSQ on a K-Quant format: W (N x K), X (T x K) as for gsq_init;
+    start_blocks (uint8 numpy array or torch tensor of gsq_kq_block_bytes
+    bytes) or None for the min-max K-Quant of W."""
+    wp, wdt, wk = _ptr_dtype(W)
+    xp, xdt, xk = _ptr_dtype(X)
+    N, K = int(W.shape[0]), int(W.shape[1])
+    T = int(X.shape[0])
+    if int(X.shape[1]) != K:
+        raise ValueError("X and W disagree on K")
+    sp, sk = None, None
+    if start_blocks is not None:
+        sk = start_blocks if hasattr(start_blocks, "data_ptr") else np.ascontiguousarray(
+            start_blocks, np.uint8)
+        nb = sk.numel() * sk.element_size() if hasattr(sk, "numel") else sk.nbytes
+        if nb != gsq_kq_block_bytes(fmt, N, K):
+            raise ValueError("start_blocks has the wrong size")
+        sp = _host_ptr(sk)
+    ctx = C.c_void_p()
+    _check(_lib.gsq_kq_init(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, fmt, sp,
+                            seed & 0xFFFFFFFFFFFFFFFF, _stream_ptr(stream)), "gsq_kq_init")
+    del wk, xk, sk
+    return KqLayer(ctx, fmt, N, K, T)
+
+
+def gsq_kq_dequant(fmt: int, blocks, N: int, K: int, out=None, stream=None):
+    """bf16 weight (N x K) of K-Quant blocks; a device tensor unless `out` is given."""
+    import torch
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    b = blocks if hasattr(blocks, "data_ptr") else np.ascontiguousarray(blocks, np.uint8)
+    nb = b.numel() * b.element_size() if hasattr(b, "numel") else b.nbytes
+    if nb != gsq_kq_block_bytes(fmt, N, K) or tuple(out.shape) != (N, K):
+        raise ValueError("gsq_kq_dequant: sizes do not match N x K")
+    _check(_lib.gsq_kq_dequant(fmt, _host_ptr(b), N, K, out.data_ptr(), _stream_ptr(stream)),
+           "gsq_kq_dequant")
+    return out
+
+
+class KqLayer:
+    """A GSQ context on a K-Quant format (owner of the C handle)."""
+
+    def __init__(self, ctx, fmt, N, K, T):
+        self.ctx, self.fmt, self.N, self.K, self.T = ctx, fmt, N, K, T
+        self.L = 4 if fmt == GSQ_KQ_Q2_K else 5
+        self.S = K // 16
+
+    _SHAPES = {GSQ_KQ_DBG_LOGITS: ("L,N,K", np.float32), GSQ_KQ_DBG_MOM: ("L,N,K", np.float32),
+               GSQ_KQ_DBG_A: ("N,S", np.float32), GSQ_KQ_DBG_MA: ("N,S", np.float32),
+               GSQ_KQ_DBG_B: ("N,S", np.float32), GSQ_KQ_DBG_MB: ("N,S", np.float32),
+               GSQ_KQ_DBG_Q0: ("N,K", np.int8), GSQ_KQ_DBG_WHAT: ("N,K", np.uint16),
+               GSQ_KQ_DBG_DW: ("N,K", np.float32), GSQ_KQ_DBG_DL: ("L,N,K", np.float32),
+               GSQ_KQ_DBG_DA: ("N,S", np.float32), GSQ_KQ_DBG_DB: ("N,S", np.float32),
+               GSQ_KQ_DBG_WSOFT32: ("N,K", np.float32)}
+
+    def _shape(self, which):
+        spec, dt = self._SHAPES[which]
+        return tuple(getattr(self, d) for d in spec.split(",")), dt
+
+    def get(self, which) -> np.ndarray:
+        shape, dt = self._shape(which)
+        out = np.zeros(shape, dt)
+        _check(_lib.gsq_kq_debug_get(self.ctx, which, out.ctypes.data, out.nbytes),
+               "gsq_kq_debug_get")
+        return out
+
+    def set(self, which, arr) -> None:
+        shape, dt = self._shape(which)
+        a = np.ascontiguousarray(arr, dtype=dt).reshape(shape)
+        _check(_lib.gsq_kq_debug_set(self.ctx, which, a.ctypes.data, a.nbytes),
+               "gsq_kq_debug_set")
+
+    def step(self, tau, lr, beta1=0.9, beta2=0.99):
+        _check(_lib.gsq_kq_step(self.ctx, tau, lr, beta1, beta2), "gsq_kq_step")
+
+    def run(self, taus, lr, beta1=0.9, beta2=0.99):
+        t = np.ascontiguousarray(taus, np.float32)
+        _check(_lib.gsq_kq_run(self.ctx, t.ctypes.data, t.size, lr, beta1, beta2), "gsq_kq_run")
+
+    def last_loss(self) -> float:
+        v = C.c_double()
+        _check(_lib.gsq_kq_last_loss(self.ctx, C.byref(v)), "gsq_kq_last_loss")
+        return v.value
+
+    def export(self) -> np.ndarray:
+        out = np.zeros(gsq_kq_block_bytes(self.fmt, self.N, self.K), np.uint8)
+        _check(_lib.gsq_kq_export(self.ctx, out.ctypes.data), "gsq_kq_export")
+        return out
+
+    def start_blocks(self) -> np.ndarray:
+        out = np.zeros(gsq_kq_block_bytes(self.fmt, self.N, self.K), np.uint8)
+        _check(_lib.gsq_kq_start_blocks(self.ctx, out.ctypes.data), "gsq_kq_start_blocks")
+        return out
+
+    def recon_error(self, which: int = 0):
+        a, r = C.c_double(), C.c_double()
+        _check(_lib.gsq_kq_recon_error(self.ctx, which, C.byref(a), C.byref(r)),
+               "gsq_kq_recon_error")
+        return a.value, r.value
+
+    def soft_weight(self, tau: float) -> None:
+        _check(_lib.gsq_kq_debug_soft_weight(self.ctx, tau), "gsq_kq_debug_soft_weight")
+
+    def backward(self, tau, lr, beta1=0.9, beta2=0.99) -> None:
+        _check(_lib.gsq_kq_debug_backward(self.ctx, tau, lr, beta1, beta2),
+               "gsq_kq_debug_backward")
+
+    def noise(self, on: bool) -> None:
+        _check(_lib.gsq_kq_debug_noise(self.ctx, int(on)), "gsq_kq_debug_noise")
+
+    def close(self):
+        if self.ctx:
+            _lib.gsq_kq_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # pragma: no cover
+            pass
