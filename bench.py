@@ -669,6 +669,70 @@ def run_gptq_stage(args, rank, world, local_rank):
             "clocks": clk}
 
 
+def run_kquant_stage(args, rank, world, local_rank):
+    """GSQ on a GGUF K-Quant format (--kq-format q2k | q3k) on the --config
+    layer: whole steps through gsq_kq_run from the min-max K-Quant start."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    cfg = synth.CONFIGS[args.config]
+    fmt = gsq.GSQ_KQ_Q2_K if args.kq_format == "q2k" else gsq.GSQ_KQ_Q3_K
+    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
+    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    lay = gsq.gsq_kq_init(torch.from_numpy(W).to(torch.bfloat16).cuda(),
+                          torch.from_numpy(X).to(torch.bfloat16).cuda(), fmt, seed=rank)
+    e_start = lay.recon_error(1)[1]
+    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
+    sched = np.array([taus[i % len(taus)] for i in range(args.warmup + args.steps)], np.float32)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    lay.run(sched[:args.warmup], 1e-4)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    lay.run(sched[args.warmup:], 1e-4)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    loss = lay.last_loss()
+    e_end = lay.recon_error(0)[1]
+    lay.close()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    per = ms / args.steps
+    flops = 4.0 * cfg.N * cfg.T * cfg.K
+    ach = flops / (per / 1e3) / 1e12
+    coords = cfg.N * cfg.K
+    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
+            "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
+            "config": {"workload": cfg.name + "_" + args.kq_format, "N": cfg.N, "K": cfg.K,
+                       "T": cfg.T, "format": args.kq_format.upper().replace("K", "_K"),
+                       "step": "soft weight, 2 GEMMs, backward + Lion (16-weight sub-blocks)"},
+            "roofline": {"bound": "tensor", "kernel": "whole step (2 GEMMs + elementwise)",
+                         "achieved": round(ach, 1), "peak": tf_sus, "unit": "TFLOP/s",
+                         "frac": round(ach / tf_sus, 4),
+                         "peak_kind": f"{peak_kind} (sustained bf16)", "traffic": None},
+            "gpu_launches": int(args.steps * 4), "clocks": clk, "last_loss": loss,
+            "recon_rel": {"start": e_start, "after": e_end}}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -702,8 +766,10 @@ def main():
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq", "block"],
+    ap.add_argument("--stage", default=None, choices=["mlp", "attn", "scale", "gptq", "block", "kquant"],
                     help="time a block stage instead of a single layer")
+    ap.add_argument("--kq-format", default="q2k", choices=["q2k", "q3k"],
+                    help="K-Quant format of --stage kquant")
     ap.add_argument("--state", default="fp32", choices=["fp32", "bf16"],
                     help="logit / momentum storage of the single-layer step")
     ap.add_argument("--no-e2e", action="store_true",
@@ -737,6 +803,8 @@ def main():
         out = run_gptq_stage(args, rank, world, local_rank)
     elif args.stage == "block":
         out = run_block_pipeline(args, rank, world, local_rank)
+    elif args.stage == "kquant":
+        out = run_kquant_stage(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:
