@@ -107,11 +107,10 @@ __device__ __forceinline__ void kq_encode(uint8_t* blk, int r, const int* q, con
     }
     if (r < 16) blk[r] = (uint8_t)(sc[r] | (m[r] << 4));
     if (r == 0) {
-      const uint16_t dh = float_to_half_bits(d), mh = float_to_half_bits(dmin);
-      blk[80] = (uint8_t)(dh & 0xFF);
-      blk[81] = (uint8_t)(dh >> 8);
-      blk[82] = (uint8_t)(mh & 0xFF);
-      blk[83] = (uint8_t)(mh >> 8);
+      // both fp16 factors in one aligned 4-byte store (84 bi + 80 is a
+      // multiple of 4), little-endian
+      *reinterpret_cast<uint32_t*>(blk + 80) =
+          (uint32_t)float_to_half_bits(d) | ((uint32_t)float_to_half_bits(dmin) << 16);
     }
   } else {
     uint32_t hib = 0;
@@ -136,9 +135,8 @@ __device__ __forceinline__ void kq_encode(uint8_t* blk, int r, const int* q, con
       blk[104 + r] = (uint8_t)byte;
     }
     if (r == 0) {
-      const uint16_t dh = float_to_half_bits(d);
-      blk[108] = (uint8_t)(dh & 0xFF);
-      blk[109] = (uint8_t)(dh >> 8);
+      // one aligned 2-byte store (110 bi + 108 is even), little-endian
+      *reinterpret_cast<uint16_t*>(blk + 108) = float_to_half_bits(d);
     }
   }
 }
