@@ -669,6 +669,11 @@ def run_gptq_stage(args, rank, world, local_rank):
             "clocks": clk}
 
 
+# one lr for the logits and the sub-block scales/mins: small enough that the
+# noisy early steps leave the 16-weight sub-blocks' parameters near the start
+KQ_LR = 1e-5
+
+
 def run_kquant_stage(args, rank, world, local_rank):
     """GSQ on a GGUF K-Quant format (--kq-format q2k | q3k) on the --config
     layer: whole steps through gsq_kq_run from the min-max K-Quant start."""
@@ -689,7 +694,7 @@ def run_kquant_stage(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    lay.run(sched[:args.warmup], 1e-4)
+    lay.run(sched[:args.warmup], KQ_LR)
     torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
@@ -698,7 +703,7 @@ def run_kquant_stage(args, rank, world, local_rank):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    lay.run(sched[args.warmup:], 1e-4)
+    lay.run(sched[args.warmup:], KQ_LR)
     e1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
