@@ -415,16 +415,23 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
   };
   int64_t gi = warp;
   if (gi < groups) prefetch(gi, 0);
+  // the group's scale and its momentum, one group ahead like the staging
+  // (each group's scale is read and written by its own warp only)
+  float s_nx = gi < groups ? s[gi] : 0.f, ms_nx = gi < groups ? ms[gi] : 0.f;
   cp_async_commit();
   for (int buf = 0; gi < groups; gi += nwarps, buf ^= 1) {
-    if (gi + nwarps < groups) prefetch(gi + nwarps, buf ^ 1);
+    const float sg = s_nx;
+    const float msg = ms_nx;
+    if (gi + nwarps < groups) {
+      prefetch(gi + nwarps, buf ^ 1);
+      s_nx = s[gi + nwarps];
+      ms_nx = ms[gi + nwarps];
+    }
     cp_async_commit();
     cp_async_wait<1>();  // this lane's copies of group gi have landed
     const uint8_t* sb = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
     const uint8_t* sb_s = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + (S16 ? 8 : 16) * lane;
     const int64_t c0 = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
-    const float sg = s[gi];
-    const float msg = ms[gi];
     float Dr[4], Lr[L][4], Mr[L][4], Gr[L][4];
     *reinterpret_cast<float4*>(Dr) = *reinterpret_cast<const float4*>(sb);
 #pragma unroll
