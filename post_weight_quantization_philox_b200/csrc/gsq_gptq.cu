@@ -91,19 +91,21 @@ __global__ void k_reverse(const float* __restrict__ src, float* __restrict__ dst
 }
 
 // Lower Cholesky factor of the 64 x 64 diagonal block at (k0, k0), in place
-// (lower triangle only).  A pivot that is not positive is recorded and
-// replaced by 1 so that nothing downstream turns into NaN.
-__global__ void __launch_bounds__(256) k_potrf64(float* __restrict__ A, int64_t K, int64_t k0,
+// (lower triangle only).  Thread r owns row r; column by column the pivot
+// row divides its entry and every later row updates its own entries right of
+// the column.  A pivot that is not positive is recorded and replaced by 1
+// so that nothing downstream turns into NaN.
+__global__ void __launch_bounds__(kNb) k_potrf64(float* __restrict__ A, int64_t K, int64_t k0,
                                                  int* __restrict__ err) {
   __shared__ float a[kNb][kNb + 1];
-  const int tid = threadIdx.x;
-  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
-    const int r = e / kNb, c = e % kNb;
-    a[r][c] = c <= r ? A[(k0 + r) * K + k0 + c] : 0.f;
+  const int r = threadIdx.x;
+  for (int e = r; e < kNb * kNb; e += kNb) {
+    const int rr = e / kNb, c = e % kNb;
+    a[rr][c] = c <= rr ? A[(k0 + rr) * K + k0 + c] : 0.f;
   }
   __syncthreads();
   for (int c = 0; c < kNb; ++c) {
-    if (tid == 0) {
+    if (r == c) {
       float d = a[c][c];
       if (!(d > 0.f) || !isfinite(d)) {
         atomicCAS(err, 0, DEV_ERR_NONFINITE);
@@ -112,51 +114,64 @@ __global__ void __launch_bounds__(256) k_potrf64(float* __restrict__ A, int64_t 
       a[c][c] = sqrtf(d);
     }
     __syncthreads();
-    const float piv = a[c][c];
-    for (int r = c + 1 + tid; r < kNb; r += blockDim.x) a[r][c] /= piv;
+    if (r > c) a[r][c] /= a[c][c];
     __syncthreads();
-    for (int e = tid; e < kNb * kNb; e += blockDim.x) {
-      const int r = e / kNb, s = e % kNb;
-      if (s > c && s <= r) a[r][s] -= a[r][c] * a[s][c];
+    if (r > c) {
+      const float l = a[r][c];
+      for (int s2 = c + 1; s2 <= r; ++s2) a[r][s2] -= l * a[s2][c];
     }
     __syncthreads();
   }
-  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
-    const int r = e / kNb, c = e % kNb;
-    if (c <= r) A[(k0 + r) * K + k0 + c] = a[r][c];
+  for (int e = r; e < kNb * kNb; e += kNb) {
+    const int rr = e / kNb, c = e % kNb;
+    if (c <= rr) A[(k0 + rr) * K + k0 + c] = a[rr][c];
   }
 }
 
 // For each of `rows` vectors x (element c at X[r rs + c cs]) solve
 // x L^T = b in place, L the 64 x 64 lower triangle at L (leading dim ldl):
-// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector.
+// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector; the 64
+// vectors of a CTA move between global and shared memory cooperatively,
+// along whichever of rs, cs is 1, so the transfers coalesce.
 __global__ void __launch_bounds__(64) k_trsm64(float* __restrict__ X, int64_t rows, int64_t rs,
                                                int64_t cs, const float* __restrict__ L,
                                                int64_t ldl) {
   __shared__ float ls[kNb][kNb];
-  __shared__ float xs[kNb][64];
+  __shared__ float xs[kNb][64 + 1];
   const int tid = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * 64;
   for (int e = tid; e < kNb * kNb; e += blockDim.x) {
     const int r = e / kNb, c = e % kNb;
     ls[r][c] = c <= r ? L[r * ldl + c] : 0.f;
   }
-  const int64_t r = (int64_t)blockIdx.x * 64 + tid;
-  if (r < rows)
-    for (int c = 0; c < kNb; ++c) xs[c][tid] = X[r * rs + c * cs];
-  __syncthreads();
-  if (r >= rows) return;
-  for (int c = 0; c < kNb; ++c) {
-    float acc = xs[c][tid];
-    for (int s = 0; s < c; ++s) acc = fmaf(-xs[s][tid], ls[c][s], acc);
-    xs[c][tid] = acc / ls[c][c];
+  const bool along_c = cs == 1;
+  for (int e = tid; e < kNb * 64; e += blockDim.x) {
+    const int v = along_c ? e / kNb : e % 64, c = along_c ? e % kNb : e / 64;
+    if (r0 + v < rows) xs[c][v] = X[(r0 + v) * rs + c * cs];
   }
-  for (int c = 0; c < kNb; ++c) X[r * rs + c * cs] = xs[c][tid];
+  __syncthreads();
+  if (r0 + tid < rows)
+    for (int c = 0; c < kNb; ++c) {
+      float acc = xs[c][tid];
+      for (int s = 0; s < c; ++s) acc = fmaf(-xs[s][tid], ls[c][s], acc);
+      xs[c][tid] = acc / ls[c][c];
+    }
+  __syncthreads();
+  for (int e = tid; e < kNb * 64; e += blockDim.x) {
+    const int v = along_c ? e / kNb : e % 64, c = along_c ? e % kNb : e / 64;
+    if (r0 + v < rows) X[(r0 + v) * rs + c * cs] = xs[c][v];
+  }
 }
 
 // C[m][n] -= sum_k A(m, k) B(k, n) with A(m, k) = A[m a_rs + k a_cs] and
-// B(k, n) = B[k b_rs + n b_cs]; C has leading dimension ldc.  64 x 64 tiles,
-// 16-deep K slices in shared memory, 4 x 4 outputs per thread.  With lower,
-// tiles wholly above the diagonal (n0 > m0 + 63) are skipped.
+// B(k, n) = B[k b_rs + n b_cs]; C has leading dimension ldc; Kd % 8 == 0.
+// 128 x 128 tiles, 8-deep K slices double-buffered in shared memory (the
+// next slice is fetched into registers while the current one computes),
+// 8 x 8 outputs per thread in two 4-wide row and column strips 64 apart (so
+// the shared-memory reads of a warp are contiguous 16-byte vectors).  Global
+// reads run along whichever operand axis is contiguous (a_cs == 1: along k,
+// else along m; likewise for B), so they coalesce at every call site.  With
+// lower, tiles wholly above the diagonal (n0 > m0 + 127) are skipped.
 struct SubGemm {
   int64_t M, N, Kd;
   const float* A;
@@ -168,48 +183,96 @@ struct SubGemm {
   int lower;
 };
 
+constexpr int kGT = 128, kGK = 8;
+
 __global__ void __launch_bounds__(256) k_gemm_sub(const SubGemm g) {
-  __shared__ float as[16][64 + 4];
-  __shared__ float bs[16][64 + 4];
-  const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
-  if (g.lower && n0 > m0 + 63) return;
+  __shared__ __align__(16) float as[2][kGK][kGT + 4];
+  __shared__ __align__(16) float bs[2][kGK][kGT + 4];
+  const int64_t m0 = (int64_t)blockIdx.y * kGT, n0 = (int64_t)blockIdx.x * kGT;
+  if (g.lower && n0 > m0 + kGT - 1) return;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  float acc[4][4] = {};
-  for (int64_t k0 = 0; k0 < g.Kd; k0 += 16) {
-    for (int e = tid; e < 16 * 64; e += 256) {
-      const int kk = e / 64, mm = e % 64;
+  const bool a_k = g.a_cs == 1, b_k = g.b_rs == 1;
+  // this thread's four elements of each slice: (row of the tile, k)
+  auto a_pos = [&](int e, int& mm, int& kk) {
+    const int idx = tid + 256 * e;  // 0..1023
+    if (a_k) { kk = idx & 7; mm = idx >> 3; } else { mm = idx & 127; kk = idx >> 7; }
+  };
+  auto b_pos = [&](int e, int& nn, int& kk) {
+    const int idx = tid + 256 * e;
+    if (b_k) { kk = idx & 7; nn = idx >> 3; } else { nn = idx & 127; kk = idx >> 7; }
+  };
+  float ra[4], rb[4];
+  auto fetch = [&](int64_t k0) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      int mm, kk;
+      a_pos(e, mm, kk);
       const int64_t m = m0 + mm, k = k0 + kk;
-      as[kk][mm] = (m < g.M && k < g.Kd) ? g.A[m * g.a_rs + k * g.a_cs] : 0.f;
-      const int64_t n = n0 + mm;
-      bs[kk][mm] = (n < g.N && k < g.Kd) ? g.B[k * g.b_rs + n * g.b_cs] : 0.f;
+      ra[e] = m < g.M ? g.A[m * g.a_rs + k * g.a_cs] : 0.f;
+      int nn, kb;
+      b_pos(e, nn, kb);
+      const int64_t n = n0 + nn, kq = k0 + kb;
+      rb[e] = n < g.N ? g.B[kq * g.b_rs + n * g.b_cs] : 0.f;
     }
-    __syncthreads();
+  };
+  auto stash = [&](int buf) {
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        av[i] = as[kk][ty * 4 + i];
-        bv[i] = bs[kk][tx * 4 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    for (int e = 0; e < 4; ++e) {
+      int mm, kk;
+      a_pos(e, mm, kk);
+      as[buf][kk][mm] = ra[e];
+      int nn, kb;
+      b_pos(e, nn, kb);
+      bs[buf][kb][nn] = rb[e];
     }
-    __syncthreads();
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
+  for (int64_t k0 = 0; k0 < g.Kd; k0 += kGK) {
+    const bool more = k0 + kGK < g.Kd;
+    if (more) fetch(k0 + kGK);
+#pragma unroll
+    for (int kk = 0; kk < kGK; ++kk) {
+      float av[8], bv[8];
+      *reinterpret_cast<float4*>(av) = *reinterpret_cast<const float4*>(&as[buf][kk][ty * 4]);
+      *reinterpret_cast<float4*>(av + 4) =
+          *reinterpret_cast<const float4*>(&as[buf][kk][64 + ty * 4]);
+      *reinterpret_cast<float4*>(bv) = *reinterpret_cast<const float4*>(&bs[buf][kk][tx * 4]);
+      *reinterpret_cast<float4*>(bv + 4) =
+          *reinterpret_cast<const float4*>(&bs[buf][kk][64 + tx * 4]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    if (more) {
+      stash(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+    for (int j = 0; j < 8; ++j) {
+      const int64_t m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+      const int64_t n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
       if (m < g.M && n < g.N) g.C[m * g.ldc + n] -= acc[i][j];
     }
 }
 
-__global__ void k_unit_diag_block(float* __restrict__ M, int64_t K, int64_t r0) {
-  if (threadIdx.x < kNb) M[(r0 + threadIdx.x) * K + r0 + threadIdx.x] = 1.f;
+// M[i][i] = 1 for all i
+__global__ void k_unit_diag(float* __restrict__ M, int64_t K) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K;
+       i += (int64_t)gridDim.x * blockDim.x)
+    M[i * K + i] = 1.f;
 }
 
 // Nearest level of w / s (first level on ties; s = 0 gives w / s := 0), in fp32.
@@ -230,50 +293,64 @@ __device__ __forceinline__ int gptq_round(float w, float s) {
   return best;
 }
 
-// One block of 128 columns [j0, j0 + 128) for 128 rows per CTA (one thread
-// per row).  The block's rows of W and the 128 x 128 block of U sit in
-// shared memory (padded rows: conflict-free column access); the row's group
-// scale is set from the updated weights at the block start; every column is
-// rounded, its error fed forward inside the block; the levels go out through
-// shared memory with coalesced stores, the errors as E[j][n].
-constexpr int kColsSmem = 2 * kCols * (kCols + 1) * 4 + kCols * (kCols + 4);
+// One block of 128 columns [j0, j0 + 128): one warp per row, lane l holding
+// the row's columns l, l + 32, l + 64, l + 96; 16 rows per CTA share the
+// block's 128 x 128 upper triangle of U in shared memory (rows of U read
+// across lanes: conflict-free).  The row's group scale is set from its
+// updated weights at the block start (warp max); then column by column the
+// owner lane's weight is broadcast, rounded to the nearest level (first on
+// ties), its error e = (w - s c) / U_jj written to E[j][n] and fed forward
+// to the later columns of the block, every lane updating its own columns.
+constexpr int kColRows = 16;
+constexpr int kColsSmem = kCols * kCols * 4;
 
 template <int MODE>
-__global__ void __launch_bounds__(kCols) k_gptq_cols(const float* __restrict__ W, int64_t N,
-                                                    int64_t K, const float* __restrict__ U,
-                                                    int64_t j0, int8_t* __restrict__ levels,
-                                                    float* __restrict__ scales,
-                                                    float* __restrict__ E) {
+__global__ void __launch_bounds__(kColRows * 32) k_gptq_cols(
+    const float* __restrict__ W, int64_t N, int64_t K, const float* __restrict__ U, int64_t j0,
+    int8_t* __restrict__ levels, float* __restrict__ scales, float* __restrict__ E) {
   using Gr = GridT<MODE>;
   extern __shared__ __align__(16) uint8_t gsm[];
-  float (*us)[kCols + 1] = reinterpret_cast<float (*)[kCols + 1]>(gsm);
-  float (*ws)[kCols + 1] = reinterpret_cast<float (*)[kCols + 1]>(gsm + kCols * (kCols + 1) * 4);
-  int8_t (*lv)[kCols + 4] = reinterpret_cast<int8_t (*)[kCols + 4]>(gsm + 2 * kCols * (kCols + 1) * 4);
-  const int tid = threadIdx.x;
-  const int64_t n0 = (int64_t)blockIdx.x * kCols;
-  for (int r = 0; r < kCols; ++r) {
-    us[r][tid] = tid >= r ? U[(j0 + r) * K + j0 + tid] : 0.f;
-    ws[tid][r] = n0 + r < N ? W[(n0 + r) * K + j0 + tid] : 0.f;
+  float (*us)[kCols] = reinterpret_cast<float (*)[kCols]>(gsm);
+  for (int e = threadIdx.x; e < kCols * kCols; e += blockDim.x) {
+    const int r = e / kCols, c = e % kCols;
+    us[r][c] = c >= r ? U[(j0 + r) * K + j0 + c] : 0.f;
   }
   __syncthreads();
-  const int64_t n = n0 + tid;
-  if (n < N) {
-    float amax = 0.f;
-    for (int c = 0; c < kCols; ++c) amax = fmaxf(amax, fabsf(ws[c][tid]));
-    const float s = amax / Gr::CMAX;
-    scales[n * (K / kCols) + j0 / kCols] = s;
-    for (int j = 0; j < kCols; ++j) {
-      const float w = ws[j][tid];
-      const int lev = gptq_round<MODE>(w, s);
-      const float e = (w - s * Gr::level(lev)) / us[j][j];
-      lv[tid][j] = (int8_t)lev;
-      E[j * N + n] = e;
-      for (int c = j + 1; c < kCols; ++c) ws[c][tid] = fmaf(-e, us[j][c], ws[c][tid]);
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * kColRows + (threadIdx.x >> 5);
+  if (n >= N) return;  // whole warps
+  float w[4];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[i] = W[n * K + j0 + lane + 32 * i];
+    amax = fmaxf(amax, fabsf(w[i]));
+  }
+  amax = warp_max(amax);
+  const float s = amax / Gr::CMAX;
+  if (lane == 0) scales[n * (K / kCols) + j0 / kCols] = s;
+  int lev_own[4] = {0, 0, 0, 0};
+  for (int j = 0; j < kCols; ++j) {
+    const int slot = j >> 5;
+    const float mine = slot == 0 ? w[0] : slot == 1 ? w[1] : slot == 2 ? w[2] : w[3];
+    const float wj = __shfl_sync(0xffffffffu, mine, j & 31);
+    const int lev = gptq_round<MODE>(wj, s);
+    const float e = (wj - s * Gr::level(lev)) / us[j][j];
+    if (lane == (j & 31)) {
+      lev_own[0] = slot == 0 ? lev : lev_own[0];
+      lev_own[1] = slot == 1 ? lev : lev_own[1];
+      lev_own[2] = slot == 2 ? lev : lev_own[2];
+      lev_own[3] = slot == 3 ? lev : lev_own[3];
+    }
+    if (lane == 0) E[(int64_t)j * N + n] = e;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      if (c > j) w[i] = fmaf(-e, us[j][c], w[i]);
     }
   }
-  __syncthreads();
-  for (int r = 0; r < kCols; ++r)
-    if (n0 + r < N) levels[(n0 + r) * K + j0 + tid] = lv[r][tid];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) levels[n * K + j0 + lane + 32 * i] = (int8_t)lev_own[i];
 }
 
 }  // namespace
@@ -290,14 +367,15 @@ cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const unsigned rb = (unsigned)((N + kCols - 1) / kCols);
+  const unsigned rb = (unsigned)((N + kColRows - 1) / kColRows);
   for (int64_t j0 = 0; j0 < K; j0 += kCols) {
-    k_gptq_cols<MODE><<<rb, kCols, kColsSmem, st>>>(W32, N, K, U, j0, levels, scales, E);
+    k_gptq_cols<MODE><<<rb, kColRows * 32, kColsSmem, st>>>(W32, N, K, U, j0, levels, scales, E);
     const int64_t j1 = j0 + kCols, rest = K - j1;
     if (rest > 0) {
       // W[:, j1:] -= E^T U[j0:j1, j1:]
       const SubGemm g{N, rest, kCols, E, 1, N, U + j0 * K + j1, K, 1, W32 + j1, K, 0};
-      k_gemm_sub<<<dim3((unsigned)((rest + 63) / 64), (unsigned)((N + 63) / 64)), 256, 0, st>>>(g);
+      k_gemm_sub<<<dim3((unsigned)((rest + kGT - 1) / kGT), (unsigned)((N + kGT - 1) / kGT)),
+                   256, 0, st>>>(g);
     }
   }
   return cudaGetLastError();
@@ -306,7 +384,9 @@ cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_
 }  // namespace
 
 // GPTQ on device inputs; levels (N x K int8) and scales (N x K/128 fp32) are
-// device buffers.  Allocates its workspace, synchronises the stream, frees.
+// device buffers.  Allocates its workspace stream-ordered on `st` (no device
+// synchronisation, unlike cudaMalloc / cudaFree), synchronises the stream,
+// frees.
 int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype, int64_t N,
              int64_t K, int64_t T, float damp, int8_t* levels, float* scales, int sm_count,
              cudaStream_t st) {
@@ -315,7 +395,7 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   bool oom = false;
   auto alloc = [&](size_t bytes) -> void* {
     void* p = nullptr;
-    if (oom || cudaMalloc(&p, bytes) != cudaSuccess) {
+    if (oom || cudaMallocAsync(&p, bytes, st) != cudaSuccess) {
       cudaGetLastError();
       oom = true;
       return nullptr;
@@ -335,9 +415,10 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   double* partials = (double*)alloc(4096 * 8);
   unsigned* ticket = (unsigned*)alloc(16);
   auto finish = [&](int status) {
+    cudaGetLastError();
+    for (void* p : bufs) cudaFreeAsync(p, st);
     cudaStreamSynchronize(st);
     cudaGetLastError();
-    for (void* p : bufs) cudaFree(p);
     return status;
   };
   if (oom) return finish(GSQ_ERR_OOM);
@@ -377,28 +458,34 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   k_reverse<<<rgrid, 256, 0, st>>>(B1, B2, K);
   float* A = B2;
   for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
-    k_potrf64<<<1, 256, 0, st>>>(A, K, k0, err);
+    k_potrf64<<<1, kNb, 0, st>>>(A, K, k0, err);
     const int64_t rest = K - k0 - kNb;
     if (rest > 0) {
       float* P = A + (k0 + kNb) * K + k0;
       k_trsm64<<<(unsigned)((rest + 63) / 64), 64, 0, st>>>(P, rest, K, 1, A + k0 * K + k0, K);
       const SubGemm g{rest, rest, kNb, P, K, 1, P, 1, K, P + kNb, K, 1};
-      const unsigned t = (unsigned)((rest + 63) / 64);
+      const unsigned t = (unsigned)((rest + kGT - 1) / kGT);
       k_gemm_sub<<<dim3(t, t), 256, 0, st>>>(g);
     }
     ok(cudaGetLastError());
   }
-  // M = L^-1 into B1 by block forward substitution
+  // M = L^-1 into B1, right-looking block forward substitution: M starts
+  // as I; row block k0 is solved against its diagonal block once every
+  // earlier block has been subtracted from it, then subtracted from all
+  // later row blocks at once (one wide GEMM per block instead of a 64-row
+  // strip with the whole K depth)
   float* M = B1;
   ok(cudaMemsetAsync(M, 0, (size_t)KK * 4, st));
-  for (int64_t r0 = 0; r0 < K && e == cudaSuccess; r0 += kNb) {
-    const int64_t c1 = r0 + kNb;
-    k_unit_diag_block<<<1, kNb, 0, st>>>(M, K, r0);
-    if (r0 > 0) {
-      const SubGemm g{kNb, c1, r0, A + r0 * K, K, 1, M, K, 1, M + r0 * K, K, 0};
-      k_gemm_sub<<<dim3((unsigned)((c1 + 63) / 64), 1), 256, 0, st>>>(g);
+  k_unit_diag<<<grid_cap(K, 256, 1024), 256, 0, st>>>(M, K);
+  for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
+    const int64_t c1 = k0 + kNb, rest = K - c1;
+    k_trsm64<<<(unsigned)((c1 + 63) / 64), 64, 0, st>>>(M + k0 * K, c1, 1, K, A + k0 * K + k0, K);
+    if (rest > 0) {
+      // M[c1:, :c1] -= L[c1:, k0:c1] M[k0:c1, :c1]
+      const SubGemm g{rest, c1, kNb, A + c1 * K + k0, K, 1, M + k0 * K, K, 1, M + c1 * K, K, 0};
+      k_gemm_sub<<<dim3((unsigned)((c1 + kGT - 1) / kGT), (unsigned)((rest + kGT - 1) / kGT)),
+                   256, 0, st>>>(g);
     }
-    k_trsm64<<<(unsigned)((c1 + 63) / 64), 64, 0, st>>>(M + r0 * K, c1, 1, K, A + r0 * K + r0, K);
     ok(cudaGetLastError());
   }
   // U = J M J into B2
