@@ -268,12 +268,12 @@ __device__ __forceinline__ void candidates(int lev0, float* cand) {
 }
 
 // Gumbel noise of one coordinate at step t (zeros when noise is off).
-template <int L>
+template <int MODE, int L = GridT<MODE>::L>
 __device__ __forceinline__ void noise1(int64_t c, uint32_t t, uint32_t k0,
                                        uint32_t k1, int noise, float (&g)[L]) {
   float gg[5];
   if (noise) {
-    coord_noise5((uint64_t)c, t, k0, k1, L == 5, gg);
+    coord_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c, t, k0, k1, L == 5, gg);
   } else {
 #pragma unroll
     for (int p = 0; p < 5; ++p) gg[p] = 0.f;
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 #pragma unroll
       for (int p = 0; p < L; ++p) l[p] = St<TS>::ld(logits + p * NK + c);
       const int lev0 = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
-      noise1<L>(c, t, k0, k1, noise, gz);
+      noise1<MODE>(c, t, k0, k1, noise, gz);
       candidates<MODE>(lev0, cand);
       const float w = sg * coord_soft<MODE>(l, gz, inv_tau, cand, y);
       What[c] = __float2bfloat16_rn(w);
@@ -475,12 +475,14 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
 #pragma unroll
         for (int p = 0; p < L; ++p) {
           rsr[S16 ? j : 0][p] = wd[p];
-          if (NEXT) gnext[NEXT ? j : 0][p] = noise ? gumbel(word_to_unit(wd[p])) : 0.f;
+          if (NEXT)
+            gnext[NEXT ? j : 0][p] =
+                noise ? gumbel<GridT<MODE>::FAST_GUMBEL>(word_to_unit(wd[p])) : 0.f;
         }
       }
     } else if (NEXT) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) noise1<L>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
+      for (int j = 0; j < 4; ++j) noise1<MODE>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
     }
     float ds_part = 0.f;
     float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
