@@ -131,8 +131,10 @@ GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const
  * W (N x K) and X (T x K): fp32 or bf16 (w_dtype, x_dtype), host or device,
  * read only.  levels (N x K int8 level indices, the init_idx of gsq_init)
  * and scales (N x K/group fp32): caller-owned, host or device.  damp >= 0
- * (GPTQ's default 0.01).  Synchronises the stream; allocates and frees its
- * own workspace (about 8 K^2 + 8 N K bytes).
+ * (GPTQ's default 0.01).  Synchronises the stream.  Its workspace (about
+ * 8 K^2 + 8 N K bytes) comes from a memory pool the library owns per device,
+ * which keeps up to 4 GiB reserved after the call so that the next call maps
+ * no new memory; gsq_gptq_release_workspace returns it to the device.
  * Errors: GSQ_ERR_INVALID_ARG for bad sizes / pointers / dtypes / damp or
  * K > 65536; GSQ_ERR_UNSUPPORTED for group != 128 or a non-sm_100 device;
  * GSQ_ERR_NONFINITE if the damped Hessian is not positive definite in fp32
@@ -140,6 +142,10 @@ GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const
 GSQ_API int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N,
                      int64_t K, int64_t T, int group, int grid_mode, float damp,
                      int8_t* levels, float* scales, void* stream);
+/* Returns the GPTQ workspace the library's pools keep reserved (all
+ * devices) to the driver.  Call it with no gsq_gptq / gsq_init_gptq running.
+ * Errors: GSQ_ERR_CUDA. */
+GSQ_API int gsq_gptq_release_workspace(void);
 /* gsq_init from the GPTQ assignment: the initial levels (init_idx) and the
  * group scales both come from gsq_gptq (instead of round-to-nearest with
  * absmax scales); everything else as gsq_init.  Synchronises the stream. */

@@ -28,6 +28,7 @@
 // This runs once per layer before the reconstruction steps; none of it is on
 // the per-step path.
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include "../../include/gsq.h"
@@ -91,38 +92,46 @@ __global__ void k_reverse(const float* __restrict__ src, float* __restrict__ dst
 }
 
 // Lower Cholesky factor of the 64 x 64 diagonal block at (k0, k0), in place
-// (lower triangle only).  Thread r owns row r; column by column the pivot
-// row divides its entry and every later row updates its own entries right of
-// the column.  A pivot that is not positive is recorded and replaced by 1
-// so that nothing downstream turns into NaN.
-__global__ void __launch_bounds__(kNb) k_potrf64(float* __restrict__ A, int64_t K, int64_t k0,
-                                                 int* __restrict__ err) {
+// (lower triangle only), right-looking: column by column every thread takes
+// the pivot's square root, the rows below divide their entry of the column,
+// and the trailing lower triangle takes its rank-1 update, 1024 threads
+// owning 4 entries each (column t % 64 of rows t / 64 + 16 j, so a warp's
+// accesses fall in distinct banks).  A pivot that is not positive is recorded and
+// replaced by 1 so that nothing downstream turns into NaN.
+constexpr int kPotrfThreads = 1024;
+__global__ void __launch_bounds__(kPotrfThreads) k_potrf64(float* __restrict__ A, int64_t K,
+                                                           int64_t k0, int* __restrict__ err) {
   __shared__ float a[kNb][kNb + 1];
-  const int r = threadIdx.x;
-  for (int e = r; e < kNb * kNb; e += kNb) {
+  const int t = threadIdx.x;
+  for (int e = t; e < kNb * kNb; e += kPotrfThreads) {
     const int rr = e / kNb, c = e % kNb;
     a[rr][c] = c <= rr ? A[(k0 + rr) * K + k0 + c] : 0.f;
   }
   __syncthreads();
+  const int s2 = t & (kNb - 1), rb = t / kNb;  // entries (rb + 16 j, s2)
   for (int c = 0; c < kNb; ++c) {
-    if (r == c) {
-      float d = a[c][c];
-      if (!(d > 0.f) || !isfinite(d)) {
-        atomicCAS(err, 0, DEV_ERR_NONFINITE);
-        d = 1.f;
-      }
-      a[c][c] = sqrtf(d);
+    float d = a[c][c];
+    const bool bad = !(d > 0.f) || !isfinite(d);
+    if (bad) d = 1.f;
+    const float sd = sqrtf(d);
+    __syncthreads();  // every thread has read the pivot
+    if (t == c) {
+      if (bad) atomicCAS(err, 0, DEV_ERR_NONFINITE);
+      a[c][c] = sd;
     }
+    if (t > c && t < kNb) a[t][c] /= sd;
     __syncthreads();
-    if (r > c) a[r][c] /= a[c][c];
-    __syncthreads();
-    if (r > c) {
-      const float l = a[r][c];
-      for (int s2 = c + 1; s2 <= r; ++s2) a[r][s2] -= l * a[s2][c];
+    if (s2 > c) {
+      const float u = a[s2][c];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = rb + 16 * j;
+        if (s2 <= r) a[r][s2] -= a[r][c] * u;
+      }
     }
     __syncthreads();
   }
-  for (int e = r; e < kNb * kNb; e += kNb) {
+  for (int e = t; e < kNb * kNb; e += kPotrfThreads) {
     const int rr = e / kNb, c = e % kNb;
     if (c <= rr) A[(k0 + rr) * K + k0 + c] = a[rr][c];
   }
@@ -130,9 +139,12 @@ __global__ void __launch_bounds__(kNb) k_potrf64(float* __restrict__ A, int64_t 
 
 // For each of `rows` vectors x (element c at X[r rs + c cs]) solve
 // x L^T = b in place, L the 64 x 64 lower triangle at L (leading dim ldl):
-// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector; the 64
-// vectors of a CTA move between global and shared memory cooperatively,
-// along whichever of rs, cs is 1, so the transfers coalesce.
+// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector, the
+// vector in registers: once x_c is known it is taken off every later b_s
+// (the same products in the same order as the dot-product form, but
+// independent of one another, so they pipeline).  The 64 vectors of a CTA
+// move between global and shared memory cooperatively, along whichever of
+// rs, cs is 1, so the transfers coalesce.
 __global__ void __launch_bounds__(64) k_trsm64(float* __restrict__ X, int64_t rows, int64_t rs,
                                                int64_t cs, const float* __restrict__ L,
                                                int64_t ldl) {
@@ -150,12 +162,19 @@ __global__ void __launch_bounds__(64) k_trsm64(float* __restrict__ X, int64_t ro
     if (r0 + v < rows) xs[c][v] = X[(r0 + v) * rs + c * cs];
   }
   __syncthreads();
-  if (r0 + tid < rows)
+  if (r0 + tid < rows) {
+    float x[kNb];
+#pragma unroll
+    for (int c = 0; c < kNb; ++c) x[c] = xs[c][tid];
+#pragma unroll
     for (int c = 0; c < kNb; ++c) {
-      float acc = xs[c][tid];
-      for (int s = 0; s < c; ++s) acc = fmaf(-xs[s][tid], ls[c][s], acc);
-      xs[c][tid] = acc / ls[c][c];
+      x[c] = x[c] / ls[c][c];
+#pragma unroll
+      for (int s2 = c + 1; s2 < kNb; ++s2) x[s2] = fmaf(-x[c], ls[s2][c], x[s2]);
     }
+#pragma unroll
+    for (int c = 0; c < kNb; ++c) xs[c][tid] = x[c];
+  }
   __syncthreads();
   for (int e = tid; e < kNb * 64; e += blockDim.x) {
     const int v = along_c ? e / kNb : e % 64, c = along_c ? e % kNb : e / 64;
@@ -383,19 +402,55 @@ cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_
 
 }  // namespace
 
+// The GPTQ workspace comes from a memory pool of the library's own per
+// device, which keeps up to kPoolKeep bytes reserved between calls (a later
+// call of the same size then maps no new memory); gsq_gptq_release_workspace
+// hands it back.
+namespace {
+constexpr uint64_t kPoolKeep = 4ull << 30;
+constexpr int kMaxDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+}  // namespace
+
+cudaMemPool_t workspace_pool(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    uint64_t keep = kPoolKeep;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    cudaGetLastError();
+    g_pool[dev] = p;
+  }
+  return g_pool[dev];
+}
+
 // GPTQ on device inputs; levels (N x K int8) and scales (N x K/128 fp32) are
-// device buffers.  Allocates its workspace stream-ordered on `st` (no device
-// synchronisation, unlike cudaMalloc / cudaFree), synchronises the stream,
-// frees.
+// device buffers.  Allocates its workspace stream-ordered on `st` from the
+// library's pool (no device synchronisation, unlike cudaMalloc / cudaFree),
+// synchronises the stream, frees.
 int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype, int64_t N,
              int64_t K, int64_t T, float damp, int8_t* levels, float* scales, int sm_count,
              cudaStream_t st) {
   const int64_t Tp = (T + 63) / 64 * 64, NK = N * K, KK = K * K;
   std::vector<void*> bufs;
-  bool oom = false;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaMemPool_t pool = workspace_pool(dev);
+  bool oom = pool == nullptr;
   auto alloc = [&](size_t bytes) -> void* {
     void* p = nullptr;
-    if (oom || cudaMallocAsync(&p, bytes, st) != cudaSuccess) {
+    if (oom || cudaMallocFromPoolAsync(&p, bytes, pool, st) != cudaSuccess) {
       cudaGetLastError();
       oom = true;
       return nullptr;
@@ -458,7 +513,7 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   k_reverse<<<rgrid, 256, 0, st>>>(B1, B2, K);
   float* A = B2;
   for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
-    k_potrf64<<<1, kNb, 0, st>>>(A, K, k0, err);
+    k_potrf64<<<1, kPotrfThreads, 0, st>>>(A, K, k0, err);
     const int64_t rest = K - k0 - kNb;
     if (rest > 0) {
       float* P = A + (k0 + kNb) * K + k0;
@@ -525,13 +580,14 @@ int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, 
       T > ((int64_t)1 << 31) || K > 65536)
     return GSQ_ERR_INVALID_ARG;
   if (group != kStageGroup) return GSQ_ERR_UNSUPPORTED;
-  int dev = 0;
-  cudaDeviceProp prop;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+  int dev = 0, major = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     return GSQ_ERR_CUDA;
   }
-  if (prop.major != 10) return GSQ_ERR_UNSUPPORTED;
+  if (major != 10) return GSQ_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t wbytes = (size_t)N * K * (w_dtype == GSQ_F32 ? 4 : 2);
   const size_t xbytes = (size_t)T * K * (x_dtype == GSQ_F32 ? 4 : 2);
@@ -560,7 +616,7 @@ int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, 
   if (!rc && e != cudaSuccess) rc = GSQ_ERR_CUDA;
   if (!rc)
     rc = gptq_run(grid_mode, Wd, w_dtype, Xd, x_dtype, N, K, T, damp, (int8_t*)Ld, (float*)Sd,
-                  prop.multiProcessorCount, st);
+                  sms, st);
   if (!rc && Ld != levels &&
       cudaMemcpy(levels, Ld, lbytes, cudaMemcpyDeviceToHost) != cudaSuccess)
     rc = GSQ_ERR_CUDA;
@@ -570,6 +626,18 @@ int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, 
   cudaStreamSynchronize(st);
   cudaGetLastError();
   for (void* p : tmp) cudaFree(p);
+  return rc;
+}
+
+int gsq_gptq_release_workspace(void) {
+  using namespace gsq;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  int rc = GSQ_OK;
+  for (int d = 0; d < kMaxDevices; ++d)
+    if (g_pool[d] && cudaMemPoolTrimTo(g_pool[d], 0) != cudaSuccess) {
+      cudaGetLastError();
+      rc = GSQ_ERR_CUDA;
+    }
   return rc;
 }
 

@@ -86,6 +86,12 @@ def test_null_context_handling(gsq):
                         None) == gsq.GSQ_ERR_INVALID_ARG
 
 
+def test_gptq_release_without_pools(gsq):
+    """With no GPTQ call made there is no pool to trim: a no-op that succeeds
+    without touching a device."""
+    assert gsq.lib().gsq_gptq_release_workspace() == gsq.GSQ_OK
+
+
 def test_binding_has_no_fallback(monkeypatch, tmp_path):
     """Importing the binding without the shared library raises."""
     import importlib.util
