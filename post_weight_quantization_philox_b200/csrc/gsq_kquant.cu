@@ -376,14 +376,20 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
 // Backward + Lion from dW and the step's probabilities: per coordinate
 // dl_k = (a_j dw / tau) y_k sum_m y_m (c_k - c_m); per sub-block
 // da_j = sum dw v, db_j = -sum dw (the four threads of a sub-block combine
-// by shuffles); Lion on the logits, a_j and (Q2_K) b_j.
-template <int F, bool DBG>
+// by shuffles, which leaves the same sum in all four); Lion on the logits,
+// a_j and (Q2_K) b_j.  With NEXT the kernel goes on to the soft weight of
+// step t_next at 1 / inv_tau_next from the updated logits, a_j and b_j --
+// the same arithmetic as k_kq_soft -- and writes it to What and its
+// probabilities over the ones it has just read.
+template <int F, bool DBG, bool NEXT>
 __global__ void __launch_bounds__(256) k_kq_backward(
     float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ a,
     float* __restrict__ ma, float* __restrict__ b, float* __restrict__ mb,
-    const int8_t* __restrict__ q0, const float* __restrict__ dW, const float* __restrict__ probs,
+    const int8_t* __restrict__ q0, const float* __restrict__ dW, float* __restrict__ probs,
     int64_t NK, float inv_tau, float lr, float b1, float omb1, float b2, float omb2,
-    float* __restrict__ dl_dbg, float* __restrict__ da_dbg, float* __restrict__ db_dbg) {
+    float* __restrict__ dl_dbg, float* __restrict__ da_dbg, float* __restrict__ db_dbg,
+    uint32_t k0, uint32_t k1, uint32_t t_next, int noise, float inv_tau_next,
+    __nv_bfloat16* __restrict__ What) {
   constexpr int L = KqT<F>::L;
   // NK / 4 is a multiple of 64 (K % 256 == 0), so this exit takes whole
   // warps and the shuffles below always see all 32 lanes
@@ -445,14 +451,17 @@ __global__ void __launch_bounds__(256) k_kq_backward(
   da_part += __shfl_xor_sync(0xffffffffu, da_part, 2);
   db_part += __shfl_xor_sync(0xffffffffu, db_part, 1);
   db_part += __shfl_xor_sync(0xffffffffu, db_part, 2);
+  // every lane of the sub-block updates its parameters alike; the first stores
+  float av = aj, mav = ma[sb], bv = b[sb], mbv = 0.f;
+  lion_update(av, mav, da_part, lr, b1, omb1, b2, omb2);
+  if (F == KQ_Q2) {
+    mbv = mb[sb];
+    lion_update(bv, mbv, db_part, lr, b1, omb1, b2, omb2);
+  }
   if ((threadIdx.x & 3) == 0) {
-    float av = aj, mav = ma[sb];
-    lion_update(av, mav, da_part, lr, b1, omb1, b2, omb2);
     a[sb] = av;
     ma[sb] = mav;
     if (F == KQ_Q2) {
-      float bv = b[sb], mbv = mb[sb];
-      lion_update(bv, mbv, db_part, lr, b1, omb1, b2, omb2);
       b[sb] = bv;
       mb[sb] = mbv;
     }
@@ -460,6 +469,34 @@ __global__ void __launch_bounds__(256) k_kq_backward(
       da_dbg[sb] = da_part;
       db_dbg[sb] = db_part;
     }
+  }
+  if (NEXT) {
+    float wv[4], yy[4][L];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[L], g[5], c[L];
+#pragma unroll
+      for (int p = 0; p < L; ++p) l[p] = lo[p][j];
+      if (noise) {
+        coord_noise5((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
+      } else {
+#pragma unroll
+        for (int p = 0; p < 5; ++p) g[p] = 0.f;
+      }
+      kq_cand<F>(qq[j], c);
+      const float v = kq_soft<L>(l, g, inv_tau_next, c, yy[j]);
+      wv[j] = fmaf(av, v, -bv);
+    }
+    __nv_bfloat162 p01 = __floats2bfloat162_rn(wv[0], wv[1]);
+    __nv_bfloat162 p23 = __floats2bfloat162_rn(wv[2], wv[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&p01);
+    pk.y = *reinterpret_cast<uint32_t*>(&p23);
+    *reinterpret_cast<uint2*>(What + c0) = pk;
+#pragma unroll
+    for (int p = 0; p < L; ++p)
+      *reinterpret_cast<float4*>(probs + p * NK + c0) =
+          make_float4(yy[0][p], yy[1][p], yy[2][p], yy[3][p]);
   }
 }
 
@@ -544,6 +581,10 @@ struct gsq_kq {
   int64_t N = 0, K = 0, T = 0, Tp = 0, nblk = 0;
   uint64_t seed = 0, t = 0;
   int noise = 1;
+  // What and probs hold the soft weight of step what_t at what_tau
+  // (what_t < 0: nothing precomputed)
+  int64_t what_t = -1;
+  float what_tau = 0.f;
   cudaStream_t st = nullptr;
   int sms = 148, failed = 0;
   __nv_bfloat16 *Xb = nullptr, *Xt = nullptr, *What = nullptr, *dYt = nullptr;
@@ -637,18 +678,29 @@ cudaError_t kq_launch_soft(gsq_kq* c, float tau, float* wsoft32) {
   return cudaGetLastError();
 }
 
-cudaError_t kq_launch_backward(gsq_kq* c, float tau, float lr, float b1, float b2, bool dbg) {
+// The backward of step t; next_tau > 0 (not with dbg): also the soft weight
+// of step t + 1 at next_tau.
+cudaError_t kq_launch_backward(gsq_kq* c, float tau, float lr, float b1, float b2, bool dbg,
+                               float next_tau = 0.f) {
   const int64_t NK = c->N * c->K;
   const unsigned g = (unsigned)((NK / 4 + 255) / 256);
   const float omb1 = 1.f - b1, omb2 = 1.f - b2, it = 1.f / tau;
-#define KQ_BWD(F, D)                                                                        \
-  k_kq_backward<F, D><<<g, 256, 0, c->st>>>(c->logits, c->mom, c->a, c->ma, c->b, c->mb,     \
-                                            c->q0, c->dW, c->probs, NK, it, lr, b1, omb1,   \
-                                            b2, omb2, c->dl, c->da, c->db)
+  const uint32_t k0 = (uint32_t)c->seed, k1 = (uint32_t)(c->seed >> 32);
+  const bool next = !dbg && next_tau > 0.f;
+  const float itn = next ? 1.f / next_tau : 0.f;
+#define KQ_BWD(F, D, X)                                                                    \
+  k_kq_backward<F, D, X><<<g, 256, 0, c->st>>>(                                              \
+      c->logits, c->mom, c->a, c->ma, c->b, c->mb, c->q0, c->dW, c->probs, NK, it, lr, b1,   \
+      omb1, b2, omb2, c->dl, c->da, c->db, k0, k1, (uint32_t)(c->t + 1), c->noise, itn,      \
+      c->What)
   if (c->fmt == KQ_Q2) {
-    if (dbg) KQ_BWD(KQ_Q2, true); else KQ_BWD(KQ_Q2, false);
+    if (dbg) KQ_BWD(KQ_Q2, true, false);
+    else if (next) KQ_BWD(KQ_Q2, false, true);
+    else KQ_BWD(KQ_Q2, false, false);
   } else {
-    if (dbg) KQ_BWD(KQ_Q3, true); else KQ_BWD(KQ_Q3, false);
+    if (dbg) KQ_BWD(KQ_Q3, true, false);
+    else if (next) KQ_BWD(KQ_Q3, false, true);
+    else KQ_BWD(KQ_Q3, false, false);
   }
 #undef KQ_BWD
   return cudaGetLastError();
@@ -662,17 +714,25 @@ cudaError_t kq_launch_dequant(int fmt, const uint8_t* blocks, int64_t nblk, __nv
   return cudaGetLastError();
 }
 
-int kq_step(gsq_kq* c, float tau, float lr, float b1, float b2) {
+// One step at tau; next_tau > 0: the backward also forms the soft weight of
+// the next step at next_tau (What and probs then hold step t + 1's, recorded
+// in what_t / what_tau, and the next step at that tau skips its own).
+int kq_step(gsq_kq* c, float tau, float lr, float b1, float b2, float next_tau = 0.f) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;
-  CKQ(kq_launch_soft(c, tau, nullptr));
+  if (!(c->what_t == (int64_t)c->t && c->what_tau == tau)) CKQ(kq_launch_soft(c, tau, nullptr));
+  c->what_t = -1;
   EpiParams ep = kq_epi(c, c->loss_hist + (c->t % kStageLossRing));
   CKQ(launch_gemm(c->tm_What, c->tm_Xb, c->em_forward, c->N, c->Tp, c->K, EPI_LOSS_DY, ep,
                   c->sms, c->st));
   EpiParams ep2 = kq_epi(c, nullptr);
   CKQ(launch_gemm(c->tm_dYt, c->tm_Xt, c->em_wgrad, c->N, c->K, c->Tp, EPI_STORE_F32, ep2,
                   c->sms, c->st));
-  CKQ(kq_launch_backward(c, tau, lr, b1, b2, false));
+  CKQ(kq_launch_backward(c, tau, lr, b1, b2, false, next_tau));
   c->t += 1;
+  if (next_tau > 0.f) {
+    c->what_t = (int64_t)c->t;
+    c->what_tau = next_tau;
+  }
   return GSQ_OK;
 }
 
@@ -890,7 +950,7 @@ int gsq_kq_run(gsq_kq* c, const float* taus, int64_t n, float lr, float beta1, f
   for (int64_t i = 0; i < n; ++i)
     if (!stage_step_args_ok(taus[i], lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
   for (int64_t i = 0; i < n; ++i) {
-    const int rc = kq_step(c, taus[i], lr, beta1, beta2);
+    const int rc = kq_step(c, taus[i], lr, beta1, beta2, i + 1 < n ? taus[i + 1] : 0.f);
     if (rc) return rc;
   }
   return GSQ_OK;
@@ -947,6 +1007,7 @@ int gsq_kq_recon_error(gsq_kq* c, int which, double* abs_err, double* rel_err) {
       k_kq_export<KQ_Q3><<<gq, 256, 0, c->st>>>(c->logits, c->a, c->b, c->q0, c->nblk, NK, c->exp);
     CKQ(cudaGetLastError());
   }
+  c->what_t = -1;  // What now holds the dequantized blocks
   CKQ(kq_launch_dequant(c->fmt, which == 0 ? c->exp : c->start, c->nblk, c->What, nullptr,
                         c->sms, c->st));
   CKQ(launch_gemm(c->tm_What, c->tm_Xb, c->em_forward, c->N, c->Tp, c->K, EPI_LOSS,
@@ -1029,6 +1090,7 @@ int gsq_kq_debug_set(gsq_kq* c, int which, const void* host, size_t bytes) {
   if (!host || bytes != need) return GSQ_ERR_INVALID_ARG;
   CKQ(cudaStreamSynchronize(c->st));
   CKQ(cudaMemcpy(p, host, need, cudaMemcpyHostToDevice));
+  c->what_t = -1;
   return GSQ_OK;
 }
 
@@ -1040,6 +1102,7 @@ int gsq_kq_debug_soft_weight(gsq_kq* c, float tau) {
   size_t need = 0;
   int rc = kq_buffer(c, GSQ_KQ_DBG_WSOFT32, &p, &need);
   if (rc) return rc;
+  c->what_t = -1;
   CKQ(kq_launch_soft(c, tau, c->wsoft32));
   return kq_check_device(c);
 }
@@ -1056,6 +1119,7 @@ int gsq_kq_debug_backward(gsq_kq* c, float tau, float lr, float beta1, float bet
   if (rc) return rc;
   // the step's probabilities (soft weight of step t), then the backward from
   // the current dW
+  c->what_t = -1;
   CKQ(kq_launch_soft(c, tau, nullptr));
   CKQ(kq_launch_backward(c, tau, lr, beta1, beta2, true));
   return kq_check_device(c);
@@ -1064,6 +1128,7 @@ int gsq_kq_debug_backward(gsq_kq* c, float tau, float lr, float beta1, float bet
 int gsq_kq_debug_noise(gsq_kq* c, int on) {
   if (!c) return GSQ_ERR_INVALID_ARG;
   c->noise = on ? 1 : 0;
+  c->what_t = -1;
   return GSQ_OK;
 }
 

@@ -202,3 +202,29 @@ def test_full_size_q_proj_row_slices(g, KQ):
             KQ.step(st, X, Y, float(tau), 1e-4)
         assert (logits[:, r] == st.logits[:, 0]).mean() > 0.995, r
         assert np.allclose(a[r], st.a[0], rtol=0, atol=3e-4)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_run_equals_step_loop(g, fmt):
+    """gsq_kq_run forms each next step's soft weight inside the backward;
+    a loop of gsq_kq_step forms it in a soft-weight pass of its own.  The two
+    must agree bit for bit, also after the debug entry points and the
+    reconstruction error (which reuse the soft-weight buffer) intervene."""
+    N, K, T = 136, 512, 120
+    W, X = case(N, K, T, number=97)
+    taus = synth.tau_schedule(1.0, 0.05, 12)
+    a, b = layer(g, W, X, fmt, seed=4), layer(g, W, X, fmt, seed=4)
+    for tau in taus[:6]:
+        a.step(float(tau), 1e-4)
+    b.run(taus[:6], 1e-4)
+    b.recon_error(1)
+    a.run(taus[6:], 1e-4)
+    for tau in taus[6:]:
+        b.step(float(tau), 1e-4)
+    for which in (g.GSQ_KQ_DBG_LOGITS, g.GSQ_KQ_DBG_MOM, g.GSQ_KQ_DBG_A, g.GSQ_KQ_DBG_MA,
+                  g.GSQ_KQ_DBG_B, g.GSQ_KQ_DBG_MB):
+        assert np.array_equal(a.get(which), b.get(which)), which
+    assert a.last_loss() == b.last_loss()
+    assert np.array_equal(a.export(), b.export())
+    a.close()
+    b.close()
