@@ -25,7 +25,8 @@
 // -2..+2 around the start code, clamped to [-4, 3]); soft weight
 // w = a_j sum_k y_k c_k - b_j with a_j, b_j continuous and trained by Lion
 // beside the logits (starting at d sc_j, dmin m_j); Gumbel noise as the 2-bit
-// (Q2_K) and 3-bit local (Q3_K) grids draw it.  Projection back: hard codes
+// (Q2_K) and 3-bit local (Q3_K) grids draw it, the outer logarithm as they
+// take it (logf for Q2_K, __logf for Q3_K).  Projection back: hard codes
 // by argmax, a_j and b_j re-encoded as the start encodes them.
 #include <cmath>
 #include <cstring>
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
       for (int p = 0; p < L; ++p)
         l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
       if (noise) {
-        coord_noise5((uint64_t)(c0 + j), t, k0, k1, L == 5, g);
+        coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t, k0, k1, L == 5, g);
       } else {
 #pragma unroll
         for (int p = 0; p < 5; ++p) g[p] = 0.f;
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(256) k_kq_backward(
 #pragma unroll
       for (int p = 0; p < L; ++p) l[p] = lo[p][j];
       if (noise) {
-        coord_noise5((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
+        coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
       } else {
 #pragma unroll
         for (int p = 0; p < 5; ++p) g[p] = 0.f;
