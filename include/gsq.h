@@ -132,9 +132,8 @@ GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const
  * read only.  levels (N x K int8 level indices, the init_idx of gsq_init)
  * and scales (N x K/group fp32): caller-owned, host or device.  damp >= 0
  * (GPTQ's default 0.01).  Synchronises the stream.  Its workspace (about
- * 8 K^2 + 8 N K bytes) comes from a memory pool the library owns per device,
- * which keeps up to 4 GiB reserved after the call so that the next call maps
- * no new memory; gsq_gptq_release_workspace returns it to the device.
+ * 8 K^2 + 8 N K bytes) comes from the library's memory pool (see
+ * gsq_release_cached_memory).
  * Errors: GSQ_ERR_INVALID_ARG for bad sizes / pointers / dtypes / damp or
  * K > 65536; GSQ_ERR_UNSUPPORTED for group != 128 or a non-sm_100 device;
  * GSQ_ERR_NONFINITE if the damped Hessian is not positive definite in fp32
@@ -142,10 +141,15 @@ GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const
 GSQ_API int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N,
                      int64_t K, int64_t T, int group, int grid_mode, float damp,
                      int8_t* levels, float* scales, void* stream);
-/* Returns the GPTQ workspace the library's pools keep reserved (all
- * devices) to the driver.  Call it with no gsq_gptq / gsq_init_gptq running.
- * Errors: GSQ_ERR_CUDA. */
-GSQ_API int gsq_gptq_release_workspace(void);
+/* Device memory: every buffer the library allocates (contexts of all kinds,
+ * init-time staging, the GPTQ workspace) comes from one memory pool per
+ * device that the library owns.  Freed memory stays reserved in the pool, up
+ * to 8 GiB per device, so that the next context or call of a similar size
+ * maps no new pages (mapping costs tens of milliseconds per GB).
+ * gsq_release_cached_memory returns what the pools hold in reserve (all
+ * devices) to the driver; memory of live contexts stays.  Call it with no
+ * library call running.  Errors: GSQ_ERR_CUDA. */
+GSQ_API int gsq_release_cached_memory(void);
 /* gsq_init from the GPTQ assignment: the initial levels (init_idx) and the
  * group scales both come from gsq_gptq (instead of round-to-nearest with
  * absmax scales); everything else as gsq_init.  Synchronises the stream. */

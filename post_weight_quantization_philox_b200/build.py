@@ -8,7 +8,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["gsq_api.cu", "gsq_gemm.cu", "gsq_gemm_pair.cu", "gsq_kernels.cu", "gsq_mlp.cu", "gsq_attn.cu", "gsq_noalloc.cu", "gsq_gptq.cu", "gsq_block.cu", "gsq_kquant.cu"]
+SOURCES = ["gsq_api.cu", "gsq_gemm.cu", "gsq_gemm_pair.cu", "gsq_kernels.cu", "gsq_mlp.cu", "gsq_attn.cu", "gsq_noalloc.cu", "gsq_gptq.cu", "gsq_block.cu", "gsq_kquant.cu", "gsq_pool.cu"]
 HEADERS = ["gsq_device.cuh", "gsq_internal.h", "gsq_gemm_epi.cuh", "gsq_stage.h"]
 LIB = os.path.join(PKG, "libgsq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -93,7 +93,7 @@ int fail(gsq_ctx* c, int status) {
 template <typename T>
 int dalloc(gsq_ctx* c, T** p, size_t count) {
   void* q = nullptr;
-  cudaError_t e = cudaMalloc(&q, count * sizeof(T) + 16);
+  cudaError_t e = pool_malloc(&q, count * sizeof(T) + 16);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GSQ_ERR_OOM;
@@ -104,7 +104,7 @@ int dalloc(gsq_ctx* c, T** p, size_t count) {
 }
 
 void free_all(gsq_ctx* c) {
-  for (void* p : c->allocs) cudaFree(p);
+  for (void* p : c->allocs) pool_free(p);
   c->allocs.clear();
   for (auto& te : c->tev)
     for (auto& e : te.ev) cudaEventDestroy(e);
@@ -224,10 +224,10 @@ int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void* X, int 
   if (N <= 0 || K <= 0 || group <= 0 || K % group != 0) return GSQ_ERR_INVALID_ARG;
   int8_t* lev = nullptr;
   float* sc = nullptr;
-  if (cudaMalloc(&lev, (size_t)N * K) != cudaSuccess ||
-      cudaMalloc(&sc, (size_t)N * (K / group) * 4) != cudaSuccess) {
+  if (pool_malloc(&lev, (size_t)N * K) != cudaSuccess ||
+      pool_malloc(&sc, (size_t)N * (K / group) * 4) != cudaSuccess) {
     cudaGetLastError();
-    cudaFree(lev);
+    pool_free(lev);
     return GSQ_ERR_OOM;
   }
   int rc = gsq_gptq(W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, damp, lev, sc, stream);
@@ -244,8 +244,8 @@ int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void* X, int 
       rc = GSQ_ERR_CUDA;
     }
   }
-  cudaFree(lev);
-  cudaFree(sc);
+  pool_free(lev);
+  pool_free(sc);
   return rc;
 }
 
@@ -330,7 +330,7 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   std::vector<void*> staging;
   auto salloc = [&](void** p, size_t bytes) {
     if (rc != GSQ_OK) return;
-    if (cudaMalloc(p, bytes) != cudaSuccess) {
+    if (pool_malloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
       rc = GSQ_ERR_OOM;
       return;
@@ -355,7 +355,7 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   auto cleanup_fail = [&](int status) {
     cudaStreamSynchronize(c->st);
     cudaGetLastError();
-    for (void* p : staging) cudaFree(p);
+    for (void* p : staging) pool_free(p);
     free_all(c);
     delete c;
     return status;
@@ -423,7 +423,7 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   if (h == DEV_ERR_BAD_INIT) return cleanup_fail(GSQ_ERR_INVALID_ARG);
   if (h != DEV_OK) return cleanup_fail(h == DEV_ERR_TIMEOUT ? GSQ_ERR_TIMEOUT : GSQ_ERR_CUDA);
   c->yref_sq = ysq;
-  for (void* p : staging) cudaFree(p);
+  for (void* p : staging) pool_free(p);
   *out = c;
   return GSQ_OK;
 #undef AL
@@ -604,7 +604,7 @@ int gsq_harden_pack(gsq_ctx* c, void* packed, uint16_t* scales_f16,
   const bool fd = !scales_f32 || is_device_ptr(scales_f32);
   void* stage = nullptr;
   size_t sbytes = (pd ? 0 : pbytes) + (hd ? 0 : ng * 2) + (fd ? 0 : ng * 4) + 64;
-  CK(cudaMalloc(&stage, sbytes));
+  CK(pool_malloc(&stage, sbytes));
   char* sp = static_cast<char*>(stage);
   uint32_t* pk = pd ? static_cast<uint32_t*>(packed) : reinterpret_cast<uint32_t*>(sp);
   if (!pd) sp += (pbytes + 15) / 16 * 16;
@@ -622,7 +622,7 @@ int gsq_harden_pack(gsq_ctx* c, void* packed, uint16_t* scales_f16,
   if (e == cudaSuccess && scales_f32 && !fd)
     e = cudaMemcpyAsync(scales_f32, f32, ng * 4, cudaMemcpyDefault, c->st);
   cudaError_t e2 = cudaStreamSynchronize(c->st);
-  cudaFree(stage);
+  pool_free(stage);
   if (e != cudaSuccess) return fail(c, cuda_status(e));
   if (e2 != cudaSuccess) return fail(c, cuda_status(e2));
   return check_device(c);
@@ -833,12 +833,12 @@ int gsq_debug_uniforms(gsq_ctx* c, uint32_t t, uint64_t coord0, int64_t count,
   if (u) return u;
   if (!host_out || count <= 0) return GSQ_ERR_INVALID_ARG;
   float* d = nullptr;
-  CK(cudaMalloc(&d, (size_t)count * c->L * 4));
+  CK(pool_malloc(&d, (size_t)count * c->L * 4));
   cudaError_t e = launch_uniforms(c->mode, c->seed, t, coord0, count, d, c->st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(c->st);
   if (e == cudaSuccess)
     e = cudaMemcpy(host_out, d, (size_t)count * c->L * 4, cudaMemcpyDeviceToHost);
-  cudaFree(d);
+  pool_free(d);
   if (e != cudaSuccess) return fail(c, cuda_status(e));
   return GSQ_OK;
 }
@@ -931,7 +931,7 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
       make_tmap_bf16(&tb, B, N, Kc, Kc, kGemmBoxRowsB))
     return GSQ_ERR_CUDA;
   int* err = nullptr;
-  if (cudaMalloc(&err, 16) != cudaSuccess) {
+  if (pool_malloc(&err, 16) != cudaSuccess) {
     cudaGetLastError();
     return GSQ_ERR_OOM;
   }
@@ -940,7 +940,7 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
   ep.err = err;
   EpiMaps em;
   if (make_tmap_epi_f32(&em.out, Cout, M, N, N)) {
-    cudaFree(err);
+    pool_free(err);
     return GSQ_ERR_CUDA;
   }
   em.yref = em.out;
@@ -950,7 +950,7 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   int h = 0;
   if (e == cudaSuccess) e = cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost);
-  cudaFree(err);
+  pool_free(err);
   if (e != cudaSuccess) return cuda_status(e);
   return h == DEV_OK ? GSQ_OK : GSQ_ERR_TIMEOUT;
 }

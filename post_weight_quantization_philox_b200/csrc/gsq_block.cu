@@ -223,13 +223,13 @@ struct Arena {
   ~Arena() {
     if (st) cudaStreamSynchronize(st);
     cudaGetLastError();
-    for (void* p : ptrs) cudaFree(p);
+    for (void* p : ptrs) pool_free(p);
   }
   template <typename T>
   T* get(size_t count) {
     if (status != GSQ_OK) return nullptr;
     void* p = nullptr;
-    if (cudaMalloc(&p, count * sizeof(T) + 16) != cudaSuccess) {
+    if (pool_malloc(&p, count * sizeof(T) + 16) != cudaSuccess) {
       cudaGetLastError();
       status = GSQ_ERR_OOM;
       return nullptr;
@@ -242,7 +242,7 @@ struct Arena {
     for (auto& q : ptrs)
       if (q == p) {
         cudaStreamSynchronize(st);
-        cudaFree(q);
+        pool_free(q);
         q = nullptr;
       }
   }

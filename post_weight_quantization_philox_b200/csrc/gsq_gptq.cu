@@ -28,7 +28,6 @@
 // This runs once per layer before the reconstruction steps; none of it is on
 // the per-step path.
 #include <cmath>
-#include <mutex>
 #include <vector>
 
 #include "../../include/gsq.h"
@@ -402,43 +401,10 @@ cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_
 
 }  // namespace
 
-// The GPTQ workspace comes from a memory pool of the library's own per
-// device, which keeps up to kPoolKeep bytes reserved between calls (a later
-// call of the same size then maps no new memory); gsq_gptq_release_workspace
-// hands it back.
-namespace {
-constexpr uint64_t kPoolKeep = 4ull << 30;
-constexpr int kMaxDevices = 64;
-std::mutex g_pool_mu;
-cudaMemPool_t g_pool[kMaxDevices] = {};
-}  // namespace
-
-cudaMemPool_t workspace_pool(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_pool_mu);
-  if (!g_pool[dev]) {
-    cudaMemPoolProps props = {};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.handleTypes = cudaMemHandleTypeNone;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t p = nullptr;
-    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
-      cudaGetLastError();
-      return nullptr;
-    }
-    uint64_t keep = kPoolKeep;
-    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
-    cudaGetLastError();
-    g_pool[dev] = p;
-  }
-  return g_pool[dev];
-}
-
 // GPTQ on device inputs; levels (N x K int8) and scales (N x K/128 fp32) are
 // device buffers.  Allocates its workspace stream-ordered on `st` from the
-// library's pool (no device synchronisation, unlike cudaMalloc / cudaFree),
-// synchronises the stream, frees.
+// library's pool (no device synchronisation, and the pool keeps the memory
+// for the next call), synchronises the stream, frees.
 int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype, int64_t N,
              int64_t K, int64_t T, float damp, int8_t* levels, float* scales, int sm_count,
              cudaStream_t st) {
@@ -446,7 +412,7 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   std::vector<void*> bufs;
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaMemPool_t pool = workspace_pool(dev);
+  cudaMemPool_t pool = library_pool(dev);
   bool oom = pool == nullptr;
   auto alloc = [&](size_t bytes) -> void* {
     void* p = nullptr;
@@ -598,7 +564,7 @@ int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, 
       *out = const_cast<void*>(p);
       return GSQ_OK;
     }
-    if (cudaMalloc(out, bytes) != cudaSuccess) {
+    if (pool_malloc(out, bytes) != cudaSuccess) {
       cudaGetLastError();
       return GSQ_ERR_OOM;
     }
@@ -625,19 +591,7 @@ int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int64_t N, 
     rc = GSQ_ERR_CUDA;
   cudaStreamSynchronize(st);
   cudaGetLastError();
-  for (void* p : tmp) cudaFree(p);
-  return rc;
-}
-
-int gsq_gptq_release_workspace(void) {
-  using namespace gsq;
-  std::lock_guard<std::mutex> lk(g_pool_mu);
-  int rc = GSQ_OK;
-  for (int d = 0; d < kMaxDevices; ++d)
-    if (g_pool[d] && cudaMemPoolTrimTo(g_pool[d], 0) != cudaSuccess) {
-      cudaGetLastError();
-      rc = GSQ_ERR_CUDA;
-    }
+  for (void* p : tmp) pool_free(p);
   return rc;
 }
 

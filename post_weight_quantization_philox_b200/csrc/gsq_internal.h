@@ -39,6 +39,19 @@ struct EpiMaps {
   CUtensorMap yref;
 };
 
+// Device memory of the library (gsq_pool.cu): one pool per device that keeps
+// freed memory reserved for the next allocation.  pool_malloc behaves as
+// cudaMalloc on the current device (usable on any stream once it returns),
+// pool_free as cudaFree (nothing in flight may still use the memory; null is
+// ignored).  library_pool gives the pool itself for stream-ordered use.
+cudaError_t pool_malloc(void** p, size_t bytes);
+template <typename T>
+inline cudaError_t pool_malloc(T** p, size_t bytes) {
+  return pool_malloc(reinterpret_cast<void**>(p), bytes);
+}
+void pool_free(void* p);
+cudaMemPool_t library_pool(int dev);
+
 // Encodes a 2-D bf16 tensor map (rows x cols, row stride ld elements) with
 // a box of box_rows x 64 elements and 128-byte swizzling (GEMM operands).
 int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows,

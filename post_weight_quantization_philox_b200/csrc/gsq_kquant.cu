@@ -619,7 +619,7 @@ int kq_fail(gsq_kq* c, int status) {
 template <typename T>
 int kq_alloc(gsq_kq* c, T** p, size_t count) {
   void* q = nullptr;
-  if (cudaMalloc(&q, count * sizeof(T) + 16) != cudaSuccess) {
+  if (pool_malloc(&q, count * sizeof(T) + 16) != cudaSuccess) {
     cudaGetLastError();
     return GSQ_ERR_OOM;
   }
@@ -629,7 +629,7 @@ int kq_alloc(gsq_kq* c, T** p, size_t count) {
 }
 
 void kq_free_all(gsq_kq* c) {
-  for (void* p : c->allocs) cudaFree(p);
+  for (void* p : c->allocs) pool_free(p);
   c->allocs.clear();
 }
 
@@ -838,7 +838,7 @@ int gsq_kq_init(gsq_kq** out, const void* W, int w_dtype, const void* X, int x_d
   std::vector<void*> staging;
   auto salloc = [&](void** p, size_t bytes) {
     if (rc != GSQ_OK) return;
-    if (cudaMalloc(p, bytes) != cudaSuccess) {
+    if (pool_malloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
       rc = GSQ_ERR_OOM;
       return;
@@ -848,7 +848,7 @@ int gsq_kq_init(gsq_kq** out, const void* W, int w_dtype, const void* X, int x_d
   auto cleanup_fail = [&](int status) {
     cudaStreamSynchronize(c->st);
     cudaGetLastError();
-    for (void* p : staging) cudaFree(p);
+    for (void* p : staging) pool_free(p);
     kq_free_all(c);
     delete c;
     return status;
@@ -932,7 +932,7 @@ int gsq_kq_init(gsq_kq** out, const void* W, int w_dtype, const void* X, int x_d
   if (h == DEV_ERR_NONFINITE) return cleanup_fail(GSQ_ERR_NONFINITE);
   if (h != DEV_OK) return cleanup_fail(h == DEV_ERR_TIMEOUT ? GSQ_ERR_TIMEOUT : GSQ_ERR_CUDA);
   c->yref_sq = ysq;
-  for (void* p : staging) cudaFree(p);
+  for (void* p : staging) pool_free(p);
   *out = c;
   return GSQ_OK;
 }
@@ -1041,7 +1041,7 @@ int gsq_kq_dequant(int format, const void* blocks, int64_t N, int64_t K, void* W
   auto dev_or_copy = [&](const void* p, size_t bytes, bool in) -> void* {
     if (stage_is_device_ptr(p)) return const_cast<void*>(p);
     void* q = nullptr;
-    if (cudaMalloc(&q, bytes) != cudaSuccess) {
+    if (pool_malloc(&q, bytes) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
@@ -1063,7 +1063,7 @@ int gsq_kq_dequant(int format, const void* blocks, int64_t N, int64_t K, void* W
     rc = GSQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess && rc == GSQ_OK) rc = GSQ_ERR_CUDA;
   cudaGetLastError();
-  for (void* p : tmp) cudaFree(p);
+  for (void* p : tmp) pool_free(p);
   return rc;
 }
 

@@ -91,7 +91,7 @@ int fail(gsq_mlp* c, int status) {
 template <typename T>
 int alloc(gsq_mlp* c, T** p, size_t count) {
   void* q = nullptr;
-  if (cudaMalloc(&q, count * sizeof(T) + 16) != cudaSuccess) {
+  if (pool_malloc(&q, count * sizeof(T) + 16) != cudaSuccess) {
     cudaGetLastError();
     return GSQ_ERR_OOM;
   }
@@ -101,7 +101,7 @@ int alloc(gsq_mlp* c, T** p, size_t count) {
 }
 
 void free_all(gsq_mlp* c) {
-  for (void* p : c->allocs) cudaFree(p);
+  for (void* p : c->allocs) pool_free(p);
   c->allocs.clear();
 }
 
@@ -304,7 +304,7 @@ int gsq_mlp_init(gsq_mlp** out, const void* Xn, int x_dtype, const void* R,
   std::vector<void*> staging;
   auto salloc = [&](void** p, size_t bytes) {
     if (rc != GSQ_OK) return;
-    if (cudaMalloc(p, bytes) != cudaSuccess) {
+    if (pool_malloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
       rc = GSQ_ERR_OOM;
       return;
@@ -314,7 +314,7 @@ int gsq_mlp_init(gsq_mlp** out, const void* Xn, int x_dtype, const void* R,
   auto cleanup_fail = [&](int status) {
     cudaStreamSynchronize(c->st);
     cudaGetLastError();
-    for (void* p : staging) cudaFree(p);
+    for (void* p : staging) pool_free(p);
     free_all(c);
     delete c;
     return status;
@@ -409,7 +409,7 @@ int gsq_mlp_init(gsq_mlp** out, const void* Xn, int x_dtype, const void* R,
   if (h == DEV_ERR_NONFINITE) return cleanup_fail(GSQ_ERR_NONFINITE);
   if (h != DEV_OK) return cleanup_fail(GSQ_ERR_CUDA);
   c->r_sq = rsq;
-  for (void* p : staging) cudaFree(p);
+  for (void* p : staging) pool_free(p);
   *out = c;
   return GSQ_OK;
 }
@@ -485,7 +485,7 @@ int gsq_mlp_harden_pack(gsq_mlp* c, int which, void* packed, uint16_t* scales_f1
   gsq_packed_bytes(c->mode, w.N, w.K, &pbytes);
   const int64_t ng = w.N * w.G;
   void* buf = nullptr;
-  CKM(cudaMalloc(&buf, pbytes + (size_t)ng * 6 + 64));
+  CKM(pool_malloc(&buf, pbytes + (size_t)ng * 6 + 64));
   uint32_t* pk = static_cast<uint32_t*>(buf);
   uint16_t* h16 = reinterpret_cast<uint16_t*>(static_cast<char*>(buf) + (pbytes + 15) / 16 * 16);
   float* f32 = reinterpret_cast<float*>(reinterpret_cast<char*>(h16) + ((size_t)ng * 2 + 15) / 16 * 16);
@@ -497,7 +497,7 @@ int gsq_mlp_harden_pack(gsq_mlp* c, int which, void* packed, uint16_t* scales_f1
   if (e == cudaSuccess && scales_f32)
     e = cudaMemcpyAsync(scales_f32, f32, (size_t)ng * 4, cudaMemcpyDefault, c->st);
   cudaError_t e2 = cudaStreamSynchronize(c->st);
-  cudaFree(buf);
+  pool_free(buf);
   if (e != cudaSuccess) return fail(c, cuda_status(e));
   if (e2 != cudaSuccess) return fail(c, cuda_status(e2));
   return check_device(c);

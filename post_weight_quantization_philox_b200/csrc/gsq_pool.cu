@@ -1,0 +1,131 @@
+// gsq_pool.cu -- the library's device memory.  Every buffer of a context
+// (layer, block stage, K-Quant), the init-time staging and the GPTQ
+// workspace come from one memory pool per device that the library owns.  The
+// pool keeps up to kPoolKeep bytes reserved after they are freed, so that the
+// next context or GPTQ call of a similar size maps no new pages: mapping
+// device memory costs tens of milliseconds per GB here, as much as hundreds
+// of reconstruction steps of a layer.  gsq_release_cached_memory hands the
+// reserve back to the driver.
+//
+// pool_malloc has cudaMalloc's contract (the memory may be used on any stream
+// once it returns): it allocates on a private stream of the device and
+// waits for that stream.  pool_free has cudaFree's (nothing in flight still
+// uses the memory): it frees on the same private stream, so a later
+// pool_malloc reuses the memory in stream order.
+#include <mutex>
+
+#include "../../include/gsq.h"
+#include "gsq_internal.h"
+
+namespace gsq {
+
+namespace {
+
+constexpr uint64_t kPoolKeep = 8ull << 30;
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+cudaStream_t g_stream[kMaxDevices] = {};
+
+// pool and private stream of device dev (created on first use); false when
+// either cannot be created
+bool device_pool(int dev, cudaMemPool_t* pool, cudaStream_t* stream) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    uint64_t keep = kPoolKeep;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    cudaGetLastError();
+    g_pool[dev] = p;
+  }
+  if (!g_stream[dev]) {
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    cudaStream_t s = nullptr;
+    const bool switched = cur != dev && cudaSetDevice(dev) == cudaSuccess;
+    const cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+    if (switched) cudaSetDevice(cur);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    g_stream[dev] = s;
+  }
+  *pool = g_pool[dev];
+  *stream = g_stream[dev];
+  return true;
+}
+
+}  // namespace
+
+cudaMemPool_t library_pool(int dev) {
+  cudaMemPool_t p = nullptr;
+  cudaStream_t s = nullptr;
+  return device_pool(dev, &p, &s) ? p : nullptr;
+}
+
+cudaError_t pool_malloc(void** p, size_t bytes) {
+  *p = nullptr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaMemPool_t pool = nullptr;
+  cudaStream_t s = nullptr;
+  if (!device_pool(dev, &pool, &s)) return cudaErrorMemoryAllocation;
+  e = cudaMallocFromPoolAsync(p, bytes, pool, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    if (*p) cudaFreeAsync(*p, s);
+    *p = nullptr;
+  }
+  return e;
+}
+
+void pool_free(void* p) {
+  if (!p) return;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  cudaMemPool_t pool = nullptr;
+  cudaStream_t s = nullptr;
+  if (device_pool(at.device, &pool, &s)) cudaFreeAsync(p, s);
+  cudaGetLastError();
+}
+
+}  // namespace gsq
+
+extern "C" {
+
+int gsq_release_cached_memory(void) {
+  using namespace gsq;
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = GSQ_OK;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (!g_pool[d]) continue;
+    // the frees queued on the private stream are done before the trim
+    if ((g_stream[d] && cudaStreamSynchronize(g_stream[d]) != cudaSuccess) ||
+        cudaMemPoolTrimTo(g_pool[d], 0) != cudaSuccess) {
+      cudaGetLastError();
+      rc = GSQ_ERR_CUDA;
+    }
+  }
+  return rc;
+}
+
+}  // extern "C"

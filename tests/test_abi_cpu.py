@@ -86,10 +86,10 @@ def test_null_context_handling(gsq):
                         None) == gsq.GSQ_ERR_INVALID_ARG
 
 
-def test_gptq_release_without_pools(gsq):
-    """With no GPTQ call made there is no pool to trim: a no-op that succeeds
+def test_release_without_pools(gsq):
+    """With no device allocation made there is no pool to trim: a no-op that succeeds
     without touching a device."""
-    assert gsq.lib().gsq_gptq_release_workspace() == gsq.GSQ_OK
+    assert gsq.lib().gsq_release_cached_memory() == gsq.GSQ_OK
 
 
 def test_binding_has_no_fallback(monkeypatch, tmp_path):

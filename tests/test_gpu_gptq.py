@@ -159,15 +159,15 @@ def test_full_size_q_proj_row_slices(g, oracle_mod):
 
 def test_repeat_calls_and_workspace_release(g):
     """The workspace pool changes nothing in the results: calls before and
-    after gsq_gptq_release_workspace agree bit for bit."""
+    after gsq_release_cached_memory agree bit for bit."""
     N, K, T = 200, 768, 384
     X = correlated(T, K, 9, outliers=3)
     W = np.random.default_rng(21).normal(0, 0.02, (N, K)).astype(np.float32)
     a = g.gsq_gptq(W, X, grid_mode=2)
     b = g.gsq_gptq(W, X, grid_mode=2)
-    g.gsq_gptq_release_workspace()
+    g.gsq_release_cached_memory()
     c = g.gsq_gptq(W, X, grid_mode=2)
-    g.gsq_gptq_release_workspace()
+    g.gsq_release_cached_memory()
     for x, y in ((a, b), (a, c)):
         assert np.array_equal(x[0], y[0])
         assert np.array_equal(x[1], y[1])
