@@ -376,14 +376,33 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
 
 // Backward + Lion from dW and the step's probabilities: per coordinate
 // dl_k = (a_j dw / tau) y_k sum_m y_m (c_k - c_m); per sub-block
-// da_j = sum dw v, db_j = -sum dw (the four threads of a sub-block combine
-// by shuffles, which leaves the same sum in all four); Lion on the logits,
-// a_j and (Q2_K) b_j.  With NEXT the kernel goes on to the soft weight of
-// step t_next at 1 / inv_tau_next from the updated logits, a_j and b_j --
-// the same arithmetic as k_kq_soft -- and writes it to What and its
-// probabilities over the ones it has just read.
+// da_j = sum dw v, db_j = -sum dw (the four lanes of a sub-block combine by
+// shuffles, which leaves the same sum in all four); Lion on the logits, a_j
+// and (Q2_K) b_j.  With NEXT the kernel goes on to the soft weight of step
+// t_next at 1 / inv_tau_next from the updated logits, a_j and b_j -- the same
+// arithmetic as k_kq_soft -- and writes it to What and its probabilities
+// over the ones it has just read.
+//
+// One warp per 128 consecutive coordinates (8 sub-blocks); lane j owns the
+// four coordinates 4j..4j+3.  The warp's next 128 coordinates are staged in
+// shared memory by per-lane 16-byte async copies (each lane copies exactly
+// what it will read) and their sub-block parameters loaded into registers
+// while the current ones are computed, so the loads of one group overlap the
+// arithmetic of the previous one.
+template <int F>
+struct KqBwdCfg {
+  static constexpr int L = KqT<F>::L;
+  // per-warp staging of 128 coordinates: dW, logits, momenta, probabilities, q0
+  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * 512, OFF_Y = OFF_M + L * 512;
+  static constexpr int OFF_Q = OFF_Y + L * 512;
+  static constexpr int BUF = OFF_Q + 128;
+  static constexpr int WARPS = L == 5 ? 4 : 8;  // warps per CTA
+  static constexpr int CTAS = L == 5 ? 3 : 2;   // CTAs per SM
+  static constexpr int SMEM = WARPS * 2 * BUF;
+};
+
 template <int F, bool DBG, bool NEXT>
-__global__ void __launch_bounds__(256) k_kq_backward(
+__global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_kq_backward(
     float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ a,
     float* __restrict__ ma, float* __restrict__ b, float* __restrict__ mb,
     const int8_t* __restrict__ q0, const float* __restrict__ dW, float* __restrict__ probs,
@@ -391,114 +410,154 @@ __global__ void __launch_bounds__(256) k_kq_backward(
     float* __restrict__ dl_dbg, float* __restrict__ da_dbg, float* __restrict__ db_dbg,
     uint32_t k0, uint32_t k1, uint32_t t_next, int noise, float inv_tau_next,
     __nv_bfloat16* __restrict__ What) {
-  constexpr int L = KqT<F>::L;
-  // NK / 4 is a multiple of 64 (K % 256 == 0), so this exit takes whole
-  // warps and the shuffles below always see all 32 lanes
-  const int64_t qd = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (qd >= NK / 4) return;
-  const int64_t c0 = qd * 4;
-  const int64_t sb = c0 / kSub;
-  const float aj = a[sb];
-  const float4 d4 = *reinterpret_cast<const float4*>(dW + c0);
-  const float dw[4] = {d4.x, d4.y, d4.z, d4.w};
-  const char4 qv = *reinterpret_cast<const char4*>(q0 + c0);
-  const int qq[4] = {qv.x, qv.y, qv.z, qv.w};
-  float4 lp[L], mp[L], yp[L];
-#pragma unroll
-  for (int p = 0; p < L; ++p) {
-    lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
-    mp[p] = *reinterpret_cast<const float4*>(mom + p * NK + c0);
-    yp[p] = *reinterpret_cast<const float4*>(probs + p * NK + c0);
-  }
-  float da_part = 0.f, db_part = 0.f;
-  float lo[L][4], mo[L][4], dlo[DBG ? L : 1][4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    float y[L], c[L];
-#pragma unroll
-    for (int p = 0; p < L; ++p)
-      y[p] = j == 0 ? yp[p].x : j == 1 ? yp[p].y : j == 2 ? yp[p].z : yp[p].w;
-    kq_cand<F>(qq[j], c);
-    float v = 0.f;
-#pragma unroll
-    for (int k = 0; k < L; ++k) v = fmaf(y[k], c[k], v);
-    da_part = fmaf(dw[j], v, da_part);
-    db_part -= dw[j];
-    const float s = aj * dw[j] * inv_tau;
+  using C = KqBwdCfg<F>;
+  constexpr int L = C::L;
+  extern __shared__ __align__(16) uint8_t kq_smem[];
+  const int64_t groups = NK / 128;  // K % 256 == 0
+  const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
+  const int64_t nwarps = (int64_t)gridDim.x * C::WARPS;
+  const uint32_t wbuf = smem_u32(kq_smem) + (uint32_t)(wic * 2 * C::BUF);
+  auto prefetch = [&](int64_t gi, int buf) {
+    const int64_t c = gi * 128 + 4 * lane;
+    const uint32_t d = wbuf + (uint32_t)(buf * C::BUF + 16 * lane);
+    cp_async16(d, dW + c);
 #pragma unroll
     for (int p = 0; p < L; ++p) {
-      float acc = 0.f;
+      cp_async16(d + (uint32_t)(C::OFF_L + p * 512), logits + p * NK + c);
+      cp_async16(d + (uint32_t)(C::OFF_M + p * 512), mom + p * NK + c);
+      cp_async16(d + (uint32_t)(C::OFF_Y + p * 512), probs + p * NK + c);
+    }
+    cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::OFF_Q + 4 * lane), q0 + c);
+  };
+  int64_t gi = (int64_t)blockIdx.x * C::WARPS + wic;
+  // the lane's sub-block parameters, one group ahead like the staging (each
+  // sub-block is read and written by the four lanes of one warp only)
+  auto params = [&](int64_t g, float* v) {
+    const int64_t sb = (g * 128 + 4 * lane) / kSub;
+    v[0] = a[sb];
+    v[1] = ma[sb];
+    v[2] = b[sb];
+    v[3] = F == KQ_Q2 ? mb[sb] : 0.f;
+  };
+  float pn[4] = {0.f, 0.f, 0.f, 0.f};
+  if (gi < groups) {
+    prefetch(gi, 0);
+    params(gi, pn);
+  }
+  cp_async_commit();
+  for (int buf = 0; gi < groups; gi += nwarps, buf ^= 1) {
+    const float aj = pn[0], maj = pn[1], bj = pn[2], mbj = pn[3];
+    if (gi + nwarps < groups) {
+      prefetch(gi + nwarps, buf ^ 1);
+      params(gi + nwarps, pn);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();  // this lane's copies of group gi have landed
+    const uint8_t* sbuf = kq_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
+    const int64_t c0 = gi * 128 + 4 * lane;
+    const int64_t sb = c0 / kSub;
+    float dw[4], lr_[L][4], mr[L][4], yr[L][4];
+    *reinterpret_cast<float4*>(dw) = *reinterpret_cast<const float4*>(sbuf);
 #pragma unroll
-      for (int k = 0; k < L; ++k) acc = fmaf(y[k], c[p] - c[k], acc);
-      const float g = s * y[p] * acc;
-      float th = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
-      float mm = j == 0 ? mp[p].x : j == 1 ? mp[p].y : j == 2 ? mp[p].z : mp[p].w;
-      lion_update(th, mm, g, lr, b1, omb1, b2, omb2);
-      lo[p][j] = th;
-      mo[p][j] = mm;
-      if (DBG) dlo[DBG ? p : 0][j] = g;
+    for (int p = 0; p < L; ++p) {
+      *reinterpret_cast<float4*>(lr_[p]) =
+          *reinterpret_cast<const float4*>(sbuf + C::OFF_L + p * 512);
+      *reinterpret_cast<float4*>(mr[p]) =
+          *reinterpret_cast<const float4*>(sbuf + C::OFF_M + p * 512);
+      *reinterpret_cast<float4*>(yr[p]) =
+          *reinterpret_cast<const float4*>(sbuf + C::OFF_Y + p * 512);
     }
-  }
+    const uint32_t q4 = *reinterpret_cast<const uint32_t*>(
+        kq_smem + wic * 2 * C::BUF + buf * C::BUF + C::OFF_Q + 4 * lane);
+    int qq[4];
 #pragma unroll
-  for (int p = 0; p < L; ++p) {
-    *reinterpret_cast<float4*>(logits + p * NK + c0) = make_float4(lo[p][0], lo[p][1], lo[p][2], lo[p][3]);
-    *reinterpret_cast<float4*>(mom + p * NK + c0) = make_float4(mo[p][0], mo[p][1], mo[p][2], mo[p][3]);
-    if (DBG)
-      *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
-          make_float4(dlo[DBG ? p : 0][0], dlo[DBG ? p : 0][1], dlo[DBG ? p : 0][2], dlo[DBG ? p : 0][3]);
-  }
-  // the four threads of the sub-block (lanes 4k..4k+3)
-  da_part += __shfl_xor_sync(0xffffffffu, da_part, 1);
-  da_part += __shfl_xor_sync(0xffffffffu, da_part, 2);
-  db_part += __shfl_xor_sync(0xffffffffu, db_part, 1);
-  db_part += __shfl_xor_sync(0xffffffffu, db_part, 2);
-  // every lane of the sub-block updates its parameters alike; the first stores
-  float av = aj, mav = ma[sb], bv = b[sb], mbv = 0.f;
-  lion_update(av, mav, da_part, lr, b1, omb1, b2, omb2);
-  if (F == KQ_Q2) {
-    mbv = mb[sb];
-    lion_update(bv, mbv, db_part, lr, b1, omb1, b2, omb2);
-  }
-  if ((threadIdx.x & 3) == 0) {
-    a[sb] = av;
-    ma[sb] = mav;
-    if (F == KQ_Q2) {
-      b[sb] = bv;
-      mb[sb] = mbv;
-    }
-    if (DBG) {
-      da_dbg[sb] = da_part;
-      db_dbg[sb] = db_part;
-    }
-  }
-  if (NEXT) {
-    float wv[4], yy[4][L];
+    for (int j = 0; j < 4; ++j) qq[j] = (int)(int8_t)((q4 >> (8 * j)) & 0xFFu);
+    float da_part = 0.f, db_part = 0.f;
+    float lo[L][4], mo[L][4], dlo[DBG ? L : 1][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float l[L], g[5], c[L];
+      float y[L], c[L];
 #pragma unroll
-      for (int p = 0; p < L; ++p) l[p] = lo[p][j];
-      if (noise) {
-        coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
-      } else {
-#pragma unroll
-        for (int p = 0; p < 5; ++p) g[p] = 0.f;
-      }
+      for (int p = 0; p < L; ++p) y[p] = yr[p][j];
       kq_cand<F>(qq[j], c);
-      const float v = kq_soft<L>(l, g, inv_tau_next, c, yy[j]);
-      wv[j] = fmaf(av, v, -bv);
-    }
-    __nv_bfloat162 p01 = __floats2bfloat162_rn(wv[0], wv[1]);
-    __nv_bfloat162 p23 = __floats2bfloat162_rn(wv[2], wv[3]);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&p01);
-    pk.y = *reinterpret_cast<uint32_t*>(&p23);
-    *reinterpret_cast<uint2*>(What + c0) = pk;
+      float v = 0.f;
 #pragma unroll
-    for (int p = 0; p < L; ++p)
-      *reinterpret_cast<float4*>(probs + p * NK + c0) =
-          make_float4(yy[0][p], yy[1][p], yy[2][p], yy[3][p]);
+      for (int k = 0; k < L; ++k) v = fmaf(y[k], c[k], v);
+      da_part = fmaf(dw[j], v, da_part);
+      db_part -= dw[j];
+      const float sc = aj * dw[j] * inv_tau;
+#pragma unroll
+      for (int p = 0; p < L; ++p) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < L; ++k) acc = fmaf(y[k], c[p] - c[k], acc);
+        const float g = sc * y[p] * acc;
+        float th = lr_[p][j], mm = mr[p][j];
+        lion_update(th, mm, g, lr, b1, omb1, b2, omb2);
+        lo[p][j] = th;
+        mo[p][j] = mm;
+        if (DBG) dlo[DBG ? p : 0][j] = g;
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < L; ++p) {
+      *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(lo[p]);
+      *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(mo[p]);
+      if (DBG)
+        *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
+            *reinterpret_cast<float4*>(dlo[DBG ? p : 0]);
+    }
+    // the four lanes of the sub-block (lanes 4k..4k+3)
+    da_part += __shfl_xor_sync(0xffffffffu, da_part, 1);
+    da_part += __shfl_xor_sync(0xffffffffu, da_part, 2);
+    db_part += __shfl_xor_sync(0xffffffffu, db_part, 1);
+    db_part += __shfl_xor_sync(0xffffffffu, db_part, 2);
+    // every lane of the sub-block updates its parameters alike; the first stores
+    float av = aj, mav = maj, bv = bj, mbv = mbj;
+    lion_update(av, mav, da_part, lr, b1, omb1, b2, omb2);
+    if (F == KQ_Q2) lion_update(bv, mbv, db_part, lr, b1, omb1, b2, omb2);
+    if ((lane & 3) == 0) {
+      a[sb] = av;
+      ma[sb] = mav;
+      if (F == KQ_Q2) {
+        b[sb] = bv;
+        mb[sb] = mbv;
+      }
+      if (DBG) {
+        da_dbg[sb] = da_part;
+        db_dbg[sb] = db_part;
+      }
+    }
+    if (NEXT) {
+      float wv[4], yy[4][L];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float l[L], g[5], c[L];
+#pragma unroll
+        for (int p = 0; p < L; ++p) l[p] = lo[p][j];
+        if (noise) {
+          coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
+        } else {
+#pragma unroll
+          for (int p = 0; p < 5; ++p) g[p] = 0.f;
+        }
+        kq_cand<F>(qq[j], c);
+        const float v = kq_soft<L>(l, g, inv_tau_next, c, yy[j]);
+        wv[j] = fmaf(av, v, -bv);
+      }
+      __nv_bfloat162 p01 = __floats2bfloat162_rn(wv[0], wv[1]);
+      __nv_bfloat162 p23 = __floats2bfloat162_rn(wv[2], wv[3]);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&p01);
+      pk.y = *reinterpret_cast<uint32_t*>(&p23);
+      *reinterpret_cast<uint2*>(What + c0) = pk;
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        *reinterpret_cast<float4*>(probs + p * NK + c0) =
+            make_float4(yy[0][p], yy[1][p], yy[2][p], yy[3][p]);
+    }
   }
+  cp_async_wait<0>();
 }
 
 // Projection back into the format: hard codes (argmax, first maximum) and
@@ -681,30 +740,40 @@ cudaError_t kq_launch_soft(gsq_kq* c, float tau, float* wsoft32) {
 
 // The backward of step t; next_tau > 0 (not with dbg): also the soft weight
 // of step t + 1 at next_tau.
+template <int F, bool DBG, bool NEXT>
+cudaError_t kq_backward_launch(gsq_kq* c, float it, float lr, float b1, float b2, float itn) {
+  using Cf = KqBwdCfg<F>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        k_kq_backward<F, DBG, NEXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int64_t NK = c->N * c->K, groups = NK / 128;
+  const int64_t need = (groups + Cf::WARPS - 1) / Cf::WARPS;
+  const int64_t cap = (int64_t)c->sms * Cf::CTAS;
+  const unsigned blocks = (unsigned)(need < cap ? need : cap);
+  k_kq_backward<F, DBG, NEXT><<<blocks, Cf::WARPS * 32, Cf::SMEM, c->st>>>(
+      c->logits, c->mom, c->a, c->ma, c->b, c->mb, c->q0, c->dW, c->probs, NK, it, lr, b1,
+      1.f - b1, b2, 1.f - b2, c->dl, c->da, c->db, (uint32_t)c->seed,
+      (uint32_t)(c->seed >> 32), (uint32_t)(c->t + 1), c->noise, itn, c->What);
+  return cudaGetLastError();
+}
+
 cudaError_t kq_launch_backward(gsq_kq* c, float tau, float lr, float b1, float b2, bool dbg,
                                float next_tau = 0.f) {
-  const int64_t NK = c->N * c->K;
-  const unsigned g = (unsigned)((NK / 4 + 255) / 256);
-  const float omb1 = 1.f - b1, omb2 = 1.f - b2, it = 1.f / tau;
-  const uint32_t k0 = (uint32_t)c->seed, k1 = (uint32_t)(c->seed >> 32);
+  const float it = 1.f / tau;
   const bool next = !dbg && next_tau > 0.f;
   const float itn = next ? 1.f / next_tau : 0.f;
-#define KQ_BWD(F, D, X)                                                                    \
-  k_kq_backward<F, D, X><<<g, 256, 0, c->st>>>(                                              \
-      c->logits, c->mom, c->a, c->ma, c->b, c->mb, c->q0, c->dW, c->probs, NK, it, lr, b1,   \
-      omb1, b2, omb2, c->dl, c->da, c->db, k0, k1, (uint32_t)(c->t + 1), c->noise, itn,      \
-      c->What)
   if (c->fmt == KQ_Q2) {
-    if (dbg) KQ_BWD(KQ_Q2, true, false);
-    else if (next) KQ_BWD(KQ_Q2, false, true);
-    else KQ_BWD(KQ_Q2, false, false);
-  } else {
-    if (dbg) KQ_BWD(KQ_Q3, true, false);
-    else if (next) KQ_BWD(KQ_Q3, false, true);
-    else KQ_BWD(KQ_Q3, false, false);
+    if (dbg) return kq_backward_launch<KQ_Q2, true, false>(c, it, lr, b1, b2, itn);
+    if (next) return kq_backward_launch<KQ_Q2, false, true>(c, it, lr, b1, b2, itn);
+    return kq_backward_launch<KQ_Q2, false, false>(c, it, lr, b1, b2, itn);
   }
-#undef KQ_BWD
-  return cudaGetLastError();
+  if (dbg) return kq_backward_launch<KQ_Q3, true, false>(c, it, lr, b1, b2, itn);
+  if (next) return kq_backward_launch<KQ_Q3, false, true>(c, it, lr, b1, b2, itn);
+  return kq_backward_launch<KQ_Q3, false, false>(c, it, lr, b1, b2, itn);
 }
 
 cudaError_t kq_launch_dequant(int fmt, const uint8_t* blocks, int64_t nblk, __nv_bfloat16* W,
