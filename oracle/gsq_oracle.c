@@ -105,24 +105,34 @@ float gsqo_u01(uint32_t x) {
     return (float)u;
 }
 
-/* Counter layout: ctr = (coord low word, coord high word, step t, block w),
- * key = (seed low word, seed high word).  Words used per coordinate:
- *   2-bit       block 0 words 0..3  -> logits 0..3
+/* Counter layout: ctr = (low word, high word, step t, block), key = (seed
+ * low word, seed high word).  Words used per coordinate:
+ *   2-bit       block 0 of the coordinate, words 0..3  -> logits 0..3
  *   ternary     block 0 words 0,1   -> mask (zero, nonzero)
  *               block 0 words 2,3   -> sign (minus, plus)
- *   3-bit local block 0 words 0..3 and block 1 word 0 -> shifts -2..+2 */
-static void coord_uniforms(int mode, uint64_t seed, uint32_t t, uint64_t coord,
-                           float* u) {
+ *   3-bit local block 0 words 0..3 -> shifts -2..+1, and for shift +2 word
+ *               coord % 4 of block 1 of the aligned quad's first coordinate
+ *               coord - coord % 4 (the quad's four coordinates take the four
+ *               words of one block-1 draw). */
+static void coord_words(int mode, uint64_t seed, uint32_t t, uint64_t coord,
+                        uint32_t* w) {
     uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
     uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t, 0u};
-    uint32_t out[4];
-    gsqo_philox4x32_10(ctr, key, out);
-    for (int j = 0; j < 4; ++j) u[j] = gsqo_u01(out[j]);
+    gsqo_philox4x32_10(ctr, key, w);
     if (mode == GSQO_GRID_3BIT_LOCAL) {
-        ctr[3] = 1u;
-        gsqo_philox4x32_10(ctr, key, out);
-        u[4] = gsqo_u01(out[0]);
+        uint32_t out[4];
+        uint64_t q = coord - coord % 4;
+        uint32_t ctr1[4] = {(uint32_t)q, (uint32_t)(q >> 32), t, 1u};
+        gsqo_philox4x32_10(ctr1, key, out);
+        w[4] = out[coord % 4];
     }
+}
+
+static void coord_uniforms(int mode, uint64_t seed, uint32_t t, uint64_t coord,
+                           float* u) {
+    uint32_t w[5];
+    coord_words(mode, seed, t, coord, w);
+    for (int j = 0; j < gsqo_num_logits(mode); ++j) u[j] = gsqo_u01(w[j]);
 }
 
 void gsqo_uniforms(int mode, uint64_t seed, uint32_t t, uint64_t coord0,
@@ -553,16 +563,10 @@ void gsqo_state16_store(int mode, int64_t row0, int64_t N, int64_t K,
                         float* mom) {
     const int L = gsqo_num_logits(mode);
     const int64_t NK = N * K;
-    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
     for (int64_t i = 0; i < NK; ++i) {
         const uint64_t coord = (uint64_t)(row0 * K + i);
-        uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next, 0u};
-        uint32_t w[8];
-        gsqo_philox4x32_10(ctr, key, w);
-        if (L == 5) {
-            ctr[3] = 1u;
-            gsqo_philox4x32_10(ctr, key, w + 4);
-        }
+        uint32_t w[5];
+        coord_words(mode, seed, t_next, coord, w);
         for (int p = 0; p < L; ++p) {
             logits[p * NK + i] = gsqo_bf16_sr(logits[p * NK + i], w[p]);
             mom[p * NK + i] = (float)gsqo_bf16_round((double)mom[p * NK + i]);

@@ -88,9 +88,13 @@ MUTATIONS = [
      ["state16:test_rounding_follows_fp32_lion_on_average",
       "state16:test_thresholds_are_next_step_philox_words"]),
     ("state16_thresholds_this_step",
-     "uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next, 0u};",
-     "uint32_t ctr[4] = {(uint32_t)coord, (uint32_t)(coord >> 32), t_next - 1u, 0u};",
+     "coord_words(mode, seed, t_next, coord, w);",
+     "coord_words(mode, seed, t_next - 1u, coord, w);",
      ["state16:test_thresholds_are_next_step_philox_words"]),
+    ("quad_word_fixed", "w[4] = out[coord % 4];", "w[4] = out[0];",
+     ["test_counter_layout"]),
+    ("quad_block_per_coordinate", "uint64_t q = coord - coord % 4;", "uint64_t q = coord;",
+     ["test_counter_layout"]),
     ("state16_threshold_scale", "b += (r9 & 0x1FFu) << 7;", "b += (r9 & 0x1FFu) << 6;",
      ["state16:test_stochastic_rounding_brackets_and_is_unbiased"]),
     ("state16_momenta_truncated",

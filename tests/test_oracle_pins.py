@@ -61,8 +61,10 @@ def test_counter_layout(oracle_mod):
             w0 = oracle_mod.philox4x32_10([c & 0xFFFFFFFF, c >> 32, 7, 0], key)
             ref = [oracle_mod.u01(int(x)) for x in w0]
             if mode == 2:
-                w1 = oracle_mod.philox4x32_10([c & 0xFFFFFFFF, c >> 32, 7, 1], key)
-                ref.append(oracle_mod.u01(int(w1[0])))
+                # word c % 4 of the block-1 draw of the aligned quad's first coordinate
+                q = c - c % 4
+                w1 = oracle_mod.philox4x32_10([q & 0xFFFFFFFF, q >> 32, 7, 1], key)
+                ref.append(oracle_mod.u01(int(w1[c % 4])))
             assert list(u[i]) == ref
 
 
