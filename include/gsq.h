@@ -17,7 +17,9 @@
  * Notation: W (N x K) is the layer weight, X (T x K) the calibration inputs,
  * G = K / group groups per row, L logits per coordinate (4, 2+2, 5),
  * coord = n*K + k.  One step t computes
- *     u   = Philox4x32-10(key = seed, ctr = (coord lo, coord hi, t, block))
+ *     u   = Philox4x32-10(key = seed, ctr = (coord lo, coord hi, t, 0)), words
+ *           0..3; the 3-bit grid's fifth: word coord % 4 of the block of
+ *           ctr = (q lo, q hi, t, 1), q = coord - coord % 4
  *     g   = -log(-log u),  y = softmax((l + g) / tau),  v = sum y_k c_k,
  *     What = bf16(s_g * v),
  *     loss = || X What^T - X W^T ||_F^2,   dY = 2 E,   dWhat = dY^T X,

@@ -468,21 +468,33 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     if (S16) {
       // the Philox words of step t + 1 give the next step's noise (NEXT) and
       // the rounding thresholds of this step's update
+      uint32_t wd[4][5];
+      quad_words5((uint64_t)c0, t_next, k0, k1, L == 5, wd);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        uint32_t wd[5];
-        coord_words5((uint64_t)(c0 + j), t_next, k0, k1, L == 5, wd);
 #pragma unroll
         for (int p = 0; p < L; ++p) {
-          rsr[S16 ? j : 0][p] = wd[p];
+          rsr[S16 ? j : 0][p] = wd[j][p];
           if (NEXT)
             gnext[NEXT ? j : 0][p] =
-                noise ? gumbel<GridT<MODE>::FAST_GUMBEL>(word_to_unit(wd[p])) : 0.f;
+                noise ? gumbel<GridT<MODE>::FAST_GUMBEL>(word_to_unit(wd[j][p])) : 0.f;
         }
       }
     } else if (NEXT) {
+      // the lane's four coordinates form an aligned quad (c0 % 4 == 0)
+      float gq[4][5];
+      if (noise) {
+        quad_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c0, t_next, k0, k1, L == 5, gq);
+      } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) noise1<MODE>(c0 + j, t_next, k0, k1, noise, gnext[NEXT ? j : 0]);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int p = 0; p < L; ++p) gnext[NEXT ? j : 0][p] = gq[j][p];
     }
     float ds_part = 0.f;
     float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
@@ -790,17 +802,10 @@ __global__ void k_uniforms(uint64_t seed, uint32_t t, uint64_t coord0,
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
        i += (int64_t)gridDim.x * blockDim.x) {
     const uint64_t c = coord0 + (uint64_t)i;
-    const uint4 r = philox4x32_10(
-        make_uint4((uint32_t)c, (uint32_t)(c >> 32), t, 0u), k0, k1);
-    out[i * L + 0] = word_to_unit(r.x);
-    out[i * L + 1] = word_to_unit(r.y);
-    out[i * L + 2] = word_to_unit(r.z);
-    out[i * L + 3] = word_to_unit(r.w);
-    if (L == 5) {
-      const uint4 r2 = philox4x32_10(
-          make_uint4((uint32_t)c, (uint32_t)(c >> 32), t, 1u), k0, k1);
-      out[i * L + 4] = word_to_unit(r2.x);
-    }
+    uint32_t w[5];
+    coord_words5(c, t, k0, k1, L == 5, w);
+#pragma unroll
+    for (int p = 0; p < L; ++p) out[i * L + p] = word_to_unit(w[p]);
   }
 }
 

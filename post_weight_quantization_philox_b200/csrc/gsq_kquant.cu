@@ -341,19 +341,22 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
     float4 lp[L];
 #pragma unroll
     for (int p = 0; p < L; ++p) lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
-    float wv[4], yy[4][L];
+    float wv[4], yy[4][L], gq[4][5];
+    if (noise) {
+      quad_noise5<F == KQ_Q3>((uint64_t)c0, t, k0, k1, L == 5, gq);  // c0 % 4 == 0
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float l[L], g[5], c[L];
+      float l[L], c[L];
+      const float* g = gq[j];
 #pragma unroll
       for (int p = 0; p < L; ++p)
         l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
-      if (noise) {
-        coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t, k0, k1, L == 5, g);
-      } else {
-#pragma unroll
-        for (int p = 0; p < 5; ++p) g[p] = 0.f;
-      }
       kq_cand<F>(qq[j], c);
       const float v = kq_soft<L>(l, g, inv_tau, c, yy[j]);
       wv[j] = fmaf(aj, v, -bj);
@@ -529,18 +532,21 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
       }
     }
     if (NEXT) {
-      float wv[4], yy[4][L];
+      float wv[4], yy[4][L], gq[4][5];
+      if (noise) {
+        quad_noise5<F == KQ_Q3>((uint64_t)c0, t_next, k0, k1, L == 5, gq);  // c0 % 4 == 0
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float l[L], g[5], c[L];
+        float l[L], c[L];
+        const float* g = gq[j];
 #pragma unroll
         for (int p = 0; p < L; ++p) l[p] = lo[p][j];
-        if (noise) {
-          coord_noise5<F == KQ_Q3>((uint64_t)(c0 + j), t_next, k0, k1, L == 5, g);
-        } else {
-#pragma unroll
-          for (int p = 0; p < 5; ++p) g[p] = 0.f;
-        }
         kq_cand<F>(qq[j], c);
         const float v = kq_soft<L>(l, g, inv_tau_next, c, yy[j]);
         wv[j] = fmaf(av, v, -bv);
