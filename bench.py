@@ -130,13 +130,14 @@ def run_gsq(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     cfg = synth.CONFIGS[args.config]
     # each rank quantizes its own independent layer of the same shape
-    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
-    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    w_seed, x_seed, _ = layer_seeds(cfg, rank)
+    W = synth.make_weight(cfg, seed=w_seed)
+    X = synth.make_calib(cfg, seed=x_seed)
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
     stream = torch.cuda.current_stream()
     state16 = args.state == "bf16"
-    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=rank, state_bf16=state16)
+    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=layer_seeds(cfg, rank)[2], state_bf16=state16)
     taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
     nt = len(taus)
 
@@ -171,11 +172,7 @@ def run_gsq(args, rank, world, local_rank):
     del Wd, Xd
     torch.cuda.empty_cache()
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
 
     # ---- end to end: host buffers through the C ABI, whole quantization job
     e2e = None if args.no_e2e else run_e2e(gsq, torch, cfg, W, X, rank)
@@ -185,7 +182,7 @@ def run_gsq(args, rank, world, local_rank):
     hbm, tf_burst, tf_sus, peak_kind = peaks()
     steps_per_s = args.steps / (ms / 1e3)
     coords = cfg.N * cfg.K
-    value = world * coords * steps_per_s
+    value = whole_job_rate(world, coords * args.steps, ms)
     names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion",
              "backward_lion_next_soft"]
     es = 2 if state16 else 4
@@ -319,6 +316,33 @@ def kernel_sources_hash():
     return hashlib.sha256(blob).hexdigest()[:16]
 
 
+def rank_seed(base: int, rank: int) -> int:
+    """Data seed of rank's own problem: every rank quantizes an independent
+    layer (or stage) of the same shape, so the ranks never exchange data."""
+    return base + 7919 * rank
+
+
+def layer_seeds(cfg, rank):
+    """(W seed, X seed, Philox seed) of rank's independent layer."""
+    return rank_seed(1000 + cfg.number, rank), rank_seed(2000 + cfg.number, rank), rank
+
+
+def max_over_ranks(ms: float, world: int, device="cuda") -> float:
+    """The job's time: the slowest rank's device-timed region."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Units all ranks processed per second of the job's (max-over-ranks) time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def run_mlp_stage(args, rank, world, local_rank):
     """The 70B block's MLP stage (gate/up/down quantized jointly on 16384
     tokens): whole-stage steps through gsq_mlp_run."""
@@ -329,8 +353,8 @@ def run_mlp_stage(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     cfg = synth.MLP_STAGE["c5_70b_mlp"]
     T, H, F = cfg["T"], cfg["H"], cfg["F"]
-    Xn, Wg, Wu, Wd = synth.make_mlp_stage(T, H, F, seed=5005 + 7919 * rank)
-    R = synth.random_target(T, H, 0.05, seed=5006 + 7919 * rank)
+    Xn, Wg, Wu, Wd = synth.make_mlp_stage(T, H, F, seed=rank_seed(5005, rank))
+    R = synth.random_target(T, H, 0.05, seed=rank_seed(5006, rank))
     dev = lambda x: torch.from_numpy(x).to(torch.bfloat16).cuda()
     m = gsq.gsq_mlp_init(dev(Xn), torch.from_numpy(R).cuda(), dev(Wg), dev(Wu), dev(Wd),
                          grid_mode=cfg["grid"], seed=rank)
@@ -356,11 +380,7 @@ def run_mlp_stage(args, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     loss = m.last_loss()
     m.close()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     hbm, tf_burst, tf_sus, peak_kind = peaks()
@@ -368,7 +388,7 @@ def run_mlp_stage(args, rank, world, local_rank):
     coords = 3 * H * F
     flops = 7 * 2.0 * T * H * F
     ach = flops / (per / 1e3) / 1e12
-    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
             "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
@@ -391,9 +411,9 @@ def run_attn_stage(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     cfg = synth.ATTN_STAGE["c5_70b_attn"]
     dims = dict(nseq=cfg["nseq"], S=cfg["S"], nh=cfg["nh"], nkv=cfg["nkv"], d=cfg["d"])
-    Xa, Wq, Wk, Wv, Wo = synth.make_attn_stage(**dims, seed=6006 + 7919 * rank)
+    Xa, Wq, Wk, Wv, Wo = synth.make_attn_stage(**dims, seed=rank_seed(6006, rank))
     T, H = Xa.shape
-    R = synth.random_target(T, H, 0.05, seed=6007 + 7919 * rank)
+    R = synth.random_target(T, H, 0.05, seed=rank_seed(6007, rank))
     dev = lambda x: torch.from_numpy(x).to(torch.bfloat16).cuda()
     a = gsq.gsq_attn_init(dev(Xa), torch.from_numpy(R).cuda(), dev(Wq), dev(Wk), dev(Wv),
                           dev(Wo), dims["nseq"], dims["S"], dims["nh"], dims["nkv"],
@@ -420,11 +440,7 @@ def run_attn_stage(args, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     loss = a.last_loss()
     a.close()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     hbm, tf_burst, tf_sus, peak_kind = peaks()
@@ -436,7 +452,7 @@ def run_attn_stage(args, rank, world, local_rank):
     # products with the causal P count its nonzero half only
     flops = 2.0 * (2 * T * H * Hk + 3 * T * H * H) + 2 * 2.0 * dims["nseq"] * nh * d * S * (S + 1) / 2
     ach = flops / (per / 1e3) / 1e12
-    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
             "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
@@ -459,8 +475,9 @@ def run_scale_stage(args, rank, world, local_rank):
     from post_weight_quantization_philox_b200 import gsq
     torch.cuda.set_device(local_rank)
     cfg = synth.CONFIGS[args.config]
-    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
-    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    w_seed, x_seed, _ = layer_seeds(cfg, rank)
+    W = synth.make_weight(cfg, seed=w_seed)
+    X = synth.make_calib(cfg, seed=x_seed)
     lay = gsq.gsq_init(torch.from_numpy(W).to(torch.bfloat16).cuda(),
                        torch.from_numpy(X).to(torch.bfloat16).cuda(), 128, cfg.grid, seed=rank)
     lay.run(synth.tau_schedule(cfg.tau0, cfg.tau1, 20), cfg.lr)  # assignments to freeze
@@ -483,11 +500,7 @@ def run_scale_stage(args, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     loss = lay.last_loss()
     lay.close()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     hbm, tf_burst, tf_sus, peak_kind = peaks()
@@ -495,7 +508,7 @@ def run_scale_stage(args, rank, world, local_rank):
     flops = 4.0 * cfg.N * cfg.T * cfg.K  # forward + weight-gradient GEMMs
     ach = flops / (per / 1e3) / 1e12
     coords = cfg.N * cfg.K
-    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
             "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
@@ -537,7 +550,7 @@ def run_block_pipeline(args, rank, world, local_rank):
     dm = BLOCK_70B
     T, H, Hk, F = dm["nseq"] * dm["S"], dm["nh"] * dm["d"], dm["nkv"] * dm["d"], dm["F"]
     # seeded synthetic block: x ~ N(0, 1) residual stream, weights N(0, 0.02^2)
-    gen = torch.Generator(device="cuda").manual_seed(7007 + 7919 * rank)
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(7007, rank))
     x = torch.randn((T, H), generator=gen, device="cuda")
     shapes = gsq.block_weight_shapes(dm["nh"], dm["nkv"], dm["d"], F)
     W = {n: (torch.randn(shp, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
@@ -562,11 +575,7 @@ def run_block_pipeline(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     hbm, tf_burst, tf_sus, peak_kind = peaks()
@@ -578,7 +587,7 @@ def run_block_pipeline(args, rank, world, local_rank):
     per_stage = {s: {"ms_per_step": m / args.steps,
                      "tflops": round(f * args.steps / (m / 1e3) / 1e12, 1) if m > 0 else None}
                  for s, m, f in zip(gsq.BLOCK_STAGES, stage_ms, flops)}
-    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "steps_per_s": 1e3 * args.steps / ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -614,8 +623,9 @@ def run_gptq_stage(args, rank, world, local_rank):
     from post_weight_quantization_philox_b200 import gsq
     torch.cuda.set_device(local_rank)
     cfg = synth.CONFIGS[args.config]
-    W = torch.from_numpy(synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank))
-    X = torch.from_numpy(synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank))
+    w_seed, x_seed, _ = layer_seeds(cfg, rank)
+    W = torch.from_numpy(synth.make_weight(cfg, seed=w_seed))
+    X = torch.from_numpy(synth.make_calib(cfg, seed=x_seed))
     dt = torch.bfloat16 if cfg.w_bf16 else torch.float32
     W, X = W.to(dt).cuda(), X.to(dt).cuda()
     lev = torch.empty((cfg.N, cfg.K), dtype=torch.int8, device="cuda")
@@ -638,11 +648,7 @@ def run_gptq_stage(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     per = ms / args.steps
@@ -653,7 +659,7 @@ def run_gptq_stage(args, rank, world, local_rank):
     flops = gptq_simt_flops(cfg.N, cfg.K)
     ach = flops / (per / 1e3) / 1e12
     coords = cfg.N * cfg.K
-    return {"metric": METRIC, "value": world * coords / (per / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords, per), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
             "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp32 (Hessian: bf16 operands, fp32 accumulate)",
@@ -684,8 +690,9 @@ def run_kquant_stage(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     cfg = synth.CONFIGS[args.config]
     fmt = gsq.GSQ_KQ_Q2_K if args.kq_format == "q2k" else gsq.GSQ_KQ_Q3_K
-    W = synth.make_weight(cfg, seed=1000 + cfg.number + 7919 * rank)
-    X = synth.make_calib(cfg, seed=2000 + cfg.number + 7919 * rank)
+    w_seed, x_seed, _ = layer_seeds(cfg, rank)
+    W = synth.make_weight(cfg, seed=w_seed)
+    X = synth.make_calib(cfg, seed=x_seed)
     lay = gsq.gsq_kq_init(torch.from_numpy(W).to(torch.bfloat16).cuda(),
                           torch.from_numpy(X).to(torch.bfloat16).cuda(), fmt, seed=rank)
     e_start = lay.recon_error(1)[1]
@@ -711,11 +718,7 @@ def run_kquant_stage(args, rank, world, local_rank):
     loss = lay.last_loss()
     e_end = lay.recon_error(0)[1]
     lay.close()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     if rank != 0:
         return None
     hbm, tf_burst, tf_sus, peak_kind = peaks()
@@ -723,7 +726,7 @@ def run_kquant_stage(args, rank, world, local_rank):
     flops = 4.0 * cfg.N * cfg.T * cfg.K
     ach = flops / (per / 1e3) / 1e12
     coords = cfg.N * cfg.K
-    return {"metric": METRIC, "value": world * coords * args.steps / (ms / 1e3), "unit": UNIT,
+    return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per,
             "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state", "data": "synthetic",
