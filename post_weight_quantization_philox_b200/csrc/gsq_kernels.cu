@@ -317,16 +317,26 @@ __global__ void __launch_bounds__(256) k_soft_weight(
     const int64_t n = gi / G, g = gi - n * G;
     const int64_t base = n * K + g * kGroup + lane;
     const float sg = __ldg(s + gi);
+    // every load of the lane's four coordinates first, then their noise
+    // (which needs none of them) while the loads are in flight
+    float lj[kPerLane][L];
+    int levj[kPerLane];
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) {
       const int64_t c = base + 32 * j;
-      float l[L], gz[L], y[L], cand[5];
 #pragma unroll
-      for (int p = 0; p < L; ++p) l[p] = St<TS>::ld(logits + p * NK + c);
-      const int lev0 = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
-      noise1<MODE>(c, t, k0, k1, noise, gz);
-      candidates<MODE>(lev0, cand);
-      const float w = sg * coord_soft<MODE>(l, gz, inv_tau, cand, y);
+      for (int p = 0; p < L; ++p) lj[j][p] = St<TS>::ld(logits + p * NK + c);
+      levj[j] = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
+    }
+    float gzj[kPerLane][L];
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) noise1<MODE>(base + 32 * j, t, k0, k1, noise, gzj[j]);
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+      const int64_t c = base + 32 * j;
+      float y[L], cand[5];
+      candidates<MODE>(levj[j], cand);
+      const float w = sg * coord_soft<MODE>(lj[j], gzj[j], inv_tau, cand, y);
       What[c] = __float2bfloat16_rn(w);
       if (gbuf) {
 #pragma unroll
