@@ -145,12 +145,17 @@ GSQ_API int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int
                      int8_t* levels, float* scales, void* stream);
 /* Device memory: every buffer the library allocates (contexts of all kinds,
  * init-time staging, the GPTQ workspace) comes from one memory pool per
- * device that the library owns.  Freed memory stays reserved in the pool, up
- * to 8 GiB per device, so that the next context or call of a similar size
- * maps no new pages (mapping costs tens of milliseconds per GB).
- * gsq_release_cached_memory returns what the pools hold in reserve (all
- * devices) to the driver; memory of live contexts stays.  Call it with no
- * library call running.  Errors: GSQ_ERR_CUDA. */
+ * device that the library owns.  Freed memory stays reserved in the pool --
+ * all of it by default -- so that the next context or call of a similar size
+ * maps no new pages (mapping costs tens of milliseconds per GB; a block's MLP
+ * stage holds about 45 GB).
+ * gsq_set_cached_memory_limit: keep at most `bytes` reserved per device
+ * (applies to the pools that exist and to later ones; the excess goes back
+ * at the next synchronisation).  gsq_release_cached_memory: return what the
+ * pools hold in reserve (all devices) to the driver now; memory of live
+ * contexts stays.  Call either with no library call running.
+ * Errors: GSQ_ERR_CUDA. */
+GSQ_API int gsq_set_cached_memory_limit(uint64_t bytes);
 GSQ_API int gsq_release_cached_memory(void);
 /* gsq_init from the GPTQ assignment: the initial levels (init_idx) and the
  * group scales both come from gsq_gptq (instead of round-to-nearest with

@@ -1,11 +1,12 @@
 // gsq_pool.cu -- the library's device memory.  Every buffer of a context
 // (layer, block stage, K-Quant), the init-time staging and the GPTQ
 // workspace come from one memory pool per device that the library owns.  The
-// pool keeps up to kPoolKeep bytes reserved after they are freed, so that the
-// next context or GPTQ call of a similar size maps no new pages: mapping
-// device memory costs tens of milliseconds per GB here, as much as hundreds
-// of reconstruction steps of a layer.  gsq_release_cached_memory hands the
-// reserve back to the driver.
+// pool keeps freed memory reserved (all of it by default, or up to the limit
+// gsq_set_cached_memory_limit sets), so that the next context or call of a
+// similar size maps no new pages: mapping device memory costs tens of
+// milliseconds per GB here, as much as hundreds of reconstruction steps of a
+// layer, and a block's MLP stage alone takes about 45 GB.
+// gsq_release_cached_memory hands the reserve back to the driver.
 //
 // pool_malloc has cudaMalloc's contract (the memory may be used on any stream
 // once it returns): it allocates on a private stream of the device and
@@ -21,10 +22,10 @@ namespace gsq {
 
 namespace {
 
-constexpr uint64_t kPoolKeep = 8ull << 30;
 constexpr int kMaxDevices = 64;
 
 std::mutex g_mu;
+uint64_t g_keep = ~0ull;  // release threshold of every pool
 cudaMemPool_t g_pool[kMaxDevices] = {};
 cudaStream_t g_stream[kMaxDevices] = {};
 
@@ -44,7 +45,7 @@ bool device_pool(int dev, cudaMemPool_t* pool, cudaStream_t* stream) {
       cudaGetLastError();
       return false;
     }
-    uint64_t keep = kPoolKeep;
+    uint64_t keep = g_keep;
     cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
     cudaGetLastError();
     g_pool[dev] = p;
@@ -111,6 +112,23 @@ void pool_free(void* p) {
 }  // namespace gsq
 
 extern "C" {
+
+int gsq_set_cached_memory_limit(uint64_t bytes) {
+  using namespace gsq;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_keep = bytes;
+  int rc = GSQ_OK;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (!g_pool[d]) continue;
+    uint64_t keep = bytes;
+    if (cudaMemPoolSetAttribute(g_pool[d], cudaMemPoolAttrReleaseThreshold, &keep) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      rc = GSQ_ERR_CUDA;
+    }
+  }
+  return rc;
+}
 
 int gsq_release_cached_memory(void) {
   using namespace gsq;

@@ -44,7 +44,7 @@ EXPORTS = [
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
-    "gsq_gptq", "gsq_release_cached_memory", "gsq_init_gptq", "gsq_init_bf16_state",
+    "gsq_gptq", "gsq_release_cached_memory", "gsq_set_cached_memory_limit", "gsq_init_gptq", "gsq_init_bf16_state",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
@@ -97,6 +97,7 @@ _SIGS = {
     "gsq_scale_step": [_p, _f32, _f32, _f32],
     "gsq_gptq": [_p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _p, _p, _p],
     "gsq_release_cached_memory": [],
+    "gsq_set_cached_memory_limit": [_u64],
     "gsq_init_gptq": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _f32, _u64, _p],
     "gsq_init_bf16_state": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64,
                             _p],
@@ -282,6 +283,11 @@ def gsq_gptq(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT, damp: float
            "gsq_gptq")
     del wk, xk
     return levels, scales
+
+
+def gsq_set_cached_memory_limit(nbytes: int) -> None:
+    """Keep at most nbytes of freed device memory reserved per device."""
+    _check(_lib.gsq_set_cached_memory_limit(int(nbytes)), "gsq_set_cached_memory_limit")
 
 
 def gsq_release_cached_memory() -> None:

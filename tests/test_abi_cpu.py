@@ -90,6 +90,8 @@ def test_release_without_pools(gsq):
     """With no device allocation made there is no pool to trim: a no-op that succeeds
     without touching a device."""
     assert gsq.lib().gsq_release_cached_memory() == gsq.GSQ_OK
+    assert gsq.lib().gsq_set_cached_memory_limit(1 << 30) == gsq.GSQ_OK
+    assert gsq.lib().gsq_set_cached_memory_limit(2 ** 64 - 1) == gsq.GSQ_OK
 
 
 def test_binding_has_no_fallback(monkeypatch, tmp_path):

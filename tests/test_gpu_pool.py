@@ -44,6 +44,15 @@ def test_reused_and_released_memory(g, mode):
     g.gsq_release_cached_memory()
     d, rd = trajectory(g, W, X, mode, taus)
     d.close()
-    for other in (rb, rc, rd):
+    # with no reserve kept, every context maps fresh memory
+    g.gsq_set_cached_memory_limit(0)
+    try:
+        e, re_ = trajectory(g, W, X, mode, taus)
+        e.close()
+        f, rf = trajectory(g, W, X, mode, taus)
+        f.close()
+    finally:
+        g.gsq_set_cached_memory_limit(2 ** 64 - 1)
+    for other in (rb, rc, rd, re_, rf):
         for x, y in zip(ra, other):
             assert np.array_equal(np.asarray(x), np.asarray(y))
