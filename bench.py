@@ -15,6 +15,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -128,11 +129,18 @@ def run_gsq(args, rank, world, local_rank):
     from post_weight_quantization_philox_b200 import gsq
 
     torch.cuda.set_device(local_rank)
-    cfg = synth.CONFIGS[args.config]
+    full = synth.CONFIGS[args.config]
+    cfg = full
+    if args.rows:
+        # the first rows of the layer (rows are independent problems): a
+        # smaller case of the same kernels, e.g. for profiling
+        if args.rows % 256 or not 0 < args.rows <= full.N:
+            raise SystemExit(f"--rows must be a multiple of 256 in (0, {full.N}]")
+        cfg = dataclasses.replace(full, N=args.rows, name=f"{full.name}_rows{args.rows}")
     # each rank quantizes its own independent layer of the same shape
-    w_seed, x_seed, _ = layer_seeds(cfg, rank)
-    W = synth.make_weight(cfg, seed=w_seed)
-    X = synth.make_calib(cfg, seed=x_seed)
+    w_seed, x_seed, _ = layer_seeds(full, rank)
+    W = synth.make_weight(full, seed=w_seed, rows=slice(0, cfg.N))
+    X = synth.make_calib(full, seed=x_seed)
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
     stream = torch.cuda.current_stream()
@@ -204,7 +212,7 @@ def run_gsq(args, rank, world, local_rank):
                       "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
     dom = max(phases, key=lambda n: phases[n]["ms"] * phases[n]["launches"])
     d = phases[dom]
-    traffic = load_traffic(dom, args.config + ("_bf16_state" if state16 else ""))
+    traffic = load_traffic(dom, cfg.name + ("_bf16_state" if state16 else ""))
     state_mb = 2 * lay.L * coords * es / 1e6
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -782,6 +790,8 @@ def main():
                     help="logit / momentum storage of the single-layer step")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end job (profiling runs)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="single layer: only its first ROWS rows (a multiple of 256)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
