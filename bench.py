@@ -210,6 +210,12 @@ def run_gsq(args, rank, world, local_rank):
         phases[nm] = {"ms": round(per, 5), "launches": int(phase_n[i]),
                       "bound": bound, "achieved": round(ach, 1), "unit": unit,
                       "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
+        if nm == "soft_weight":
+            # the run's first kernel: later steps get their soft weight from
+            # the fused backward; its events also span the idle GPU's start
+            # after the synchronised beginning of the timed region
+            phases[nm]["note"] = ("once per gsq_run call, the first kernel after the "
+                                  "synchronised start; includes the GPU's ramp from idle")
     dom = max(phases, key=lambda n: phases[n]["ms"] * phases[n]["launches"])
     d = phases[dom]
     traffic = load_traffic(dom, cfg.name + ("_bf16_state" if state16 else ""))
