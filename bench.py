@@ -212,10 +212,11 @@ def run_gsq(args, rank, world, local_rank):
                       "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
         if nm == "soft_weight":
             # the run's first kernel: later steps get their soft weight from
-            # the fused backward; its events also span the idle GPU's start
-            # after the synchronised beginning of the timed region
+            # the fused backward; its events are the first after the
+            # synchronised start of the timed region (0.77 ms here against
+            # 0.22 ms per launch in the ncu launch list of the same workload)
             phases[nm]["note"] = ("once per gsq_run call, the first kernel after the "
-                                  "synchronised start; includes the GPU's ramp from idle")
+                                  "synchronised start of the timed region")
     dom = max(phases, key=lambda n: phases[n]["ms"] * phases[n]["launches"])
     d = phases[dom]
     traffic = load_traffic(dom, cfg.name + ("_bf16_state" if state16 else ""))
