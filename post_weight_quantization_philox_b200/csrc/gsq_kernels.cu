@@ -291,11 +291,10 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w)
   *reinterpret_cast<uint2*>(dst) = pk;
 }
 
-// Both kernels below give one warp a group of 128 coordinates of one row;
-// lane j takes coordinates j, j+32, j+64, j+96, so every load and store of a
-// logit plane is one coalesced 128-byte access and each coordinate is
-// finished before the next one starts (few live registers).
-constexpr int kPerLane = kGroup / 32;
+// The soft weight and the fused backward give one warp a group of 128
+// coordinates of one row; lane j takes the aligned quad 4j .. 4j + 3, so every
+// access to a plane is one 16-byte access per lane (512 contiguous bytes per
+// warp) and the quad shares its 3-bit block-1 Philox draw.
 
 // Soft weight (A1 + A2): w = bf16(s * v((l + g) / tau)).  When gbuf is given
 // the step's probabilities y = softmax((l + g) / tau) are kept there (L
@@ -314,36 +313,51 @@ __global__ void __launch_bounds__(256) k_soft_weight(
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t gi = warp; gi < N * G; gi += nwarps) {
+    // lane j owns the four consecutive coordinates 4j .. 4j + 3 of the
+    // group (an aligned quad): 16-byte loads and stores of every plane
     const int64_t n = gi / G, g = gi - n * G;
-    const int64_t base = n * K + g * kGroup + lane;
+    const int64_t c0 = n * K + g * kGroup + 4 * lane;
     const float sg = __ldg(s + gi);
-    // every load of the lane's four coordinates first, then their noise
-    // (which needs none of them) while the loads are in flight
-    float lj[kPerLane][L];
-    int levj[kPerLane];
+    float lj[4][L];
 #pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-      const int64_t c = base + 32 * j;
-#pragma unroll
-      for (int p = 0; p < L; ++p) lj[j][p] = St<TS>::ld(logits + p * NK + c);
-      levj[j] = MODE == GRID_3BIT_LOCAL ? (int)__ldg(i0 + c) : 0;
+    for (int p = 0; p < L; ++p) {
+      const float4 v = St<TS>::ld4(logits + p * NK + c0);
+      lj[0][p] = v.x;
+      lj[1][p] = v.y;
+      lj[2][p] = v.z;
+      lj[3][p] = v.w;
     }
-    float gzj[kPerLane][L];
+    int levj[4] = {0, 0, 0, 0};
+    if (MODE == GRID_3BIT_LOCAL) {
+      const uint32_t b4 = __ldg(reinterpret_cast<const uint32_t*>(i0 + c0));
 #pragma unroll
-    for (int j = 0; j < kPerLane; ++j) noise1<MODE>(base + 32 * j, t, k0, k1, noise, gzj[j]);
+      for (int j = 0; j < 4; ++j) levj[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
+    }
+    // the quad's noise (it needs none of the loads, which are in flight)
+    float gq[4][5];
+    if (noise) {
+      quad_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c0, t, k0, k1, L == 5, gq);
+    } else {
 #pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-      const int64_t c = base + 32 * j;
-      float y[L], cand[5];
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
+    }
+    float w[4], y[4][L];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float cand[5];
       candidates<MODE>(levj[j], cand);
-      const float w = sg * coord_soft<MODE>(lj[j], gzj[j], inv_tau, cand, y);
-      What[c] = __float2bfloat16_rn(w);
-      if (gbuf) {
-#pragma unroll
-        for (int p = 0; p < L; ++p) gbuf[p * NK + c] = y[p];
-      }
-      if (DBG) wsoft32[c] = w;
+      w[j] = sg * coord_soft<MODE>(lj[j], gq[j], inv_tau, cand, y[j]);
     }
+    store_bf16x4(What + c0, w);
+    if (gbuf) {
+#pragma unroll
+      for (int p = 0; p < L; ++p)
+        *reinterpret_cast<float4*>(gbuf + p * NK + c0) =
+            make_float4(y[0][p], y[1][p], y[2][p], y[3][p]);
+    }
+    if (DBG) *reinterpret_cast<float4*>(wsoft32 + c0) = make_float4(w[0], w[1], w[2], w[3]);
   }
 }
 
