@@ -544,11 +544,11 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs == 0) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair<EPI, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem_bytes<EPI, BN>());
+  {
+    const cudaError_t e = smem_optin<k_gemm_pair<EPI, BN>>(smem_bytes<EPI, BN>());
     if (e != cudaSuccess) return e;
+  }
+  if (max_pairs == 0) {
     cfg.gridDim = dim3((unsigned)(2 * (sm_count / 2)));
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<EPI, BN>, &cfg) != cudaSuccess ||

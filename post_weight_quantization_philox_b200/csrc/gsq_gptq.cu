@@ -378,12 +378,9 @@ namespace {
 template <int MODE>
 cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_t* levels,
                          float* scales, float* E, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gptq_cols<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kColsSmem);
+  {
+    const cudaError_t e = smem_optin<k_gptq_cols<MODE>>(kColsSmem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const unsigned rb = (unsigned)((N + kColRows - 1) / kColRows);
   for (int64_t j0 = 0; j0 < K; j0 += kCols) {

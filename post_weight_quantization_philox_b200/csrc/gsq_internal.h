@@ -1,6 +1,7 @@
 // gsq_internal.h -- launchers shared by the translation units of libgsq.
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,6 +39,21 @@ struct EpiMaps {
   CUtensorMap out;
   CUtensorMap yref;
 };
+
+// Opts kernel Fn in to `bytes` of dynamic shared memory on the current device,
+// once per device (the attribute is per device; a process may drive several).
+template <auto Fn>
+inline cudaError_t smem_optin(int bytes) {
+  static std::atomic<uint64_t> done{0};  // one bit per device ordinal < 64
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(Fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Device memory of the library (gsq_pool.cu): one pool per device that keeps
 // freed memory reserved for the next allocation.  pool_malloc behaves as

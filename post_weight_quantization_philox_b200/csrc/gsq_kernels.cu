@@ -1193,20 +1193,16 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   using C = BwdCfg<MODE, TS>;
   TS* lg = reinterpret_cast<TS*>(a.logits_w);
   TS* mm = reinterpret_cast<TS*>(a.mom);
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaFuncSetAttribute(k_backward_lion<MODE, true, NEXT, TS>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    cudaFuncSetAttribute(k_backward_lion<MODE, false, NEXT, TS>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    attr_set = true;
-  }
+  // a failed opt-in leaves the launch to fail, and the launcher's caller
+  // reads that error from cudaGetLastError
   if (dl_dbg) {
+    smem_optin<k_backward_lion<MODE, true, NEXT, TS>>(C::SMEM);
     k_backward_lion<MODE, true, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
         lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
         dl_dbg, ds_dbg);
   } else {
+    smem_optin<k_backward_lion<MODE, false, NEXT, TS>>(C::SMEM);
     k_backward_lion<MODE, false, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
         lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
         a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,

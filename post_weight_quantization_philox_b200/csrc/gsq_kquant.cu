@@ -749,12 +749,9 @@ cudaError_t kq_launch_soft(gsq_kq* c, float tau, float* wsoft32) {
 template <int F, bool DBG, bool NEXT>
 cudaError_t kq_backward_launch(gsq_kq* c, float it, float lr, float b1, float b2, float itn) {
   using Cf = KqBwdCfg<F>;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        k_kq_backward<F, DBG, NEXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  {
+    const cudaError_t e = smem_optin<k_kq_backward<F, DBG, NEXT>>(Cf::SMEM);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int64_t NK = c->N * c->K, groups = NK / 128;
   const int64_t need = (groups + Cf::WARPS - 1) / Cf::WARPS;
