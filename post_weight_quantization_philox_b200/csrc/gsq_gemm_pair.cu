@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const __grid_constant__ CUtensorMap tmO,
                 const __grid_constant__ CUtensorMap tmY, int64_t M, int64_t N,
                 int64_t Kc, EpiParams ep, const __grid_constant__ GemmSched sc) {
+  pdl_trigger();  // our CTAs are all resident (persistent grid)
   using C = Cfg<BN>;
   constexpr int PN = C::PN, STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
   constexpr int TMEM_COLS = C::TMEM_COLS;
@@ -226,6 +227,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote access
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  // the setup above overlapped the previous kernel's tail; its outputs (our
+  // operands) and its reads of what we write are complete after this
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -533,17 +537,19 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
                             int64_t Kc, const GemmSched& sc, const EpiParams& ep,
                             int sm_count, cudaStream_t st) {
   static int max_pairs = 0;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = smem_bytes<EPI, BN>();
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below takes the cluster shape only
   {
     const cudaError_t e = smem_optin<k_gemm_pair<EPI, BN>>(smem_bytes<EPI, BN>());
     if (e != cudaSuccess) return e;
@@ -562,6 +568,7 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
       ((M + PM - 1) / PM) * ((N + BN - 1) / BN) * (int64_t)sc.count;
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI, BN>, tmA, tmB, maps.out, maps.yref,
                             M, N, Kc, ep, sc);
 }

@@ -412,6 +412,8 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
   constexpr int L = C::L;
   constexpr bool S16 = sizeof(TS) == 2;
   extern __shared__ __align__(16) uint8_t bwd_smem[];
+  pdl_trigger();  // persistent grid: every CTA is resident
+  pdl_wait();     // dW (and the state) of the previous kernels are complete
   const int64_t NK = N * K, G = K / kGroup, groups = N * G;
   const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
   const int64_t warp = (int64_t)blockIdx.x * C::WARPS + wic;
@@ -1195,18 +1197,29 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   TS* mm = reinterpret_cast<TS*>(a.mom);
   // a failed opt-in leaves the launch to fail, and the launcher's caller
   // reads that error from cudaGetLastError
+  // launched with programmatic stream serialisation: the CTAs start as the
+  // weight-gradient GEMM's finish and wait in the kernel for its dW
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(C::WARPS * 32);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (dl_dbg) {
     smem_optin<k_backward_lion<MODE, true, NEXT, TS>>(C::SMEM);
-    k_backward_lion<MODE, true, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
-        a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
-        dl_dbg, ds_dbg);
+    cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, true, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
+                       dW, gbuf, a.N, a.K, k0, k1, (uint32_t)(a.t + 1), a.noise, inv_tau,
+                       inv_tau_next, lr, b1, omb1, b2, omb2, What, dl_dbg, ds_dbg);
   } else {
     smem_optin<k_backward_lion<MODE, false, NEXT, TS>>(C::SMEM);
-    k_backward_lion<MODE, false, NEXT, TS><<<blocks, C::WARPS * 32, C::SMEM, st>>>(
-        lg, mm, a.s, a.ms, a.i0, dW, gbuf, a.N, a.K, k0, k1,
-        a.t + 1, a.noise, inv_tau, inv_tau_next, lr, b1, omb1, b2, omb2, What,
-        nullptr, nullptr);
+    cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, false, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
+                       dW, gbuf, a.N, a.K, k0, k1, (uint32_t)(a.t + 1), a.noise, inv_tau,
+                       inv_tau_next, lr, b1, omb1, b2, omb2, What, (float*)nullptr,
+                       (float*)nullptr);
   }
 }
 
