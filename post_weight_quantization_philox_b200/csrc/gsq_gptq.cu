@@ -90,17 +90,22 @@ __global__ void k_reverse(const float* __restrict__ src, float* __restrict__ dst
     dst[i] = src[KK - 1 - i];
 }
 
-// Lower Cholesky factor of the 64 x 64 diagonal block at (k0, k0), in place
+// Lower Cholesky factor L of the 64 x 64 diagonal block at (k0, k0), in place
 // (lower triangle only), right-looking: column by column every thread takes
 // the pivot's square root, the rows below divide their entry of the column,
 // and the trailing lower triangle takes its rank-1 update, 1024 threads
 // owning 4 entries each (column t % 64 of rows t / 64 + 16 j, so a warp's
-// accesses fall in distinct banks).  A pivot that is not positive is recorded and
-// replaced by 1 so that nothing downstream turns into NaN.
+// accesses fall in distinct banks).  A pivot that is not positive is
+// recorded and replaced by 1 so that nothing downstream turns into NaN.
+// Then X = L^-T into Xinv (64 x 64, row-major): row r of X solves
+// x L^T = e_r by forward substitution, 16 threads per row sharing each
+// column's dot product.  The triangular solves against L become GEMMs with X.
 constexpr int kPotrfThreads = 1024;
 __global__ void __launch_bounds__(kPotrfThreads) k_potrf64(float* __restrict__ A, int64_t K,
-                                                           int64_t k0, int* __restrict__ err) {
+                                                           int64_t k0, int* __restrict__ err,
+                                                           float* __restrict__ Xinv) {
   __shared__ float a[kNb][kNb + 1];
+  __shared__ float xs[kNb][kNb + 1];
   const int t = threadIdx.x;
   for (int e = t; e < kNb * kNb; e += kPotrfThreads) {
     const int rr = e / kNb, c = e % kNb;
@@ -134,54 +139,21 @@ __global__ void __launch_bounds__(kPotrfThreads) k_potrf64(float* __restrict__ A
     const int rr = e / kNb, c = e % kNb;
     if (c <= rr) A[(k0 + rr) * K + k0 + c] = a[rr][c];
   }
-}
-
-// For each of `rows` vectors x (element c at X[r rs + c cs]) solve
-// x L^T = b in place, L the 64 x 64 lower triangle at L (leading dim ldl):
-// x_c = (b_c - sum_{s<c} x_s L_cs) / L_cc.  One thread per vector, the
-// vector in registers: once x_c is known it is taken off every later b_s
-// (the same products in the same order as the dot-product form, but
-// independent of one another, so they pipeline).  The 64 vectors of a CTA
-// move between global and shared memory cooperatively, along whichever of
-// rs, cs is 1, so the transfers coalesce.
-__global__ void __launch_bounds__(64) k_trsm64(float* __restrict__ X, int64_t rows, int64_t rs,
-                                               int64_t cs, const float* __restrict__ L,
-                                               int64_t ldl) {
-  __shared__ float ls[kNb][kNb];
-  __shared__ float xs[kNb][64 + 1];
-  const int tid = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * 64;
-  for (int e = tid; e < kNb * kNb; e += blockDim.x) {
-    const int r = e / kNb, c = e % kNb;
-    ls[r][c] = c <= r ? L[r * ldl + c] : 0.f;
-  }
-  const bool along_c = cs == 1;
-  for (int e = tid; e < kNb * 64; e += blockDim.x) {
-    const int v = along_c ? e / kNb : e % 64, c = along_c ? e % kNb : e / 64;
-    if (r0 + v < rows) xs[c][v] = X[(r0 + v) * rs + c * cs];
+  // X = L^-T: x_c = (delta_rc - sum_{s<c} x_s L_cs) / L_cc, x_c = 0 for c < r
+  const int r = t >> 4, sub = t & 15;
+  for (int c = 0; c < kNb; ++c) {
+    float part = 0.f;
+    for (int q = sub; q < c; q += 16) part = fmaf(xs[r][q], a[c][q], part);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (sub == 0) xs[r][c] = c < r ? 0.f : ((c == r ? 1.f : 0.f) - part) / a[c][c];
+    __syncwarp();
   }
   __syncthreads();
-  if (r0 + tid < rows) {
-    float x[kNb];
-#pragma unroll
-    for (int c = 0; c < kNb; ++c) x[c] = xs[c][tid];
-#pragma unroll
-    for (int c = 0; c < kNb; ++c) {
-      x[c] = x[c] / ls[c][c];
-#pragma unroll
-      for (int s2 = c + 1; s2 < kNb; ++s2) x[s2] = fmaf(-x[c], ls[s2][c], x[s2]);
-    }
-#pragma unroll
-    for (int c = 0; c < kNb; ++c) xs[c][tid] = x[c];
-  }
-  __syncthreads();
-  for (int e = tid; e < kNb * 64; e += blockDim.x) {
-    const int v = along_c ? e / kNb : e % 64, c = along_c ? e % kNb : e / 64;
-    if (r0 + v < rows) X[(r0 + v) * rs + c * cs] = xs[c][v];
-  }
+  for (int e = t; e < kNb * kNb; e += kPotrfThreads) Xinv[e] = xs[e / kNb][e % kNb];
 }
 
-// C[m][n] -= sum_k A(m, k) B(k, n) with A(m, k) = A[m a_rs + k a_cs] and
+// C[m][n] -= sum_k A(m, k) B(k, n) (or =, with assign) with A(m, k) = A[m a_rs + k a_cs] and
 // B(k, n) = B[k b_rs + n b_cs]; C has leading dimension ldc; Kd % 8 == 0.
 // 128 x 128 tiles, 8-deep K slices double-buffered in shared memory (the
 // next slice is fetched into registers while the current one computes),
@@ -199,6 +171,7 @@ struct SubGemm {
   float* C;
   int64_t ldc;
   int lower;
+  int assign = 0;  // C = A B instead of C -= A B
 };
 
 constexpr int kGT = 128, kGK = 8;
@@ -282,7 +255,10 @@ __global__ void __launch_bounds__(256) k_gemm_sub(const SubGemm g) {
     for (int j = 0; j < 8; ++j) {
       const int64_t m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
       const int64_t n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-      if (m < g.M && n < g.N) g.C[m * g.ldc + n] -= acc[i][j];
+      if (m < g.M && n < g.N) {
+        if (g.assign) g.C[m * g.ldc + n] = acc[i][j];
+        else g.C[m * g.ldc + n] -= acc[i][j];
+      }
     }
 }
 
@@ -429,6 +405,7 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   float* B2 = (float*)alloc((size_t)KK * 4);
   int* dead = (int*)alloc((size_t)K * 4);
   float* E = (float*)alloc((size_t)kCols * N * 4);
+  float* Xinv = (float*)alloc((size_t)K * kNb * 4);  // L_kk^-T of every diagonal block
   int* err = (int*)alloc(64);
   double* partials = (double*)alloc(4096 * 8);
   unsigned* ticket = (unsigned*)alloc(16);
@@ -476,11 +453,15 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   k_reverse<<<rgrid, 256, 0, st>>>(B1, B2, K);
   float* A = B2;
   for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
-    k_potrf64<<<1, kPotrfThreads, 0, st>>>(A, K, k0, err);
+    float* Xk = Xinv + (k0 / kNb) * kNb * kNb;  // L_kk^-T
+    k_potrf64<<<1, kPotrfThreads, 0, st>>>(A, K, k0, err, Xk);
     const int64_t rest = K - k0 - kNb;
     if (rest > 0) {
       float* P = A + (k0 + kNb) * K + k0;
-      k_trsm64<<<(unsigned)((rest + 63) / 64), 64, 0, st>>>(P, rest, K, 1, A + k0 * K + k0, K);
+      // the panel below: P = P L_kk^-T, in place (each CTA's rows are its own)
+      SubGemm gs{rest, kNb, kNb, P, K, 1, Xk, kNb, 1, P, K, 0};
+      gs.assign = 1;
+      k_gemm_sub<<<dim3(1, (unsigned)((rest + kGT - 1) / kGT)), 256, 0, st>>>(gs);
       const SubGemm g{rest, rest, kNb, P, K, 1, P, 1, K, P + kNb, K, 1};
       const unsigned t = (unsigned)((rest + kGT - 1) / kGT);
       k_gemm_sub<<<dim3(t, t), 256, 0, st>>>(g);
@@ -497,7 +478,14 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   k_unit_diag<<<grid_cap(K, 256, 1024), 256, 0, st>>>(M, K);
   for (int64_t k0 = 0; k0 < K && e == cudaSuccess; k0 += kNb) {
     const int64_t c1 = k0 + kNb, rest = K - c1;
-    k_trsm64<<<(unsigned)((c1 + 63) / 64), 64, 0, st>>>(M + k0 * K, c1, 1, K, A + k0 * K + k0, K);
+    // the row block: M[k0:c1, :c1] = L_kk^-1 M[k0:c1, :c1], in place (each
+    // CTA's columns are its own); L_kk^-1 (m, k) = Xinv_k (k, m)
+    {
+      SubGemm gs{kNb, c1, kNb, Xinv + (k0 / kNb) * kNb * kNb, 1, kNb, M + k0 * K, K, 1,
+                 M + k0 * K, K, 0};
+      gs.assign = 1;
+      k_gemm_sub<<<dim3((unsigned)((c1 + kGT - 1) / kGT), 1), 256, 0, st>>>(gs);
+    }
     if (rest > 0) {
       // M[c1:, :c1] -= L[c1:, k0:c1] M[k0:c1, :c1]
       const SubGemm g{rest, c1, kNb, A + c1 * K + k0, K, 1, M + k0 * K, K, 1, M + c1 * K, K, 0};
