@@ -536,7 +536,9 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
                             const EpiMaps& maps, int64_t M, int64_t N,
                             int64_t Kc, const GemmSched& sc, const EpiParams& ep,
                             int sm_count, cudaStream_t st) {
-  static int max_pairs = 0;
+  // co-resident CTA pairs of this kernel (the same on every B200; computed once)
+  static std::atomic<int> max_pairs_cache{0};
+  int max_pairs = max_pairs_cache.load(std::memory_order_relaxed);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -563,6 +565,7 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
       n = sm_count / 2;
     }
     max_pairs = n;
+    max_pairs_cache.store(n, std::memory_order_relaxed);
   }
   const int64_t tiles =
       ((M + PM - 1) / PM) * ((N + BN - 1) / BN) * (int64_t)sc.count;
