@@ -101,10 +101,11 @@ def phase_bytes_flops(cfg, layer, es=4):
     the bytes of one logit / momentum element (4, or 2 in the bf16 state).
 
     soft weight:        read L logit planes + scale (+ initial level),
-                        write bf16 weight and the L fp32 noise planes;
-    backward + Lion:    read dW, logits, momenta, noise (+ initial level),
-                        write logits and momenta, 16 B per group of scales;
-    ... + next soft:    also write the next bf16 weight and noise planes."""
+                        write bf16 weight and the L fp32 probability planes;
+    backward + Lion:    read dW, logits, momenta, probabilities (+ initial
+                        level), write logits and momenta, 16 B per group of
+                        scales;
+    ... + next soft:    also write the next bf16 weight and probability planes."""
     NK = cfg.N * cfg.K
     L = layer.L
     extra = 1 if cfg.grid == synth.GRID_3BIT_LOCAL else 0  # initial level (int8)

@@ -1,0 +1,54 @@
+"""The bench's roofline arithmetic on CPU: the algorithmic bytes and flops per
+launch behind every achieved figure, and the whole-step roofline."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from post_weight_quantization_philox_b200 import synth  # noqa: E402
+
+
+class _Layer:
+    def __init__(self, L):
+        self.L = L
+
+
+@pytest.mark.parametrize("name,L,per_coord", [
+    # 4 dW + 2 W_hat + logits and momenta read and written (16 L) + probabilities
+    # read and written (8 L), + 1 initial level for the 3-bit grid
+    ("c2_qproj_4096x4096", 4, 102), ("c4_gateproj_14336x4096", 4, 102),
+    ("c3_downproj_4096x14336", 5, 127)])
+def test_fused_backward_bytes_per_coordinate(name, L, per_coord):
+    cfg = synth.CONFIGS[name]
+    w = bench.phase_bytes_flops(cfg, _Layer(L), 4)
+    groups = cfg.N * cfg.K // 128
+    assert w["backward_lion_next_soft"] == ("hbm", cfg.N * cfg.K * per_coord + 16 * groups)
+    # without the next soft weight: no probabilities written, no W_hat
+    assert w["backward_lion"][1] == cfg.N * cfg.K * (per_coord - 2 - 4 * L) + 16 * groups
+    assert w["forward_gemm"] == ("tensor", 2.0 * cfg.N * cfg.T * cfg.K)
+    assert w["weight_grad_gemm"] == w["forward_gemm"]
+
+
+def test_bf16_state_halves_the_state_bytes():
+    cfg = synth.CONFIGS["c2_qproj_4096x4096"]
+    w32 = bench.phase_bytes_flops(cfg, _Layer(4), 4)["backward_lion_next_soft"][1]
+    w16 = bench.phase_bytes_flops(cfg, _Layer(4), 2)["backward_lion_next_soft"][1]
+    # logits and momenta, read and written: 4 planes x 4 logits x 2 bytes saved
+    assert w32 - w16 == cfg.N * cfg.K * 32
+
+
+def test_step_roofline_q_proj():
+    cfg = synth.CONFIGS["c2_qproj_4096x4096"]
+    w = bench.phase_bytes_flops(cfg, _Layer(4), 4)
+    r = bench.step_roofline(w, 0.5, 1374.8, 6457.4)
+    gemm_ms = 2 * 2 * 4096 ** 3 / 1374.8e12 * 1e3
+    hbm_ms = w["backward_lion_next_soft"][1] / 6457.4e9 * 1e3
+    assert r["gemm_ms"] == pytest.approx(gemm_ms, abs=1e-4)
+    assert r["hbm_ms"] == pytest.approx(hbm_ms, abs=1e-4)
+    assert r["frac"] == pytest.approx((gemm_ms + hbm_ms) / 0.5, abs=1e-4)
+    # the whole-job rate counts every rank's units over the slowest rank's time
+    assert bench.whole_job_rate(4, 10.0, 2.0) == pytest.approx(4 * 10.0 / 2e-3)
