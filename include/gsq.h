@@ -522,7 +522,10 @@ GSQ_API int gsq_block_quantize(const float* x_in, const void* const* W, int64_t 
  *   weight (Q3_K), projected as above, each weight's code its nearest level
  *   (first on ties).  Syncs.
  * gsq_kq_step / gsq_kq_run / gsq_kq_last_loss: as gsq_step / gsq_run /
- *   gsq_last_loss (gsq_kq_run is a loop of steps).
+ *   gsq_last_loss.  gsq_kq_run gives the same result as a loop of
+ *   gsq_kq_step bit for bit; inside it each step's backward also forms the
+ *   next step's soft weight (at the next temperature), so a step is three
+ *   launches instead of four.
  * gsq_kq_export: the projected blocks (host or device).  Syncs.
  * gsq_kq_start_blocks: the starting blocks.  Syncs.
  * gsq_kq_recon_error: abs = ||bf16(X) Wq^T - Y_ref||^2 and rel = abs /
