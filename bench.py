@@ -203,6 +203,12 @@ def run_gsq(args, rank, world, local_rank):
 
     # ---- end to end: host buffers through the C ABI, whole quantization job
     e2e = None if args.no_e2e else run_e2e(gsq, torch, cfg, W, X, rank)
+    if e2e is not None and world > 1:
+        # every rank ran its own job; the whole job ends with the slowest
+        sec = max_over_ranks(e2e["seconds"] * 1e3, world) / 1e3
+        e2e["seconds"] = sec
+        e2e["value"] = whole_job_rate(world, cfg.N * cfg.K * cfg.steps, sec * 1e3)
+        e2e["ranks"] = world
 
     if rank != 0:
         return None
