@@ -97,38 +97,42 @@ class ClockSampler:
 
 
 def phase_bytes_flops(cfg, layer, es=4):
-    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch; es is
-    the bytes of one logit / momentum element (4, or 2 in the bf16 state).
+    """Algorithmic bytes (HBM phases) and flops (GEMMs) of one launch: what
+    the method itself must move per coordinate, es being the bytes of one
+    logit / momentum element (4, or 2 in the bf16 state).
 
-    soft weight:        read L logit planes + scale (+ initial level),
-                        write bf16 weight and the L fp32 probability planes;
-    backward + Lion:    read dW, logits, momenta, probabilities (+ initial
-                        level), write logits and momenta, 16 B per group of
-                        scales;
-    ... + next soft:    also write the next bf16 weight and probability planes."""
+    soft weight:        read the L logit planes (+ the int8 initial level of
+                        the 3-bit grid), write the bf16 weight; 4 B per group
+                        of scales;
+    backward + Lion:    read dW, read and write the L logit and L momentum
+                        planes (+ initial level); 16 B per group (scale and
+                        its momentum, read and written);
+    ... + next soft:    also write the next step's bf16 weight.
+    The kernels keep nothing else between launches: the backward draws the
+    step's noise again from its counters."""
     NK = cfg.N * cfg.K
     L = layer.L
     extra = 1 if cfg.grid == synth.GRID_3BIT_LOCAL else 0  # initial level (int8)
     groups = cfg.N * (cfg.K // 128)
-    soft = NK * (es * L + 4 * L + 2 + extra) + groups * 4
-    back = NK * (4 + 4 * es * L + 4 * L + extra) + groups * 16
-    back_next = NK * (6 + 4 * es * L + 8 * L + extra) + groups * 16
+    soft = NK * (es * L + 2 + extra) + groups * 4
+    back = NK * (4 + 4 * es * L + extra) + groups * 16
+    back_next = back + NK * 2
     gemm = 2.0 * cfg.N * cfg.T * cfg.K
     return {"soft_weight": ("hbm", soft), "forward_gemm": ("tensor", gemm),
             "weight_grad_gemm": ("tensor", gemm), "backward_lion": ("hbm", back),
             "backward_lion_next_soft": ("hbm", back_next)}
 
 
-def step_roofline(work, ms_step, tf_sus, hbm):
+def step_roofline(work, ms_step, tf, hbm):
     """A steady step (both GEMMs and the fused backward with the next soft
-    weight) at the peaks: the GEMM flops at the sustained bf16 rate plus the
+    weight) at the peaks: the GEMM flops at the bf16 rate tf plus the
     backward's algorithmic bytes at the copy rate, against the measured step."""
-    gemm_ms = (work["forward_gemm"][1] + work["weight_grad_gemm"][1]) / (tf_sus * 1e12) * 1e3
+    gemm_ms = (work["forward_gemm"][1] + work["weight_grad_gemm"][1]) / (tf * 1e12) * 1e3
     hbm_ms = work["backward_lion_next_soft"][1] / (hbm * 1e9) * 1e3
     return {"gemm_ms": round(gemm_ms, 4), "hbm_ms": round(hbm_ms, 4),
             "ms": round(gemm_ms + hbm_ms, 4), "frac": round((gemm_ms + hbm_ms) / ms_step, 4),
-            "how": "GEMM flops at the sustained bf16 rate + the fused backward's bytes at "
-                   "the copy rate, over the measured step"}
+            "how": "GEMM flops at the burst bf16 rate + the fused backward's algorithmic "
+                   "bytes at the copy rate, over the measured step"}
 
 
 def run_gsq(args, rank, world, local_rank):
@@ -230,11 +234,14 @@ def run_gsq(args, rank, world, local_rank):
             ach = amount / (per / 1e3) / 1e9
             peak, unit = hbm, "GB/s"
         else:
+            # each GEMM launch is a ~0.1 ms burst: the burst bf16 rate
             ach = amount / (per / 1e3) / 1e12
-            peak, unit = tf_sus, "TFLOP/s"
+            peak, unit = tf_burst, "TFLOP/s"
         phases[nm] = {"ms": round(per, 5), "launches": int(phase_n[i]),
                       "bound": bound, "achieved": round(ach, 1), "unit": unit,
                       "peak": peak, "frac": round(ach / peak, 4), "per_launch": amount}
+        if bound == "tensor":
+            phases[nm]["frac_of_sustained"] = round(ach / tf_sus, 4)
         if nm == "soft_weight":
             # the run's first kernel: later steps get their soft weight from
             # the fused backward; its events are the first after the
@@ -261,10 +268,10 @@ def run_gsq(args, rank, world, local_rank):
                    "l2": f"state (logits + Lion momenta, {state_mb:.0f} MB) larger than L2; no flush"},
         "roofline": {"bound": d["bound"], "kernel": dom, "achieved": d["achieved"],
                      "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
-                     "peak_kind": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})",
+                     "peak_kind": f"{peak_kind} ({'burst bf16' if d['bound'] == 'tensor' else 'HBM copy'})",
                      "traffic": traffic},
         "phases": phases,
-        "step_roofline": step_roofline(work, ms / args.steps, tf_sus, hbm),
+        "step_roofline": step_roofline(work, ms / args.steps, tf_burst, hbm),
         "gpu_launches": int(sum(phase_n)),
         "clocks": clk,
         "last_loss": loss,

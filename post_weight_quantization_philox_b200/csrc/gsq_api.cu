@@ -51,10 +51,9 @@ struct gsq_ctx {
   double *partials = nullptr, *loss_hist = nullptr, *scratch = nullptr;
   unsigned* ticket = nullptr;
   int* err = nullptr;
-  float* gbuf = nullptr;  // probabilities of the pending step (L x N x K)
   float *wsoft32 = nullptr, *dl = nullptr, *ds = nullptr;  // debug, lazy
-  // What and gbuf hold the soft weight and probabilities of step what_t at
-  // temperature what_tau (what_t < 0: nothing precomputed)
+  // What holds the soft weight of step what_t at temperature what_tau
+  // (what_t < 0: nothing precomputed)
   int64_t what_t = -1;
   float what_tau = 0.f;
   // level codes of the hard choice of the current logits (scale-only steps)
@@ -312,7 +311,6 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   // bf16 state: half as many 4-byte words
   AL(c->logits, state16 ? (c->L * NK + 1) / 2 : c->L * NK);
   AL(c->mom, state16 ? (c->L * NK + 1) / 2 : c->L * NK);
-  AL(c->gbuf, c->L * NK);
   AL(c->s, N * c->G);
   AL(c->ms, N * c->G);
   AL(c->i0, NK);
@@ -454,8 +452,7 @@ int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const void* X
 namespace {
 
 // One step t at temperature tau; with tau_next > 0 the backward also builds
-// the soft weight and probabilities of step t + 1 (which the next call then
-// skips).
+// the soft weight of step t + 1 (which the next call then skips).
 int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
              float beta2) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;  // 32-bit counter word
@@ -471,7 +468,7 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
     CK(cudaEventRecord(tm->ev[0], c->st));
   }
   const bool soft = !(c->what_t == (int64_t)c->t && c->what_tau == tau);
-  if (soft) CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));
+  if (soft) CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
   if (tm) {
     tm->soft = soft;
     tm->next = tau_next > 0.f;
@@ -481,7 +478,7 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
   if (tm) CK(cudaEventRecord(tm->ev[2], c->st));
   CK(run_weight_grad(c));
   if (tm) CK(cudaEventRecord(tm->ev[3], c->st));
-  CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, tau_next,
+  CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, tau_next,
                           c->What, nullptr, nullptr, c->sms, c->st));
   if (tm) CK(cudaEventRecord(tm->ev[4], c->st));
   c->t += 1;
@@ -642,7 +639,7 @@ int gsq_recon_error(gsq_ctx* c, int mode, float tau, double* abs_err,
   } else {
     StepArgs a = step_args(c, tau);
     a.noise = 0;
-    CK(launch_soft_weight(a, c->What, nullptr, nullptr, c->sms, c->st));
+    CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
   }
   CK(run_forward(c, c->scratch, EPI_LOSS));
   int rc = check_device(c);
@@ -851,8 +848,7 @@ int gsq_debug_soft_weight(gsq_ctx* c, float tau) {
   size_t nb;
   int rc = debug_buffer(c, GSQ_DBG_WSOFT32, &p, &nb);
   if (rc) return rc;
-  CK(launch_soft_weight(step_args(c, tau), c->What, c->gbuf, c->wsoft32, c->sms,
-                        c->st));
+  CK(launch_soft_weight(step_args(c, tau), c->What, c->wsoft32, c->sms, c->st));
   c->what_t = (int64_t)c->t;
   c->what_tau = tau;
   return check_device(c);
@@ -886,11 +882,9 @@ int gsq_debug_backward(gsq_ctx* c, float tau, float lr, float beta1,
   int rc = debug_buffer(c, GSQ_DBG_DL, &p, &nb);
   if (!rc) rc = debug_buffer(c, GSQ_DBG_DS, &p, &nb);
   if (rc) return rc;
-  // the step's soft weight first (the backward takes its probabilities)
+  // the backward draws the step's probabilities itself
   const StepArgs a = step_args(c, tau);
-  if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
-    CK(launch_soft_weight(a, c->What, c->gbuf, nullptr, c->sms, c->st));
-  CK(launch_backward_lion(a, c->dW, c->gbuf, lr, beta1, beta2, 0.f, c->What,
+  CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, 0.f, c->What,
                           c->dl, c->ds, c->sms, c->st));
   c->what_t = -1;
   c->hcode_valid = false;

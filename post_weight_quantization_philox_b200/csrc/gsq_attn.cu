@@ -149,7 +149,7 @@ int run_step(gsq_attn* c, float tau, float tau_next, float lr, float b1, float b
   if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
     for (int i = 0; i < 2; ++i)
       CKA(launch_soft_weight(stage_weight_args(c->w[i], c->mode, c->t, c->noise, tau),
-                             c->w[i].What, c->w[i].gbuf, nullptr, c->sms, c->st));
+                             c->w[i].What, nullptr, c->sms, c->st));
   CKA(forward(c, c->loss_hist + (c->t % kStageLossRing), true));
   EpiParams ep = epi(c, nullptr);
   // dWo = dp^T . o
@@ -169,7 +169,7 @@ int run_step(gsq_attn* c, float tau, float tau_next, float lr, float b1, float b
                   c->sms, c->st));
   for (int i = 0; i < 2; ++i)
     CKA(launch_backward_lion(stage_weight_args(c->w[i], c->mode, c->t, c->noise, tau),
-                             c->w[i].dW, c->w[i].gbuf, lr, b1, b2, tau_next,
+                             c->w[i].dW, lr, b1, b2, tau_next,
                              c->w[i].What, nullptr, nullptr, c->sms, c->st));
   c->t += 1;
   if (tau_next > 0.f) {
@@ -256,7 +256,6 @@ int gsq_attn_init(gsq_attn** out, const void* Xa, int x_dtype, const void* R,
     const int64_t NK = w.N * w.K;
     ALA(w.logits, c->L * NK);
     ALA(w.mom, c->L * NK);
-    ALA(w.gbuf, c->L * NK);
     ALA(w.s, w.N * w.G);
     ALA(w.ms, w.N * w.G);
     ALA(w.i0, NK);
@@ -528,7 +527,7 @@ int gsq_attn_recon_error(gsq_attn* c, int mode, float tau, double* abs_err,
       CKA(launch_hard_weight(c->mode, w.N, w.K, w.logits, w.s, w.i0, w.What, c->st));
     } else {
       StepArgs a = stage_weight_args(w, c->mode, c->t, 0, tau);
-      CKA(launch_soft_weight(a, w.What, nullptr, nullptr, c->sms, c->st));
+      CKA(launch_soft_weight(a, w.What, nullptr, c->sms, c->st));
     }
   }
   CKA(forward(c, c->scratch, false));

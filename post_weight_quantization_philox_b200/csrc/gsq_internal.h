@@ -170,17 +170,15 @@ cudaError_t launch_convert_w(const void* W, int dtype, int64_t N, int64_t K,
 cudaError_t launch_init_state(int mode, const float* W32, const int8_t* init_idx,
                               int64_t N, int64_t K, float* s, int8_t* i0,
                               float* logits, int* err, cudaStream_t st, int state16 = 0);
-// Soft weight of step a.t; keeps the step's probabilities (softmax of the
-// noisy, tempered logits; L planes of N x K fp32) in gbuf when not null.
-cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
-                               float* gbuf, float* wsoft32, int sm_count,
-                               cudaStream_t st);
-// Backward + Lion of step a.t from dW and the probabilities in gbuf; with
-// tau_next > 0 also the soft weight (into What) and probabilities (into
-// gbuf) of step a.t + 1.
-cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
-                                 float* gbuf, float lr, float b1, float b2,
-                                 float tau_next, __nv_bfloat16* What,
+// Soft weight of step a.t into What (and its fp32 values before rounding
+// into wsoft32 when not null).
+cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What, float* wsoft32,
+                               int sm_count, cudaStream_t st);
+// Backward + Lion of step a.t from dW (the step's probabilities are drawn
+// again from the pre-update logits and the step's counters); with
+// tau_next > 0 also the soft weight of step a.t + 1 into What.
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr, float b1,
+                                 float b2, float tau_next, __nv_bfloat16* What,
                                  float* dl_dbg, float* ds_dbg, int sm_count,
                                  cudaStream_t st);
 cudaError_t launch_hard_weight(int mode, int64_t N, int64_t K,

@@ -198,61 +198,6 @@ __global__ void k_init_state(const float* __restrict__ W32,
 
 // ----------------------------------------------------- soft weight (A1+A2)
 
-// Per coordinate: probabilities y and unit value v from logits l, noise g
-// and 1/tau.  Categorical modes use candidate values cand[]; ternary forms
-// v = p1 (q+ - q-).
-template <int MODE>
-__device__ __forceinline__ float coord_soft(const float* l, const float* g,
-                                            float inv_tau, const float* cand,
-                                            float* y) {
-  constexpr int L = GridT<MODE>::L;
-  float z[L];
-#pragma unroll
-  for (int k = 0; k < L; ++k) z[k] = (l[k] + g[k]) * inv_tau;
-  if (MODE == GRID_TERNARY) {
-    const float m0 = fmaxf(z[0], z[1]);
-    const float e0 = __expf(z[0] - m0), e1 = __expf(z[1] - m0);
-    const float r0 = 1.f / (e0 + e1);
-    y[0] = e0 * r0;
-    y[1] = e1 * r0;
-    const float m1 = fmaxf(z[2], z[3]);
-    const float e2 = __expf(z[2] - m1), e3 = __expf(z[3] - m1);
-    const float r1 = 1.f / (e2 + e3);
-    y[2] = e2 * r1;
-    y[3] = e3 * r1;
-    return y[1] * (y[3] - y[2]);
-  } else {
-    float zm = z[0];
-#pragma unroll
-    for (int k = 1; k < L; ++k) zm = fmaxf(zm, z[k]);
-    float sum = 0.f;
-#pragma unroll
-    for (int k = 0; k < L; ++k) {
-      y[k] = __expf(z[k] - zm);
-      sum += y[k];
-    }
-    const float r = 1.f / sum;
-    float v = 0.f;
-#pragma unroll
-    for (int k = 0; k < L; ++k) {
-      y[k] *= r;
-      v = fmaf(y[k], cand[k], v);
-    }
-    return v;
-  }
-}
-
-// The unit value v from probabilities y, with the same operations in the same
-// order as coord_soft, so it equals the v coord_soft returned for them.
-template <int MODE>
-__device__ __forceinline__ float value_of(const float* y, const float* cand) {
-  if (MODE == GRID_TERNARY) return y[1] * (y[3] - y[2]);
-  float v = 0.f;
-#pragma unroll
-  for (int k = 0; k < GridT<MODE>::L; ++k) v = fmaf(y[k], cand[k], v);
-  return v;
-}
-
 template <int MODE>
 __device__ __forceinline__ void candidates(int lev0, float* cand) {
   if (MODE == GRID_2BIT) {
@@ -267,19 +212,55 @@ __device__ __forceinline__ void candidates(int lev0, float* cand) {
   }
 }
 
-// Gumbel noise of one coordinate at step t (zeros when noise is off).
-template <int MODE, int L = GridT<MODE>::L>
-__device__ __forceinline__ void noise1(int64_t c, uint32_t t, uint32_t k0,
-                                       uint32_t k1, int noise, float (&g)[L]) {
-  float gg[5];
-  if (noise) {
-    coord_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c, t, k0, k1, L == 5, gg);
+// Tempered Gumbel-softmax of one coordinate at a step, from its logits l and
+// its Philox words w, and its unit value v.  Categorical modes: e holds the
+// unnormalised e_k, r[0] = 1 / sum e, and v = r[0] sum_k e_k c_k over the
+// candidate values cand[].  Ternary (one softmax over the mask pair, one over
+// the sign pair): e holds the normalised probabilities p0, p1, q-, q+ and
+// v = p1 (q+ - q-).
+template <int MODE>
+__device__ __forceinline__ float coord_value(const float* l, const uint32_t* w, bool noise,
+                                             float inv_tau, const float* cand, float* e,
+                                             float* r) {
+  if (MODE == GRID_TERNARY) {
+    const float rm = gsoftmax2<2>(l, w, noise, inv_tau, e);
+    const float rs = gsoftmax2<2>(l + 2, w + 2, noise, inv_tau, e + 2);
+    e[0] *= rm;
+    e[1] *= rm;
+    e[2] *= rs;
+    e[3] *= rs;
+    r[0] = 1.f;
+    return e[1] * (e[3] - e[2]);
   } else {
+    r[0] = gsoftmax2<GridT<MODE>::L>(l, w, noise, inv_tau, e);
+    float v = 0.f;
 #pragma unroll
-    for (int p = 0; p < 5; ++p) gg[p] = 0.f;
+    for (int k = 0; k < GridT<MODE>::L; ++k) v = fmaf(e[k], cand[k], v);
+    return v * r[0];
   }
-#pragma unroll
-  for (int p = 0; p < L; ++p) g[p] = gg[p];
+}
+
+// Block-0 words of coordinate c at step t (words 0..3 of its noise).  The
+// callers pass the high word of the aligned quad's first coordinate: the four
+// coordinates of a quad share it (a quad never straddles a multiple of
+// 2^32), so the rounds that depend only on it and on t are formed once.
+__device__ __forceinline__ void block0_words(uint64_t c, uint32_t c_hi, uint32_t t,
+                                             const PhiloxKeys& ks, uint32_t* w) {
+  const uint4 r = philox4x32_10(make_uint4((uint32_t)c, c_hi, t, 0u), ks);
+  w[0] = r.x;
+  w[1] = r.y;
+  w[2] = r.z;
+  w[3] = r.w;
+}
+// Block-1 draw of the aligned quad starting at c0 (the 3-bit grid's fifth
+// word: coordinate c0 + j takes word j).
+__device__ __forceinline__ void block1_words(uint64_t c0, uint32_t t, const PhiloxKeys& ks,
+                                             uint32_t* w) {
+  const uint4 r = philox4x32_10(make_uint4((uint32_t)c0, (uint32_t)(c0 >> 32), t, 1u), ks);
+  w[0] = r.x;
+  w[1] = r.y;
+  w[2] = r.z;
+  w[3] = r.w;
 }
 
 __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w) {
@@ -296,16 +277,14 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* dst, const float* w)
 // access to a plane is one 16-byte access per lane (512 contiguous bytes per
 // warp) and the quad shares its 3-bit block-1 Philox draw.
 
-// Soft weight (A1 + A2): w = bf16(s * v((l + g) / tau)).  When gbuf is given
-// the step's probabilities y = softmax((l + g) / tau) are kept there (L
-// planes) for the backward, which then needs neither the noise nor a second
-// softmax.
+// Soft weight (A1 + A2): w = bf16(s * v), v the unit value of the tempered
+// Gumbel-softmax of the logits.  Nothing else is kept: the backward draws the
+// same noise again from the same counters.
 template <int MODE, bool DBG, typename TS>
 __global__ void __launch_bounds__(256) k_soft_weight(
     const TS* __restrict__ logits, const float* __restrict__ s,
-    const int8_t* __restrict__ i0, int64_t N, int64_t K, uint32_t k0,
-    uint32_t k1, uint32_t t, int noise, float inv_tau,
-    __nv_bfloat16* __restrict__ What, float* __restrict__ gbuf,
+    const int8_t* __restrict__ i0, int64_t N, int64_t K, const PhiloxKeys ks,
+    uint32_t t, int noise, float inv_tau, __nv_bfloat16* __restrict__ What,
     float* __restrict__ wsoft32) {
   constexpr int L = GridT<MODE>::L;
   const int64_t NK = N * K, G = K / kGroup;
@@ -313,10 +292,8 @@ __global__ void __launch_bounds__(256) k_soft_weight(
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t gi = warp; gi < N * G; gi += nwarps) {
-    // lane j owns the four consecutive coordinates 4j .. 4j + 3 of the
-    // group (an aligned quad): 16-byte loads and stores of every plane
-    const int64_t n = gi / G, g = gi - n * G;
-    const int64_t c0 = n * K + g * kGroup + 4 * lane;
+    // K = G * 128: group gi starts at coordinate 128 gi
+    const int64_t c0 = gi * kGroup + 4 * lane;
     const float sg = __ldg(s + gi);
     float lj[4][L];
 #pragma unroll
@@ -333,64 +310,51 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 #pragma unroll
       for (int j = 0; j < 4; ++j) levj[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
-    // the quad's noise (it needs none of the loads, which are in flight)
-    float gq[4][5];
-    if (noise) {
-      quad_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c0, t, k0, k1, L == 5, gq);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
-    }
-    float w[4], y[4][L];
+    uint32_t q1[4] = {0u, 0u, 0u, 0u};
+    if (L == 5 && noise) block1_words((uint64_t)c0, t, ks, q1);
+    float w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float cand[5];
+      uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
+      if (noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t, ks, wd);
+      wd[4] = q1[j];
+      float cand[5], e[L], r;
       candidates<MODE>(levj[j], cand);
-      w[j] = sg * coord_soft<MODE>(lj[j], gq[j], inv_tau, cand, y[j]);
+      w[j] = sg * coord_value<MODE>(lj[j], wd, noise, inv_tau, cand, e, &r);
     }
     store_bf16x4(What + c0, w);
-    if (gbuf) {
-#pragma unroll
-      for (int p = 0; p < L; ++p)
-        *reinterpret_cast<float4*>(gbuf + p * NK + c0) =
-            make_float4(y[0][p], y[1][p], y[2][p], y[3][p]);
-    }
     if (DBG) *reinterpret_cast<float4*>(wsoft32 + c0) = make_float4(w[0], w[1], w[2], w[3]);
   }
 }
 
 // ------------------------------------------------- backward + Lion (A5)
 
-// Takes the step's probabilities y from gbuf (written by the soft weight of
-// the same step, from the pre-update logits and the step's noise) and forms
-//   a = s dW / tau,  dl_k = a y_k sum_j y_j (c_k - c_j)   (categorical),
-//   dl_mask1 = a (q+ - q-) p1 p0 = -dl_mask0, dl_sign+ = 2 a p1 q+ q- =
-//   -dl_sign- (ternary),  ds = sum over the group of dW v (warp shuffle),
-// then applies Lion to the logits and the group scale.  With NEXT it also
-// computes the soft weight of step t+1 from the updated logits and scale
-// (fresh Philox noise; its probabilities go to gbuf for the next backward):
-// the same values a separate soft-weight launch would produce.  All loads of the group are
-// issued first and the next step's noise (which needs none of them) is
-// computed while they are in flight.
 // Backward + Lion (A5), optionally fused with the next step's A1 + A2.  One
 // warp per 128-group; lane j owns the four consecutive coordinates 4j..4j+3.
 // The warp's next group is staged into shared memory with per-lane 16-byte
 // async copies (each lane copies exactly the pieces it will read) while the
 // current group is computed, so the loads of one group overlap the
-// arithmetic of the previous one.  Every global access is 16 bytes wide.
+// arithmetic of the previous one.  Every global access is 16 bytes wide
+// (8 bytes for bf16 state planes).
+//
+// Per coordinate, from the pre-update logits and the step's Philox words
+// (the counters of the step's soft weight, so the same probabilities):
+//   a = s dW / tau,  dl_k = a y_k sum_j y_j (c_k - c_j)   (categorical),
+//   dl_mask1 = a (q+ - q-) p1 p0 = -dl_mask0, dl_sign+ = 2 a p1 q+ q- =
+//   -dl_sign- (ternary),  ds = sum over the group of dW v (warp shuffle),
+// then Lion on the logits and the group scale.  With NEXT it also forms the
+// soft weight of step t + 1 from the updated logits and scale with the words
+// of step t + 1: the values a separate soft-weight launch would produce.
 template <int MODE, typename TS = float>
 struct BwdCfg {
   static constexpr int L = GridT<MODE>::L;
-  // per-warp staging of one group: dW, logits, momenta, probabilities (, i0); the
-  // logit and momentum planes take 128 sizeof(TS) bytes each
+  // per-warp staging of one group: dW, logits, momenta (, i0); the logit and
+  // momentum planes take 128 sizeof(TS) bytes each
   static constexpr int SP = 128 * (int)sizeof(TS);
-  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * SP, OFF_G = OFF_M + L * SP;
-  static constexpr int OFF_I = OFF_G + L * 512;
+  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * SP, OFF_I = OFF_M + L * SP;
   static constexpr int BUF = OFF_I + (MODE == GRID_3BIT_LOCAL ? 128 : 0);
-  static constexpr int WARPS = L == 5 ? 4 : 8;  // warps per CTA
-  static constexpr int CTAS = L == 5 ? 3 : 2;   // CTAs per SM
+  static constexpr int WARPS = L == 5 ? 8 : 12;  // warps per CTA
+  static constexpr int CTAS = 2;                 // CTAs per SM
   static constexpr int SMEM = WARPS * 2 * BUF;
 };
 
@@ -403,10 +367,9 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     k_backward_lion(TS* __restrict__ logits, TS* __restrict__ mom,
                     float* __restrict__ s, float* __restrict__ ms,
                     const int8_t* __restrict__ i0, const float* __restrict__ dW,
-                    float* __restrict__ gbuf, int64_t N, int64_t K, uint32_t k0,
-                    uint32_t k1, uint32_t t_next, int noise, float inv_tau,
-                    float inv_tau_next, float lr, float b1, float omb1, float b2,
-                    float omb2, __nv_bfloat16* __restrict__ What,
+                    int64_t N, int64_t K, const PhiloxKeys ks, uint32_t t, int noise,
+                    float inv_tau, float inv_tau_next, float lr, float b1, float omb1,
+                    float b2, float omb2, __nv_bfloat16* __restrict__ What,
                     float* __restrict__ dl_dbg, float* __restrict__ ds_dbg) {
   using C = BwdCfg<MODE, TS>;
   constexpr int L = C::L;
@@ -419,9 +382,10 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
   const int64_t warp = (int64_t)blockIdx.x * C::WARPS + wic;
   const int64_t nwarps = (int64_t)gridDim.x * C::WARPS;
   const uint32_t wbuf = smem_u32(bwd_smem) + (uint32_t)(wic * 2 * C::BUF);
-  // shared-memory plane order: dW, logits 0..L-1, momenta, noise, (i0)
+  const uint32_t t1 = t + 1u;
+  // shared-memory plane order: dW, logits 0..L-1, momenta, (i0)
   auto prefetch = [&](int64_t gi, int buf) {
-    const int64_t c = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
+    const int64_t c = gi * kGroup + 4 * lane;  // K = G * 128
     const uint32_t d = wbuf + (uint32_t)(buf * C::BUF + 16 * lane);
     cp_async16(d, dW + c);
     const uint32_t ds_ = wbuf + (uint32_t)(buf * C::BUF + (S16 ? 8 : 16) * lane);
@@ -434,7 +398,6 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
         cp_async16(ds_ + (uint32_t)(C::OFF_L + p * C::SP), logits + p * NK + c);
         cp_async16(ds_ + (uint32_t)(C::OFF_M + p * C::SP), mom + p * NK + c);
       }
-      cp_async16(d + (uint32_t)(C::OFF_G + p * 512), gbuf + p * NK + c);
     }
     if (MODE == GRID_3BIT_LOCAL)
       cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::OFF_I + 4 * lane), i0 + c);
@@ -457,8 +420,8 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     cp_async_wait<1>();  // this lane's copies of group gi have landed
     const uint8_t* sb = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
     const uint8_t* sb_s = bwd_smem + wic * 2 * C::BUF + buf * C::BUF + (S16 ? 8 : 16) * lane;
-    const int64_t c0 = (gi / G) * K + (gi % G) * kGroup + 4 * lane;
-    float Dr[4], Lr[L][4], Mr[L][4], Gr[L][4];
+    const int64_t c0 = gi * kGroup + 4 * lane;
+    float Dr[4], Lr[L][4], Mr[L][4];
     *reinterpret_cast<float4*>(Dr) = *reinterpret_cast<const float4*>(sb);
 #pragma unroll
     for (int p = 0; p < L; ++p) {
@@ -479,8 +442,6 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
         *reinterpret_cast<float4*>(Mr[p]) =
             *reinterpret_cast<const float4*>(sb + C::OFF_M + p * C::SP);
       }
-      *reinterpret_cast<float4*>(Gr[p]) =
-          *reinterpret_cast<const float4*>(sb + C::OFF_G + p * 512);
     }
     int lev[4] = {0, 0, 0, 0};
     if (MODE == GRID_3BIT_LOCAL) {
@@ -489,81 +450,61 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
 #pragma unroll
       for (int j = 0; j < 4; ++j) lev[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
-    float gnext[NEXT ? 4 : 1][L];
-    uint32_t rsr[S16 ? 4 : 1][L];  // stochastic-rounding thresholds (bf16 state)
-    if (S16) {
-      // the Philox words of step t + 1 give the next step's noise (NEXT) and
-      // the rounding thresholds of this step's update
-      uint32_t wd[4][5];
-      quad_words5((uint64_t)c0, t_next, k0, k1, L == 5, wd);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int p = 0; p < L; ++p) {
-          rsr[S16 ? j : 0][p] = wd[j][p];
-          if (NEXT)
-            gnext[NEXT ? j : 0][p] =
-                noise ? gumbel<GridT<MODE>::FAST_GUMBEL>(word_to_unit(wd[j][p])) : 0.f;
-        }
-      }
-    } else if (NEXT) {
-      // the lane's four coordinates form an aligned quad (c0 % 4 == 0)
-      float gq[4][5];
-      if (noise) {
-        quad_noise5<GridT<MODE>::FAST_GUMBEL>((uint64_t)c0, t_next, k0, k1, L == 5, gq);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int p = 0; p < L; ++p) gnext[NEXT ? j : 0][p] = gq[j][p];
-    }
+    // pass 1: this step's probabilities (pre-update logits, words of step t),
+    // gradients and Lion
+    uint32_t q1[4] = {0u, 0u, 0u, 0u};
+    if (L == 5 && noise) block1_words((uint64_t)c0, t, ks, q1);
     float ds_part = 0.f;
-    float Lo[L][4], Mo[L][4], Do[DBG ? L : 1][4];
+    float Do[DBG ? L : 1][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float l[L], y[L], cand[5];
+      uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
+      if (noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t, ks, wd);
+      wd[4] = q1[j];
+      // e: unnormalised e_k (categorical) or the probabilities (ternary)
+      float l[L], e[L], cand[5], r;
 #pragma unroll
-      for (int p = 0; p < L; ++p) {
-        l[p] = Lr[p][j];
-        y[p] = Gr[p][j];  // this step's probabilities, kept by its soft weight
-      }
-      const float dw = Dr[j];
+      for (int p = 0; p < L; ++p) l[p] = Lr[p][j];
       candidates<MODE>(lev[j], cand);
-      const float v = value_of<MODE>(y, cand);
+      const float v = coord_value<MODE>(l, wd, noise, inv_tau, cand, e, &r);
+      const float dw = Dr[j];
       ds_part = fmaf(dw, v, ds_part);
       const float a = sg * dw * inv_tau;
       float dl[L];
       if (MODE == GRID_TERNARY) {
-        const float gm = a * (y[3] - y[2]) * y[1] * y[0];
-        const float gs = 2.f * a * y[1] * y[3] * y[2];
+        const float gm = a * (e[3] - e[2]) * e[1] * e[0];
+        const float gs = 2.f * a * e[1] * e[3] * e[2];
         dl[0] = -gm;
         dl[1] = gm;
         dl[2] = -gs;
         dl[3] = gs;
       } else {
+        // y_k = e_k r: dl_k = (a r^2) e_k sum_j e_j (c_k - c_j); the j = k
+        // term is zero and skipped
+        const float a2 = a * r * r;
+        float dc[L][L];
+#pragma unroll
+        for (int p = 0; p < L; ++p)
+#pragma unroll
+          for (int q = p + 1; q < L; ++q) {
+            dc[p][q] = cand[p] - cand[q];
+            dc[q][p] = -dc[p][q];
+          }
 #pragma unroll
         for (int p = 0; p < L; ++p) {
           float acc = 0.f;
 #pragma unroll
-          for (int q = 0; q < L; ++q) acc = fmaf(y[q], cand[p] - cand[q], acc);
-          dl[p] = a * y[p] * acc;
+          for (int q = 0; q < L; ++q)
+            if (q != p) acc = fmaf(e[q], dc[p][q], acc);
+          dl[p] = a2 * e[p] * acc;
         }
       }
 #pragma unroll
       for (int p = 0; p < L; ++p) {
         float th = l[p], mm = Mr[p][j];
         lion_update(th, mm, dl[p], lr, b1, omb1, b2, omb2);
-        if (S16) {
-          th = bf16_sr(th, rsr[S16 ? j : 0][p]);
-          mm = bf16_rn(mm);
-        }
-        Lo[p][j] = th;
-        Mo[p][j] = mm;
+        Lr[p][j] = th;  // fp32; rounded in pass 2 with bf16 state
+        Mr[p][j] = S16 ? bf16_rn(mm) : mm;
         if (DBG) Do[DBG ? p : 0][j] = dl[p];
       }
     }
@@ -571,15 +512,12 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     for (int p = 0; p < L; ++p) {
       if (S16) {
         // the values are bf16 already: keep their top halves
-        *reinterpret_cast<uint2*>(logits + p * NK + c0) =
-            make_uint2((__float_as_uint(Lo[p][0]) >> 16) | (__float_as_uint(Lo[p][1]) & 0xFFFF0000u),
-                       (__float_as_uint(Lo[p][2]) >> 16) | (__float_as_uint(Lo[p][3]) & 0xFFFF0000u));
         *reinterpret_cast<uint2*>(mom + p * NK + c0) =
-            make_uint2((__float_as_uint(Mo[p][0]) >> 16) | (__float_as_uint(Mo[p][1]) & 0xFFFF0000u),
-                       (__float_as_uint(Mo[p][2]) >> 16) | (__float_as_uint(Mo[p][3]) & 0xFFFF0000u));
+            make_uint2((__float_as_uint(Mr[p][0]) >> 16) | (__float_as_uint(Mr[p][1]) & 0xFFFF0000u),
+                       (__float_as_uint(Mr[p][2]) >> 16) | (__float_as_uint(Mr[p][3]) & 0xFFFF0000u));
       } else {
-        *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(Lo[p]);
-        *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(Mo[p]);
+        *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(Lr[p]);
+        *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(Mr[p]);
       }
       if (DBG)
         *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
@@ -594,23 +532,38 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
       ms[gi] = ms_new;
       if (DBG) ds_dbg[gi] = ds;
     }
-    if (NEXT) {
-      float w[4], yn[4][L];
+    // pass 2 (NEXT, or bf16 state): the words of step t + 1 give the
+    // stochastic-rounding thresholds of the updated logits and the next
+    // step's noise
+    if (NEXT || S16) {
+      uint32_t r1[4] = {0u, 0u, 0u, 0u};
+      if (L == 5 && (S16 || noise)) block1_words((uint64_t)c0, t1, ks, r1);
+      float w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float l[L], cand[5];
+        uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
+        if (S16 || noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t1, ks, wd);
+        wd[4] = r1[j];
+        float l[L];
 #pragma unroll
-        for (int p = 0; p < L; ++p) l[p] = Lo[p][j];
-        candidates<MODE>(lev[j], cand);
-        w[j] = s_new * coord_soft<MODE>(l, gnext[NEXT ? j : 0], inv_tau_next, cand, yn[j]);
+        for (int p = 0; p < L; ++p) {
+          if (S16) Lr[p][j] = bf16_sr(Lr[p][j], wd[p]);
+          l[p] = Lr[p][j];
+        }
+        if (NEXT) {
+          float e[L], cand[5], r;
+          candidates<MODE>(lev[j], cand);
+          w[j] = s_new * coord_value<MODE>(l, wd, noise, inv_tau_next, cand, e, &r);
+        }
       }
-      store_bf16x4(What + c0, w);
+      if (S16) {
 #pragma unroll
-      for (int p = 0; p < L; ++p) {
-        // the next step's probabilities, for its backward
-        float4 y4 = make_float4(yn[0][p], yn[1][p], yn[2][p], yn[3][p]);
-        *reinterpret_cast<float4*>(gbuf + p * NK + c0) = y4;
+        for (int p = 0; p < L; ++p)
+          *reinterpret_cast<uint2*>(logits + p * NK + c0) =
+              make_uint2((__float_as_uint(Lr[p][0]) >> 16) | (__float_as_uint(Lr[p][1]) & 0xFFFF0000u),
+                         (__float_as_uint(Lr[p][2]) >> 16) | (__float_as_uint(Lr[p][3]) & 0xFFFF0000u));
       }
+      if (NEXT) store_bf16x4(What + c0, w);
     }
   }
   cp_async_wait<0>();
@@ -1144,48 +1097,44 @@ cudaError_t launch_init_state(int mode, const float* W32,
 }
 
 template <int MODE, typename TS>
-static void soft_weight_ts(const StepArgs& a, __nv_bfloat16* What,
-                           float* gbuf, float* wsoft32, int blocks,
+static void soft_weight_ts(const StepArgs& a, __nv_bfloat16* What, float* wsoft32, int blocks,
                            cudaStream_t st) {
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
   const float inv_tau = 1.0f / a.tau;
   const TS* lg = reinterpret_cast<const TS*>(a.logits);
   if (wsoft32)
-    k_soft_weight<MODE, true, TS><<<blocks, 256, 0, st>>>(
-        lg, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        gbuf, wsoft32);
+    k_soft_weight<MODE, true, TS><<<blocks, 256, 0, st>>>(lg, a.s, a.i0, a.N, a.K,
+                                                          philox_keys(k0, k1), a.t, a.noise,
+                                                          inv_tau, What, wsoft32);
   else
-    k_soft_weight<MODE, false, TS><<<blocks, 256, 0, st>>>(
-        lg, a.s, a.i0, a.N, a.K, k0, k1, a.t, a.noise, inv_tau, What,
-        gbuf, nullptr);
+    k_soft_weight<MODE, false, TS><<<blocks, 256, 0, st>>>(lg, a.s, a.i0, a.N, a.K,
+                                                           philox_keys(k0, k1), a.t, a.noise,
+                                                           inv_tau, What, nullptr);
 }
 
 template <int MODE>
-static void soft_weight_mode(const StepArgs& a, __nv_bfloat16* What,
-                             float* gbuf, float* wsoft32, int blocks,
+static void soft_weight_mode(const StepArgs& a, __nv_bfloat16* What, float* wsoft32, int blocks,
                              cudaStream_t st) {
   if (a.state16)
-    soft_weight_ts<MODE, __nv_bfloat16>(a, What, gbuf, wsoft32, blocks, st);
+    soft_weight_ts<MODE, __nv_bfloat16>(a, What, wsoft32, blocks, st);
   else
-    soft_weight_ts<MODE, float>(a, What, gbuf, wsoft32, blocks, st);
+    soft_weight_ts<MODE, float>(a, What, wsoft32, blocks, st);
 }
 
-cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What,
-                               float* gbuf, float* wsoft32, int sm_count,
-                               cudaStream_t st) {
+cudaError_t launch_soft_weight(const StepArgs& a, __nv_bfloat16* What, float* wsoft32,
+                               int sm_count, cudaStream_t st) {
   const int64_t groups = a.N * (a.K / kGroup);
   const int blocks = grid_for(groups * 32, 256, sm_count * 8);
   switch (a.mode) {
-    case GRID_2BIT: soft_weight_mode<GRID_2BIT>(a, What, gbuf, wsoft32, blocks, st); break;
-    case GRID_TERNARY: soft_weight_mode<GRID_TERNARY>(a, What, gbuf, wsoft32, blocks, st); break;
-    default: soft_weight_mode<GRID_3BIT_LOCAL>(a, What, gbuf, wsoft32, blocks, st);
+    case GRID_2BIT: soft_weight_mode<GRID_2BIT>(a, What, wsoft32, blocks, st); break;
+    case GRID_TERNARY: soft_weight_mode<GRID_TERNARY>(a, What, wsoft32, blocks, st); break;
+    default: soft_weight_mode<GRID_3BIT_LOCAL>(a, What, wsoft32, blocks, st);
   }
   return cudaGetLastError();
 }
 
 template <int MODE, bool NEXT, typename TS>
-static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
-                          float lr, float b1, float b2, float tau_next,
+static void backward_mode(const StepArgs& a, const float* dW, float lr, float b1, float b2, float tau_next,
                           __nv_bfloat16* What, float* dl_dbg, float* ds_dbg,
                           int blocks, cudaStream_t st) {
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
@@ -1212,42 +1161,40 @@ static void backward_mode(const StepArgs& a, const float* dW, float* gbuf,
   if (dl_dbg) {
     smem_optin<k_backward_lion<MODE, true, NEXT, TS>>(C::SMEM);
     cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, true, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
-                       dW, gbuf, a.N, a.K, k0, k1, (uint32_t)(a.t + 1), a.noise, inv_tau,
+                       dW, a.N, a.K, philox_keys(k0, k1), a.t, a.noise, inv_tau,
                        inv_tau_next, lr, b1, omb1, b2, omb2, What, dl_dbg, ds_dbg);
   } else {
     smem_optin<k_backward_lion<MODE, false, NEXT, TS>>(C::SMEM);
     cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, false, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
-                       dW, gbuf, a.N, a.K, k0, k1, (uint32_t)(a.t + 1), a.noise, inv_tau,
+                       dW, a.N, a.K, philox_keys(k0, k1), a.t, a.noise, inv_tau,
                        inv_tau_next, lr, b1, omb1, b2, omb2, What, (float*)nullptr,
                        (float*)nullptr);
   }
 }
 
 template <int MODE>
-static void backward_dispatch(const StepArgs& a, const float* dW, float* gbuf,
-                              float lr, float b1, float b2, float tau_next,
+static void backward_dispatch(const StepArgs& a, const float* dW, float lr, float b1, float b2, float tau_next,
                               __nv_bfloat16* What, float* dl_dbg,
                               float* ds_dbg, int blocks, cudaStream_t st) {
   const bool next = tau_next > 0.f;
   if (a.state16) {
     if (next)
-      backward_mode<MODE, true, __nv_bfloat16>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+      backward_mode<MODE, true, __nv_bfloat16>(a, dW, lr, b1, b2, tau_next, What, dl_dbg,
                                                ds_dbg, blocks, st);
     else
-      backward_mode<MODE, false, __nv_bfloat16>(a, dW, gbuf, lr, b1, b2, tau_next, What,
+      backward_mode<MODE, false, __nv_bfloat16>(a, dW, lr, b1, b2, tau_next, What,
                                                 dl_dbg, ds_dbg, blocks, st);
   } else {
     if (next)
-      backward_mode<MODE, true, float>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg,
+      backward_mode<MODE, true, float>(a, dW, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg,
                                        blocks, st);
     else
-      backward_mode<MODE, false, float>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg,
+      backward_mode<MODE, false, float>(a, dW, lr, b1, b2, tau_next, What, dl_dbg,
                                         ds_dbg, blocks, st);
   }
 }
 
-cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
-                                 float* gbuf, float lr, float b1, float b2,
+cudaError_t launch_backward_lion(const StepArgs& a, const float* dW, float lr, float b1, float b2,
                                  float tau_next, __nv_bfloat16* What,
                                  float* dl_dbg, float* ds_dbg, int sm_count,
                                  cudaStream_t st) {
@@ -1262,9 +1209,9 @@ cudaError_t launch_backward_lion(const StepArgs& a, const float* dW,
                          ? blocks_for(BwdCfg<GRID_3BIT_LOCAL>::WARPS, BwdCfg<GRID_3BIT_LOCAL>::CTAS)
                          : blocks_for(BwdCfg<GRID_2BIT>::WARPS, BwdCfg<GRID_2BIT>::CTAS);
   switch (a.mode) {
-    case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
-    case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
-    default: backward_dispatch<GRID_3BIT_LOCAL>(a, dW, gbuf, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st);
+    case GRID_2BIT: backward_dispatch<GRID_2BIT>(a, dW, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    case GRID_TERNARY: backward_dispatch<GRID_TERNARY>(a, dW, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st); break;
+    default: backward_dispatch<GRID_3BIT_LOCAL>(a, dW, lr, b1, b2, tau_next, What, dl_dbg, ds_dbg, blocks, st);
   }
   return cudaGetLastError();
 }

@@ -35,7 +35,7 @@ struct Weight {
   int64_t N = 0, K = 0, G = 0;
   uint64_t seed = 0;
   float *logits = nullptr, *mom = nullptr, *s = nullptr, *ms = nullptr;
-  float *gbuf = nullptr, *dW = nullptr;
+  float* dW = nullptr;
   int8_t* i0 = nullptr;
   __nv_bfloat16* What = nullptr;
   CUtensorMap tmA;  // What as GEMM operand A
@@ -191,8 +191,8 @@ int run_step(gsq_mlp* c, float tau, float tau_next, float lr, float b1, float b2
   const int64_t T = c->T, H = c->H, F = c->F;
   if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
     for (int i = 0; i < 3; ++i)
-      CKM(launch_soft_weight(weight_args(c, i, tau), c->w[i].What, c->w[i].gbuf,
-                             nullptr, c->sms, c->st));
+      CKM(launch_soft_weight(weight_args(c, i, tau), c->w[i].What, nullptr, c->sms,
+                             c->st));
   CKM(forward(c, c->loss_hist + (c->t % kLossRing), true));
   EpiParams ep = epi(c, nullptr);
   // dD = dp^T . (h^T)^T
@@ -210,7 +210,7 @@ int run_step(gsq_mlp* c, float tau, float tau_next, float lr, float b1, float b2
   CKM(launch_gemm(c->tmA_dbT, c->tmB_XnT, c->w[1].em_dW, F, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
   for (int i = 0; i < 3; ++i)
-    CKM(launch_backward_lion(weight_args(c, i, tau), c->w[i].dW, c->w[i].gbuf, lr, b1,
+    CKM(launch_backward_lion(weight_args(c, i, tau), c->w[i].dW, lr, b1,
                              b2, tau_next, c->w[i].What, nullptr, nullptr, c->sms,
                              c->st));
   c->t += 1;
@@ -275,7 +275,6 @@ int gsq_mlp_init(gsq_mlp** out, const void* Xn, int x_dtype, const void* R,
     const int64_t NK = w.N * w.K;
     ALM(w.logits, c->L * NK);
     ALM(w.mom, c->L * NK);
-    ALM(w.gbuf, c->L * NK);
     ALM(w.s, w.N * w.G);
     ALM(w.ms, w.N * w.G);
     ALM(w.i0, NK);
@@ -462,7 +461,7 @@ int gsq_mlp_recon_error(gsq_mlp* c, int mode, float tau, double* abs_err,
     } else {
       StepArgs a = weight_args(c, i, tau);
       a.noise = 0;
-      CKM(launch_soft_weight(a, w.What, nullptr, nullptr, c->sms, c->st));
+      CKM(launch_soft_weight(a, w.What, nullptr, c->sms, c->st));
     }
   }
   CKM(forward(c, c->scratch, false));

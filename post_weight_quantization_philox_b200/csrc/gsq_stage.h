@@ -18,7 +18,7 @@ struct StageWeight {
   int64_t N = 0, K = 0, G = 0;
   uint64_t seed = 0;
   float *logits = nullptr, *mom = nullptr, *s = nullptr, *ms = nullptr;
-  float *gbuf = nullptr, *dW = nullptr;
+  float* dW = nullptr;
   int8_t* i0 = nullptr;
   __nv_bfloat16* What = nullptr;
   CUtensorMap tmA;  // What as GEMM operand A

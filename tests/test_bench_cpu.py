@@ -18,17 +18,21 @@ class _Layer:
 
 
 @pytest.mark.parametrize("name,L,per_coord", [
-    # 4 dW + 2 W_hat + logits and momenta read and written (16 L) + probabilities
-    # read and written (8 L), + 1 initial level for the 3-bit grid
-    ("c2_qproj_4096x4096", 4, 102), ("c4_gateproj_14336x4096", 4, 102),
-    ("c3_downproj_4096x14336", 5, 127)])
+    # 4 dW + 2 W_hat + logits and momenta read and written (16 L), + 1 initial
+    # level for the 3-bit grid: the algorithmic bytes 4 + 16 L (+1) of the
+    # backward plus the 2 B of the fused next soft weight
+    ("c2_qproj_4096x4096", 4, 70), ("c4_gateproj_14336x4096", 4, 70),
+    ("c3_downproj_4096x14336", 5, 87)])
 def test_fused_backward_bytes_per_coordinate(name, L, per_coord):
     cfg = synth.CONFIGS[name]
     w = bench.phase_bytes_flops(cfg, _Layer(L), 4)
     groups = cfg.N * cfg.K // 128
     assert w["backward_lion_next_soft"] == ("hbm", cfg.N * cfg.K * per_coord + 16 * groups)
-    # without the next soft weight: no probabilities written, no W_hat
-    assert w["backward_lion"][1] == cfg.N * cfg.K * (per_coord - 2 - 4 * L) + 16 * groups
+    # without the next soft weight: no W_hat
+    assert w["backward_lion"][1] == cfg.N * cfg.K * (per_coord - 2) + 16 * groups
+    # the soft weight alone: logits read, bf16 weight written (4 L + 2, + 1)
+    extra = 1 if L == 5 else 0
+    assert w["soft_weight"][1] == cfg.N * cfg.K * (4 * L + 2 + extra) + 4 * groups
     assert w["forward_gemm"] == ("tensor", 2.0 * cfg.N * cfg.T * cfg.K)
     assert w["weight_grad_gemm"] == w["forward_gemm"]
 
@@ -44,8 +48,8 @@ def test_bf16_state_halves_the_state_bytes():
 def test_step_roofline_q_proj():
     cfg = synth.CONFIGS["c2_qproj_4096x4096"]
     w = bench.phase_bytes_flops(cfg, _Layer(4), 4)
-    r = bench.step_roofline(w, 0.5, 1374.8, 6457.4)
-    gemm_ms = 2 * 2 * 4096 ** 3 / 1374.8e12 * 1e3
+    r = bench.step_roofline(w, 0.5, 1662.4, 6457.4)
+    gemm_ms = 2 * 2 * 4096 ** 3 / 1662.4e12 * 1e3
     hbm_ms = w["backward_lion_next_soft"][1] / 6457.4e9 * 1e3
     assert r["gemm_ms"] == pytest.approx(gemm_ms, abs=1e-4)
     assert r["hbm_ms"] == pytest.approx(hbm_ms, abs=1e-4)
