@@ -1,13 +1,18 @@
 """Benchmark of the GSQ layer-reconstruction step on B200.
 
-One step = one pass of the whole hot path over one synthetic layer: Philox
-Gumbel soft weight, forward GEMM with fused loss / output gradient, weight-
-gradient GEMM, fused logit/scale gradients with Lion.  The default workload is
-the Llama-3.1-8B q_proj-shaped layer (4096 x 4096, 4096 calibration tokens,
-2-bit grid).  Under torchrun each rank quantizes its own independent layer of
-that shape (weak scaling, no data-path collective).
+Default workload: the Llama-3.1-70B-shaped transformer block (hidden 8192,
+64 query / 8 key-value heads of 128, SwiGLU 28672, 8 x 2048 tokens, 2-bit
+grid).  One bench step is one GSQ step of every stage of the block: the Q
+and K layers, the V/O joint stage and the MLP joint stage (seven weights,
+8.55e8 grid coordinates).  Each stage step is the whole hot path: Philox
+Gumbel soft weight, forward GEMMs with the fused loss / output gradient,
+weight-gradient GEMMs, fused logit/scale gradients with Lion (and the next
+step's soft weight).  Under torchrun each rank quantizes its own block (weak
+scaling, no data-path collective).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W]     # the 70B block step
+    python bench.py --config NAME [--split rows] ...          # one layer
+    python bench.py --stage mlp|attn|scale|gptq|block|kquant  # one stage
     python bench.py --impl reference ...   # the oracle on the host cores
 
 Prints one JSON line on rank 0.
@@ -154,15 +159,25 @@ def run_gsq(args, rank, world, local_rank):
         if args.rows % 256 or not 0 < args.rows <= full.N:
             raise SystemExit(f"--rows must be a multiple of 256 in (0, {full.N}]")
         cfg = dataclasses.replace(full, N=args.rows, name=f"{full.name}_rows{args.rows}")
-    # each rank quantizes its own independent layer of the same shape
-    w_seed, x_seed, _ = layer_seeds(full, rank)
-    W = synth.make_weight(full, seed=w_seed, rows=slice(0, cfg.N))
+    split = args.split == "rows"
+    row0 = None
+    if split:
+        # one layer split by rows over the ranks: the same layer and Philox
+        # seed everywhere, rank r holds band r keyed by its global row offset
+        w_seed, x_seed, philox_seed = layer_seeds(cfg, 0)
+        row0, n = row_shard(cfg.N, rank, world)
+        W = synth.make_weight(full, seed=w_seed, rows=slice(row0, row0 + n))
+        cfg = dataclasses.replace(cfg, N=n)
+    else:
+        # each rank quantizes its own independent layer of the same shape
+        w_seed, x_seed, philox_seed = layer_seeds(full, rank)
+        W = synth.make_weight(full, seed=w_seed, rows=slice(0, cfg.N))
     X = synth.make_calib(full, seed=x_seed)
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
     stream = torch.cuda.current_stream()
     state16 = args.state == "bf16"
-    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=layer_seeds(cfg, rank)[2], state_bf16=state16)
+    lay = gsq.gsq_init(Wd, Xd, 128, cfg.grid, seed=philox_seed, state_bf16=state16, row0=row0)
     taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
     nt = len(taus)
 
@@ -204,14 +219,22 @@ def run_gsq(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     ms = max_over_ranks(ms, world)
+    if split and world > 1:
+        # the layer's loss is the sum of the bands' losses (a scalar; the
+        # steps themselves exchange nothing)
+        import torch.distributed as dist
+        lt = torch.tensor([loss], dtype=torch.float64, device="cuda")
+        dist.all_reduce(lt, op=dist.ReduceOp.SUM)
+        loss = float(lt.item())
 
     # ---- end to end: host buffers through the C ABI, whole quantization job
-    e2e = None if args.no_e2e else run_e2e(gsq, torch, cfg, W, X, rank)
+    e2e = None if args.no_e2e else run_e2e(gsq, torch, cfg, W, X, rank, row0=row0)
     if e2e is not None and world > 1:
-        # every rank ran its own job; the whole job ends with the slowest
+        # every rank ran its own job (or band); the whole job ends with the slowest
         sec = max_over_ranks(e2e["seconds"] * 1e3, world) / 1e3
         e2e["seconds"] = sec
-        e2e["value"] = whole_job_rate(world, cfg.N * cfg.K * cfg.steps, sec * 1e3)
+        units = full.N * full.K * cfg.steps if split else world * cfg.N * cfg.K * cfg.steps
+        e2e["value"] = whole_job_rate(1, units, sec * 1e3)
         e2e["ranks"] = world
 
     if rank != 0:
@@ -219,7 +242,10 @@ def run_gsq(args, rank, world, local_rank):
     hbm, tf_burst, tf_sus, peak_kind = peaks()
     steps_per_s = args.steps / (ms / 1e3)
     coords = cfg.N * cfg.K
-    value = whole_job_rate(world, coords * args.steps, ms)
+    # coordinates all ranks updated per step: the whole layer when it is
+    # split, one layer per rank otherwise
+    job_coords = (full.N if not args.rows else args.rows) * full.K if split else world * coords
+    value = whole_job_rate(1, job_coords * args.steps, ms)
     names = ["soft_weight", "forward_gemm", "weight_grad_gemm", "backward_lion",
              "backward_lion_next_soft"]
     es = 2 if state16 else 4
@@ -256,7 +282,8 @@ def run_gsq(args, rank, world, local_rank):
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-        "steps_per_s": steps_per_s, "higher_is_better": True, "scaling": "weak",
+        "steps_per_s": steps_per_s, "higher_is_better": True,
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None,
         "dtype": ("bf16 GEMM operands, bf16 logit/momentum state (stochastic rounding)"
                   if state16 else "bf16 GEMM operands, fp32 state"),
@@ -264,7 +291,8 @@ def run_gsq(args, rank, world, local_rank):
         "config": {"workload": cfg.name + ("_bf16_state" if state16 else ""),
                    "N": cfg.N, "K": cfg.K, "T": cfg.T,
                    "grid": ["2bit", "ternary", "3bit_local"][cfg.grid], "group": 128,
-                   "parallelism": f"independent layer per GPU x{world}",
+                   "parallelism": (f"one layer split by rows over {world} GPUs (global row offset)"
+                                   if split else f"independent layer per GPU x{world}"),
                    "l2": f"state (logits + Lion momenta, {state_mb:.0f} MB) larger than L2; no flush"},
         "roofline": {"bound": d["bound"], "kernel": dom, "achieved": d["achieved"],
                      "peak": d["peak"], "unit": d["unit"], "frac": d["frac"],
@@ -282,10 +310,10 @@ def run_gsq(args, rank, world, local_rank):
     return out
 
 
-def run_e2e(gsq, torch, cfg, W, X, rank):
+def run_e2e(gsq, torch, cfg, W, X, rank, row0=None):
     """Whole quantization job from pinned host buffers through the C ABI:
     upload + init, the config's steps, loss history read-back, harden+pack
-    into host memory."""
+    into host memory (of the rank's band when the layer is split by rows)."""
     Wh = torch.from_numpy(W).to(torch.bfloat16).pin_memory()
     Xh = torch.from_numpy(X).to(torch.bfloat16).pin_memory()
     taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)
@@ -295,7 +323,7 @@ def run_e2e(gsq, torch, cfg, W, X, rank):
     hist = np.zeros(min(cfg.steps, 4096), np.float64)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    lay = gsq.gsq_init(Wh, Xh, 128, cfg.grid, seed=rank)
+    lay = gsq.gsq_init(Wh, Xh, 128, cfg.grid, seed=0 if row0 is not None else rank, row0=row0)
     lay.run(taus, cfg.lr)
     gsq._check(gsq.lib().gsq_loss_history(lay.ctx, cfg.steps - hist.size, hist.size,
                                           hist.ctypes.data), "gsq_loss_history")
@@ -373,6 +401,20 @@ def rank_seed(base: int, rank: int) -> int:
 def layer_seeds(cfg, rank):
     """(W seed, X seed, Philox seed) of rank's independent layer."""
     return rank_seed(1000 + cfg.number, rank), rank_seed(2000 + cfg.number, rank), rank
+
+
+def row_shard(N: int, rank: int, world: int, align: int = 256):
+    """(row0, rows) of rank's shard when the rows of one layer are split over
+    world ranks: contiguous bands with boundaries on multiples of `align`
+    rows (the GEMM tile) where the layer allows, the last band taking the
+    remainder.  Rows are independent problems (the loss is a sum over output
+    rows and groups lie inside rows), so the bands need no exchange."""
+    units = max(1, N // align) if N >= align * world else 0
+    if units:
+        b = [min(N, (r * units // world) * align) for r in range(world)] + [N]
+    else:
+        b = [r * N // world for r in range(world)] + [N]
+    return b[rank], b[rank + 1] - b[rank]
 
 
 def max_over_ranks(ms: float, world: int, device="cuda") -> float:
@@ -654,6 +696,234 @@ def run_block_pipeline(args, rank, world, local_rank):
             "clocks": clk}
 
 
+C5_WORKLOAD = "c5_70b_block_step"
+C5_Q_LAYER = "c5_70b_qproj_8192x8192"
+
+
+def block_step_coords(nseq, S, nh, nkv, d, F):
+    """Grid coordinates of the block's seven weights: Q, K (layers), V, O
+    (joint), gate, up, down (joint)."""
+    H, Hk = nh * d, nkv * d
+    return [H * H, Hk * H, Hk * H + H * H, 3 * H * F]
+
+
+def block_backward_bytes(coords, L=4, es=4, next_soft=True):
+    """Algorithmic bytes of the fused backward over `coords` coordinates (2-bit
+    grid): dW read, L logit and L momentum planes read and written, 16 B per
+    group of 128, plus the next bf16 soft weight."""
+    return coords * (4 + 4 * es * L + (2 if next_soft else 0)) + coords // 128 * 16
+
+
+def run_block_step(args, rank, world, local_rank):
+    """The Llama-3.1-70B-shaped block (hidden 8192, 64 / 8 heads of 128, SwiGLU
+    28672, 8 x 2048 tokens, 2-bit grid), one GSQ step of every stage per
+    bench step: the Q and K layers (8192 x 8192 and 1024 x 8192 on the
+    normalised attention input), the V/O joint stage (probabilities from the
+    frozen query / key weights), the MLP joint stage (gate, up, down).  The
+    timed region runs each stage's K steps through its run call, in the
+    method's stage order.  Inputs are seeded on the device (torch generator):
+    stage inputs normalised to unit RMS per token as after a unit-gain
+    RMSNorm, weights N(0, 0.02^2) bf16, and for the joint stages N(0, 0.05^2)
+    stand-ins of their targets (the step's work does not depend on the
+    target's values).  The end-to-end leg is the whole job: gsq_block_quantize
+    from pinned host buffers (full-precision forward, the four stages' inits
+    and steps, hardening, the quantized output), outputs back in pinned host
+    memory."""
+    import torch
+    from post_weight_quantization_philox_b200 import build
+    build.build()
+    from post_weight_quantization_philox_b200 import gsq
+    torch.cuda.set_device(local_rank)
+    dm = BLOCK_70B
+    nseq, S, nh, nkv, d, F = (dm[k] for k in ("nseq", "S", "nh", "nkv", "d", "F"))
+    T, H, Hk = nseq * S, nh * d, nkv * d
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(8008, rank))
+
+    def randn(shape, std):
+        return torch.randn(shape, generator=gen, device="cuda") * std
+
+    def normalised(shape):
+        x = randn(shape, 1.0)
+        return (x / x.pow(2).mean(1, keepdim=True).sqrt()).to(torch.bfloat16)
+
+    xa, xm = normalised((T, H)), normalised((T, H))
+    shapes = gsq.block_weight_shapes(nh, nkv, d, F)
+    W = {n: randn(shp, 0.02).to(torch.bfloat16) for n, shp in shapes.items()}
+    Ra, Rm = randn((T, H), 0.05), randn((T, H), 0.05)
+    seed = rank
+    q = gsq.gsq_init(W["q"], xa, 128, synth.GRID_2BIT, seed=seed)
+    k = gsq.gsq_init(W["k"], xa, 128, synth.GRID_2BIT, seed=seed + 1)
+    a = gsq.gsq_attn_init(xa, Ra, W["q"], W["k"], W["v"], W["o"], nseq, S, nh, nkv, d,
+                          grid_mode=synth.GRID_2BIT, seed=seed + 2)
+    m = gsq.gsq_mlp_init(xm, Rm, W["gate"], W["up"], W["down"], grid_mode=synth.GRID_2BIT,
+                         seed=seed + 3)
+    del Ra, Rm
+    stages = [("q", q), ("k", k), ("vo", a), ("mlp", m)]
+    lr = 1e-3
+    taus = synth.tau_schedule(1.0, 0.05, 200)
+    sched = np.array([taus[i % len(taus)] for i in range(args.warmup + args.steps)], np.float32)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    for _, st in stages:
+        st.run(sched[:args.warmup], lr)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    # the timed region: every stage's steps, the library's launches only
+    e0.record(stream)
+    for _, st in stages:
+        st.run(sched[args.warmup:], lr)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    losses = {n: st.last_loss() for n, st in stages}
+    # per-phase device time from a second, instrumented run of the same steps
+    ph = {}
+    for n, st in (("q", q), ("k", k)):
+        gsq.gsq_set_timing(st, True)
+        gsq.gsq_phase_times(st)
+        st.run(sched[args.warmup:], lr)
+        pm, pn = gsq.gsq_phase_times(st)
+        gsq.gsq_set_timing(st, False)
+        # soft weight, GEMMs (forward + weight gradient), backward (both kinds)
+        ph[n] = (np.array([pm[0], pm[1] + pm[2], 0.0, pm[3] + pm[4]]),
+                 np.array([pn[0], pn[1] + pn[2], 0, pn[3] + pn[4]]))
+    for n, st in (("vo", a), ("mlp", m)):
+        st.set_timing(True)
+        st.phase_times()
+        st.run(sched[args.warmup:], lr)
+        ph[n] = st.phase_times()
+        st.set_timing(False)
+    for _, st in stages:
+        st.close()
+    del q, k, a, m, stages, xa, xm
+    torch.cuda.empty_cache()
+    ms = max_over_ranks(ms, world)
+
+    # ---- end to end: the whole block job from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = block_e2e(gsq, torch, W, gen, dm, args.e2e_steps, rank)
+        if world > 1:
+            sec = max_over_ranks(e2e["seconds"] * 1e3, world) / 1e3
+            e2e["seconds"] = sec
+            e2e["value"] = whole_job_rate(world, e2e["coords_per_job"], sec * 1e3)
+            e2e["ranks"] = world
+    del W
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    K_ = args.steps
+    coords = block_step_coords(nseq, S, nh, nkv, d, F)
+    flops = block_step_flops(nseq, S, nh, nkv, d, F)
+    names = ["q", "k", "vo", "mlp"]
+    stage_out = {}
+    gemm_ms = gemm_flops = bwd_ms = bwd_bytes = elem_ms = soft_ms = 0.0
+    launches = 0
+    for n, c, f in zip(names, coords, flops):
+        pm, pn = ph[n]
+        launches += int(pn.sum())
+        # backward launches of a run: all but the last step also form the
+        # next soft weight
+        bb = (K_ - 1) * block_backward_bytes(c) + block_backward_bytes(c, next_soft=False)
+        stage_out[n] = {
+            "coords": c, "ms_per_step": round(float(pm.sum()) / K_, 4),
+            "gemm": {"ms_per_step": round(pm[1] / K_, 4),
+                     "tflops": round(f * K_ / (pm[1] / 1e3) / 1e12, 1) if pm[1] else None},
+            "backward": {"ms_per_step": round(pm[3] / K_, 4),
+                         "gbs": round(bb / (pm[3] / 1e3) / 1e9, 1) if pm[3] else None},
+            "elementwise_ms_per_step": round(pm[2] / K_, 4),
+            "soft_weight_ms_per_run": round(pm[0], 4),
+            "last_loss": losses[n]}
+        gemm_ms += pm[1]
+        gemm_flops += f * K_
+        bwd_ms += pm[3]
+        bwd_bytes += bb
+        elem_ms += pm[2]
+        soft_ms += pm[0]
+    gemm_ach = gemm_flops / (gemm_ms / 1e3) / 1e12
+    bwd_ach = bwd_bytes / (bwd_ms / 1e3) / 1e9
+    phases = {
+        "gemm": {"ms": round(gemm_ms / K_, 4), "bound": "tensor", "achieved": round(gemm_ach, 1),
+                 "unit": "TFLOP/s", "peak": tf_burst, "frac": round(gemm_ach / tf_burst, 4),
+                 "frac_of_sustained": round(gemm_ach / tf_sus, 4)},
+        "backward_lion": {"ms": round(bwd_ms / K_, 4), "bound": "hbm",
+                          "achieved": round(bwd_ach, 1), "unit": "GB/s", "peak": hbm,
+                          "frac": round(bwd_ach / hbm, 4)},
+        "elementwise": {"ms": round(elem_ms / K_, 4)},
+        "soft_weight": {"ms_per_run": round(soft_ms, 4)},
+    }
+    dom = "gemm" if gemm_ms >= bwd_ms else "backward_lion"
+    dd = phases[dom]
+    per = ms / K_
+    gemm_floor = sum(flops) / (tf_burst * 1e12) * 1e3
+    hbm_floor = sum(block_backward_bytes(c) for c in coords) / (hbm * 1e9) * 1e3
+    out = {
+        "metric": METRIC, "value": whole_job_rate(world, sum(coords) * K_, ms), "unit": UNIT,
+        "n_gpus": world, "steps": K_, "warmup": args.warmup, "ms_per_step": per,
+        "steps_per_s": 1e3 / per, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 GEMM operands, fp32 state",
+        "data": ("synthetic (seeded torch generator on the device: unit-RMS stage inputs, "
+                 "weights N(0,0.02^2) bf16, joint-stage targets N(0,0.05^2) stand-ins)"),
+        "config": {"workload": C5_WORKLOAD, **dm, "T": T, "grid": "2bit", "group": 128,
+                   "weights": "q, k (layers); v, o (joint); gate, up, down (joint)",
+                   "step": "one GSQ step of every stage (Q, K, V/O, MLP), stage order",
+                   "parallelism": f"independent block per GPU x{world}",
+                   "l2": "every stage's state and activations far larger than L2; no flush"},
+        "roofline": {"bound": dd["bound"], "kernel": ("k_gemm_pair (all GEMMs of the step)"
+                                                      if dom == "gemm" else
+                                                      "k_backward_lion (all weights)"),
+                     "achieved": dd["achieved"], "peak": dd["peak"], "unit": dd["unit"],
+                     "frac": dd["frac"],
+                     "peak_kind": f"{peak_kind} ({'burst bf16' if dom == 'gemm' else 'HBM copy'})",
+                     "traffic": None},
+        "phases": phases, "stages": stage_out,
+        "step_roofline": {"gemm_ms": round(gemm_floor, 3), "hbm_ms": round(hbm_floor, 3),
+                          "ms": round(gemm_floor + hbm_floor, 3),
+                          "frac": round((gemm_floor + hbm_floor) / per, 4),
+                          "how": "all GEMM flops at the burst bf16 rate + the fused backwards' "
+                                 "algorithmic bytes at the copy rate, over the measured step"},
+        "gpu_launches": launches, "clocks": clk, "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline(synth.CONFIGS[C5_Q_LAYER], budget_s=args.cpu_seconds, steps=1)
+        cb["sample"] += " (the block's query projection, one step)"
+        out["cpu_baseline"] = cb
+    return out
+
+
+def block_e2e(gsq, torch, W, gen, dm, steps, rank):
+    """One gsq_block_quantize call (the whole block job, `steps` steps per
+    stage) from pinned host buffers, outputs into pinned host memory."""
+    nseq, S, nh, nkv, d, F = (dm[k] for k in ("nseq", "S", "nh", "nkv", "d", "F"))
+    T, H = nseq * S, nh * d
+    x = torch.randn((T, H), generator=gen, device="cuda").cpu().pin_memory()
+    Wh = {n: w.cpu().pin_memory() for n, w in W.items()}
+    taus = [synth.tau_schedule(1.0, 0.05, steps)] * 4
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    r = gsq.gsq_block_quantize(x, Wh, nseq, S, nh, nkv, d, F, taus, 1e-3, seed=rank,
+                               host_outputs=True)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    coords = sum(a * b for a, b in gsq.block_weight_shapes(nh, nkv, d, F).values())
+    h2d = x.numel() * 4 + sum(w.numel() * 2 for w in Wh.values())
+    d2h = (r["x_out"].numel() * 4 + sum(p.numel() * 4 for p in r["packed"].values())
+           + sum(s.numel() * 4 for s in r["scales"].values()))
+    return {"value": coords * steps / dt, "unit": UNIT, "seconds": dt,
+            "coords_per_job": coords * steps,
+            "h2d_bytes_per_step": h2d / steps, "d2h_bytes_per_step": d2h / steps,
+            "job": (f"gsq_block_quantize from pinned host buffers: full-precision forward, "
+                    f"Q, K, V/O, MLP stages x {steps} steps, hardening, quantized output, "
+                    f"outputs to pinned host memory")}
+
+
 def gptq_simt_flops(N: int, K: int) -> float:
     """fp32 SIMT flops of one GPTQ call: Cholesky of the damped K x K
     Hessian (K^3 / 3), inverse of its triangular factor (K^3 / 3), the
@@ -803,8 +1073,12 @@ def run_kquant_stage(args, rank, world, local_rank):
             "recon_rel": {"start": e_start, "after": e_end}}
 
 
-def run_reference(args, rank, world):
-    """The oracle as the reference arm (rank 0 only)."""
+def run_reference(args, rank, world, block_default=False):
+    """The oracle as the reference arm (rank 0 only), on the same workload
+    as the GPU arm: for the 70B block step, rows of the block's query
+    projection (every weight of the block costs the same two T-long
+    contractions per coordinate, and the oracle's stage steps are the layer
+    step's arithmetic)."""
     if rank != 0:
         return None
     cfg = synth.CONFIGS[args.config]
@@ -820,7 +1094,10 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": cfg.name, "N": cfg.N, "K": cfg.K, "T": cfg.T},
+            "config": ({"workload": C5_WORKLOAD, **BLOCK_70B, "T": cfg.T, "grid": "2bit",
+                        "group": 128} if block_default else
+                       {"workload": cfg.name, "N": cfg.N, "K": cfg.K, "T": cfg.T,
+                        "grid": ["2bit", "ternary", "3bit_local"][cfg.grid], "group": 128}),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cb["cores"],
                              "kind": "oracle", "sample": cb["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -832,7 +1109,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="c2_qproj_4096x4096", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default=None, choices=sorted(synth.CONFIGS),
+                    help="time one layer of this shape (default: the 70B block step)")
     ap.add_argument("--impl", default="gsq", choices=["gsq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -846,14 +1124,22 @@ def main():
                     help="skip the end-to-end job (profiling runs)")
     ap.add_argument("--rows", type=int, default=0,
                     help="single layer: only its first ROWS rows (a multiple of 256)")
+    ap.add_argument("--split", default="layers", choices=["layers", "rows"],
+                    help="N > 1: one independent layer per GPU (weak scaling), or one "
+                         "layer's rows split over the GPUs (strong scaling)")
+    ap.add_argument("--e2e-steps", type=int, default=200,
+                    help="block step: steps per stage of the end-to-end block job")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    block_default = args.config is None and args.stage is None
+    if args.config is None:
+        args.config = C5_Q_LAYER if block_default else "c2_qproj_4096x4096"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        out = run_reference(args, rank, world)
+        out = run_reference(args, rank, world, block_default)
         if out:
             print(json.dumps(out))
         return
@@ -877,6 +1163,8 @@ def main():
         out = run_block_pipeline(args, rank, world, local_rank)
     elif args.stage == "kquant":
         out = run_kquant_stage(args, rank, world, local_rank)
+    elif block_default:
+        out = run_block_step(args, rank, world, local_rank)
     else:
         out = run_gsq(args, rank, world, local_rank)
     if out:

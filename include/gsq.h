@@ -119,6 +119,27 @@ GSQ_API int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const
                                 int grid_mode, const int8_t* init_idx, uint64_t seed,
                                 void* stream);
 
+/* gsq_init_rows -- gsq_init for the rows [row0, row0 + N) of a larger layer
+ * (a shard; state_bf16 = 1 as gsq_init_bf16_state).  W holds those N rows
+ * (N x K), X the whole calibration input, init_idx (nullable) the shard's
+ * N x K initial levels.  The layer loss is a sum over output rows and every
+ * group lies inside one row, so the shards of a layer are independent
+ * problems: Y_ref of the shard is X W_shard^T, i.e. the columns row0 ..
+ * row0 + N of the whole layer's reference output.  The Philox counters take
+ * the global coordinate (row0 + n) K + k, so the shard draws exactly the
+ * noise that a context holding the whole layer draws for those rows, and
+ * the shards' steps together reproduce the whole layer's step (the sum of
+ * the shards' losses is the layer's loss).  This is how a layer is split
+ * over GPUs: one shard per GPU, no exchange during the steps.  (agihunt.info
+ * summary, cost paragraph: the pages run the search on 8 GPUs.)
+ * gsq_debug_uniforms keeps taking global coordinates.
+ * Errors: as gsq_init, and GSQ_ERR_INVALID_ARG for row0 < 0, state_bf16
+ * other than 0 or 1, or global coordinates beyond 2^62. */
+GSQ_API int gsq_init_rows(gsq_ctx** out, const void* W, int w_dtype, const void* X,
+                          int x_dtype, int64_t N, int64_t K, int64_t T, int group,
+                          int grid_mode, const int8_t* init_idx, uint64_t seed,
+                          int64_t row0, int state_bf16, void* stream);
+
 /* GPTQ initial assignment (agihunt.info summary, optimisation paragraph: GSQ
  * starts from GPTQ; the algorithm of Frantar et al., "GPTQ: Accurate
  * Post-Training Quantization for Generative Pre-trained Transformers",
@@ -157,6 +178,17 @@ GSQ_API int gsq_gptq(const void* W, int w_dtype, const void* X, int x_dtype, int
  * Errors: GSQ_ERR_CUDA. */
 GSQ_API int gsq_set_cached_memory_limit(uint64_t bytes);
 GSQ_API int gsq_release_cached_memory(void);
+/* Failure-injection hooks for tests (host side; no GPU fault is involved).
+ * gsq_debug_fail_alloc(after): the library's device allocation that comes
+ * after `after` more successful ones fails as if the device were out of
+ * memory (so 0 fails the next one); a negative value switches the hook off.
+ * Process-wide, all devices.  gsq_debug_pool_used(device, bytes): the bytes
+ * of the device's pool that are handed out (contexts, workspaces) -- 0
+ * before the library first allocates on that device; waits for frees the
+ * library queued.  Errors: GSQ_ERR_INVALID_ARG (null bytes, bad device),
+ * GSQ_ERR_CUDA. */
+GSQ_API int gsq_debug_fail_alloc(int64_t after);
+GSQ_API int gsq_debug_pool_used(int device, uint64_t* bytes);
 /* gsq_init from the GPTQ assignment: the initial levels (init_idx) and the
  * group scales both come from gsq_gptq (instead of round-to-nearest with
  * absmax scales); everything else as gsq_init.  Synchronises the stream. */
@@ -170,7 +202,16 @@ GSQ_API int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void*
  * weight-gradient GEMM, fused logit/scale gradients and Lion update
  * (c = beta1 m + (1-beta1) g; theta -= lr sign(c); m = beta2 m + (1-beta2) g),
  * then t += 1.  tau > 0, lr >= 0, 0 <= beta < 1.  The annealing schedule is
- * the caller's.
+ * the caller's.  Source: agihunt.info summary, method paragraph (the soft
+ * weighted sum of grid points under Gumbel-Softmax sampling, trained on the
+ * output reconstruction error and annealed towards a hard choice) and
+ * optimisation paragraph (Lion, logits trained jointly with the group
+ * scales); atlas.scime.ai, Approach.  Lion itself: Chen et al., "Symbolic
+ * Discovery of Optimization Algorithms", 2023.
+ * Errors: GSQ_ERR_INVALID_ARG for tau <= 0 or not finite, lr < 0 or beta
+ * outside [0, 1); GSQ_ERR_UNSUPPORTED once t reaches 2^32 - 2 (the counter
+ * word); GSQ_ERR_STATE after an earlier failure (a device-side failure of
+ * this step surfaces at the next call that syncs).
  */
 GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2);
 
@@ -183,8 +224,6 @@ GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2
 GSQ_API int gsq_run(gsq_ctx* ctx, const float* taus, int64_t n, float lr,
                     float beta1, float beta2);
 
-/* gsq_last_loss -- loss (sum of squared errors) of the last step.  Syncs.
- * GSQ_ERR_NONFINITE if it was NaN / Inf; GSQ_ERR_STATE before any step. */
 /* Scale-only step (agihunt.info summary, optimisation paragraph: the 2-bit
  * models get one more round that changes only the group scales), on the
  * layer objective of gsq_step:
@@ -202,6 +241,9 @@ GSQ_API int gsq_run(gsq_ctx* ctx, const float* taus, int64_t n, float lr,
 GSQ_API int gsq_scale_step(gsq_ctx* ctx, float lr, float beta1, float beta2);
 /* n scale-only steps (n > 0) */
 GSQ_API int gsq_scale_run(gsq_ctx* ctx, int64_t n, float lr, float beta1, float beta2);
+
+/* gsq_last_loss -- loss (sum of squared errors) of the last step.  Syncs.
+ * GSQ_ERR_NONFINITE if it was NaN / Inf; GSQ_ERR_STATE before any step. */
 GSQ_API int gsq_last_loss(gsq_ctx* ctx, double* loss);
 
 /* gsq_loss_history -- losses of steps [t0, t0 + n) (the last 4096 steps are
@@ -217,7 +259,12 @@ GSQ_API int gsq_packed_bytes(int grid_mode, int64_t N, int64_t K, size_t* bytes)
  * no noise; 3-bit: clamp(i0 + argmax - 2, 0, 7); ternary: zero if the mask
  * pair prefers zero, else the sign pair's choice), packed as an LSB-first
  * bitstream per row of 32-bit little-endian words (code j of a row at bits
- * [j b, j b + b)); the code is the level index (ternary: v + 1).
+ * [j b, j b + b)); the code is the level index (ternary: v + 1).  Source:
+ * agihunt.info summary, method paragraph (as the temperature falls the soft
+ * sum collapses to a hard choice of grid point) and its conclusion
+ * (symmetric group-128 grids, no zero-point, so one fp16 scale per group is
+ * the whole side information: 2.13 bits per weight at 2 bits in the
+ * zero-shot table).  The bit layout is this library's.
  *   packed      gsq_packed_bytes() bytes, host or device.
  *   scales_f16  N x G binary16 (round to nearest even), host or device,
  *               nullable.
@@ -231,7 +278,12 @@ GSQ_API int gsq_harden_pack(gsq_ctx* ctx, void* packed, uint16_t* scales_f16,
  * gsq_recon_error -- A7: abs = || bf16(X) Wq^T - Y_ref ||_F^2 and
  * rel = abs / || Y_ref ||_F^2 with Wq the hard weight (GSQ_RECON_HARD) or
  * the noiseless soft weight at tau (GSQ_RECON_SOFT; tau ignored for hard).
- * Syncs.  Leaves the optimiser state untouched.
+ * Syncs.  Leaves the optimiser state untouched.  Source: the layer's output
+ * reconstruction error on the calibration inputs, the objective named in the
+ * agihunt.info summary, method paragraph.
+ * Errors: GSQ_ERR_INVALID_ARG for a bad mode, a null output or a soft tau
+ * that is not positive and finite; GSQ_ERR_STATE after an earlier failure;
+ * GSQ_ERR_NONFINITE if the error is NaN / Inf.
  */
 GSQ_API int gsq_recon_error(gsq_ctx* ctx, int mode, float tau, double* abs_err,
                     double* rel_err);
@@ -304,6 +356,16 @@ GSQ_API int gsq_debug_backward(gsq_ctx* ctx, float tau, float lr, float beta1,
                        float beta2);
 /* scale-only backward + Lion from the current dW (fills GSQ_DBG_DS) */
 GSQ_API int gsq_debug_scale_backward(gsq_ctx* ctx, float lr, float beta1, float beta2);
+/* gsq_debug_stall_probe -- test hook of the bounded device waits: the next
+ * forward GEMM of the context (in the next gsq_step / gsq_run) first lets
+ * one thread of every CTA wait, with a short bound (about 10 ms), on a
+ * barrier that nothing arrives at, before the CTA issues any load or MMA;
+ * the wait runs out, the kernel records a timeout in the context's error
+ * word and processes no tile, so no copy or MMA is ever in flight.  The
+ * next call that syncs returns GSQ_ERR_TIMEOUT and the context turns
+ * sticky-failed (GSQ_ERR_STATE afterwards), as after a real timeout.
+ * Errors: GSQ_ERR_STATE after an earlier failure. */
+GSQ_API int gsq_debug_stall_probe(gsq_ctx* ctx);
 
 /* ----------------------------------------------- block stage: SwiGLU MLP --
  * The GSQ pages quantize a transformer block in stages; the last stage trains
@@ -362,6 +424,15 @@ GSQ_API int gsq_mlp_debug_set(gsq_mlp* ctx, int which, int buf,
                               const void* host, size_t bytes);
 GSQ_API int gsq_mlp_get_step(gsq_mlp* ctx, uint64_t* t);
 GSQ_API int gsq_mlp_destroy(gsq_mlp* ctx);
+/* gsq_mlp_set_timing / gsq_mlp_phase_times: per-phase device time of the
+ * stage's steps, as gsq_set_timing / gsq_phase_times for a layer: ms[4] and
+ * launches[4] for 0 soft weights, 1 GEMMs (the seven contractions of a
+ * step), 2 elementwise (SwiGLU forward and backward, transposes), 3 fused
+ * backward + Lion of the three weights.  The events between launches keep
+ * each kernel from starting early, so time a separate run.  phase_times
+ * syncs and starts over.  Errors: GSQ_ERR_INVALID_ARG, GSQ_ERR_STATE. */
+GSQ_API int gsq_mlp_set_timing(gsq_mlp* ctx, int on);
+GSQ_API int gsq_mlp_phase_times(gsq_mlp* ctx, double* ms, int64_t* launches);
 
 /* ------------------------------------------- block stage: attention V/O --
  * The GSQ pages quantize a block's query and key projections first, then the
@@ -415,6 +486,11 @@ GSQ_API int gsq_attn_debug_set(gsq_attn* ctx, int which, int buf,
                                const void* host, size_t bytes);
 GSQ_API int gsq_attn_get_step(gsq_attn* ctx, uint64_t* t);
 GSQ_API int gsq_attn_destroy(gsq_attn* ctx);
+/* gsq_attn_set_timing / gsq_attn_phase_times: as gsq_mlp_set_timing, for the
+ * V/O stage (GEMMs: V, the batched P V, the output projection with the
+ * loss, dWo, do, the batched P^T do, dWv; elementwise: transposes). */
+GSQ_API int gsq_attn_set_timing(gsq_attn* ctx, int on);
+GSQ_API int gsq_attn_phase_times(gsq_attn* ctx, double* ms, int64_t* launches);
 
 /* ------------------------------------------- staged block pipeline ------
  * GSQ quantizes the blocks of a model one after another: every block is
@@ -592,7 +668,8 @@ GSQ_API int gsq_kq_destroy(gsq_kq* ctx);
  * GSQ_NOALLOC_MAX_COORDS x 5 floats (1.25 MiB), which every GPU that loads
  * the library holds until exit; count above GSQ_NOALLOC_MAX_COORDS returns
  * GSQ_ERR_INVALID_ARG.  The first call on a device looks up that array's
- * device address (once per device); make that first call before any stream
+ * device address (once per device, and again if the device's context changed
+ * since, e.g. after cudaDeviceReset); make that first call before any stream
  * capture.  All calls share the array: calls whose work overlaps on the GPU
  * (for example on two streams) race and may return each other's values.
  * Enqueued on `stream` (NULL = legacy default stream); syncs.

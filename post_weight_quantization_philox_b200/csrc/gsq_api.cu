@@ -39,10 +39,13 @@ struct gsq_ctx {
   int state16 = 0;
   int64_t N = 0, K = 0, T = 0, Tp = 0, G = 0;
   uint64_t seed = 0, t = 0;
+  // global coordinate of local coordinate 0 (row0 K for a shard of rows)
+  uint64_t coord0 = 0;
   int noise = 1;
   cudaStream_t st = nullptr;
   int dev = 0, sms = 148;
   int failed = 0;  // sticky status (negative) once something went wrong
+  int stall_probe = 0;  // test hook: the next forward GEMM runs the probe
 
   __nv_bfloat16 *Xb = nullptr, *Xt = nullptr, *What = nullptr, *dYt = nullptr;
   float *YrefT = nullptr, *dW = nullptr, *logits = nullptr, *mom = nullptr;
@@ -158,6 +161,7 @@ StepArgs step_args(gsq_ctx* c, float tau) {
   a.noise = c->noise;
   a.tau = tau;
   a.state16 = c->state16;
+  a.coord0 = c->coord0;
   return a;
 }
 
@@ -178,6 +182,8 @@ EpiParams forward_params(gsq_ctx* c, double* loss_out) {
 
 cudaError_t run_forward(gsq_ctx* c, double* loss_out, int epi) {
   EpiParams ep = forward_params(c, loss_out);
+  ep.stall_probe = c->stall_probe;
+  c->stall_probe = 0;
   return launch_gemm(c->tm_What, c->tm_Xb, c->em_forward, c->N, c->Tp, c->K,
                      epi, ep, c->sms,
                      c->st);
@@ -263,9 +269,12 @@ namespace {
 int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
               int x_dtype, int64_t N, int64_t K, int64_t T, int group,
               int grid_mode, const int8_t* init_idx, uint64_t seed,
-              void* stream, int state16) {
+              void* stream, int state16, int64_t row0 = 0) {
   if (!out) return GSQ_ERR_INVALID_ARG;
   *out = nullptr;
+  // the global coordinates row0 K .. (row0 + N) K must fit the 64-bit
+  // counter words
+  if (row0 < 0 || (K > 0 && row0 > (((int64_t)1 << 62) / K) - N)) return GSQ_ERR_INVALID_ARG;
   if (!W || !X || N <= 0 || K <= 0 || T <= 0 || group <= 0 ||
       (w_dtype != GSQ_F32 && w_dtype != GSQ_BF16) ||
       (x_dtype != GSQ_F32 && x_dtype != GSQ_BF16) || num_logits(grid_mode) < 0 ||
@@ -293,6 +302,7 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   c->Tp = (T + 63) / 64 * 64;
   c->G = K / kGroup;
   c->seed = seed;
+  c->coord0 = (uint64_t)row0 * (uint64_t)K;
   c->st = static_cast<cudaStream_t>(stream);
   c->dev = dev;
   c->sms = prop.multiProcessorCount;
@@ -447,6 +457,15 @@ int gsq_init_bf16_state(gsq_ctx** out, const void* W, int w_dtype, const void* X
                    stream, 1);
 }
 
+int gsq_init_rows(gsq_ctx** out, const void* W, int w_dtype, const void* X, int x_dtype,
+                  int64_t N, int64_t K, int64_t T, int group, int grid_mode,
+                  const int8_t* init_idx, uint64_t seed, int64_t row0, int state_bf16,
+                  void* stream) {
+  if (state_bf16 != 0 && state_bf16 != 1) return GSQ_ERR_INVALID_ARG;
+  return init_impl(out, W, w_dtype, X, x_dtype, N, K, T, group, grid_mode, init_idx, seed,
+                   stream, state_bf16, row0);
+}
+
 }  // extern "C"
 
 namespace {
@@ -467,19 +486,32 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
     tm = &c->tev[c->tev_used++];
     CK(cudaEventRecord(tm->ev[0], c->st));
   }
+  NvtxRange step_range("gsq_step");
   const bool soft = !(c->what_t == (int64_t)c->t && c->what_tau == tau);
-  if (soft) CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
+  if (soft) {
+    NvtxRange r("gsq_step/soft_weight");
+    CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
+  }
   if (tm) {
     tm->soft = soft;
     tm->next = tau_next > 0.f;
     CK(cudaEventRecord(tm->ev[1], c->st));
   }
-  CK(run_forward(c, c->loss_hist + (c->t % kLossRing), EPI_LOSS_DY));
+  {
+    NvtxRange r("gsq_step/forward_gemm");
+    CK(run_forward(c, c->loss_hist + (c->t % kLossRing), EPI_LOSS_DY));
+  }
   if (tm) CK(cudaEventRecord(tm->ev[2], c->st));
-  CK(run_weight_grad(c));
+  {
+    NvtxRange r("gsq_step/weight_grad_gemm");
+    CK(run_weight_grad(c));
+  }
   if (tm) CK(cudaEventRecord(tm->ev[3], c->st));
-  CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, tau_next,
-                          c->What, nullptr, nullptr, c->sms, c->st));
+  {
+    NvtxRange r(tau_next > 0.f ? "gsq_step/backward_lion_next_soft" : "gsq_step/backward_lion");
+    CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, tau_next, c->What, nullptr, nullptr,
+                            c->sms, c->st));
+  }
   if (tm) CK(cudaEventRecord(tm->ev[4], c->st));
   c->t += 1;
   c->hcode_valid = false;  // the logits moved
@@ -837,6 +869,13 @@ int gsq_debug_uniforms(gsq_ctx* c, uint32_t t, uint64_t coord0, int64_t count,
     e = cudaMemcpy(host_out, d, (size_t)count * c->L * 4, cudaMemcpyDeviceToHost);
   pool_free(d);
   if (e != cudaSuccess) return fail(c, cuda_status(e));
+  return GSQ_OK;
+}
+
+int gsq_debug_stall_probe(gsq_ctx* c) {
+  int u = usable(c);
+  if (u) return u;
+  c->stall_probe = 1;
   return GSQ_OK;
 }
 

@@ -35,6 +35,7 @@ using namespace gsq;
 
 struct gsq_attn {
   int mode = 0, L = 0;
+  PhaseClock clock;  // per-phase device time (gsq_attn_set_timing)
   int64_t nseq = 0, S = 0, nh = 0, nkv = 0, d = 0, grp = 0, T = 0, H = 0, Hk = 0;
   uint64_t t = 0;
   int noise = 1;
@@ -133,44 +134,63 @@ cudaError_t forward(gsq_attn* c, double* loss_out, bool with_dp) {
   const int64_t T = c->T, H = c->H, Hk = c->Hk, S = c->S;
   cudaError_t e;
   EpiParams ep = epi(c, loss_out);
+  PhaseClock& k = c->clock;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   if ((e = launch_gemm(c->w[0].tmA, c->tmB_Xa, c->em_VT, Hk, T, H, EPI_STORE_BF16, ep,
                        c->sms, c->st)) != cudaSuccess) return e;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   if ((e = launch_gemm_batched(c->tmA_P, c->tmB_VT, c->tm_o, c->grp * S, c->d, S, 128,
                                c->sc_pv, EPI_STORE_BF16, ep, c->sms, c->st)) != cudaSuccess)
     return e;
+  if ((e = k.mark(c->st, PH_ELEM)) != cudaSuccess) return e;
   if ((e = launch_transpose_bf16(c->o, T, H, c->oT, c->st)) != cudaSuccess) return e;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   return launch_gemm(c->w[1].tmA, c->tmB_o, c->em_pred, H, T, H,
                      with_dp ? EPI_LOSS_DY : EPI_LOSS, ep, c->sms, c->st);
 }
 
 int run_step(gsq_attn* c, float tau, float tau_next, float lr, float b1, float b2) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;
+  NvtxRange step_range("gsq_attn_step");
   const int64_t T = c->T, H = c->H, Hk = c->Hk, S = c->S;
+  PhaseClock& k = c->clock;
   if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 2; ++i) {
+      CKA(k.mark(c->st, PH_SOFT));
       CKA(launch_soft_weight(stage_weight_args(c->w[i], c->mode, c->t, c->noise, tau),
                              c->w[i].What, nullptr, c->sms, c->st));
+    }
   CKA(forward(c, c->loss_hist + (c->t % kStageLossRing), true));
   EpiParams ep = epi(c, nullptr);
   // dWo = dp^T . o
+  CKA(k.mark(c->st, PH_GEMM));
   CKA(launch_gemm(c->tmA_dpT, c->tmB_oT, c->w[1].em_dW, H, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
   // do^T = Wo^T . dp^T
+  CKA(k.mark(c->st, PH_ELEM));
   CKA(launch_transpose_bf16(c->w[1].What, H, H, c->WoT, c->st));
+  CKA(k.mark(c->st, PH_ELEM));
   CKA(launch_transpose_bf16(c->dpT, H, T, c->dp, c->st));
+  CKA(k.mark(c->st, PH_GEMM));
   CKA(launch_gemm(c->tmA_WoT, c->tmB_dp, c->em_doT, H, T, H, EPI_STORE_BF16, ep, c->sms,
                   c->st));
   // dV_(s,g) = P^T_(s,g) . do_(s, g's heads)
+  CKA(k.mark(c->st, PH_GEMM));
   CKA(launch_gemm_batched(c->tmA_PT, c->tmB_doT, c->tm_dV, S, c->d, c->grp * S, 128,
                           c->sc_dv, EPI_STORE_BF16, ep, c->sms, c->st));
   // dWv = dV^T . Xa
+  CKA(k.mark(c->st, PH_ELEM));
   CKA(launch_transpose_bf16(c->dVb, T, Hk, c->dVT, c->st));
+  CKA(k.mark(c->st, PH_GEMM));
   CKA(launch_gemm(c->tmA_dVT, c->tmB_XaT, c->w[0].em_dW, Hk, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 2; ++i) {
+    CKA(k.mark(c->st, PH_BACKWARD));
     CKA(launch_backward_lion(stage_weight_args(c->w[i], c->mode, c->t, c->noise, tau),
                              c->w[i].dW, lr, b1, b2, tau_next,
                              c->w[i].What, nullptr, nullptr, c->sms, c->st));
+  }
+  CKA(k.mark(c->st, -1));
   c->t += 1;
   if (tau_next > 0.f) {
     c->what_t = (int64_t)c->t;
@@ -607,7 +627,22 @@ int gsq_attn_destroy(gsq_attn* c) {
   cudaStreamSynchronize(c->st);
   cudaGetLastError();
   free_all(c);
+  c->clock.release();
   delete c;
+  return GSQ_OK;
+}
+
+int gsq_attn_set_timing(gsq_attn* c, int on) {
+  if (!c) return GSQ_ERR_INVALID_ARG;
+  if (c->failed) return GSQ_ERR_STATE;
+  c->clock.on = on != 0;
+  return GSQ_OK;
+}
+
+int gsq_attn_phase_times(gsq_attn* c, double* ms, int64_t* launches) {
+  if (!c || !ms || !launches) return GSQ_ERR_INVALID_ARG;
+  if (c->failed) return GSQ_ERR_STATE;
+  CKA(c->clock.collect(PH_COUNT, ms, launches));
   return GSQ_OK;
 }
 

@@ -35,6 +35,7 @@ constexpr int PM = 256, HALF = 128, BK = 64;
 constexpr int A_BYTES = HALF * BK * 2;
 constexpr int NUM_THREADS = 192;
 constexpr long long WAIT_LIMIT = 4000000000LL;  // clock cycles (~2 s)
+constexpr long long PROBE_LIMIT = 20000000LL;   // the test hook's wait (~10 ms)
 
 // Output tile width BN (256, or 128 for N = 128 problems): each CTA loads
 // BN / 2 rows of B per stage; two BN-column TMEM accumulators per CTA.
@@ -58,6 +59,7 @@ struct Ctl {
   uint64_t tempty[2];
   uint64_t done;
   uint64_t ybar[4][2];  // Y_ref tile loads of each epilogue warp
+  uint64_t probe;       // test hook: a barrier nothing arrives at
   uint32_t tmem_base;
   int abort;
   double red[4];
@@ -196,7 +198,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int m_tiles = (int)((M + PM - 1) / PM);
   const int n_tiles = (int)((N + PN - 1) / PN);
-  const int num_tiles = m_tiles * n_tiles * sc.count;
+  // the test hook's launch processes no tile: nothing is ever in flight
+  const int num_tiles = ep.stall_probe ? 0 : m_tiles * n_tiles * sc.count;
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0 && lane == 0) {
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&ctl->done), 1);
     for (int w = 0; w < 4; ++w)
       for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&ctl->ybar[w][b]), 1);
+    mbar_init(smem_u32(&ctl->probe), 1);
     ctl->abort = 0;
     mbar_fence_init();
     if (EPI != EPI_LOSS) tma_prefetch_desc(&tmO);
@@ -230,6 +234,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // the setup above overlapped the previous kernel's tail; its outputs (our
   // operands) and its reads of what we write are complete after this
   pdl_wait();
+  if (ep.stall_probe && threadIdx.x == 0) {
+    // a bounded wait that runs out: the error word reports it
+    if (!mbar_wait_bounded(smem_u32(&ctl->probe), 0, PROBE_LIMIT))
+      atomicCAS(ep.err, 0, DEV_ERR_TIMEOUT);
+  }
 
   if (warp == 0) {
     if (lane == 0) {

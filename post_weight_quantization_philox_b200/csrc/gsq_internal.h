@@ -2,12 +2,24 @@
 #pragma once
 
 #include <atomic>
+#include <vector>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace gsq {
+
+// NVTX range around the host-side issue of a step or phase (names such as
+// "gsq_step/backward"), so a profiler's timeline shows where each step's
+// kernels come from; inert when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // device-side error codes written into the context's error word
 enum : int {
@@ -30,6 +42,10 @@ struct EpiParams {
   unsigned* ticket;      // zero between launches
   double* loss_out;      // final loss (fp64)
   int* err;              // device error word
+  // test hook: before any load or MMA is issued, one thread per CTA waits
+  // (bounded, about 10 ms) on a barrier nothing arrives at, records
+  // DEV_ERR_TIMEOUT, and the CTA then processes no tile
+  int stall_probe = 0;
 };
 
 // The epilogue's tensor maps: out = C (EPI_STORE_F32, fp32 map; EPI_STORE_BF16,
@@ -39,6 +55,60 @@ struct EpiMaps {
   CUtensorMap out;
   CUtensorMap yref;
 };
+
+// Per-phase device time of a block stage's steps: when on, an event is
+// recorded on the stage's stream before each launch, tagged with the phase
+// of that launch, and one tagged -1 after the step's last launch; the time
+// between an event and the next is the tagged launch's.  collect() syncs,
+// sums milliseconds and launches per phase, and starts over.  (The events
+// keep each kernel from starting before the previous one ends, so timings
+// come from a separate run of the same steps.)
+struct PhaseClock {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> tag;
+  size_t used = 0;
+  cudaError_t mark(cudaStream_t st, int phase) {
+    if (!on) return cudaSuccess;
+    if (used == ev.size()) {
+      cudaEvent_t e;
+      const cudaError_t r = cudaEventCreate(&e);
+      if (r != cudaSuccess) return r;
+      ev.push_back(e);
+      tag.push_back(-1);
+    }
+    tag[used] = phase;
+    return cudaEventRecord(ev[used++], st);
+  }
+  cudaError_t collect(int nphase, double* ms, int64_t* launches) {
+    for (int i = 0; i < nphase; ++i) {
+      ms[i] = 0.0;
+      launches[i] = 0;
+    }
+    if (used > 0) {
+      const cudaError_t r = cudaEventSynchronize(ev[used - 1]);
+      if (r != cudaSuccess) return r;
+    }
+    for (size_t i = 0; i + 1 < used; ++i) {
+      if (tag[i] < 0 || tag[i] >= nphase) continue;
+      float t = 0.f;
+      const cudaError_t r = cudaEventElapsedTime(&t, ev[i], ev[i + 1]);
+      if (r != cudaSuccess) return r;
+      ms[tag[i]] += t;
+      launches[tag[i]] += 1;
+    }
+    used = 0;
+    return cudaSuccess;
+  }
+  void release() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    ev.clear();
+    tag.clear();
+    used = 0;
+  }
+};
+// phases of a block stage's step
+enum : int { PH_SOFT = 0, PH_GEMM = 1, PH_ELEM = 2, PH_BACKWARD = 3, PH_COUNT = 4 };
 
 // Opts kernel Fn in to `bytes` of dynamic shared memory on the current device,
 // once per device (the attribute is per device; a process may drive several).
@@ -54,6 +124,9 @@ inline cudaError_t smem_optin(int bytes) {
   if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
   return e;
 }
+
+// Pool test hook (gsq_debug_fail_alloc): true when this allocation is to fail.
+bool pool_fail_injected();
 
 // Device memory of the library (gsq_pool.cu): one pool per device that keeps
 // freed memory reserved for the next allocation.  pool_malloc behaves as
@@ -157,6 +230,10 @@ struct StepArgs {
   uint32_t t;
   int noise;
   float tau;
+  // global coordinate of local coordinate 0 (row0 K for a shard of rows
+  // [row0, row0 + N) of a larger layer): the Philox counters take global
+  // coordinates, so a shard draws the noise the whole layer would
+  uint64_t coord0 = 0;
 };
 
 cudaError_t launch_convert_x(const void* X, int dtype, int64_t T, int64_t K,

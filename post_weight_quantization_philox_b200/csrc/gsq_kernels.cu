@@ -284,7 +284,7 @@ template <int MODE, bool DBG, typename TS>
 __global__ void __launch_bounds__(256) k_soft_weight(
     const TS* __restrict__ logits, const float* __restrict__ s,
     const int8_t* __restrict__ i0, int64_t N, int64_t K, const PhiloxKeys ks,
-    uint32_t t, int noise, float inv_tau, __nv_bfloat16* __restrict__ What,
+    uint64_t coord0, uint32_t t, int noise, float inv_tau, __nv_bfloat16* __restrict__ What,
     float* __restrict__ wsoft32) {
   constexpr int L = GridT<MODE>::L;
   const int64_t NK = N * K, G = K / kGroup;
@@ -310,13 +310,15 @@ __global__ void __launch_bounds__(256) k_soft_weight(
 #pragma unroll
       for (int j = 0; j < 4; ++j) levj[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
+    // Philox counters take the global coordinate (a multiple of 4 here)
+    const uint64_t gc0 = coord0 + (uint64_t)c0;
     uint32_t q1[4] = {0u, 0u, 0u, 0u};
-    if (L == 5 && noise) block1_words((uint64_t)c0, t, ks, q1);
+    if (L == 5 && noise) block1_words(gc0, t, ks, q1);
     float w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
-      if (noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t, ks, wd);
+      if (noise) block0_words(gc0 + j, (uint32_t)(gc0 >> 32), t, ks, wd);
       wd[4] = q1[j];
       float cand[5], e[L], r;
       candidates<MODE>(levj[j], cand);
@@ -367,8 +369,8 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     k_backward_lion(TS* __restrict__ logits, TS* __restrict__ mom,
                     float* __restrict__ s, float* __restrict__ ms,
                     const int8_t* __restrict__ i0, const float* __restrict__ dW,
-                    int64_t N, int64_t K, const PhiloxKeys ks, uint32_t t, int noise,
-                    float inv_tau, float inv_tau_next, float lr, float b1, float omb1,
+                    int64_t N, int64_t K, const PhiloxKeys ks, uint64_t coord0, uint32_t t,
+                    int noise, float inv_tau, float inv_tau_next, float lr, float b1, float omb1,
                     float b2, float omb2, __nv_bfloat16* __restrict__ What,
                     float* __restrict__ dl_dbg, float* __restrict__ ds_dbg) {
   using C = BwdCfg<MODE, TS>;
@@ -451,15 +453,16 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
       for (int j = 0; j < 4; ++j) lev[j] = (int)(int8_t)((b4 >> (8 * j)) & 0xFFu);
     }
     // pass 1: this step's probabilities (pre-update logits, words of step t),
-    // gradients and Lion
+    // gradients and Lion.  Philox counters take the global coordinate.
+    const uint64_t gc0 = coord0 + (uint64_t)c0;
     uint32_t q1[4] = {0u, 0u, 0u, 0u};
-    if (L == 5 && noise) block1_words((uint64_t)c0, t, ks, q1);
+    if (L == 5 && noise) block1_words(gc0, t, ks, q1);
     float ds_part = 0.f;
     float Do[DBG ? L : 1][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
-      if (noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t, ks, wd);
+      if (noise) block0_words(gc0 + j, (uint32_t)(gc0 >> 32), t, ks, wd);
       wd[4] = q1[j];
       // e: unnormalised e_k (categorical) or the probabilities (ternary)
       float l[L], e[L], cand[5], r;
@@ -537,12 +540,12 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
     // step's noise
     if (NEXT || S16) {
       uint32_t r1[4] = {0u, 0u, 0u, 0u};
-      if (L == 5 && (S16 || noise)) block1_words((uint64_t)c0, t1, ks, r1);
+      if (L == 5 && (S16 || noise)) block1_words(gc0, t1, ks, r1);
       float w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t wd[5] = {0u, 0u, 0u, 0u, 0u};
-        if (S16 || noise) block0_words((uint64_t)(c0 + j), (uint32_t)((uint64_t)c0 >> 32), t1, ks, wd);
+        if (S16 || noise) block0_words(gc0 + j, (uint32_t)(gc0 >> 32), t1, ks, wd);
         wd[4] = r1[j];
         float l[L];
 #pragma unroll
@@ -1104,12 +1107,12 @@ static void soft_weight_ts(const StepArgs& a, __nv_bfloat16* What, float* wsoft3
   const TS* lg = reinterpret_cast<const TS*>(a.logits);
   if (wsoft32)
     k_soft_weight<MODE, true, TS><<<blocks, 256, 0, st>>>(lg, a.s, a.i0, a.N, a.K,
-                                                          philox_keys(k0, k1), a.t, a.noise,
-                                                          inv_tau, What, wsoft32);
+                                                          philox_keys(k0, k1), a.coord0, a.t,
+                                                          a.noise, inv_tau, What, wsoft32);
   else
     k_soft_weight<MODE, false, TS><<<blocks, 256, 0, st>>>(lg, a.s, a.i0, a.N, a.K,
-                                                           philox_keys(k0, k1), a.t, a.noise,
-                                                           inv_tau, What, nullptr);
+                                                           philox_keys(k0, k1), a.coord0, a.t,
+                                                           a.noise, inv_tau, What, nullptr);
 }
 
 template <int MODE>
@@ -1161,12 +1164,12 @@ static void backward_mode(const StepArgs& a, const float* dW, float lr, float b1
   if (dl_dbg) {
     smem_optin<k_backward_lion<MODE, true, NEXT, TS>>(C::SMEM);
     cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, true, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
-                       dW, a.N, a.K, philox_keys(k0, k1), a.t, a.noise, inv_tau,
+                       dW, a.N, a.K, philox_keys(k0, k1), a.coord0, a.t, a.noise, inv_tau,
                        inv_tau_next, lr, b1, omb1, b2, omb2, What, dl_dbg, ds_dbg);
   } else {
     smem_optin<k_backward_lion<MODE, false, NEXT, TS>>(C::SMEM);
     cudaLaunchKernelEx(&cfg, k_backward_lion<MODE, false, NEXT, TS>, lg, mm, a.s, a.ms, a.i0,
-                       dW, a.N, a.K, philox_keys(k0, k1), a.t, a.noise, inv_tau,
+                       dW, a.N, a.K, philox_keys(k0, k1), a.coord0, a.t, a.noise, inv_tau,
                        inv_tau_next, lr, b1, omb1, b2, omb2, What, (float*)nullptr,
                        (float*)nullptr);
   }

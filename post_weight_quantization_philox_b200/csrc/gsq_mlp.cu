@@ -46,6 +46,7 @@ struct Weight {
 
 struct gsq_mlp {
   int mode = 0, L = 0;
+  PhaseClock clock;  // per-phase device time (gsq_mlp_set_timing)
   int64_t T = 0, H = 0, F = 0;
   uint64_t t = 0;
   int noise = 1;
@@ -170,13 +171,19 @@ cudaError_t forward(gsq_mlp* c, double* loss_out, bool with_dp) {
   const int64_t T = c->T, H = c->H, F = c->F;
   cudaError_t e;
   EpiParams ep = epi(c, loss_out);
+  PhaseClock& k = c->clock;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   if ((e = launch_gemm(c->w[0].tmA, c->tmB_Xn, c->em_aT, F, T, H, EPI_STORE_F32, ep,
                        c->sms, c->st)) != cudaSuccess) return e;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   if ((e = launch_gemm(c->w[1].tmA, c->tmB_Xn, c->em_bT, F, T, H, EPI_STORE_F32, ep,
                        c->sms, c->st)) != cudaSuccess) return e;
+  if ((e = k.mark(c->st, PH_ELEM)) != cudaSuccess) return e;
   if ((e = launch_swiglu_fwd(c->aT, c->bT, F * T, c->hT, c->sms, c->st)) != cudaSuccess)
     return e;
+  if ((e = k.mark(c->st, PH_ELEM)) != cudaSuccess) return e;
   if ((e = launch_transpose_bf16(c->hT, F, T, c->h, c->st)) != cudaSuccess) return e;
+  if ((e = k.mark(c->st, PH_GEMM)) != cudaSuccess) return e;
   return launch_gemm(c->w[2].tmA, c->tmB_h, c->em_pred, H, T, F,
                      with_dp ? EPI_LOSS_DY : EPI_LOSS, ep, c->sms, c->st);
 }
@@ -188,31 +195,45 @@ bool step_args_ok(float tau, float lr, float b1, float b2) {
 
 int run_step(gsq_mlp* c, float tau, float tau_next, float lr, float b1, float b2) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;
+  NvtxRange step_range("gsq_mlp_step");
   const int64_t T = c->T, H = c->H, F = c->F;
+  PhaseClock& k = c->clock;
   if (!(c->what_t == (int64_t)c->t && c->what_tau == tau))
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 3; ++i) {
+      CKM(k.mark(c->st, PH_SOFT));
       CKM(launch_soft_weight(weight_args(c, i, tau), c->w[i].What, nullptr, c->sms,
                              c->st));
+    }
   CKM(forward(c, c->loss_hist + (c->t % kLossRing), true));
   EpiParams ep = epi(c, nullptr);
   // dD = dp^T . (h^T)^T
+  CKM(k.mark(c->st, PH_GEMM));
   CKM(launch_gemm(c->tmA_dpT, c->tmB_hT, c->w[2].em_dW, H, F, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
   // dh^T = D^T . dp^T  (transposed copies of D and dp^T)
+  CKM(k.mark(c->st, PH_ELEM));
   CKM(launch_transpose_bf16(c->w[2].What, H, F, c->WdT, c->st));
+  CKM(k.mark(c->st, PH_ELEM));
   CKM(launch_transpose_bf16(c->dpT, H, T, c->dp, c->st));
+  CKM(k.mark(c->st, PH_GEMM));
   CKM(launch_gemm(c->tmA_WdT, c->tmB_dp, c->em_dhT, F, T, H, EPI_STORE_F32, ep,
                   c->sms, c->st));
+  CKM(k.mark(c->st, PH_ELEM));
   CKM(launch_swiglu_bwd(c->aT, c->bT, c->dhT, F * T, c->daT, c->dbT, c->sms, c->st));
   // dG = da^T . Xn, dU = db^T . Xn
+  CKM(k.mark(c->st, PH_GEMM));
   CKM(launch_gemm(c->tmA_daT, c->tmB_XnT, c->w[0].em_dW, F, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
+  CKM(k.mark(c->st, PH_GEMM));
   CKM(launch_gemm(c->tmA_dbT, c->tmB_XnT, c->w[1].em_dW, F, H, T, EPI_STORE_F32, ep,
                   c->sms, c->st));
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 3; ++i) {
+    CKM(k.mark(c->st, PH_BACKWARD));
     CKM(launch_backward_lion(weight_args(c, i, tau), c->w[i].dW, lr, b1,
                              b2, tau_next, c->w[i].What, nullptr, nullptr, c->sms,
                              c->st));
+  }
+  CKM(k.mark(c->st, -1));
   c->t += 1;
   if (tau_next > 0.f) {
     c->what_t = (int64_t)c->t;
@@ -570,8 +591,23 @@ int gsq_mlp_destroy(gsq_mlp* c) {
   if (!c) return GSQ_OK;
   cudaStreamSynchronize(c->st);
   cudaGetLastError();
+  c->clock.release();
   free_all(c);
   delete c;
+  return GSQ_OK;
+}
+
+int gsq_mlp_set_timing(gsq_mlp* c, int on) {
+  if (!c) return GSQ_ERR_INVALID_ARG;
+  if (c->failed) return GSQ_ERR_STATE;
+  c->clock.on = on != 0;
+  return GSQ_OK;
+}
+
+int gsq_mlp_phase_times(gsq_mlp* c, double* ms, int64_t* launches) {
+  if (!c || !ms || !launches) return GSQ_ERR_INVALID_ARG;
+  if (c->failed) return GSQ_ERR_STATE;
+  CKM(c->clock.collect(PH_COUNT, ms, launches));
   return GSQ_OK;
 }
 

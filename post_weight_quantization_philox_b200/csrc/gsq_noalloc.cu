@@ -25,10 +25,29 @@ static __device__ __align__(256) float g_uniform_scratch[kScratchFloats];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 float* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+// The calling thread's current driver context (null if it cannot be read).
+CUcontext current_context() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return (CtxGetCurrentFn) nullptr;
+  }();
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, with that device current: once per device, and again
+// whenever the device's context is no longer the one the address was taken
+// in (after cudaDeviceReset the old address is gone).
 int scratch_address(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -36,14 +55,18 @@ int scratch_address(float** out) {
     return GSQ_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return GSQ_ERR_UNSUPPORTED;
+  // null until the runtime has made the device's context current; the
+  // lookup below does that, and the context is read again after it
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_uniform_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
       return GSQ_ERR_CUDA;
     }
     g_scratch_ptr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = ctx ? ctx : current_context();
   }
   *out = g_scratch_ptr[dev];
   return GSQ_OK;

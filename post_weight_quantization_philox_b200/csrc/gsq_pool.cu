@@ -13,6 +13,7 @@
 // waits for that stream.  pool_free has cudaFree's (nothing in flight still
 // uses the memory): it frees on the same private stream, so a later
 // pool_malloc reuses the memory in stream order.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/gsq.h"
@@ -26,6 +27,8 @@ constexpr int kMaxDevices = 64;
 
 std::mutex g_mu;
 uint64_t g_keep = ~0ull;  // release threshold of every pool
+// test hook: allocations left before one fails (negative: none fails)
+std::atomic<int64_t> g_fail_after{-1};
 cudaMemPool_t g_pool[kMaxDevices] = {};
 cudaStream_t g_stream[kMaxDevices] = {};
 
@@ -73,6 +76,14 @@ bool device_pool(int dev, cudaMemPool_t* pool, cudaStream_t* stream) {
 
 }  // namespace
 
+bool pool_fail_injected() {
+  int64_t n = g_fail_after.load();
+  while (n >= 0) {
+    if (g_fail_after.compare_exchange_weak(n, n - 1)) return n == 0;
+  }
+  return false;
+}
+
 cudaMemPool_t library_pool(int dev) {
   cudaMemPool_t p = nullptr;
   cudaStream_t s = nullptr;
@@ -81,6 +92,7 @@ cudaMemPool_t library_pool(int dev) {
 
 cudaError_t pool_malloc(void** p, size_t bytes) {
   *p = nullptr;
+  if (pool_fail_injected()) return cudaErrorMemoryAllocation;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -128,6 +140,34 @@ int gsq_set_cached_memory_limit(uint64_t bytes) {
     }
   }
   return rc;
+}
+
+int gsq_debug_fail_alloc(int64_t after) {
+  gsq::g_fail_after.store(after < 0 ? -1 : after);
+  return GSQ_OK;
+}
+
+int gsq_debug_pool_used(int device, uint64_t* bytes) {
+  using namespace gsq;
+  if (!bytes || device < 0 || device >= kMaxDevices) return GSQ_ERR_INVALID_ARG;
+  *bytes = 0;
+  cudaMemPool_t pool = nullptr;
+  cudaStream_t s = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    pool = g_pool[device];
+    s = g_stream[device];
+  }
+  if (!pool) return GSQ_OK;  // nothing allocated on that device yet
+  uint64_t used = 0;
+  // frees queued on the private stream are done before the count is read
+  if ((s && cudaStreamSynchronize(s) != cudaSuccess) ||
+      cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemCurrent, &used) != cudaSuccess) {
+    cudaGetLastError();
+    return GSQ_ERR_CUDA;
+  }
+  *bytes = used;
+  return GSQ_OK;
 }
 
 int gsq_release_cached_memory(void) {

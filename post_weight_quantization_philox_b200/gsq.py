@@ -45,6 +45,8 @@ EXPORTS = [
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
     "gsq_gptq", "gsq_release_cached_memory", "gsq_set_cached_memory_limit", "gsq_init_gptq", "gsq_init_bf16_state",
+    "gsq_init_rows", "gsq_mlp_set_timing", "gsq_mlp_phase_times", "gsq_attn_set_timing",
+    "gsq_attn_phase_times", "gsq_debug_stall_probe", "gsq_debug_fail_alloc", "gsq_debug_pool_used",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
     "gsq_mlp_debug_set", "gsq_mlp_get_step", "gsq_mlp_destroy",
@@ -71,6 +73,15 @@ _pp = C.POINTER(C.c_void_p)
 
 _SIGS = {
     "gsq_init": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64, _p],
+    "gsq_debug_stall_probe": [_p],
+    "gsq_mlp_set_timing": [_p, _i32],
+    "gsq_mlp_phase_times": [_p, _p, _p],
+    "gsq_attn_set_timing": [_p, _i32],
+    "gsq_attn_phase_times": [_p, _p, _p],
+    "gsq_debug_fail_alloc": [_i64],
+    "gsq_debug_pool_used": [_i32, C.POINTER(_u64)],
+    "gsq_init_rows": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64, _i64,
+                      _i32, _p],
     "gsq_step": [_p, _f32, _f32, _f32, _f32],
     "gsq_run": [_p, _p, _i64, _f32, _f32, _f32],
     "gsq_last_loss": [_p, C.POINTER(C.c_double)],
@@ -228,9 +239,12 @@ def gsq_packed_bytes(grid_mode: int, N: int, K: int) -> int:
 
 
 def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
-             init_idx=None, seed: int = 0, stream=None, state_bf16: bool = False) -> "Layer":
+             init_idx=None, seed: int = 0, stream=None, state_bf16: bool = False,
+             row0=None) -> "Layer":
     """W (N x K) and X (T x K): numpy fp32 or torch fp32/bf16, host or device.
-    state_bf16 selects gsq_init_bf16_state (bf16 logits and momenta)."""
+    state_bf16 selects gsq_init_bf16_state (bf16 logits and momenta).  With
+    row0, W holds the rows [row0, row0 + N) of a larger layer
+    (gsq_init_rows: the noise is keyed by the global coordinate)."""
     wp, wdt, wk = _ptr_dtype(W)
     xp, xdt, xk = _ptr_dtype(X)
     N, K = int(W.shape[0]), int(W.shape[1])
@@ -251,10 +265,15 @@ def gsq_init(W, X, group: int = 128, grid_mode: int = GSQ_GRID_2BIT,
             ip = ik.ctypes.data
     ctx = C.c_void_p()
     st = _stream_ptr(stream)
-    fn = _lib.gsq_init_bf16_state if state_bf16 else _lib.gsq_init
-    _check(fn(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group,
-              grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
-           "gsq_init_bf16_state" if state_bf16 else "gsq_init")
+    if row0 is not None:
+        _check(_lib.gsq_init_rows(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group, grid_mode,
+                                  ip, seed & 0xFFFFFFFFFFFFFFFF, int(row0), int(bool(state_bf16)),
+                                  st), "gsq_init_rows")
+    else:
+        fn = _lib.gsq_init_bf16_state if state_bf16 else _lib.gsq_init
+        _check(fn(C.byref(ctx), wp, wdt, xp, xdt, N, K, T, group,
+                  grid_mode, ip, seed & 0xFFFFFFFFFFFFFFFF, st),
+               "gsq_init_bf16_state" if state_bf16 else "gsq_init")
     del wk, xk, ik
     return Layer(ctx, grid_mode, N, K, T, group, state16=state_bf16)
 
@@ -549,6 +568,18 @@ class Mlp:
         _check(_lib.gsq_mlp_run(self.ctx, t.ctypes.data, t.size, lr, beta1, beta2),
                "gsq_mlp_run")
 
+    def set_timing(self, on: bool) -> None:
+        _check(_lib.gsq_mlp_set_timing(self.ctx, int(bool(on))), "gsq_mlp_set_timing")
+
+    def phase_times(self):
+        """(ms[4], launches[4]) of soft weights, GEMMs, elementwise, backward
+        since the last call (syncs)."""
+        ms = np.zeros(4, np.float64)
+        n = np.zeros(4, np.int64)
+        _check(_lib.gsq_mlp_phase_times(self.ctx, ms.ctypes.data, n.ctypes.data),
+               "gsq_mlp_phase_times")
+        return ms, n
+
     def last_loss(self):
         v = C.c_double()
         _check(_lib.gsq_mlp_last_loss(self.ctx, C.byref(v)), "gsq_mlp_last_loss")
@@ -655,6 +686,18 @@ class Attn:
         t = np.ascontiguousarray(taus, dtype=np.float32).ravel()
         _check(_lib.gsq_attn_run(self.ctx, t.ctypes.data, t.size, lr, beta1, beta2),
                "gsq_attn_run")
+
+    def set_timing(self, on: bool) -> None:
+        _check(_lib.gsq_attn_set_timing(self.ctx, int(bool(on))), "gsq_attn_set_timing")
+
+    def phase_times(self):
+        """(ms[4], launches[4]) of soft weights, GEMMs, elementwise, backward
+        since the last call (syncs)."""
+        ms = np.zeros(4, np.float64)
+        n = np.zeros(4, np.int64)
+        _check(_lib.gsq_attn_phase_times(self.ctx, ms.ctypes.data, n.ctypes.data),
+               "gsq_attn_phase_times")
+        return ms, n
 
     def last_loss(self):
         v = C.c_double()
@@ -803,26 +846,31 @@ def gsq_block_forward(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn,
 
 def gsq_block_quantize(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn, taus,
                        lr, beta1=0.9, beta2=0.99, seed=0, grid_mode=GSQ_GRID_2BIT,
-                       group=128, rope_theta=500000.0, rms_eps=1e-5, stream=None):
+                       group=128, rope_theta=500000.0, rms_eps=1e-5, stream=None,
+                       host_outputs=False):
     """GSQ's staged reconstruction of one block (Q, K, then V/O, then the MLP
     on the block output).  taus: four temperature schedules (one per stage).
-    Returns a dict: x_out (device fp32, the next block's input), packed and
-    scales_f32 per weight (device tensors), stats per stage (first loss, last
-    loss, hard abs / rel error, ms)."""
+    Returns a dict: x_out (fp32, the next block's input), packed and
+    scales_f32 per weight, stats per stage (first loss, last loss, hard abs /
+    rel error, ms).  Outputs are device tensors, or pinned host tensors with
+    host_outputs (the library writes them through unified addressing)."""
     import torch
     x = _f32_tensor(x)
     _block_shapes_ok(x, W, n_seq, seq_len, n_heads, n_kv_heads, head_dim, ffn)
     keep, arr = _bf16_weights(W)
     T, H = int(x.shape[0]), int(x.shape[1])
     dev = x.device if x.is_cuda else torch.device("cuda")
+    if host_outputs:
+        dev = torch.device("cpu")
     shapes = block_weight_shapes(n_heads, n_kv_heads, head_dim, ffn)
-    x_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    pin = dict(pin_memory=True) if host_outputs else {}
+    x_out = torch.empty((T, H), dtype=torch.float32, device=dev, **pin)
     packed, scales = {}, {}
     for name in BLOCK_WEIGHTS:
         N, K = shapes[name]
         packed[name] = torch.empty(gsq_packed_bytes(grid_mode, N, K) // 4, dtype=torch.int32,
-                                   device=dev)
-        scales[name] = torch.empty((N, K // group), dtype=torch.float32, device=dev)
+                                   device=dev, **pin)
+        scales[name] = torch.empty((N, K // group), dtype=torch.float32, device=dev, **pin)
     tau_arr = [np.ascontiguousarray(t, np.float32) for t in taus]
     if len(tau_arr) != 4:
         raise ValueError("taus: one schedule per stage (4)")

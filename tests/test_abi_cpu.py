@@ -104,3 +104,27 @@ def test_binding_has_no_fallback(monkeypatch, tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_failure_hooks_are_host_only(gsq):
+    """The allocation-failure hook and the pool query need no device until
+    the library has allocated on one."""
+    lib = gsq.lib()
+    assert lib.gsq_debug_fail_alloc(3) == gsq.GSQ_OK
+    assert lib.gsq_debug_fail_alloc(-1) == gsq.GSQ_OK
+    b = C.c_uint64(7)
+    assert lib.gsq_debug_pool_used(0, C.byref(b)) == gsq.GSQ_OK and b.value == 0
+    assert lib.gsq_debug_pool_used(-1, C.byref(b)) == gsq.GSQ_ERR_INVALID_ARG
+    assert lib.gsq_debug_pool_used(0, None) == gsq.GSQ_ERR_INVALID_ARG
+    assert lib.gsq_debug_stall_probe(None) == gsq.GSQ_ERR_INVALID_ARG
+
+
+def test_row_shard_init_rejects_bad_offsets_on_host(gsq):
+    import numpy as np
+    W = np.zeros((8, 256), np.float32)
+    X = np.zeros((4, 256), np.float32)
+    for row0, st16 in [(-1, 0), (0, 2), (1 << 60, 0)]:
+        out = C.c_void_p()
+        rc = gsq.lib().gsq_init_rows(C.byref(out), W.ctypes.data, gsq.GSQ_F32, X.ctypes.data,
+                                     gsq.GSQ_F32, 8, 256, 4, 128, 0, None, 0, row0, st16, None)
+        assert rc == gsq.GSQ_ERR_INVALID_ARG and not out.value

@@ -56,3 +56,20 @@ def test_step_roofline_q_proj():
     assert r["frac"] == pytest.approx((gemm_ms + hbm_ms) / 0.5, abs=1e-4)
     # the whole-job rate counts every rank's units over the slowest rank's time
     assert bench.whole_job_rate(4, 10.0, 2.0) == pytest.approx(4 * 10.0 / 2e-3)
+
+
+def test_block_step_accounting():
+    """The 70B block step: seven weights, 8.55e8 coordinates per step; the
+    fused backward's algorithmic bytes are 70 B per coordinate (2-bit, with
+    the next soft weight) plus 16 B per group; the GEMM flops per stage."""
+    dm = bench.BLOCK_70B
+    dims = (dm["nseq"], dm["S"], dm["nh"], dm["nkv"], dm["d"], dm["F"])
+    c = bench.block_step_coords(*dims)
+    assert c == [8192 * 8192, 1024 * 8192, 1024 * 8192 + 8192 * 8192, 3 * 8192 * 28672]
+    assert sum(c) == 855638016
+    assert bench.block_backward_bytes(128) == 128 * 70 + 16
+    assert bench.block_backward_bytes(128, next_soft=False) == 128 * 68 + 16
+    f = bench.block_step_flops(*dims)
+    T = 8 * 2048
+    assert f[0] == 4.0 * T * 8192 * 8192 and f[1] == 4.0 * T * 1024 * 8192
+    assert f[3] == 14.0 * T * 8192 * 28672

@@ -188,8 +188,25 @@ def test_full_70b_shape(g, oracle_mod):
     s_chk = 5
     Ps = bits_to_f32(P[s_chk]).astype(np.float64)  # nh x S x S
     del P
+
+    def prefix_loss_vs_oracle(n=64):
+        """The step's loss over the first n tokens of sequence s_chk from the
+        GPU's output gradient, against the oracle's V/O forward of that prefix
+        with the GPU's probabilities and soft weights of the step (causal: the
+        prefix's outputs need no later token)."""
+        dpt = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_DPT)).astype(np.float64)
+        gpu_tok = ((dpt / 2.0) ** 2).sum(0)
+        assert gpu_tok.sum() == pytest.approx(a.last_loss(), rel=1e-2)
+        lo = s_chk * S
+        Wv_h = bits_to_f32(a.get(0, g.GSQ_DBG_WHAT))
+        Wo_h = bits_to_f32(a.get(1, g.GSQ_DBG_WHAT))
+        Pp = np.ascontiguousarray(Ps[None, :, :n, :n], np.float32)
+        ref = oracle_mod.attn_vo_forward_backward(Xa[lo:lo + n], Pp, R[lo:lo + n], Wv_h, Wo_h,
+                                                  1, n, nh, nkv, d)[0]
+        assert gpu_tok[lo:lo + n].sum() == pytest.approx(ref, rel=1e-2)
+
     a.step(1.0, 1e-3)
-    assert np.isfinite(a.last_loss()) and a.last_loss() > 0
+    prefix_loss_vs_oracle()
     rows = slice(s_chk * S, (s_chk + 1) * S)
     VT = bits_to_f32(a.get(g.GSQ_ATTN_STAGE, g.GSQ_ATTN_DBG_VT)).astype(np.float64)  # Hk x T
     Wv_hat = bits_to_f32(a.get(0, g.GSQ_DBG_WHAT)).astype(np.float64)
@@ -224,5 +241,5 @@ def test_full_70b_shape(g, oracle_mod):
         assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref) + 1e-12, key
     taus = synth.tau_schedule(1.0, 0.05, cfg["steps"])
     a.run(taus[1:3], 1e-3)
-    assert np.isfinite(a.last_loss()) and a.last_loss() > 0
+    prefix_loss_vs_oracle()
     a.close()

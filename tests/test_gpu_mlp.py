@@ -122,9 +122,24 @@ def test_mlp_run_equals_step_loop_bit_exact(g):
     a.close(); b.close()
 
 
+def token_losses_vs_oracle(g, oracle_mod, m, Xn, R, tokens):
+    """The step's loss per token from the GPU's output gradient (bf16 of
+    2 (pred - R), H x T) against the oracle's MLP forward of that token with
+    the GPU's own soft weights of the step (the loss is a sum over tokens)."""
+    dpt = bits_to_f32(m.get(g.GSQ_MLP_STAGE, g.GSQ_MLP_DBG_DPT)).astype(np.float64)
+    gpu = ((dpt / 2.0) ** 2).sum(0)
+    assert gpu.sum() == pytest.approx(m.last_loss(), rel=1e-2)
+    Wh = [bits_to_f32(m.get(i, g.GSQ_DBG_WHAT)) for i in range(3)]
+    for t in tokens:
+        ref = oracle_mod.mlp_forward_backward(Xn[t:t + 1], R[t:t + 1], *Wh)[0]
+        assert gpu[t] == pytest.approx(ref, rel=1e-2), t
+
+
 def test_mlp_full_70b_shape(g, oracle_mod):
     """The 70B block MLP (H 8192, F 28672) on 8 x 2048 tokens in the bench's
-    launch configuration: GEMM identities on sampled entries, finite losses."""
+    launch configuration: GEMM identities on sampled entries; each step's loss
+    on sampled tokens against the oracle, after the first step and after a
+    fused run."""
     import torch
     cfg = synth.MLP_STAGE["c5_70b_mlp"]
     T, H, F = cfg["T"], cfg["H"], cfg["F"]
@@ -134,8 +149,10 @@ def test_mlp_full_70b_shape(g, oracle_mod):
     m = g.gsq_mlp_init(dev(Xn), torch.from_numpy(R).cuda(), dev(Wg), dev(Wu), dev(Wd),
                        grid_mode=cfg["grid"], seed=0)
     taus = synth.tau_schedule(1.0, 0.05, cfg["steps"])
-    m.run(taus[:2], 1e-3)
-    assert np.isfinite(m.last_loss()) and m.last_loss() > 0
+    m.step(float(taus[0]), 1e-3)
+    token_losses_vs_oracle(g, oracle_mod, m, Xn, R, [0, 5000, T - 1])
+    m.run(taus[1:3], 1e-3)
+    token_losses_vs_oracle(g, oracle_mod, m, Xn, R, [1, 12345])
     rng = np.random.default_rng(0)
     for i in range(3):
         assert np.isfinite(bits_to_f32(m.get(i, g.GSQ_DBG_WHAT))).all()

@@ -127,6 +127,62 @@ def test_nonfinite_input_is_reported(g):
     assert e.value.status == g.GSQ_ERR_NONFINITE
 
 
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("state16", [False, True])
+def test_row_shards_equal_whole_layer(g, oracle_mod, mode, state16):
+    """gsq_init_rows: the shards [0, 256) and [256, 456) of a layer, each
+    keyed by its global row offset, follow the whole layer's trajectory bit
+    for bit (every output row of the GEMMs is the same dot products in the
+    same order whatever the row tile), and their losses add up to the
+    layer's; the shard's noise equals the oracle's at the global coordinates."""
+    import torch
+    N, K, T = 456, 640, 200
+    cfg, W, X = make_case(mode, N, K, T)
+    Xd = torch.from_numpy(X).cuda()
+    full = g.gsq_init(torch.from_numpy(W).cuda(), Xd, 128, mode, seed=31, state_bf16=state16)
+    bands = [(0, 256), (256, N - 256)]
+    shards = [g.gsq_init(torch.from_numpy(np.ascontiguousarray(W[r0:r0 + n])).cuda(), Xd, 128,
+                         mode, seed=31, state_bf16=state16, row0=r0) for r0, n in bands]
+    taus = np.array([1.0, 0.6, 0.3, 0.15], np.float32)
+    full.run(taus, 1e-3)
+    for sh in shards:
+        sh.run(taus, 1e-3)
+    for which in (g.GSQ_DBG_LOGITS, g.GSQ_DBG_MOM, g.GSQ_DBG_SCALES, g.GSQ_DBG_SMOM,
+                  g.GSQ_DBG_WHAT, g.GSQ_DBG_DW):
+        whole = full.get(which)
+        axis = 1 if which in (g.GSQ_DBG_LOGITS, g.GSQ_DBG_MOM) else 0
+        parts = np.concatenate([sh.get(which) for sh in shards], axis=axis)
+        assert np.array_equal(parts.view(np.uint8), whole.view(np.uint8)), which
+    assert sum(sh.last_loss() for sh in shards) == pytest.approx(full.last_loss(), rel=1e-12)
+    # the soft weight of the second shard at step 4 from the oracle's noise at
+    # the global coordinates (the oracle state takes row0 likewise)
+    st = oracle_mod.State(mode, N - 256, K, 128, shards[1].get(g.GSQ_DBG_LOGITS).astype(np.float32),
+                          shards[1].get(g.GSQ_DBG_MOM).astype(np.float32),
+                          shards[1].get(g.GSQ_DBG_SCALES), shards[1].get(g.GSQ_DBG_SMOM),
+                          shards[1].get(g.GSQ_DBG_I0), row0=256, seed=31, t=4)
+    if not state16:
+        shards[1].soft_weight(0.2)
+        _, _, w, _ = oracle_mod.soft_weight(st, 0.2)
+        w_gpu = shards[1].get(g.GSQ_DBG_WSOFT32).astype(np.float64)
+        floor = np.repeat(st.s, 128, 1) * LEVEL_MAX[mode]
+        assert np.all(np.abs(w_gpu - w) <= 1e-5 * (np.abs(w) + floor))
+    full.close()
+    for sh in shards:
+        sh.close()
+
+
+def test_row_offset_rejected_on_host(g):
+    cfg, W, X = make_case(0, 8, 128, 8)
+    import ctypes as C
+    ctx = C.c_void_p()
+    rc = g.lib().gsq_init_rows(C.byref(ctx), W.ctypes.data, g.GSQ_F32, X.ctypes.data, g.GSQ_F32,
+                               8, 128, 8, 128, 0, None, 0, -1, 0, None)
+    assert rc == g.GSQ_ERR_INVALID_ARG and not ctx.value
+    rc = g.lib().gsq_init_rows(C.byref(ctx), W.ctypes.data, g.GSQ_F32, X.ctypes.data, g.GSQ_F32,
+                               8, 128, 8, 128, 0, None, 0, 0, 2, None)
+    assert rc == g.GSQ_ERR_INVALID_ARG and not ctx.value
+
+
 # ---------------------------------------------------------- soft weight
 
 @pytest.mark.parametrize("mode", [0, 1, 2])
@@ -430,33 +486,104 @@ def test_bad_step_arguments(g):
 
 # ------------------------------------------- full-size row-slice parity
 
+def _row_state(oracle_mod, mode, arrays, r, t):
+    """The oracle state of row r from the GPU's buffers (identical values)."""
+    logits, mom, s, ms, i0 = arrays
+    return oracle_mod.State(mode, 1, logits.shape[2], 128,
+                            np.ascontiguousarray(logits[:, r:r + 1], np.float32),
+                            np.ascontiguousarray(mom[:, r:r + 1], np.float32),
+                            np.ascontiguousarray(s[r:r + 1]), np.ascontiguousarray(ms[r:r + 1]),
+                            np.ascontiguousarray(i0[r:r + 1]), row0=r, seed=0, t=t)
+
+
 @pytest.mark.parametrize("name", ["c2_qproj_4096x4096", "c3_downproj_4096x14336",
                                   "c4_gateproj_14336x4096"])
-def test_full_size_row_slices(g, oracle_mod, name):
-    """Full layers in the benchmark's launch configuration; the oracle follows
-    a slice of rows (the loss decomposes over rows and the noise is keyed by
-    the global coordinate)."""
+def test_full_size_fused_run_against_oracle_rows(g, oracle_mod, name):
+    """Full layers in the benchmark's launch configuration (gsq_run: every
+    backward but a run's last also forms the next step's soft weight).
+
+    1. gsq_run over 5 steps equals a loop of gsq_step bit for bit, all
+       buffers of the whole layer (the fused path computes what the unfused
+       one does, at full size and in every GEMM wave);
+    2. on sampled rows (first, last, both sides of a 256-row tile edge, the
+       last row tile) the state after 5 fused steps follows the oracle's own
+       5-step trajectory of those rows (Lion near-ties aside);
+    3. one more step from the GPU's exact state, row by row against the
+       oracle: the soft weight (fp32 contract, then bf16 rounding), each
+       row's loss from the GPU's output gradient at 1e-2, the dW rows at
+       1e-2, and -- given the GPU's own dW -- the fused backward: logits and
+       scales bit-identical wherever Lion's blend is not a near-tie, momenta
+       within their bound.
+    The loss decomposes over rows and the noise is keyed by the global
+    coordinate, so each row is an independent oracle problem."""
     import torch
     cfg = synth.CONFIGS[name]
     W, X = synth.make_weight(cfg), synth.make_calib(cfg)
-    lay = g.gsq_init(torch.from_numpy(W).cuda().to(torch.bfloat16),
-                     torch.from_numpy(X).cuda().to(torch.bfloat16), 128, cfg.grid, seed=0)
-    steps = 2
-    taus = synth.tau_schedule(cfg.tau0, cfg.tau1, cfg.steps)[:steps]
-    for tau in taus:
-        lay.step(float(tau), cfg.lr)
-    loss_gpu = lay.last_loss()
-    logits = lay.get(g.GSQ_DBG_LOGITS)
-    scales = lay.get(g.GSQ_DBG_SCALES)
+    Wd = torch.from_numpy(W).cuda().to(torch.bfloat16)
+    Xd = torch.from_numpy(X).cuda().to(torch.bfloat16)
+    taus = np.array([1.0, 0.6, 0.35, 0.2, 0.1, 0.05], np.float32)
+    lr = cfg.lr
+    N, K, T, mode = cfg.N, cfg.K, cfg.T, cfg.grid
+    lay = g.gsq_init(Wd, Xd, 128, mode, seed=0)
+    lay.run(taus[:5], lr)
+    bufs = (g.GSQ_DBG_LOGITS, g.GSQ_DBG_MOM, g.GSQ_DBG_SCALES, g.GSQ_DBG_SMOM, g.GSQ_DBG_I0)
+    s5 = [lay.get(b) for b in bufs]
+    # 1. the same five steps one gsq_step at a time
+    ref = g.gsq_init(Wd, Xd, 128, mode, seed=0)
+    for tau in taus[:5]:
+        ref.step(float(tau), lr)
+    for b, a in zip(bufs, s5):
+        assert np.array_equal(ref.get(b).view(np.uint8), a.view(np.uint8)), b
+    assert ref.last_loss() == lay.last_loss()
+    ref.close()
+    # step 5 on the GPU
+    lay.run(taus[5:6], lr)
+    w5 = bits_to_f32(lay.get(g.GSQ_DBG_WHAT))
+    dW5 = lay.get(g.GSQ_DBG_DW)
+    dyt = lay.get(g.GSQ_DBG_DYT)[:, :T]
+    s6 = [lay.get(b) for b in bufs[:4]]
+    loss5 = lay.last_loss()
     lay.close()
-    rows = [0, 1, cfg.N // 2 + 3, cfg.N - 1]
+    E = bits_to_f32(dyt).astype(np.float64) / 2.0
+    row_loss_gpu = (E * E).sum(1)
+    assert row_loss_gpu.sum() == pytest.approx(loss5, rel=1e-2)
+    rows = sorted({0, 1, 255, 256, N // 2 + 3, N - 257, N - 200, N - 1})
+    agree = []
     for r in rows:
-        Wr = W[r:r + 1]
-        st = oracle_mod.init(cfg.grid, Wr, seed=0, row0=r)
+        Wr = np.ascontiguousarray(W[r:r + 1])
         Y = oracle_mod.reference_output(Wr, X)
-        for tau in taus:
-            oracle_mod.step(st, X, Y, float(tau), cfg.lr)
-        agree = (logits[:, r] == st.logits[:, 0]).mean()
-        assert agree > 0.995, (r, agree)
-        assert np.allclose(scales[r], st.s[0], rtol=0, atol=3 * cfg.lr * steps)
-    assert np.isfinite(loss_gpu) and loss_gpu > 0
+        # 2. the oracle's own trajectory of this row
+        tr = oracle_mod.init(mode, Wr, seed=0, row0=r)
+        for tau in taus[:5]:
+            oracle_mod.step(tr, X, Y, float(tau), lr)
+        agree.append((tr.logits[:, 0] == s5[0][:, r]).mean())
+        # 3. step 5 from the GPU's state of the row
+        st = _row_state(oracle_mod, mode, s5, r, 5)
+        _, v, w, wb = oracle_mod.soft_weight(st, float(taus[5]))
+        floor = np.repeat(st.s, 128, 1) * LEVEL_MAX[mode]
+        half_ulp = np.where(w5[r:r + 1] != 0,
+                            2.0 ** (np.floor(np.log2(np.abs(w5[r:r + 1]) + 1e-300)) - 8), 0)
+        assert np.all(np.abs(w5[r:r + 1] - w) <= 1e-5 * (np.abs(w) + floor) + half_ulp), r
+        assert (w5[r:r + 1] != wb).mean() < 1e-2, r
+        loss_r, dY = oracle_mod.forward(X, wb, Y)
+        assert row_loss_gpu[r] == pytest.approx(loss_r, rel=1e-2), r
+        dW_ref = oracle_mod.weight_grad(dY, X)
+        assert np.linalg.norm(dW5[r] - dW_ref[0]) <= 1e-2 * np.linalg.norm(dW_ref[0]), r
+        # the fused backward given the GPU's dW of the row
+        dWr = np.ascontiguousarray(dW5[r:r + 1])
+        m_before = st.mom.copy()
+        dl_ref, ds_ref = oracle_mod.backward_lion(st, dWr, float(taus[5]), lr)
+        a = np.abs(np.repeat(s5[2][r:r + 1], 128, 1) * dWr) / float(taus[5])
+        c = 0.9 * m_before.astype(np.float64) + 0.1 * dl_ref
+        clear = np.abs(c) > 0.1 * 1e-5 * (np.abs(dl_ref) + a[None]) + 1e-12
+        assert clear.mean() > 0.99, r
+        assert np.array_equal(s6[0][:, r:r + 1][clear], st.logits[clear]), r
+        mtol = 0.01 * 1e-5 * (np.abs(dl_ref) + a[None]) + 2.0 ** -22 * np.abs(st.mom)
+        assert np.all(np.abs(s6[1][:, r:r + 1] - st.mom) <= mtol), r
+        bound = np.abs(dWr.astype(np.float64) * v).reshape(1, -1, 128).sum(-1)
+        sclear = np.abs(0.9 * s5[3][r:r + 1].astype(np.float64) + 0.1 * ds_ref) > 1e-6 * bound
+        assert sclear.mean() > 0.9, r
+        assert np.array_equal(s6[2][r:r + 1][sclear], st.s[sclear]), r
+    assert min(agree) > 0.99, agree
+
+

@@ -86,6 +86,88 @@ def test_two_ranks_independent_layers_and_max_time(oracle_mod):
     assert out[0]["rate"] == pytest.approx(2 * 16 * 256 * 3 / 0.015)
 
 
+def _shard_worker(rank, world, port, out):
+    """One layer split by rows over the ranks (bench.py --split rows): each
+    rank steps its band with the band's global row offset, then the states
+    and losses are gathered on rank 0."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        import oracle
+        from post_weight_quantization_philox_b200 import synth
+        mode = int(os.environ.get("SHARD_MODE", "0"))
+        cfg = synth.small_config(24, 256, 32, mode, number=93)
+        W = synth.make_weight(cfg)          # the same layer on every rank
+        X = synth.make_calib(cfg)
+        r0, n = bench.row_shard(cfg.N, rank, world, align=8)
+        st = oracle.init(cfg.grid, W[r0:r0 + n], seed=5, row0=r0)
+        Y = oracle.reference_output(W[r0:r0 + n], X)
+        losses = [oracle.step(st, X, Y, tau, 1e-3) for tau in (1.0, 0.4, 0.1)]
+        got = [None] * world
+        dist.all_gather_object(got, (r0, n, st.logits, st.mom, st.s, st.ms, losses))
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_row_shards_reproduce_the_whole_layer(oracle_mod, mode):
+    """Two ranks holding rows [0, 8) and [8, 24) of one layer, each keyed by
+    its global row offset, end in exactly the whole layer's state for those
+    rows, and their losses add up to the layer's loss, step by step."""
+    import torch.multiprocessing as mp
+    os.environ["SHARD_MODE"] = str(mode)
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    shards = out[0]
+    assert [(r0, n) for r0, n, *_ in shards] == [(0, 8), (8, 16)]
+    sys.path.insert(0, ROOT)
+    import oracle
+    from post_weight_quantization_philox_b200 import synth
+    cfg = synth.small_config(24, 256, 32, mode, number=93)
+    W, X = synth.make_weight(cfg), synth.make_calib(cfg)
+    full = oracle.init(cfg.grid, W, seed=5)
+    Y = oracle.reference_output(W, X)
+    full_losses = [oracle.step(full, X, Y, tau, 1e-3) for tau in (1.0, 0.4, 0.1)]
+    for r0, n, logits, mom, s, ms, _ in shards:
+        assert np.array_equal(logits, full.logits[:, r0:r0 + n])
+        assert np.array_equal(mom, full.mom[:, r0:r0 + n])
+        assert np.array_equal(s, full.s[r0:r0 + n])
+        assert np.array_equal(ms, full.ms[r0:r0 + n])
+    summed = np.sum([sh[6] for sh in shards], axis=0)
+    assert np.allclose(summed, full_losses, rtol=1e-12, atol=0)
+    # a shard keyed with the wrong offset draws other noise
+    wrong = oracle.init(cfg.grid, W[8:24], seed=5, row0=0)
+    oracle.step(wrong, X, oracle.reference_output(W[8:24], X), 1.0, 1e-3)
+    assert not np.array_equal(wrong.logits, shards[1][2])
+
+
+def test_row_shard_bounds():
+    sys.path.insert(0, ROOT)
+    import bench
+    for N, world in [(4096, 8), (14336, 8), (8192, 3), (24, 2), (100, 4)]:
+        bands = [bench.row_shard(N, r, world) for r in range(world)]
+        assert bands[0][0] == 0
+        assert sum(n for _, n in bands) == N
+        assert all(bands[r][0] + bands[r][1] == bands[r + 1][0] for r in range(world - 1))
+    assert [bench.row_shard(4096, r, 8) for r in range(8)] == [(512 * r, 512) for r in range(8)]
+
+
 def test_single_rank_needs_no_process_group():
     sys.path.insert(0, ROOT)
     import bench

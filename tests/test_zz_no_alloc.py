@@ -4,7 +4,9 @@ their framework forbids device allocation on its execution path).  Its device
 staging is a fixed array inside the library instead of an allocation; this
 checks, through the C ABI, that two calls in a row return exactly what the
 allocating entry point gsq_debug_uniforms returns (uniforms are bit-exact),
-and that counts above the array's capacity are refused."""
+that they equal the oracle's Philox uniforms directly (including counters
+whose low word wraps past 2^32), and that counts above the array's capacity
+are refused."""
 import ctypes as C
 
 import numpy as np
@@ -42,6 +44,16 @@ def test_noalloc_uniforms_match_allocating_entry_point(g, mode):
         out = np.full((n, L), -1.0, np.float32)
         st = lib.gsq_uniforms_noalloc(mode, seed, t, c0, n, out.ctypes.data, None)
         assert st == g.GSQ_OK, g.error_string(st)
+        assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
+    # directly against the oracle's uniforms (the oracle is test
+    # infrastructure: plain C from the published Philox definition), across
+    # the 2^32 boundary of the counter's low word
+    import oracle
+    for t, c0, n in [(0, 0, 4096), (12, (1 << 32) - 2048, 4096)]:
+        out = np.full((n, L), -1.0, np.float32)
+        st = lib.gsq_uniforms_noalloc(mode, seed, t, c0, n, out.ctypes.data, None)
+        assert st == g.GSQ_OK, g.error_string(st)
+        ref = oracle.uniforms(mode, seed, t, c0, n)
         assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
     # device output buffer
     dev = torch.zeros((513, L), dtype=torch.float32, device="cuda")
