@@ -216,6 +216,19 @@ GSQ_API int gsq_init_gptq(gsq_ctx** out, const void* W, int w_dtype, const void*
 GSQ_API int gsq_step(gsq_ctx* ctx, float tau, float lr, float beta1, float beta2);
 
 /*
+ * gsq_step_next -- gsq_step at tau whose fused backward also forms the soft
+ * weight of the next step at tau_next (its noise and tempered softmax from
+ * the updated logits and scales), so that the next gsq_step or
+ * gsq_step_next call at that temperature starts at its forward GEMM: a
+ * caller-driven loop of gsq_step_next(tau_t, tau_{t+1}) costs what gsq_run
+ * costs and gives the same results bit for bit.  A next call at another
+ * temperature recomputes its soft weight.  Errors: as gsq_step, and
+ * GSQ_ERR_INVALID_ARG for tau_next <= 0 or not finite.
+ */
+GSQ_API int gsq_step_next(gsq_ctx* ctx, float tau, float tau_next, float lr, float beta1,
+                          float beta2);
+
+/*
  * gsq_run -- n consecutive steps at temperatures taus[0..n) (host array),
  * asynchronous.  Same results, bit for bit, as n calls of gsq_step; the
  * backward of each step but the last also builds the next step's soft weight

@@ -489,7 +489,7 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
   NvtxRange step_range("gsq_step");
   const bool soft = !(c->what_t == (int64_t)c->t && c->what_tau == tau);
   if (soft) {
-    NvtxRange r("gsq_step/soft_weight");
+    NvtxRange r("soft_weight");
     CK(launch_soft_weight(a, c->What, nullptr, c->sms, c->st));
   }
   if (tm) {
@@ -498,17 +498,17 @@ int run_step(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
     CK(cudaEventRecord(tm->ev[1], c->st));
   }
   {
-    NvtxRange r("gsq_step/forward_gemm");
+    NvtxRange r("forward_gemm");
     CK(run_forward(c, c->loss_hist + (c->t % kLossRing), EPI_LOSS_DY));
   }
   if (tm) CK(cudaEventRecord(tm->ev[2], c->st));
   {
-    NvtxRange r("gsq_step/weight_grad_gemm");
+    NvtxRange r("weight_grad_gemm");
     CK(run_weight_grad(c));
   }
   if (tm) CK(cudaEventRecord(tm->ev[3], c->st));
   {
-    NvtxRange r(tau_next > 0.f ? "gsq_step/backward_lion_next_soft" : "gsq_step/backward_lion");
+    NvtxRange r(tau_next > 0.f ? "backward_lion_next_soft" : "backward_lion");
     CK(launch_backward_lion(a, c->dW, lr, beta1, beta2, tau_next, c->What, nullptr, nullptr,
                             c->sms, c->st));
   }
@@ -575,6 +575,15 @@ int gsq_step(gsq_ctx* c, float tau, float lr, float beta1, float beta2) {
   if (u) return u;
   if (!step_args_ok(tau, lr, beta1, beta2)) return GSQ_ERR_INVALID_ARG;
   return run_step(c, tau, 0.f, lr, beta1, beta2);
+}
+
+int gsq_step_next(gsq_ctx* c, float tau, float tau_next, float lr, float beta1,
+                  float beta2) {
+  int u = usable(c);
+  if (u) return u;
+  if (!step_args_ok(tau, lr, beta1, beta2) || !(tau_next > 0.f && std::isfinite(tau_next)))
+    return GSQ_ERR_INVALID_ARG;
+  return run_step(c, tau, tau_next, lr, beta1, beta2);
 }
 
 int gsq_run(gsq_ctx* c, const float* taus, int64_t n, float lr, float beta1,

@@ -45,7 +45,7 @@ EXPORTS = [
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
     "gsq_gptq", "gsq_release_cached_memory", "gsq_set_cached_memory_limit", "gsq_init_gptq", "gsq_init_bf16_state",
-    "gsq_init_rows", "gsq_mlp_set_timing", "gsq_mlp_phase_times", "gsq_attn_set_timing",
+    "gsq_init_rows", "gsq_step_next", "gsq_mlp_set_timing", "gsq_mlp_phase_times", "gsq_attn_set_timing",
     "gsq_attn_phase_times", "gsq_debug_stall_probe", "gsq_debug_fail_alloc", "gsq_debug_pool_used",
     "gsq_mlp_init", "gsq_mlp_step", "gsq_mlp_run", "gsq_mlp_last_loss",
     "gsq_mlp_recon_error", "gsq_mlp_harden_pack", "gsq_mlp_debug_get",
@@ -83,6 +83,7 @@ _SIGS = {
     "gsq_init_rows": [_pp, _p, _i32, _p, _i32, _i64, _i64, _i64, _i32, _i32, _p, _u64, _i64,
                       _i32, _p],
     "gsq_step": [_p, _f32, _f32, _f32, _f32],
+    "gsq_step_next": [_p, _f32, _f32, _f32, _f32, _f32],
     "gsq_run": [_p, _p, _i64, _f32, _f32, _f32],
     "gsq_last_loss": [_p, C.POINTER(C.c_double)],
     "gsq_loss_history": [_p, _u64, _i64, _p],
@@ -498,8 +499,14 @@ class Layer:
                "gsq_debug_scale_backward")
 
     # convenience -------------------------------------------------------
-    def step(self, tau, lr, beta1=0.9, beta2=0.99):
-        gsq_step(self, tau, lr, beta1, beta2)
+    def step(self, tau, lr, beta1=0.9, beta2=0.99, tau_next=None):
+        """One step; with tau_next, gsq_step_next (the backward also forms the
+        next step's soft weight at tau_next)."""
+        if tau_next is None:
+            gsq_step(self, tau, lr, beta1, beta2)
+        else:
+            _check(_lib.gsq_step_next(self.ctx, tau, tau_next, lr, beta1, beta2),
+                   "gsq_step_next")
 
     def scale_step(self, lr, beta1=0.9, beta2=0.99):
         gsq_scale_step(self, lr, beta1, beta2)
