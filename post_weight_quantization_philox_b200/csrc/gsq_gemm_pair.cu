@@ -99,10 +99,24 @@ __device__ __forceinline__ TileAt tile_at(int tile, int m_tiles, int n_tiles,
   t.r0 = 0;
   t.kps = 0;
   if (sc.causal == 0) {
-    mb = tile % m_tiles;
-    const int r = tile / m_tiles;
-    nb = r % n_tiles;
-    p = r / n_tiles;
+    const int per = m_tiles * n_tiles;
+    p = tile / per;
+    const int local = tile - p * per;
+    if (sc.group_m > 1) {
+      // bands of group_m row tiles: a wave of CTA pairs then shares a few
+      // row tiles of A and a few column tiles of B instead of streaming one
+      // row tile of A per pair
+      const int band_tiles = sc.group_m * n_tiles;
+      const int band = local / band_tiles;
+      const int within = local - band * band_tiles;
+      const int first = band * sc.group_m;
+      const int gm = m_tiles - first < sc.group_m ? m_tiles - first : sc.group_m;
+      mb = first + within % gm;
+      nb = within / gm;
+    } else {
+      mb = local % m_tiles;
+      nb = local / m_tiles;
+    }
     t.nk = (int)((Kc + BK - 1) / BK);
     if (sc.nseg > 1) t.kps = (int)(sc.seg / BK);
   } else {
@@ -540,11 +554,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Band height of the tile order (GemmSched::group_m) when the caller leaves it
+// to the launcher: bands of 8 row tiles once A has 24 or more row tiles (its
+// row tiles then no longer stay in L2 from one column tile to the next; a
+// wave of 74 pairs reads about 19 distinct operand tiles instead of about 75
+// on the 70B MLP shapes), row tiles fastest otherwise.
+inline int auto_group_m(int m_tiles, int n_tiles) {
+  return (m_tiles >= 24 && n_tiles > 1) ? 8 : 1;
+}
+
 template <int EPI, int BN>
 cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
                             const EpiMaps& maps, int64_t M, int64_t N,
-                            int64_t Kc, const GemmSched& sc, const EpiParams& ep,
+                            int64_t Kc, const GemmSched& sc_in, const EpiParams& ep,
                             int sm_count, cudaStream_t st) {
+  GemmSched sc = sc_in;
+  if (sc.causal == 0 && sc.group_m == 0)
+    sc.group_m = auto_group_m((int)((M + PM - 1) / PM), (int)((N + BN - 1) / BN));
   // co-resident CTA pairs of this kernel (the same on every B200; computed once)
   static std::atomic<int> max_pairs_cache{0};
   int max_pairs = max_pairs_cache.load(std::memory_order_relaxed);

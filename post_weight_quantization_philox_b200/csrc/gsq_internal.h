@@ -197,6 +197,10 @@ struct GemmSched {
   int nseg = 1;
   int64_t a_seg_k = 0, a_seg_row = 0, b_seg_k = 0, b_seg_row = 0;
   int64_t o_fold = 0, o_fold_col = 0;
+  // tile order of a non-causal schedule: row tiles fastest within bands of
+  // group_m row tiles, every column tile of a band before the next band
+  // (1: row tiles fastest over all of them; 0: chosen by the launcher)
+  int group_m = 0;
 };
 // Box rows of the B tensor map for the 128-wide output tiles (bn = 128).
 constexpr int kGemmBoxRowsBNarrow = 64;
