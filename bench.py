@@ -286,6 +286,12 @@ def run_gsq(args, rank, world, local_rank):
     phase_ms = list(phase_ms)
     phase_n = list(phase_n)
     phase_ms[0], phase_n[0] = loop_ms[0], loop_n[0]
+    if phase_n[2] == 0 and phase_n[1] > 0:
+        # both GEMMs of a step ran as one launch (layers with fewer than 24
+        # row tiles): the forward slot holds them both
+        names = list(names)
+        names[1] = "gemms_merged"
+        work["gemms_merged"] = ("tensor", work["forward_gemm"][1] + work["weight_grad_gemm"][1])
     for i, nm in enumerate(names):
         if phase_n[i] == 0:
             continue

@@ -72,8 +72,9 @@ constexpr int DY_TILE = 32 * 32 * 2;
 template <int EPI>
 __host__ __device__ constexpr int warp_stage_bytes() {
   return EPI == EPI_STORE_BF16 ? 2 * DY_TILE
-                               : (EPI == EPI_LOSS_DY ? 2 * OUT_TILE + 2 * DY_TILE
-                                                     : 2 * OUT_TILE);
+                               : ((EPI == EPI_LOSS_DY || EPI == EPI_MERGED)
+                                      ? 2 * OUT_TILE + 2 * DY_TILE
+                                      : 2 * OUT_TILE);
 }
 template <int EPI, int BN>
 __host__ __device__ constexpr int smem_bytes() {
@@ -185,6 +186,36 @@ __device__ __forceinline__ uint32_t swz64(int r, int j) {
   return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
+// acquire load of a counter another CTA releases; then the fence that orders
+// it before this thread's later async-proxy (TMA) reads of global memory
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Row band of a merged launch's tile and whether it is a weight-gradient
+// tile: forward tiles [0, tiles_f) first, then the weight-gradient tiles,
+// each problem with its column tiles fastest inside a band of 256 rows.
+__device__ __forceinline__ TileAt merged_tile_at(int tile, int tiles_f, int n_tiles,
+                                                 int n_tiles2, int64_t Kc, int64_t Kc2,
+                                                 bool& wgrad) {
+  TileAt t;
+  wgrad = tile >= tiles_f;
+  const int local = wgrad ? tile - tiles_f : tile;
+  const int nt = wgrad ? n_tiles2 : n_tiles;
+  t.a_row = t.a_k = t.b_row = t.b_k = t.o_row = t.o_col = 0;
+  t.r0 = 0;
+  t.kps = 0;
+  t.m0 = (int64_t)(local / nt) * PM;
+  t.n0 = (int64_t)(local % nt) * 256;
+  t.nk = (int)(((wgrad ? Kc2 : Kc) + BK - 1) / BK);
+  return t;
+}
+
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   const bool ok = mbar_wait_bounded(bar, parity, WAIT_LIMIT);
   return __all_sync(0xffffffffu, ok);
@@ -196,9 +227,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmO,
                 const __grid_constant__ CUtensorMap tmY, int64_t M, int64_t N,
-                int64_t Kc, EpiParams ep, const __grid_constant__ GemmSched sc) {
+                int64_t Kc, EpiParams ep, const __grid_constant__ GemmSched sc,
+                const __grid_constant__ MergeArgs mg) {
   pdl_trigger();  // our CTAs are all resident (persistent grid)
   using C = Cfg<BN>;
+  // a merged launch: forward tiles (loss + dY epilogue) then weight-gradient
+  // tiles (fp32 store into mg.tmO2)
+  constexpr bool MERGED = EPI == EPI_MERGED;
   constexpr int PN = C::PN, STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
   constexpr int TMEM_COLS = C::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -212,8 +247,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int m_tiles = (int)((M + PM - 1) / PM);
   const int n_tiles = (int)((N + PN - 1) / PN);
+  const int n_tiles2 = MERGED ? (int)((mg.N2 + PN - 1) / PN) : 0;
+  const int tiles_f = m_tiles * n_tiles * sc.count;
   // the test hook's launch processes no tile: nothing is ever in flight
-  const int num_tiles = ep.stall_probe ? 0 : m_tiles * n_tiles * sc.count;
+  const int num_tiles = ep.stall_probe ? 0 : tiles_f + (MERGED ? m_tiles * n_tiles2 : 0);
+  // where tile `tile` sits, and whether it is a merged launch's weight-gradient tile
+  auto at = [&](int tile, bool& wgrad) -> TileAt {
+    if (MERGED) return merged_tile_at(tile, tiles_f, n_tiles, n_tiles2, Kc, mg.Kc2, wgrad);
+    wgrad = false;
+    return tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
+  };
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0 && lane == 0) {
@@ -234,7 +277,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ctl->abort = 0;
     mbar_fence_init();
     if (EPI != EPI_LOSS) tma_prefetch_desc(&tmO);
-    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS) tma_prefetch_desc(&tmY);
+    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED) tma_prefetch_desc(&tmY);
+    if (MERGED) {
+      tma_prefetch_desc(&mg.tmA2);
+      tma_prefetch_desc(&mg.tmB2);
+      tma_prefetch_desc(&mg.tmO2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -262,9 +310,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       long long issued = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        const TileAt ta = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
+        bool wgrad;
+        const TileAt ta = at(tile, wgrad);
         const int32_t ya = (int32_t)(ta.a_row + ta.m0 + (int)rank * HALF);
         const int32_t yb = (int32_t)(ta.b_row + ta.n0 + (int)rank * C::HALFN);
+        const void* mapA = &tmA;
+        const void* mapB = &tmB;
+        if (MERGED && wgrad) {
+          mapA = &mg.tmA2;
+          mapB = &mg.tmB2;
+          // this band's dY rows must be in memory: every forward tile of the
+          // band has counted its stores (bounded wait)
+          const unsigned* flag = mg.band_done + ta.m0 / PM;
+          if (ld_acquire_u32(flag) < mg.target) {
+            const long long t0 = clock64();
+            while (ld_acquire_u32(flag) < mg.target) {
+              if (clock64() - t0 > WAIT_LIMIT || *(volatile int*)&ctl->abort) {
+                ok = false;
+                break;
+              }
+              __nanosleep(128);
+            }
+            if (!ok) break;
+          }
+          fence_proxy_async_global();
+        }
         for (int kb = 0; kb < ta.nk; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&ctl->empty[stage]), ph ^ 1,
                                  WAIT_LIMIT) ||
@@ -277,8 +347,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (leader) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
           const uint32_t sa = sbase + stage * STAGE_BYTES;
           const KAt kx = tile_k(ta, kb, sc);
-          tma_load_2d_pair(sa, &tmA, fb_leader, (int32_t)kx.ak, ya + (int32_t)kx.arow);
-          tma_load_2d_pair(sa + A_BYTES, &tmB, fb_leader, (int32_t)kx.bk,
+          tma_load_2d_pair(sa, mapA, fb_leader, (int32_t)kx.ak, ya + (int32_t)kx.arow);
+          tma_load_2d_pair(sa + A_BYTES, mapB, fb_leader, (int32_t)kx.bk,
                            yb + (int32_t)kx.brow);
           ++issued;
           if (++stage == STAGES) {
@@ -319,7 +389,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PN);
-        const int nk = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc).nk;
+        bool wgrad_unused;
+        const int nk = at(tile, wgrad_unused).nk;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&ctl->full[stage]), ph,
                                  WAIT_LIMIT) ||
@@ -372,12 +443,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t dy_s = smem_u32(wst + 2 * OUT_TILE);    // 2 x DY_TILE
     constexpr int UNITS = C::UNITS;
     const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
-    const int64_t total_units = (int64_t)my_tiles * UNITS;
+    // units that read Y_ref: all of them, or a merged launch's forward ones
+    // (a pair's forward tiles come before its weight-gradient tiles)
+    const int fwd_tiles_mine =
+        MERGED ? (pair < tiles_f ? (tiles_f - 1 - pair) / npairs + 1 : 0) : my_tiles;
+    const int64_t y_units = (int64_t)(fwd_tiles_mine < my_tiles ? fwd_tiles_mine : my_tiles) * UNITS;
     // coordinates (x = column, y = first row) of unit u of this warp; false
     // when the unit lies wholly outside its problem's M x N
     auto unit_xy = [&](int64_t u, int32_t& x, int32_t& y) {
       const int tile = pair + (int)(u / UNITS) * npairs;
-      const TileAt ta = tile_at<BN>(tile, m_tiles, n_tiles, Kc, sc);
+      bool wgrad;
+      const TileAt ta = at(tile, wgrad);
+      const int64_t ncols = (MERGED && wgrad) ? mg.N2 : N;
       const int64_t lx = ta.n0 + (int)(u % UNITS) * 32;
       const int64_t ly = ta.m0 + (int)rank * HALF + q * 32;
       if (sc.o_fold > 0) {
@@ -388,7 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         x = (int32_t)(ta.o_col + lx);
         y = (int32_t)(ta.o_row + ly);
       }
-      return lx < N && ly < M;
+      return lx < ncols && ly < M;
     };
     int64_t y_issued = 0;
     auto issue_y = [&](int64_t u) {  // lane 0: Y_ref tile of unit u
@@ -398,8 +475,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive_expect_tx(bar, OUT_TILE);
       tma_load_2d(y_s + (uint32_t)((u & 1) * OUT_TILE), &tmY, bar, x, y);
     };
-    if ((EPI == EPI_LOSS_DY || EPI == EPI_LOSS) && lane == 0) {
-      for (; y_issued < 2 && y_issued < total_units; ++y_issued) issue_y(y_issued);
+    if ((EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED) && lane == 0) {
+      for (; y_issued < 2 && y_issued < y_units; ++y_issued) issue_y(y_issued);
     }
     int acc = 0;
     uint32_t aph = 0;
@@ -408,6 +485,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int last_buf = -1;  // staging buffer of the newest committed store (lane 0)
     bool ok = true;
     for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+      // a merged launch's weight-gradient tile takes the fp32-store epilogue,
+      // its forward tiles the loss + dY one
+      bool wtile = false;
+      int64_t band = 0;
+      if (MERGED) band = at(tile, wtile).m0 / PM;
+      const bool store_f32 = EPI == EPI_STORE_F32 || (MERGED && wtile);
+      const bool store_any = store_f32 || EPI == EPI_STORE_BF16;
+      const bool with_dy = EPI == EPI_LOSS_DY || (MERGED && !wtile);
+      const void* mapO = (MERGED && wtile) ? (const void*)&mg.tmO2 : (const void*)&tmO;
       if (!warp_wait(smem_u32(&ctl->tfull[acc]), aph) ||
           *(volatile int*)&ctl->abort) {
         ok = false;
@@ -425,7 +511,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int32_t x, y;
         const bool inside = unit_xy(u, x, y);
         const int b = (int)(u & 1);
-        if (EPI == EPI_STORE_F32 || EPI == EPI_STORE_BF16) {
+        if (store_any) {
           // this buffer may be rewritten once the store that last read it is
           // done: the newest group if it used this buffer, else the one before
           if (lane == 0) {
@@ -433,9 +519,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else bulk_wait_read<1>();
           }
           __syncwarp();
-          const uint32_t base =
-              out_s + (uint32_t)(b * (EPI == EPI_STORE_F32 ? OUT_TILE : DY_TILE));
-          if (EPI == EPI_STORE_F32) {
+          const uint32_t base = out_s + (uint32_t)(b * (store_f32 ? OUT_TILE : DY_TILE));
+          if (store_f32) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const uint32_t a = base + swz128(lane, j);
@@ -458,7 +543,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0 && inside) {  // no store for a box wholly outside C
-            tma_store_2d(&tmO, base, x, y);
+            tma_store_2d(mapO, base, x, y);
             bulk_commit();
             last_buf = b;
           }
@@ -483,13 +568,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             e[4 * j + 3] = __uint_as_float(v[4 * j + 3]) - y4.w;
           }
           __syncwarp();  // every lane has read this Y_ref buffer
-          if (lane == 0 && y_issued < total_units && y_issued == u + 2) {
+          if (lane == 0 && y_issued < y_units && y_issued == u + 2) {
             issue_y(y_issued);
             ++y_issued;
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) part = fmaf(e[j], e[j], part);
-          if (EPI == EPI_LOSS_DY) {
+          if (with_dy) {
             if (lane == 0) {
               if (last_buf == b) bulk_wait_read<0>();
               else bulk_wait_read<1>();
@@ -509,7 +594,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0 && inside) {
-              tma_store_2d(&tmO, dbase, x, y);
+              tma_store_2d(mapO, dbase, x, y);
               bulk_commit();
               last_buf = b;
             }
@@ -520,6 +605,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tempty[acc]), 0));
+      if (MERGED && !wtile && ok && lane == 0) {
+        // this warp's dY stores of the tile are complete: count them for the
+        // band's weight-gradient tiles (the async-proxy writes are ordered
+        // before the release of the count)
+        bulk_wait_all();
+        fence_proxy_async_global();
+        __threadfence();
+        atomicAdd(mg.band_done + band, 1u);
+      }
       acc ^= 1;
       if (acc == 0) aph ^= 1;
     }
@@ -536,7 +630,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bulk_wait_all();  // stores complete before the CTA exits
     }
     __syncwarp();
-    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS) {
+    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED) {
       lsum = warp_sum_d(lsum);
       if (lane == 0) ctl->red[q] = lsum;
       asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -567,7 +661,8 @@ template <int EPI, int BN>
 cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
                             const EpiMaps& maps, int64_t M, int64_t N,
                             int64_t Kc, const GemmSched& sc_in, const EpiParams& ep,
-                            int sm_count, cudaStream_t st) {
+                            int sm_count, cudaStream_t st,
+                            const MergeArgs& mg = MergeArgs()) {
   GemmSched sc = sc_in;
   if (sc.causal == 0 && sc.group_m == 0)
     sc.group_m = auto_group_m((int)((M + PM - 1) / PM), (int)((N + BN - 1) / BN));
@@ -602,13 +697,13 @@ cudaError_t launch_pair_epi(const CUtensorMap& tmA, const CUtensorMap& tmB,
     max_pairs = n;
     max_pairs_cache.store(n, std::memory_order_relaxed);
   }
-  const int64_t tiles =
-      ((M + PM - 1) / PM) * ((N + BN - 1) / BN) * (int64_t)sc.count;
+  int64_t tiles = ((M + PM - 1) / PM) * ((N + BN - 1) / BN) * (int64_t)sc.count;
+  if (EPI == EPI_MERGED) tiles = merged_tiles(M, N, mg.N2);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_gemm_pair<EPI, BN>, tmA, tmB, maps.out, maps.yref,
-                            M, N, Kc, ep, sc);
+                            M, N, Kc, ep, sc, mg);
 }
 
 }  // namespace
@@ -632,6 +727,23 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
       return launch_pair_epi<EPI_LOSS, 256>(tmA, tmB, maps, M, N, Kc, one, ep, sm_count,
                                             st);
   }
+}
+
+int64_t merged_band_tiles(int64_t N) { return (N + 255) / 256; }
+
+int64_t merged_tiles(int64_t M, int64_t N, int64_t N2) {
+  return ((M + PM - 1) / PM) * (merged_band_tiles(N) + merged_band_tiles(N2));
+}
+
+cudaError_t launch_gemm_merged(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                               const EpiMaps& maps, int64_t M, int64_t N, int64_t Kc,
+                               const MergeArgs& mg, const EpiParams& ep, int sm_count,
+                               cudaStream_t st) {
+  if (M <= 0 || N <= 0 || Kc <= 0 || mg.N2 <= 0 || mg.Kc2 <= 0 || !mg.band_done)
+    return cudaErrorInvalidValue;
+  const GemmSched one;
+  return launch_pair_epi<EPI_MERGED, 256>(tmA, tmB, maps, M, N, Kc, one, ep, sm_count, st,
+                                           mg);
 }
 
 cudaError_t launch_gemm_batched(const CUtensorMap& tmA, const CUtensorMap& tmB,

@@ -34,7 +34,9 @@ enum EpiMode : int {
   EPI_STORE_F32 = 0,  // C = acc (fp32 store)
   EPI_LOSS_DY = 1,    // E = acc - Yref; loss += sum E^2; dY = bf16(2E)
   EPI_LOSS = 2,       // E = acc - Yref; loss += sum E^2
-  EPI_STORE_BF16 = 3  // C = bf16(acc)
+  EPI_STORE_BF16 = 3,  // C = bf16(acc)
+  EPI_MERGED = 4       // a forward (EPI_LOSS_DY) and a weight-gradient
+                       // (EPI_STORE_F32) problem in one launch (MergeArgs)
 };
 
 struct EpiParams {
@@ -110,6 +112,20 @@ struct PhaseClock {
 // phases of a block stage's step
 enum : int { PH_SOFT = 0, PH_GEMM = 1, PH_ELEM = 2, PH_BACKWARD = 3, PH_COUNT = 4 };
 
+// The weight-gradient problem of a merged launch (launch_gemm_merged).  The
+// forward problem's tiles [0, TF) come first, then the weight-gradient tiles
+// (both in row-band order: every column tile of a band of 256 rows before the
+// next band); both problems have the same M (the rows of W).  Every epilogue
+// warp adds 1 to band_done[band] once a forward tile's dY stores are complete;
+// a weight-gradient tile of a band waits until band_done[band] reaches target,
+// i.e. until that band's dY rows (its A operand) are in memory.
+struct MergeArgs {
+  CUtensorMap tmA2, tmB2, tmO2;  // dY^T rows, X^T rows, dW (fp32 epilogue map)
+  int64_t N2 = 0, Kc2 = 0;
+  unsigned* band_done = nullptr;  // one counter per row band, never reset
+  unsigned target = 0;            // generation x column tiles x 8 epilogue warps
+};
+
 // Opts kernel Fn in to `bytes` of dynamic shared memory on the current device,
 // once per device (the attribute is per device; a process may drive several).
 template <auto Fn>
@@ -168,6 +184,18 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const EpiMaps& maps, int64_t M, int64_t N,
                              int64_t Kc, int mode, const EpiParams& ep,
                              int sm_count, cudaStream_t st);
+// Forward (C = A . B^T with the loss + dY epilogue, maps as launch_gemm) and
+// weight gradient (mg) in one persistent launch: the weight-gradient tiles of
+// a row band start as soon as that band's forward tiles are done, so the two
+// problems share one tail.  mg.band_done: M / 256 counters (rounded up).
+cudaError_t launch_gemm_merged(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                               const EpiMaps& maps, int64_t M, int64_t N, int64_t Kc,
+                               const MergeArgs& mg, const EpiParams& ep, int sm_count,
+                               cudaStream_t st);
+// Tiles of the two problems of a merged launch (its grid sizing) and the
+// forward tiles per row band.
+int64_t merged_tiles(int64_t M, int64_t N, int64_t N2);
+int64_t merged_band_tiles(int64_t N);
 
 // Many equal GEMMs in one launch.  Problem p = p1 * inner + p2 (p < count)
 // is C_p[M x N] = A_p[M x Kc] . B_p[N x Kc]^T, where the operands and the
