@@ -215,16 +215,18 @@ __device__ __forceinline__ void candidates(int lev0, float* cand) {
 // Tempered Gumbel-softmax of one coordinate at a step, from its logits l and
 // its Philox words w, and its unit value v.  Categorical modes: e holds the
 // unnormalised e_k, r[0] = 1 / sum e, and v = r[0] sum_k e_k c_k over the
-// candidate values cand[].  Ternary (one softmax over the mask pair, one over
-// the sign pair): e holds the normalised probabilities p0, p1, q-, q+ and
-// v = p1 (q+ - q-).
+// candidate values cand[]; an e_k below 2^-126 is flushed (its share of v is
+// far below v's rounding, as the largest e_k is 1).  Ternary (one softmax
+// over the mask pair, one over the sign pair): e holds the normalised
+// probabilities p0, p1, q-, q+ and v = p1 (q+ - q-); v is itself as small as
+// p1, so subnormal probabilities are kept.
 template <int MODE>
 __device__ __forceinline__ float coord_value(const float* l, const uint32_t* w, bool noise,
-                                             float inv_tau, const float* cand, float* e,
-                                             float* r) {
+                                             float inv_tau, const float2* cells,
+                                             const float* cand, float* e, float* r) {
   if (MODE == GRID_TERNARY) {
-    const float rm = gsoftmax2<2>(l, w, noise, inv_tau, e);
-    const float rs = gsoftmax2<2>(l + 2, w + 2, noise, inv_tau, e + 2);
+    const float rm = gsoftmax2<2, true>(l, w, noise, inv_tau, cells, e);
+    const float rs = gsoftmax2<2, true>(l + 2, w + 2, noise, inv_tau, cells, e + 2);
     e[0] *= rm;
     e[1] *= rm;
     e[2] *= rs;
@@ -232,7 +234,7 @@ __device__ __forceinline__ float coord_value(const float* l, const uint32_t* w, 
     r[0] = 1.f;
     return e[1] * (e[3] - e[2]);
   } else {
-    r[0] = gsoftmax2<GridT<MODE>::L>(l, w, noise, inv_tau, e);
+    r[0] = gsoftmax2<GridT<MODE>::L, false>(l, w, noise, inv_tau, cells, e);
     float v = 0.f;
 #pragma unroll
     for (int k = 0; k < GridT<MODE>::L; ++k) v = fmaf(e[k], cand[k], v);
@@ -287,6 +289,9 @@ __global__ void __launch_bounds__(256) k_soft_weight(
     uint64_t coord0, uint32_t t, int noise, float inv_tau, __nv_bfloat16* __restrict__ What,
     float* __restrict__ wsoft32) {
   constexpr int L = GridT<MODE>::L;
+  __shared__ float2 l2cells[2 * kLog2Cells];
+  log2_cells_init(l2cells);
+  __syncthreads();
   const int64_t NK = N * K, G = K / kGroup;
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
       wd[4] = q1[j];
       float cand[5], e[L], r;
       candidates<MODE>(levj[j], cand);
-      w[j] = sg * coord_value<MODE>(lj[j], wd, noise, inv_tau, cand, e, &r);
+      w[j] = sg * coord_value<MODE>(lj[j], wd, noise, inv_tau, l2cells, cand, e, &r);
     }
     store_bf16x4(What + c0, w);
     if (DBG) *reinterpret_cast<float4*>(wsoft32 + c0) = make_float4(w[0], w[1], w[2], w[3]);
@@ -377,8 +382,11 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
   constexpr int L = C::L;
   constexpr bool S16 = sizeof(TS) == 2;
   extern __shared__ __align__(16) uint8_t bwd_smem[];
+  __shared__ float2 l2cells[2 * kLog2Cells];
   pdl_trigger();  // persistent grid: every CTA is resident
+  log2_cells_init(l2cells);
   pdl_wait();     // dW (and the state) of the previous kernels are complete
+  __syncthreads();
   const int64_t NK = N * K, G = K / kGroup, groups = N * G;
   const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
   const int64_t warp = (int64_t)blockIdx.x * C::WARPS + wic;
@@ -469,7 +477,7 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
 #pragma unroll
       for (int p = 0; p < L; ++p) l[p] = Lr[p][j];
       candidates<MODE>(lev[j], cand);
-      const float v = coord_value<MODE>(l, wd, noise, inv_tau, cand, e, &r);
+      const float v = coord_value<MODE>(l, wd, noise, inv_tau, l2cells, cand, e, &r);
       const float dw = Dr[j];
       ds_part = fmaf(dw, v, ds_part);
       const float a = sg * dw * inv_tau;
@@ -556,7 +564,7 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
         if (NEXT) {
           float e[L], cand[5], r;
           candidates<MODE>(lev[j], cand);
-          w[j] = s_new * coord_value<MODE>(l, wd, noise, inv_tau_next, cand, e, &r);
+          w[j] = s_new * coord_value<MODE>(l, wd, noise, inv_tau_next, l2cells, cand, e, &r);
         }
       }
       if (S16) {
