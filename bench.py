@@ -1096,12 +1096,13 @@ def run_kquant_stage(args, rank, world, local_rank):
     ach = flops / (per / 1e3) / 1e12
     coords = cfg.N * cfg.K
     # the step at the peaks: both GEMMs at the tensor rate plus the fused
-    # backward's bytes at the copy rate (read dW 4, q0 1, logits, momenta and
-    # probabilities 12 L; write logits and momenta 8 L, probabilities 4 L, the
-    # bf16 soft weight 2; sub-block parameters and momenta 2 (Q2_K) or 1 B)
+    # backward's bytes at the copy rate (read dW 4, q0 1, logits and momenta
+    # 8 L; write logits and momenta 8 L, the bf16 soft weight 2; sub-block
+    # parameters and momenta 2 (Q2_K) or 1 B; the probabilities are drawn
+    # again, not stored)
     q2 = args.kq_format == "q2k"
     L = 4 if q2 else 5
-    bwd_bytes = coords * (7 + 24 * L + (2 if q2 else 1))
+    bwd_bytes = coords * (7 + 16 * L + (2 if q2 else 1))
     gemm_ms = flops / (tf_sus * 1e12) * 1e3
     hbm_ms = bwd_bytes / (hbm * 1e9) * 1e3
     return {"metric": METRIC, "value": whole_job_rate(world, coords * args.steps, ms), "unit": UNIT,

@@ -333,6 +333,10 @@ GSQ_API int gsq_phase_times(gsq_ctx* ctx, double* ms, int64_t* launches);
  *
  * gsq_debug_uniforms: the L Philox uniforms of coords [coord0, coord0+count)
  *   at step t, coordinate-major, into host memory.  Syncs.
+ * gsq_debug_noise_log2: log2(u) as every step's noise forms it (the
+ *   table-driven logarithm of the kernels) for the uniforms
+ *   u = (m + 1/2) 2^-23, m = m0 .. m0 + count - 1, into host memory (count
+ *   floats); m0 + count <= 2^23, else GSQ_ERR_INVALID_ARG.  Syncs.
  * gsq_debug_get / gsq_debug_set: copy an internal buffer to / from host
  *   memory; bytes must equal the buffer size.  Syncs.  Buffers:          */
 enum {
@@ -354,6 +358,8 @@ enum {
 };
 GSQ_API int gsq_debug_uniforms(gsq_ctx* ctx, uint32_t t, uint64_t coord0,
                        int64_t count, float* host_out);
+GSQ_API int gsq_debug_noise_log2(gsq_ctx* ctx, uint32_t m0, int64_t count,
+                                 float* host_out);
 GSQ_API int gsq_debug_get(gsq_ctx* ctx, int which, void* host, size_t bytes);
 GSQ_API int gsq_debug_set(gsq_ctx* ctx, int which, const void* host, size_t bytes);
 /* noise on (default) / off; off sets g = 0 */
@@ -622,8 +628,9 @@ GSQ_API int gsq_block_quantize(const float* x_in, const void* const* W, int64_t 
  * gsq_kq_dequant: bf16 weight (N x K) of blocks, w = bf16((d sc_j) q -
  *   dmin m_j) with each product and the difference rounded in fp32.  Syncs.
  * gsq_kq_debug_get / _set (GSQ_KQ_DBG_*), gsq_kq_debug_soft_weight (fills
- *   GSQ_KQ_DBG_WSOFT32), gsq_kq_debug_backward (soft weight of the current
- *   step, then backward + Lion from the current dW, filling DL, DA, DB),
+ *   GSQ_KQ_DBG_WSOFT32), gsq_kq_debug_backward (backward + Lion from the
+ *   current dW, filling DL, DA, DB; the step's probabilities are drawn
+ *   again inside, as in a step; What is left as it was),
  *   gsq_kq_debug_noise: test entry points as their single-layer
  *   counterparts.
  * Errors: GSQ_ERR_INVALID_ARG (sizes, K % 256, format, null pointers),

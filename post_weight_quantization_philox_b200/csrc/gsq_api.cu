@@ -934,6 +934,21 @@ int gsq_debug_uniforms(gsq_ctx* c, uint32_t t, uint64_t coord0, int64_t count,
   return GSQ_OK;
 }
 
+int gsq_debug_noise_log2(gsq_ctx* c, uint32_t m0, int64_t count, float* host_out) {
+  int u = usable(c);
+  if (u) return u;
+  if (!host_out || count <= 0 || (int64_t)m0 + count > ((int64_t)1 << 23))
+    return GSQ_ERR_INVALID_ARG;
+  float* d = nullptr;
+  CK(pool_malloc(&d, (size_t)count * 4));
+  cudaError_t e = launch_log2_unit(m0, count, d, c->st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(c->st);
+  if (e == cudaSuccess) e = cudaMemcpy(host_out, d, (size_t)count * 4, cudaMemcpyDeviceToHost);
+  pool_free(d);
+  if (e != cudaSuccess) return fail(c, cuda_status(e));
+  return GSQ_OK;
+}
+
 int gsq_debug_stall_probe(gsq_ctx* c) {
   int u = usable(c);
   if (u) return u;

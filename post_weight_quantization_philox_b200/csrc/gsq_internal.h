@@ -312,6 +312,8 @@ cudaError_t launch_export_scales(const float* s, int64_t n, uint16_t* f16,
 cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
                             uint64_t coord0, int64_t count, float* out,
                             cudaStream_t st);
+// log2(u) of u = (m + 1/2) 2^-23 for m = m0 .. m0 + count - 1 (the noise's log2_unit)
+cudaError_t launch_log2_unit(uint32_t m0, int64_t count, float* out, cudaStream_t st);
 cudaError_t launch_sumsq(const float* x, int64_t n, double* partials,
                          unsigned* ticket, double* out, cudaStream_t st);
 // SwiGLU MLP stage: h = bf16(silu(a) b); da = bf16(dh b silu'(a)),

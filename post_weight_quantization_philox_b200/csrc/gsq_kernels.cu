@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(256) k_soft_weight(
     uint64_t coord0, uint32_t t, int noise, float inv_tau, __nv_bfloat16* __restrict__ What,
     float* __restrict__ wsoft32) {
   constexpr int L = GridT<MODE>::L;
-  __shared__ float2 l2cells[2 * kLog2Cells];
+  __shared__ float2 l2cells[kLog2Cells];
   log2_cells_init(l2cells);
   __syncthreads();
   const int64_t NK = N * K, G = K / kGroup;
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
   constexpr int L = C::L;
   constexpr bool S16 = sizeof(TS) == 2;
   extern __shared__ __align__(16) uint8_t bwd_smem[];
-  __shared__ float2 l2cells[2 * kLog2Cells];
+  __shared__ float2 l2cells[kLog2Cells];
   pdl_trigger();  // persistent grid: every CTA is resident
   log2_cells_init(l2cells);
   pdl_wait();     // dW (and the state) of the previous kernels are complete
@@ -797,6 +797,18 @@ __global__ void k_uniforms(uint64_t seed, uint32_t t, uint64_t coord0,
 #pragma unroll
     for (int p = 0; p < L; ++p) out[i * L + p] = word_to_unit(w[p]);
   }
+}
+
+// log2(u) of the uniforms u = (m + 1/2) 2^-23, m = m0 .. m0 + count - 1, as
+// the noise of every step forms it (log2_unit on the word m << 9).
+__global__ void __launch_bounds__(256) k_log2_unit(uint32_t m0, int64_t count,
+                                                   float* __restrict__ out) {
+  __shared__ float2 l2cells[kLog2Cells];
+  log2_cells_init(l2cells);
+  __syncthreads();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = log2_unit((m0 + (uint32_t)i) << 9, l2cells);
 }
 
 // sum of squares with per-block fp64 partials; the last block to finish
@@ -1323,6 +1335,11 @@ cudaError_t launch_uniforms(int mode, uint64_t seed, uint32_t t,
     case GRID_TERNARY: k_uniforms<GRID_TERNARY><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out); break;
     default: k_uniforms<GRID_3BIT_LOCAL><<<blocks, 256, 0, st>>>(seed, t, coord0, count, out);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_log2_unit(uint32_t m0, int64_t count, float* out, cudaStream_t st) {
+  k_log2_unit<<<grid_for(count, 256, 4096), 256, 0, st>>>(m0, count, out);
   return cudaGetLastError();
 }
 

@@ -24,10 +24,12 @@
 // GSQ on the format: logits over q (Q2_K: 4, the full grid; Q3_K: 5 shifts
 // -2..+2 around the start code, clamped to [-4, 3]); soft weight
 // w = a_j sum_k y_k c_k - b_j with a_j, b_j continuous and trained by Lion
-// beside the logits (starting at d sc_j, dmin m_j); Gumbel noise as the 2-bit
-// (Q2_K) and 3-bit local (Q3_K) grids draw it, the outer logarithm as they
-// take it (logf for Q2_K, __logf for Q3_K).  Projection back: hard codes
-// by argmax, a_j and b_j re-encoded as the start encodes them.
+// beside the logits (starting at d sc_j, dmin m_j); Gumbel noise and the
+// tempered softmax exactly as the 2-bit (Q2_K) and 3-bit local (Q3_K) grids
+// draw and form them (the same counters and the same function), drawn again
+// in the backward instead of kept between the soft weight and the backward.
+// Projection back: hard codes by argmax, a_j and b_j re-encoded as the start
+// encodes them.
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -294,44 +296,58 @@ __device__ __forceinline__ void kq_cand(int q0, float* c) {
     c[k] = F == KQ_Q2 ? (float)k : (float)min(max(q0 + k - 2, -4), 3);
 }
 
-// y = softmax((l + g) / tau) and v = sum_k y_k c_k
-template <int L>
-__device__ __forceinline__ float kq_soft(const float* l, const float* g, float inv_tau,
-                                         const float* c, float* y) {
-  float z[L], zm = -INFINITY;
+// Philox words of the aligned quad c0 .. c0 + 3 (c0 % 4 == 0) at step t:
+// block 0 of each coordinate and, with `five` (Q3_K), the quad's one block-1
+// draw, coordinate c0 + j taking its word j -- the counters of the GSQ grids.
+__device__ __forceinline__ void kq_quad_words(uint64_t c0, uint32_t t, const PhiloxKeys& ks,
+                                              bool five, uint32_t w[4][5]) {
+  const uint32_t hi = (uint32_t)(c0 >> 32);
 #pragma unroll
-  for (int k = 0; k < L; ++k) {
-    z[k] = (l[k] + g[k]) * inv_tau;
-    zm = fmaxf(zm, z[k]);
+  for (int j = 0; j < 4; ++j) {
+    const uint4 r = philox4x32_10(make_uint4((uint32_t)c0 + (uint32_t)j, hi, t, 0u), ks);
+    w[j][0] = r.x;
+    w[j][1] = r.y;
+    w[j][2] = r.z;
+    w[j][3] = r.w;
   }
-  float sum = 0.f;
-#pragma unroll
-  for (int k = 0; k < L; ++k) {
-    y[k] = __expf(z[k] - zm);
-    sum += y[k];
-  }
-  const float rs = 1.f / sum;
-  float v = 0.f;
-#pragma unroll
-  for (int k = 0; k < L; ++k) {
-    y[k] *= rs;
-    v = fmaf(y[k], c[k], v);
-  }
-  return v;
+  uint4 r1 = make_uint4(0u, 0u, 0u, 0u);
+  if (five) r1 = philox4x32_10(make_uint4((uint32_t)c0, hi, t, 1u), ks);
+  w[0][4] = r1.x;
+  w[1][4] = r1.y;
+  w[2][4] = r1.z;
+  w[3][4] = r1.w;
 }
 
-// Soft weight w = bf16(a_j v - b_j) of step t; the step's probabilities go
-// to probs (L planes) for the backward.  Four coordinates per thread.
+// y = softmax((l + g) / tau) with the GSQ grids' noise (gsoftmax2: the same
+// words, the same arithmetic) and v = sum_k y_k c_k
+template <int L>
+__device__ __forceinline__ float kq_value(const float* l, const uint32_t* w, bool noise,
+                                          float inv_tau, const float2* cells, const float* c,
+                                          float* y) {
+  const float r = gsoftmax2<L, false>(l, w, noise, inv_tau, cells, y);
+  float v = 0.f;
+#pragma unroll
+  for (int k = 0; k < L; ++k) v = fmaf(y[k], c[k], v);
+#pragma unroll
+  for (int k = 0; k < L; ++k) y[k] *= r;
+  return v * r;
+}
+
+// Soft weight w = bf16(a_j v - b_j) of step t.  Nothing else is kept: the
+// backward draws the same noise again from the same counters.  Four
+// coordinates per thread.
 template <int F>
 __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logits,
                                                  const float* __restrict__ a,
                                                  const float* __restrict__ b,
                                                  const int8_t* __restrict__ q0, int64_t NK,
-                                                 uint32_t k0, uint32_t k1, uint32_t t, int noise,
+                                                 const PhiloxKeys ks, uint32_t t, int noise,
                                                  float inv_tau, __nv_bfloat16* __restrict__ What,
-                                                 float* __restrict__ probs,
                                                  float* __restrict__ wsoft32) {
   constexpr int L = KqT<F>::L;
+  __shared__ float2 l2cells[kLog2Cells];
+  log2_cells_init(l2cells);
+  __syncthreads();
   for (int64_t qd = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; qd < NK / 4;
        qd += (int64_t)gridDim.x * blockDim.x) {
     const int64_t c0 = qd * 4;
@@ -341,24 +357,17 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
     float4 lp[L];
 #pragma unroll
     for (int p = 0; p < L; ++p) lp[p] = *reinterpret_cast<const float4*>(logits + p * NK + c0);
-    float wv[4], yy[4][L], gq[4][5];
-    if (noise) {
-      quad_noise5<F == KQ_Q3>((uint64_t)c0, t, k0, k1, L == 5, gq);  // c0 % 4 == 0
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
-    }
+    uint32_t wd[4][5] = {};
+    if (noise) kq_quad_words((uint64_t)c0, t, ks, L == 5, wd);
+    float wv[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float l[L], c[L];
-      const float* g = gq[j];
+      float l[L], c[L], y[L];
 #pragma unroll
       for (int p = 0; p < L; ++p)
         l[p] = j == 0 ? lp[p].x : j == 1 ? lp[p].y : j == 2 ? lp[p].z : lp[p].w;
       kq_cand<F>(qq[j], c);
-      const float v = kq_soft<L>(l, g, inv_tau, c, yy[j]);
+      const float v = kq_value<L>(l, wd[j], noise, inv_tau, l2cells, c, y);
       wv[j] = fmaf(aj, v, -bj);
     }
     __nv_bfloat162 p01 = __floats2bfloat162_rn(wv[0], wv[1]);
@@ -367,24 +376,19 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
     pk.x = *reinterpret_cast<uint32_t*>(&p01);
     pk.y = *reinterpret_cast<uint32_t*>(&p23);
     *reinterpret_cast<uint2*>(What + c0) = pk;
-    if (probs) {
-#pragma unroll
-      for (int p = 0; p < L; ++p)
-        *reinterpret_cast<float4*>(probs + p * NK + c0) =
-            make_float4(yy[0][p], yy[1][p], yy[2][p], yy[3][p]);
-    }
     if (wsoft32) *reinterpret_cast<float4*>(wsoft32 + c0) = make_float4(wv[0], wv[1], wv[2], wv[3]);
   }
 }
 
-// Backward + Lion from dW and the step's probabilities: per coordinate
+// Backward + Lion from dW: per coordinate the step's probabilities are drawn
+// again from the pre-update logits and the words of step t (the soft
+// weight's counters, so the same values), then
 // dl_k = (a_j dw / tau) y_k sum_m y_m (c_k - c_m); per sub-block
 // da_j = sum dw v, db_j = -sum dw (the four lanes of a sub-block combine by
 // shuffles, which leaves the same sum in all four); Lion on the logits, a_j
 // and (Q2_K) b_j.  With NEXT the kernel goes on to the soft weight of step
-// t_next at 1 / inv_tau_next from the updated logits, a_j and b_j -- the same
-// arithmetic as k_kq_soft -- and writes it to What and its probabilities
-// over the ones it has just read.
+// t + 1 at 1 / inv_tau_next from the updated logits, a_j and b_j -- the
+// same arithmetic as k_kq_soft -- and writes it to What.
 //
 // One warp per 128 consecutive coordinates (8 sub-blocks); lane j owns the
 // four coordinates 4j..4j+3.  The warp's next 128 coordinates are staged in
@@ -395,12 +399,12 @@ __global__ void __launch_bounds__(256) k_kq_soft(const float* __restrict__ logit
 template <int F>
 struct KqBwdCfg {
   static constexpr int L = KqT<F>::L;
-  // per-warp staging of 128 coordinates: dW, logits, momenta, probabilities, q0
-  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * 512, OFF_Y = OFF_M + L * 512;
-  static constexpr int OFF_Q = OFF_Y + L * 512;
+  // per-warp staging of 128 coordinates: dW, logits, momenta, q0
+  static constexpr int OFF_L = 512, OFF_M = OFF_L + L * 512;
+  static constexpr int OFF_Q = OFF_M + L * 512;
   static constexpr int BUF = OFF_Q + 128;
-  static constexpr int WARPS = L == 5 ? 4 : 8;  // warps per CTA
-  static constexpr int CTAS = L == 5 ? 3 : 2;   // CTAs per SM
+  static constexpr int WARPS = 8;  // warps per CTA
+  static constexpr int CTAS = 2;   // CTAs per SM
   static constexpr int SMEM = WARPS * 2 * BUF;
 };
 
@@ -408,14 +412,16 @@ template <int F, bool DBG, bool NEXT>
 __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_kq_backward(
     float* __restrict__ logits, float* __restrict__ mom, float* __restrict__ a,
     float* __restrict__ ma, float* __restrict__ b, float* __restrict__ mb,
-    const int8_t* __restrict__ q0, const float* __restrict__ dW, float* __restrict__ probs,
-    int64_t NK, float inv_tau, float lr, float b1, float omb1, float b2, float omb2,
-    float* __restrict__ dl_dbg, float* __restrict__ da_dbg, float* __restrict__ db_dbg,
-    uint32_t k0, uint32_t k1, uint32_t t_next, int noise, float inv_tau_next,
-    __nv_bfloat16* __restrict__ What) {
+    const int8_t* __restrict__ q0, const float* __restrict__ dW, int64_t NK, float inv_tau,
+    float lr, float b1, float omb1, float b2, float omb2, float* __restrict__ dl_dbg,
+    float* __restrict__ da_dbg, float* __restrict__ db_dbg, const PhiloxKeys ks, uint32_t t,
+    int noise, float inv_tau_next, __nv_bfloat16* __restrict__ What) {
   using C = KqBwdCfg<F>;
   constexpr int L = C::L;
   extern __shared__ __align__(16) uint8_t kq_smem[];
+  __shared__ float2 l2cells[kLog2Cells];
+  log2_cells_init(l2cells);
+  __syncthreads();
   const int64_t groups = NK / 128;  // K % 256 == 0
   const int lane = threadIdx.x & 31, wic = threadIdx.x >> 5;
   const int64_t nwarps = (int64_t)gridDim.x * C::WARPS;
@@ -428,7 +434,6 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
     for (int p = 0; p < L; ++p) {
       cp_async16(d + (uint32_t)(C::OFF_L + p * 512), logits + p * NK + c);
       cp_async16(d + (uint32_t)(C::OFF_M + p * 512), mom + p * NK + c);
-      cp_async16(d + (uint32_t)(C::OFF_Y + p * 512), probs + p * NK + c);
     }
     cp_async4(wbuf + (uint32_t)(buf * C::BUF + C::OFF_Q + 4 * lane), q0 + c);
   };
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
     const uint8_t* sbuf = kq_smem + wic * 2 * C::BUF + buf * C::BUF + 16 * lane;
     const int64_t c0 = gi * 128 + 4 * lane;
     const int64_t sb = c0 / kSub;
-    float dw[4], lr_[L][4], mr[L][4], yr[L][4];
+    float dw[4], lr_[L][4], mr[L][4];
     *reinterpret_cast<float4*>(dw) = *reinterpret_cast<const float4*>(sbuf);
 #pragma unroll
     for (int p = 0; p < L; ++p) {
@@ -467,25 +472,24 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
           *reinterpret_cast<const float4*>(sbuf + C::OFF_L + p * 512);
       *reinterpret_cast<float4*>(mr[p]) =
           *reinterpret_cast<const float4*>(sbuf + C::OFF_M + p * 512);
-      *reinterpret_cast<float4*>(yr[p]) =
-          *reinterpret_cast<const float4*>(sbuf + C::OFF_Y + p * 512);
     }
     const uint32_t q4 = *reinterpret_cast<const uint32_t*>(
         kq_smem + wic * 2 * C::BUF + buf * C::BUF + C::OFF_Q + 4 * lane);
     int qq[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) qq[j] = (int)(int8_t)((q4 >> (8 * j)) & 0xFFu);
+    // pass 1: this step's probabilities (pre-update logits, words of step t)
+    uint32_t wd[4][5] = {};
+    if (noise) kq_quad_words((uint64_t)c0, t, ks, L == 5, wd);
     float da_part = 0.f, db_part = 0.f;
-    float lo[L][4], mo[L][4], dlo[DBG ? L : 1][4];
+    float dlo[DBG ? L : 1][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float y[L], c[L];
+      float l[L], y[L], c[L];
 #pragma unroll
-      for (int p = 0; p < L; ++p) y[p] = yr[p][j];
+      for (int p = 0; p < L; ++p) l[p] = lr_[p][j];
       kq_cand<F>(qq[j], c);
-      float v = 0.f;
-#pragma unroll
-      for (int k = 0; k < L; ++k) v = fmaf(y[k], c[k], v);
+      const float v = kq_value<L>(l, wd[j], noise, inv_tau, l2cells, c, y);
       da_part = fmaf(dw[j], v, da_part);
       db_part -= dw[j];
       const float sc = aj * dw[j] * inv_tau;
@@ -497,15 +501,15 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
         const float g = sc * y[p] * acc;
         float th = lr_[p][j], mm = mr[p][j];
         lion_update(th, mm, g, lr, b1, omb1, b2, omb2);
-        lo[p][j] = th;
-        mo[p][j] = mm;
+        lr_[p][j] = th;
+        mr[p][j] = mm;
         if (DBG) dlo[DBG ? p : 0][j] = g;
       }
     }
 #pragma unroll
     for (int p = 0; p < L; ++p) {
-      *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(lo[p]);
-      *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(mo[p]);
+      *reinterpret_cast<float4*>(logits + p * NK + c0) = *reinterpret_cast<float4*>(lr_[p]);
+      *reinterpret_cast<float4*>(mom + p * NK + c0) = *reinterpret_cast<float4*>(mr[p]);
       if (DBG)
         *reinterpret_cast<float4*>(dl_dbg + p * NK + c0) =
             *reinterpret_cast<float4*>(dlo[DBG ? p : 0]);
@@ -532,23 +536,16 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
       }
     }
     if (NEXT) {
-      float wv[4], yy[4][L], gq[4][5];
-      if (noise) {
-        quad_noise5<F == KQ_Q3>((uint64_t)c0, t_next, k0, k1, L == 5, gq);  // c0 % 4 == 0
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int p = 0; p < 5; ++p) gq[j][p] = 0.f;
-      }
+      // pass 2: the soft weight of step t + 1 (updated logits and parameters)
+      if (noise) kq_quad_words((uint64_t)c0, t + 1u, ks, L == 5, wd);
+      float wv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float l[L], c[L];
-        const float* g = gq[j];
+        float l[L], c[L], y[L];
 #pragma unroll
-        for (int p = 0; p < L; ++p) l[p] = lo[p][j];
+        for (int p = 0; p < L; ++p) l[p] = lr_[p][j];
         kq_cand<F>(qq[j], c);
-        const float v = kq_soft<L>(l, g, inv_tau_next, c, yy[j]);
+        const float v = kq_value<L>(l, wd[j], noise, inv_tau_next, l2cells, c, y);
         wv[j] = fmaf(av, v, -bv);
       }
       __nv_bfloat162 p01 = __floats2bfloat162_rn(wv[0], wv[1]);
@@ -557,10 +554,6 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
       pk.x = *reinterpret_cast<uint32_t*>(&p01);
       pk.y = *reinterpret_cast<uint32_t*>(&p23);
       *reinterpret_cast<uint2*>(What + c0) = pk;
-#pragma unroll
-      for (int p = 0; p < L; ++p)
-        *reinterpret_cast<float4*>(probs + p * NK + c0) =
-            make_float4(yy[0][p], yy[1][p], yy[2][p], yy[3][p]);
     }
   }
   cp_async_wait<0>();
@@ -647,14 +640,14 @@ struct gsq_kq {
   int64_t N = 0, K = 0, T = 0, Tp = 0, nblk = 0;
   uint64_t seed = 0, t = 0;
   int noise = 1;
-  // What and probs hold the soft weight of step what_t at what_tau
+  // What holds the soft weight of step what_t at what_tau
   // (what_t < 0: nothing precomputed)
   int64_t what_t = -1;
   float what_tau = 0.f;
   cudaStream_t st = nullptr;
   int sms = 148, failed = 0;
   __nv_bfloat16 *Xb = nullptr, *Xt = nullptr, *What = nullptr, *dYt = nullptr;
-  float *YrefT = nullptr, *dW = nullptr, *logits = nullptr, *mom = nullptr, *probs = nullptr;
+  float *YrefT = nullptr, *dW = nullptr, *logits = nullptr, *mom = nullptr;
   float *a = nullptr, *ma = nullptr, *b = nullptr, *mb = nullptr;
   float *dl = nullptr, *da = nullptr, *db = nullptr, *wsoft32 = nullptr;  // debug, lazy
   int8_t* q0 = nullptr;
@@ -734,13 +727,13 @@ cudaError_t kq_launch_soft(gsq_kq* c, float tau, float* wsoft32) {
   const int64_t NK = c->N * c->K;
   const int g = kq_grid(NK / 4, c->sms);
   if (c->fmt == KQ_Q2)
-    k_kq_soft<KQ_Q2><<<g, 256, 0, c->st>>>(c->logits, c->a, c->b, c->q0, NK, k0, k1,
-                                           (uint32_t)c->t, c->noise, 1.f / tau, c->What,
-                                           c->probs, wsoft32);
+    k_kq_soft<KQ_Q2><<<g, 256, 0, c->st>>>(c->logits, c->a, c->b, c->q0, NK,
+                                           philox_keys(k0, k1), (uint32_t)c->t, c->noise,
+                                           1.f / tau, c->What, wsoft32);
   else
-    k_kq_soft<KQ_Q3><<<g, 256, 0, c->st>>>(c->logits, c->a, c->b, c->q0, NK, k0, k1,
-                                           (uint32_t)c->t, c->noise, 1.f / tau, c->What,
-                                           c->probs, wsoft32);
+    k_kq_soft<KQ_Q3><<<g, 256, 0, c->st>>>(c->logits, c->a, c->b, c->q0, NK,
+                                           philox_keys(k0, k1), (uint32_t)c->t, c->noise,
+                                           1.f / tau, c->What, wsoft32);
   return cudaGetLastError();
 }
 
@@ -758,9 +751,9 @@ cudaError_t kq_backward_launch(gsq_kq* c, float it, float lr, float b1, float b2
   const int64_t cap = (int64_t)c->sms * Cf::CTAS;
   const unsigned blocks = (unsigned)(need < cap ? need : cap);
   k_kq_backward<F, DBG, NEXT><<<blocks, Cf::WARPS * 32, Cf::SMEM, c->st>>>(
-      c->logits, c->mom, c->a, c->ma, c->b, c->mb, c->q0, c->dW, c->probs, NK, it, lr, b1,
-      1.f - b1, b2, 1.f - b2, c->dl, c->da, c->db, (uint32_t)c->seed,
-      (uint32_t)(c->seed >> 32), (uint32_t)(c->t + 1), c->noise, itn, c->What);
+      c->logits, c->mom, c->a, c->ma, c->b, c->mb, c->q0, c->dW, NK, it, lr, b1, 1.f - b1, b2,
+      1.f - b2, c->dl, c->da, c->db, philox_keys((uint32_t)c->seed, (uint32_t)(c->seed >> 32)),
+      (uint32_t)c->t, c->noise, itn, c->What);
   return cudaGetLastError();
 }
 
@@ -788,7 +781,7 @@ cudaError_t kq_launch_dequant(int fmt, const uint8_t* blocks, int64_t nblk, __nv
 }
 
 // One step at tau; next_tau > 0: the backward also forms the soft weight of
-// the next step at next_tau (What and probs then hold step t + 1's, recorded
+// the next step at next_tau (What then holds step t + 1's, recorded
 // in what_t / what_tau, and the next step at that tau skips its own).
 int kq_step(gsq_kq* c, float tau, float lr, float b1, float b2, float next_tau = 0.f) {
   if (c->t >= 0xFFFFFFFEull) return GSQ_ERR_UNSUPPORTED;
@@ -893,7 +886,6 @@ int gsq_kq_init(gsq_kq** out, const void* W, int w_dtype, const void* X, int x_d
   ALQ(c->dW, NK);
   ALQ(c->logits, c->L * NK);
   ALQ(c->mom, c->L * NK);
-  ALQ(c->probs, c->L * NK);
   ALQ(c->a, NS);
   ALQ(c->ma, NS);
   ALQ(c->b, NS);
@@ -1190,10 +1182,9 @@ int gsq_kq_debug_backward(gsq_kq* c, float tau, float lr, float beta1, float bet
   if (!rc) rc = kq_buffer(c, GSQ_KQ_DBG_DA, &p, &need);
   if (!rc) rc = kq_buffer(c, GSQ_KQ_DBG_DB, &p, &need);
   if (rc) return rc;
-  // the step's probabilities (soft weight of step t), then the backward from
-  // the current dW
+  // the backward from the current dW (it draws the step's probabilities
+  // again itself, as inside a step)
   c->what_t = -1;
-  CKQ(kq_launch_soft(c, tau, nullptr));
   CKQ(kq_launch_backward(c, tau, lr, beta1, beta2, true));
   return kq_check_device(c);
 }

@@ -40,7 +40,7 @@ EXPORTS = [
     "gsq_packed_bytes", "gsq_harden_pack", "gsq_recon_error",
     "gsq_state_bytes", "gsq_export_state", "gsq_import_state", "gsq_get_step",
     "gsq_destroy", "gsq_error_string", "gsq_set_timing", "gsq_phase_times",
-    "gsq_debug_uniforms", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
+    "gsq_debug_uniforms", "gsq_debug_noise_log2", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
     "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
@@ -99,6 +99,7 @@ _SIGS = {
     "gsq_set_timing": [_p, _i32],
     "gsq_phase_times": [_p, _p, _p],
     "gsq_debug_uniforms": [_p, _u32, _u64, _i64, _p],
+    "gsq_debug_noise_log2": [_p, _u32, _i64, _p],
     "gsq_debug_get": [_p, _i32, _p, _sz],
     "gsq_debug_set": [_p, _i32, _p, _sz],
     "gsq_debug_noise": [_p, _i32],
@@ -474,6 +475,12 @@ class Layer:
         out = np.zeros((count, self.L), np.float32)
         _check(_lib.gsq_debug_uniforms(self.ctx, t, coord0, count, out.ctypes.data),
                "gsq_debug_uniforms")
+        return out
+
+    def noise_log2(self, m0: int, count: int) -> np.ndarray:
+        out = np.zeros(count, np.float32)
+        _check(_lib.gsq_debug_noise_log2(self.ctx, m0, count, out.ctypes.data),
+               "gsq_debug_noise_log2")
         return out
 
     def noise(self, on: bool) -> None:

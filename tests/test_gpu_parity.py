@@ -74,6 +74,29 @@ def test_uniforms_bit_exact(g, oracle_mod, mode):
     lay.close()
 
 
+def test_noise_log2_every_uniform(g):
+    """The logarithm inside every step's noise, log2(u) for each of the 2^23
+    uniforms u = (m + 1/2) 2^-23, against fp64: relative error within 1.5e-7
+    everywhere, in particular next to u = 1 where log2(u) is tiny and a
+    logarithm with an absolute error (the hardware lg2) is off by up to 86%.
+    The Gumbel noise -ln(-ln u) takes log2 of -log2(u), so its absolute error
+    is this relative error over ln 2."""
+    cfg, W, X = make_case(0, 8, 128, 8)
+    lay = gpu_layer(g, W, X, 0)
+    n = 1 << 23
+    got = np.concatenate([lay.noise_log2(m0, 1 << 21) for m0 in range(0, n, 1 << 21)])
+    u = (np.arange(n, dtype=np.float64) + 0.5) * 2.0 ** -23
+    ref = np.log2(u)
+    rel = np.abs(got.astype(np.float64) - ref) / np.abs(ref)
+    assert rel.max() <= 1.5e-7, (rel.max(), int(rel.argmax()))
+    assert np.all(got < 0)
+    # the last uniform below 1: log2(1 - 2^-24) = -8.6e-8, relatively exact
+    assert abs(got[-1] / ref[-1] - 1) <= 1.5e-7
+    with pytest.raises(g.GSQError):
+        lay.noise_log2(n - 10, 11)
+    lay.close()
+
+
 @pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("shape", SHAPES)
 def test_init_bit_exact(g, oracle_mod, mode, shape):
