@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ctl->abort = 0;
     mbar_fence_init();
     if (EPI != EPI_LOSS) tma_prefetch_desc(&tmO);
-    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED) tma_prefetch_desc(&tmY);
+    if (EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED || EPI == EPI_SUB_F32)
+      tma_prefetch_desc(&tmY);
     if (MERGED) {
       tma_prefetch_desc(&mg.tmA2);
       tma_prefetch_desc(&mg.tmB2);
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive_expect_tx(bar, OUT_TILE);
       tma_load_2d(y_s + (uint32_t)((u & 1) * OUT_TILE), &tmY, bar, x, y);
     };
-    if ((EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED) && lane == 0) {
+    if ((EPI == EPI_LOSS_DY || EPI == EPI_LOSS || MERGED || EPI == EPI_SUB_F32) && lane == 0) {
       for (; y_issued < 2 && y_issued < y_units; ++y_issued) issue_y(y_issued);
     }
     int acc = 0;
@@ -567,13 +568,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             e[4 * j + 2] = __uint_as_float(v[4 * j + 2]) - y4.z;
             e[4 * j + 3] = __uint_as_float(v[4 * j + 3]) - y4.w;
           }
+          if (EPI == EPI_SUB_F32) {
+            // C - acc = -e goes back into the slots this lane just read,
+            // and out by TMA; the buffer is loaded again only after the
+            // store has read it
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               ybase + swz128(lane, j)),
+                           "f"(-e[4 * j]), "f"(-e[4 * j + 1]), "f"(-e[4 * j + 2]),
+                           "f"(-e[4 * j + 3])
+                           : "memory");
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (inside) {
+                tma_store_2d(&tmO, ybase, x, y);
+                bulk_commit();
+              }
+              bulk_wait_read<0>();
+            }
+          }
           __syncwarp();  // every lane has read this Y_ref buffer
           if (lane == 0 && y_issued < y_units && y_issued == u + 2) {
             issue_y(y_issued);
             ++y_issued;
           }
+          if (EPI != EPI_SUB_F32) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) part = fmaf(e[j], e[j], part);
+            for (int j = 0; j < 32; ++j) part = fmaf(e[j], e[j], part);
+          }
           if (with_dy) {
             if (lane == 0) {
               if (last_buf == b) bulk_wait_read<0>();
@@ -723,6 +747,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
     case EPI_STORE_BF16:
       return launch_pair_epi<EPI_STORE_BF16, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
                                                   sm_count, st);
+    case EPI_SUB_F32:
+      return launch_pair_epi<EPI_SUB_F32, 256>(tmA, tmB, maps, M, N, Kc, one, ep,
+                                               sm_count, st);
     default:
       return launch_pair_epi<EPI_LOSS, 256>(tmA, tmB, maps, M, N, Kc, one, ep, sm_count,
                                             st);

@@ -14,16 +14,23 @@
 //   U      = J L^-1 J with L L^T = J H J (J reverses the index order), so
 //            U^T U = J (J H J)^-1 J = H^-1 and U is upper triangular;
 //            L from a blocked right-looking Cholesky (64 x 64 diagonal
-//            blocks in one CTA, a row-wise triangular solve for the panel,
-//            a SIMT fp32 GEMM for the trailing update), L^-1 by block
-//            forward substitution with the same two kernels
+//            blocks in one CTA, the panel times the block's inverse, the
+//            trailing update on the tensor cores), L^-1 by block forward
+//            substitution (the row block times the diagonal block's inverse,
+//            the update of the later row blocks on the tensor cores)
 //   per group of 128 columns: one thread per row carries the row's 128
 //            weights in shared memory, sets the group scale absmax / c_max
 //            from the updated weights, rounds each column to the nearest
 //            level (first on ties) and feeds its error
 //            e_j = (w_j - s c) / U_jj forward within the group; the error
 //            block E (128 x N) then updates every later column at once:
-//            W[:, j1:] -= E^T U[j0:j1, j1:]   (SIMT fp32 GEMM)
+//            W[:, j1:] -= E^T U[j0:j1, j1:]   (tensor cores)
+//
+// The tensor-core updates keep fp32 accuracy: each fp32 operand is split
+// into three bf16 terms and every product is formed from six bf16 products
+// (one GEMM of six-fold depth, fp32 accumulation) whose epilogue subtracts
+// the result from the fp32 matrix in place.  The small products with the
+// diagonal blocks' inverses stay on a SIMT fp32 kernel.
 //
 // This runs once per layer before the reconstruction steps; none of it is on
 // the per-step path.
@@ -262,6 +269,72 @@ __global__ void __launch_bounds__(256) k_gemm_sub(const SubGemm g) {
     }
 }
 
+// Products of fp32 matrices on the bf16 tensor cores, to fp32 accuracy:
+// every value is split into three bf16 terms, x = x1 + x2 + x3 + r with each
+// term the bf16 rounding of what the earlier ones leave (|r| about 2^-24 |x|,
+// every subtraction exact), and sum_k x_k y_k is formed from the six products
+// x1 y1 + x1 y2 + x2 y1 + x1 y3 + x2 y2 + x3 y1 (the dropped ones are below
+// 2^-24 of the product).  The six go into one GEMM with a six-fold depth: A's
+// K blocks hold the terms (1, 1, 2, 1, 2, 3) of x, B's (1, 2, 1, 3, 2, 1) of
+// y.  bf16 x bf16 products are exact in the fp32 accumulator.
+__device__ __forceinline__ void split3_bf16(float x, __nv_bfloat16* t) {
+  t[0] = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(t[0]);
+  t[1] = __float2bfloat16_rn(r1);
+  t[2] = __float2bfloat16_rn(r1 - __bfloat162float(t[1]));
+}
+__device__ __forceinline__ int split_term(int b_side, int q) {
+  // A: 0 0 1 0 1 2, B: 0 1 0 2 1 0
+  return b_side ? (0x010210 >> (4 * (5 - q))) & 15 : (0x001012 >> (4 * (5 - q))) & 15;
+}
+
+// dst (cols x 6 depth, row-major, leading dimension 6 depth) from the
+// transpose of src (depth x cols, leading dimension lds): row n of dst holds
+// the split terms of column n of src, K block q holding term split_term(q).
+// 32 x 32 tiles through shared memory so that both sides coalesce.
+__global__ void __launch_bounds__(256) k_split_t(const float* __restrict__ src, int64_t lds,
+                                                 int depth, int64_t cols,
+                                                 __nv_bfloat16* __restrict__ dst, int b_side) {
+  __shared__ float tile[32][33];
+  const int64_t c0 = (int64_t)blockIdx.x * 32;
+  const int r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i;
+    const int64_t c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < depth && c < cols) ? src[(int64_t)r * lds + c] : 0.f;
+  }
+  __syncthreads();
+  const int64_t ldd = 6 * (int64_t)depth;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int64_t c = c0 + i;
+    const int r = r0 + threadIdx.x;
+    if (c < cols && r < depth) {
+      __nv_bfloat16 t[3];
+      split3_bf16(tile[threadIdx.x][i], t);
+#pragma unroll
+      for (int q = 0; q < 6; ++q) dst[c * ldd + q * depth + r] = t[split_term(b_side, q)];
+    }
+  }
+}
+
+// dst (rows x 6 depth) from src (rows x depth, leading dimension lds), no
+// transpose.
+__global__ void __launch_bounds__(256) k_split_rows(const float* __restrict__ src, int64_t lds,
+                                                    int64_t rows, int depth,
+                                                    __nv_bfloat16* __restrict__ dst,
+                                                    int b_side) {
+  const int64_t ldd = 6 * (int64_t)depth;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * depth;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / depth;
+    const int k = (int)(i - r * depth);
+    __nv_bfloat16 t[3];
+    split3_bf16(src[r * lds + k], t);
+#pragma unroll
+    for (int q = 0; q < 6; ++q) dst[r * ldd + q * depth + k] = t[split_term(b_side, q)];
+  }
+}
+
 // M[i][i] = 1 for all i
 __global__ void k_unit_diag(float* __restrict__ M, int64_t K) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < K;
@@ -351,9 +424,42 @@ __global__ void __launch_bounds__(kColRows * 32) k_gptq_cols(
 
 namespace {
 
+// C (rows x cols, leading dimension ldc) -= X Y^T with X rows x depth
+// (leading dimension ldx) and Y^T given either as cols x depth (ldy, b_t
+// false) or as depth x cols (b_t true), on the tensor cores with the
+// three-term split: X and Y are split into Sa and Sb, and the GEMM's
+// epilogue subtracts the product from C in place.  depth <= 128.
+cudaError_t sub_split_gemm(const float* X, int64_t ldx, int64_t rows, const float* Y,
+                           int64_t ldy, int64_t cols, int depth, bool b_t, float* C,
+                           int64_t ldc, __nv_bfloat16* Sa, __nv_bfloat16* Sb,
+                           const EpiParams& ep, int sm_count, cudaStream_t st) {
+  const int kd = 6 * depth;
+  k_split_rows<<<grid_cap(rows * depth, 256, sm_count * 8), 256, 0, st>>>(X, ldx, rows, depth,
+                                                                          Sa, 0);
+  if (b_t)
+    k_split_t<<<dim3((unsigned)((cols + 31) / 32), (unsigned)((depth + 31) / 32)), dim3(32, 8),
+                0, st>>>(Y, ldy, depth, cols, Sb, 1);
+  else
+    k_split_rows<<<grid_cap(cols * depth, 256, sm_count * 8), 256, 0, st>>>(Y, ldy, cols,
+                                                                            depth, Sb, 1);
+  CUtensorMap ta, tb;
+  EpiMaps em;
+  if (make_tmap_bf16(&ta, Sa, rows, kd, kd, kGemmBoxRowsA) ||
+      make_tmap_bf16(&tb, Sb, cols, kd, kd, kGemmBoxRowsB) ||
+      make_tmap_epi_f32(&em.out, C, rows, cols, ldc))
+    return cudaErrorInvalidValue;
+  em.yref = em.out;
+  return launch_gemm(ta, tb, em, rows, cols, kd, EPI_SUB_F32, ep, sm_count, st);
+}
+
+// W[:, j1:] -= E^T U[j0:j1, j1:] for each block of 128 columns, on the tensor
+// cores with the three-term split (fp32 accuracy): A = split of E^T (N x
+// 768), B = split of U[j0:j1, j1:]^T (rest x 768), and the GEMM's epilogue
+// subtracts the product from W's columns j1.. in place.
 template <int MODE>
 cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_t* levels,
-                         float* scales, float* E, cudaStream_t st) {
+                         float* scales, float* E, __nv_bfloat16* Es, __nv_bfloat16* Us,
+                         const EpiParams& ep, int sm_count, cudaStream_t st) {
   {
     const cudaError_t e = smem_optin<k_gptq_cols<MODE>>(kColsSmem);
     if (e != cudaSuccess) return e;
@@ -363,10 +469,20 @@ cudaError_t gptq_columns(float* W32, int64_t N, int64_t K, const float* U, int8_
     k_gptq_cols<MODE><<<rb, kColRows * 32, kColsSmem, st>>>(W32, N, K, U, j0, levels, scales, E);
     const int64_t j1 = j0 + kCols, rest = K - j1;
     if (rest > 0) {
-      // W[:, j1:] -= E^T U[j0:j1, j1:]
-      const SubGemm g{N, rest, kCols, E, 1, N, U + j0 * K + j1, K, 1, W32 + j1, K, 0};
-      k_gemm_sub<<<dim3((unsigned)((rest + kGT - 1) / kGT), (unsigned)((N + kGT - 1) / kGT)),
-                   256, 0, st>>>(g);
+      k_split_t<<<dim3((unsigned)((N + 31) / 32), kCols / 32), dim3(32, 8), 0, st>>>(
+          E, N, kCols, N, Es, 0);
+      k_split_t<<<dim3((unsigned)((rest + 31) / 32), kCols / 32), dim3(32, 8), 0, st>>>(
+          U + j0 * K + j1, K, kCols, rest, Us, 1);
+      CUtensorMap ta, tb;
+      EpiMaps em;
+      if (make_tmap_bf16(&ta, Es, N, 6 * kCols, 6 * kCols, kGemmBoxRowsA) ||
+          make_tmap_bf16(&tb, Us, rest, 6 * kCols, 6 * kCols, kGemmBoxRowsB) ||
+          make_tmap_epi_f32(&em.out, W32 + j1, N, rest, K))
+        return cudaErrorInvalidValue;
+      em.yref = em.out;
+      const cudaError_t e =
+          launch_gemm(ta, tb, em, N, rest, 6 * kCols, EPI_SUB_F32, ep, sm_count, st);
+      if (e != cudaSuccess) return e;
     }
   }
   return cudaGetLastError();
@@ -405,6 +521,9 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   float* B2 = (float*)alloc((size_t)KK * 4);
   int* dead = (int*)alloc((size_t)K * 4);
   float* E = (float*)alloc((size_t)kCols * N * 4);
+  // split operands of the tensor-core updates (up to 6 x 128 bf16 per row)
+  __nv_bfloat16* Sa = (__nv_bfloat16*)alloc((size_t)(N > K ? N : K) * 6 * kCols * 2);
+  __nv_bfloat16* Sb = (__nv_bfloat16*)alloc((size_t)K * 6 * kCols * 2);
   float* Xinv = (float*)alloc((size_t)K * kNb * 4);  // L_kk^-T of every diagonal block
   int* err = (int*)alloc(64);
   double* partials = (double*)alloc(4096 * 8);
@@ -462,9 +581,10 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
       SubGemm gs{rest, kNb, kNb, P, K, 1, Xk, kNb, 1, P, K, 0};
       gs.assign = 1;
       k_gemm_sub<<<dim3(1, (unsigned)((rest + kGT - 1) / kGT)), 256, 0, st>>>(gs);
-      const SubGemm g{rest, rest, kNb, P, K, 1, P, 1, K, P + kNb, K, 1};
-      const unsigned t = (unsigned)((rest + kGT - 1) / kGT);
-      k_gemm_sub<<<dim3(t, t), 256, 0, st>>>(g);
+      // the trailing matrix: A[c1:, c1:] -= P P^T on the tensor cores (the
+      // whole square; only its lower triangle is ever read)
+      ok(sub_split_gemm(P, K, rest, P, K, rest, kNb, false, A + (k0 + kNb) * K + k0 + kNb, K,
+                        Sa, Sb, ep, sm_count, st));
     }
     ok(cudaGetLastError());
   }
@@ -487,10 +607,9 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
       k_gemm_sub<<<dim3((unsigned)((c1 + kGT - 1) / kGT), 1), 256, 0, st>>>(gs);
     }
     if (rest > 0) {
-      // M[c1:, :c1] -= L[c1:, k0:c1] M[k0:c1, :c1]
-      const SubGemm g{rest, c1, kNb, A + c1 * K + k0, K, 1, M + k0 * K, K, 1, M + c1 * K, K, 0};
-      k_gemm_sub<<<dim3((unsigned)((c1 + kGT - 1) / kGT), (unsigned)((rest + kGT - 1) / kGT)),
-                   256, 0, st>>>(g);
+      // M[c1:, :c1] -= L[c1:, k0:c1] M[k0:c1, :c1] on the tensor cores
+      ok(sub_split_gemm(A + c1 * K + k0, K, rest, M + k0 * K, K, c1, kNb, true, M + c1 * K, K,
+                        Sa, Sb, ep, sm_count, st));
     }
     ok(cudaGetLastError());
   }
@@ -500,9 +619,16 @@ int gptq_run(int mode, const void* Wd, int w_dtype, const void* Xd, int x_dtype,
   const float* U = B2;
   if (e == cudaSuccess) {
     switch (mode) {
-      case GRID_2BIT: ok(gptq_columns<GRID_2BIT>(W32, N, K, U, levels, scales, E, st)); break;
-      case GRID_TERNARY: ok(gptq_columns<GRID_TERNARY>(W32, N, K, U, levels, scales, E, st)); break;
-      default: ok(gptq_columns<GRID_3BIT_LOCAL>(W32, N, K, U, levels, scales, E, st));
+      case GRID_2BIT:
+        ok(gptq_columns<GRID_2BIT>(W32, N, K, U, levels, scales, E, Sa, Sb, ep, sm_count, st));
+        break;
+      case GRID_TERNARY:
+        ok(gptq_columns<GRID_TERNARY>(W32, N, K, U, levels, scales, E, Sa, Sb, ep, sm_count,
+                                      st));
+        break;
+      default:
+        ok(gptq_columns<GRID_3BIT_LOCAL>(W32, N, K, U, levels, scales, E, Sa, Sb, ep, sm_count,
+                                         st));
     }
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);

@@ -35,8 +35,10 @@ enum EpiMode : int {
   EPI_LOSS_DY = 1,    // E = acc - Yref; loss += sum E^2; dY = bf16(2E)
   EPI_LOSS = 2,       // E = acc - Yref; loss += sum E^2
   EPI_STORE_BF16 = 3,  // C = bf16(acc)
-  EPI_MERGED = 4       // a forward (EPI_LOSS_DY) and a weight-gradient
+  EPI_MERGED = 4,      // a forward (EPI_LOSS_DY) and a weight-gradient
                        // (EPI_STORE_F32) problem in one launch (MergeArgs)
+  EPI_SUB_F32 = 5      // C = C - acc in place (fp32; C read through the
+                       // Y_ref map, written through the out map)
 };
 
 struct EpiParams {
