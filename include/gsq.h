@@ -707,6 +707,15 @@ GSQ_API int gsq_uniforms_noalloc(int grid_mode, uint64_t seed, uint32_t t,
  */
 GSQ_API int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
                       int64_t N, int64_t Kc, void* stream);
+/*
+ * gsq_gemm_bf16_abt_sub -- the same GEMM with the subtracting epilogue that
+ * GPTQ's tensor-core updates use: C (M x N fp32, row-major, ldc = N) -=
+ * A . B^T, in place (each output tile is read, reduced by the fp32 product
+ * and written back by the tile's own CTA).  Same argument rules and errors
+ * as gsq_gemm_bf16_abt; C is read and written.  Enqueued on `stream`; syncs.
+ */
+GSQ_API int gsq_gemm_bf16_abt_sub(const void* A, const void* B, float* C, int64_t M,
+                                  int64_t N, int64_t Kc, void* stream);
 
 #ifdef __cplusplus
 }

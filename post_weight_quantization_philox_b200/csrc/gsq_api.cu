@@ -1021,8 +1021,13 @@ int gsq_debug_scale_backward(gsq_ctx* c, float lr, float beta1, float beta2) {
   return check_device(c);
 }
 
-int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
-                      int64_t N, int64_t Kc, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// C (M x N fp32, ldc = N) = A B^T (EPI_STORE_F32) or C -= A B^T (EPI_SUB_F32)
+int gemm_bf16_abt_mode(const void* A, const void* B, float* Cout, int64_t M, int64_t N,
+                       int64_t Kc, int mode, void* stream) {
   if (!A || !B || !Cout || M <= 0 || N <= 0 || Kc <= 0 || Kc % 8 != 0 ||
       N % 4 != 0 || (reinterpret_cast<uintptr_t>(Cout) & 15) ||
       (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(B) & 15))
@@ -1056,13 +1061,27 @@ int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
   em.yref = em.out;
   cudaError_t e = cudaMemsetAsync(err, 0, 16, st);
   if (e == cudaSuccess)
-    e = launch_gemm(ta, tb, em, M, N, Kc, EPI_STORE_F32, ep, prop.multiProcessorCount, st);
+    e = launch_gemm(ta, tb, em, M, N, Kc, mode, ep, prop.multiProcessorCount, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   int h = 0;
   if (e == cudaSuccess) e = cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost);
   pool_free(err);
   if (e != cudaSuccess) return cuda_status(e);
   return h == DEV_OK ? GSQ_OK : GSQ_ERR_TIMEOUT;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gsq_gemm_bf16_abt(const void* A, const void* B, float* Cout, int64_t M,
+                      int64_t N, int64_t Kc, void* stream) {
+  return gemm_bf16_abt_mode(A, B, Cout, M, N, Kc, EPI_STORE_F32, stream);
+}
+
+int gsq_gemm_bf16_abt_sub(const void* A, const void* B, float* C, int64_t M, int64_t N,
+                          int64_t Kc, void* stream) {
+  return gemm_bf16_abt_mode(A, B, C, M, N, Kc, EPI_SUB_F32, stream);
 }
 
 }  // extern "C"

@@ -42,7 +42,7 @@ EXPORTS = [
     "gsq_destroy", "gsq_error_string", "gsq_set_timing", "gsq_phase_times",
     "gsq_debug_uniforms", "gsq_debug_noise_log2", "gsq_debug_get", "gsq_debug_set", "gsq_debug_noise",
     "gsq_debug_soft_weight", "gsq_debug_forward", "gsq_debug_weight_grad",
-    "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_uniforms_noalloc",
+    "gsq_debug_backward", "gsq_gemm_bf16_abt", "gsq_gemm_bf16_abt_sub", "gsq_uniforms_noalloc",
     "gsq_scale_step", "gsq_scale_run", "gsq_debug_scale_backward",
     "gsq_gptq", "gsq_release_cached_memory", "gsq_set_cached_memory_limit", "gsq_init_gptq", "gsq_init_bf16_state",
     "gsq_init_rows", "gsq_step_next", "gsq_mlp_set_timing", "gsq_mlp_phase_times", "gsq_attn_set_timing",
@@ -117,6 +117,7 @@ _SIGS = {
     "gsq_scale_run": [_p, _i64, _f32, _f32, _f32],
     "gsq_debug_scale_backward": [_p, _f32, _f32, _f32],
     "gsq_gemm_bf16_abt": [_p, _p, _p, _i64, _i64, _i64, _p],
+    "gsq_gemm_bf16_abt_sub": [_p, _p, _p, _i64, _i64, _i64, _p],
     "gsq_uniforms_noalloc": [_i32, _u64, _u32, _u64, _i64, _p, _p],
     "gsq_mlp_init": [_pp, _p, _i32, _p, _i32, _p, _p, _p, _i32, _i64, _i64, _i64,
                      _i32, _i32, _u64, _p],
@@ -430,6 +431,16 @@ def gsq_gemm_bf16_abt(A, B, Cout, stream=None) -> None:
     _check(_lib.gsq_gemm_bf16_abt(A.data_ptr(), B.data_ptr(), Cout.data_ptr(),
                                   M, N, Kc, _stream_ptr(stream)),
            "gsq_gemm_bf16_abt")
+
+
+def gsq_gemm_bf16_abt_sub(A, B, C, stream=None) -> None:
+    """C (M x N fp32) -= A (M x Kc bf16) . B (N x Kc bf16)^T in place; torch
+    device tensors."""
+    M, Kc = A.shape
+    N = B.shape[0]
+    _check(_lib.gsq_gemm_bf16_abt_sub(A.data_ptr(), B.data_ptr(), C.data_ptr(),
+                                      M, N, Kc, _stream_ptr(stream)),
+           "gsq_gemm_bf16_abt_sub")
 
 
 class Layer:

@@ -256,6 +256,30 @@ def test_gemm_entry_matches_oracle(g, oracle_mod, shape):
     assert np.max(np.abs(got - ref)) < 1e-4 * np.sqrt(Kc)
 
 
+@pytest.mark.parametrize("shape", [(401, 552, 200), (300, 1000, 4160), (4096, 3968, 768)])
+def test_subtracting_gemm_entry(g, oracle_mod, shape):
+    """C -= A B^T in place (the epilogue of GPTQ's tensor-core updates): ragged
+    tiles, a deep K, and the q_proj column-block shape; C's old values and the
+    product of the library's GEMM entry both come back exactly as fp32 sums."""
+    import torch
+    M, N, Kc = shape
+    rng = np.random.default_rng(M + 7 * N)
+    A = synth.bf16_values(rng.normal(size=(M, Kc)).astype(np.float32))
+    B = synth.bf16_values(rng.normal(size=(N, Kc)).astype(np.float32))
+    C0 = rng.normal(0, 10, size=(M, N)).astype(np.float32)
+    C = torch.from_numpy(C0).cuda()
+    Ad = torch.from_numpy(A).cuda().to(torch.bfloat16)
+    Bd = torch.from_numpy(B).cuda().to(torch.bfloat16)
+    g.gsq_gemm_bf16_abt_sub(Ad, Bd, C)
+    ref = C0.astype(np.float64) - oracle_mod.gemm_abt(A, B)
+    got = C.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - ref)) < 1e-4 * np.sqrt(Kc)
+    # the same product from the storing entry, subtracted in fp32 on the host
+    P = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    g.gsq_gemm_bf16_abt(Ad, Bd, P)
+    assert np.array_equal(got.astype(np.float32), C0 - P.cpu().numpy())
+
+
 @pytest.mark.parametrize("shape", SHAPES)
 def test_forward_loss_and_dy(g, oracle_mod, shape):
     N, K, T = shape
