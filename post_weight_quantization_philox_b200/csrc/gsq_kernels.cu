@@ -490,25 +490,18 @@ __global__ void __launch_bounds__(BwdCfg<MODE, TS>::WARPS * 32, BwdCfg<MODE, TS>
         dl[2] = -gs;
         dl[3] = gs;
       } else {
-        // y_k = e_k r: dl_k = (a r^2) e_k sum_j e_j (c_k - c_j); the j = k
-        // term is zero and skipped
+        // y_k = e_k r: dl_k = (a r^2) e_k sum_j e_j (c_k - c_j)
+        //                   = (a r^2) e_k (c_k S - V),
+        // S = sum_j e_j and V = sum_j e_j c_j (the sums coord_value formed,
+        // in the same order)
         const float a2 = a * r * r;
-        float dc[L][L];
+        float S = 0.f, V = 0.f;
 #pragma unroll
-        for (int p = 0; p < L; ++p)
+        for (int q = 0; q < L; ++q) S += e[q];
 #pragma unroll
-          for (int q = p + 1; q < L; ++q) {
-            dc[p][q] = cand[p] - cand[q];
-            dc[q][p] = -dc[p][q];
-          }
+        for (int q = 0; q < L; ++q) V = fmaf(e[q], cand[q], V);
 #pragma unroll
-        for (int p = 0; p < L; ++p) {
-          float acc = 0.f;
-#pragma unroll
-          for (int q = 0; q < L; ++q)
-            if (q != p) acc = fmaf(e[q], dc[p][q], acc);
-          dl[p] = a2 * e[p] * acc;
-        }
+        for (int p = 0; p < L; ++p) dl[p] = a2 * e[p] * fmaf(cand[p], S, -V);
       }
 #pragma unroll
       for (int p = 0; p < L; ++p) {
