@@ -437,10 +437,19 @@ STEP_KERNEL_SOURCES = ("gsq_device.cuh", "gsq_gemm.cu", "gsq_gemm_epi.cuh",
 
 
 def kernel_sources_hash():
+    """Hash of the step kernels' code: the sources with comments and blank
+    space removed, so that a comment edit keeps the counters valid and any
+    code change drops them."""
     import hashlib
+    import re
     csrc = os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc")
-    blob = b"".join(open(os.path.join(csrc, f), "rb").read() for f in STEP_KERNEL_SOURCES)
-    return hashlib.sha256(blob).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in STEP_KERNEL_SOURCES:
+        text = open(os.path.join(csrc, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()[:16]
 
 
 def rank_seed(base: int, rank: int) -> int:

@@ -22,7 +22,8 @@
 // MMA thread signals each CTA's "empty" and "accumulator full" barriers with
 // one tcgen05.commit per CTA (shared::cluster addresses from mapa); the
 // epilogue warps of both CTAs release an accumulator on the leader's
-// barrier.  No cluster multicast of any load is used.  Every mbarrier wait
+// barrier.  Every TMA load lands in the issuing CTA's own shared memory
+// only, from this GPU's own memory.  Every mbarrier wait
 // is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, drains what it
 // issued, frees TMEM and returns.
 #include "gsq_gemm_epi.cuh"

@@ -98,66 +98,91 @@ __global__ void k_reverse(const float* __restrict__ src, float* __restrict__ dst
 }
 
 // Lower Cholesky factor L of the 64 x 64 diagonal block at (k0, k0), in place
-// (lower triangle only), right-looking: column by column every thread takes
-// the pivot's square root, the rows below divide their entry of the column,
-// and the trailing lower triangle takes its rank-1 update, 1024 threads
-// owning 4 entries each (column t % 64 of rows t / 64 + 16 j, so a warp's
-// accesses fall in distinct banks).  A pivot that is not positive is
-// recorded and replaced by 1 so that nothing downstream turns into NaN.
-// Then X = L^-T into Xinv (64 x 64, row-major): row r of X solves
-// x L^T = e_r by forward substitution, 16 threads per row sharing each
-// column's dot product.  The triangular solves against L become GEMMs with X.
-constexpr int kPotrfThreads = 1024;
+// (lower triangle only), right-looking, and X = L^-T into Xinv (64 x 64,
+// row-major).  64 threads, thread r holding row r of the block in registers
+// (every loop below is unrolled, so the row is indexed statically):
+//   column c: thread c takes the pivot's square root, every row r > c forms
+//   l_rc = a_rc / sqrt(a_cc) and publishes it, then each row takes the
+//   rank-1 update a_rs -= l_rc l_sc of its entries c < s <= r;
+//   row r of X solves x L^T = e_r by forward substitution
+//   (x_c = (delta_rc - sum_{s<c} x_s L_cs) / L_cc, x_c = 0 for c < r, so the
+//   dot product needs no bound on s).
+// A pivot that is not positive is recorded and replaced by 1 so that nothing
+// downstream turns into NaN.  The triangular solves against L become GEMMs
+// with X.
+constexpr int kPotrfThreads = kNb;
 __global__ void __launch_bounds__(kPotrfThreads) k_potrf64(float* __restrict__ A, int64_t K,
                                                            int64_t k0, int* __restrict__ err,
                                                            float* __restrict__ Xinv) {
-  __shared__ float a[kNb][kNb + 1];
-  __shared__ float xs[kNb][kNb + 1];
-  const int t = threadIdx.x;
-  for (int e = t; e < kNb * kNb; e += kPotrfThreads) {
-    const int rr = e / kNb, c = e % kNb;
-    a[rr][c] = c <= rr ? A[(k0 + rr) * K + k0 + c] : 0.f;
+  __shared__ float ls[kNb][kNb + 1];  // the block (rows), then L
+  __shared__ float col[kNb];          // the current column of L
+  __shared__ float piv;               // its diagonal entry
+  const int r = threadIdx.x;
+  {
+    // coalesced: thread r loads column r of each row, all 64 loads in
+    // flight before the first store (the block is often not in L2)
+    float v[kNb];
+#pragma unroll
+    for (int i = 0; i < kNb; ++i) v[i] = A[(k0 + i) * K + k0 + r];
+#pragma unroll
+    for (int i = 0; i < kNb; ++i) ls[i][r] = v[i];
   }
   __syncthreads();
-  const int s2 = t & (kNb - 1), rb = t / kNb;  // entries (rb + 16 j, s2)
-  for (int c = 0; c < kNb; ++c) {
-    float d = a[c][c];
-    const bool bad = !(d > 0.f) || !isfinite(d);
-    if (bad) d = 1.f;
-    const float sd = sqrtf(d);
-    __syncthreads();  // every thread has read the pivot
-    if (t == c) {
-      if (bad) atomicCAS(err, 0, DEV_ERR_NONFINITE);
-      a[c][c] = sd;
-    }
-    if (t > c && t < kNb) a[t][c] /= sd;
-    __syncthreads();
-    if (s2 > c) {
-      const float u = a[s2][c];
+  float a[kNb];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = rb + 16 * j;
-        if (s2 <= r) a[r][s2] -= a[r][c] * u;
+  for (int s = 0; s < kNb; ++s) a[s] = s <= r ? ls[r][s] : 0.f;
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kNb; ++c) {
+    if (r == c) {
+      float d = a[c];
+      const bool bad = !(d > 0.f) || !isfinite(d);
+      if (bad) {
+        d = 1.f;
+        atomicCAS(err, 0, DEV_ERR_NONFINITE);
       }
+      piv = sqrtf(d);
     }
+    // the pivot's root; every row is also done with the previous column's
+    // update, so col can be rewritten (and piv was read before the barrier
+    // below in the previous column)
     __syncthreads();
-  }
-  for (int e = t; e < kNb * kNb; e += kPotrfThreads) {
-    const int rr = e / kNb, c = e % kNb;
-    if (c <= rr) A[(k0 + rr) * K + k0 + c] = a[rr][c];
-  }
-  // X = L^-T: x_c = (delta_rc - sum_{s<c} x_s L_cs) / L_cc, x_c = 0 for c < r
-  const int r = t >> 4, sub = t & 15;
-  for (int c = 0; c < kNb; ++c) {
-    float part = 0.f;
-    for (int q = sub; q < c; q += 16) part = fmaf(xs[r][q], a[c][q], part);
+    const float sd = piv;
+    const float l = r > c ? a[c] / sd : (r == c ? sd : 0.f);
+    if (r > c) col[r] = l;
+    __syncthreads();  // the column
+    if (r >= c) a[c] = l;
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (sub == 0) xs[r][c] = c < r ? 0.f : ((c == r ? 1.f : 0.f) - part) / a[c][c];
-    __syncwarp();
+    for (int s = c + 1; s < kNb; ++s)
+      if (r > c && s <= r) a[s] -= l * col[s];
   }
+#pragma unroll
+  for (int s = 0; s < kNb; ++s) ls[r][s] = s <= r ? a[s] : 0.f;
   __syncthreads();
-  for (int e = t; e < kNb * kNb; e += kPotrfThreads) Xinv[e] = xs[e / kNb][e % kNb];
+  for (int i = 0; i < kNb; ++i)
+    if (r <= i) A[(k0 + i) * K + k0 + r] = ls[i][r];
+  // X = L^-T, row r in registers; four partial sums for the dot products
+  float x[kNb];
+#pragma unroll
+  for (int c = 0; c < kNb; ++c) {
+    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+    for (int q = 0; q + 3 < c; q += 4) {
+      p0 = fmaf(x[q], ls[c][q], p0);
+      p1 = fmaf(x[q + 1], ls[c][q + 1], p1);
+      p2 = fmaf(x[q + 2], ls[c][q + 2], p2);
+      p3 = fmaf(x[q + 3], ls[c][q + 3], p3);
+    }
+#pragma unroll
+    for (int q = c & ~3; q < c; ++q) p0 = fmaf(x[q], ls[c][q], p0);
+    const float part = (p0 + p1) + (p2 + p3);
+    x[c] = c < r ? 0.f : ((c == r ? 1.f : 0.f) - part) / ls[c][c];
+  }
+  __syncthreads();  // L is read by every thread above; reuse ls for X
+#pragma unroll
+  for (int c = 0; c < kNb; ++c) ls[r][c] = x[c];
+  __syncthreads();
+  for (int i = 0; i < kNb; ++i) Xinv[i * kNb + r] = ls[i][r];
 }
 
 // C[m][n] -= sum_k A(m, k) B(k, n) (or =, with assign) with A(m, k) = A[m a_rs + k a_cs] and
@@ -378,9 +403,23 @@ __global__ void __launch_bounds__(kColRows * 32) k_gptq_cols(
   using Gr = GridT<MODE>;
   extern __shared__ __align__(16) uint8_t gsm[];
   float (*us)[kCols] = reinterpret_cast<float (*)[kCols]>(gsm);
-  for (int e = threadIdx.x; e < kCols * kCols; e += blockDim.x) {
-    const int r = e / kCols, c = e % kCols;
-    us[r][c] = c >= r ? U[(j0 + r) * K + j0 + c] : 0.f;
+  // eight loads in flight per thread before their stores (the block of U
+  // is usually not in L2); kCols * kCols is a multiple of 8 x the block
+  constexpr int kBatch = 8;
+  static_assert((kCols * kCols) % (kBatch * kColRows * 32) == 0, "U block load batches");
+  for (int e0 = threadIdx.x; e0 < kCols * kCols; e0 += kBatch * blockDim.x) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int e = e0 + u * blockDim.x;
+      const int r = e / kCols, c = e % kCols;
+      v[u] = c >= r ? U[(j0 + r) * K + j0 + c] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int e = e0 + u * blockDim.x;
+      us[e / kCols][e % kCols] = v[u];
+    }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
