@@ -436,20 +436,25 @@ STEP_KERNEL_SOURCES = ("gsq_device.cuh", "gsq_gemm.cu", "gsq_gemm_epi.cuh",
                        "gsq_gemm_pair.cu", "gsq_internal.h", "gsq_kernels.cu")
 
 
-def kernel_sources_hash():
-    """Hash of the step kernels' code: the sources with comments and blank
-    space removed, so that a comment edit keeps the counters valid and any
-    code change drops them."""
+def code_hash(texts) -> str:
+    """Hash of C/CUDA sources with comments and blank space removed."""
     import hashlib
     import re
-    csrc = os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc")
     h = hashlib.sha256()
-    for f in STEP_KERNEL_SOURCES:
-        text = open(os.path.join(csrc, f), encoding="utf-8").read()
+    for text in texts:
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
         text = re.sub(r"//[^\n]*", " ", text)
         h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
+
+
+def kernel_sources_hash():
+    """Hash of the step kernels' code (comments and blank space removed), so
+    that a comment edit keeps the counters valid and any code change drops
+    them."""
+    csrc = os.path.join(ROOT, "post_weight_quantization_philox_b200", "csrc")
+    return code_hash(open(os.path.join(csrc, f), encoding="utf-8").read()
+                     for f in STEP_KERNEL_SOURCES)
 
 
 def rank_seed(base: int, rank: int) -> int:

@@ -73,3 +73,11 @@ def test_block_step_accounting():
     T = 8 * 2048
     assert f[0] == 4.0 * T * 8192 * 8192 and f[1] == 4.0 * T * 1024 * 8192
     assert f[3] == 14.0 * T * 8192 * 28672
+
+
+def test_traffic_counters_follow_the_code_not_the_comments():
+    a = "int f(int x) {  // doubles\n  return 2 * x; /* fast */ }\n"
+    b = "int f(int x) {  // twice x\n\n  return 2 * x;   }\n"
+    c = "int f(int x) {  // doubles\n  return 3 * x; /* fast */ }\n"
+    assert bench.code_hash([a]) == bench.code_hash([b])
+    assert bench.code_hash([a]) != bench.code_hash([c])
