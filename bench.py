@@ -992,7 +992,7 @@ def block_e2e(gsq, torch, W, gen, dm, steps, rank):
                     f"outputs to pinned host memory")}
 
 
-def gptq_simt_flops(N: int, K: int) -> float:
+def gptq_flops(N: int, K: int) -> float:
     """fp32 flops of one GPTQ call (algorithmic): Cholesky of the damped K x K
     Hessian (K^3 / 3), inverse of its triangular factor (K^3 / 3), the
     trailing-column error updates (N K^2 in total) and the in-group feedback
@@ -1047,7 +1047,7 @@ def run_gptq_stage(args, rank, world, local_rank):
     # measured burst bf16 rate / 6
     hbm, tf_burst, tf_sus, peak_kind = peaks()
     split_peak = tf_burst / 6.0
-    flops = gptq_simt_flops(cfg.N, cfg.K)
+    flops = gptq_flops(cfg.N, cfg.K)
     ach = flops / (per / 1e3) / 1e12
     coords = cfg.N * cfg.K
     return {"metric": METRIC, "value": whole_job_rate(world, coords, per), "unit": UNIT,
