@@ -287,8 +287,8 @@ def run_gsq(args, rank, world, local_rank):
     phase_n = list(phase_n)
     phase_ms[0], phase_n[0] = loop_ms[0], loop_n[0]
     if phase_n[2] == 0 and phase_n[1] > 0:
-        # both GEMMs of a step ran as one launch (layers with fewer than 24
-        # row tiles): the forward slot holds them both
+        # both GEMMs of a step ran as one launch (layers whose X is at most
+        # 64 MB): the forward slot holds them both
         names = list(names)
         names[1] = "gemms_merged"
         work["gemms_merged"] = ("tensor", work["forward_gemm"][1] + work["weight_grad_gemm"][1])

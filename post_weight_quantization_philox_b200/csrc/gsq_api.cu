@@ -356,15 +356,16 @@ int init_impl(gsq_ctx** out, const void* W, int w_dtype, const void* X,
   AL(c->ticket, 4);
   AL(c->err, 4);
   {
-    // both GEMMs of a step in one launch when the layer has fewer than 24
-    // row tiles and the GEMMs' B operand (X, Tp x K bf16) fits well inside
-    // L2: the merged launch runs each band's column tiles together, so a
-    // wave reads every column tile of B.  (Measured on one B200: q_proj
-    // 4096 x 4096 -4.5% per step; with a 117 MB or 268 MB B, down_proj
-    // 4096 x 14336 and the 70B k_proj, +3% and +10%.)  Larger layers keep
-    // two launches, with the banded tile order from 24 row tiles.
+    // both GEMMs of a step in one launch when the GEMMs' B operand (X, Tp x
+    // K bf16) fits well inside L2: the merged launch runs each 256-row
+    // band's column tiles together, so a wave reads every column tile of B
+    // and one band of A.  (Measured on one B200: q_proj 4096 x 4096 -4.5%
+    // per step, gate_proj 14336 x 4096 -0.8% (its GEMMs -6%); with a 117 MB
+    // or 268 MB B, down_proj 4096 x 14336 and the 70B k_proj, +3% and +10%.)
+    // Larger B keeps two launches, with the banded tile order from 24 row
+    // tiles.
     const int64_t m_tiles = (N + 255) / 256;
-    c->merged = m_tiles < 24 && (double)Tp * (double)K * 2.0 <= 64.0 * 1024 * 1024;
+    c->merged = (double)Tp * (double)K * 2.0 <= 64.0 * 1024 * 1024;
     AL(c->band_done, m_tiles);
   }
   // init-only staging
