@@ -493,12 +493,16 @@ __global__ void __launch_bounds__(KqBwdCfg<F>::WARPS * 32, KqBwdCfg<F>::CTAS) k_
       da_part = fmaf(dw[j], v, da_part);
       db_part -= dw[j];
       const float sc = aj * dw[j] * inv_tau;
+      // sum_k y_k (c_p - c_k) = c_p Sy - Vy, Sy = sum_k y_k, Vy = sum_k y_k c_k
+      float Sy = 0.f, Vy = 0.f;
+#pragma unroll
+      for (int k = 0; k < L; ++k) {
+        Sy += y[k];
+        Vy = fmaf(y[k], c[k], Vy);
+      }
 #pragma unroll
       for (int p = 0; p < L; ++p) {
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < L; ++k) acc = fmaf(y[k], c[p] - c[k], acc);
-        const float g = sc * y[p] * acc;
+        const float g = sc * y[p] * fmaf(c[p], Sy, -Vy);
         float th = lr_[p][j], mm = mr[p][j];
         lion_update(th, mm, g, lr, b1, omb1, b2, omb2);
         lr_[p][j] = th;
