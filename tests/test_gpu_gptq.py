@@ -141,6 +141,16 @@ def test_dead_inputs_and_bad_arguments(g):
         g.gsq_gptq(W, X, group=64)
     with pytest.raises(g.GSQError):
         g.gsq_gptq(W[:, :200], X[:, :200])
+    # a non-finite calibration value reaches the factorisation's pivots (or is
+    # caught converting X): reported as GSQ_ERR_NONFINITE, and the next call
+    # on clean inputs is unaffected
+    Xbad = X.copy()
+    Xbad[7, 5] = np.nan
+    with pytest.raises(g.GSQError) as e:
+        g.gsq_gptq(W, Xbad)
+    assert e.value.status == g.GSQ_ERR_NONFINITE
+    lev2, s2 = g.gsq_gptq(W, X)
+    assert np.array_equal(lev2, lev) and np.array_equal(s2, s)
 
 
 def test_full_size_q_proj_row_slices(g, oracle_mod):
